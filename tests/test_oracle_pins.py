@@ -1,0 +1,334 @@
+"""Pins for the float64 oracle, each against something other than the oracle
+itself: hand-derived cases (tests/golden), closed forms, brute force on tiny
+inputs, exact rational arithmetic, and independent library routines (torch's
+float32 -> bfloat16 cast, torch's float64 scaled_dot_product_attention,
+numpy's argpartition).  CPU only.
+"""
+
+import itertools
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_worked_cases.json")
+
+
+def _bf16_bits(x):
+    return torch.tensor(np.asarray(x, np.float32)).to(torch.bfloat16).view(torch.int16).numpy().astype(np.int64) & 0xFFFF
+
+
+def _bf16_from_bits(bits):
+    b = torch.tensor(np.asarray(bits, np.int64).astype(np.int16)).view(torch.bfloat16)
+    return b.to(torch.float64).numpy()
+
+
+# ---------------------------------------------------------------- bf16 rounding
+
+def test_bf16_round_matches_torch_cast_on_float32_inputs():
+    rng = np.random.default_rng(1)
+    mags = np.concatenate([
+        rng.standard_normal(20000),
+        rng.standard_normal(2000) * 1e-38,    # subnormal range
+        rng.standard_normal(2000) * 1e-30,
+        rng.uniform(-1.0, 1.0, 2000) * 3.3e38,  # near overflow
+        rng.standard_normal(2000) * 1e6,
+    ]).astype(np.float32)
+    mags = mags[np.isfinite(mags)]
+    ref = torch.tensor(mags).to(torch.bfloat16).to(torch.float64).numpy()
+    got = O.bf16_round(mags.astype(np.float64))
+    np.testing.assert_array_equal(got, ref)
+
+
+def test_bf16_round_ties_to_even_from_the_exact_value():
+    # near 1.0 the bf16 quantum is 2^-7
+    cases = {
+        1.0 + 2.0 ** -8: 1.0,                              # tie -> even (1.0)
+        1.0 + 3 * 2.0 ** -8: 1.0 + 2.0 ** -6,               # tie -> even mantissa
+        1.0 + 2.0 ** -8 + 2.0 ** -30: 1.0 + 2.0 ** -7,      # just above the tie: up
+        -(1.0 + 2.0 ** -8 + 2.0 ** -40): -(1.0 + 2.0 ** -7),
+        1.0 + 2.0 ** -8 - 2.0 ** -40: 1.0,                 # just below the tie: down
+    }
+    for x, want in cases.items():
+        assert O.bf16_round(np.array([x]))[0] == want, x
+    # rounding through float32 first would turn 1 + 2^-8 + 2^-30 into the tie 1 + 2^-8
+    # and then into 1.0; the oracle must not do that.
+    assert np.float32(1.0 + 2.0 ** -8 + 2.0 ** -30) == np.float32(1.0 + 2.0 ** -8)
+
+
+def test_bf16_round_special_values():
+    x = np.array([0.0, -0.0, np.inf, -np.inf, 1e39, -1e39])
+    y = O.bf16_round(x)
+    assert y[0] == 0.0 and y[1] == 0.0 and np.signbit(y[1])
+    assert np.isposinf(y[2]) and np.isneginf(y[3]) and np.isposinf(y[4]) and np.isneginf(y[5])
+
+
+# ---------------------------------------------------------------- index keys
+
+def test_index_keys_coordinate_selection_pins_operand_orientation():
+    # P_g picks coordinate perm[j] of k for output j: k~_j = k[perm[j]] exactly.
+    rng = np.random.default_rng(2)
+    d, r = 16, 16
+    perm = (3 * np.arange(r) + 1) % d           # not an involution
+    P = np.zeros((d, r))
+    P[perm, np.arange(r)] = 1.0
+    k = O.bf16_round(rng.standard_normal((5, d)))
+    got = O.index_keys(P, k)
+    np.testing.assert_array_equal(got, k[:, perm])
+    assert not np.array_equal(got, k[:, np.argsort(perm)])   # the transpose differs
+
+
+def test_index_keys_is_the_nearest_bf16_of_the_exact_sum():
+    rng = np.random.default_rng(3)
+    d, r, n = 64, 16, 6
+    P = O.bf16_round(rng.standard_normal((d, r)) / 8.0)
+    K = O.bf16_round(rng.standard_normal((n, d)))
+    got = O.index_keys(P, K)
+    bits = _bf16_bits(got.astype(np.float32))
+    assert np.array_equal(_bf16_from_bits(bits), got)        # representable in bf16
+    lo, hi = _bf16_from_bits(bits - 1), _bf16_from_bits(bits + 1)   # bf16 neighbours
+    for t in range(n):
+        for j in range(r):
+            exact = sum(Fraction(float(K[t, i])) * Fraction(float(P[i, j])) for i in range(d))
+            err = abs(Fraction(float(got[t, j])) - exact)
+            for nb in (lo[t, j], hi[t, j]):
+                e_nb = abs(Fraction(float(nb)) - exact)
+                assert err <= e_nb
+                if err == e_nb:                                # a tie: even bit pattern
+                    assert bits[t, j] % 2 == 0
+
+
+def test_index_scores_with_identity_projection_are_full_dot_products():
+    rng = np.random.default_rng(4)
+    d = r = 16
+    P = np.eye(d)
+    q = O.bf16_round(rng.standard_normal(d))
+    K = O.bf16_round(rng.standard_normal((40, d)))
+    s = O.index_scores(O.query_index(P, q), O.index_keys(P, K), 0.25)
+    want = np.array([0.25 * math.fsum(float(q[i]) * float(K[j, i]) for i in range(d)) for j in range(40)])
+    np.testing.assert_allclose(s, want, rtol=0, atol=1e-12)
+
+
+def test_query_index_uses_the_group_projection_columns():
+    # q~_j = <q, P[:, j]>: with P = e_i e_j^T only output j is non-zero and equals q_i.
+    d, r = 8, 4
+    q = np.arange(1.0, d + 1)
+    P = np.zeros((d, r)); P[5, 2] = 1.0
+    np.testing.assert_array_equal(O.query_index(P, q), [0, 0, 6.0, 0])
+
+
+# ---------------------------------------------------------------- golden cases
+
+def _golden():
+    with open(GOLDEN) as f:
+        return json.load(f)
+
+
+def test_top_p_hand_worked_cases():
+    for c in _golden()["top_p"]:
+        s = np.log(np.array(c["scores_ln"], dtype=np.float64))
+        got = O.select_top_p(s, c["p"]).tolist()
+        assert got == c["expected"], c
+
+
+def test_top_k_hand_worked_cases():
+    for c in _golden()["top_k"]:
+        got = O.select_top_k(np.array(c["scores"], np.float64), c["k"]).tolist()
+        assert got == c["expected"], c
+
+
+def test_local_positions_hand_worked_cases():
+    for c in _golden()["local"]:
+        want = [j for a, b in c["expected_ranges"] for j in range(a, b)]
+        assert O.local_positions(c["n"], c["window"], c["sinks"]).tolist() == want, c
+
+
+# ---------------------------------------------------------------- top-p
+
+def _mass(s):
+    w = np.exp(s - s.max())
+    return w / w.sum()
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_top_p_brute_force_over_all_subsets(seed):
+    rng = np.random.default_rng(100 + seed)
+    n = int(rng.integers(1, 11))
+    s = rng.standard_normal(n) * rng.uniform(0.2, 4.0)      # distinct almost surely
+    p = float(rng.uniform(0.05, 0.99))
+    w = _mass(s)
+    best = None
+    for m in range(1, n + 1):
+        reach = [T for T in itertools.combinations(range(n), m) if w[list(T)].sum() >= p]
+        if reach:
+            best = max(reach, key=lambda T: w[list(T)].sum())
+            break
+    assert best is not None
+    assert O.select_top_p(s, p).tolist() == sorted(best)
+
+
+@pytest.mark.parametrize("seed", range(10))
+def test_top_p_defining_property(seed):
+    rng = np.random.default_rng(200 + seed)
+    n = int(rng.integers(50, 5000))
+    s = rng.standard_normal(n) * rng.uniform(0.5, 6.0)
+    p = float(rng.uniform(0.1, 0.99))
+    S = O.select_top_p(s, p)
+    w = _mass(s)
+    inS = np.zeros(n, bool); inS[S] = True
+    assert math.fsum(w[S]) >= p - 1e-12
+    lowest = S[np.argmin(s[S])]
+    assert math.fsum(w[S]) - w[lowest] < p + 1e-12          # minimal
+    if (~inS).any():
+        assert s[S].min() > s[~inS].max()                    # a prefix of the ranking
+
+
+@pytest.mark.parametrize("alpha", [0.8, 1.2])
+@pytest.mark.parametrize("p", [0.5, 0.9, 0.99])
+def test_top_p_zipf_closed_form(alpha, p):
+    # scores -alpha*ln(rank) give softmax masses proportional to rank^-alpha, so
+    # |S| is the smallest n with sum_{r<=n} r^-alpha >= p * sum_{r<=N} r^-alpha.
+    N = 262144
+    rng = np.random.default_rng(7)
+    rank = rng.permutation(N) + 1
+    s = -alpha * np.log(rank.astype(np.float64))
+    terms = [r ** -alpha for r in range(1, N + 1)]
+    total = math.fsum(terms)
+    acc, n_expect = 0.0, None
+    partial = np.cumsum(np.array(terms))                     # monotone; exact check below
+    n_expect = int(np.searchsorted(partial, p * total, side="left")) + 1
+    # confirm the boundary with exact summation on both sides
+    assert math.fsum(terms[:n_expect]) >= p * total
+    assert math.fsum(terms[:n_expect - 1]) < p * total
+    S = O.select_top_p(s, p)
+    assert len(S) == n_expect
+    assert set(rank[S].tolist()) == set(range(1, n_expect + 1))
+
+
+def test_top_p_one_keeps_everything_and_scale_invariance_of_order():
+    s = np.array([3.0, -1.0, 2.0])
+    assert O.select_top_p(s, 1.0).tolist() == [0, 1, 2]
+    assert O.select_top_p(s + 1000.0, 0.6).tolist() == O.select_top_p(s, 0.6).tolist()
+
+
+# ---------------------------------------------------------------- top-k
+
+@pytest.mark.parametrize("seed", range(20))
+def test_top_k_brute_force_and_argpartition(seed):
+    rng = np.random.default_rng(300 + seed)
+    n = int(rng.integers(1, 10))
+    s = rng.standard_normal(n)
+    k = int(rng.integers(1, n + 1))
+    best = max(itertools.combinations(range(n), k), key=lambda T: s[list(T)].sum())
+    assert O.select_top_k(s, k).tolist() == sorted(best)
+    big = rng.standard_normal(3000)
+    kk = int(rng.integers(1, 3000))
+    assert O.select_top_k(big, kk).tolist() == sorted(np.argpartition(-big, kk - 1)[:kk].tolist())
+
+
+def test_top_k_budget():
+    assert O.top_k_budget(131072, 0, 0.02) == 2621       # 2% of 128K, float32 fraction
+    assert O.top_k_budget(100, 0, 0.001) == 1
+    assert O.top_k_budget(100, 5000, 0.0) == 100
+    assert O.top_k_budget(512, 7, 0.5) == 7
+
+
+# ---------------------------------------------------------------- attention
+
+def _sdpa64(q, K, V, scale):
+    qt = torch.tensor(q, dtype=torch.float64)[None, None, None, :]
+    Kt = torch.tensor(K, dtype=torch.float64)[None, None]
+    Vt = torch.tensor(V, dtype=torch.float64)[None, None]
+    return torch.nn.functional.scaled_dot_product_attention(qt, Kt, Vt, scale=scale)[0, 0, 0].numpy()
+
+
+def test_attend_full_set_is_dense_sdpa():
+    rng = np.random.default_rng(5)
+    n, d = 300, 64
+    q, K, V = (O.bf16_round(rng.standard_normal(sh)) for sh in [(d,), (n, d), (n, d)])
+    got = O.attend_set(q, K, V, np.arange(n), 1 / 8)
+    np.testing.assert_allclose(got, _sdpa64(q, K, V, 1 / 8), rtol=1e-12, atol=1e-13)
+
+
+def test_attend_single_and_pair_closed_forms():
+    rng = np.random.default_rng(6)
+    d = 16
+    q, K, V = rng.standard_normal(d), rng.standard_normal((5, d)), rng.standard_normal((5, d))
+    np.testing.assert_array_equal(O.attend_set(q, K, V, [3], 0.3), V[3])
+    l1, l4 = 0.3 * K[1] @ q, 0.3 * K[4] @ q
+    a = 1.0 / (1.0 + math.exp(l4 - l1))
+    np.testing.assert_allclose(O.attend_set(q, K, V, [1, 4], 0.3), a * V[1] + (1 - a) * V[4], rtol=1e-13)
+    assert np.all(O.attend_set(q, K, V, [], 0.3) == 0)
+
+
+def _tiny_problem(seed, page_perm=False, n_list=(37, 20), Hq=4, Hkv=2, d=32, r=16):
+    rng = np.random.default_rng(seed)
+    ps = 16
+    B = len(n_list)
+    pages_per = [math.ceil(n / ps) for n in n_list]
+    total = sum(pages_per)
+    ids = rng.permutation(total) if page_perm else np.arange(total)
+    pt = -np.ones((B, max(pages_per)), np.int64)
+    c = 0
+    for b, m in enumerate(pages_per):
+        pt[b, :m] = ids[c:c + m]
+        c += m
+    kc = O.bf16_round(rng.standard_normal((total, Hkv, ps, d)))
+    vc = O.bf16_round(rng.standard_normal((total, Hkv, ps, d)))
+    proj = O.bf16_round(rng.standard_normal((Hkv, d, r)) / math.sqrt(d))
+    q = O.bf16_round(rng.standard_normal((B, Hq, d)))
+    return dict(proj=proj, q_pre=q, q=q, k_cache=kc, v_cache=vc, page_table=pt,
+                seq_lens=np.array(n_list)), Hq, Hkv, d, r
+
+
+@pytest.mark.parametrize("mode", ["top_p1", "top_kN", "windowN"])
+def test_decode_step_degenerate_cases_are_dense_sdpa(mode):
+    # p = 1, k >= N and window >= N all reduce to dense attention ([NHA] §2.3:
+    # a window as long as the sequence is full attention).
+    prob, Hq, Hkv, d, r = _tiny_problem(11, page_perm=True)
+    retr = [1, 1, 0, 0]
+    if mode == "top_p1":
+        cfg = O.OracleConfig(Hq, Hkv, d, r, 16, retr, 10 ** 6, 2, "top_p", top_p=1.0)
+    elif mode == "top_kN":
+        cfg = O.OracleConfig(Hq, Hkv, d, r, 16, retr, 10 ** 6, 2, "top_k", top_k=10 ** 6)
+    else:
+        cfg = O.OracleConfig(Hq, Hkv, d, r, 16, [0, 0, 0, 0], 10 ** 6, 0, "top_p")
+    res = O.decode_reference(cfg, **prob)
+    G = Hq // Hkv
+    for (b, h), o in res.out.items():
+        n = prob["seq_lens"][b]
+        K = O.gather_rows(prob["k_cache"], prob["page_table"][b], n, h // G, 16)
+        V = O.gather_rows(prob["v_cache"], prob["page_table"][b], n, h // G, 16)
+        np.testing.assert_allclose(o, _sdpa64(prob["q"][b, h], K, V, 1 / math.sqrt(d)),
+                                   rtol=1e-11, atol=1e-12)
+
+
+def test_decode_step_page_table_permutation_invariance():
+    # the same logical cache stored under a permuted page table gives the same result
+    prob, Hq, Hkv, d, r = _tiny_problem(12, page_perm=False)
+    cfg = O.OracleConfig(Hq, Hkv, d, r, 16, [1, 1, 0, 0], 8, 2, "top_p", top_p=0.7)
+    a = O.decode_reference(cfg, **prob)
+    rng = np.random.default_rng(0)
+    total = prob["k_cache"].shape[0]
+    perm = rng.permutation(total)           # new physical location of old page i
+    kc = np.empty_like(prob["k_cache"]); kc[perm] = prob["k_cache"]
+    vc = np.empty_like(prob["v_cache"]); vc[perm] = prob["v_cache"]
+    pt = prob["page_table"].copy()
+    pt[pt >= 0] = perm[pt[pt >= 0]]
+    b_ = O.decode_reference(cfg, **{**prob, "k_cache": kc, "v_cache": vc, "page_table": pt})
+    for key in a.out:
+        np.testing.assert_array_equal(a.out[key], b_.out[key])
+    for key in a.sets:
+        np.testing.assert_array_equal(a.sets[key], b_.sets[key])
+
+
+def test_widen_accepts_bf16_bit_patterns():
+    x = O.bf16_round(np.random.default_rng(9).standard_normal(100))
+    bits = _bf16_bits(x.astype(np.float32)).astype(np.uint16)
+    np.testing.assert_array_equal(O.widen(bits), x)
