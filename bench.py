@@ -1,0 +1,498 @@
+"""Decode-step benchmark of head-wise sparse attention on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload topk_128k]
+
+A step is one pass of the whole decode path over one batch: index_keys for
+the B appended tokens, select (index scoring + top-k / top-p) and attend
+(gathered retrieval rows, sinks + window for local heads, split merge).  The
+default workload is the 128K-context fixed-budget decode: 16 sequences of
+131072 tokens, 32 q / 8 KV heads, d = 128, all heads retrieval with top-k 2%
+(2621 tokens per head).  Inputs are synthetic and seeded; each rank runs its
+own batch (weak scaling, no collective on the data path).
+
+Rank 0 prints one JSON line.  `value` is whole-job head-steps/s (one
+head-step = one (sequence, q head) output of one decode step), timed with
+CUDA events over K steps after W warm-up steps, max over ranks.  The touched
+bytes per step (~1.2 GB) exceed the 126 MB L2, so no flush is needed between
+steps.  `--impl reference` times the float64 CPU oracle on the host cores on
+a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "sparse decode head-steps/s and achieved HBM GB/s vs 8 TB/s at 128K ctx"
+UNIT = "head-steps/s"
+CONTRACT_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ---------------------------------------------------------------- rank plumbing
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Each rank draws its own batch (weak scaling)."""
+    return base + 7919 * rank
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed
+    region (200 ms period)."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- measurements
+
+def load_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+KERNEL_SOURCES = {
+    "select": ["head_wise_sparse_02_b200/csrc/sd_select.cu", "head_wise_sparse_02_b200/csrc/sd_internal.cuh"],
+    "attend": ["head_wise_sparse_02_b200/csrc/sd_attend.cu", "head_wise_sparse_02_b200/csrc/sd_internal.cuh"],
+    "index_keys": ["head_wise_sparse_02_b200/csrc/sd_index.cu", "head_wise_sparse_02_b200/csrc/sd_internal.cuh"],
+}
+
+
+def ncu_traffic(kernel: str, workload: str, units: float):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source (else None).  The summary stores bytes per unit
+    of work so that a capture on a smaller case scales to this launch."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        e = d[kernel]
+        if e.get("source_hash") != kernel_source_hash(KERNEL_SOURCES[kernel]):
+            return None
+        return float(e["dram_bytes_per_unit"]) * units
+    except Exception:
+        return None
+
+
+def union_rows(sel_idx, sel_count, w):
+    """Distinct K/V rows each (sequence, KV group) reads: union over the
+    group's retrieval heads plus the local set of its local heads."""
+    import torch
+    G = w.num_q_heads // w.num_kv_heads
+    rows = {}
+    r = 0
+    ret_rows = {}
+    for h in range(w.num_q_heads):
+        if w.head_is_retrieval[h]:
+            ret_rows[h] = r
+            r += 1
+    cnt = sel_count.cpu()
+    lens = w.seq_lens.cpu().tolist()
+    total = 0
+    index_tokens = 0
+    for b in range(w.batch):
+        n = lens[b]
+        for g in range(w.num_kv_heads):
+            heads = range(g * G, (g + 1) * G)
+            parts = []
+            has_ret = False
+            has_loc = False
+            for h in heads:
+                if w.head_is_retrieval[h]:
+                    has_ret = True
+                    k = int(cnt[b, ret_rows[h]])
+                    parts.append(sel_idx[b, ret_rows[h], :k])
+                else:
+                    has_loc = True
+            if has_loc:
+                a = min(w.num_sinks, n)
+                ws_ = max(a, n - w.window)
+                parts.append(torch.arange(0, a, device=sel_idx.device, dtype=torch.int32))
+                parts.append(torch.arange(ws_, n, device=sel_idx.device, dtype=torch.int32))
+            if parts:
+                total += int(torch.unique(torch.cat(parts)).numel())
+            if has_ret:
+                index_tokens += n
+    return total, index_tokens
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from head_wise_sparse_02_b200.decode import DecodeStep
+    from workloads import keys_at, make_workload, slots_of
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    w = make_workload(args.workload, dev, seed=rank_seed(args.seed, rank))
+    B, Hq, d = w.batch, w.num_q_heads, w.head_dim
+    st = DecodeStep(k_cache=w.k_cache, v_cache=w.v_cache, page_table=w.page_table, seq_lens=w.seq_lens,
+                    proj=w.proj, num_q_heads=Hq, head_is_retrieval=w.head_is_retrieval, window=w.window,
+                    num_sinks=w.num_sinks, mode=w.mode, top_p=w.top_p, top_k=w.top_k,
+                    top_k_frac=w.top_k_frac)
+    slots_all = slots_of(w)
+    st.build_index(slots_all, keys_at(w, slots_all))          # prefill-time index (setup, untimed)
+    # per step: the appended token of every sequence is position N_b - 1
+    lens = w.seq_lens.long()
+    new_slots = (w.page_table[torch.arange(B, device=dev), (lens - 1) // 16].long() * 16 + (lens - 1) % 16).to(torch.int32)
+    new_keys = keys_at(w, new_slots)
+    stream = torch.cuda.current_stream()
+
+    ev = {k: [] for k in ("index_keys", "select", "attend")}
+
+    def step(record=False):
+        if record:
+            e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
+            e2 = torch.cuda.Event(enable_timing=True); e3 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        st.sd.index_keys(new_keys, new_slots, st.index_cache, stream)
+        if record:
+            e1.record(stream)
+        st.select(w.q_pre, stream)
+        if record:
+            e2.record(stream)
+        st.attend(w.q, stream=stream)
+        if record:
+            e3.record(stream)
+            ev["index_keys"].append((e0, e1)); ev["select"].append((e1, e2)); ev["attend"].append((e2, e3))
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    word = st.error_word()
+    if word:
+        raise RuntimeError(f"device error word {word:#x} after warm-up")
+    rows, index_tokens = union_rows(st.sel_idx, st.sel_count, w)
+    sel_sizes = st.sel_count.float()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True); t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step(record=True)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms = t0.elapsed_time(t1) / args.steps
+    ms_max = max_over_ranks(ms, dev)
+    per = {k: sum(a.elapsed_time(b) for a, b in v) / len(v) for k, v in ev.items()}
+
+    # ---- end to end through the public API with host buffers ----
+    q_h = w.q.cpu().pin_memory()
+    qp_h = w.q_pre.cpu().pin_memory()
+    nk_h = new_keys.cpu().pin_memory()
+    ns_h = new_slots.cpu().pin_memory()
+    out_h = torch.empty(st.out.shape, dtype=torch.float32).pin_memory()
+    q_d, qp_d = torch.empty_like(w.q), torch.empty_like(w.q_pre)
+    nk_d, ns_d = torch.empty_like(new_keys), torch.empty_like(new_slots)
+
+    def e2e_step():
+        q_d.copy_(q_h, non_blocking=True); qp_d.copy_(qp_h, non_blocking=True)
+        nk_d.copy_(nk_h, non_blocking=True); ns_d.copy_(ns_h, non_blocking=True)
+        st.sd.index_keys(nk_d, ns_d, st.index_cache, stream)
+        st.select(qp_d, stream)
+        st.attend(q_d, stream=stream)
+        out_h.copy_(st.out, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    a0 = torch.cuda.Event(enable_timing=True); a1 = torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    a1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(a0.elapsed_time(a1) / args.steps, dev)
+    word = st.error_word()
+    if word:
+        raise RuntimeError(f"device error word {word:#x} after timing")
+
+    # ---- roofline of the dominant kernel ----
+    row_bytes = 4 * d                                   # K + V row, bf16
+    index_bytes = 32 * index_tokens
+    kv_bytes = row_bytes * rows
+    kern_bytes = {"select": index_bytes, "attend": kv_bytes, "index_keys": B * w.num_kv_heads * (2 * d + 32)}
+    dominant = max(per, key=per.get)
+    peak, peak_kind = load_peak()
+    achieved = kern_bytes[dominant] / (per[dominant] * 1e-3) / 1e9
+    units = {"select": index_tokens, "attend": rows, "index_keys": B}[dominant]
+    step_bytes = index_bytes + kv_bytes
+    head_steps = ws * B * Hq
+    value = head_steps / (ms_max * 1e-3)
+    res = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_max, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "storage_dtype": "bf16",
+        "data": "synthetic (seeded; no datasets or trained weights)",
+        "config": {
+            "workload": f"{args.workload}: B={B}, Hq={Hq}/Hkv={w.num_kv_heads}, d={d}, "
+                        f"N={int(w.seq_lens.max())}, mode={w.mode}"
+                        + (f", top-k frac {w.top_k_frac}" if w.mode == "top_k" else f", top-p {w.top_p}"),
+            "batch_per_gpu": B, "seq_len": int(w.seq_lens.max()), "parallelism": f"replicas x{ws} (sequences sharded, no collective)",
+            "l2": "no flush: bytes touched per step exceed the 126 MB L2",
+        },
+        "tokens_per_s": round(ws * B / (ms_max * 1e-3), 1),
+        "hbm_gbs_achieved_step": round(step_bytes / (ms * 1e-3) / 1e9, 1),
+        "frac_of_8tbs_step": round(step_bytes / (ms * 1e-3) / 1e9 / CONTRACT_GBS, 4),
+        "algorithmic_bytes_per_step": step_bytes,
+        "ms_per_call": {k: round(v, 4) for k, v in per.items()},
+        "selected_per_head": {"mean": round(float(sel_sizes.mean()), 1), "min": int(sel_sizes.min()),
+                              "max": int(sel_sizes.max())},
+        "roofline": {"kernel": dominant, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                     "peak_kind": f"{peak_kind} hbm_gbs (copy bandwidth)", "unit": "GB/s",
+                     "frac": round(achieved / peak, 4),
+                     "algorithmic_bytes_per_launch": kern_bytes[dominant],
+                     "traffic": ncu_traffic(dominant, args.workload, units)},
+        "e2e": {"value": round(head_steps / (e2e_ms * 1e-3), 1), "unit": UNIT,
+                "h2d_bytes_per_step": int(q_h.numel() * 2 + qp_h.numel() * 2 + nk_h.numel() * 2 + ns_h.numel() * 4),
+                "d2h_bytes_per_step": int(out_h.numel() * 4)},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
+    st.close()
+    if ws > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+# ---------------------------------------------------------------- oracle legs
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return len(os.sched_getaffinity(0))
+
+
+def oracle_slab_step(inp, cfg, b, g, index_g):
+    """One decode step of the oracle for the heads of KV group g of sequence
+    b, with the slab's index already built (as the GPU's index cache is)."""
+    import numpy as np
+
+    import oracle as O
+    G = cfg.num_q_heads // cfg.num_kv_heads
+    n = int(inp["seq_lens"][b])
+    attn_scale, index_scale = cfg.scales()
+    K = O.gather_rows(inp["k_cache"], inp["page_table"][b], n, g, cfg.page_size)
+    V = O.gather_rows(inp["v_cache"], inp["page_table"][b], n, g, cfg.page_size)
+    O.index_keys(inp["proj"][g], K[n - 1:n])                 # the appended token
+    outs = []
+    for h in range(g * G, (g + 1) * G):
+        if cfg.head_is_retrieval[h]:
+            s = O.index_scores(O.query_index(inp["proj"][g], inp["q_pre"][b, h]), index_g, index_scale)
+            S = (O.select_top_p(s, cfg.top_p) if cfg.mode == "top_p"
+                 else O.select_top_k(s, O.top_k_budget(n, cfg.top_k, cfg.top_k_frac)))
+        else:
+            S = O.local_positions(n, cfg.window, cfg.num_sinks)
+        outs.append(O.attend_set(inp["q"][b, h], K, V, S, attn_scale))
+    return np.stack(outs)
+
+
+def cpu_baseline(w, budget_s=15.0):
+    """Time the oracle as it stands on (b, KV group) slabs of the workload
+    until ~budget_s of CPU work; head-steps/s over the slabs processed."""
+    import numpy as np
+
+    import oracle as O
+    from tests.helpers import oracle_config, oracle_inputs
+    cfg = oracle_config(w)
+    G = w.num_q_heads // w.num_kv_heads
+    done = 0
+    elapsed = 0.0
+    slabs = []
+    b = 0
+    while elapsed < budget_s and b < w.batch:
+        inp = oracle_inputs(w, [b])
+        n = int(inp["seq_lens"][0])
+        for g in range(w.num_kv_heads):
+            K = O.gather_rows(inp["k_cache"], inp["page_table"][0], n, g, cfg.page_size)
+            index_g = O.index_keys(inp["proj"][g], K)          # setup (prefill), untimed
+            t = time.perf_counter()
+            oracle_slab_step(inp, cfg, 0, g, index_g)
+            elapsed += time.perf_counter() - t
+            done += G
+            slabs.append((b, g))
+            if elapsed >= budget_s:
+                break
+        b += 1
+    return {"value": round(done / elapsed, 3), "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{len(slabs)} (sequence, KV group) slabs = {done} head-steps of the same workload, "
+                      f"float64 numpy oracle, index prebuilt (untimed) as on the GPU; {elapsed:.1f} s"}
+
+
+def run_reference(args):
+    ws, rank, local = dist_env()
+    if rank != 0:
+        return
+    import torch
+
+    from tests.helpers import oracle_config, oracle_inputs
+    from workloads import make_workload
+    import oracle as O
+    dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
+    w = make_workload(args.workload, dev, seed=rank_seed(args.seed, 0))
+    cfg = oracle_config(w)
+    G = w.num_q_heads // w.num_kv_heads
+    inp = oracle_inputs(w, [0])
+    n = int(inp["seq_lens"][0])
+    idx = {}
+    for g in range(w.num_kv_heads):
+        K = O.gather_rows(inp["k_cache"], inp["page_table"][0], n, g, cfg.page_size)
+        idx[g] = O.index_keys(inp["proj"][g], K)
+    # each step: one (sequence, KV group) slab = G head-steps
+    for i in range(args.warmup):
+        oracle_slab_step(inp, cfg, 0, i % w.num_kv_heads, idx[i % w.num_kv_heads])
+    t = time.perf_counter()
+    for i in range(args.steps):
+        oracle_slab_step(inp, cfg, 0, i % w.num_kv_heads, idx[i % w.num_kv_heads])
+    el = time.perf_counter() - t
+    v = G * args.steps / el
+    res = {"impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": UNIT, "n_gpus": ws,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic (seeded)",
+           "config": {"workload": f"{args.workload}: B={w.batch}, Hq={w.num_q_heads}/Hkv={w.num_kv_heads}, "
+                                  f"d={w.head_dim}, N={int(w.seq_lens.max())}",
+                      "step_sample": f"one (sequence, KV group) slab = {G} head-steps per step"},
+           "cpu_baseline": {"kind": "oracle", "cores": _blas_threads(), "value": round(v, 3), "unit": UNIT,
+                            "sample": f"{args.steps} slabs of {G} heads, float64 numpy oracle"},
+           "e2e": {"value": round(v, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="topk_128k")
+    ap.add_argument("--seed", type=int, default=2)
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    args.warmup = max(args.warmup, 3)          # timing rule: at least 3 warm-up steps
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

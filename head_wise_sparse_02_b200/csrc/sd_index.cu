@@ -1,0 +1,82 @@
+// Index keys: k~ = bf16_rne(P_g^T k_pre) for newly cached tokens.
+//
+// RTPurbo page (gist.science/ar/paper/2605.16928), Methodology 2: retrieval
+// heads estimate relevance in an r = 16 dimensional space obtained by
+// projecting pre-RoPE keys (and queries).  The index entry of a token is the
+// projection of its key, stored as bf16 (32 bytes per token and KV head).
+//
+// Accumulation is float64: every product of two bf16 values is exact in
+// float64 and the running sum is rounded at 2^-53, so the single final
+// rounding to bf16 (round to nearest even, from the float64 value) agrees with
+// rounding the exact dot product except when that exact value lies within
+// ~2^-45 relative of a bf16 rounding midpoint.
+#include "sd_internal.cuh"
+
+namespace sd {
+namespace {
+
+constexpr int kRows = 16;          // (token) rows per block, one KV head per block
+constexpr int kThreads = kRows * kIndexDim;
+
+// float64 -> bf16 bits, round to nearest even, from the float64 value itself.
+__device__ __forceinline__ uint16_t f64_to_bf16_rne(double x) {
+  if (isnan(x)) return 0x7FC0u;
+  const uint16_t sign = (__double_as_longlong(x) < 0) ? 0x8000u : 0u;
+  const double a = fabs(x);
+  if (a == 0.0) return sign;
+  int e;
+  frexp(a, &e);                                  // a = m * 2^e, 0.5 <= m < 1
+  const int q = max(e - 8, -133);                // bf16 quantum (subnormal floor 2^-133)
+  const double r = rint(ldexp(a, -q));           // exact scaling, ties to even
+  const float y = (float)ldexp(r, q);            // exactly representable, or +inf on overflow
+  return sign | (uint16_t)(__float_as_uint(y) >> 16);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads)
+index_keys_kernel(const uint16_t *__restrict__ k_pre, const int32_t *__restrict__ slots, int T,
+                  uint16_t *__restrict__ index_cache, const uint16_t *__restrict__ proj, int Hkv,
+                  int num_pages, unsigned *err) {
+  __shared__ double Ps[D][kIndexDim];
+  __shared__ double Ks[kRows][D + 1];
+  const int g = blockIdx.y;
+  const int t0 = blockIdx.x * kRows;
+  const uint16_t *P = proj + (size_t)g * D * kIndexDim;
+  for (int i = threadIdx.x; i < D * kIndexDim; i += kThreads)
+    Ps[i / kIndexDim][i % kIndexDim] = (double)bf16_to_f32(P[i]);
+  for (int i = threadIdx.x; i < kRows * D; i += kThreads) {
+    const int row = i / D, c = i % D, t = t0 + row;
+    Ks[row][c] = (t < T) ? (double)bf16_to_f32(k_pre[((size_t)t * Hkv + g) * D + c]) : 0.0;
+  }
+  __syncthreads();
+  const int row = threadIdx.x / kIndexDim, j = threadIdx.x % kIndexDim;
+  const int t = t0 + row;
+  if (t >= T) return;
+  double acc = 0.0;
+#pragma unroll 8
+  for (int i = 0; i < D; ++i) acc = fma(Ks[row][i], Ps[i][j], acc);
+  const long long slot = slots[t];
+  if (slot < 0 || slot >= (long long)num_pages * kPage) {
+    if (j == 0) raise_error(err, SD_EBIT_SLOT);
+    return;
+  }
+  const long long page = slot / kPage, off = slot % kPage;
+  index_cache[((page * Hkv + g) * kPage + off) * kIndexDim + j] = f64_to_bf16_rne(acc);
+}
+
+}  // namespace
+
+cudaError_t launch_index_keys(const uint16_t *k_pre, const int32_t *slots, int T, uint16_t *index_cache,
+                              const uint16_t *proj, const Shape &sh, unsigned *err, cudaStream_t st) {
+  if (T <= 0) return cudaSuccess;
+  dim3 grid((T + kRows - 1) / kRows, sh.Hkv);
+  if (sh.d == 128)
+    index_keys_kernel<128><<<grid, kThreads, 0, st>>>(k_pre, slots, T, index_cache, proj, sh.Hkv,
+                                                      sh.num_pages, err);
+  else
+    index_keys_kernel<64><<<grid, kThreads, 0, st>>>(k_pre, slots, T, index_cache, proj, sh.Hkv,
+                                                     sh.num_pages, err);
+  return cudaGetLastError();
+}
+
+}  // namespace sd

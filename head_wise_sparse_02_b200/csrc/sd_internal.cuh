@@ -1,0 +1,106 @@
+// Internal declarations of the sparse decode library (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "sparse_decode.h"
+
+namespace sd {
+
+constexpr int kMaxGroup = 16;     // q heads per KV head (GQA group) supported
+constexpr int kIndexDim = 16;     // r
+constexpr int kPage = 16;         // tokens per page
+
+// One KV head's heads of one role (retrieval or local).
+struct Group {
+  int kv_head;
+  int n;                          // heads of this role in the group
+  int q_head[kMaxGroup];          // their q-head ids, ascending
+  int row[kMaxGroup];             // retrieval: row in sel_idx (rank among retrieval heads)
+};
+
+// Device-side view of a context's tables.
+struct Tables {
+  const Group *ret;               // [n_ret] groups with >= 1 retrieval head
+  const Group *loc;               // [n_loc] groups with >= 1 local head
+  int n_ret, n_loc;
+  int max_ret;                    // largest n over ret groups
+  int max_loc;                    // largest n over loc groups
+};
+
+struct Shape {
+  int Hq, Hkv, d, num_pages, max_pages, H_ret;
+  long long max_len;              // max_pages * kPage
+};
+
+// ----------------------------------------------------------------- helpers
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+__device__ __forceinline__ float bf16_to_f32(uint16_t h) { return __uint_as_float(uint32_t(h) << 16); }
+
+// Order-preserving map of a float to an unsigned key (-0 folded onto +0).
+__device__ __forceinline__ uint32_t order_key(float f) {
+  uint32_t u = __float_as_uint(__fadd_rn(f, 0.0f));
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_to_float(uint32_t k) {
+  uint32_t u = (k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k;
+  return __uint_as_float(u);
+}
+
+__device__ __forceinline__ void raise_error(unsigned *err, unsigned bit) {
+  if (err) atomicOr(err, bit);
+}
+
+// ---------------------------------------------------------------- launchers
+// Each returns cudaSuccess or the launch error.
+
+cudaError_t launch_index_keys(const uint16_t *k_pre, const int32_t *slots, int T, uint16_t *index_cache,
+                              const uint16_t *proj, const Shape &sh, unsigned *err, cudaStream_t st);
+
+struct SelectArgs {
+  const uint16_t *q_pre;
+  const uint16_t *index_cache;
+  const int32_t *page_table;
+  const int32_t *seq_lens;
+  int32_t *sel_idx;
+  int32_t *sel_count;
+  long long sel_stride;
+  const uint16_t *proj;
+  float index_scale;
+  int mode;
+  float top_p;
+  int top_k;
+  float top_k_frac;
+  float *score_ws;                // global score rows when they do not fit on chip
+  unsigned *err;
+  int batch;
+};
+
+size_t select_workspace_bytes(const Shape &sh, const Tables &tb, int batch);
+cudaError_t launch_select(const SelectArgs &a, const Shape &sh, const Tables &tb, cudaStream_t st);
+
+struct AttendArgs {
+  const uint16_t *q;
+  const uint16_t *k_cache;
+  const uint16_t *v_cache;
+  const int32_t *page_table;
+  const int32_t *seq_lens;
+  const int32_t *sel_idx;
+  const int32_t *sel_count;
+  long long sel_stride;
+  float *out;
+  float attn_scale;
+  int window, num_sinks;
+  float *partials;
+  unsigned *tickets;
+  unsigned *err;
+  int batch;
+};
+
+size_t attend_workspace_bytes(const Shape &sh, const Tables &tb, int batch, size_t *tickets_off);
+cudaError_t launch_attend(const AttendArgs &a, const Shape &sh, const Tables &tb, cudaStream_t st);
+
+}  // namespace sd

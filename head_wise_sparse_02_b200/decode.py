@@ -1,0 +1,70 @@
+"""One decode step wired through the C ABI: index_keys for the appended
+tokens, select, attend.  Torch is used only to hold device buffers."""
+
+from __future__ import annotations
+
+from typing import Optional, Sequence
+
+import torch
+
+from .sparse_decode import SparseDecode
+
+
+class DecodeStep:
+    """Holds a context, the index cache and the per-batch buffers of one layer.
+
+    k_cache / v_cache: bf16 [num_pages, Hkv, 16, d]; page_table int32 [B, MAXP];
+    seq_lens int32 [B]; proj bf16 [Hkv, d, 16].
+    """
+
+    def __init__(self, *, k_cache: torch.Tensor, v_cache: torch.Tensor, page_table: torch.Tensor,
+                 seq_lens: torch.Tensor, proj: torch.Tensor, num_q_heads: int,
+                 head_is_retrieval: Sequence[int], window: int, num_sinks: int, mode: str,
+                 top_p: float = 0.9, top_k: int = 0, top_k_frac: float = 0.0,
+                 attn_scale: float = 0.0, index_scale: float = 0.0,
+                 index_cache: Optional[torch.Tensor] = None):
+        num_pages, Hkv, page, d = k_cache.shape
+        self.k_cache, self.v_cache = k_cache, v_cache
+        self.page_table, self.seq_lens = page_table, seq_lens
+        self.batch = int(seq_lens.shape[0])
+        self.num_q_heads, self.head_dim = num_q_heads, d
+        self.sd = SparseDecode(num_q_heads=num_q_heads, num_kv_heads=Hkv, head_dim=d,
+                               head_is_retrieval=list(head_is_retrieval), num_pages=num_pages,
+                               max_batch=self.batch, max_pages_per_seq=int(page_table.shape[1]),
+                               proj=proj, window=window, num_sinks=num_sinks, mode=mode,
+                               top_p=top_p, top_k=top_k, top_k_frac=top_k_frac,
+                               attn_scale=attn_scale, index_scale=index_scale)
+        dev = k_cache.device
+        self.index_cache = index_cache if index_cache is not None else torch.zeros(
+            (num_pages, Hkv, page, 16), dtype=torch.bfloat16, device=dev)
+        self.workspace, self.sel_idx, self.sel_count = self.sd.alloc(self.batch)
+        self.out = torch.empty((self.batch, num_q_heads, d), dtype=torch.float32, device=dev)
+
+    def build_index(self, slots: torch.Tensor, keys: torch.Tensor, stream=None):
+        """index_keys over the given slots (e.g. every cached position at setup)."""
+        self.sd.index_keys(keys, slots, self.index_cache, stream)
+
+    def select(self, q_pre: torch.Tensor, stream=None):
+        self.sd.select(q_pre, self.index_cache, self.page_table, self.seq_lens, self.sel_idx,
+                       self.sel_count, self.workspace, stream)
+
+    def attend(self, q: torch.Tensor, sel_idx=None, sel_count=None, stream=None):
+        self.sd.attend(q, self.k_cache, self.v_cache, self.page_table, self.seq_lens,
+                       self.sel_idx if sel_idx is None else sel_idx,
+                       self.sel_count if sel_count is None else sel_count,
+                       self.out, self.workspace, stream)
+        return self.out
+
+    def step(self, q_pre: torch.Tensor, q: torch.Tensor, new_keys: Optional[torch.Tensor] = None,
+             new_slots: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """One decode step: index the appended tokens, select, attend."""
+        if new_keys is not None:
+            self.sd.index_keys(new_keys, new_slots, self.index_cache, stream)
+        self.select(q_pre, stream)
+        return self.attend(q, stream=stream)
+
+    def error_word(self, stream=None) -> int:
+        return self.sd.error_word(stream)
+
+    def close(self):
+        self.sd.close()

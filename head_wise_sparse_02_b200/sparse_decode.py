@@ -1,0 +1,235 @@
+"""Thin ctypes binding of libsparsedecode.so (see include/sparse_decode.h).
+
+Argument marshalling only: every step of the decode path runs in the CUDA
+library.  Functions carry the C names and take torch tensors (for device
+memory and streams); they check dtype, device and contiguity, pass raw
+pointers and raise :class:`SparseDecodeError` on a non-zero status.  There is
+no fallback: if the library is missing or fails to load, importing this
+module raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import POINTER, c_char_p, c_float, c_int, c_int32, c_size_t, c_uint32, c_void_p
+from typing import Optional, Sequence
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libsparsedecode.so")
+
+SD_OK, SD_ERR_INVALID_ARG, SD_ERR_UNSUPPORTED, SD_ERR_WORKSPACE, SD_ERR_CUDA, SD_ERR_TIMEOUT, \
+    SD_ERR_DEVICE_DATA = range(7)
+SD_TOP_P, SD_TOP_K = 0, 1
+SD_EBIT_PAGE, SD_EBIT_SEQLEN, SD_EBIT_SEL, SD_EBIT_SLOT, SD_EBIT_TIMEOUT = 1, 2, 4, 8, 16
+
+
+class SparseDecodeError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{message} (status {status})")
+        self.status = status
+
+
+class SdConfig(ctypes.Structure):
+    _fields_ = [
+        ("num_q_heads", c_int), ("num_kv_heads", c_int), ("head_dim", c_int), ("index_dim", c_int),
+        ("page_size", c_int), ("num_pages", c_int), ("head_is_retrieval", POINTER(c_int32)),
+        ("window", c_int), ("num_sinks", c_int), ("mode", c_int), ("top_p", c_float),
+        ("top_k", c_int), ("top_k_frac", c_float), ("attn_scale", c_float),
+        ("index_scale", c_float), ("max_batch", c_int), ("max_pages_per_seq", c_int),
+    ]
+
+
+def _load(path: str = LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with `python -m head_wise_sparse_02_b200.build`")
+    lib = ctypes.CDLL(path)
+    P = c_void_p
+    sig = {
+        "sparse_decode_init": (c_int, [POINTER(SdConfig), P, POINTER(P)]),
+        "sparse_decode_workspace_size": (c_int, [P, c_int, POINTER(c_size_t)]),
+        "sparse_decode_index_keys": (c_int, [P, P, P, c_int, P, P]),
+        "sparse_decode_select": (c_int, [P, P, P, P, P, c_int, P, P, c_int, P, c_size_t, P]),
+        "sparse_decode_attend": (c_int, [P, P, P, P, P, P, c_int, P, P, c_int, P, P, c_size_t, P]),
+        "sparse_decode_error_word": (c_int, [P, P, POINTER(c_uint32)]),
+        "sparse_decode_num_retrieval_heads": (c_int, [P]),
+        "sparse_decode_last_error": (c_char_p, [P]),
+        "sparse_decode_status_string": (c_char_p, [c_int]),
+        "sparse_decode_destroy": (None, [P]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+LIB = _load()
+
+
+def status_string(status: int) -> str:
+    return LIB.sparse_decode_status_string(status).decode()
+
+
+def _check(status: int, ctx: Optional[int] = None) -> None:
+    if status != SD_OK:
+        msg = status_string(status)
+        if ctx:
+            detail = LIB.sparse_decode_last_error(ctx).decode()
+            if detail:
+                msg = f"{msg}: {detail}"
+        raise SparseDecodeError(status, msg)
+
+
+def _ptr(t: Optional[torch.Tensor], dtype: torch.dtype, name: str) -> Optional[int]:
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+# ------------------------------------------------------------ C-named calls
+
+def sparse_decode_init(*, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                       head_is_retrieval: Sequence[int], num_pages: int, max_batch: int,
+                       max_pages_per_seq: int, proj: torch.Tensor, window: int = 0,
+                       num_sinks: int = 0, mode: str = "top_p", top_p: float = 0.9,
+                       top_k: int = 0, top_k_frac: float = 0.0, attn_scale: float = 0.0,
+                       index_scale: float = 0.0, index_dim: int = 16, page_size: int = 16) -> int:
+    """Create a context (returns the opaque handle)."""
+    retr = (c_int32 * num_q_heads)(*[int(x) for x in head_is_retrieval])
+    cfg = SdConfig(num_q_heads, num_kv_heads, head_dim, index_dim, page_size, num_pages,
+                   ctypes.cast(retr, POINTER(c_int32)), window, num_sinks,
+                   SD_TOP_P if mode == "top_p" else SD_TOP_K, top_p, top_k, top_k_frac,
+                   attn_scale, index_scale, max_batch, max_pages_per_seq)
+    out = c_void_p()
+    with torch.cuda.device(proj.device):
+        _check(LIB.sparse_decode_init(ctypes.byref(cfg), _ptr(proj, torch.bfloat16, "proj"), ctypes.byref(out)))
+    return out.value
+
+
+def sparse_decode_workspace_size(ctx: int, batch: int) -> int:
+    n = c_size_t()
+    _check(LIB.sparse_decode_workspace_size(ctx, batch, ctypes.byref(n)), ctx)
+    return n.value
+
+
+def sparse_decode_index_keys(ctx: int, k_pre: torch.Tensor, slots: torch.Tensor,
+                             index_cache: torch.Tensor, stream=None) -> None:
+    _check(LIB.sparse_decode_index_keys(ctx, _ptr(k_pre, torch.bfloat16, "k_pre"),
+                                        _ptr(slots, torch.int32, "slots"), int(slots.numel()),
+                                        _ptr(index_cache, torch.bfloat16, "index_cache"),
+                                        _stream(stream)), ctx)
+
+
+def sparse_decode_select(ctx: int, q_pre, index_cache, page_table, seq_lens, sel_idx, sel_count,
+                         workspace, stream=None) -> None:
+    _check(LIB.sparse_decode_select(
+        ctx, _ptr(q_pre, torch.bfloat16, "q_pre"), _ptr(index_cache, torch.bfloat16, "index_cache"),
+        _ptr(page_table, torch.int32, "page_table"), _ptr(seq_lens, torch.int32, "seq_lens"),
+        int(seq_lens.numel()), _ptr(sel_idx, torch.int32, "sel_idx"),
+        _ptr(sel_count, torch.int32, "sel_count"), int(sel_idx.shape[-1]),
+        _ptr(workspace, torch.uint8, "workspace"), int(workspace.numel()), _stream(stream)), ctx)
+
+
+def sparse_decode_attend(ctx: int, q, k_cache, v_cache, page_table, seq_lens, sel_idx, sel_count,
+                         out, workspace, stream=None) -> None:
+    stride = int(sel_idx.shape[-1]) if sel_idx is not None else 0
+    _check(LIB.sparse_decode_attend(
+        ctx, _ptr(q, torch.bfloat16, "q"), _ptr(k_cache, torch.bfloat16, "k_cache"),
+        _ptr(v_cache, torch.bfloat16, "v_cache"), _ptr(page_table, torch.int32, "page_table"),
+        _ptr(seq_lens, torch.int32, "seq_lens"), int(seq_lens.numel()),
+        _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_count, torch.int32, "sel_count"), stride,
+        _ptr(out, torch.float32, "out"), _ptr(workspace, torch.uint8, "workspace"),
+        int(workspace.numel()), _stream(stream)), ctx)
+
+
+def sparse_decode_error_word(ctx: int, stream=None) -> int:
+    """Wait for the stream, read and clear the device error word (0 = clean)."""
+    w = c_uint32()
+    st = LIB.sparse_decode_error_word(ctx, _stream(stream), ctypes.byref(w))
+    if st not in (SD_OK, SD_ERR_DEVICE_DATA, SD_ERR_TIMEOUT):
+        _check(st, ctx)
+    return int(w.value)
+
+
+def sparse_decode_num_retrieval_heads(ctx: int) -> int:
+    return int(LIB.sparse_decode_num_retrieval_heads(ctx))
+
+
+def sparse_decode_destroy(ctx: int) -> None:
+    LIB.sparse_decode_destroy(ctx)
+
+
+# ------------------------------------------------------------ convenience
+
+class SparseDecode:
+    """Owns one context; methods forward to the C-named calls above."""
+
+    def __init__(self, **cfg):
+        self.cfg = dict(cfg)
+        self.handle = sparse_decode_init(**cfg)
+        self.num_retrieval_heads = sparse_decode_num_retrieval_heads(self.handle)
+        self.device = cfg["proj"].device
+        self.max_len = cfg["max_pages_per_seq"] * cfg.get("page_size", 16)
+
+    def close(self):
+        if self.handle:
+            sparse_decode_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def workspace_size(self, batch: int) -> int:
+        return sparse_decode_workspace_size(self.handle, batch)
+
+    def sel_stride(self) -> int:
+        if self.cfg.get("mode", "top_p") == "top_p":
+            return self.max_len
+        k = self.cfg.get("top_k", 0)
+        if k > 0:
+            return min(k, self.max_len)
+        import math
+        import numpy as np
+        return min(self.max_len, max(1, math.floor(float(np.float32(self.cfg["top_k_frac"])) * self.max_len)))
+
+    def alloc(self, batch: int):
+        """Workspace, selection rows and counts for `batch` sequences."""
+        ws = torch.empty(self.workspace_size(batch), dtype=torch.uint8, device=self.device)
+        h = max(1, self.num_retrieval_heads)
+        sel = torch.empty((batch, h, self.sel_stride()), dtype=torch.int32, device=self.device)
+        cnt = torch.zeros((batch, h), dtype=torch.int32, device=self.device)
+        return ws, sel, cnt
+
+    def index_keys(self, k_pre, slots, index_cache, stream=None):
+        sparse_decode_index_keys(self.handle, k_pre, slots, index_cache, stream)
+
+    def select(self, q_pre, index_cache, page_table, seq_lens, sel_idx, sel_count, workspace, stream=None):
+        sparse_decode_select(self.handle, q_pre, index_cache, page_table, seq_lens, sel_idx, sel_count,
+                             workspace, stream)
+
+    def attend(self, q, k_cache, v_cache, page_table, seq_lens, sel_idx, sel_count, out, workspace,
+               stream=None):
+        sparse_decode_attend(self.handle, q, k_cache, v_cache, page_table, seq_lens, sel_idx, sel_count,
+                             out, workspace, stream)
+
+    def error_word(self, stream=None) -> int:
+        return sparse_decode_error_word(self.handle, stream)

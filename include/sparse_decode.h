@@ -1,0 +1,277 @@
+/*
+ * sparse_decode.h -- C ABI of the head-wise sparse decode attention library
+ * (libsparsedecode.so, sm_100a).
+ *
+ * One decode step of one attention layer, for a batch of sequences whose
+ * keys and values live in a paged bf16 cache:
+ *
+ *   retrieval heads  score every cached token in an r = 16 dimensional index
+ *                    space built from pre-RoPE keys, keep a per-(sequence,
+ *                    head) token set by dynamic top-p or fixed top-k, and run
+ *                    exact softmax attention over the kept rows only;
+ *   local heads      attend to a few sink tokens plus a recent window.
+ *
+ * Sources (gist.science summary pages):
+ *   RTPurbo page  "Full attention strikes back: moving full attention to sparse
+ *                 attention within hundreds of training steps",
+ *                 gist.science/ar/paper/2605.16928, Methodology 1 (retrieval vs
+ *                 local heads; local heads use a sliding window with attention
+ *                 sinks, retrieval heads keep the full KV and select sparsely at
+ *                 decode), 2 (r << d, r = 16, projection of pre-RoPE q and k),
+ *                 3 (dynamic top-p: accumulate low-dimensional attention mass to
+ *                 the cumulative threshold p, e.g. 0.9; fixed top-k as the
+ *                 alternative), 5 (histogram-based, sort-free threshold and a
+ *                 bandwidth-optimised sparse decode kernel).
+ *   ICS page      "Inference-time context sparsity: illusion or opportunity?",
+ *                 gist.science/ar/paper/2605.24168, 2 (Oracle Top-K), 3a (50x
+ *                 sparsity = ~2% of tokens), 3c (decode traffic O(N d) -> O(k d)).
+ *   AoH page      "Autonomy-of-Heads: Data-Free Sparse Attention from Frozen
+ *                 Query-Key Geometry", gist.science/ar/paper/2608.06849,
+ *                 Methodology 4 (streaming heads keep sinks + recent window;
+ *                 head roles pooled per GQA group).
+ *
+ * Conventions for every call:
+ *   - Pointers named "device" must point to memory of the device that was
+ *     current when sparse_decode_init ran.  The caller owns all of them; the
+ *     library never frees caller memory.
+ *   - bf16 tensors are raw IEEE bfloat16 bit patterns (uint16), row-major and
+ *     densely packed in the order of their stated shapes.
+ *   - Hot calls (index_keys, select, attend) allocate nothing, never
+ *     synchronise the host, and enqueue their work on `stream` (a
+ *     cudaStream_t; NULL = the legacy default stream).  Argument errors are
+ *     detected on the host before any launch and nothing is enqueued.
+ *   - Data-dependent errors found on the device (a page id outside
+ *     [0, num_pages), a sequence length above max_pages_per_seq * page_size,
+ *     a selected position out of range) never fault: the kernel skips the bad
+ *     access, sets a bit in a device error word and carries on; results are
+ *     then unspecified.  sparse_decode_error_word reads and clears the word.
+ *   - The context is not thread-safe: one host thread at a time per context.
+ *     Calls on the same context and stream are ordered; calls that share a
+ *     workspace must not overlap on the device.
+ *
+ * Shapes: B = batch, Hq = query heads, Hkv = KV heads, G = Hq / Hkv (GQA
+ * group), d = head_dim (64 or 128), r = index_dim (16), P = page_size (16),
+ * H_ret = number of retrieval heads, MAXP = max_pages_per_seq,
+ * L = MAXP * P (longest supported context).
+ *
+ * Caches (caller-owned, device):
+ *   k_cache, v_cache  bf16 [num_pages, Hkv, P, d]; token j of sequence b, KV
+ *                     head g lives at [page_table[b][j / P], g, j % P, :].
+ *   index_cache       bf16 [num_pages, Hkv, P, r]; same addressing.
+ *   page_table        int32 [B, MAXP]; entries at and past ceil(N_b / P) are
+ *                     never read.
+ *   seq_lens          int32 [B]; N_b, 0 <= N_b <= L.  The current token is
+ *                     position N_b - 1 and is already in the caches.
+ */
+#ifndef SPARSE_DECODE_H
+#define SPARSE_DECODE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SD_API __attribute__((visibility("default")))
+#else
+#define SD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct sd_ctx sd_ctx;          /* opaque, host-side */
+typedef void *sd_stream;               /* a cudaStream_t */
+
+typedef enum {
+  SD_OK = 0,
+  SD_ERR_INVALID_ARG = 1,   /* a null pointer, a bad size or an inconsistent shape */
+  SD_ERR_UNSUPPORTED = 2,   /* a valid request this build does not implement */
+  SD_ERR_WORKSPACE = 3,     /* workspace missing or smaller than the size query */
+  SD_ERR_CUDA = 4,          /* a CUDA runtime call or a kernel launch failed */
+  SD_ERR_TIMEOUT = 5,       /* a bounded device-side wait gave up */
+  SD_ERR_DEVICE_DATA = 6    /* a device-side check rejected input data */
+} sd_status;
+
+/* Selection mode of retrieval heads (RTPurbo page, Methodology 3). */
+enum { SD_TOP_P = 0, SD_TOP_K = 1 };
+
+/* Bits of the device error word. */
+enum {
+  SD_EBIT_PAGE = 1u,       /* page id outside [0, num_pages) */
+  SD_EBIT_SEQLEN = 2u,     /* N_b < 0 or N_b > L */
+  SD_EBIT_SEL = 4u,        /* sel_idx entry outside [0, N_b), not ascending, or sel_count > sel_stride */
+  SD_EBIT_SLOT = 8u,       /* index_keys slot outside [0, num_pages * P) */
+  SD_EBIT_TIMEOUT = 16u    /* a bounded device-side wait gave up */
+};
+
+/*
+ * Layer configuration, copied by sparse_decode_init.
+ *
+ *   num_q_heads, num_kv_heads  Hq and Hkv; Hkv divides Hq; G = Hq/Hkv <= 16.
+ *   head_dim                   d, 64 or 128.
+ *   index_dim                  r, must be 16 (RTPurbo page, Methodology 2).
+ *   page_size                  P, must be 16.
+ *   num_pages                  pages in the caller's cache pool (bounds checks).
+ *   head_is_retrieval          host int32 [Hq]: 1 = retrieval head, 0 = local
+ *                              head (RTPurbo page, Methodology 1).  Copied.
+ *   window, num_sinks          local heads attend to positions
+ *                              [0, num_sinks) U [N_b - window, N_b), clamped to
+ *                              [0, N_b) (RTPurbo Methodology 1; AoH Methodology 4).
+ *   mode                       SD_TOP_P or SD_TOP_K.
+ *   top_p                      in (0, 1]; keeps the smallest set of highest index
+ *                              scores whose softmax mass reaches top_p; every
+ *                              token tied with the threshold score is kept;
+ *                              top_p = 1 keeps every token.
+ *   top_k, top_k_frac          top-k budget k_b = top_k if top_k > 0, else
+ *                              max(1, floor(top_k_frac * N_b)) (frac in (0, 1]),
+ *                              capped at N_b; ties go to the lower position.
+ *   attn_scale                 logit scale of the attention; <= 0 selects 1/sqrt(d).
+ *   index_scale                c in s_j = c * <P^T q, k~_j>; <= 0 selects
+ *                              sqrt(d) / r, which makes the index score an
+ *                              unbiased estimate of q.k/sqrt(d) for a projection
+ *                              with i.i.d. N(0, 1/d) entries.
+ *   max_batch                  largest B of any later call.
+ *   max_pages_per_seq          MAXP, the page-table row length.
+ */
+typedef struct {
+  int num_q_heads;
+  int num_kv_heads;
+  int head_dim;
+  int index_dim;
+  int page_size;
+  int num_pages;
+  const int32_t *head_is_retrieval;
+  int window;
+  int num_sinks;
+  int mode;
+  float top_p;
+  int top_k;
+  float top_k_frac;
+  float attn_scale;
+  float index_scale;
+  int max_batch;
+  int max_pages_per_seq;
+} sd_config;
+
+/*
+ * sparse_decode_init -- validate `cfg`, copy it and the index projection, and
+ * create a context bound to the current CUDA device.
+ *
+ *   proj  device bf16 [Hkv, d, r]: one r x d projection per KV head, applied
+ *         to pre-RoPE keys of that head and to pre-RoPE queries of its GQA
+ *         group (RTPurbo page, Methodology 2).  Copied; the caller may free
+ *         it after the call.
+ *   out   receives the context; NULL on failure.
+ *
+ * Allocates the device copy of the projection, a head table and a 4-byte
+ * device error word.  Returns SD_ERR_INVALID_ARG or SD_ERR_UNSUPPORTED for a
+ * bad or unsupported configuration, SD_ERR_CUDA if an allocation fails.
+ */
+SD_API sd_status sparse_decode_init(const sd_config *cfg, const void *proj, sd_ctx **out);
+
+/*
+ * sparse_decode_workspace_size -- bytes of device workspace that select and
+ * attend need for a batch of `batch` sequences (batch <= max_batch).  The
+ * same workspace serves both calls.  `bytes` receives the size.
+ */
+SD_API sd_status sparse_decode_workspace_size(const sd_ctx *ctx, int batch, size_t *bytes);
+
+/*
+ * sparse_decode_index_keys -- write index entries for `num_tokens` keys
+ * (RTPurbo page, Methodology 2):
+ *
+ *   index_cache[slot_t / P, g, slot_t % P, :] = bf16_rne( P_g^T k_pre[t, g, :] )
+ *
+ * with the dot products accumulated in float64 and rounded once to bf16,
+ * round to nearest even.
+ *
+ *   k_pre        device bf16 [num_tokens, Hkv, d], pre-RoPE keys.
+ *   slots        device int32 [num_tokens], page * P + offset of each token.
+ *   index_cache  device bf16 [num_pages, Hkv, P, r], written in place.
+ *
+ * num_tokens == 0 is a no-op.  A slot outside [0, num_pages * P) sets
+ * SD_EBIT_SLOT and is skipped.
+ */
+SD_API sd_status sparse_decode_index_keys(sd_ctx *ctx, const void *k_pre, const int32_t *slots,
+                                   int num_tokens, void *index_cache, sd_stream stream);
+
+/*
+ * sparse_decode_select -- per (sequence b, retrieval head h) token sets
+ * (RTPurbo page, Methodology 2-3 and 5; ICS page, 2):
+ *
+ *   q~_h = P_g^T q_pre[b, h]                    (float64, then float32)
+ *   s_j  = index_scale * <q~_h, k~_j>           j < N_b, float32
+ *   top-p: S = { j : s_j >= tau }, tau the largest score whose
+ *          upper set {s >= tau} holds softmax(s) mass >= top_p
+ *   top-k: the k_b highest s_j, ties to the lower position
+ *
+ *   q_pre       device bf16 [B, Hq, d], pre-RoPE queries (only retrieval
+ *               heads are read).
+ *   index_cache device bf16, filled by sparse_decode_index_keys.
+ *   sel_idx     device int32 [B, H_ret, sel_stride]: row (b, i) receives the
+ *               positions of the i-th retrieval head (retrieval heads in
+ *               ascending q-head order), ascending.
+ *   sel_count   device int32 [B, H_ret]: set sizes.
+ *   sel_stride  row capacity: >= L for SD_TOP_P; >= the largest k_b for
+ *               SD_TOP_K (min(top_k, L), or max(1, floor(top_k_frac * L))).
+ *   workspace   device memory of at least sparse_decode_workspace_size bytes.
+ *
+ * N_b == 0 yields an empty set.  Returns SD_ERR_WORKSPACE if ws_bytes is too
+ * small.  A configuration without retrieval heads is a no-op.
+ */
+SD_API sd_status sparse_decode_select(sd_ctx *ctx, const void *q_pre, const void *index_cache,
+                               const int32_t *page_table, const int32_t *seq_lens, int batch,
+                               int32_t *sel_idx, int32_t *sel_count, int sel_stride,
+                               void *workspace, size_t ws_bytes, sd_stream stream);
+
+/*
+ * sparse_decode_attend -- attention output of every head (ICS page, 3c;
+ * RTPurbo Methodology 1):
+ *
+ *   out[b, h] = sum_{j in S} e^{l_j - max l} v_j / sum_{j in S} e^{l_j - max l},
+ *   l_j = attn_scale * <q[b, h], k_j>
+ *
+ * with S the selected set of a retrieval head (from sel_idx / sel_count, as
+ * written by sparse_decode_select or by the caller) and the sinks + window of a
+ * local head.  One softmax over the whole set; fp32 accumulation; an empty
+ * set gives zeros.  Each KV row of a GQA group is read once per call even
+ * when several heads of the group selected it.
+ *
+ *   q          device bf16 [B, Hq, d], post-RoPE queries.
+ *   k_cache, v_cache, page_table, seq_lens   as described above.
+ *   sel_idx, sel_count, sel_stride           as for select (ascending rows);
+ *              may be NULL when there are no retrieval heads.
+ *   out        device float32 [B, Hq, d].
+ *   workspace  device memory of at least sparse_decode_workspace_size bytes.
+ */
+SD_API sd_status sparse_decode_attend(sd_ctx *ctx, const void *q, const void *k_cache,
+                               const void *v_cache, const int32_t *page_table,
+                               const int32_t *seq_lens, int batch, const int32_t *sel_idx,
+                               const int32_t *sel_count, int sel_stride, float *out,
+                               void *workspace, size_t ws_bytes, sd_stream stream);
+
+/*
+ * sparse_decode_error_word -- wait for `stream`, copy the device error word
+ * into *word (may be NULL) and clear it.  Returns SD_OK when the word was 0,
+ * SD_ERR_TIMEOUT when SD_EBIT_TIMEOUT was set, SD_ERR_DEVICE_DATA otherwise.
+ * This call synchronises the stream.
+ */
+SD_API sd_status sparse_decode_error_word(sd_ctx *ctx, sd_stream stream, uint32_t *word);
+
+/* Number of retrieval heads (rows per sequence in sel_idx / sel_count). */
+SD_API int sparse_decode_num_retrieval_heads(const sd_ctx *ctx);
+
+/* Message describing the last failure on this context ("" if none). */
+SD_API const char *sparse_decode_last_error(const sd_ctx *ctx);
+
+/* Static description of a status code. */
+SD_API const char *sparse_decode_status_string(sd_status status);
+
+/* Release the context and its device allocations.  NULL is a no-op. */
+SD_API void sparse_decode_destroy(sd_ctx *ctx);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARSE_DECODE_H */

@@ -1,0 +1,4 @@
+"""Seeded synthetic inputs shared by the tests, the bench and the oracle legs."""
+
+from .synthetic import (BUILDERS, WORKLOAD_NAMES, Workload, keys_at, make_workload,  # noqa: F401
+                        slots_of)
