@@ -74,60 +74,71 @@ def barrier():
 # ---------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons during the timed
-    region (200 ms period)."""
+    """SM clock and throttle-reason samples during the timed region, read
+    through NVML every 10 ms (the data nvidia-smi reports; nothing is set).
+    Falls back to `nvidia-smi -lms 200` when NVML is unavailable."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clocks-event reason bits
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown"}
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.lines = []
+    def __init__(self, cuda_index: int):
+        self.cuda_index = cuda_index
+        self.samples = []
+        self.stop_evt = threading.Event()
+        self.handle = None
+        self.nvml = None
+
+    def _handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        self.nvml = pynvml
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(self.cuda_index).uuid)
+            return pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            idx = int(vis.split(",")[self.cuda_index]) if vis and vis.split(",")[0].isdigit() else self.cuda_index
+            return pynvml.nvmlDeviceGetHandleByIndex(idx)
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
-            self.thread.start()
+            self.handle = self._handle()
+            self.max_mhz = self.nvml.nvmlDeviceGetMaxClockInfo(self.handle, self.nvml.NVML_CLOCK_SM)
         except Exception:
-            self.proc = None
+            self.handle = None
+            return
+        getr = getattr(self.nvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(self.nvml, "nvmlDeviceGetCurrentClocksThrottleReasons")
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+        def loop():
+            while not self.stop_evt.is_set():
+                try:
+                    self.samples.append((self.nvml.nvmlDeviceGetClockInfo(self.handle, self.nvml.NVML_CLOCK_SM),
+                                         int(getr(self.handle))))
+                except Exception:
+                    pass
+                time.sleep(0.01)
+
+        self.thread = threading.Thread(target=loop, daemon=True)
+        self.thread.start()
 
     def stop(self):
-        if self.proc is None:
+        if self.handle is None:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
+        self.stop_evt.set()
         self.thread.join(timeout=2)
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 8:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                smax.append(float(parts[1]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[4:8]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
+        if not self.samples:
             return None
-        sm.sort()
-        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": max(smax), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        sm = sorted(x for x, _ in self.samples)
+        reasons = set()
+        for _, r in self.samples:
+            for bit, name in self.REASONS.items():
+                if r & bit:
+                    reasons.add(name)
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons),
+                "samples": len(sm), "source": "nvml 10 ms"}
 
 
 # ---------------------------------------------------------------- measurements
@@ -214,6 +225,17 @@ def union_rows(sel_idx, sel_count, w):
     return total, index_tokens
 
 
+def size_overrides(args):
+    """--batch / --seq-len shrink the workload (profiling cases); the JSON
+    config reports the sizes actually run."""
+    kw = {}
+    if args.batch:
+        kw["B"] = args.batch
+    if args.seq_len:
+        kw["N"] = args.seq_len
+    return kw
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -228,7 +250,7 @@ def run_ours(args):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
-    w = make_workload(args.workload, dev, seed=rank_seed(args.seed, rank))
+    w = make_workload(args.workload, dev, seed=rank_seed(args.seed, rank), **size_overrides(args))
     B, Hq, d = w.batch, w.num_q_heads, w.head_dim
     st = DecodeStep(k_cache=w.k_cache, v_cache=w.v_cache, page_table=w.page_table, seq_lens=w.seq_lens,
                     proj=w.proj, num_q_heads=Hq, head_is_retrieval=w.head_is_retrieval, window=w.window,
@@ -446,7 +468,7 @@ def run_reference(args):
     from workloads import make_workload
     import oracle as O
     dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
-    w = make_workload(args.workload, dev, seed=rank_seed(args.seed, 0))
+    w = make_workload(args.workload, dev, seed=rank_seed(args.seed, 0), **size_overrides(args))
     cfg = oracle_config(w)
     G = w.num_q_heads // w.num_kv_heads
     inp = oracle_inputs(w, [0])
@@ -486,6 +508,8 @@ def main(argv=None):
     ap.add_argument("--seed", type=int, default=2)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling)")
+    ap.add_argument("--seq-len", type=int, default=0, help="override the workload's context length")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)          # timing rule: at least 3 warm-up steps
     if args.impl == "reference":

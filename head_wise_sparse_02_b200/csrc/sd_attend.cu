@@ -24,6 +24,8 @@
 // finish (atomic ticket, no waiting) merges the partials with a log-sum-exp
 // combine into out[b, h, :] and resets the ticket.
 #include <algorithm>
+#include <map>
+#include <mutex>
 
 #include "sd_internal.cuh"
 
@@ -45,10 +47,12 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 // First index i in [0, n) with arr[i] >= x (n if none); whole warp cooperates.
+// Lanes 0..30 probe inside [lo, hi); lane 31 always lands at or past hi and
+// acts as the sentinel, so some lane is always true.
 __device__ int warp_lower_bound(const int32_t *arr, int n, int x, int lane) {
-  int lo = 0, hi = n;
-  while (hi - lo > 32) {
-    const int step = (hi - lo + 31) / 32;
+  int lo = 0, hi = n;                      // answer in [lo, hi]
+  while (hi - lo > 31) {
+    const int step = (hi - lo + 30) / 31;  // 31 * step >= hi - lo
     const int p = lo + lane * step;
     const bool ge = (p < hi) ? (__ldg(arr + p) >= x) : true;
     const int first = __ffs(__ballot_sync(kFull, ge)) - 1;
@@ -57,7 +61,7 @@ __device__ int warp_lower_bound(const int32_t *arr, int n, int x, int lane) {
     lo = nlo;
     hi = nhi;
   }
-  const int p = lo + lane;
+  const int p = lo + lane;                 // hi - lo <= 31: lane 31 is past hi
   const bool ge = (p < hi) ? (__ldg(arr + p) >= x) : true;
   return lo + (__ffs(__ballot_sync(kFull, ge)) - 1);
 }
@@ -392,8 +396,19 @@ AttPlan make_plan(const Shape &sh, const Tables &tb, int D) {
 template <int D, int GR>
 cudaError_t launch_t(const AttendArgs &a, const Shape &sh, const Tables &tb, const AttPlan &p, cudaStream_t st) {
   auto kern = attend_kernel<D, GR>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.dyn_bytes);
-  if (e != cudaSuccess) return e;
+  static std::mutex mu;
+  static std::map<int, size_t> configured;     // device -> dynamic smem bytes set
+  int dev = 0;
+  cudaGetDevice(&dev);
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    auto it = configured.find(dev);
+    if (it == configured.end() || it->second < p.dyn_bytes) {
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.dyn_bytes);
+      if (e != cudaSuccess) return e;
+      configured[dev] = p.dyn_bytes;
+    }
+  }
   const long long blocks = (long long)a.batch * ((long long)tb.n_ret * p.ns_r + (long long)tb.n_loc * p.ns_l);
   if (blocks == 0) return cudaSuccess;
   kern<<<(unsigned)blocks, kThreads, p.dyn_bytes, st>>>(a, sh, tb, p.ns_r, p.span_r, p.ns_l, p.ns_max);

@@ -29,6 +29,9 @@
 #include <cooperative_groups.h>
 
 #include <algorithm>
+#include <map>
+#include <mutex>
+#include <tuple>
 
 #include "sd_internal.cuh"
 
@@ -254,7 +257,7 @@ select_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__ grou
 #pragma unroll
     for (int h = 0; h < HPB; ++h) {
       const float m = warp_max_strided(tmax[h], HB);
-      if (lane == 0 && hb * HPB + h < nr && m > -INFINITY) atomicMax(&S.cmax_key[hb * HPB + h], order_key(m));
+      if (lane < HB && hb * HPB + h < nr && m > -INFINITY) atomicMax(&S.cmax_key[hb * HPB + h], order_key(m));
     }
   }
   if (!SMEM) __threadfence_block();
@@ -263,10 +266,11 @@ select_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__ grou
   // ---- cluster max (top-p needs the softmax reference) --------------------
   if (TOPP) {
     cluster.sync();
-    if (tid < nr) {
-      uint32_t m = 0;
-      for (int c = 0; c < C; ++c) m = std::max(m, *cluster.map_shared_rank(&S.cmax_key[tid], c));
-      S.M[tid] = key_to_float(m);
+    if (warp < nr) {                   // warp h reads the C CTA maxima, one per lane
+      uint32_t m = lane < C ? *cluster.map_shared_rank(&S.cmax_key[warp], lane) : 0u;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = std::max(m, __shfl_xor_sync(kFull, m, o));
+      if (lane == 0) S.M[warp] = key_to_float(m);
     }
   }
   if (tid < nr) {
@@ -303,82 +307,137 @@ select_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__ grou
     }
     __syncthreads();
     cluster.sync();
-    // owner reduction of this CTA's digit slice
-    for (int o = tid; o < nr * per; o += kThreads) {
-      const int h = o / per, dg = d0 + o % per;
-      uint32_t sc = 0;
-      double sm = 0.0;
-      for (int c = 0; c < C; ++c) {
-        sc += *cluster.map_shared_rank(&hcnt[h * kRadix + dg], c);
-        if (TOPP) sm += *cluster.map_shared_rank(&hmass[h * kRadix + dg], c);
+    // owner reduction of this CTA's digit slice: one remote load per lane,
+    // items ordered (head, digit, cta) with the CTA index fastest so that the
+    // C values of one digit sit in C adjacent lanes (C divides 32)
+    for (int base = 0; base < nr * kRadix; base += kThreads) {
+      const int it = base + tid;
+      const bool ok = it < nr * kRadix;
+      const int c = it % C, rest = it / C;
+      const int h = rest / per, dg = d0 + rest % per;
+      uint32_t vc = 0u;
+      double vm = 0.0;
+      if (ok) {
+        vc = *cluster.map_shared_rank(&hcnt[h * kRadix + dg], c);
+        if (TOPP) vm = *cluster.map_shared_rank(&hmass[h * kRadix + dg], c);
       }
-      rcnt[h * kRadix + dg] = sc;
-      if (TOPP) rmass[h * kRadix + dg] = sm;
+      for (int o = 1; o < C; o <<= 1) {
+        vc += __shfl_xor_sync(kFull, vc, o);
+        if (TOPP) vm += __shfl_xor_sync(kFull, vm, o);
+      }
+      if (ok && c == 0) {
+        rcnt[h * kRadix + dg] = vc;
+        if (TOPP) rmass[h * kRadix + dg] = vm;
+      }
     }
     __syncthreads();
-    if (tid < nr) {
-      uint32_t sc = 0;
+    if (warp < nr) {                   // slice totals, warp h
+      uint32_t sc = 0u;
       double sm = 0.0;
-      for (int dg = d0; dg < d0 + per; ++dg) {
-        sc += rcnt[tid * kRadix + dg];
-        if (TOPP) sm += rmass[tid * kRadix + dg];
+      for (int j = lane; j < per; j += 32) {
+        sc += rcnt[warp * kRadix + d0 + j];
+        if (TOPP) sm += rmass[warp * kRadix + d0 + j];
       }
-      S.slice_cnt[tid] = sc;
-      S.slice_mass[tid] = sm;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        sc += __shfl_xor_sync(kFull, sc, o);
+        if (TOPP) sm += __shfl_xor_sync(kFull, sm, o);
+      }
+      if (lane == 0) {
+        S.slice_cnt[warp] = sc;
+        S.slice_mass[warp] = sm;
+      }
     }
     __syncthreads();
     cluster.sync();
-    // every CTA: locate the cut digit (scanning from the highest digit down)
-    if (tid < nr) {
-      const int h = tid;
-      uint32_t scnt[kMaxCluster];
-      double smass[kMaxCluster];
-      for (int c = 0; c < C; ++c) {
-        scnt[c] = *cluster.map_shared_rank(&S.slice_cnt[h], c);
-        smass[c] = TOPP ? *cluster.map_shared_rank(&S.slice_mass[h], c) : 0.0;
-      }
+    // every CTA, warp h: locate the cut digit scanning from the highest digit
+    // down; lanes hold slices (then digits) and suffix sums give the running
+    // amount above each of them
+    if (warp < nr) {
+      const int h = warp;
+      const uint32_t lc = lane < C ? *cluster.map_shared_rank(&S.slice_cnt[h], lane) : 0u;
+      const double lm = (TOPP && lane < C) ? *cluster.map_shared_rank(&S.slice_mass[h], lane) : 0.0;
       if (TOPP && pass == 0) {
-        double Z = 0.0;
-        for (int c = 0; c < C; ++c) Z += smass[c];
-        S.target[h] = (double)a.top_p * Z;
+        double Z = lm;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) Z += __shfl_xor_sync(kFull, Z, o);
+        if (lane == 0) S.target[h] = (double)a.top_p * Z;
       }
+      __syncwarp();
       const double need_m = TOPP ? S.target[h] : 0.0;
       const long long need_k = S.need[h];
-      double acc_m = 0.0;
-      long long acc_k = 0;
-      int cs = -1, last_nz = -1;
-      for (int c = C - 1; c >= 0; --c) {
-        if (scnt[c] == 0) continue;
-        const bool reach = TOPP ? (acc_m + smass[c] >= need_m) : (acc_k + (long long)scnt[c] >= need_k);
-        if (reach) { cs = c; break; }
-        acc_m += smass[c];
-        acc_k += scnt[c];
-        last_nz = c;
+      // suffix sums over lanes: value at lane c = sum over lanes >= c
+      long long suf_k = lc;
+      double suf_m = lm;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const long long yk = __shfl_down_sync(kFull, suf_k, o);
+        const double ym = __shfl_down_sync(kFull, suf_m, o);
+        if (lane + o < 32) {
+          suf_k += yk;
+          suf_m += ym;
+        }
       }
-      if (cs < 0) {                      // rounding left the target unreached: take the lowest
-        cs = last_nz < 0 ? 0 : last_nz;  // non-empty slice and, in it, the lowest digit
-        acc_m -= smass[cs];
-        acc_k -= scnt[cs];
+      bool reach = lane < C && lc > 0u && (TOPP ? suf_m >= need_m : suf_k >= need_k);
+      unsigned bal = __ballot_sync(kFull, reach);
+      int cs;
+      if (bal) {
+        cs = 31 - __clz(bal);          // highest slice where the amount is reached
+      } else {                         // rounding left it unreached: lowest non-empty slice
+        const unsigned nz = __ballot_sync(kFull, lane < C && lc > 0u);
+        cs = nz ? __ffs(nz) - 1 : 0;
       }
-      int cut = -1, last_d = -1;
-      for (int dg = (cs + 1) * per - 1; dg >= cs * per; --dg) {
-        const uint32_t dc = *cluster.map_shared_rank(&rcnt[h * kRadix + dg], cs);
-        if (dc == 0) continue;
-        const double dm = TOPP ? *cluster.map_shared_rank(&rmass[h * kRadix + dg], cs) : 0.0;
-        const bool reach = TOPP ? (acc_m + dm >= need_m) : (acc_k + (long long)dc >= need_k);
-        if (reach) { cut = dg; break; }
-        acc_m += dm;
-        acc_k += dc;
-        last_d = dg;
+      // amount strictly above slice cs
+      long long acc_k = __shfl_sync(kFull, suf_k, cs) - (long long)__shfl_sync(kFull, lc, cs);
+      double acc_m = __shfl_sync(kFull, suf_m, cs) - __shfl_sync(kFull, lm, cs);
+      int cut = -1;
+      int lowest_nz = -1;
+      for (int top = per; top > 0 && cut < 0; top -= 32) {
+        const int j = top - 32 + lane;          // digits of this chunk, highest chunk first
+        const int dg = cs * per + j;
+        const bool in = j >= 0 && j < per;
+        const uint32_t dc = in ? *cluster.map_shared_rank(&rcnt[h * kRadix + dg], cs) : 0u;
+        const double dm = (TOPP && in) ? *cluster.map_shared_rank(&rmass[h * kRadix + dg], cs) : 0.0;
+        long long sk = dc;
+        double smv = dm;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const long long yk = __shfl_down_sync(kFull, sk, o);
+          const double ym = __shfl_down_sync(kFull, smv, o);
+          if (lane + o < 32) {
+            sk += yk;
+            smv += ym;
+          }
+        }
+        const bool r2 = in && dc > 0u && (TOPP ? acc_m + smv >= need_m : acc_k + sk >= need_k);
+        const unsigned b2 = __ballot_sync(kFull, r2);
+        const unsigned nz2 = __ballot_sync(kFull, in && dc > 0u);
+        if (b2) {
+          const int l = 31 - __clz(b2);
+          cut = cs * per + top - 32 + l;
+          acc_k += __shfl_sync(kFull, sk, l) - (long long)__shfl_sync(kFull, dc, l);
+          acc_m += __shfl_sync(kFull, smv, l) - __shfl_sync(kFull, dm, l);
+        } else {
+          if (nz2) {
+            const int l = __ffs(nz2) - 1;
+            lowest_nz = cs * per + top - 32 + l;
+          }
+          acc_k += __shfl_sync(kFull, sk, 0);
+          acc_m += __shfl_sync(kFull, smv, 0);
+        }
       }
-      if (cut < 0) {
-        cut = last_d < 0 ? cs * per : last_d;
-        acc_m -= TOPP ? *cluster.map_shared_rank(&rmass[h * kRadix + cut], cs) : 0.0;
-        acc_k -= *cluster.map_shared_rank(&rcnt[h * kRadix + cut], cs);
+      if (cut < 0) {                   // rounding: take the lowest non-empty digit of the slice
+        cut = lowest_nz < 0 ? cs * per : lowest_nz;
+        const uint32_t dc = *cluster.map_shared_rank(&rcnt[h * kRadix + cut], cs);
+        const double dm = TOPP ? *cluster.map_shared_rank(&rmass[h * kRadix + cut], cs) : 0.0;
+        acc_k -= dc;
+        acc_m -= dm;
       }
-      S.prefix[h] = (S.prefix[h] << 8) | (uint32_t)cut;
-      if (TOPP) S.target[h] = need_m - acc_m;
-      S.need[h] = need_k - acc_k;
+      if (lane == 0) {
+        S.prefix[h] = (S.prefix[h] << 8) | (uint32_t)cut;
+        if (TOPP) S.target[h] = need_m - acc_m;
+        S.need[h] = need_k - acc_k;
+      }
     }
     __syncthreads();
   }
@@ -414,27 +473,29 @@ select_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__ grou
   }
   __syncthreads();
   cluster.sync();
-  if (tid < nr) {
-    const int h = tid;
-    long long gt_before = 0, eq_before = 0, tot_gt = 0, tot_eq = 0;
-    for (int c = 0; c < C; ++c) {
-      const long long gc = *cluster.map_shared_rank(&S.cgt[h], c);
-      const long long ec = *cluster.map_shared_rank(&S.ceq[h], c);
-      if (c < rank) {
-        gt_before += gc;
-        eq_before += ec;
-      }
-      tot_gt += gc;
-      tot_eq += ec;
+  if (warp < nr) {
+    const int h = warp;
+    const long long gc = lane < C ? (long long)*cluster.map_shared_rank(&S.cgt[h], lane) : 0LL;
+    const long long ec = lane < C ? (long long)*cluster.map_shared_rank(&S.ceq[h], lane) : 0LL;
+    long long gt_before = lane < rank ? gc : 0, eq_before = lane < rank ? ec : 0;
+    long long tot_gt = gc, tot_eq = ec;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      gt_before += __shfl_xor_sync(kFull, gt_before, o);
+      eq_before += __shfl_xor_sync(kFull, eq_before, o);
+      tot_gt += __shfl_xor_sync(kFull, tot_gt, o);
+      tot_eq += __shfl_xor_sync(kFull, tot_eq, o);
     }
-    const long long ties_total = TOPP ? tot_eq : std::min(S.need[h], tot_eq);
-    const long long ties_before = std::min(eq_before, ties_total);
-    S.my_ties[h] = std::max(0LL, std::min((long long)S.ceq[h], ties_total - eq_before));
-    S.out_off[h] = gt_before + ties_before;
-    const long long total = tot_gt + ties_total;
-    if (rank == 0) {
-      if (total > a.sel_stride) raise_error(a.err, SD_EBIT_SEL);
-      *count_slot(h) = (int32_t)std::min(total, a.sel_stride);
+    if (lane == 0) {
+      const long long ties_total = TOPP ? tot_eq : std::min(S.need[h], tot_eq);
+      const long long ties_before = std::min(eq_before, ties_total);
+      S.my_ties[h] = std::max(0LL, std::min((long long)S.ceq[h], ties_total - eq_before));
+      S.out_off[h] = gt_before + ties_before;
+      const long long total = tot_gt + ties_total;
+      if (rank == 0) {
+        if (total > a.sel_stride) raise_error(a.err, SD_EBIT_SEL);
+        *count_slot(h) = (int32_t)std::min(total, a.sel_stride);
+      }
     }
   }
   cluster.sync();   // no CTA leaves while others still read its shared memory
@@ -516,37 +577,47 @@ Plan make_plan(const Shape &sh, const Tables &tb, int batch, bool topp, int smem
   return p;
 }
 
+// Per kernel instantiation and device: the dynamic shared memory attribute
+// and the cluster occupancy check are set / queried once, not per call.
 template <int GR, bool TOPP, bool SMEM>
-cudaError_t launch_t(const SelectArgs &a, const Shape &sh, const Tables &tb, const Plan &p, cudaStream_t st) {
-  auto kern = select_kernel<GR, TOPP, SMEM>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.dyn_bytes);
-  if (e != cudaSuccess) return e;
-  if (p.cluster > 8) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e != cudaSuccess) return e;
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.cluster, a.batch * tb.n_ret, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = p.dyn_bytes;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = p.cluster;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, a, sh, tb.ret, tb.n_ret, p.tc_cap);
+struct KernelCache {
+  std::mutex mu;
+  std::map<int, size_t> attr_bytes;                      // device -> bytes configured
+  std::map<std::tuple<int, size_t, int>, int> clusters;  // (device, bytes, cluster) -> active clusters
+};
+
+template <int GR, bool TOPP, bool SMEM>
+KernelCache<GR, TOPP, SMEM> &kcache() {
+  static KernelCache<GR, TOPP, SMEM> c;
+  return c;
 }
 
 template <int GR, bool TOPP, bool SMEM>
-int active_clusters(const Plan &p) {
+cudaError_t ensure_attrs(int dev, size_t bytes) {
+  auto &c = kcache<GR, TOPP, SMEM>();
+  std::lock_guard<std::mutex> lk(c.mu);
+  auto it = c.attr_bytes.find(dev);
+  if (it != c.attr_bytes.end() && it->second >= bytes) return cudaSuccess;
   auto kern = select_kernel<GR, TOPP, SMEM>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.dyn_bytes) != cudaSuccess)
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e == cudaSuccess) c.attr_bytes[dev] = bytes;
+  return e;
+}
+
+template <int GR, bool TOPP, bool SMEM>
+int active_clusters(int dev, const Plan &p) {
+  if (ensure_attrs<GR, TOPP, SMEM>(dev, p.dyn_bytes) != cudaSuccess) {
+    cudaGetLastError();
     return 0;
-  if (p.cluster > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
-    return 0;
+  }
+  auto &c = kcache<GR, TOPP, SMEM>();
+  const auto key = std::make_tuple(dev, p.dyn_bytes, p.cluster);
+  {
+    std::lock_guard<std::mutex> lk(c.mu);
+    auto it = c.clusters.find(key);
+    if (it != c.clusters.end()) return it->second;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.cluster, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -559,32 +630,55 @@ int active_clusters(const Plan &p) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, select_kernel<GR, TOPP, SMEM>, &cfg) != cudaSuccess) {
     cudaGetLastError();
-    return 0;
+    n = 0;
   }
+  std::lock_guard<std::mutex> lk(c.mu);
+  c.clusters[key] = n;
   return n;
 }
 
+template <int GR, bool TOPP, bool SMEM>
+cudaError_t launch_t(const SelectArgs &a, const Shape &sh, const Tables &tb, const Plan &p, int dev,
+                     cudaStream_t st) {
+  cudaError_t e = ensure_attrs<GR, TOPP, SMEM>(dev, p.dyn_bytes);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.cluster, a.batch * tb.n_ret, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = p.dyn_bytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = p.cluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, select_kernel<GR, TOPP, SMEM>, a, sh, tb.ret, tb.n_ret, p.tc_cap);
+}
+
 template <bool TOPP, bool SMEM>
-int active_clusters_gr(const Tables &tb, const Plan &p) {
+int active_clusters_gr(const Tables &tb, const Plan &p, int dev) {
   switch (group_rows(tb)) {
-    case 1: return active_clusters<1, TOPP, SMEM>(p);
-    case 2: return active_clusters<2, TOPP, SMEM>(p);
-    case 4: return active_clusters<4, TOPP, SMEM>(p);
-    case 8: return active_clusters<8, TOPP, SMEM>(p);
-    default: return active_clusters<16, TOPP, SMEM>(p);
+    case 1: return active_clusters<1, TOPP, SMEM>(dev, p);
+    case 2: return active_clusters<2, TOPP, SMEM>(dev, p);
+    case 4: return active_clusters<4, TOPP, SMEM>(dev, p);
+    case 8: return active_clusters<8, TOPP, SMEM>(dev, p);
+    default: return active_clusters<16, TOPP, SMEM>(dev, p);
   }
 }
 
 template <bool TOPP, bool SMEM>
-cudaError_t dispatch_gr(const SelectArgs &a, const Shape &sh, const Tables &tb, const Plan &p, cudaStream_t st) {
+cudaError_t dispatch_gr(const SelectArgs &a, const Shape &sh, const Tables &tb, const Plan &p, int dev,
+                        cudaStream_t st) {
   switch (group_rows(tb)) {
-    case 1: return launch_t<1, TOPP, SMEM>(a, sh, tb, p, st);
-    case 2: return launch_t<2, TOPP, SMEM>(a, sh, tb, p, st);
-    case 4: return launch_t<4, TOPP, SMEM>(a, sh, tb, p, st);
-    case 8: return launch_t<8, TOPP, SMEM>(a, sh, tb, p, st);
-    default: return launch_t<16, TOPP, SMEM>(a, sh, tb, p, st);
+    case 1: return launch_t<1, TOPP, SMEM>(a, sh, tb, p, dev, st);
+    case 2: return launch_t<2, TOPP, SMEM>(a, sh, tb, p, dev, st);
+    case 4: return launch_t<4, TOPP, SMEM>(a, sh, tb, p, dev, st);
+    case 8: return launch_t<8, TOPP, SMEM>(a, sh, tb, p, dev, st);
+    default: return launch_t<16, TOPP, SMEM>(a, sh, tb, p, dev, st);
   }
 }
 
@@ -604,12 +698,23 @@ size_t select_workspace_bytes(const Shape &sh, const Tables &tb, int batch) {
 
 cudaError_t launch_select(const SelectArgs &a, const Shape &sh, const Tables &tb, cudaStream_t st) {
   if (tb.n_ret == 0 || a.batch == 0) return cudaSuccess;
+  int dev = 0;
+  cudaGetDevice(&dev);
   const bool topp = a.mode == SD_TOP_P;
-  Plan p = make_plan(sh, tb, a.batch, topp, smem_limit_bytes());
+  static std::mutex mu;
+  static std::map<int, int> smem_limit;
+  int lim;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    auto it = smem_limit.find(dev);
+    if (it == smem_limit.end()) it = smem_limit.emplace(dev, smem_limit_bytes()).first;
+    lim = it->second;
+  }
+  Plan p = make_plan(sh, tb, a.batch, topp, lim);
   // A cluster whose CTAs cannot be co-resident would fail to launch: fall back
   // to the portable size with scores in the workspace.
-  const int fits = topp ? (p.smem ? active_clusters_gr<true, true>(tb, p) : active_clusters_gr<true, false>(tb, p))
-                        : (p.smem ? active_clusters_gr<false, true>(tb, p) : active_clusters_gr<false, false>(tb, p));
+  const int fits = topp ? (p.smem ? active_clusters_gr<true, true>(tb, p, dev) : active_clusters_gr<true, false>(tb, p, dev))
+                        : (p.smem ? active_clusters_gr<false, true>(tb, p, dev) : active_clusters_gr<false, false>(tb, p, dev));
   if (fits == 0) {
     const int c = std::min(p.cluster, 8);
     p.cluster = c;
@@ -617,8 +722,8 @@ cudaError_t launch_select(const SelectArgs &a, const Shape &sh, const Tables &tb
     p.tc_cap = (int)(((sh.max_len + c - 1) / c + kPage - 1) / kPage * kPage);
     p.dyn_bytes = hist_bytes(group_rows(tb), topp);
   }
-  if (topp) return p.smem ? dispatch_gr<true, true>(a, sh, tb, p, st) : dispatch_gr<true, false>(a, sh, tb, p, st);
-  return p.smem ? dispatch_gr<false, true>(a, sh, tb, p, st) : dispatch_gr<false, false>(a, sh, tb, p, st);
+  if (topp) return p.smem ? dispatch_gr<true, true>(a, sh, tb, p, dev, st) : dispatch_gr<true, false>(a, sh, tb, p, dev, st);
+  return p.smem ? dispatch_gr<false, true>(a, sh, tb, p, dev, st) : dispatch_gr<false, false>(a, sh, tb, p, dev, st);
 }
 
 }  // namespace sd

@@ -155,8 +155,11 @@ def _plant_needles(w: Workload, counts: Dict[int, List[int]], gen, noise: float 
                 m = counts[b][i]
                 if m == 0:
                     continue
-                p = pos[c:c + m]
+                p = pos[c:c + m]              # fewer when the context is shorter than the needles
                 c += m
+                m = int(p.numel())
+                if m == 0:
+                    continue
                 qh = w.q[b, h].float()
                 key = 0.8 * math.sqrt(d) * qh / qh.norm()
                 eps = noise * torch.randn((m, d), generator=gen, device=dev, dtype=torch.float32)
