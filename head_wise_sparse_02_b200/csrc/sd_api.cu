@@ -47,13 +47,15 @@ sd_status cuda_fail(sd_ctx *ctx, cudaError_t e, const char *what) {
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct WsLayout {
-  size_t scores_off, scores_bytes, part_off, tickets_off, total;
+  size_t scores_off, flags_off, scores_bytes, part_off, tickets_off, total;
 };
 
 WsLayout layout(const sd_ctx *ctx, int batch) {
   WsLayout w{};
   w.scores_off = 0;
-  w.scores_bytes = align256(sd::select_workspace_bytes(ctx->sh, ctx->tb, batch));
+  size_t foff = 0;
+  w.scores_bytes = align256(sd::select_workspace_bytes(ctx->sh, ctx->tb, batch, &foff));
+  w.flags_off = w.scores_off + foff;
   w.part_off = w.scores_off + w.scores_bytes;
   size_t toff = 0;
   const size_t att = sd::attend_workspace_bytes(ctx->sh, ctx->tb, batch, &toff);
@@ -221,6 +223,7 @@ sd_status sparse_decode_select(sd_ctx *ctx, const void *q_pre, const void *index
   a.top_k = ctx->cfg.top_k;
   a.top_k_frac = ctx->cfg.top_k_frac;
   a.score_ws = reinterpret_cast<float *>(static_cast<char *>(workspace) + w.scores_off);
+  a.flags = reinterpret_cast<uint32_t *>(static_cast<char *>(workspace) + w.flags_off);
   a.err = ctx->err_d;
   a.batch = batch;
   cudaError_t e = sd::launch_select(a, ctx->sh, ctx->tb, static_cast<cudaStream_t>(stream));

@@ -18,20 +18,6 @@ namespace {
 constexpr int kRows = 16;          // (token) rows per block, one KV head per block
 constexpr int kThreads = kRows * kIndexDim;
 
-// float64 -> bf16 bits, round to nearest even, from the float64 value itself.
-__device__ __forceinline__ uint16_t f64_to_bf16_rne(double x) {
-  if (isnan(x)) return 0x7FC0u;
-  const uint16_t sign = (__double_as_longlong(x) < 0) ? 0x8000u : 0u;
-  const double a = fabs(x);
-  if (a == 0.0) return sign;
-  int e;
-  frexp(a, &e);                                  // a = m * 2^e, 0.5 <= m < 1
-  const int q = max(e - 8, -133);                // bf16 quantum (subnormal floor 2^-133)
-  const double r = rint(ldexp(a, -q));           // exact scaling, ties to even
-  const float y = (float)ldexp(r, q);            // exactly representable, or +inf on overflow
-  return sign | (uint16_t)(__float_as_uint(y) >> 16);
-}
-
 template <int D>
 __global__ void __launch_bounds__(kThreads)
 index_keys_kernel(const uint16_t *__restrict__ k_pre, const int32_t *__restrict__ slots, int T,

@@ -50,6 +50,23 @@ __device__ __forceinline__ float key_to_float(uint32_t k) {
   return __uint_as_float(u);
 }
 
+// float64 -> bf16 bits, round to nearest even, from the float64 value itself
+// (never through float32).  bf16 keeps 8 significant bits and float32's
+// exponent range; the quantum of a value in [2^(e-1), 2^e) is 2^(e-8), with
+// the subnormal floor 2^-133.
+__device__ __forceinline__ uint16_t f64_to_bf16_rne(double x) {
+  if (isnan(x)) return 0x7FC0u;
+  const uint16_t sign = (__double_as_longlong(x) < 0) ? 0x8000u : 0u;
+  const double a = fabs(x);
+  if (a == 0.0) return sign;
+  int e;
+  frexp(a, &e);                                  // a = m * 2^e, 0.5 <= m < 1
+  const int q = max(e - 8, -133);
+  const double r = rint(ldexp(a, -q));           // exact scaling, ties to even
+  const float y = (float)ldexp(r, q);            // exactly representable, or +inf on overflow
+  return sign | (uint16_t)(__float_as_uint(y) >> 16);
+}
+
 __device__ __forceinline__ void raise_error(unsigned *err, unsigned bit) {
   if (err) atomicOr(err, bit);
 }
@@ -75,12 +92,15 @@ struct SelectArgs {
   int top_k;
   float top_k_frac;
   float *score_ws;                // global score rows when they do not fit on chip
+  uint32_t *flags;                // [batch * n_ret] streaming top-k misses
   unsigned *err;
   int batch;
 };
 
-size_t select_workspace_bytes(const Shape &sh, const Tables &tb, int batch);
+size_t select_workspace_bytes(const Shape &sh, const Tables &tb, int batch, size_t *flags_off);
 cudaError_t launch_select(const SelectArgs &a, const Shape &sh, const Tables &tb, cudaStream_t st);
+cudaError_t launch_select_topk_stream(const SelectArgs &a, const Shape &sh, const Tables &tb, uint32_t *fail,
+                                      cudaStream_t st, bool *used);
 
 struct AttendArgs {
   const uint16_t *q;

@@ -106,18 +106,14 @@ struct SelShared {
 
 // GR: score rows held per CTA (power of two >= the group's retrieval heads).
 template <int GR, bool TOPP, bool SMEM>
-__global__ void __launch_bounds__(kThreads, 1)
-select_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__ groups, int n_groups,
-              int tc_cap) {
+__device__ __forceinline__ void select_item(const SelectArgs &a, const Shape &sh, const Group *__restrict__ groups,
+                                            int n_groups, int tc_cap, int item, SelShared &S, unsigned char *dyn) {
   cg::cluster_group cluster = cg::this_cluster();
   const int C = (int)cluster.num_blocks();
   const int rank = (int)cluster.block_rank();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int b = blockIdx.y / n_groups;
-  const int gi = blockIdx.y % n_groups;
-
-  __shared__ SelShared S;
-  extern __shared__ __align__(16) unsigned char dyn[];
+  const int b = item / n_groups;
+  const int gi = item % n_groups;
   double *hmass = reinterpret_cast<double *>(dyn);                    // [GR][256] (top-p)
   double *rmass = hmass + (TOPP ? GR * kRadix : 0);                  // [GR][256] (top-p)
   uint32_t *hcnt = reinterpret_cast<uint32_t *>(rmass + (TOPP ? GR * kRadix : 0));
@@ -532,6 +528,24 @@ select_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__ grou
   }
 }
 
+// One cluster per work item (sequence, retrieval KV group).  With `flags`,
+// the grid's clusters stride over all items and process only the flagged
+// ones (items whose streaming top-k window missed); otherwise item =
+// blockIdx.y.
+template <int GR, bool TOPP, bool SMEM>
+__global__ void __launch_bounds__(kThreads, 1)
+select_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__ groups, int n_groups,
+              int tc_cap, const uint32_t *__restrict__ flags) {
+  __shared__ SelShared S;
+  extern __shared__ __align__(16) unsigned char dyn[];
+  const int n_items = a.batch * n_groups;
+  for (int item = blockIdx.y; item < n_items; item += gridDim.y) {
+    if (flags && flags[item] == 0u) continue;
+    __syncthreads();
+    select_item<GR, TOPP, SMEM>(a, sh, groups, n_groups, tc_cap, item, S, dyn);
+  }
+}
+
 struct Plan {
   int cluster;
   bool smem;
@@ -641,11 +655,11 @@ int active_clusters(int dev, const Plan &p) {
 
 template <int GR, bool TOPP, bool SMEM>
 cudaError_t launch_t(const SelectArgs &a, const Shape &sh, const Tables &tb, const Plan &p, int dev,
-                     cudaStream_t st) {
+                     cudaStream_t st, const uint32_t *flags, int grid_y) {
   cudaError_t e = ensure_attrs<GR, TOPP, SMEM>(dev, p.dyn_bytes);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.cluster, a.batch * tb.n_ret, 1);
+  cfg.gridDim = dim3(p.cluster, grid_y, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = p.dyn_bytes;
   cfg.stream = st;
@@ -656,7 +670,7 @@ cudaError_t launch_t(const SelectArgs &a, const Shape &sh, const Tables &tb, con
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, select_kernel<GR, TOPP, SMEM>, a, sh, tb.ret, tb.n_ret, p.tc_cap);
+  return cudaLaunchKernelEx(&cfg, select_kernel<GR, TOPP, SMEM>, a, sh, tb.ret, tb.n_ret, p.tc_cap, flags);
 }
 
 template <bool TOPP, bool SMEM>
@@ -672,13 +686,13 @@ int active_clusters_gr(const Tables &tb, const Plan &p, int dev) {
 
 template <bool TOPP, bool SMEM>
 cudaError_t dispatch_gr(const SelectArgs &a, const Shape &sh, const Tables &tb, const Plan &p, int dev,
-                        cudaStream_t st) {
+                        cudaStream_t st, const uint32_t *flags, int grid_y) {
   switch (group_rows(tb)) {
-    case 1: return launch_t<1, TOPP, SMEM>(a, sh, tb, p, dev, st);
-    case 2: return launch_t<2, TOPP, SMEM>(a, sh, tb, p, dev, st);
-    case 4: return launch_t<4, TOPP, SMEM>(a, sh, tb, p, dev, st);
-    case 8: return launch_t<8, TOPP, SMEM>(a, sh, tb, p, dev, st);
-    default: return launch_t<16, TOPP, SMEM>(a, sh, tb, p, dev, st);
+    case 1: return launch_t<1, TOPP, SMEM>(a, sh, tb, p, dev, st, flags, grid_y);
+    case 2: return launch_t<2, TOPP, SMEM>(a, sh, tb, p, dev, st, flags, grid_y);
+    case 4: return launch_t<4, TOPP, SMEM>(a, sh, tb, p, dev, st, flags, grid_y);
+    case 8: return launch_t<8, TOPP, SMEM>(a, sh, tb, p, dev, st, flags, grid_y);
+    default: return launch_t<16, TOPP, SMEM>(a, sh, tb, p, dev, st, flags, grid_y);
   }
 }
 
@@ -691,9 +705,13 @@ int smem_limit_bytes() {
 
 }  // namespace
 
-size_t select_workspace_bytes(const Shape &sh, const Tables &tb, int batch) {
-  // global score rows, used when the scores of a chunk do not fit on chip
-  return (size_t)batch * sh.H_ret * (size_t)sh.max_len * sizeof(float);
+size_t select_workspace_bytes(const Shape &sh, const Tables &tb, int batch, size_t *flags_off) {
+  // global score rows (used when the scores of a chunk do not fit on chip),
+  // then one flag per work item
+  size_t rows = (size_t)batch * sh.H_ret * (size_t)sh.max_len * sizeof(float);
+  rows = (rows + 255) / 256 * 256;
+  if (flags_off) *flags_off = rows;
+  return rows + (size_t)batch * std::max(1, tb.n_ret) * sizeof(uint32_t);
 }
 
 cudaError_t launch_select(const SelectArgs &a, const Shape &sh, const Tables &tb, cudaStream_t st) {
@@ -722,8 +740,22 @@ cudaError_t launch_select(const SelectArgs &a, const Shape &sh, const Tables &tb
     p.tc_cap = (int)(((sh.max_len + c - 1) / c + kPage - 1) / kPage * kPage);
     p.dyn_bytes = hist_bytes(group_rows(tb), topp);
   }
-  if (topp) return p.smem ? dispatch_gr<true, true>(a, sh, tb, p, dev, st) : dispatch_gr<true, false>(a, sh, tb, p, dev, st);
-  return p.smem ? dispatch_gr<false, true>(a, sh, tb, p, dev, st) : dispatch_gr<false, false>(a, sh, tb, p, dev, st);
+  const int items = a.batch * tb.n_ret;
+  if (!topp) {
+    bool used = false;
+    cudaError_t e = launch_select_topk_stream(a, sh, tb, a.flags, st, &used);
+    if (e != cudaSuccess) return e;
+    if (used) {
+      // exact recomputation of the items whose window missed (usually none)
+      const int gy = std::min(items, 16);
+      return p.smem ? dispatch_gr<false, true>(a, sh, tb, p, dev, st, a.flags, gy)
+                    : dispatch_gr<false, false>(a, sh, tb, p, dev, st, a.flags, gy);
+    }
+    return p.smem ? dispatch_gr<false, true>(a, sh, tb, p, dev, st, nullptr, items)
+                  : dispatch_gr<false, false>(a, sh, tb, p, dev, st, nullptr, items);
+  }
+  return p.smem ? dispatch_gr<true, true>(a, sh, tb, p, dev, st, nullptr, items)
+                : dispatch_gr<true, false>(a, sh, tb, p, dev, st, nullptr, items);
 }
 
 }  // namespace sd
