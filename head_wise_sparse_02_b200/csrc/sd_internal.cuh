@@ -93,14 +93,17 @@ struct SelectArgs {
   float top_k_frac;
   float *score_ws;                // global score rows when they do not fit on chip
   uint32_t *flags;                // [batch * n_ret] streaming top-k misses
+  void *topk_ws;                  // streaming top-k scratch (histograms, buffers)
   unsigned *err;
   int batch;
 };
 
 size_t select_workspace_bytes(const Shape &sh, const Tables &tb, int batch, size_t *flags_off);
+size_t select_topk_offset(const Shape &sh, const Tables &tb, int batch);
 cudaError_t launch_select(const SelectArgs &a, const Shape &sh, const Tables &tb, cudaStream_t st);
+size_t topk_workspace_bytes(const Shape &sh, const Tables &tb, int batch);
 cudaError_t launch_select_topk_stream(const SelectArgs &a, const Shape &sh, const Tables &tb, uint32_t *fail,
-                                      cudaStream_t st, bool *used);
+                                      void *ws_base, cudaStream_t st, bool *used);
 
 struct AttendArgs {
   const uint16_t *q;

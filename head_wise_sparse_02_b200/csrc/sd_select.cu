@@ -714,6 +714,11 @@ size_t select_workspace_bytes(const Shape &sh, const Tables &tb, int batch, size
   return rows + (size_t)batch * std::max(1, tb.n_ret) * sizeof(uint32_t);
 }
 
+size_t select_topk_offset(const Shape &sh, const Tables &tb, int batch) {
+  size_t f = 0;
+  return (select_workspace_bytes(sh, tb, batch, &f) + 255) / 256 * 256;
+}
+
 cudaError_t launch_select(const SelectArgs &a, const Shape &sh, const Tables &tb, cudaStream_t st) {
   if (tb.n_ret == 0 || a.batch == 0) return cudaSuccess;
   int dev = 0;
@@ -743,7 +748,7 @@ cudaError_t launch_select(const SelectArgs &a, const Shape &sh, const Tables &tb
   const int items = a.batch * tb.n_ret;
   if (!topp) {
     bool used = false;
-    cudaError_t e = launch_select_topk_stream(a, sh, tb, a.flags, st, &used);
+    cudaError_t e = launch_select_topk_stream(a, sh, tb, a.flags, a.topk_ws, st, &used);
     if (e != cudaSuccess) return e;
     if (used) {
       // exact recomputation of the items whose window missed (usually none)

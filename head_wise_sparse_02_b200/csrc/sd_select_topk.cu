@@ -1,86 +1,57 @@
-// Fixed-budget (top-k) selection in one pass over the index.
+// Fixed-budget (top-k) selection: one streaming pass over the index.
 //
 // RTPurbo page (gist.science/ar/paper/2605.16928), Methodology 2-3 and 5: the
 // tokens of a retrieval head are scored in the r = 16 index space and a fixed
-// top-k budget is taken; the threshold comes from a histogram, without
+// top-k budget is kept; the threshold comes from a histogram, without
 // sorting.  ICS page (gist.science/ar/paper/2605.24168), 2 and 3a: exact
 // ("Oracle") top-k at ~2% of the context.
 //
-// One thread-block cluster of C CTAs per (sequence, KV group); each CTA owns a
-// page-aligned chunk of the context and reads its index entries once.
-//
-//   1. Scores on the tensor cores: a 16-token page of the index of one KV
-//      head (16 x 16 bf16) is the A operand of mma.m16n8k16; the B operand
-//      holds q~ of the group's heads split into three bf16 terms
-//      (q~ = hi + mid + lo, each the bf16 rounding of the remainder), so the
-//      float32 accumulation reproduces the float32 score to ~2^-24 relative.
-//   2. Each CTA first scores a strided sample of its pages (<= 64 pages) and
-//      derives from it a conservative score window [t_lo, t_hi): t_lo is a
-//      sample quantile safely below the k-th score, t_hi the sample maximum.
-//      The cluster agrees on the widest window (min of t_lo, max of t_hi).
-//   3. Streaming the rest of the chunk, every score at or above t_lo goes to
-//      a small per-head list (score, position) and, when below t_hi, to a
-//      512-bin linear histogram of the window.  Nothing else is kept.
-//   4. The histograms are reduced across the cluster (distributed shared
-//      memory); the bin holding the k-th score is found scanning down from
-//      the top, and the few tokens of that bin are sent to the head's owner
-//      CTA, which ranks them exactly by (score desc, position asc).  This
-//      yields the threshold as a (score, position) pair.
-//   5. Each CTA marks its selected list entries in a bitmap of its chunk and
-//      writes their positions in ascending order at its cluster offset.
-// If the window misses (list overflow, k-th score outside the window, too
-// many candidates in the cut bin), the cluster flags its work item and the
-// exact general kernel recomputes it.
-#include <cooperative_groups.h>
+// Three launches, none of which waits on another CTA:
+//   K0 window  one CTA per (sequence, KV group).  Computes q~ = c P_g^T q_pre
+//              (float64, rounded to float32, split exactly into three bf16
+//              terms) and scores a strided sample of <= 256 pages; from the
+//              sample it sets, per head, a conservative score window
+//              [t_lo, t_hi): t_lo a sample quantile safely below the k-th
+//              score, t_hi the sample maximum.  Zeroes the head's histogram
+//              and buffer counter.
+//   K1 stream  many CTAs, each 512 pages of one (sequence, KV group): pages
+//              arrive through a per-warp cp.async ring (16 bytes per lane,
+//              XOR-swizzled rows), ldmatrix + mma.m16n8k16 score all heads of
+//              the group at once (A = the 16 x 16 bf16 index page, B = the q~
+//              terms), and every score at or above t_lo goes to a global
+//              512-bin histogram of the window (or a count of scores at or
+//              above t_hi) and, with its position, to a per-head buffer
+//              (staged per warp in shared memory, flushed in batches).
+//   K2 resolve one CTA per (sequence, retrieval head): scans the histogram
+//              from the top for the bin holding the k-th score, ranks the
+//              tokens of that bin exactly by (score desc, position asc),
+//              marks the selected positions in a bitmap of the context and
+//              writes them in ascending order.
+// If the window misses (buffer overflow, k-th score outside the window, too
+// many tokens in the cut bin), K2 flags the work item and the exact general
+// kernel recomputes it.
+#include <cuda_bf16.h>
 
 #include <algorithm>
 #include <map>
 #include <mutex>
-#include <tuple>
 
 #include "sd_internal.cuh"
-
-namespace cg = cooperative_groups;
 
 namespace sd {
 namespace {
 
-constexpr int kT = 256;
-constexpr int kW = kT / 32;
-constexpr int kBins = 512;            // window histogram
-constexpr int kTopClass = kBins;      // class of scores at or above t_hi
-constexpr int kSampleTiles = 64;      // sampled pages per CTA
-constexpr int kSampleBins = 64;
-constexpr int kCap = 1024;            // cut-bin candidates ranked exactly per head
-constexpr int kMaxCluster = 16;
-constexpr int kUnroll = 4;            // pages in flight per warp
+constexpr int kBins = 512;            // window histogram bins (+1 slot: scores >= t_hi)
+// K0: sampled pages per (sequence, group); the sample store is capped at 96 KB
+__host__ __device__ constexpr int sample_pages(int GR) { return GR <= 4 ? 256 : (GR == 8 ? 192 : 96); }
+constexpr int kSampleBins = 256;
+constexpr int kChunkPages = 512;      // K1: pages per CTA
+constexpr int kRing = 8;              // K1: pages in flight per warp
+// K1: staged buffer entries per (warp, head)
+__host__ __device__ constexpr int stage_entries(int GR) { return GR <= 4 ? 64 : 32; }
+constexpr int kCap = 2048;            // K2: cut-bin tokens ranked exactly
+constexpr int kPageBytes = kPage * kIndexDim * 2;   // 512 B: one page of one KV head
 constexpr unsigned kFull = 0xFFFFFFFFu;
-
-struct TopkParams {
-  int tc_cap;                         // tokens per CTA (capacity, multiple of 16)
-  int list_cap;                       // list entries per head per CTA
-  int own_slots;                      // heads owned per CTA
-  uint32_t *fail;                     // [items]: 1 = needs the exact general kernel
-};
-
-struct TkShared {
-  Group grp;
-  uint32_t qs[3][kMaxGroup][kIndexDim / 2];   // q~ terms hi / mid / lo, bf16 pairs
-  uint32_t smax[kMaxGroup], smin[kMaxGroup];
-  uint32_t tlo_key[kMaxGroup], thi_key[kMaxGroup];
-  float tlo[kMaxGroup], thi[kMaxGroup], inv[kMaxGroup];
-  uint32_t list_n[kMaxGroup];
-  uint32_t top_n[kMaxGroup];
-  uint32_t overflow;
-  uint32_t slice_cnt[kMaxGroup];
-  int cut[kMaxGroup];
-  long long need_c[kMaxGroup];
-  int fail;
-  uint32_t above_local[kMaxGroup];
-  uint32_t cand_n[kMaxGroup];
-  unsigned long long tau_sk[kMaxGroup];
-  uint32_t wtot[kW];
-};
 
 __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -89,194 +60,209 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
       : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.0f));
 }
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
+// byte offset of the 16-byte half `half` of row `row` inside a staged page;
+// halves of rows 4-7 and 12-15 are swapped so that the eight rows an ldmatrix
+// phase reads fall in distinct banks
+__device__ __forceinline__ uint32_t page_off(int row, int half) {
+  return (uint32_t)(row * 32 + ((half ^ ((row >> 2) & 1)) << 4));
+}
+__device__ __forceinline__ uint16_t bf16_rn(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
+__device__ __forceinline__ float bf16_val(uint16_t h) { return __uint_as_float(uint32_t(h) << 16); }
 
-__device__ __forceinline__ double bf16_bits_to_f64(uint16_t h) { return (double)__uint_as_float(uint32_t(h) << 16); }
-
-__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory"); }
-__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory"); }
-
-// sort key: ascending order = score descending, then position ascending
-__device__ __forceinline__ unsigned long long sort_key(float s, uint32_t pos) {
-  return ((unsigned long long)(~order_key(s)) << 32) | pos;
+// class of a score in the window of its head: kBins for scores >= t_hi, else
+// the linear bin of [t_lo, t_hi); the same arithmetic in K1 and K2
+__device__ __forceinline__ int window_bin(float s, float tlo, float thi, float inv) {
+  if (s >= thi) return kBins;
+  return min(kBins - 1, max(0, __float2int_rz((s - tlo) * inv)));
 }
 
-struct TkLayout {
-  size_t sample, whist, wred, list, cand, occ, bitmap, total;
+struct TopkWs {
+  uint32_t *qsplit;                   // [rows][24]: bf16 pairs of the q~ terms hi, mid, lo
+  float4 *win;                        // [rows]: t_lo, t_hi, 1 / bin width, unused
+  uint32_t *hist;                     // [rows][kBins + 1]
+  uint32_t *bcount;                   // [rows] buffer entries written
+  int *rowitem;                       // [rows] work item of the row
+  unsigned long long *buf;            // [rows][cap]: order key << 32 | position
+  uint32_t *fail;                     // [items]
+  int cap;
 };
 
-__host__ __device__ inline TkLayout tk_layout(int GR, int tc_cap, int list_cap, int own_slots) {
-  TkLayout L{};
-  size_t o = 0;
-  L.list = o;   o += (size_t)GR * list_cap * 8;
-  L.cand = o;   o += (size_t)own_slots * kCap * 8;
-  L.sample = o; o += (size_t)GR * kSampleTiles * 16 * 4;
-  L.whist = o;  o += (size_t)GR * kBins * 4;
-  L.wred = o;   o += (size_t)GR * kBins * 4;
-  L.occ = o;    o += (size_t)own_slots * kMaxCluster * 4;
-  L.bitmap = o; o += (size_t)GR * (tc_cap / 32) * 4;
-  L.total = o;
-  return L;
+// B fragments of mma.m16n8k16 for head block hb: column n = gq of the first
+// MMA carries head 4hb + gq/2, term gq%2 (hi, mid); of the second, the lo term
+// for even gq and zero for odd gq.
+struct BFrag {
+  uint32_t v[2][2];
+};
+__device__ __forceinline__ BFrag load_bfrag(const uint32_t *qs /* [16 heads][24] */, int hb, int gq, int tq) {
+  const int head = hb * 4 + (gq >> 1);
+  const int part = gq & 1;
+  const uint32_t *q = qs + head * 24;
+  BFrag f;
+  f.v[0][0] = q[part * 8 + tq];
+  f.v[0][1] = q[part * 8 + tq + 4];
+  f.v[1][0] = part == 0 ? q[16 + tq] : 0u;
+  f.v[1][1] = part == 0 ? q[16 + tq + 4] : 0u;
+  return f;
 }
-
-template <int GR>
-__global__ void __launch_bounds__(kT, 2)
-topk_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__ groups, int n_groups,
-            const TopkParams tp) {
-  constexpr int HB = (GR + 3) / 4;                   // 4-head blocks of the MMA
-  cg::cluster_group cluster = cg::this_cluster();
-  const int C = (int)cluster.num_blocks();
-  const int rank = (int)cluster.block_rank();
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int gq = lane >> 2, tq = lane & 3;
-  const int item = blockIdx.y;
-  const int b = item / n_groups, gi = item % n_groups;
-
-  __shared__ TkShared S;
-  extern __shared__ __align__(16) unsigned char dyn[];
-  const TkLayout L = tk_layout(GR, tp.tc_cap, tp.list_cap, tp.own_slots);
-  unsigned long long *list = reinterpret_cast<unsigned long long *>(dyn + L.list);
-  unsigned long long *cand = reinterpret_cast<unsigned long long *>(dyn + L.cand);
-  float *sample = reinterpret_cast<float *>(dyn + L.sample);
-  uint32_t *whist = reinterpret_cast<uint32_t *>(dyn + L.whist);
-  uint32_t *wred = reinterpret_cast<uint32_t *>(dyn + L.wred);
-  uint32_t *occ = reinterpret_cast<uint32_t *>(dyn + L.occ);
-  uint32_t *bitmap = reinterpret_cast<uint32_t *>(dyn + L.bitmap);
-  const int words = tp.tc_cap / 32;
-
-  if (tid == 0) S.grp = groups[gi];
-  __syncthreads();
-  const int nr = S.grp.n;
-  const int g = S.grp.kv_head;
-
-  long long N = a.seq_lens[b];
-  if (N < 0 || N > sh.max_len) {
-    if (tid == 0 && rank == 0) raise_error(a.err, SD_EBIT_SEQLEN);
-    N = N < 0 ? 0 : sh.max_len;
-  }
-  const long long per_cta = ((N + C - 1) / C + kPage - 1) / kPage * kPage;
-  const long long t0 = std::min(N, (long long)rank * per_cta);
-  const long long t1 = std::min(N, t0 + per_cta);
-  const int cnt = (int)(t1 - t0);
-  const int ntiles = (cnt + kPage - 1) / kPage;
-
-  auto sel_row = [&](int i) { return a.sel_idx + ((long long)b * sh.H_ret + S.grp.row[i]) * a.sel_stride; };
-  auto count_slot = [&](int i) { return a.sel_count + (long long)b * sh.H_ret + S.grp.row[i]; };
-
-  long long kb = a.top_k > 0 ? (long long)a.top_k
-                             : std::max(1LL, (long long)floor((double)a.top_k_frac * (double)N));
-  kb = std::min(kb, N);
-  if (N == 0 || kb >= N) {                           // the whole context (or nothing)
-    for (int i = 0; i < nr; ++i) {
-      int32_t *row = sel_row(i);
-      for (long long t = t0 + tid; t < t1; t += kT) {
-        if (t < a.sel_stride) row[t] = (int32_t)t;
-        else raise_error(a.err, SD_EBIT_SEL);
-      }
-      if (rank == 0 && tid == 0) *count_slot(i) = (int32_t)std::min(N, a.sel_stride);
-    }
-    if (rank == 0 && tid == 0) tp.fail[item] = 0u;
-    return;
-  }
-
-  // ---- q~ = c P_g^T q_pre in float64, split into three bf16 terms ----------
-  for (int o = tid; o < kMaxGroup * kIndexDim; o += kT) {
-    const int i = o / kIndexDim, j = o % kIndexDim;
-    uint16_t hi = 0, mid = 0, lo = 0;
-    if (i < nr) {
-      const uint16_t *qrow = a.q_pre + ((long long)b * sh.Hq + S.grp.q_head[i]) * sh.d;
-      const uint16_t *P = a.proj + (long long)g * sh.d * kIndexDim;
-      double acc = 0.0;
-      for (int e = 0; e < sh.d; ++e)
-        acc = fma((double)bf16_to_f32(qrow[e]), (double)bf16_to_f32(P[e * kIndexDim + j]), acc);
-      acc *= (double)a.index_scale;
-      hi = f64_to_bf16_rne(acc);
-      const double r1 = acc - bf16_bits_to_f64(hi);
-      mid = f64_to_bf16_rne(r1);
-      lo = f64_to_bf16_rne(r1 - bf16_bits_to_f64(mid));
-    }
-    uint16_t *q0 = reinterpret_cast<uint16_t *>(&S.qs[0][i][0]);
-    uint16_t *q1 = reinterpret_cast<uint16_t *>(&S.qs[1][i][0]);
-    uint16_t *q2 = reinterpret_cast<uint16_t *>(&S.qs[2][i][0]);
-    q0[j] = hi;
-    q1[j] = mid;
-    q2[j] = lo;
-  }
-  if (tid < kMaxGroup) {
-    S.smax[tid] = 0u;
-    S.smin[tid] = 0xFFFFFFFFu;
-    S.list_n[tid] = 0u;
-    S.top_n[tid] = 0u;
-    S.cand_n[tid] = 0u;
-    S.above_local[tid] = 0u;
-  }
-  if (tid == 0) {
-    S.overflow = 0u;
-    S.fail = 0;
-  }
-  for (int o = tid; o < GR * kBins; o += kT) whist[o] = 0u;
-  for (int o = tid; o < tp.own_slots * kMaxCluster; o += kT) occ[o] = 0u;
-  for (int o = tid; o < GR * words; o += kT) bitmap[o] = 0u;
-  __syncthreads();
-
-  // B fragments: column n = gq of the first MMA carries head 4hb + gq/2, term
-  // gq%2 (hi, mid); of the second MMA, the lo term for even gq, zero for odd.
-  uint32_t bf[HB][2][2];
+template <int HB>
+__device__ __forceinline__ void score_frag(const uint32_t (&af)[4], const BFrag (&bf)[HB], float (&out)[HB][2]) {
 #pragma unroll
   for (int hb = 0; hb < HB; ++hb) {
-    const int head = hb * 4 + (gq >> 1);
-    const int part = gq & 1;
-    bf[hb][0][0] = S.qs[part][head][tq];
-    bf[hb][0][1] = S.qs[part][head][tq + 4];
-    bf[hb][1][0] = part == 0 ? S.qs[2][head][tq] : 0u;
-    bf[hb][1][1] = part == 0 ? S.qs[2][head][tq + 4] : 0u;
+    float d[4], e[4];
+    mma_16816(d, af, bf[hb].v[0][0], bf[hb].v[0][1]);
+    mma_16816(e, af, bf[hb].v[1][0], bf[hb].v[1][1]);
+    out[hb][0] = (d[0] + d[1]) + e[0];               // row gq
+    out[hb][1] = (d[2] + d[3]) + e[2];               // row gq + 8
   }
+}
+
+__device__ __forceinline__ long long topk_budget(const SelectArgs &a, long long N) {
+  long long kb = a.top_k > 0 ? (long long)a.top_k
+                             : std::max(1LL, (long long)floor((double)a.top_k_frac * (double)N));
+  return std::min(kb, N);
+}
+
+// ------------------------------------------------------------------- K0
+constexpr int kT0 = 256;
+
+template <int GR>
+__global__ void __launch_bounds__(kT0)
+topk_window_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__ groups, int n_groups,
+                   const TopkWs ws) {
+  constexpr int HB = (GR + 3) / 4;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gq = lane >> 2, tq = lane & 3;
+  const int item = blockIdx.x;
+  const int b = item / n_groups, gi = item % n_groups;
+  constexpr int SP = sample_pages(GR);
+  __shared__ Group grp;
+  __shared__ uint32_t qs[16 * 24];
+  __shared__ uint32_t smax[GR], smin[GR];
+  extern __shared__ __align__(16) unsigned char dyn0[];
+  float (*sample)[SP * 16] = reinterpret_cast<float (*)[SP * 16]>(dyn0);
+  uint32_t (*shist)[kSampleBins] = reinterpret_cast<uint32_t (*)[kSampleBins]>(dyn0 + (size_t)GR * SP * 16 * 4);
+  if (tid == 0) grp = groups[gi];
+  __syncthreads();
+  const int nr = grp.n, g = grp.kv_head;
+  long long N = a.seq_lens[b];
+  N = N < 0 ? 0 : std::min<long long>(N, sh.max_len);
+  const long long kb = topk_budget(a, N);
+  if (tid == 0) ws.fail[item] = 0u;
+  for (int o = tid; o < nr * (kBins + 1); o += kT0) {
+    const int i = o / (kBins + 1);
+    ws.hist[((long long)b * sh.H_ret + grp.row[i]) * (kBins + 1) + o % (kBins + 1)] = 0u;
+  }
+  if (tid < nr) {
+    ws.bcount[(long long)b * sh.H_ret + grp.row[tid]] = 0u;
+    ws.rowitem[(long long)b * sh.H_ret + grp.row[tid]] = item;
+  }
+  if (N == 0 || kb >= N) return;                     // K1 skips, K2 keeps everything
+
+  // q~ in float64 (one warp per head, lanes split d) -> float32 -> hi/mid/lo
+  for (int i = warp; i < 16; i += kT0 / 32) {
+    double acc[kIndexDim];
+#pragma unroll
+    for (int j = 0; j < kIndexDim; ++j) acc[j] = 0.0;
+    if (i < nr) {
+      const uint16_t *qrow = a.q_pre + ((long long)b * sh.Hq + grp.q_head[i]) * sh.d;
+      const uint16_t *P = a.proj + (long long)g * sh.d * kIndexDim;
+      for (int e = lane; e < sh.d; e += 32) {
+        const double qe = (double)bf16_to_f32(qrow[e]);
+        const uint4 p0 = __ldg(reinterpret_cast<const uint4 *>(P + e * kIndexDim));
+        const uint4 p1 = __ldg(reinterpret_cast<const uint4 *>(P + e * kIndexDim + 8));
+        const uint32_t pw[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          acc[2 * j] = fma(qe, (double)bf16_lo(pw[j]), acc[2 * j]);
+          acc[2 * j + 1] = fma(qe, (double)bf16_hi(pw[j]), acc[2 * j + 1]);
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kIndexDim; ++j)
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc[j] += __shfl_xor_sync(kFull, acc[j], o);
+    if (lane < kIndexDim) {
+      double v = 0.0;
+#pragma unroll
+      for (int j = 0; j < kIndexDim; ++j) v = (lane == j) ? acc[j] : v;
+      const float x = (float)(v * (double)a.index_scale);
+      const uint16_t hi = bf16_rn(x);
+      const float r1 = x - bf16_val(hi);             // exact in float32
+      const uint16_t mid = bf16_rn(r1);
+      const uint16_t lo = bf16_rn(r1 - bf16_val(mid));
+      uint16_t *q16 = reinterpret_cast<uint16_t *>(qs + i * 24);
+      q16[lane] = hi;
+      q16[16 + lane] = mid;
+      q16[32 + lane] = lo;
+    }
+  }
+  if (tid < GR) {
+    smax[tid] = 0u;
+    smin[tid] = 0xFFFFFFFFu;
+  }
+  for (int o = tid; o < GR * kSampleBins; o += kT0) (&shist[0][0])[o] = 0u;
+  __syncthreads();
+  for (int o = tid; o < nr * 24; o += kT0)           // publish the q~ terms for K1
+    ws.qsplit[((long long)b * sh.H_ret + grp.row[o / 24]) * 24 + o % 24] = qs[o];
+
+  // sample: pages j * st, j < ns
+  const int pages = (int)((N + kPage - 1) / kPage);
+  int st = 1;
+  while ((long long)st * SP < pages) st <<= 1;
+  const int ns = (pages + st - 1) / st;
+  BFrag bf[HB];
+#pragma unroll
+  for (int hb = 0; hb < HB; ++hb) bf[hb] = load_bfrag(qs, hb, gq, tq);
   const int32_t *pt = a.page_table + (long long)b * sh.max_pages;
-  const uint16_t *icache = a.index_cache;
-
-  auto load_tile = [&](int tile, uint32_t (&af)[4]) -> bool {
-    const long long pos0 = t0 + (long long)tile * kPage;
-    const int page = pt[pos0 / kPage];
-    if (page < 0 || page >= sh.num_pages) {
-      if (lane == 0) raise_error(a.err, SD_EBIT_PAGE);
-      af[0] = af[1] = af[2] = af[3] = 0u;
-      return false;
-    }
-    const uint32_t *pg =
-        reinterpret_cast<const uint32_t *>(icache + ((long long)page * sh.Hkv + g) * (kPage * kIndexDim));
-    af[0] = __ldg(pg + gq * 8 + tq);
-    af[1] = __ldg(pg + (gq + 8) * 8 + tq);
-    af[2] = __ldg(pg + gq * 8 + tq + 4);
-    af[3] = __ldg(pg + (gq + 8) * 8 + tq + 4);
-    return true;
-  };
-  // scores of rows gq and gq + 8 for head 4hb + tq
-  auto score_tile = [&](const uint32_t (&af)[4], float (&out)[HB][2]) {
+  const uint16_t *icache = a.index_cache + (long long)g * (kPage * kIndexDim);
+  const long long page_stride = (long long)sh.Hkv * (kPage * kIndexDim);
+  float smx[HB], smn[HB];
 #pragma unroll
-    for (int hb = 0; hb < HB; ++hb) {
-      float d[4], e[4];
-      mma_16816(d, af, bf[hb][0][0], bf[hb][0][1]);
-      mma_16816(e, af, bf[hb][1][0], bf[hb][1][1]);
-      out[hb][0] = (d[0] + d[1]) + e[0];
-      out[hb][1] = (d[2] + d[3]) + e[2];
-    }
-  };
-
-  // ---- 1. sample --------------------------------------------------------------
-  const int st = std::max(1, (ntiles + kSampleTiles - 1) / kSampleTiles);
-  const int ns = (ntiles + st - 1) / st;
-  {
-    float smx[HB], smn[HB];
+  for (int hb = 0; hb < HB; ++hb) {
+    smx[hb] = -INFINITY;
+    smn[hb] = INFINITY;
+  }
+  constexpr int U = 8;
+  for (int j0 = warp; j0 < ns; j0 += (kT0 / 32) * U) {
+    uint32_t af[U][4];
+    bool ok[U];
 #pragma unroll
-    for (int hb = 0; hb < HB; ++hb) {
-      smx[hb] = -INFINITY;
-      smn[hb] = INFINITY;
+    for (int u = 0; u < U; ++u) {
+      const int j = j0 + u * (kT0 / 32);
+      ok[u] = false;
+      af[u][0] = af[u][1] = af[u][2] = af[u][3] = 0u;
+      if (j < ns) {
+        const int page = pt[j * st];
+        if (page >= 0 && page < sh.num_pages) {
+          const uint32_t *pg = reinterpret_cast<const uint32_t *>(icache + page * page_stride);
+          af[u][0] = __ldg(pg + gq * 8 + tq);
+          af[u][1] = __ldg(pg + (gq + 8) * 8 + tq);
+          af[u][2] = __ldg(pg + gq * 8 + tq + 4);
+          af[u][3] = __ldg(pg + (gq + 8) * 8 + tq + 4);
+          ok[u] = true;
+        } else if (lane == 0) {
+          raise_error(a.err, SD_EBIT_PAGE);
+        }
+      }
     }
-    for (int j = warp; j < ns; j += kW) {
-      const int tile = j * st;
-      uint32_t af[4];
-      const bool ok = load_tile(tile, af);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int j = j0 + u * (kT0 / 32);
+      if (j >= ns) break;
       float sc[HB][2];
-      score_tile(af, sc);
+      score_frag<HB>(af[u], bf, sc);
 #pragma unroll
       for (int hb = 0; hb < HB; ++hb) {
         const int h = hb * 4 + tq;
@@ -284,9 +270,9 @@ topk_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__ groups
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
           const int row = gq + 8 * r;
-          const bool valid = ok && tile * kPage + row < cnt;
+          const bool valid = ok[u] && (long long)j * st * kPage + row < N;
           const float v = valid ? sc[hb][r] : -INFINITY;
-          sample[h * (kSampleTiles * 16) + j * 16 + row] = v;
+          sample[h][j * 16 + row] = v;
           if (valid) {
             smx[hb] = fmaxf(smx[hb], v);
             smn[hb] = fminf(smn[hb], v);
@@ -294,457 +280,439 @@ topk_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__ groups
         }
       }
     }
+  }
 #pragma unroll
-    for (int hb = 0; hb < HB; ++hb) {
+  for (int hb = 0; hb < HB; ++hb) {
 #pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
-        smx[hb] = fmaxf(smx[hb], __shfl_xor_sync(kFull, smx[hb], o));
-        smn[hb] = fminf(smn[hb], __shfl_xor_sync(kFull, smn[hb], o));
-      }
-      const int h = hb * 4 + tq;
-      if (gq == 0 && h < nr && smx[hb] > -INFINITY) {
-        atomicMax(&S.smax[h], order_key(smx[hb]));
-        atomicMin(&S.smin[h], order_key(smn[hb]));
-      }
+    for (int o = 4; o < 32; o <<= 1) {
+      smx[hb] = fmaxf(smx[hb], __shfl_xor_sync(kFull, smx[hb], o));
+      smn[hb] = fminf(smn[hb], __shfl_xor_sync(kFull, smn[hb], o));
+    }
+    const int h = hb * 4 + tq;
+    if (gq == 0 && h < nr && smx[hb] > -INFINITY) {
+      atomicMax(&smax[h], order_key(smx[hb]));
+      atomicMin(&smin[h], order_key(smn[hb]));
     }
   }
   __syncthreads();
-  // local window estimate from a 64-bin histogram of the sample
-  uint32_t *shist = wred;                            // scratch until the reduction
-  for (int o = tid; o < GR * kSampleBins; o += kT) shist[o] = 0u;
-  __syncthreads();
-  int n_sample = 0;                                  // valid sample tokens (same for every head)
-  for (int j = 0; j < ns; ++j) n_sample += std::max(0, std::min(16, cnt - j * st * kPage));
-  for (int o = tid; o < nr * ns * 16; o += kT) {
+  for (int o = tid; o < nr * ns * 16; o += kT0) {
     const int h = o / (ns * 16), r = o % (ns * 16);
-    const float v = sample[h * (kSampleTiles * 16) + r];
+    const float v = sample[h][r];
     if (v == -INFINITY) continue;
-    const float lo = key_to_float(S.smin[h]), hi = key_to_float(S.smax[h]);
+    const float lo = key_to_float(smin[h]), hi = key_to_float(smax[h]);
     const float inv = hi > lo ? (float)kSampleBins / (hi - lo) : 0.0f;
-    const int bin = std::min(kSampleBins - 1, std::max(0, __float2int_rz((v - lo) * inv)));
-    atomicAdd(&shist[h * kSampleBins + bin], 1u);
+    atomicAdd(&shist[h][std::min(kSampleBins - 1, std::max(0, __float2int_rz((v - lo) * inv)))], 1u);
   }
   __syncthreads();
   if (tid < nr) {
     const int h = tid;
-    uint32_t lo_key = 0xFFFFFFFFu, hi_key = 0u;      // neutral for the cluster min / max
-    if (n_sample > 0 && S.smax[h] != 0u) {
-      const double mu = (double)n_sample * (double)kb / (double)N;
+    long long m = 0;                                 // valid sample tokens
+    for (int j = 0; j < ns; ++j) m += std::max(0LL, std::min<long long>(16, N - (long long)j * st * kPage));
+    float tlo = -INFINITY, thi = INFINITY;
+    if (smax[h] != 0u) {
+      const float lo = key_to_float(smin[h]), hi = key_to_float(smax[h]);
+      thi = hi;
+      const double mu = (double)m * (double)kb / (double)N;
       const double r = ceil(mu + 6.0 * sqrt(mu) + 8.0);
-      hi_key = S.smax[h];
-      if (r < (double)n_sample) {
-        const float lo = key_to_float(S.smin[h]), hi = key_to_float(S.smax[h]);
+      if (r < (double)m) {
         uint32_t cum = 0;
         int blo = 0;
         for (int bin = kSampleBins - 1; bin >= 0; --bin) {
-          cum += shist[h * kSampleBins + bin];
+          cum += shist[h][bin];
           if ((double)cum >= r) {
             blo = bin;
             break;
           }
         }
-        const float edge = lo + (float)blo * ((hi - lo) / (float)kSampleBins);
-        lo_key = order_key(edge);
-      } else {
-        lo_key = 0u;                                 // no estimate: the window starts at -inf
+        tlo = lo + (float)blo * ((hi - lo) / (float)kSampleBins);
       }
     }
-    S.tlo_key[h] = lo_key;
-    S.thi_key[h] = hi_key;
+    const float inv = (tlo > -INFINITY && thi > tlo) ? (float)kBins / (thi - tlo) : 0.0f;
+    ws.win[(long long)b * sh.H_ret + grp.row[h]] = make_float4(tlo, thi, inv, 0.0f);
   }
-  cluster.sync();                                    // B1: local windows published
-  for (int h = warp; h < nr; h += kW) {
-    uint32_t lo = lane < C ? *cluster.map_shared_rank(&S.tlo_key[h], lane) : 0xFFFFFFFFu;
-    uint32_t hi = lane < C ? *cluster.map_shared_rank(&S.thi_key[h], lane) : 0u;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      lo = std::min(lo, __shfl_xor_sync(kFull, lo, o));
-      hi = std::max(hi, __shfl_xor_sync(kFull, hi, o));
+}
+
+// ------------------------------------------------------------------- K1
+constexpr int kT1 = 256;
+constexpr int kW1 = kT1 / 32;
+
+template <int GR>
+__global__ void __launch_bounds__(kT1)
+topk_stream_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__ groups, int n_groups,
+                   const TopkWs ws) {
+  constexpr int HB = (GR + 3) / 4;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gq = lane >> 2, tq = lane & 3;
+  const int item = blockIdx.y;
+  const int b = item / n_groups, gi = item % n_groups;
+  constexpr int SE = stage_entries(GR);
+  extern __shared__ __align__(128) unsigned char dyn1[];
+  unsigned char (*ring)[kRing][kPageBytes] = reinterpret_cast<unsigned char (*)[kRing][kPageBytes]>(dyn1);
+  unsigned long long (*stage)[GR][SE] =
+      reinterpret_cast<unsigned long long (*)[GR][SE]>(dyn1 + (size_t)kW1 * kRing * kPageBytes);
+  __shared__ int32_t pt_s[kChunkPages];
+  __shared__ uint32_t qs[16 * 24];
+  __shared__ Group grp;
+  if (tid == 0) grp = groups[gi];
+  __syncthreads();
+  const int nr = grp.n, g = grp.kv_head;
+  long long N = a.seq_lens[b];
+  N = N < 0 ? 0 : std::min<long long>(N, sh.max_len);
+  const long long kb = topk_budget(a, N);
+  if (N == 0 || kb >= N) return;
+  const int pages = (int)((N + kPage - 1) / kPage);
+  const int p0 = blockIdx.x * kChunkPages;
+  if (p0 >= pages) return;
+  const int np = pages - p0 < kChunkPages ? pages - p0 : kChunkPages;
+  {
+    const int32_t *pt = a.page_table + (long long)b * sh.max_pages + p0;
+    for (int o = tid; o < np; o += kT1) {
+      const int page = pt[o];
+      const bool ok = page >= 0 && page < sh.num_pages;
+      pt_s[o] = ok ? page : -1;
+      if (!ok) raise_error(a.err, SD_EBIT_PAGE);
     }
-    if (lane == 0) {
-      const float flo = (lo == 0u || lo == 0xFFFFFFFFu) ? -INFINITY : key_to_float(lo);
-      const float fhi = key_to_float(hi);
-      S.tlo[h] = flo;
-      S.thi[h] = fhi;
-      S.inv[h] = (flo > -INFINITY && fhi > flo) ? (float)kBins / (fhi - flo) : 0.0f;
+    for (int o = tid; o < 16 * 24; o += kT1) {
+      const int i = o / 24;
+      qs[o] = i < nr ? ws.qsplit[((long long)b * sh.H_ret + grp.row[i]) * 24 + o % 24] : 0u;
     }
   }
   __syncthreads();
 
-  // ---- 2. stream the chunk, keep the window ----------------------------------
-  auto classify = [&](int h, int i, float s) {
-    int cls;
-    if (s >= S.thi[h]) {
-      cls = kTopClass;
-      atomicAdd(&S.top_n[h], 1u);
-    } else if (s >= S.tlo[h]) {
-      cls = std::min(kBins - 1, std::max(0, __float2int_rz((s - S.tlo[h]) * S.inv[h])));
-      atomicAdd(&whist[h * kBins + cls], 1u);
-    } else {
-      return;
+  // per-warp ring: this warp reads pages warp, warp + 8, ... of the chunk
+  const uint32_t ring_base = (uint32_t)__cvta_generic_to_shared(&ring[warp][0][0]);
+  const uint16_t *icache = a.index_cache + (long long)g * (kPage * kIndexDim) + lane * 8;
+  const long long page_stride = (long long)sh.Hkv * (kPage * kIndexDim);
+  const uint32_t st_off = page_off(lane >> 1, lane & 1);
+  const int nq = np > warp ? (np - warp + kW1 - 1) / kW1 : 0;
+  auto issue = [&](int q) {
+    if (q < nq) {
+      const int page = pt_s[warp + q * kW1];
+      cp_async16(ring_base + (q % kRing) * kPageBytes + st_off, page >= 0 ? icache + page * page_stride : icache,
+                 page >= 0 ? 16 : 0);
     }
-    const uint32_t slot = atomicAdd(&S.list_n[h], 1u);
-    if (slot < (uint32_t)tp.list_cap)
-      list[(size_t)h * tp.list_cap + slot] = ((unsigned long long)__float_as_uint(s) << 32) | (uint32_t)i;
-    else
-      S.overflow = 1u;
+    cp_async_commit();
   };
-  for (int base = warp; base < ntiles; base += kW * kUnroll) {
-    uint32_t af[kUnroll][4];
-    bool ok[kUnroll];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int tile = base + u * kW;
-      ok[u] = false;
-      if (tile < ntiles && tile % st != 0) ok[u] = load_tile(tile, af[u]);
-    }
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      if (!ok[u]) continue;
-      const int tile = base + u * kW;
-      float sc[HB][2];
-      score_tile(af[u], sc);
-#pragma unroll
-      for (int hb = 0; hb < HB; ++hb) {
-        const int h = hb * 4 + tq;
-        if (h >= nr) continue;
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const int i = tile * kPage + gq + 8 * r;
-          if (i < cnt) classify(h, i, sc[hb][r]);
-        }
-      }
-    }
-  }
-  for (int o = tid; o < nr * ns * 16; o += kT) {     // sampled pages
-    const int h = o / (ns * 16), r = o % (ns * 16);
-    const int i = (r / 16) * st * kPage + (r % 16);
-    const float v = sample[h * (kSampleTiles * 16) + r];
-    if (i < cnt && v > -INFINITY) classify(h, i, v);
-  }
-  __syncthreads();
-  cluster.sync();                                    // B2: histograms and lists complete
+  for (int q = 0; q < kRing; ++q) issue(q);
 
-  // ---- 3. cluster reduction of the window histogram, cut bin ----------------
-  const int per = kBins / C;
-  const int d0 = rank * per;
-  for (int base = 0; base < nr * kBins; base += kT) {
-    const int it = base + tid;
-    const bool okk = it < nr * kBins;
-    const int c = it % C, rest = it / C;
-    const int h = rest / per, bin = d0 + rest % per;
-    uint32_t v = okk ? *cluster.map_shared_rank(&whist[h * kBins + bin], c) : 0u;
-    for (int o = 1; o < C; o <<= 1) v += __shfl_xor_sync(kFull, v, o);
-    if (okk && c == 0) wred[h * kBins + bin] = v;
-  }
-  __syncthreads();
-  for (int h = warp; h < nr; h += kW) {
-    uint32_t sc = 0u;
-    for (int j = lane; j < per; j += 32) sc += wred[h * kBins + d0 + j];
+  BFrag bf[HB];
+  float tlo[HB], thi[HB], inv[HB];
+  long long row_of[HB];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sc += __shfl_xor_sync(kFull, sc, o);
-    if (lane == 0) S.slice_cnt[h] = sc;
+  for (int hb = 0; hb < HB; ++hb) {
+    bf[hb] = load_bfrag(qs, hb, gq, tq);
+    const int h = hb * 4 + tq;
+    row_of[hb] = h < nr ? (long long)b * sh.H_ret + grp.row[h] : 0;
+    const float4 w = h < nr ? ws.win[row_of[hb]] : make_float4(INFINITY, INFINITY, 0.f, 0.f);
+    tlo[hb] = w.x;
+    thi[hb] = w.y;
+    inv[hb] = w.z;
   }
-  __syncthreads();
-  cluster.sync();                                    // B3: owner slices reduced
-  if (warp == 0) {
-    uint32_t f = lane < C ? *cluster.map_shared_rank(&S.overflow, lane) : 0u;
-    f = __reduce_or_sync(kFull, f);
-    if (lane == 0 && f) S.fail = 1;
-  }
-  for (int h = warp; h < nr; h += kW) {
-    const uint32_t topc = lane < C ? *cluster.map_shared_rank(&S.top_n[h], lane) : 0u;
-    const long long top_total = __reduce_add_sync(kFull, topc);
-    const long long need = kb - top_total;
-    const uint32_t lc = lane < C ? *cluster.map_shared_rank(&S.slice_cnt[h], lane) : 0u;
-    long long suf = lc;
+  const unsigned head_lanes = 0x11111111u << tq;
+  const unsigned lt = (1u << lane) - 1u;
+  uint32_t staged[HB];
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const long long y = __shfl_down_sync(kFull, suf, o);
-      if (lane + o < 32) suf += y;
-    }
-    const bool reach = lane < C && lc > 0u && need > 0 && suf >= need;
-    const unsigned bal = __ballot_sync(kFull, reach);
-    bool bad = need <= 0 || bal == 0u;
-    int cut = -1;
-    long long above = 0, ncut = 0;
-    if (!bad) {
-      const int cs = 31 - __clz(bal);
-      above = __shfl_sync(kFull, suf, cs) - (long long)__shfl_sync(kFull, lc, cs);
-      for (int top = per; top > 0 && cut < 0; top -= 32) {
-        const int j = top - 32 + lane;
-        const bool in = j >= 0 && j < per;
-        const uint32_t dc = in ? *cluster.map_shared_rank(&wred[h * kBins + cs * per + j], cs) : 0u;
-        long long sk = dc;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const long long y = __shfl_down_sync(kFull, sk, o);
-          if (lane + o < 32) sk += y;
-        }
-        const unsigned b2 = __ballot_sync(kFull, in && dc > 0u && above + sk >= need);
-        if (b2) {
-          const int l = 31 - __clz(b2);
-          cut = cs * per + top - 32 + l;
-          ncut = __shfl_sync(kFull, (long long)dc, l);
-          above += __shfl_sync(kFull, sk, l) - ncut;
-        } else {
-          above += __shfl_sync(kFull, sk, 0);
-        }
+  for (int hb = 0; hb < HB; ++hb) staged[hb] = 0u;
+  // move this warp's staged entries of head block hb to the heads' buffers:
+  // lane tq reserves the space for head 4hb + tq, the head's 8 lanes copy
+  auto flush = [&](int hb) {
+    const int h = hb * 4 + tq;
+    uint32_t base = 0u;
+    if (gq == 0 && h < nr && staged[hb] > 0u) base = atomicAdd(&ws.bcount[row_of[hb]], staged[hb]);
+    base = __shfl_sync(kFull, base, tq);
+    if (h < nr) {
+      unsigned long long *dst = ws.buf + row_of[hb] * ws.cap;
+      for (uint32_t e = gq; e < staged[hb]; e += 8) {
+        const uint32_t at = base + e;
+        if (at < (uint32_t)ws.cap) dst[at] = stage[warp][h][e];
       }
-      bad = cut < 0 || ncut > kCap;
     }
-    if (lane == 0) {
-      S.cut[h] = cut;
-      S.need_c[h] = need - above;
-      if (bad) S.fail = 1;
+    __syncwarp();
+    staged[hb] = 0u;
+  };
+  const uint32_t ld = ring_base + page_off((lane & 7) + ((lane >> 3) & 1) * 8, lane >> 4);
+  for (int q = 0; q < nq; ++q) {
+    cp_async_wait<kRing - 1>();
+    __syncwarp();
+    uint32_t af[4];
+    ldmatrix_x4(af, ld + (q % kRing) * kPageBytes);
+    __syncwarp();
+    const int pl = warp + q * kW1;                   // page within the chunk
+    const bool ok = pt_s[pl] >= 0;
+    issue(q + kRing);
+    float sc[HB][2];
+    score_frag<HB>(af, bf, sc);
+    const long long pos0 = (long long)(p0 + pl) * kPage + gq;
+#pragma unroll
+    for (int hb = 0; hb < HB; ++hb) {
+      const int h = hb * 4 + tq;
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const long long pos = pos0 + 8 * r;
+        const float s = sc[hb][r];
+        const bool in = ok && h < nr && pos < N && s >= tlo[hb];
+        const unsigned m = __ballot_sync(kFull, in) & head_lanes;
+        if (in) {
+          const int cls = window_bin(s, tlo[hb], thi[hb], inv[hb]);
+          atomicAdd(&ws.hist[row_of[hb] * (kBins + 1) + cls], 1u);
+          stage[warp][h][staged[hb] + __popc(m & lt)] = ((unsigned long long)order_key(s) << 32) | (uint32_t)pos;
+        }
+        staged[hb] += __popc(m);
+      }
+      // all lanes of a head share staged[hb]; flush when another page could overflow
+      const bool full = __any_sync(kFull, staged[hb] > (uint32_t)(SE - 16));
+      if (full) flush(hb);
     }
   }
-  __syncthreads();
-  if (S.fail) {                                      // uniform across the cluster
-    if (rank == 0 && tid == 0) tp.fail[item] = 1u;
-    cluster.sync();                                  // peers may still read this CTA's memory
+#pragma unroll
+  for (int hb = 0; hb < HB; ++hb) flush(hb);
+  cp_async_wait<0>();
+}
+
+// ------------------------------------------------------------------- K2
+constexpr int kT2 = 512;
+
+__global__ void __launch_bounds__(kT2)
+topk_resolve_kernel(const SelectArgs a, const Shape sh, const TopkWs ws) {
+  extern __shared__ uint32_t bitmap[];               // [max_len / 32]
+  __shared__ unsigned long long cand[kCap];
+  __shared__ uint32_t n_cand;
+  __shared__ int cut_s, fail_s;
+  __shared__ long long need_s;
+  __shared__ uint32_t wtot[kT2 / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int b = blockIdx.y, hr = blockIdx.x;
+  const long long row = (long long)b * sh.H_ret + hr;
+  int32_t *out = a.sel_idx + row * a.sel_stride;
+  long long N = a.seq_lens[b];
+  N = N < 0 ? 0 : std::min<long long>(N, sh.max_len);
+  const long long kb = topk_budget(a, N);
+  if (N == 0 || kb >= N) {
+    for (long long t = tid; t < N; t += kT2) {
+      if (t < a.sel_stride) out[t] = (int32_t)t;
+      else raise_error(a.err, SD_EBIT_SEL);
+    }
+    if (tid == 0) a.sel_count[row] = (int32_t)std::min(N, a.sel_stride);
     return;
   }
-  if (rank == 0 && tid == 0) tp.fail[item] = 0u;
-
-  // ---- 4. candidates of the cut bin to the owner; local counts above it -----
-  auto class_of = [&](int h, float s) -> int {
-    if (s >= S.thi[h]) return kTopClass;
-    return std::min(kBins - 1, std::max(0, __float2int_rz((s - S.tlo[h]) * S.inv[h])));
-  };
-  for (int h = 0; h < nr; ++h) {
-    const int n = (int)std::min<uint32_t>(S.list_n[h], (uint32_t)tp.list_cap);
-    const int cut = S.cut[h];
-    const int owner = h % C, slot = h / C;
-    uint32_t above = 0u;
-    for (int e = tid; e < n; e += kT) {
-      const unsigned long long ent = list[(size_t)h * tp.list_cap + e];
-      const float s = __uint_as_float((uint32_t)(ent >> 32));
-      const uint32_t i = (uint32_t)ent;
-      const int cls = class_of(h, s);
-      if (cls > cut) {
-        ++above;
-      } else if (cls == cut) {
-        uint32_t *cn = cluster.map_shared_rank(&S.cand_n[slot], owner);
-        const uint32_t idx = atomicAdd(cn, 1u);
-        if (idx < (uint32_t)kCap) {
-          unsigned long long *dst = cluster.map_shared_rank(cand + (size_t)slot * kCap + idx, owner);
-          *dst = sort_key(s, (uint32_t)(t0 + i));
+  const uint32_t *hist = ws.hist + row * (kBins + 1);
+  const float4 w = ws.win[row];
+  // cut bin: warp 0 scans the histogram from the top, 32 bins at a time
+  if (warp == 0) {
+    const long long top = hist[kBins];
+    const long long need = kb - top;
+    long long acc = 0;
+    int cut = -1;
+    long long ncut = 0;
+    if (need > 0) {
+      for (int hi = kBins; hi > 0 && cut < 0; hi -= 32) {
+        const int bin = hi - 32 + lane;
+        const uint32_t c = hist[bin];
+        long long suf = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const long long y = __shfl_down_sync(kFull, suf, o);
+          if (lane + o < 32) suf += y;
+        }
+        const unsigned bal = __ballot_sync(kFull, c > 0u && acc + suf >= need);
+        if (bal) {
+          const int l = 31 - __clz(bal);
+          cut = hi - 32 + l;
+          ncut = __shfl_sync(kFull, (long long)c, l);
+          acc += __shfl_sync(kFull, suf, l) - ncut;
+        } else {
+          acc += __shfl_sync(kFull, suf, 0);
         }
       }
     }
-    above = __reduce_add_sync(kFull, above);
-    if (lane == 0 && above) atomicAdd(&S.above_local[h], above);
-  }
-  __syncthreads();
-  cluster.sync();                                    // B4: candidates delivered
-
-  // ---- 5. owners rank their candidates exactly --------------------------------
-  for (int slot = 0; slot < tp.own_slots; ++slot) {
-    const int h = rank + slot * C;
-    if (h >= nr) break;
-    const int n = (int)std::min<uint32_t>(S.cand_n[slot], (uint32_t)kCap);
-    const long long need_c = S.need_c[h];
-    const unsigned long long *cs = cand + (size_t)slot * kCap;
-    for (int e = tid; e < n; e += kT) {
-      const unsigned long long me = cs[e];
-      int rk = 0;
-      for (int j = 0; j < n; ++j) rk += cs[j] < me;
-      if (rk == need_c - 1) S.tau_sk[slot] = me;
-      if (rk < need_c) {
-        const long long pos = (long long)(me & 0xFFFFFFFFull);
-        const int c = (int)std::min<long long>(C - 1, pos / per_cta);
-        atomicAdd(&occ[slot * kMaxCluster + c], 1u);
-      }
+    if (lane == 0) {
+      const bool bad = need <= 0 || cut < 0 || ncut > kCap || ws.bcount[row] > (uint32_t)ws.cap;
+      fail_s = bad;
+      cut_s = cut;
+      need_s = need - acc;                           // tokens to take from the cut bin
+      n_cand = 0u;
     }
   }
   __syncthreads();
-  cluster.sync();                                    // B5: thresholds published
-
-  // ---- 6. offsets, ordered write ---------------------------------------------
-  unsigned long long tau[kMaxGroup];
-  long long off[kMaxGroup];
-  for (int h = 0; h < nr; ++h) {
-    const int owner = h % C, slot = h / C;
-    tau[h] = *cluster.map_shared_rank(&S.tau_sk[slot], owner);
-    const long long ab = lane < C ? (long long)*cluster.map_shared_rank(&S.above_local[h], lane) : 0LL;
-    const long long oc = lane < C ? (long long)*cluster.map_shared_rank(&occ[slot * kMaxCluster + lane], owner) : 0LL;
-    const long long mine = ab + oc;
-    const long long before = __reduce_add_sync(kFull, (unsigned)(lane < rank ? mine : 0LL));
-    const long long total = __reduce_add_sync(kFull, (unsigned)mine);
-    off[h] = before;
-    if (rank == 0 && tid == 0) {
-      if (total > a.sel_stride) raise_error(a.err, SD_EBIT_SEL);
-      *count_slot(h) = (int32_t)std::min(total, a.sel_stride);
-    }
+  if (fail_s) {
+    if (tid == 0) atomicOr(&ws.fail[ws.rowitem[row]], 1u);
+    return;
   }
-  cluster_arrive();                                  // no more reads of peer memory
-  for (int h = 0; h < nr; ++h) {
-    const int n = (int)std::min<uint32_t>(S.list_n[h], (uint32_t)tp.list_cap);
-    const int cut = S.cut[h];
-    for (int e = tid; e < n; e += kT) {
-      const unsigned long long ent = list[(size_t)h * tp.list_cap + e];
-      const float s = __uint_as_float((uint32_t)(ent >> 32));
-      const uint32_t i = (uint32_t)ent;
-      const int cls = class_of(h, s);
-      const bool sel = cls > cut || (cls == cut && sort_key(s, (uint32_t)(t0 + i)) <= tau[h]);
-      if (sel) atomicOr(&bitmap[h * words + (i >> 5)], 1u << (i & 31));
+  const int words = (int)((N + 31) / 32);
+  for (int o = tid; o < words; o += kT2) bitmap[o] = 0u;
+  __syncthreads();
+  const int cut = cut_s;
+  const unsigned long long *buf = ws.buf + row * ws.cap;
+  const int n = (int)ws.bcount[row];
+  for (int e = tid; e < n; e += kT2) {
+    const unsigned long long ent = buf[e];
+    const uint32_t key = (uint32_t)(ent >> 32), pos = (uint32_t)ent;
+    const int cls = window_bin(key_to_float(key), w.x, w.y, w.z);
+    if (cls > cut) {
+      atomicOr(&bitmap[pos >> 5], 1u << (pos & 31));
+    } else if (cls == cut) {
+      const uint32_t at = atomicAdd(&n_cand, 1u);
+      if (at < (uint32_t)kCap) cand[at] = ((unsigned long long)(~key) << 32) | pos;   // ascending = better first
     }
   }
   __syncthreads();
-  const int nwords = (cnt + 31) / 32;
-  const int wpt = (nwords + kT - 1) / kT;            // bitmap words per thread
-  for (int h = 0; h < nr; ++h) {
-    int32_t *row = sel_row(h);
-    const int w0 = tid * wpt;
-    uint32_t c = 0;
-    for (int w = w0; w < std::min(nwords, w0 + wpt); ++w) c += __popc(bitmap[h * words + w]);
-    uint32_t incl = c;
+  // rank the cut bin exactly: the need_c best by (score desc, position asc)
+  const int nc = (int)std::min<uint32_t>(n_cand, (uint32_t)kCap);
+  const long long need_c = need_s;
+  for (int e = tid; e < nc; e += kT2) {
+    const unsigned long long me = cand[e];
+    int rk = 0;
+    for (int j = 0; j < nc; ++j) rk += cand[j] < me;
+    if (rk < need_c) {
+      const uint32_t pos = (uint32_t)me;
+      atomicOr(&bitmap[pos >> 5], 1u << (pos & 31));
+    }
+  }
+  __syncthreads();
+  // ordered write: contiguous word ranges per thread, block-wide prefix
+  const int wpt = (words + kT2 - 1) / kT2;
+  const int w0 = tid * wpt, w1 = std::min(words, w0 + wpt);
+  uint32_t c = 0;
+  for (int x = w0; x < w1; ++x) c += __popc(bitmap[x]);
+  uint32_t incl = c;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(kFull, incl, o);
-      if (lane >= o) incl += y;
-    }
-    if (lane == 31) S.wtot[warp] = incl;
-    __syncthreads();
-    uint32_t wbase = 0;
-    for (int w = 0; w < warp; ++w) wbase += S.wtot[w];
-    long long o = off[h] + wbase + incl - c;
-    for (int w = w0; w < std::min(nwords, w0 + wpt); ++w) {
-      uint32_t bits = bitmap[h * words + w];
-      while (bits) {
-        const int bit = __ffs(bits) - 1;
-        bits &= bits - 1;
-        if (o < a.sel_stride) row[o] = (int32_t)(t0 + w * 32 + bit);
-        else raise_error(a.err, SD_EBIT_SEL);
-        ++o;
-      }
-    }
-    __syncthreads();
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(kFull, incl, o);
+    if (lane >= o) incl += y;
   }
-  cluster_wait();
+  if (lane == 31) wtot[warp] = incl;
+  __syncthreads();
+  uint32_t base = 0, total = 0;
+  for (int x = 0; x < kT2 / 32; ++x) {
+    if (x < warp) base += wtot[x];
+    total += wtot[x];
+  }
+  long long o = base + incl - c;
+  for (int x = w0; x < w1; ++x) {
+    uint32_t bits = bitmap[x];
+    while (bits) {
+      const int bit = __ffs(bits) - 1;
+      bits &= bits - 1;
+      if (o < a.sel_stride) out[o] = x * 32 + bit;
+      else raise_error(a.err, SD_EBIT_SEL);
+      ++o;
+    }
+  }
+  if (tid == 0) {
+    if ((long long)total > a.sel_stride) raise_error(a.err, SD_EBIT_SEL);
+    a.sel_count[row] = (int32_t)std::min<long long>(total, a.sel_stride);
+  }
 }
 
-int pow2_floor(int x) {
-  int p = 1;
-  while (p * 2 <= x) p <<= 1;
+// ------------------------------------------------------------------- host
+struct TopkPlan {
+  int cap;
+  size_t bitmap_bytes;
+  bool ok;
+};
+
+TopkPlan topk_plan(const Shape &sh, const Tables &tb) {
+  TopkPlan p{};
+  p.cap = (int)std::min<long long>(sh.max_len, std::max<long long>(4096, sh.max_len / 8));
+  p.bitmap_bytes = (size_t)((sh.max_len + 31) / 32) * 4;
+  p.ok = tb.max_ret <= 16 && p.bitmap_bytes <= 160 * 1024 && sh.max_len < (1LL << 31);
   return p;
 }
 
-template <int GR>
-struct TkCache {
-  std::mutex mu;
-  std::map<int, size_t> attr;
-  std::map<std::tuple<int, size_t, int>, int> clusters;
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+struct TopkLayout {
+  size_t qsplit, win, hist, bcount, rowitem, buf, total;
 };
 
-template <int GR>
-TkCache<GR> &tk_cache() {
-  static TkCache<GR> c;
-  return c;
+TopkLayout topk_layout(const Shape &sh, int batch, int cap) {
+  TopkLayout L{};
+  const size_t rows = (size_t)batch * std::max(1, sh.H_ret);
+  size_t o = 0;
+  L.qsplit = o;  o = align256(o + rows * 24 * 4);
+  L.win = o;     o = align256(o + rows * 16);
+  L.hist = o;    o = align256(o + rows * (kBins + 1) * 4);
+  L.bcount = o;  o = align256(o + rows * 4);
+  L.rowitem = o; o = align256(o + rows * 4);
+  L.buf = o;     o = align256(o + rows * (size_t)cap * 8);
+  L.total = o;
+  return L;
 }
 
-template <int GR>
-cudaError_t tk_attrs(int dev, size_t bytes) {
-  auto &c = tk_cache<GR>();
-  std::lock_guard<std::mutex> lk(c.mu);
-  auto it = c.attr.find(dev);
-  if (it != c.attr.end() && it->second >= bytes) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(topk_kernel<GR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(topk_kernel<GR>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-  if (e == cudaSuccess) c.attr[dev] = bytes;
+// dynamic shared memory attributes, set once per kernel and device
+template <typename K>
+cudaError_t set_smem_once(K kern, size_t bytes) {
+  static std::mutex mu;
+  static std::map<std::pair<const void *, int>, size_t> done;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lk(mu);
+  const auto key = std::make_pair((const void *)kern, dev);
+  auto it = done.find(key);
+  if (it != done.end() && it->second >= bytes) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) done[key] = bytes;
   return e;
 }
 
 template <int GR>
-cudaLaunchConfig_t tk_config(int C, int items, size_t bytes, cudaStream_t st, cudaLaunchAttribute *attr) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(C, items, 1);
-  cfg.blockDim = dim3(kT, 1, 1);
-  cfg.dynamicSmemBytes = bytes;
-  cfg.stream = st;
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = C;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cfg;
-}
-
-template <int GR>
-int tk_fits(int dev, int C, size_t bytes) {
-  if (tk_attrs<GR>(dev, bytes) != cudaSuccess) {
-    cudaGetLastError();
-    return 0;
-  }
-  auto &c = tk_cache<GR>();
-  const auto key = std::make_tuple(dev, bytes, C);
-  {
-    std::lock_guard<std::mutex> lk(c.mu);
-    auto it = c.clusters.find(key);
-    if (it != c.clusters.end()) return it->second;
-  }
-  cudaLaunchAttribute attr[1];
-  cudaLaunchConfig_t cfg = tk_config<GR>(C, 1, bytes, 0, attr);
-  int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, topk_kernel<GR>, &cfg) != cudaSuccess) {
-    cudaGetLastError();
-    n = 0;
-  }
-  std::lock_guard<std::mutex> lk(c.mu);
-  c.clusters[key] = n;
-  return n;
-}
-
-struct TkPlan {
-  int C, tc_cap, list_cap, own_slots;
-  size_t bytes;
-};
-
-TkPlan tk_plan(const Shape &sh, int GR) {
-  TkPlan p{};
-  p.C = std::min(kMaxCluster, pow2_floor(std::max(1, sh.max_pages)));
-  p.tc_cap = (int)(((sh.max_len + p.C - 1) / p.C + kPage - 1) / kPage * kPage);
-  p.tc_cap = (p.tc_cap + 31) / 32 * 32;
-  p.list_cap = std::max(256, (p.tc_cap / 8 + 31) / 32 * 32);
-  p.own_slots = (GR + p.C - 1) / p.C;
-  p.bytes = tk_layout(GR, p.tc_cap, p.list_cap, p.own_slots).total;
-  return p;
-}
-
-template <int GR>
-cudaError_t tk_launch(const SelectArgs &a, const Shape &sh, const Tables &tb, uint32_t *fail, int dev,
-                      cudaStream_t st, bool *used) {
-  *used = false;
-  const TkPlan p = tk_plan(sh, GR);
-  if (p.bytes + sizeof(TkShared) > 227 * 1024) return cudaSuccess;
-  if (tk_fits<GR>(dev, p.C, p.bytes) == 0) return cudaSuccess;
-  cudaError_t e = tk_attrs<GR>(dev, p.bytes);
+cudaError_t topk_launch(const SelectArgs &a, const Shape &sh, const Tables &tb, const TopkWs &ws,
+                        size_t bitmap_bytes, cudaStream_t st) {
+  const int items = a.batch * tb.n_ret;
+  const size_t smem0 = (size_t)GR * sample_pages(GR) * 16 * 4 + (size_t)GR * kSampleBins * 4;
+  const size_t smem1 = (size_t)kW1 * kRing * kPageBytes + (size_t)kW1 * GR * stage_entries(GR) * 8;
+  cudaError_t e = set_smem_once(topk_window_kernel<GR>, smem0);
+  if (e == cudaSuccess) e = set_smem_once(topk_stream_kernel<GR>, smem1);
+  if (e == cudaSuccess) e = set_smem_once(topk_resolve_kernel, bitmap_bytes);
   if (e != cudaSuccess) return e;
-  TopkParams tp{p.tc_cap, p.list_cap, p.own_slots, fail};
-  cudaLaunchAttribute attr[1];
-  cudaLaunchConfig_t cfg = tk_config<GR>(p.C, a.batch * tb.n_ret, p.bytes, st, attr);
-  e = cudaLaunchKernelEx(&cfg, topk_kernel<GR>, a, sh, tb.ret, tb.n_ret, tp);
-  if (e == cudaSuccess) *used = true;
-  return e;
+  topk_window_kernel<GR><<<items, kT0, smem0, st>>>(a, sh, tb.ret, tb.n_ret, ws);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int chunks = (int)((sh.max_pages + kChunkPages - 1) / kChunkPages);
+  topk_stream_kernel<GR><<<dim3(chunks, items), kT1, smem1, st>>>(a, sh, tb.ret, tb.n_ret, ws);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  topk_resolve_kernel<<<dim3(sh.H_ret, a.batch), kT2, bitmap_bytes, st>>>(a, sh, ws);
+  return cudaGetLastError();
 }
 
 }  // namespace
 
+size_t topk_workspace_bytes(const Shape &sh, const Tables &tb, int batch) {
+  const TopkPlan p = topk_plan(sh, tb);
+  if (!p.ok) return 0;
+  return topk_layout(sh, batch, p.cap).total;
+}
+
 cudaError_t launch_select_topk_stream(const SelectArgs &a, const Shape &sh, const Tables &tb, uint32_t *fail,
-                                      cudaStream_t st, bool *used) {
-  int dev = 0;
-  cudaGetDevice(&dev);
+                                      void *ws_base, cudaStream_t st, bool *used) {
+  *used = false;
+  const TopkPlan p = topk_plan(sh, tb);
+  if (!p.ok || ws_base == nullptr) return cudaSuccess;
+  const TopkLayout L = topk_layout(sh, a.batch, p.cap);
+  char *base = static_cast<char *>(ws_base);
+  TopkWs ws{};
+  ws.qsplit = reinterpret_cast<uint32_t *>(base + L.qsplit);
+  ws.win = reinterpret_cast<float4 *>(base + L.win);
+  ws.hist = reinterpret_cast<uint32_t *>(base + L.hist);
+  ws.bcount = reinterpret_cast<uint32_t *>(base + L.bcount);
+  ws.rowitem = reinterpret_cast<int *>(base + L.rowitem);
+  ws.buf = reinterpret_cast<unsigned long long *>(base + L.buf);
+  ws.fail = fail;
+  ws.cap = p.cap;
   int gr = 1;
   while (gr < tb.max_ret) gr <<= 1;
+  cudaError_t e;
   switch (gr) {
-    case 1: return tk_launch<1>(a, sh, tb, fail, dev, st, used);
-    case 2: return tk_launch<2>(a, sh, tb, fail, dev, st, used);
-    case 4: return tk_launch<4>(a, sh, tb, fail, dev, st, used);
-    case 8: return tk_launch<8>(a, sh, tb, fail, dev, st, used);
-    default: return tk_launch<16>(a, sh, tb, fail, dev, st, used);
+    case 1: e = topk_launch<1>(a, sh, tb, ws, p.bitmap_bytes, st); break;
+    case 2: e = topk_launch<2>(a, sh, tb, ws, p.bitmap_bytes, st); break;
+    case 4: e = topk_launch<4>(a, sh, tb, ws, p.bitmap_bytes, st); break;
+    case 8: e = topk_launch<8>(a, sh, tb, ws, p.bitmap_bytes, st); break;
+    default: e = topk_launch<16>(a, sh, tb, ws, p.bitmap_bytes, st); break;
   }
+  if (e == cudaSuccess) *used = true;
+  return e;
 }
 
 }  // namespace sd

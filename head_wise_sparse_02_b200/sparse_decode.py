@@ -17,7 +17,8 @@ from typing import Optional, Sequence
 
 import torch
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libsparsedecode.so")
+LIB_PATH = os.environ.get("SPARSE_DECODE_LIB") or os.path.join(
+    os.path.dirname(os.path.abspath(__file__)), "lib", "libsparsedecode.so")
 
 SD_OK, SD_ERR_INVALID_ARG, SD_ERR_UNSUPPORTED, SD_ERR_WORKSPACE, SD_ERR_CUDA, SD_ERR_TIMEOUT, \
     SD_ERR_DEVICE_DATA = range(7)
