@@ -47,7 +47,7 @@ sd_status cuda_fail(sd_ctx *ctx, cudaError_t e, const char *what) {
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct WsLayout {
-  size_t scores_off, flags_off, scores_bytes, topk_off, topk_bytes, part_off, tickets_off, total;
+  size_t scores_off, flags_off, scores_bytes, topk_off, topk_bytes, att_off, total;
 };
 
 WsLayout layout(const sd_ctx *ctx, int batch) {
@@ -58,11 +58,8 @@ WsLayout layout(const sd_ctx *ctx, int batch) {
   w.flags_off = w.scores_off + foff;
   w.topk_off = w.scores_off + w.scores_bytes;
   w.topk_bytes = ctx->cfg.mode == SD_TOP_K ? align256(sd::topk_workspace_bytes(ctx->sh, ctx->tb, batch)) : 0;
-  w.part_off = w.topk_off + w.topk_bytes;
-  size_t toff = 0;
-  const size_t att = sd::attend_workspace_bytes(ctx->sh, ctx->tb, batch, &toff);
-  w.tickets_off = w.part_off + toff;
-  w.total = align256(w.part_off + att);
+  w.att_off = w.topk_off + w.topk_bytes;
+  w.total = align256(w.att_off + sd::attend_workspace_bytes(ctx->sh, ctx->tb, batch));
   return w;
 }
 
@@ -105,7 +102,9 @@ sd_status sparse_decode_init(const sd_config *cfg, const void *proj, sd_ctx **ou
   if (c.head_dim != 64 && c.head_dim != 128) return SD_ERR_UNSUPPORTED;
   if (c.index_dim != sd::kIndexDim || c.page_size != sd::kPage) return SD_ERR_UNSUPPORTED;
   if (c.num_pages <= 0 || c.max_batch <= 0 || c.max_pages_per_seq <= 0) return SD_ERR_INVALID_ARG;
-  if ((long long)c.max_pages_per_seq * sd::kPage > (1LL << 30)) return SD_ERR_UNSUPPORTED;
+  if ((long long)c.max_pages_per_seq * sd::kPage > (1LL << 25)) return SD_ERR_UNSUPPORTED;
+  // cache rows are addressed with 32-bit row numbers inside the kernels
+  if ((long long)c.num_pages * c.num_kv_heads * sd::kPage >= 0xFFFFFFFFLL) return SD_ERR_UNSUPPORTED;
   if (c.window < 0 || c.num_sinks < 0) return SD_ERR_INVALID_ARG;
   if (c.mode != SD_TOP_P && c.mode != SD_TOP_K) return SD_ERR_INVALID_ARG;
   if (c.mode == SD_TOP_P && !(c.top_p > 0.0f && c.top_p <= 1.0f)) return SD_ERR_INVALID_ARG;
@@ -260,8 +259,7 @@ sd_status sparse_decode_attend(sd_ctx *ctx, const void *q, const void *k_cache, 
   a.attn_scale = ctx->attn_scale;
   a.window = ctx->cfg.window;
   a.num_sinks = ctx->cfg.num_sinks;
-  a.partials = reinterpret_cast<float *>(static_cast<char *>(workspace) + w.part_off);
-  a.tickets = reinterpret_cast<unsigned *>(static_cast<char *>(workspace) + w.tickets_off);
+  a.ws = static_cast<char *>(workspace) + w.att_off;
   a.err = ctx->err_d;
   a.batch = batch;
   cudaError_t e = sd::launch_attend(a, ctx->sh, ctx->tb, static_cast<cudaStream_t>(stream));

@@ -117,13 +117,12 @@ struct AttendArgs {
   float *out;
   float attn_scale;
   int window, num_sinks;
-  float *partials;
-  unsigned *tickets;
+  void *ws;                       // attend's part of the workspace (partials, union lists, tickets)
   unsigned *err;
   int batch;
 };
 
-size_t attend_workspace_bytes(const Shape &sh, const Tables &tb, int batch, size_t *tickets_off);
+size_t attend_workspace_bytes(const Shape &sh, const Tables &tb, int batch);
 cudaError_t launch_attend(const AttendArgs &a, const Shape &sh, const Tables &tb, cudaStream_t st);
 
 }  // namespace sd

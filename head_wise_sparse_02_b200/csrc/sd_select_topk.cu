@@ -12,21 +12,22 @@
 //              terms) and scores a strided sample of <= 256 pages; from the
 //              sample it sets, per head, a conservative score window
 //              [t_lo, t_hi): t_lo a sample quantile safely below the k-th
-//              score, t_hi the sample maximum.  Zeroes the head's histogram
-//              and buffer counter.
+//              score, t_hi the sample maximum.  Zeroes the head's buffer
+//              counter.
 //   K1 stream  many CTAs, each 512 pages of one (sequence, KV group): pages
 //              arrive through a per-warp cp.async ring (16 bytes per lane,
 //              XOR-swizzled rows), ldmatrix + mma.m16n8k16 score all heads of
 //              the group at once (A = the 16 x 16 bf16 index page, B = the q~
-//              terms), and every score at or above t_lo goes to a global
-//              512-bin histogram of the window (or a count of scores at or
-//              above t_hi) and, with its position, to a per-head buffer
-//              (staged per warp in shared memory, flushed in batches).
-//   K2 resolve one CTA per (sequence, retrieval head): scans the histogram
-//              from the top for the bin holding the k-th score, ranks the
-//              tokens of that bin exactly by (score desc, position asc),
-//              marks the selected positions in a bitmap of the context and
-//              writes them in ascending order.
+//              terms), and every score at or above t_lo goes, with its
+//              position, to a lane-private staging area in shared memory and
+//              from there, in batches, to a per-head buffer.  Most scores
+//              fail the single compare and cost nothing more.
+//   K2 resolve one CTA per (sequence, retrieval head): histograms the
+//              buffered scores over 512 bins of [t_lo, t_hi) (plus one bin for
+//              scores >= t_hi), scans from the top for the bin holding the
+//              k-th score, ranks the tokens of that bin exactly by (score
+//              desc, position asc), marks the selected positions in a bitmap
+//              of the context and writes them in ascending order.
 // If the window misses (buffer overflow, k-th score outside the window, too
 // many tokens in the cut bin), K2 flags the work item and the exact general
 // kernel recomputes it.
@@ -46,9 +47,9 @@ constexpr int kBins = 512;            // window histogram bins (+1 slot: scores 
 __host__ __device__ constexpr int sample_pages(int GR) { return GR <= 4 ? 256 : (GR == 8 ? 192 : 96); }
 constexpr int kSampleBins = 256;
 constexpr int kChunkPages = 512;      // K1: pages per CTA
-constexpr int kRing = 8;              // K1: pages in flight per warp
-// K1: staged buffer entries per (warp, head)
-__host__ __device__ constexpr int stage_entries(int GR) { return GR <= 4 ? 64 : 32; }
+constexpr int kRing = 12;             // K1: pages in flight per warp (even)
+// K1: staged buffer entries per (lane, head block); an iteration adds <= 4
+__host__ __device__ constexpr int stage_lane(int GR) { return GR <= 4 ? 10 : (GR == 8 ? 8 : 5); }
 constexpr int kCap = 2048;            // K2: cut-bin tokens ranked exactly
 constexpr int kPageBytes = kPage * kIndexDim * 2;   // 512 B: one page of one KV head
 constexpr unsigned kFull = 0xFFFFFFFFu;
@@ -90,7 +91,6 @@ __device__ __forceinline__ int window_bin(float s, float tlo, float thi, float i
 struct TopkWs {
   uint32_t *qsplit;                   // [rows][24]: bf16 pairs of the q~ terms hi, mid, lo
   float4 *win;                        // [rows]: t_lo, t_hi, 1 / bin width, unused
-  uint32_t *hist;                     // [rows][kBins + 1]
   uint32_t *bcount;                   // [rows] buffer entries written
   int *rowitem;                       // [rows] work item of the row
   unsigned long long *buf;            // [rows][cap]: order key << 32 | position
@@ -149,6 +149,8 @@ topk_window_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__
   __shared__ Group grp;
   __shared__ uint32_t qs[16 * 24];
   __shared__ uint32_t smax[GR], smin[GR];
+  __shared__ float hlo[GR], hinv[GR];
+  __shared__ int spage[SP];
   extern __shared__ __align__(16) unsigned char dyn0[];
   float (*sample)[SP * 16] = reinterpret_cast<float (*)[SP * 16]>(dyn0);
   uint32_t (*shist)[kSampleBins] = reinterpret_cast<uint32_t (*)[kSampleBins]>(dyn0 + (size_t)GR * SP * 16 * 4);
@@ -159,10 +161,6 @@ topk_window_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__
   N = N < 0 ? 0 : std::min<long long>(N, sh.max_len);
   const long long kb = topk_budget(a, N);
   if (tid == 0) ws.fail[item] = 0u;
-  for (int o = tid; o < nr * (kBins + 1); o += kT0) {
-    const int i = o / (kBins + 1);
-    ws.hist[((long long)b * sh.H_ret + grp.row[i]) * (kBins + 1) + o % (kBins + 1)] = 0u;
-  }
   if (tid < nr) {
     ws.bcount[(long long)b * sh.H_ret + grp.row[tid]] = 0u;
     ws.rowitem[(long long)b * sh.H_ret + grp.row[tid]] = item;
@@ -217,15 +215,22 @@ topk_window_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__
   for (int o = tid; o < nr * 24; o += kT0)           // publish the q~ terms for K1
     ws.qsplit[((long long)b * sh.H_ret + grp.row[o / 24]) * 24 + o % 24] = qs[o];
 
-  // sample: pages j * st, j < ns
+  // sample: pages j * st, j < ns; their page ids first, all at once
   const int pages = (int)((N + kPage - 1) / kPage);
   int st = 1;
   while ((long long)st * SP < pages) st <<= 1;
   const int ns = (pages + st - 1) / st;
+  const int32_t *pt = a.page_table + (long long)b * sh.max_pages;
+  for (int j = tid; j < ns; j += kT0) {
+    const int page = pt[j * st];
+    const bool ok = page >= 0 && page < sh.num_pages;
+    spage[j] = ok ? page : -1;
+    if (!ok) raise_error(a.err, SD_EBIT_PAGE);
+  }
+  __syncthreads();
   BFrag bf[HB];
 #pragma unroll
   for (int hb = 0; hb < HB; ++hb) bf[hb] = load_bfrag(qs, hb, gq, tq);
-  const int32_t *pt = a.page_table + (long long)b * sh.max_pages;
   const uint16_t *icache = a.index_cache + (long long)g * (kPage * kIndexDim);
   const long long page_stride = (long long)sh.Hkv * (kPage * kIndexDim);
   float smx[HB], smn[HB];
@@ -234,33 +239,27 @@ topk_window_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__
     smx[hb] = -INFINITY;
     smn[hb] = INFINITY;
   }
-  constexpr int U = 8;
+  constexpr int U = 16;
   for (int j0 = warp; j0 < ns; j0 += (kT0 / 32) * U) {
     uint32_t af[U][4];
-    bool ok[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int j = j0 + u * (kT0 / 32);
-      ok[u] = false;
       af[u][0] = af[u][1] = af[u][2] = af[u][3] = 0u;
-      if (j < ns) {
-        const int page = pt[j * st];
-        if (page >= 0 && page < sh.num_pages) {
-          const uint32_t *pg = reinterpret_cast<const uint32_t *>(icache + page * page_stride);
-          af[u][0] = __ldg(pg + gq * 8 + tq);
-          af[u][1] = __ldg(pg + (gq + 8) * 8 + tq);
-          af[u][2] = __ldg(pg + gq * 8 + tq + 4);
-          af[u][3] = __ldg(pg + (gq + 8) * 8 + tq + 4);
-          ok[u] = true;
-        } else if (lane == 0) {
-          raise_error(a.err, SD_EBIT_PAGE);
-        }
+      const int page = j < ns ? spage[j] : -1;
+      if (page >= 0) {
+        const uint32_t *pg = reinterpret_cast<const uint32_t *>(icache + page * page_stride);
+        af[u][0] = __ldg(pg + gq * 8 + tq);
+        af[u][1] = __ldg(pg + (gq + 8) * 8 + tq);
+        af[u][2] = __ldg(pg + gq * 8 + tq + 4);
+        af[u][3] = __ldg(pg + (gq + 8) * 8 + tq + 4);
       }
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int j = j0 + u * (kT0 / 32);
       if (j >= ns) break;
+      const bool ok = spage[j] >= 0;
       float sc[HB][2];
       score_frag<HB>(af[u], bf, sc);
 #pragma unroll
@@ -270,7 +269,7 @@ topk_window_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
           const int row = gq + 8 * r;
-          const bool valid = ok[u] && (long long)j * st * kPage + row < N;
+          const bool valid = ok && (long long)j * st * kPage + row < N;
           const float v = valid ? sc[hb][r] : -INFINITY;
           sample[h][j * 16 + row] = v;
           if (valid) {
@@ -295,40 +294,52 @@ topk_window_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__
     }
   }
   __syncthreads();
+  if (tid < nr) {
+    const float lo = key_to_float(smin[tid]), hi = key_to_float(smax[tid]);
+    hlo[tid] = lo;
+    hinv[tid] = (smax[tid] != 0u && hi > lo) ? (float)kSampleBins / (hi - lo) : 0.0f;
+  }
+  __syncthreads();
   for (int o = tid; o < nr * ns * 16; o += kT0) {
     const int h = o / (ns * 16), r = o % (ns * 16);
     const float v = sample[h][r];
     if (v == -INFINITY) continue;
-    const float lo = key_to_float(smin[h]), hi = key_to_float(smax[h]);
-    const float inv = hi > lo ? (float)kSampleBins / (hi - lo) : 0.0f;
-    atomicAdd(&shist[h][std::min(kSampleBins - 1, std::max(0, __float2int_rz((v - lo) * inv)))], 1u);
+    atomicAdd(&shist[h][std::min(kSampleBins - 1, std::max(0, __float2int_rz((v - hlo[h]) * hinv[h])))], 1u);
   }
   __syncthreads();
-  if (tid < nr) {
-    const int h = tid;
-    long long m = 0;                                 // valid sample tokens
-    for (int j = 0; j < ns; ++j) m += std::max(0LL, std::min<long long>(16, N - (long long)j * st * kPage));
+  // one warp per head: the highest bin whose suffix count reaches r
+  for (int h = warp; h < nr; h += kT0 / 32) {
+    // valid sample tokens: every sampled page is full except possibly the last
+    const long long m = (long long)(ns - 1) * kPage + std::min<long long>(kPage, N - (long long)(ns - 1) * st * kPage);
     float tlo = -INFINITY, thi = INFINITY;
     if (smax[h] != 0u) {
-      const float lo = key_to_float(smin[h]), hi = key_to_float(smax[h]);
+      const float lo = hlo[h], hi = key_to_float(smax[h]);
       thi = hi;
       const double mu = (double)m * (double)kb / (double)N;
       const double r = ceil(mu + 6.0 * sqrt(mu) + 8.0);
       if (r < (double)m) {
-        uint32_t cum = 0;
         int blo = 0;
-        for (int bin = kSampleBins - 1; bin >= 0; --bin) {
-          cum += shist[h][bin];
-          if ((double)cum >= r) {
-            blo = bin;
+        uint32_t acc = 0;
+        for (int top = kSampleBins; top > 0; top -= 32) {
+          const uint32_t c = shist[h][top - 32 + lane];
+          uint32_t suf = c;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_down_sync(kFull, suf, o);
+            if (lane + o < 32) suf += y;
+          }
+          const unsigned bal = __ballot_sync(kFull, (double)(acc + suf) >= r);
+          if (bal) {
+            blo = top - 32 + (31 - __clz(bal));
             break;
           }
+          acc += __shfl_sync(kFull, suf, 0);
         }
         tlo = lo + (float)blo * ((hi - lo) / (float)kSampleBins);
       }
     }
     const float inv = (tlo > -INFINITY && thi > tlo) ? (float)kBins / (thi - tlo) : 0.0f;
-    ws.win[(long long)b * sh.H_ret + grp.row[h]] = make_float4(tlo, thi, inv, 0.0f);
+    if (lane == 0) ws.win[(long long)b * sh.H_ret + grp.row[h]] = make_float4(tlo, thi, inv, 0.0f);
   }
 }
 
@@ -341,15 +352,16 @@ __global__ void __launch_bounds__(kT1)
 topk_stream_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__ groups, int n_groups,
                    const TopkWs ws) {
   constexpr int HB = (GR + 3) / 4;
+  constexpr int SL = stage_lane(GR);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gq = lane >> 2, tq = lane & 3;
   const int item = blockIdx.y;
   const int b = item / n_groups, gi = item % n_groups;
-  constexpr int SE = stage_entries(GR);
   extern __shared__ __align__(128) unsigned char dyn1[];
   unsigned char (*ring)[kRing][kPageBytes] = reinterpret_cast<unsigned char (*)[kRing][kPageBytes]>(dyn1);
-  unsigned long long (*stage)[GR][SE] =
-      reinterpret_cast<unsigned long long (*)[GR][SE]>(dyn1 + (size_t)kW1 * kRing * kPageBytes);
+  // lane-private staging: entry e of (warp, head block hb) for lane l at stage[warp][hb][e][l]
+  unsigned long long (*stage)[HB][SL][32] =
+      reinterpret_cast<unsigned long long (*)[HB][SL][32]>(dyn1 + (size_t)kW1 * kRing * kPageBytes);
   __shared__ int32_t pt_s[kChunkPages];
   __shared__ uint32_t qs[16 * 24];
   __shared__ Group grp;
@@ -365,11 +377,12 @@ topk_stream_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__
   if (p0 >= pages) return;
   const int np = pages - p0 < kChunkPages ? pages - p0 : kChunkPages;
   {
+    // page id -> page * Hkv + g (the 512-byte index block of this KV head), or -1
     const int32_t *pt = a.page_table + (long long)b * sh.max_pages + p0;
     for (int o = tid; o < np; o += kT1) {
       const int page = pt[o];
       const bool ok = page >= 0 && page < sh.num_pages;
-      pt_s[o] = ok ? page : -1;
+      pt_s[o] = ok ? page * sh.Hkv + g : -1;
       if (!ok) raise_error(a.err, SD_EBIT_PAGE);
     }
     for (int o = tid; o < 16 * 24; o += kT1) {
@@ -381,15 +394,14 @@ topk_stream_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__
 
   // per-warp ring: this warp reads pages warp, warp + 8, ... of the chunk
   const uint32_t ring_base = (uint32_t)__cvta_generic_to_shared(&ring[warp][0][0]);
-  const uint16_t *icache = a.index_cache + (long long)g * (kPage * kIndexDim) + lane * 8;
-  const long long page_stride = (long long)sh.Hkv * (kPage * kIndexDim);
+  const unsigned char *iblk = reinterpret_cast<const unsigned char *>(a.index_cache) + lane * 16;
   const uint32_t st_off = page_off(lane >> 1, lane & 1);
   const int nq = np > warp ? (np - warp + kW1 - 1) / kW1 : 0;
   auto issue = [&](int q) {
     if (q < nq) {
-      const int page = pt_s[warp + q * kW1];
-      cp_async16(ring_base + (q % kRing) * kPageBytes + st_off, page >= 0 ? icache + page * page_stride : icache,
-                 page >= 0 ? 16 : 0);
+      const int blk = pt_s[warp + q * kW1];
+      cp_async16(ring_base + (q % kRing) * kPageBytes + st_off, iblk + (size_t)(blk >= 0 ? blk : 0) * kPageBytes,
+                 blk >= 0 ? 16 : 0);
     }
     cp_async_commit();
   };
@@ -397,76 +409,82 @@ topk_stream_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__
   for (int q = 0; q < kRing; ++q) issue(q);
 
   BFrag bf[HB];
-  float tlo[HB], thi[HB], inv[HB];
+  float tlo[HB];
   long long row_of[HB];
 #pragma unroll
   for (int hb = 0; hb < HB; ++hb) {
     bf[hb] = load_bfrag(qs, hb, gq, tq);
     const int h = hb * 4 + tq;
     row_of[hb] = h < nr ? (long long)b * sh.H_ret + grp.row[h] : 0;
-    const float4 w = h < nr ? ws.win[row_of[hb]] : make_float4(INFINITY, INFINITY, 0.f, 0.f);
-    tlo[hb] = w.x;
-    thi[hb] = w.y;
-    inv[hb] = w.z;
+    tlo[hb] = h < nr ? ws.win[row_of[hb]].x : INFINITY;   // absent heads keep nothing
   }
-  const unsigned head_lanes = 0x11111111u << tq;
-  const unsigned lt = (1u << lane) - 1u;
-  uint32_t staged[HB];
+  uint32_t cnt[HB];
 #pragma unroll
-  for (int hb = 0; hb < HB; ++hb) staged[hb] = 0u;
-  // move this warp's staged entries of head block hb to the heads' buffers:
-  // lane tq reserves the space for head 4hb + tq, the head's 8 lanes copy
-  auto flush = [&](int hb) {
-    const int h = hb * 4 + tq;
-    uint32_t base = 0u;
-    if (gq == 0 && h < nr && staged[hb] > 0u) base = atomicAdd(&ws.bcount[row_of[hb]], staged[hb]);
-    base = __shfl_sync(kFull, base, tq);
-    if (h < nr) {
-      unsigned long long *dst = ws.buf + row_of[hb] * ws.cap;
-      for (uint32_t e = gq; e < staged[hb]; e += 8) {
-        const uint32_t at = base + e;
-        if (at < (uint32_t)ws.cap) dst[at] = stage[warp][h][e];
-      }
-    }
-    __syncwarp();
-    staged[hb] = 0u;
-  };
-  const uint32_t ld = ring_base + page_off((lane & 7) + ((lane >> 3) & 1) * 8, lane >> 4);
-  for (int q = 0; q < nq; ++q) {
-    cp_async_wait<kRing - 1>();
-    __syncwarp();
-    uint32_t af[4];
-    ldmatrix_x4(af, ld + (q % kRing) * kPageBytes);
-    __syncwarp();
-    const int pl = warp + q * kW1;                   // page within the chunk
-    const bool ok = pt_s[pl] >= 0;
-    issue(q + kRing);
-    float sc[HB][2];
-    score_frag<HB>(af, bf, sc);
-    const long long pos0 = (long long)(p0 + pl) * kPage + gq;
+  for (int hb = 0; hb < HB; ++hb) cnt[hb] = 0u;
+  // move the warp's staged entries to the heads' buffers: the 8 lanes of a
+  // head (same tq) take consecutive ranges of one reservation
+  auto flush = [&]() {
 #pragma unroll
     for (int hb = 0; hb < HB; ++hb) {
       const int h = hb * 4 + tq;
+      uint32_t incl = cnt[hb];
 #pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const long long pos = pos0 + 8 * r;
-        const float s = sc[hb][r];
-        const bool in = ok && h < nr && pos < N && s >= tlo[hb];
-        const unsigned m = __ballot_sync(kFull, in) & head_lanes;
-        if (in) {
-          const int cls = window_bin(s, tlo[hb], thi[hb], inv[hb]);
-          atomicAdd(&ws.hist[row_of[hb] * (kBins + 1) + cls], 1u);
-          stage[warp][h][staged[hb] + __popc(m & lt)] = ((unsigned long long)order_key(s) << 32) | (uint32_t)pos;
-        }
-        staged[hb] += __popc(m);
+      for (int o = 4; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += y;
       }
-      // all lanes of a head share staged[hb]; flush when another page could overflow
-      const bool full = __any_sync(kFull, staged[hb] > (uint32_t)(SE - 16));
-      if (full) flush(hb);
+      const uint32_t tot = __shfl_sync(kFull, incl, 28 + tq);
+      uint32_t base = 0u;
+      if (gq == 0 && h < nr && tot > 0u) base = atomicAdd(&ws.bcount[row_of[hb]], tot);
+      base = __shfl_sync(kFull, base, tq) + (incl - cnt[hb]);
+      if (h < nr) {
+        unsigned long long *dst = ws.buf + row_of[hb] * ws.cap;
+        for (uint32_t e = 0; e < cnt[hb]; ++e)
+          if (base + e < (uint32_t)ws.cap) dst[base + e] = stage[warp][hb][e][lane];
+      }
+      cnt[hb] = 0u;
     }
-  }
+    __syncwarp();
+  };
+  const uint32_t ld = ring_base + page_off((lane & 7) + ((lane >> 3) & 1) * 8, lane >> 4);
+  const uint32_t n32 = (uint32_t)N;
+  // two pages per iteration (q, q + 1); one cp.async group per page
+  for (int q = 0; q < nq; q += 2) {
+    cp_async_wait<kRing - 2>();
+    __syncwarp();
+    uint32_t af[2][4];
+    ldmatrix_x4(af[0], ld + (q % kRing) * kPageBytes);
+    ldmatrix_x4(af[1], ld + ((q + 1) % kRing) * kPageBytes);
+    __syncwarp();
+    const int pl = warp + q * kW1;                   // page within the chunk
+    const bool ok0 = pt_s[pl] >= 0;
+    const bool ok1 = q + 1 < nq && pt_s[pl + kW1] >= 0;
+    issue(q + kRing);
+    issue(q + kRing + 1);
+    float sc[2][HB][2];
+    score_frag<HB>(af[0], bf, sc[0]);
+    score_frag<HB>(af[1], bf, sc[1]);
+    const uint32_t pos0 = (uint32_t)(p0 + pl) * kPage + gq;
+    bool full = false;
 #pragma unroll
-  for (int hb = 0; hb < HB; ++hb) flush(hb);
+    for (int hb = 0; hb < HB; ++hb) {
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const uint32_t pos = pos0 + u * (kW1 * kPage) + 8 * r;
+          const float s = sc[u][hb][r];
+          if ((u ? ok1 : ok0) && s >= tlo[hb] && pos < n32) {
+            stage[warp][hb][cnt[hb]][lane] = ((unsigned long long)order_key(s) << 32) | pos;
+            ++cnt[hb];
+          }
+        }
+      }
+      full |= cnt[hb] > (uint32_t)(SL - 4);
+    }
+    if (__any_sync(kFull, full)) flush();
+  }
+  flush();
   cp_async_wait<0>();
 }
 
@@ -477,6 +495,7 @@ __global__ void __launch_bounds__(kT2)
 topk_resolve_kernel(const SelectArgs a, const Shape sh, const TopkWs ws) {
   extern __shared__ uint32_t bitmap[];               // [max_len / 32]
   __shared__ unsigned long long cand[kCap];
+  __shared__ uint32_t hist[kBins + 1];
   __shared__ uint32_t n_cand;
   __shared__ int cut_s, fail_s;
   __shared__ long long need_s;
@@ -496,8 +515,20 @@ topk_resolve_kernel(const SelectArgs a, const Shape sh, const TopkWs ws) {
     if (tid == 0) a.sel_count[row] = (int32_t)std::min(N, a.sel_stride);
     return;
   }
-  const uint32_t *hist = ws.hist + row * (kBins + 1);
   const float4 w = ws.win[row];
+  const uint32_t nbuf = ws.bcount[row];
+  const unsigned long long *buf = ws.buf + row * ws.cap;
+  const int n = (int)std::min<uint32_t>(nbuf, (uint32_t)ws.cap);
+  const int words = (int)((N + 31) / 32);
+  for (int o = tid; o < words; o += kT2) bitmap[o] = 0u;
+  for (int o = tid; o <= kBins; o += kT2) hist[o] = 0u;
+  __syncthreads();
+  // window histogram of the buffered scores (all >= t_lo)
+  for (int e = tid; e < n; e += kT2) {
+    const uint32_t key = (uint32_t)(buf[e] >> 32);
+    atomicAdd(&hist[window_bin(key_to_float(key), w.x, w.y, w.z)], 1u);
+  }
+  __syncthreads();
   // cut bin: warp 0 scans the histogram from the top, 32 bins at a time
   if (warp == 0) {
     const long long top = hist[kBins];
@@ -527,7 +558,7 @@ topk_resolve_kernel(const SelectArgs a, const Shape sh, const TopkWs ws) {
       }
     }
     if (lane == 0) {
-      const bool bad = need <= 0 || cut < 0 || ncut > kCap || ws.bcount[row] > (uint32_t)ws.cap;
+      const bool bad = need <= 0 || cut < 0 || ncut > kCap || nbuf > (uint32_t)ws.cap;
       fail_s = bad;
       cut_s = cut;
       need_s = need - acc;                           // tokens to take from the cut bin
@@ -539,12 +570,7 @@ topk_resolve_kernel(const SelectArgs a, const Shape sh, const TopkWs ws) {
     if (tid == 0) atomicOr(&ws.fail[ws.rowitem[row]], 1u);
     return;
   }
-  const int words = (int)((N + 31) / 32);
-  for (int o = tid; o < words; o += kT2) bitmap[o] = 0u;
-  __syncthreads();
   const int cut = cut_s;
-  const unsigned long long *buf = ws.buf + row * ws.cap;
-  const int n = (int)ws.bcount[row];
   for (int e = tid; e < n; e += kT2) {
     const unsigned long long ent = buf[e];
     const uint32_t key = (uint32_t)(ent >> 32), pos = (uint32_t)ent;
@@ -623,7 +649,7 @@ TopkPlan topk_plan(const Shape &sh, const Tables &tb) {
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct TopkLayout {
-  size_t qsplit, win, hist, bcount, rowitem, buf, total;
+  size_t qsplit, win, bcount, rowitem, buf, total;
 };
 
 TopkLayout topk_layout(const Shape &sh, int batch, int cap) {
@@ -632,7 +658,6 @@ TopkLayout topk_layout(const Shape &sh, int batch, int cap) {
   size_t o = 0;
   L.qsplit = o;  o = align256(o + rows * 24 * 4);
   L.win = o;     o = align256(o + rows * 16);
-  L.hist = o;    o = align256(o + rows * (kBins + 1) * 4);
   L.bcount = o;  o = align256(o + rows * 4);
   L.rowitem = o; o = align256(o + rows * 4);
   L.buf = o;     o = align256(o + rows * (size_t)cap * 8);
@@ -661,7 +686,7 @@ cudaError_t topk_launch(const SelectArgs &a, const Shape &sh, const Tables &tb, 
                         size_t bitmap_bytes, cudaStream_t st) {
   const int items = a.batch * tb.n_ret;
   const size_t smem0 = (size_t)GR * sample_pages(GR) * 16 * 4 + (size_t)GR * kSampleBins * 4;
-  const size_t smem1 = (size_t)kW1 * kRing * kPageBytes + (size_t)kW1 * GR * stage_entries(GR) * 8;
+  const size_t smem1 = (size_t)kW1 * kRing * kPageBytes + (size_t)kW1 * ((GR + 3) / 4) * stage_lane(GR) * 32 * 8;
   cudaError_t e = set_smem_once(topk_window_kernel<GR>, smem0);
   if (e == cudaSuccess) e = set_smem_once(topk_stream_kernel<GR>, smem1);
   if (e == cudaSuccess) e = set_smem_once(topk_resolve_kernel, bitmap_bytes);
@@ -695,7 +720,6 @@ cudaError_t launch_select_topk_stream(const SelectArgs &a, const Shape &sh, cons
   TopkWs ws{};
   ws.qsplit = reinterpret_cast<uint32_t *>(base + L.qsplit);
   ws.win = reinterpret_cast<float4 *>(base + L.win);
-  ws.hist = reinterpret_cast<uint32_t *>(base + L.hist);
   ws.bcount = reinterpret_cast<uint32_t *>(base + L.bcount);
   ws.rowitem = reinterpret_cast<int *>(base + L.rowitem);
   ws.buf = reinterpret_cast<unsigned long long *>(base + L.buf);

@@ -131,7 +131,8 @@ enum {
  *                              unbiased estimate of q.k/sqrt(d) for a projection
  *                              with i.i.d. N(0, 1/d) entries.
  *   max_batch                  largest B of any later call.
- *   max_pages_per_seq          MAXP, the page-table row length.
+ *   max_pages_per_seq          MAXP, the page-table row length; MAXP * P (the
+ *                              longest context) must not exceed 2^25 tokens.
  */
 typedef struct {
   int num_q_heads;
@@ -165,7 +166,9 @@ typedef struct {
  *
  * Allocates the device copy of the projection, a head table and a 4-byte
  * device error word.  Returns SD_ERR_INVALID_ARG or SD_ERR_UNSUPPORTED for a
- * bad or unsupported configuration, SD_ERR_CUDA if an allocation fails.
+ * bad or unsupported configuration (among them a pool whose
+ * num_pages * Hkv * P cache rows do not fit 32-bit row numbers),
+ * SD_ERR_CUDA if an allocation fails.
  */
 SD_API sd_status sparse_decode_init(const sd_config *cfg, const void *proj, sd_ctx **out);
 

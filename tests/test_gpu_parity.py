@@ -197,6 +197,88 @@ def test_host_side_argument_errors():
     st.close()
 
 
+# ------------------------------------------------------------------ top-k fallback
+
+def _group_query_keys(w, b, n, gain, noise, seed):
+    """[Hkv, n, d] bf16 keys along the mean pre-RoPE query of each GQA group
+    (times `gain`) plus N(0, noise^2) noise: their index scores sit far above
+    those of N(0, 1) keys."""
+    G = w.num_q_heads // w.num_kv_heads
+    qm = w.q_pre[b].float().view(w.num_kv_heads, G, w.head_dim).mean(1)
+    qm = qm / qm.norm(dim=-1, keepdim=True) * math.sqrt(w.head_dim)
+    gen = torch.Generator(device=w.k_cache.device)
+    gen.manual_seed(seed)
+    eps = torch.randn((w.num_kv_heads, n, w.head_dim), generator=gen, device=w.k_cache.device)
+    return (gain * qm[:, None, :] + noise * eps).to(torch.bfloat16)
+
+
+def _set_keys(w, b, positions, keys):
+    """k_cache rows of sequence b at `positions` (all KV heads) := keys [Hkv, n, d]."""
+    pos = torch.as_tensor(positions, device=w.page_table.device, dtype=torch.long)
+    pages = w.page_table[b, pos // w.page_size].long()
+    slots = pos % w.page_size
+    for g in range(w.num_kv_heads):
+        w.k_cache[pages, g, slots] = keys[g]
+
+
+def _exact_sets(w, seqs, label):
+    """Sets must equal the oracle's exactly (ties go to the lower position on
+    both sides); outputs are checked by check_workload."""
+    st = make_step(w)
+    st.select(w.q_pre)
+    torch.cuda.synchronize()
+    assert st.error_word() == 0
+    ref = O.decode_reference(oracle_config(w), **oracle_inputs(w, seqs),
+                             pairs=_pairs(w, range(len(seqs))), keep_scores=True)
+    retr = [h for h in range(w.num_q_heads) if w.head_is_retrieval[h]]
+    got = gpu_sets(st, w, [(b, h) for b in seqs for h in retr])
+    for i, b in enumerate(seqs):
+        for h in retr:
+            assert np.array_equal(got[(b, h)], np.asarray(ref.sets[(i, h)])), f"{label} b={b} h={h}"
+    st.close()
+    return ref
+
+
+def test_topk_sample_overestimate_falls_back_to_exact():
+    """High-scoring keys on every 8th page, the stride at which the score
+    window samples a 2048-page context: the sample then puts the window above
+    the k-th score, the streaming pass cannot resolve the budget, and the
+    exact selector must produce the same sets."""
+    w = make_workload("topk_128k", "cuda", B=2, N=32768)
+    for b in range(w.batch):
+        pos = [p * 16 + s for p in range(0, 2048, 8) for s in range(16)]
+        _set_keys(w, b, pos, _group_query_keys(w, b, len(pos), 2.0, 0.5, 100 + b))
+    ref = _exact_sets(w, [0, 1], "planted sample pages")
+    # the construction: for many heads every selected token is a planted one
+    # (keys follow the group's mean query, which some heads barely share), so
+    # several groups take the exact path
+    planted = set(p * 16 + s for p in range(0, 2048, 8) for s in range(16))
+    inside = [set(int(x) for x in sset) <= planted for (i, h), sset in ref.sets.items()
+              if w.head_is_retrieval[h]]
+    assert sum(inside) * 4 >= len(inside)
+    check_workload(w, seqs=[0, 1], heads=[0, 5, 31], label="planted sample pages")
+
+
+def test_topk_heavy_ties_fall_back_to_exact():
+    """Keys drawn from 6 distinct vectors besides 400 distinct high-scoring
+    ones: the k-th score is shared by thousands of tokens, more than the
+    streaming pass ranks exactly, so the exact selector takes over and must
+    break the ties by position like the definition does."""
+    w = make_workload("topk_128k", "cuda", B=1, N=40000)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(7)
+    base = torch.randn((w.num_kv_heads, 6, w.head_dim), generator=gen, device="cuda").to(torch.bfloat16)
+    pick = torch.randint(0, 6, (40000,), generator=gen, device="cuda")
+    _set_keys(w, 0, list(range(40000)), base[:, pick])
+    high = torch.randperm(40000, generator=gen, device="cuda")[:400].sort().values.cpu().tolist()
+    _set_keys(w, 0, high, _group_query_keys(w, 0, 400, 2.0, 0.5, 11))
+    ref = _exact_sets(w, [0], "heavy ties")
+    for (i, h), sset in ref.sets.items():
+        if w.head_is_retrieval[h]:
+            assert len(sset) == math.floor(float(np.float32(0.02)) * 40000)   # 799
+    check_workload(w, seqs=[0], heads=[0, 13, 31], label="heavy ties")
+
+
 # ------------------------------------------------------------------ full sizes
 
 FULL = [
