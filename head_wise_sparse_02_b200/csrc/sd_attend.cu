@@ -8,30 +8,36 @@
 // (gist.science/ar/paper/2608.06849), Methodology 4: sinks + recent window;
 // roles are shared by the heads of a GQA group.
 //
+// Work item = (sequence b, KV group g, role): a retrieval item's rows are the
+// union of its heads' selected positions, a local item's rows are
+// [0, sinks) U [N - window, N).  Rows are processed in 16-row tiles.
+//
 // Two launches:
-//   plan  one CTA per (sequence b, KV group g with retrieval heads, span of
-//         positions).  Finds each head's sub-list of its ascending selected
-//         positions inside the span (warp-cooperative search), marks them in
-//         per-head bitmaps and compacts the union into an ordered list of
-//         (cache row, head mask): every union row is read once for all the
-//         group's heads that selected it.  The page of each row is resolved
-//         here, from a shared-memory copy of the span's page-table slice.
-//   main  one CTA per (b, g, role, chunk).  A retrieval chunk is an equal share
-//         of the (b, g) union list (the span lists concatenated); a local chunk
-//         is a run of 1024 rows of [0, sinks) U [N - window, N).  Four warps
-//         stream 16-row K/V tiles through per-warp cp.async rings (XOR-swizzled
-//         16-byte chunks) and run them on the tensor cores in the
-//         FlashAttention-2 arrangement: S = Q K^T with mma.m16n8k16 (A = the
-//         group's bf16 queries, heads on M; B = K rows by ldmatrix), a masked
-//         online softmax per head in base 2, then O += P V with P taken
+//   plan  one CTA per (b, retrieval group, span of positions).  Finds each
+//         head's sub-list of its ascending selected positions inside the span
+//         (warp-cooperative search), marks them in per-head bitmaps and
+//         compacts the union into an ordered list of (cache row, head mask):
+//         every union row is read once for all the group's heads that
+//         selected it.  The page of each row is resolved here, from a
+//         shared-memory copy of the span's page-table slice.  The last plan
+//         CTA to finish (atomic ticket) lays all items end to end and writes
+//         the first tile of each (a prefix sum over the items' tile counts).
+//   main  a persistent grid, one CTA per resident slot.  CTA c takes the
+//         equal share [W c / P, W (c + 1) / P) of all W tiles and walks the
+//         items it overlaps (usually one or two), so that its rings run
+//         without the start and drain of a grid of small CTAs.  Four warps
+//         stream tiles through per-warp cp.async rings (whole rows per
+//         instruction, padded row pitch) and run them on the tensor cores in
+//         the FlashAttention-2 arrangement: S = Q K^T with mma.m16n8k16 (A =
+//         the group's bf16 queries, heads on M; B = K rows by ldmatrix), a
+//         masked online softmax per head in base 2, then O += P V with P taken
 //         straight from the S fragments, split exactly into bf16 hi + lo terms
 //         so that P keeps float32 accuracy (B = V rows by ldmatrix.trans).
-//         Each CTA merges its warps and writes one partial (m, l, acc[d]) per
-//         (b, head, chunk); the last CTA of a (b, g, role) to finish (atomic
-//         ticket, no waiting) merges the partials with a log-sum-exp combine
-//         into out[b, h, :] and resets the ticket.
+//         For every item it touched a CTA merges its warps; an item that lies
+//         inside one CTA goes to out directly, otherwise each CTA writes a
+//         partial (m, l, acc[d]) and the last to finish (atomic ticket, no
+//         waiting) merges the partials with a log-sum-exp combine.
 #include <algorithm>
-#include <cmath>
 #include <map>
 #include <mutex>
 
@@ -52,11 +58,9 @@ constexpr int kSpanMax = 8192;          // positions per plan CTA (max)
 constexpr int kThreads = 128;
 constexpr int kWarps = kThreads / 32;
 constexpr int kTileRows = 16;
-constexpr int kTileRing = 2;            // tiles in flight per warp
+constexpr int kTileRing = 3;            // tiles in flight per warp
 constexpr int kPassRows = 1024;         // list entries staged in shared memory per pass
-constexpr int kSpanLoc = 1024;          // local rows per chunk
-constexpr int kChunksRet = 16;          // retrieval chunks per (b, g), at most
-constexpr int kRowsPerChunk = 512;      // retrieval: aim for at least this many rows per chunk
+constexpr int kMaxGrid = 4096;          // persistent CTAs (partial slots are sized for this)
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, int src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
@@ -78,21 +82,21 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
 // d += a * b, bf16 inputs, float32 accumulate
 __device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};\n"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 // the same with rows 8-15 of A zero: only d0, d1 (rows 0-7) are kept, so the
-// accumulators of the empty rows need no registers
-__device__ __forceinline__ void mma_bf16_top(float (&d)[2], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
-  float j0, j1;
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%5}, {%7,%8}, "
+// accumulators of the empty rows need no registers; zu / zf hold 0 (kept in
+// one register each by the caller)
+__device__ __forceinline__ void mma_bf16_top(float (&d)[2], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1,
+                                             uint32_t zu, float zf) {
+  [[maybe_unused]] float j0, j1;                    // outputs of the empty rows, discarded
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%5}, {%7,%8}, "
       "{%0,%1,%9,%9};\n"
       : "+f"(d[0]), "+f"(d[1]), "=f"(j0), "=f"(j1)
-      : "r"(a0), "r"(0u), "r"(a2), "r"(b0), "r"(b1), "f"(0.0f));
+      : "r"(a0), "r"(zu), "r"(a2), "r"(b0), "r"(b1), "f"(zf));
 }
 // two floats -> bf16x2 (x in the low half), round to nearest even
 __device__ __forceinline__ uint32_t pack_bf16(float x, float y) {
@@ -109,12 +113,13 @@ __device__ __forceinline__ void split_bf16(float x, float y, uint32_t &hi, uint3
 // First index i in [0, n) with arr[i] >= x (n if none); whole warp cooperates.
 // Lanes 0..30 probe inside [lo, hi); lane 31 always lands at or past hi and
 // acts as the sentinel, so some lane is always true.
-__device__ int warp_lower_bound(const int32_t *arr, int n, int x, int lane) {
+template <typename T>
+__device__ int warp_lower_bound(const T *arr, int n, T x, int lane) {
   int lo = 0, hi = n;                      // answer in [lo, hi]
   while (hi - lo > 31) {
     const int step = (hi - lo + 30) / 31;  // 31 * step >= hi - lo
     const int p = lo + lane * step;
-    const bool ge = (p < hi) ? (__ldg(arr + p) >= x) : true;
+    const bool ge = (p < hi) ? (__ldcg(arr + p) >= x) : true;
     const int first = __ffs(__ballot_sync(kFull, ge)) - 1;
     const int nhi = std::min(hi, lo + first * step);
     const int nlo = first == 0 ? lo : lo + (first - 1) * step + 1;
@@ -122,52 +127,126 @@ __device__ int warp_lower_bound(const int32_t *arr, int n, int x, int lane) {
     hi = nhi;
   }
   const int p = lo + lane;                 // hi - lo <= 31: lane 31 is past hi
-  const bool ge = (p < hi) ? (__ldg(arr + p) >= x) : true;
+  const bool ge = (p < hi) ? (__ldcg(arr + p) >= x) : true;
   return lo + (__ffs(__ballot_sync(kFull, ge)) - 1);
 }
 
 struct AttParams {
   int span;                 // plan: positions per span (power of two, multiple of 32)
   int ns;                   // plan: spans per sequence
-  int c_r, c_l;             // main: chunks per retrieval / local item
-  int c_max;                // partial slots per (b, head)
+  int n_ret_items;          // B * n_ret retrieval items, numbered first
+  int ni;                   // all items: then B * n_loc local items
 };
 
 // Carving of the attend workspace.
 struct AttWs {
-  float *partials;          // [B][Hq][c_max][D + 2]
+  float *partials;          // [(kMaxGrid + ni) slots][GR][D + 2]
   uint32_t *plan_row;       // [B][n_ret][ns][span]: cache row of each union entry
   uint16_t *plan_mask;      // [B][n_ret][ns][span]: heads (bit i = i-th head of the group)
   int *plan_cnt;            // [B][n_ret][ns]
-  unsigned *tickets;        // [B][Hkv][2]
+  long long *tstart;        // [ni + 1]: first tile of each item; tstart[ni] = all tiles
+  int *item_rows;           // [ni]: rows of each item           } zeroed before
+  unsigned *tickets;        // [ni]: partials merged per item     } every call
+  unsigned *plan_ticket;    // [1]: plan CTAs finished            }
 };
 
+__device__ __forceinline__ const Group &item_group(const Tables &tb, const AttParams &ap, int i, int &b,
+                                                   bool &is_ret) {
+  is_ret = i < ap.n_ret_items;
+  if (is_ret) {
+    b = i / tb.n_ret;
+    return tb.ret[i % tb.n_ret];
+  }
+  const int j = i - ap.n_ret_items;
+  b = j / tb.n_loc;
+  return tb.loc[j % tb.n_loc];
+}
+
+__device__ __forceinline__ long long clamp_len(const AttendArgs &a, const Shape &sh, int b) {
+  const long long N = a.seq_lens[b];
+  return N < 0 ? 0 : std::min<long long>(N, sh.max_len);
+}
+
+// Tile counts and first tiles of all items, by one CTA (block size a multiple
+// of 32, at most 1024).  Retrieval items' rows were summed into item_rows by
+// the plan CTAs; local items' rows follow from N.  Items without rows get a
+// zero output here, since no main CTA visits them.
+template <int D>
+__device__ void item_prefix(const AttendArgs &a, const Shape &sh, const Tables &tb, const AttParams &ap,
+                            const AttWs &ws) {
+  __shared__ long long wsum[32];
+  __shared__ long long carry;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+  if (tid == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < ap.ni; base += blockDim.x) {
+    const int i = base + tid;
+    long long nt = 0;
+    if (i < ap.ni) {
+      int b;
+      bool is_ret;
+      const Group &grp = item_group(tb, ap, i, b, is_ret);
+      long long rows;
+      const long long N0 = a.seq_lens[b];
+      if (N0 < 0 || N0 > sh.max_len) raise_error(a.err, SD_EBIT_SEQLEN);
+      if (is_ret) {
+        rows = __ldcg(ws.item_rows + i);
+      } else {
+        const long long N = clamp_len(a, sh, b);
+        const long long la = std::min<long long>(a.num_sinks, N);
+        const long long lw = std::max<long long>(la, N - a.window);
+        rows = la + (N - lw);
+        ws.item_rows[i] = (int)rows;
+      }
+      nt = (rows + kTileRows - 1) / kTileRows;
+      if (rows == 0)
+        for (int x = 0; x < grp.n * D; ++x) a.out[((long long)b * sh.Hq + grp.q_head[x / D]) * D + x % D] = 0.0f;
+    }
+    long long incl = nt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long y = __shfl_up_sync(kFull, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    long long before = carry, total = 0;
+    for (int w = 0; w < nw; ++w) {
+      if (w < warp) before += wsum[w];
+      total += wsum[w];
+    }
+    if (i < ap.ni) ws.tstart[i] = before + incl - nt;
+    __syncthreads();
+    if (tid == 0) carry += total;
+    __syncthreads();
+  }
+  if (tid == 0) ws.tstart[ap.ni] = carry;
+}
+
+// The item layout alone, when there is no retrieval item to plan.
+template <int D>
+__global__ void __launch_bounds__(256)
+attend_prefix_kernel(const AttendArgs a, const Shape sh, const Tables tb, const AttParams ap, const AttWs ws) {
+  item_prefix<D>(a, sh, tb, ap, ws);
+}
+
 // ============================================================== plan kernel
-// dynamic shared memory: [per-head bitmaps: GR x span / 32 words][page slice: span / 16 ints]
+// Union list of the span [p0, p1) of retrieval item (b, gi): plan_cnt[slot],
+// the list in plan_row / plan_mask, and the count added to the item's rows.
+// hbm: [GR][span / 32] bitmap words; pslice: the span's pages.
 template <int GR>
-__global__ void __launch_bounds__(kPlanThreads)
-attend_plan_kernel(const AttendArgs a, const Shape sh, const Tables tb, const AttParams ap, const AttWs ws) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int split = blockIdx.x, gi = blockIdx.y, b = blockIdx.z;
-  __shared__ Group grp;
+__device__ void plan_span(const AttendArgs &a, const Shape &sh, const Tables &tb, const AttParams &ap,
+                          const AttWs &ws, const Group &grp, int b, int gi, int split, uint32_t *hbm, int *pslice) {
   __shared__ int seg_lo[kMaxGroup], seg_hi[kMaxGroup];
   __shared__ uint32_t wtot[kPlanWarps];
-  extern __shared__ uint32_t plan_dyn[];
-  const int bwords = ap.span / 32;
-  uint32_t *hbm = plan_dyn;
-  int *pslice = reinterpret_cast<int *>(plan_dyn + GR * bwords);
-  if (tid == 0) grp = tb.ret[gi];
-  __syncthreads();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nh = grp.n, g = grp.kv_head;
-  long long N = a.seq_lens[b];
-  if (N < 0 || N > sh.max_len) {
-    if (tid == 0 && split == 0 && gi == 0) raise_error(a.err, SD_EBIT_SEQLEN);
-    N = N < 0 ? 0 : sh.max_len;
-  }
+  const int bwords = ap.span / 32;
+  const long long N = clamp_len(a, sh, b);
   const long long slot = ((long long)b * tb.n_ret + gi) * ap.ns + split;
   const long long p0 = (long long)split * ap.span;
   const long long p1 = std::min(N, p0 + ap.span);
-  if (p0 >= N) {
+  if (p0 >= p1) {
     if (tid == 0) ws.plan_cnt[slot] = 0;
     return;
   }
@@ -181,7 +260,7 @@ attend_plan_kernel(const AttendArgs a, const Shape sh, const Tables tb, const At
       if (lane == 0 && (t & 1) == 0) raise_error(a.err, SD_EBIT_SEL);
       c = c < 0 ? 0 : a.sel_stride;
     }
-    const int at = warp_lower_bound(sel, (int)c, (int)((t & 1) ? p1 : p0), lane);
+    const int at = warp_lower_bound<int32_t>(sel, (int)c, (int32_t)((t & 1) ? p1 : p0), lane);
     if (lane == 0) ((t & 1) ? seg_hi : seg_lo)[i] = at;
   }
   for (int o = tid; o < nh * bwords; o += kPlanThreads) hbm[o] = 0u;
@@ -248,27 +327,57 @@ attend_plan_kernel(const AttendArgs a, const Shape sh, const Tables tb, const At
       ++o;
     }
   }
-  if (tid == 0) ws.plan_cnt[slot] = (int)total;
+  if (tid == 0) {
+    ws.plan_cnt[slot] = (int)total;
+    if (total) atomicAdd(ws.item_rows + (long long)b * tb.n_ret + gi, (int)total);
+  }
+}
+
+// dynamic shared memory: [per-head bitmaps: GR x span / 32 words][page slice: span / 16 ints]
+template <int D, int GR>
+__global__ void __launch_bounds__(kPlanThreads)
+attend_plan_kernel(const AttendArgs a, const Shape sh, const Tables tb, const AttParams ap, const AttWs ws) {
+  const int tid = threadIdx.x;
+  const int split = blockIdx.x, gi = blockIdx.y, b = blockIdx.z;
+  __shared__ Group grp;
+  __shared__ int last;
+  extern __shared__ uint32_t plan_dyn[];
+  if (tid == 0) grp = tb.ret[gi];
+  __syncthreads();
+  plan_span<GR>(a, sh, tb, ap, ws, grp, b, gi, split, plan_dyn, reinterpret_cast<int *>(plan_dyn + GR * (ap.span / 32)));
+  // the last plan CTA to finish lays out the items
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) last = atomicAdd(ws.plan_ticket, 1u) == gridDim.x * gridDim.y * gridDim.z - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  item_prefix<D>(a, sh, tb, ap, ws);
+  if (tid == 0) *ws.plan_ticket = 0u;
 }
 
 // ============================================================== main kernel
 struct MainShared {
   Group grp;
+  int item;                 // current item
   int last;
 };
 
-// dynamic shared memory: [ring: kWarps x kTileRing x (16 K rows + 16 V rows)]
+// dynamic shared memory: [ring: kWarps x kTileRing x (16 K rows + 16 V rows),
+//                         rows padded to 2d + 16 bytes: ldmatrix phases hit
+//                         distinct banks and every offset is a constant]
 //                        [pass list: kPassRows x uint32 cache row]
 //                        [kPassRows + 16 x uint16 head mask]
 //                        [span prefix: ns + 1 ints]
-// after the row loop the ring holds the warps' (m, l, acc) for the CTA merge
+// between items the ring holds the warps' (m, l, acc) for the CTA merge
 template <int D, int GR>
 __global__ void __launch_bounds__(kThreads)
 attend_main_kernel(const AttendArgs a, const Shape sh, const Tables tb, const AttParams ap, const AttWs ws) {
   constexpr int KS = D / 16;                         // k-steps of Q K^T
   constexpr int NT = D / 8;                          // n-tiles (8 dims) of P V
-  constexpr int kRowB = 2 * D;                       // bytes of one K (or V) row
-  constexpr int kTileB = 2 * kTileRows * kRowB;      // K tile + V tile
+  constexpr int kRowB = 2 * D;                       // bytes of one K (or V) row in the cache
+  constexpr int kPitch = kRowB + 16;                 // bytes of one row in shared memory
+  constexpr int kTileB = 2 * kTileRows * kPitch;     // K tile + V tile
   constexpr int CPR = kRowB / 16;                    // 16-byte chunks per row
   constexpr bool HI = GR > 8;                        // heads 8..15 present
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -280,347 +389,366 @@ attend_main_kernel(const AttendArgs a, const Shape sh, const Tables tb, const At
   uint16_t *lmask = reinterpret_cast<uint16_t *>(lrow + kPassRows);
   int *pre = reinterpret_cast<int *>(lmask + kPassRows + kTileRows);
 
-  // ---- decode the work item ------------------------------------------------
-  long long bid = blockIdx.x;
-  const long long n_ret_items = (long long)a.batch * tb.n_ret * ap.c_r;
-  const bool is_ret = bid < n_ret_items;
-  int b, gi, chunk, nc;
-  if (is_ret) {
-    b = (int)(bid / ((long long)tb.n_ret * ap.c_r));
-    const long long rem = bid % ((long long)tb.n_ret * ap.c_r);
-    gi = (int)(rem / ap.c_r);
-    chunk = (int)(rem % ap.c_r);
-    nc = ap.c_r;
-  } else {
-    bid -= n_ret_items;
-    b = (int)(bid / ((long long)tb.n_loc * ap.c_l));
-    const long long rem = bid % ((long long)tb.n_loc * ap.c_l);
-    gi = (int)(rem / ap.c_l);
-    chunk = (int)(rem % ap.c_l);
-    nc = ap.c_l;
-  }
-  if (tid == 0) S.grp = is_ret ? tb.ret[gi] : tb.loc[gi];
-  __syncthreads();
-  const int nh = S.grp.n;
-  const int g = S.grp.kv_head;
-  long long N = a.seq_lens[b];
-  if (N < 0 || N > sh.max_len) {
-    if (tid == 0 && chunk == 0 && !is_ret && gi == 0) raise_error(a.err, SD_EBIT_SEQLEN);
-    N = N < 0 ? 0 : sh.max_len;
+  // ---- this CTA's share of the tiles -----------------------------------------
+  const long long W = __ldcg(ws.tstart + ap.ni);
+  // with fewer tiles than CTAs only the first W take part (one tile each), so
+  // every CTA between an item's first and last one holds some of its tiles
+  const long long P = std::min<long long>(gridDim.x, W), c = blockIdx.x;
+  if (c >= P) return;
+  const long long t0 = W * c / P, t1 = W * (c + 1) / P;
+  // CTA holding tile x: the largest c' with floor(W c' / P) <= x
+  auto cta_of = [&](long long x) { return ((x + 1) * P - 1) / W; };
+  if (warp == 0) {
+    const int i = warp_lower_bound<long long>(ws.tstart, ap.ni + 1, t0 + 1, lane) - 1;   // tstart[i] <= t0 < tstart[i+1]
+    if (lane == 0) S.item = i;
   }
 
-  // ---- rows of this chunk: [r0, r1) of the item's row sequence ---------------
-  long long r0 = 0, r1 = 0;
-  long long loc_a = 0, loc_w = 0;
-  const long long slot0 = ((long long)b * tb.n_ret + gi) * ap.ns;
-  const int ns_item = is_ret ? (int)std::min<long long>(ap.ns, (N + ap.span - 1) / ap.span) : 0;
-  if (is_ret) {
-    // exclusive prefix of the span counts (warp 0, 32 spans at a time)
-    if (warp == 0) {
+  // cp.async mapping: one instruction copies whole rows (coalesced): for
+  // d = 128 lanes 0-15 the K row and lanes 16-31 the V row of tile row j; for
+  // d = 64 lanes 0-7 / 8-15 the K / V row of tile row 2j, lanes 16-31 row 2j + 1
+  constexpr int RPI = 32 / (2 * CPR);                // tile rows per instruction
+  const int c_sub = lane / (2 * CPR);                // which of them
+  const int c_isv = (lane / CPR) & 1;                // K or V
+  const int c_ch = lane % CPR;                       // 16-byte chunk of the row
+  const uint32_t ring_w = ring0 + warp * (kTileRing * kTileB);
+  const unsigned char *kbase = reinterpret_cast<const unsigned char *>(a.k_cache);
+  const unsigned char *vbase = reinterpret_cast<const unsigned char *>(a.v_cache);
+  // ldmatrix lane addresses inside a tile (plus a constant per k-step / n-tile)
+  const int lm = lane >> 3, lr = lane & 7;
+  const uint32_t k_lane = (lr + (lm >> 1) * 8) * kPitch + (lm & 1) * 16;   // K: rows (0-7 | 8-15) x chunk (2k | 2k+1)
+  const uint32_t v_lane = kTileRows * kPitch + (lr + (lm & 1) * 8) * kPitch + (lm >> 1) * 16;   // V: rows x chunk (n | n+1)
+  const float sc = a.attn_scale * kLog2e;
+  uint32_t zu = 0u;
+  float zf = 0.0f;
+  asm volatile("" : "+r"(zu), "+f"(zf));             // opaque zeros: one register each
+  const uint32_t head_bit0 = 1u << gq, head_bit1 = 1u << (gq + 8);
+
+  long long t = t0;
+  while (t < t1) {
+    __syncthreads();                                   // S.item set; the previous item's smem no longer read
+    int item = S.item;
+    long long ts = __ldcg(ws.tstart + item), te = __ldcg(ws.tstart + item + 1);
+    while (te <= t) {                                  // skip items without tiles
+      ++item;
+      ts = te;
+      te = __ldcg(ws.tstart + item + 1);
+    }
+    const long long seg_end = std::min(t1, te);
+    int b;
+    bool is_ret;
+    const Group &grp_g = item_group(tb, ap, item, b, is_ret);
+    if (tid == 0) S.grp = grp_g;
+    const long long N = clamp_len(a, sh, b);
+    const long long T = __ldcg(ws.item_rows + item);
+    const long long r0 = (t - ts) * kTileRows;
+    const long long r1 = std::min(T, (seg_end - ts) * kTileRows);
+    const long long first = cta_of(ts), last = cta_of(te - 1);
+    const int gi = is_ret ? item % tb.n_ret : 0;
+    const long long slot0 = ((long long)b * tb.n_ret + gi) * ap.ns;
+    const int ns_item = is_ret ? (int)((N + ap.span - 1) / ap.span) : 0;
+    if (is_ret && warp == 0) {
+      // exclusive prefix of the item's span counts (32 spans at a time)
       int run = 0;
       for (int s0 = 0; s0 < ns_item; s0 += 32) {
         const int s = s0 + lane;
-        const int c = s < ns_item ? ws.plan_cnt[slot0 + s] : 0;
-        int incl = c;
+        const int cnt = s < ns_item ? __ldcg(ws.plan_cnt + slot0 + s) : 0;
+        int incl = cnt;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
           const int y = __shfl_up_sync(kFull, incl, o);
           if (lane >= o) incl += y;
         }
-        if (s < ns_item) pre[s] = run + incl - c;
+        if (s < ns_item) pre[s] = run + incl - cnt;
         run += __shfl_sync(kFull, incl, 31);
       }
       if (lane == 0) pre[ns_item] = run;
     }
     __syncthreads();
-    const long long T = pre[ns_item];
-    const long long per = ((T + nc - 1) / nc + kTileRows - 1) / kTileRows * kTileRows;
-    r0 = std::min(T, (long long)chunk * per);
-    r1 = std::min(T, r0 + per);
-  } else {
-    loc_a = std::min<long long>(a.num_sinks, N);
-    loc_w = std::max<long long>(loc_a, N - a.window);
-    const long long L = loc_a + (N - loc_w);
-    r0 = std::min(L, (long long)chunk * kSpanLoc);
-    r1 = std::min(L, r0 + kSpanLoc);
-  }
+    const int nh = S.grp.n;
+    const int g = S.grp.kv_head;
+    const long long loc_a = std::min<long long>(a.num_sinks, N);
+    const long long loc_w = std::max<long long>(loc_a, N - a.window);
 
-  // ---- queries: A fragments of Q (heads on M), bf16 ------------------------
-  uint32_t qa[KS][4];
-  {
-    const uint16_t *q0 = gq < nh ? a.q + ((long long)b * sh.Hq + S.grp.q_head[gq]) * D : nullptr;
-    const uint16_t *q1 = (HI && gq + 8 < nh) ? a.q + ((long long)b * sh.Hq + S.grp.q_head[gq + 8]) * D : nullptr;
-#pragma unroll
-    for (int k = 0; k < KS; ++k) {
-      const int c = k * 16 + 2 * tq;
-      qa[k][0] = q0 ? *reinterpret_cast<const uint32_t *>(q0 + c) : 0u;
-      qa[k][2] = q0 ? *reinterpret_cast<const uint32_t *>(q0 + c + 8) : 0u;
-      qa[k][1] = q1 ? *reinterpret_cast<const uint32_t *>(q1 + c) : 0u;
-      qa[k][3] = q1 ? *reinterpret_cast<const uint32_t *>(q1 + c + 8) : 0u;
-    }
-  }
-  const float sc = a.attn_scale * kLog2e;
-  const uint32_t head_bit0 = 1u << gq, head_bit1 = 1u << (gq + 8);
-
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-  float o[NT][4];
-#pragma unroll
-  for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-
-  // cp.async mapping: lane -> tile row lane / 2, one half of its 16-byte chunks
-  const int crow = lane >> 1, chalf = lane & 1;
-  const uint32_t ring_w = ring0 + warp * (kTileRing * kTileB);
-  const unsigned char *kbase = reinterpret_cast<const unsigned char *>(a.k_cache);
-  const unsigned char *vbase = reinterpret_cast<const unsigned char *>(a.v_cache);
-  // byte offset of 16-byte chunk `ch` of tile row `row`: chunks XOR-swizzled by row % 8
-  auto swz = [](int row, int ch) -> uint32_t { return (uint32_t)(row * kRowB + ((ch ^ (row & 7)) << 4)); };
-  const int lm = lane >> 3, lr = lane & 7;
-  const int k_row = lr + (lm >> 1) * 8, k_chk = lm & 1;       // K: rows (0-7 | 8-15) x chunk (2k | 2k+1)
-  const int v_row = lr + (lm & 1) * 8, v_chk = lm >> 1;       // V: rows (0-7 | 8-15) x chunk (n | n+1)
-
-  for (long long ps = r0; ps < r1; ps += kPassRows) {
-    const int n = (int)std::min<long long>(kPassRows, r1 - ps);
-    __syncthreads();                                   // the previous pass no longer reads the list
-    // ---- stage the pass's list entries -------------------------------------
-    if (is_ret) {
-      for (int x = tid; x < n; x += kThreads) {
-        const long long gx = ps + x;
-        int lo = 0, hi = ns_item;                      // last span s with pre[s] <= gx
-        while (hi - lo > 1) {
-          const int mid = (lo + hi) >> 1;
-          if (pre[mid] <= gx) lo = mid;
-          else hi = mid;
-        }
-        const long long e = (slot0 + lo) * ap.span + (gx - pre[lo]);
-        lrow[x] = ws.plan_row[e];
-        lmask[x] = ws.plan_mask[e];
-      }
-    } else {
-      const int32_t *pt = a.page_table + (long long)b * sh.max_pages;
-      const uint16_t all = (uint16_t)((1u << nh) - 1u);
-      for (int x = tid; x < n; x += kThreads) {
-        const long long rr = ps + x;
-        const long long pos = rr < loc_a ? rr : loc_w + (rr - loc_a);
-        const int page = pt[pos / kPage];
-        const bool ok = page >= 0 && page < sh.num_pages;
-        if (!ok) raise_error(a.err, SD_EBIT_PAGE);
-        lrow[x] = ok ? (uint32_t)(((long long)page * sh.Hkv + g) * kPage + (pos % kPage)) : 0u;
-        lmask[x] = ok ? all : (uint16_t)0;
-      }
-    }
-    const int tiles = (n + kTileRows - 1) / kTileRows;
-    for (int x = n + tid; x < tiles * kTileRows; x += kThreads) lmask[x] = 0;
-    __syncthreads();
-
-    // ---- stream the pass's tiles: warp w takes tiles w, w + 4, ... ----------
-    const int mt = tiles > warp ? (tiles - warp + kWarps - 1) / kWarps : 0;
-    auto issue = [&](int t) {
-      if (t < mt) {
-        const int x = (warp + t * kWarps) * kTileRows + crow;
-        const bool ok = x < n;
-        const size_t row = ok ? lrow[x] : 0u;
-        const unsigned char *ks = kbase + row * kRowB;
-        const unsigned char *vs = vbase + row * kRowB;
-        const uint32_t dst = ring_w + (t % kTileRing) * kTileB;
-#pragma unroll 2                                 // full unrolling keeps 16 addresses live
-        for (int j = 0; j < CPR / 2; ++j) {
-          const int ch = chalf * (CPR / 2) + j;
-          const uint32_t off = swz(crow, ch);
-          cp_async16(dst + off, ks + ch * 16, ok ? 16 : 0);
-          cp_async16(dst + kTileRows * kRowB + off, vs + ch * 16, ok ? 16 : 0);
-        }
-      }
-      cp_async_commit();
-    };
-#pragma unroll
-    for (int t = 0; t < kTileRing; ++t) issue(t);
-
-    for (int t = 0; t < mt; ++t) {
-      cp_async_wait<kTileRing - 1>();
-      __syncwarp();
-      const uint32_t kt = ring_w + (t % kTileRing) * kTileB;
-      const uint32_t vt = kt + kTileRows * kRowB;
-      const int x0 = (warp + t * kWarps) * kTileRows;
-      // S = Q K^T: n-tile j holds rows 8j .. 8j + 7 of the tile
-      float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    // ---- queries: A fragments of Q (heads on M), bf16 ----------------------
+    uint32_t qa[KS][4];
+    {
+      const uint16_t *q0 = gq < nh ? a.q + ((long long)b * sh.Hq + S.grp.q_head[gq]) * D : nullptr;
+      const uint16_t *q1 = (HI && gq + 8 < nh) ? a.q + ((long long)b * sh.Hq + S.grp.q_head[gq + 8]) * D : nullptr;
 #pragma unroll
       for (int k = 0; k < KS; ++k) {
-        uint32_t kb[4];
-        ldsm_x4(kb, kt + swz(k_row, 2 * k + k_chk));
-        if constexpr (HI) {
-          mma_bf16(s[0], qa[k][0], qa[k][1], qa[k][2], qa[k][3], kb[0], kb[1]);
-          mma_bf16(s[1], qa[k][0], qa[k][1], qa[k][2], qa[k][3], kb[2], kb[3]);
-        } else {
-          float t0[2] = {s[0][0], s[0][1]}, t1[2] = {s[1][0], s[1][1]};
-          mma_bf16_top(t0, qa[k][0], qa[k][2], kb[0], kb[1]);
-          mma_bf16_top(t1, qa[k][0], qa[k][2], kb[2], kb[3]);
-          s[0][0] = t0[0]; s[0][1] = t0[1]; s[1][0] = t1[0]; s[1][1] = t1[1];
+        const int cc = k * 16 + 2 * tq;
+        qa[k][0] = q0 ? *reinterpret_cast<const uint32_t *>(q0 + cc) : 0u;
+        qa[k][2] = q0 ? *reinterpret_cast<const uint32_t *>(q0 + cc + 8) : 0u;
+        qa[k][1] = q1 ? *reinterpret_cast<const uint32_t *>(q1 + cc) : 0u;
+        qa[k][3] = q1 ? *reinterpret_cast<const uint32_t *>(q1 + cc + 8) : 0u;
+      }
+    }
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    float o[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+
+    for (long long ps = r0; ps < r1; ps += kPassRows) {
+      const int n = (int)std::min<long long>(kPassRows, r1 - ps);
+      __syncthreads();                                 // the previous pass no longer reads the list
+      // ---- stage the pass's list entries -----------------------------------
+      if (is_ret) {
+#pragma unroll 4
+        for (int x = tid; x < n; x += kThreads) {
+          const long long gx = ps + x;
+          int lo = 0, hi = ns_item;                    // last span s with pre[s] <= gx
+          while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (pre[mid] <= gx) lo = mid;
+            else hi = mid;
+          }
+          const long long e = (slot0 + lo) * ap.span + (gx - pre[lo]);
+          lrow[x] = __ldcg(ws.plan_row + e);
+          lmask[x] = __ldcg(ws.plan_mask + e);
+        }
+      } else {
+        const int32_t *pt = a.page_table + (long long)b * sh.max_pages;
+        const uint16_t all = (uint16_t)((1u << nh) - 1u);
+        for (int x = tid; x < n; x += kThreads) {
+          const long long rr = ps + x;
+          const long long pos = rr < loc_a ? rr : loc_w + (rr - loc_a);
+          const int page = pt[pos / kPage];
+          const bool ok = page >= 0 && page < sh.num_pages;
+          if (!ok) raise_error(a.err, SD_EBIT_PAGE);
+          lrow[x] = ok ? (uint32_t)(((long long)page * sh.Hkv + g) * kPage + (pos % kPage)) : 0u;
+          lmask[x] = ok ? all : (uint16_t)0;
         }
       }
-      // head masks of rows 2tq, 2tq + 1 (j = 0) and 8 + 2tq, 9 + 2tq (j = 1)
-      const uint32_t mk0 = *reinterpret_cast<const uint32_t *>(lmask + x0 + 2 * tq);
-      const uint32_t mk1 = *reinterpret_cast<const uint32_t *>(lmask + x0 + 8 + 2 * tq);
-      const uint32_t mr[4] = {mk0 & 0xFFFFu, mk0 >> 16, mk1 & 0xFFFFu, mk1 >> 16};
-      float p[2][4];
+      const int tiles = (n + kTileRows - 1) / kTileRows;
+      __syncthreads();
+      // pad the last tile with copies of its first row (finite data), masked out
+      for (int x = n + tid; x < tiles * kTileRows; x += kThreads) {
+        lrow[x] = lrow[(tiles - 1) * kTileRows];
+        lmask[x] = 0;
+      }
+      __syncthreads();
+
+      // ---- stream the pass's tiles: warp w takes tiles w, w + kWarps, ... ---
+      const int mt = tiles > warp ? (tiles - warp + kWarps - 1) / kWarps : 0;
+      auto issue = [&](int q) {
+        if (q < mt) {
+          const int x0 = (warp + q * kWarps) * kTileRows;
+          const uint32_t dst = ring_w + (q % kTileRing) * kTileB + c_isv * (kTileRows * kPitch) + c_ch * 16 +
+                               c_sub * kPitch;
+          const unsigned char *src = (c_isv ? vbase : kbase) + c_ch * 16;
 #pragma unroll
-      for (int j = 0; j < 2; ++j)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const uint32_t mm = mr[2 * j + e];
-          p[j][e] = (mm & head_bit0) ? s[j][e] * sc : -INFINITY;
-          p[j][2 + e] = (HI && (mm & head_bit1)) ? s[j][2 + e] * sc : -INFINITY;
+          for (int j = 0; j < kTileRows / RPI; ++j) {
+            const size_t row = lrow[x0 + j * RPI + c_sub];
+            cp_async16(dst + j * RPI * kPitch, src + row * kRowB, 16);
+          }
         }
-      // online softmax per head (head gq: p[.][0..1]; head gq + 8: p[.][2..3])
-      float x0m = fmaxf(fmaxf(p[0][0], p[0][1]), fmaxf(p[1][0], p[1][1]));
-      x0m = fmaxf(x0m, __shfl_xor_sync(kFull, x0m, 1));
-      x0m = fmaxf(x0m, __shfl_xor_sync(kFull, x0m, 2));
-      const float mn0 = fmaxf(m0, x0m);
-      const float mu0 = mn0 == -INFINITY ? 0.f : mn0;
-      const float al0 = exp2f(m0 - mu0);
-      m0 = mn0;
-      float al1 = 1.f;
-      if (HI) {
-        float x1m = fmaxf(fmaxf(p[0][2], p[0][3]), fmaxf(p[1][2], p[1][3]));
-        x1m = fmaxf(x1m, __shfl_xor_sync(kFull, x1m, 1));
-        x1m = fmaxf(x1m, __shfl_xor_sync(kFull, x1m, 2));
-        const float mn1 = fmaxf(m1, x1m);
-        const float mu1 = mn1 == -INFINITY ? 0.f : mn1;
-        al1 = exp2f(m1 - mu1);
-        m1 = mn1;
+        cp_async_commit();
+      };
+#pragma unroll
+      for (int q = 0; q < kTileRing; ++q) issue(q);
+
+      for (int q = 0; q < mt; ++q) {
+        cp_async_wait<kTileRing - 1>();
+        __syncwarp();
+        const uint32_t kt = ring_w + (q % kTileRing) * kTileB;
+        const int x0 = (warp + q * kWarps) * kTileRows;
+        // S = Q K^T: n-tile j holds rows 8j .. 8j + 7 of the tile
+        float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int k = 0; k < KS; ++k) {
+          uint32_t kb[4];
+          ldsm_x4(kb, kt + k_lane + k * 32);
+          if constexpr (HI) {
+            mma_bf16(s[0], qa[k][0], qa[k][1], qa[k][2], qa[k][3], kb[0], kb[1]);
+            mma_bf16(s[1], qa[k][0], qa[k][1], qa[k][2], qa[k][3], kb[2], kb[3]);
+          } else {
+            float u0[2] = {s[0][0], s[0][1]}, u1[2] = {s[1][0], s[1][1]};
+            mma_bf16_top(u0, qa[k][0], qa[k][2], kb[0], kb[1], zu, zf);
+            mma_bf16_top(u1, qa[k][0], qa[k][2], kb[2], kb[3], zu, zf);
+            s[0][0] = u0[0]; s[0][1] = u0[1]; s[1][0] = u1[0]; s[1][1] = u1[1];
+          }
+        }
+        // head masks of rows 2tq, 2tq + 1 (j = 0) and 8 + 2tq, 9 + 2tq (j = 1)
+        const uint32_t mk0 = *reinterpret_cast<const uint32_t *>(lmask + x0 + 2 * tq);
+        const uint32_t mk1 = *reinterpret_cast<const uint32_t *>(lmask + x0 + 8 + 2 * tq);
+        const uint32_t mr[4] = {mk0 & 0xFFFFu, mk0 >> 16, mk1 & 0xFFFFu, mk1 >> 16};
+        float p[2][4];
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const uint32_t mm = mr[2 * j + e];
+            p[j][e] = (mm & head_bit0) ? s[j][e] * sc : -INFINITY;
+            p[j][2 + e] = (HI && (mm & head_bit1)) ? s[j][2 + e] * sc : -INFINITY;
+          }
+        // online softmax per head (head gq: p[.][0..1]; head gq + 8: p[.][2..3])
+        float x0m = fmaxf(fmaxf(p[0][0], p[0][1]), fmaxf(p[1][0], p[1][1]));
+        x0m = fmaxf(x0m, __shfl_xor_sync(kFull, x0m, 1));
+        x0m = fmaxf(x0m, __shfl_xor_sync(kFull, x0m, 2));
+        const float mn0 = fmaxf(m0, x0m);
+        const float mu0 = mn0 == -INFINITY ? 0.f : mn0;
+        const float al0 = mn0 == m0 ? 1.f : exp2f(m0 - mu0);
+        m0 = mn0;
+        float al1 = 1.f;
+        if (HI) {
+          float x1m = fmaxf(fmaxf(p[0][2], p[0][3]), fmaxf(p[1][2], p[1][3]));
+          x1m = fmaxf(x1m, __shfl_xor_sync(kFull, x1m, 1));
+          x1m = fmaxf(x1m, __shfl_xor_sync(kFull, x1m, 2));
+          const float mn1 = fmaxf(m1, x1m);
+          const float mu1 = mn1 == -INFINITY ? 0.f : mn1;
+          al1 = mn1 == m1 ? 1.f : exp2f(m1 - mu1);
+          m1 = mn1;
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            p[j][2] = exp2f(p[j][2] - mu1);
+            p[j][3] = exp2f(p[j][3] - mu1);
+          }
+          l1 = fmaf(l1, al1, (p[0][2] + p[0][3]) + (p[1][2] + p[1][3]));
+        } else {
+#pragma unroll
+          for (int j = 0; j < 2; ++j) p[j][2] = p[j][3] = 0.f;
+        }
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
-          p[j][2] = exp2f(p[j][2] - mu1);
-          p[j][3] = exp2f(p[j][3] - mu1);
+          p[j][0] = exp2f(p[j][0] - mu0);
+          p[j][1] = exp2f(p[j][1] - mu0);
         }
-        l1 = fmaf(l1, al1, (p[0][2] + p[0][3]) + (p[1][2] + p[1][3]));
+        l0 = fmaf(l0, al0, (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]));
+        if (__any_sync(kFull, al0 != 1.f || al1 != 1.f)) {
+#pragma unroll
+          for (int nn = 0; nn < NT; ++nn) {
+            o[nn][0] *= al0;
+            o[nn][1] *= al0;
+            o[nn][2] *= al1;
+            o[nn][3] *= al1;
+          }
+        }
+        // P as the A operand (heads x 16 rows), hi + lo
+        uint32_t ph[4], pl[4];
+        split_bf16(p[0][0], p[0][1], ph[0], pl[0]);  // head gq,     rows 2tq, 2tq+1
+        split_bf16(p[0][2], p[0][3], ph[1], pl[1]);  // head gq + 8, rows 2tq, 2tq+1
+        split_bf16(p[1][0], p[1][1], ph[2], pl[2]);  // head gq,     rows 8+2tq, 9+2tq
+        split_bf16(p[1][2], p[1][3], ph[3], pl[3]);  // head gq + 8, rows 8+2tq, 9+2tq
+#pragma unroll
+        for (int nn = 0; nn < NT; nn += 2) {
+          uint32_t vb[4];
+          ldsm_x4_t(vb, kt + v_lane + nn * 16);
+          if constexpr (HI) {
+            mma_bf16(o[nn], ph[0], ph[1], ph[2], ph[3], vb[0], vb[1]);
+            mma_bf16(o[nn], pl[0], pl[1], pl[2], pl[3], vb[0], vb[1]);
+            mma_bf16(o[nn + 1], ph[0], ph[1], ph[2], ph[3], vb[2], vb[3]);
+            mma_bf16(o[nn + 1], pl[0], pl[1], pl[2], pl[3], vb[2], vb[3]);
+          } else {
+            float u0[2] = {o[nn][0], o[nn][1]}, u1[2] = {o[nn + 1][0], o[nn + 1][1]};
+            mma_bf16_top(u0, ph[0], ph[2], vb[0], vb[1], zu, zf);
+            mma_bf16_top(u0, pl[0], pl[2], vb[0], vb[1], zu, zf);
+            mma_bf16_top(u1, ph[0], ph[2], vb[2], vb[3], zu, zf);
+            mma_bf16_top(u1, pl[0], pl[2], vb[2], vb[3], zu, zf);
+            o[nn][0] = u0[0]; o[nn][1] = u0[1]; o[nn + 1][0] = u1[0]; o[nn + 1][1] = u1[1];
+          }
+        }
+        __syncwarp();
+        issue(q + kTileRing);
+      }
+      cp_async_wait<0>();
+    }
+    // per-lane partial sums of l -> per head
+    l0 += __shfl_xor_sync(kFull, l0, 1);
+    l0 += __shfl_xor_sync(kFull, l0, 2);
+    l1 += __shfl_xor_sync(kFull, l1, 1);
+    l1 += __shfl_xor_sync(kFull, l1, 2);
+
+    // ---- merge the warps of the CTA ------------------------------------------
+    __syncthreads();                                   // ring and lists no longer read
+    float *cm = reinterpret_cast<float *>(dyn);                  // [kWarps][16]
+    float *cl = cm + kWarps * 16;                                // [kWarps][16]
+    float *cacc = cl + kWarps * 16;                              // [kWarps][GR][D]
+    if (tq == 0) {
+      cm[warp * 16 + gq] = m0;
+      cl[warp * 16 + gq] = l0;
+      cm[warp * 16 + gq + 8] = m1;
+      cl[warp * 16 + gq + 8] = l1;
+    }
+#pragma unroll
+    for (int nn = 0; nn < NT; ++nn) {
+      const int cc = nn * 8 + 2 * tq;
+      if (gq < GR) {
+        cacc[(warp * GR + gq) * D + cc] = o[nn][0];
+        cacc[(warp * GR + gq) * D + cc + 1] = o[nn][1];
+      }
+      if (HI && gq + 8 < GR) {
+        cacc[(warp * GR + gq + 8) * D + cc] = o[nn][2];
+        cacc[(warp * GR + gq + 8) * D + cc + 1] = o[nn][3];
+      }
+    }
+    __syncthreads();
+    const bool alone = first == last;                  // the whole item is in this CTA
+    float *part = ws.partials + ((c + item) * GR) * (long long)(D + 2);
+    for (int x = tid; x < nh * (D + 2); x += kThreads) {
+      const int i = x / (D + 2), cc = x % (D + 2);
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, cm[w * 16 + i]);
+      if (alone) {
+        if (cc < 2) continue;
+        float num = 0.0f, den = 0.0f;
+        if (M > -INFINITY) {
+#pragma unroll
+          for (int w = 0; w < kWarps; ++w) {
+            const float f = exp2f(cm[w * 16 + i] - M);
+            den = fmaf(f, cl[w * 16 + i], den);
+            num = fmaf(f, cacc[(w * GR + i) * D + (cc - 2)], num);
+          }
+        }
+        a.out[((long long)b * sh.Hq + S.grp.q_head[i]) * D + (cc - 2)] = den > 0.0f ? num / den : 0.0f;
+        continue;
+      }
+      float v;
+      if (cc == 0) {
+        v = M;
       } else {
+        v = 0.0f;
+        if (M > -INFINITY) {
 #pragma unroll
-        for (int j = 0; j < 2; ++j) p[j][2] = p[j][3] = 0.f;
-      }
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        p[j][0] = exp2f(p[j][0] - mu0);
-        p[j][1] = exp2f(p[j][1] - mu0);
-      }
-      l0 = fmaf(l0, al0, (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]));
-      if (__any_sync(kFull, al0 != 1.f || al1 != 1.f)) {
-#pragma unroll
-        for (int nn = 0; nn < NT; ++nn) {
-          o[nn][0] *= al0;
-          o[nn][1] *= al0;
-          o[nn][2] *= al1;
-          o[nn][3] *= al1;
+          for (int w = 0; w < kWarps; ++w) {
+            const float f = exp2f(cm[w * 16 + i] - M);
+            v += f * (cc == 1 ? cl[w * 16 + i] : cacc[(w * GR + i) * D + (cc - 2)]);
+          }
         }
       }
-      // P as the A operand (heads x 16 rows), hi + lo
-      uint32_t ph[4], pl[4];
-      split_bf16(p[0][0], p[0][1], ph[0], pl[0]);    // head gq,     rows 2tq, 2tq+1
-      split_bf16(p[0][2], p[0][3], ph[1], pl[1]);    // head gq + 8, rows 2tq, 2tq+1
-      split_bf16(p[1][0], p[1][1], ph[2], pl[2]);    // head gq,     rows 8+2tq, 9+2tq
-      split_bf16(p[1][2], p[1][3], ph[3], pl[3]);    // head gq + 8, rows 8+2tq, 9+2tq
-#pragma unroll
-      for (int nn = 0; nn < NT; nn += 2) {
-        uint32_t vb[4];
-        ldsm_x4_t(vb, vt + swz(v_row, nn + v_chk));
-        if constexpr (HI) {
-          mma_bf16(o[nn], ph[0], ph[1], ph[2], ph[3], vb[0], vb[1]);
-          mma_bf16(o[nn], pl[0], pl[1], pl[2], pl[3], vb[0], vb[1]);
-          mma_bf16(o[nn + 1], ph[0], ph[1], ph[2], ph[3], vb[2], vb[3]);
-          mma_bf16(o[nn + 1], pl[0], pl[1], pl[2], pl[3], vb[2], vb[3]);
-        } else {
-          float u0[2] = {o[nn][0], o[nn][1]}, u1[2] = {o[nn + 1][0], o[nn + 1][1]};
-          mma_bf16_top(u0, ph[0], ph[2], vb[0], vb[1]);
-          mma_bf16_top(u0, pl[0], pl[2], vb[0], vb[1]);
-          mma_bf16_top(u1, ph[0], ph[2], vb[2], vb[3]);
-          mma_bf16_top(u1, pl[0], pl[2], vb[2], vb[3]);
-          o[nn][0] = u0[0]; o[nn][1] = u0[1]; o[nn + 1][0] = u1[0]; o[nn + 1][1] = u1[1];
-        }
-      }
-      __syncwarp();
-      issue(t + kTileRing);
+      part[i * (D + 2) + cc] = v;
     }
-    cp_async_wait<0>();
-  }
-  // per-lane partial sums of l -> per head
-  l0 += __shfl_xor_sync(kFull, l0, 1);
-  l0 += __shfl_xor_sync(kFull, l0, 2);
-  l1 += __shfl_xor_sync(kFull, l1, 1);
-  l1 += __shfl_xor_sync(kFull, l1, 2);
-
-  // ---- merge the warps of the CTA, write the partial -----------------------
-  __syncthreads();                                   // ring and lists no longer read
-  float *cm = reinterpret_cast<float *>(dyn);                    // [kWarps][16]
-  float *cl = cm + kWarps * 16;                                  // [kWarps][16]
-  float *cacc = cl + kWarps * 16;                                // [kWarps][GR][D]
-  if (tq == 0) {
-    cm[warp * 16 + gq] = m0;
-    cl[warp * 16 + gq] = l0;
-    cm[warp * 16 + gq + 8] = m1;
-    cl[warp * 16 + gq + 8] = l1;
-  }
-#pragma unroll
-  for (int nn = 0; nn < NT; ++nn) {
-    const int c = nn * 8 + 2 * tq;
-    if (gq < GR) {
-      cacc[(warp * GR + gq) * D + c] = o[nn][0];
-      cacc[(warp * GR + gq) * D + c + 1] = o[nn][1];
-    }
-    if (HI && gq + 8 < GR) {
-      cacc[(warp * GR + gq + 8) * D + c] = o[nn][2];
-      cacc[(warp * GR + gq + 8) * D + c + 1] = o[nn][3];
-    }
-  }
-  __syncthreads();
-  const int role = is_ret ? 0 : 1;
-  for (int x = tid; x < nh * (D + 2); x += kThreads) {
-    const int i = x / (D + 2), c = x % (D + 2);
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, cm[w * 16 + i]);
-    float v;
-    if (c == 0) {
-      v = M;
-    } else {
-      v = 0.0f;
-      if (M > -INFINITY) {
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
-          const float f = exp2f(cm[w * 16 + i] - M);
-          v += f * (c == 1 ? cl[w * 16 + i] : cacc[(w * GR + i) * D + (c - 2)]);
+    if (!alone) {
+      __threadfence();
+      __syncthreads();
+      if (tid == 0) S.last = (atomicAdd(ws.tickets + item, 1u) == (unsigned)(last - first));
+      __syncthreads();
+      if (S.last) {
+        __threadfence();
+        // the last segment of the item: merge partial slots first + item .. last + item
+        for (int x = tid; x < nh * D; x += kThreads) {
+          const int i = x / D, cc = x % D;
+          float M = -INFINITY;
+          for (long long s = first; s <= last; ++s)
+            M = fmaxf(M, __ldcg(ws.partials + ((s + item) * GR + i) * (long long)(D + 2)));
+          float num = 0.0f, den = 0.0f;
+          if (M > -INFINITY) {
+            for (long long s = first; s <= last; ++s) {
+              const float *pp = ws.partials + ((s + item) * GR + i) * (long long)(D + 2);
+              const float ms = __ldcg(pp);
+              if (ms == -INFINITY) continue;
+              const float f = exp2f(ms - M);
+              den = fmaf(f, __ldcg(pp + 1), den);
+              num = fmaf(f, __ldcg(pp + 2 + cc), num);
+            }
+          }
+          a.out[((long long)b * sh.Hq + S.grp.q_head[i]) * D + cc] = den > 0.0f ? num / den : 0.0f;
         }
       }
     }
-    const long long h = S.grp.q_head[i];
-    ws.partials[(((long long)b * sh.Hq + h) * ap.c_max + chunk) * (D + 2) + c] = v;
+    t = seg_end;
+    if (tid == 0) S.item = item + 1;
   }
-  __threadfence();
-  __syncthreads();
-  unsigned *ticket = ws.tickets + ((long long)b * sh.Hkv + g) * 2 + role;
-  if (tid == 0) S.last = (atomicAdd(ticket, 1u) == (unsigned)(nc - 1));
-  __syncthreads();
-  if (!S.last) return;
-  __threadfence();
-
-  // ---- last CTA of the item: merge all chunks into out ----------------------
-  for (int x = tid; x < nh * D; x += kThreads) {
-    const int i = x / D, c = x % D;
-    const long long h = S.grp.q_head[i];
-    const float *pp = ws.partials + ((long long)b * sh.Hq + h) * ap.c_max * (D + 2);
-    float M = -INFINITY;
-    for (int s = 0; s < nc; ++s) M = fmaxf(M, __ldcg(pp + (long long)s * (D + 2)));
-    float num = 0.0f, den = 0.0f;
-    if (M > -INFINITY) {
-      for (int s = 0; s < nc; ++s) {
-        const float ms = __ldcg(pp + (long long)s * (D + 2));
-        if (ms == -INFINITY) continue;
-        const float f = exp2f(ms - M);
-        den = fmaf(f, __ldcg(pp + (long long)s * (D + 2) + 1), den);
-        num = fmaf(f, __ldcg(pp + (long long)s * (D + 2) + 2 + c), num);
-      }
-    }
-    a.out[((long long)b * sh.Hq + h) * D + c] = den > 0.0f ? num / den : 0.0f;
-  }
-  if (tid == 0) atomicExch(ticket, 0u);
 }
 
 // ==================================================================== host
@@ -632,39 +760,33 @@ int pow2_ceil(long long x) {
 
 int group_rows_att(const Tables &tb) { return pow2_ceil(std::max(1, std::max(tb.max_ret, tb.max_loc))); }
 
-// bound: most union rows one retrieval item can hold in this call
-AttParams att_params(const Shape &sh, const Tables &tb, long long window, long long sinks, long long bound) {
+AttParams att_params(const Shape &sh, const Tables &tb, int batch) {
   AttParams p{};
   const long long L = sh.max_len;
   p.span = (int)std::max(256LL, std::min<long long>(kSpanMax, pow2_ceil((L + 15) / 16)));
   p.ns = (int)((L + p.span - 1) / p.span);
-  p.c_r = (int)std::max(1LL, std::min<long long>(kChunksRet, (std::min(bound, L) + kRowsPerChunk - 1) / kRowsPerChunk));
-  p.c_l = 0;
-  if (tb.n_loc > 0) {
-    const long long rows = std::min<long long>(L, window + sinks);
-    p.c_l = (int)std::max(1LL, (rows + kSpanLoc - 1) / kSpanLoc);
-  }
-  // partial slots: the largest chunk count any call can use
-  p.c_max = (int)std::max<long long>(kChunksRet, (L + kSpanLoc - 1) / kSpanLoc);
+  p.n_ret_items = batch * tb.n_ret;
+  p.ni = batch * (tb.n_ret + tb.n_loc);
   return p;
 }
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct AttLayout {
-  size_t partials, plan_row, plan_mask, plan_cnt, tickets, total;
+  size_t partials, plan_row, plan_mask, plan_cnt, tstart, counters, total;
 };
 
 AttLayout att_layout(const Shape &sh, const Tables &tb, int batch) {
-  const AttParams p = att_params(sh, tb, 0, 0, sh.max_len);
+  const AttParams p = att_params(sh, tb, batch);
   AttLayout L{};
   const size_t entries = (size_t)batch * tb.n_ret * p.ns * p.span;
   size_t o = 0;
-  L.partials = o;  o = align256(o + (size_t)batch * sh.Hq * p.c_max * (sh.d + 2) * sizeof(float));
+  L.partials = o;  o = align256(o + (size_t)(kMaxGrid + p.ni) * group_rows_att(tb) * (sh.d + 2) * sizeof(float));
   L.plan_row = o;  o = align256(o + entries * 4);
   L.plan_mask = o; o = align256(o + entries * 2);
   L.plan_cnt = o;  o = align256(o + (size_t)batch * tb.n_ret * p.ns * 4);
-  L.tickets = o;   o = align256(o + (size_t)batch * sh.Hkv * 2 * sizeof(unsigned));
+  L.tstart = o;    o = align256(o + (size_t)(p.ni + 1) * 8);
+  L.counters = o;  o = align256(o + ((size_t)p.ni * 2 + 1) * 4);     // item_rows, tickets, plan ticket
   L.total = o;
   return L;
 }
@@ -684,68 +806,51 @@ cudaError_t set_smem(K kern, size_t bytes) {
   return e;
 }
 
-// Chunks per retrieval item, at most c_hi.  Chunks are equal shares of an
-// item's rows, so CTAs finish in waves: pick the count whose last wave is
-// fullest, preferring more chunks when the difference is small.
+// resident CTAs of a kernel on this device (cached)
 template <typename K>
-int pick_chunks(K kern, size_t smem, long long items, int c_hi, long long other_blocks) {
+int resident_ctas(K kern, int threads, size_t smem) {
   static std::mutex mu;
-  static std::map<std::pair<const void *, int>, int> slots_of;
-  if (items <= 0 || c_hi <= 1) return std::max(1, c_hi);
+  static std::map<std::pair<const void *, int>, int> cache;
   int dev = 0;
   cudaGetDevice(&dev);
-  int slots = 0;
-  {
-    std::lock_guard<std::mutex> lk(mu);
-    const auto key = std::make_pair((const void *)kern, dev);
-    auto it = slots_of.find(key);
-    if (it == slots_of.end()) {
-      int occ = 0, sms = 0;
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, smem) != cudaSuccess ||
-          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
-        cudaGetLastError();
-        occ = sms = 0;
-      }
-      it = slots_of.emplace(key, occ * sms).first;
-    }
-    slots = it->second;
+  std::lock_guard<std::mutex> lk(mu);
+  const auto key = std::make_pair((const void *)kern, dev);
+  auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  int occ = 0, sms = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, threads, smem) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;                                        // not cached: retried next call
   }
-  if (slots <= 0) return c_hi;
-  auto eff = [&](int c) {
-    const double w = (double)(items * c + other_blocks) / slots;
-    return w / std::ceil(w);
-  };
-  double best = 0.0;
-  for (int c = 1; c <= c_hi; ++c) best = std::max(best, eff(c));
-  int pick = 1;
-  for (int c = 1; c <= c_hi; ++c)
-    if (eff(c) >= best - 0.03) pick = c;
-  return pick;
+  const int n = std::max(1, std::min(kMaxGrid, occ * sms));
+  cache.emplace(key, n);
+  return n;
 }
 
 template <int D, int GR>
 cudaError_t launch_t(const AttendArgs &a, const Shape &sh, const Tables &tb, const AttParams &p, const AttWs &ws,
                      cudaStream_t st) {
+  cudaError_t e;
   if (tb.n_ret > 0) {
     const size_t pbytes = (size_t)GR * (p.span / 32) * 4 + (size_t)(p.span / kPage) * 4;
-    cudaError_t e = set_smem(attend_plan_kernel<GR>, pbytes);
+    e = set_smem(attend_plan_kernel<D, GR>, pbytes);
     if (e != cudaSuccess) return e;
-    attend_plan_kernel<GR><<<dim3(p.ns, tb.n_ret, a.batch), kPlanThreads, pbytes, st>>>(a, sh, tb, p, ws);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    attend_plan_kernel<D, GR><<<dim3(p.ns, tb.n_ret, a.batch), kPlanThreads, pbytes, st>>>(a, sh, tb, p, ws);
+  } else {
+    attend_prefix_kernel<D><<<1, 256, 0, st>>>(a, sh, tb, p, ws);
   }
-  const size_t ring = (size_t)kWarps * kTileRing * (2 * kTileRows * 2 * D);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t ring = (size_t)kWarps * kTileRing * (2 * kTileRows * (2 * D + 16));
   const size_t lists = (size_t)kPassRows * 4 + (size_t)(kPassRows + kTileRows) * 2 + (size_t)(p.ns + 1) * 4;
   const size_t merge = (size_t)kWarps * 32 * 4 + (size_t)kWarps * GR * D * 4;
   const size_t bytes = std::max(ring + lists, merge);
-  cudaError_t e = set_smem(attend_main_kernel<D, GR>, bytes);
+  e = set_smem(attend_main_kernel<D, GR>, bytes);
   if (e != cudaSuccess) return e;
-  AttParams q = p;
-  q.c_r = pick_chunks(attend_main_kernel<D, GR>, bytes, (long long)a.batch * tb.n_ret, p.c_r,
-                      (long long)a.batch * tb.n_loc * p.c_l);
-  const long long blocks = (long long)a.batch * ((long long)tb.n_ret * q.c_r + (long long)tb.n_loc * q.c_l);
-  if (blocks == 0) return cudaSuccess;
-  attend_main_kernel<D, GR><<<(unsigned)blocks, kThreads, bytes, st>>>(a, sh, tb, q, ws);
+  const int grid = resident_ctas(attend_main_kernel<D, GR>, kThreads, bytes);
+  if (grid <= 0) return cudaErrorInvalidConfiguration;
+  attend_main_kernel<D, GR><<<grid, kThreads, bytes, st>>>(a, sh, tb, p, ws);
   return cudaGetLastError();
 }
 
@@ -770,16 +875,18 @@ size_t attend_workspace_bytes(const Shape &sh, const Tables &tb, int batch) {
 cudaError_t launch_attend(const AttendArgs &a, const Shape &sh, const Tables &tb, cudaStream_t st) {
   if (a.batch == 0) return cudaSuccess;
   const AttLayout L = att_layout(sh, tb, a.batch);
+  const AttParams p = att_params(sh, tb, a.batch);
   char *base = static_cast<char *>(a.ws);
   AttWs ws{};
   ws.partials = reinterpret_cast<float *>(base + L.partials);
   ws.plan_row = reinterpret_cast<uint32_t *>(base + L.plan_row);
   ws.plan_mask = reinterpret_cast<uint16_t *>(base + L.plan_mask);
   ws.plan_cnt = reinterpret_cast<int *>(base + L.plan_cnt);
-  ws.tickets = reinterpret_cast<unsigned *>(base + L.tickets);
-  const long long bound = tb.n_ret > 0 ? (long long)std::max(1, tb.max_ret) * a.sel_stride : 0;
-  const AttParams p = att_params(sh, tb, a.window, a.num_sinks, bound);
-  cudaError_t e = cudaMemsetAsync(ws.tickets, 0, (size_t)a.batch * sh.Hkv * 2 * sizeof(unsigned), st);
+  ws.tstart = reinterpret_cast<long long *>(base + L.tstart);
+  ws.item_rows = reinterpret_cast<int *>(base + L.counters);
+  ws.tickets = reinterpret_cast<unsigned *>(ws.item_rows + p.ni);
+  ws.plan_ticket = ws.tickets + p.ni;
+  cudaError_t e = cudaMemsetAsync(ws.item_rows, 0, ((size_t)p.ni * 2 + 1) * 4, st);
   if (e != cudaSuccess) return e;
   return sh.d == 128 ? dispatch_gr<128>(a, sh, tb, p, ws, st) : dispatch_gr<64>(a, sh, tb, p, ws, st);
 }
