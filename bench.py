@@ -161,16 +161,18 @@ def kernel_source_hash(files):
 
 
 KERNEL_SOURCES = {
-    "select": ["head_wise_sparse_02_b200/csrc/sd_select.cu", "head_wise_sparse_02_b200/csrc/sd_internal.cuh"],
+    "select": ["head_wise_sparse_02_b200/csrc/sd_select.cu", "head_wise_sparse_02_b200/csrc/sd_select_topk.cu",
+               "head_wise_sparse_02_b200/csrc/sd_internal.cuh"],
     "attend": ["head_wise_sparse_02_b200/csrc/sd_attend.cu", "head_wise_sparse_02_b200/csrc/sd_internal.cuh"],
     "index_keys": ["head_wise_sparse_02_b200/csrc/sd_index.cu", "head_wise_sparse_02_b200/csrc/sd_internal.cuh"],
 }
 
 
-def ncu_traffic(kernel: str, workload: str, units: float):
-    """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel source (else None).  The summary stores bytes per unit
-    of work so that a capture on a smaller case scales to this launch."""
+def ncu_traffic(kernel: str, algorithmic_bytes: float):
+    """DRAM bytes per call from a committed ncu summary, if it was taken on
+    the current kernel source (else None).  The summary stores DRAM bytes per
+    algorithmic byte of the captured (smaller) case; both grow with the rows
+    a call processes, so the ratio scales the capture to this call."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(p) as f:
@@ -178,9 +180,17 @@ def ncu_traffic(kernel: str, workload: str, units: float):
         e = d[kernel]
         if e.get("source_hash") != kernel_source_hash(KERNEL_SOURCES[kernel]):
             return None
-        return float(e["dram_bytes_per_unit"]) * units
+        return round(float(e["dram_bytes_per_algorithmic_byte"]) * algorithmic_bytes)
     except Exception:
         return None
+
+
+def kernels_per_step(w) -> int:
+    """Kernels of this library one step launches: index_keys; select (top-k:
+    window, stream, resolve and the exact selector for flagged items; top-p:
+    the exact selector); attend (plan, or the item layout alone, and main)."""
+    n_sel = 0 if not any(w.head_is_retrieval) else (4 if w.mode == "top_k" else 1)
+    return 1 + n_sel + 2
 
 
 def union_rows(sel_idx, sel_count, w):
@@ -348,7 +358,6 @@ def run_ours(args):
     dominant = max(per, key=per.get)
     peak, peak_kind = load_peak()
     achieved = kern_bytes[dominant] / (per[dominant] * 1e-3) / 1e9
-    units = {"select": index_tokens, "attend": rows, "index_keys": B}[dominant]
     step_bytes = index_bytes + kv_bytes
     head_steps = ws * B * Hq
     value = head_steps / (ms_max * 1e-3)
@@ -369,17 +378,18 @@ def run_ours(args):
         "frac_of_8tbs_step": round(step_bytes / (ms * 1e-3) / 1e9 / CONTRACT_GBS, 4),
         "algorithmic_bytes_per_step": step_bytes,
         "ms_per_call": {k: round(v, 4) for k, v in per.items()},
+        "algorithmic_bytes_per_call": kern_bytes,
         "selected_per_head": {"mean": round(float(sel_sizes.mean()), 1), "min": int(sel_sizes.min()),
                               "max": int(sel_sizes.max())},
         "roofline": {"kernel": dominant, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                      "peak_kind": f"{peak_kind} hbm_gbs (copy bandwidth)", "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
                      "algorithmic_bytes_per_launch": kern_bytes[dominant],
-                     "traffic": ncu_traffic(dominant, args.workload, units)},
+                     "traffic": ncu_traffic(dominant, kern_bytes[dominant])},
         "e2e": {"value": round(head_steps / (e2e_ms * 1e-3), 1), "unit": UNIT,
                 "h2d_bytes_per_step": int(q_h.numel() * 2 + qp_h.numel() * 2 + nk_h.numel() * 2 + ns_h.numel() * 4),
                 "d2h_bytes_per_step": int(out_h.numel() * 4)},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": kernels_per_step(w) * args.steps,
         "clocks": clk,
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
