@@ -266,6 +266,46 @@ sd_status sparse_decode_attend(sd_ctx *ctx, const void *q, const void *k_cache, 
   return e == cudaSuccess ? SD_OK : cuda_fail(ctx, e, "attend launch");
 }
 
+sd_status sparse_decode_attend_noalloc(sd_ctx *ctx, const void *q, const void *k_cache, const void *v_cache,
+                                       const int32_t *page_table, const int32_t *seq_lens, int batch,
+                                       const int32_t *sel_idx, const int32_t *sel_count, int sel_stride,
+                                       float *out, sd_stream stream) {
+  if (!ctx) return SD_ERR_INVALID_ARG;
+  if (batch < 0 || batch > ctx->cfg.max_batch) return fail(ctx, SD_ERR_INVALID_ARG, "batch out of range");
+  if (batch == 0) return SD_OK;
+  if (!q || !k_cache || !v_cache || !page_table || !seq_lens || !out)
+    return fail(ctx, SD_ERR_INVALID_ARG, "null pointer");
+  if (ctx->sh.H_ret > 0 && (!sel_idx || !sel_count || sel_stride <= 0))
+    return fail(ctx, SD_ERR_INVALID_ARG, "selection lists required for retrieval heads");
+  const size_t need = sd::attend_workspace_bytes(ctx->sh, ctx->tb, batch);
+  if (need > sd::kNoAllocScratchBytes)
+    return fail(ctx, SD_ERR_WORKSPACE,
+                "attend needs " + std::to_string(need) + " bytes of scratch for this batch; the built-in scratch holds " +
+                    std::to_string(sd::kNoAllocScratchBytes) + " (use sparse_decode_attend with a caller workspace)");
+  DeviceGuard dg(ctx->device);
+  void *scratch = nullptr;
+  cudaError_t e = sd::noalloc_scratch(&scratch);
+  if (e != cudaSuccess) return cuda_fail(ctx, e, "scratch lookup");
+  sd::AttendArgs a{};
+  a.q = static_cast<const uint16_t *>(q);
+  a.k_cache = static_cast<const uint16_t *>(k_cache);
+  a.v_cache = static_cast<const uint16_t *>(v_cache);
+  a.page_table = page_table;
+  a.seq_lens = seq_lens;
+  a.sel_idx = sel_idx;
+  a.sel_count = sel_count;
+  a.sel_stride = sel_stride;
+  a.out = out;
+  a.attn_scale = ctx->attn_scale;
+  a.window = ctx->cfg.window;
+  a.num_sinks = ctx->cfg.num_sinks;
+  a.ws = scratch;
+  a.err = ctx->err_d;
+  a.batch = batch;
+  e = sd::launch_attend(a, ctx->sh, ctx->tb, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SD_OK : cuda_fail(ctx, e, "attend launch");
+}
+
 sd_status sparse_decode_error_word(sd_ctx *ctx, sd_stream stream, uint32_t *word) {
   if (!ctx) return SD_ERR_INVALID_ARG;
   DeviceGuard dg(ctx->device);

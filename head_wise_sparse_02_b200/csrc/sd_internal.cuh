@@ -125,4 +125,9 @@ struct AttendArgs {
 size_t attend_workspace_bytes(const Shape &sh, const Tables &tb, int batch);
 cudaError_t launch_attend(const AttendArgs &a, const Shape &sh, const Tables &tb, cudaStream_t st);
 
+// Size of the built-in attend scratch of sparse_decode_attend_noalloc.
+constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;
+// This device's scratch address (looked up on the first call per device).
+cudaError_t noalloc_scratch(void **ptr);
+
 }  // namespace sd

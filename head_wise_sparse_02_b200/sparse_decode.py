@@ -53,6 +53,7 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sparse_decode_index_keys": (c_int, [P, P, P, c_int, P, P]),
         "sparse_decode_select": (c_int, [P, P, P, P, P, c_int, P, P, c_int, P, c_size_t, P]),
         "sparse_decode_attend": (c_int, [P, P, P, P, P, P, c_int, P, P, c_int, P, P, c_size_t, P]),
+        "sparse_decode_attend_noalloc": (c_int, [P, P, P, P, P, P, c_int, P, P, c_int, P, P]),
         "sparse_decode_error_word": (c_int, [P, P, POINTER(c_uint32)]),
         "sparse_decode_num_retrieval_heads": (c_int, [P]),
         "sparse_decode_last_error": (c_char_p, [P]),
@@ -157,6 +158,18 @@ def sparse_decode_attend(ctx: int, q, k_cache, v_cache, page_table, seq_lens, se
         _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_count, torch.int32, "sel_count"), stride,
         _ptr(out, torch.float32, "out"), _ptr(workspace, torch.uint8, "workspace"),
         int(workspace.numel()), _stream(stream)), ctx)
+
+
+def sparse_decode_attend_noalloc(ctx: int, q, k_cache, v_cache, page_table, seq_lens, sel_idx, sel_count,
+                                 out, stream=None) -> None:
+    """attend on the library's built-in scratch (no workspace argument)."""
+    stride = int(sel_idx.shape[-1]) if sel_idx is not None else 0
+    _check(LIB.sparse_decode_attend_noalloc(
+        ctx, _ptr(q, torch.bfloat16, "q"), _ptr(k_cache, torch.bfloat16, "k_cache"),
+        _ptr(v_cache, torch.bfloat16, "v_cache"), _ptr(page_table, torch.int32, "page_table"),
+        _ptr(seq_lens, torch.int32, "seq_lens"), int(seq_lens.numel()),
+        _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_count, torch.int32, "sel_count"), stride,
+        _ptr(out, torch.float32, "out"), _stream(stream)), ctx)
 
 
 def sparse_decode_error_word(ctx: int, stream=None) -> int:

@@ -254,6 +254,40 @@ SD_API sd_status sparse_decode_attend(sd_ctx *ctx, const void *q, const void *k_
                                void *workspace, size_t ws_bytes, sd_stream stream);
 
 /*
+ * sparse_decode_attend_noalloc -- sparse_decode_attend without a workspace
+ * argument: the call uses a fixed scratch area compiled into the library
+ * (64 MiB per device) and allocates nothing.  An addition of this library;
+ * the pages describe no such call.
+ *
+ * For callers that cannot hand over device memory on the decode path: an
+ * engine whose device memory is all planned before it starts serving, where
+ * an allocation in the middle of a step could synchronise the device or fail
+ * under memory pressure, or a host program without a device allocator of its
+ * own.
+ *
+ * Arguments, layouts and results are those of sparse_decode_attend.
+ *   - Returns SD_ERR_WORKSPACE, with the sizes in sparse_decode_last_error,
+ *     when this batch needs more than the built-in scratch (the amount
+ *     sparse_decode_workspace_size reports for attend grows with the batch,
+ *     the retrieval groups and max_pages_per_seq); nothing is launched then.
+ *   - Nothing in the scratch has to start at zero: the call clears the
+ *     counters it uses, on `stream`, before its kernels run.
+ *   - The scratch is one area per device, shared by every context and stream
+ *     of the process: two of these calls on the same device that are not
+ *     ordered on one stream (other streams, threads or contexts) race and may
+ *     give wrong outputs.  Order them, or use sparse_decode_attend with
+ *     separate workspaces.
+ *   - The first call on a device does a one-time set-up (it looks up the
+ *     scratch address with cudaGetSymbolAddress); make that first call
+ *     outside any stream capture.
+ */
+SD_API sd_status sparse_decode_attend_noalloc(sd_ctx *ctx, const void *q, const void *k_cache,
+                                      const void *v_cache, const int32_t *page_table,
+                                      const int32_t *seq_lens, int batch, const int32_t *sel_idx,
+                                      const int32_t *sel_count, int sel_stride, float *out,
+                                      sd_stream stream);
+
+/*
  * sparse_decode_error_word -- wait for `stream`, copy the device error word
  * into *word (may be NULL) and clear it.  Returns SD_OK when the word was 0,
  * SD_ERR_TIMEOUT when SD_EBIT_TIMEOUT was set, SD_ERR_DEVICE_DATA otherwise.
