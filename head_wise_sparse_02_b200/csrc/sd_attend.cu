@@ -12,22 +12,25 @@
 // union of its heads' selected positions, a local item's rows are
 // [0, sinks) U [N - window, N).  Rows are processed in 16-row tiles.
 //
-// Two launches:
+// Three launches:
 //   plan  one CTA per (b, retrieval group, span of positions).  Finds each
 //         head's sub-list of its ascending selected positions inside the span
 //         (warp-cooperative search), marks them in per-head bitmaps and
 //         compacts the union into an ordered list of (cache row, head mask):
 //         every union row is read once for all the group's heads that
 //         selected it.  The page of each row is resolved here, from a
-//         shared-memory copy of the span's page-table slice.  The last plan
-//         CTA to finish (atomic ticket) lays all items end to end and writes
-//         the first tile of each (a prefix sum over the items' tile counts).
+//         shared-memory copy of the span's page-table slice; the union sizes
+//         are summed per item.
+//   layout one CTA lays all items end to end and writes the first tile of
+//         each (a prefix sum over the items' tile counts).
 //   main  a persistent grid, one CTA per resident slot.  CTA c takes the
 //         equal share [W c / P, W (c + 1) / P) of all W tiles and walks the
 //         items it overlaps (usually one or two), so that its rings run
 //         without the start and drain of a grid of small CTAs.  Four warps
 //         stream tiles through per-warp cp.async rings (whole rows per
-//         instruction, padded row pitch) and run them on the tensor cores in
+//         instruction, padded row pitch; each warp fetches its tiles' rows
+//         from the union lists itself, one tile ahead, so nothing stops the
+//         rings inside an item) and run them on the tensor cores in
 //         the FlashAttention-2 arrangement: S = Q K^T with mma.m16n8k16 (A =
 //         the group's bf16 queries, heads on M; B = K rows by ldmatrix), a
 //         masked online softmax per head in base 2, then O += P V with P taken
@@ -59,7 +62,6 @@ constexpr int kThreads = 128;
 constexpr int kWarps = kThreads / 32;
 constexpr int kTileRows = 16;
 constexpr int kTileRing = 3;            // tiles in flight per warp
-constexpr int kPassRows = 1024;         // list entries staged in shared memory per pass
 constexpr int kMaxGrid = 4096;          // persistent CTAs (partial slots are sized for this)
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, int src_bytes) {
@@ -110,17 +112,27 @@ __device__ __forceinline__ void split_bf16(float x, float y, uint32_t &hi, uint3
   lo = pack_bf16(x - bf16_lo(hi), y - bf16_hi(hi));
 }
 
-// First index i in [0, n) with arr[i] >= x (n if none); whole warp cooperates.
-// Lanes 0..30 probe inside [lo, hi); lane 31 always lands at or past hi and
-// acts as the sentinel, so some lane is always true.
+// First index i in [0, n) with arr[i] >= x (n if none), arr ascending; the
+// whole warp cooperates.  While the bracket is wider than 31, each lane
+// probes 4 of 128 evenly spaced points, the last of which lies at or past hi
+// (one dependent round narrows the bracket ~127-fold); then lane j probes
+// lo + j, and lane 31 lands at or past hi.  Either way some lane is true.
 template <typename T>
 __device__ int warp_lower_bound(const T *arr, int n, T x, int lane) {
   int lo = 0, hi = n;                      // answer in [lo, hi]
   while (hi - lo > 31) {
-    const int step = (hi - lo + 30) / 31;  // 31 * step >= hi - lo
-    const int p = lo + lane * step;
-    const bool ge = (p < hi) ? (__ldcg(arr + p) >= x) : true;
-    const int first = __ffs(__ballot_sync(kFull, ge)) - 1;
+    const int step = (hi - lo + 126) / 127;  // 127 * step >= hi - lo: probe 127 is past hi
+    bool ge[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int p = lo + (lane * 4 + j) * step;
+      ge[j] = (p < hi) ? (__ldcg(arr + p) >= x) : true;
+    }
+    const int jf = ge[0] ? 0 : (ge[1] ? 1 : (ge[2] ? 2 : (ge[3] ? 3 : 4)));
+    const unsigned bal = __ballot_sync(kFull, jf < 4);
+    // probe k = 4 l + j is at lo + k step; probe 127 (lane 31) is always true
+    const int l = __ffs(bal) - 1;
+    const int first = l * 4 + __shfl_sync(kFull, jf, l);
     const int nhi = std::min(hi, lo + first * step);
     const int nlo = first == 0 ? lo : lo + (first - 1) * step + 1;
     lo = nlo;
@@ -147,7 +159,6 @@ struct AttWs {
   long long *tstart;        // [ni + 1]: first tile of each item; tstart[ni] = all tiles
   int *item_rows;           // [ni]: rows of each item           } zeroed before
   unsigned *tickets;        // [ni]: partials merged per item     } every call
-  unsigned *plan_ticket;    // [1]: plan CTAs finished            }
 };
 
 __device__ __forceinline__ const Group &item_group(const Tables &tb, const AttParams &ap, int i, int &b,
@@ -223,9 +234,10 @@ __device__ void item_prefix(const AttendArgs &a, const Shape &sh, const Tables &
   if (tid == 0) ws.tstart[ap.ni] = carry;
 }
 
-// The item layout alone, when there is no retrieval item to plan.
+// The item layout, one CTA, after the plan (when there is one) has summed the
+// retrieval items' rows.
 template <int D>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(1024)
 attend_prefix_kernel(const AttendArgs a, const Shape sh, const Tables tb, const AttParams ap, const AttWs ws) {
   item_prefix<D>(a, sh, tb, ap, ws);
 }
@@ -237,7 +249,7 @@ attend_prefix_kernel(const AttendArgs a, const Shape sh, const Tables tb, const 
 template <int GR>
 __device__ void plan_span(const AttendArgs &a, const Shape &sh, const Tables &tb, const AttParams &ap,
                           const AttWs &ws, const Group &grp, int b, int gi, int split, uint32_t *hbm, int *pslice) {
-  __shared__ int seg_lo[kMaxGroup], seg_hi[kMaxGroup];
+  __shared__ int seg_lo[kMaxGroup], seg_hi[kMaxGroup], seg_at[kMaxGroup + 1];
   __shared__ uint32_t wtot[kPlanWarps];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nh = grp.n, g = grp.kv_head;
@@ -273,17 +285,27 @@ __device__ void plan_span(const AttendArgs &a, const Shape &sh, const Tables &tb
     }
   }
   __syncthreads();
-  for (int i = 0; i < nh; ++i) {
-    const int32_t *sel = a.sel_idx + ((long long)b * sh.H_ret + grp.row[i]) * a.sel_stride;
-    for (int e = seg_lo[i] + tid; e < seg_hi[i]; e += kPlanThreads) {
-      const long long pos = sel[e];
-      if (pos < p0 || pos >= p1) {                  // not ascending
-        raise_error(a.err, SD_EBIT_SEL);
-        continue;
-      }
-      const int off = (int)(pos - p0);
-      atomicOr(&hbm[i * bwords + (off >> 5)], 1u << (off & 31));
+  if (tid == 0) {                                    // where each head's entries start in one flat range
+    int run = 0;
+    for (int i = 0; i < nh; ++i) {
+      seg_at[i] = run;
+      run += seg_hi[i] - seg_lo[i];
     }
+    seg_at[nh] = run;
+  }
+  __syncthreads();
+  // all heads' entries of the span in one flat loop, so that their loads overlap
+#pragma unroll 4
+  for (int x = tid; x < seg_at[nh]; x += kPlanThreads) {
+    int i = 0;
+    while (seg_at[i + 1] <= x) ++i;
+    const long long pos = a.sel_idx[((long long)b * sh.H_ret + grp.row[i]) * a.sel_stride + seg_lo[i] + (x - seg_at[i])];
+    if (pos < p0 || pos >= p1) {                    // not ascending
+      raise_error(a.err, SD_EBIT_SEL);
+      continue;
+    }
+    const int off = (int)(pos - p0);
+    atomicOr(&hbm[i * bwords + (off >> 5)], 1u << (off & 31));
   }
   __syncthreads();
   // ordered compaction of the union: contiguous word ranges per thread
@@ -340,20 +362,10 @@ attend_plan_kernel(const AttendArgs a, const Shape sh, const Tables tb, const At
   const int tid = threadIdx.x;
   const int split = blockIdx.x, gi = blockIdx.y, b = blockIdx.z;
   __shared__ Group grp;
-  __shared__ int last;
   extern __shared__ uint32_t plan_dyn[];
   if (tid == 0) grp = tb.ret[gi];
   __syncthreads();
   plan_span<GR>(a, sh, tb, ap, ws, grp, b, gi, split, plan_dyn, reinterpret_cast<int *>(plan_dyn + GR * (ap.span / 32)));
-  // the last plan CTA to finish lays out the items
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) last = atomicAdd(ws.plan_ticket, 1u) == gridDim.x * gridDim.y * gridDim.z - 1;
-  __syncthreads();
-  if (!last) return;
-  __threadfence();
-  item_prefix<D>(a, sh, tb, ap, ws);
-  if (tid == 0) *ws.plan_ticket = 0u;
 }
 
 // ============================================================== main kernel
@@ -366,9 +378,8 @@ struct MainShared {
 // dynamic shared memory: [ring: kWarps x kTileRing x (16 K rows + 16 V rows),
 //                         rows padded to 2d + 16 bytes: ldmatrix phases hit
 //                         distinct banks and every offset is a constant]
-//                        [pass list: kPassRows x uint32 cache row]
-//                        [kPassRows + 16 x uint16 head mask]
-//                        [span prefix: ns + 1 ints]
+//                        [head masks of the tiles in the rings: kWarps x kTileRing x 16 x uint16]
+//                        [span prefix of the current item: ns + 1 ints]
 // between items the ring holds the warps' (m, l, acc) for the CTA merge
 template <int D, int GR>
 __global__ void __launch_bounds__(kThreads)
@@ -385,9 +396,9 @@ attend_main_kernel(const AttendArgs a, const Shape sh, const Tables tb, const At
   __shared__ MainShared S;
   extern __shared__ __align__(128) unsigned char dyn[];
   const uint32_t ring0 = (uint32_t)__cvta_generic_to_shared(dyn);
-  uint32_t *lrow = reinterpret_cast<uint32_t *>(dyn + (size_t)kWarps * kTileRing * kTileB);
-  uint16_t *lmask = reinterpret_cast<uint16_t *>(lrow + kPassRows);
-  int *pre = reinterpret_cast<int *>(lmask + kPassRows + kTileRows);
+  uint16_t *wmask = reinterpret_cast<uint16_t *>(dyn + (size_t)kWarps * kTileRing * kTileB) +
+                    warp * (kTileRing * kTileRows);                       // this warp's tile masks
+  int *pre = reinterpret_cast<int *>(dyn + (size_t)kWarps * kTileRing * kTileB + kWarps * kTileRing * kTileRows * 2);
 
   // ---- this CTA's share of the tiles -----------------------------------------
   const long long W = __ldcg(ws.tstart + ap.ni);
@@ -488,14 +499,22 @@ attend_main_kernel(const AttendArgs a, const Shape sh, const Tables tb, const At
 #pragma unroll
     for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
 
-    for (long long ps = r0; ps < r1; ps += kPassRows) {
-      const int n = (int)std::min<long long>(kPassRows, r1 - ps);
-      __syncthreads();                                 // the previous pass no longer reads the list
-      // ---- stage the pass's list entries -----------------------------------
-      if (is_ret) {
-#pragma unroll 4
-        for (int x = tid; x < n; x += kThreads) {
-          const long long gx = ps + x;
+    // ---- stream the segment's tiles: warp w takes tiles w, w + kWarps, ... -----
+    // Lane r < 16 fetches the cache row and head mask of row r of a tile one
+    // tile ahead of its copy (registers), so the rings run across the whole
+    // segment without staging the list in shared memory.
+    const long long rows = r1 - r0;
+    const int tiles = (int)((rows + kTileRows - 1) / kTileRows);
+    const int mt = tiles > warp ? (tiles - warp + kWarps - 1) / kWarps : 0;
+    const uint16_t all = (uint16_t)((1u << nh) - 1u);
+    const int32_t *pt = a.page_table + (long long)b * sh.max_pages;
+    auto fetch = [&](int q, uint32_t &row, uint32_t &mask) {
+      row = 0u;
+      mask = 0u;
+      if (q >= mt) return;
+      const long long gx = r0 + (long long)(warp + q * kWarps) * kTileRows + (lane & 15);
+      if (gx < r1) {
+        if (is_ret) {
           int lo = 0, hi = ns_item;                    // last span s with pre[s] <= gx
           while (hi - lo > 1) {
             const int mid = (lo + hi) >> 1;
@@ -503,55 +522,50 @@ attend_main_kernel(const AttendArgs a, const Shape sh, const Tables tb, const At
             else hi = mid;
           }
           const long long e = (slot0 + lo) * ap.span + (gx - pre[lo]);
-          lrow[x] = __ldcg(ws.plan_row + e);
-          lmask[x] = __ldcg(ws.plan_mask + e);
-        }
-      } else {
-        const int32_t *pt = a.page_table + (long long)b * sh.max_pages;
-        const uint16_t all = (uint16_t)((1u << nh) - 1u);
-        for (int x = tid; x < n; x += kThreads) {
-          const long long rr = ps + x;
-          const long long pos = rr < loc_a ? rr : loc_w + (rr - loc_a);
+          row = __ldcg(ws.plan_row + e);
+          mask = __ldcg(ws.plan_mask + e);
+        } else {
+          const long long pos = gx < loc_a ? gx : loc_w + (gx - loc_a);
           const int page = pt[pos / kPage];
           const bool ok = page >= 0 && page < sh.num_pages;
           if (!ok) raise_error(a.err, SD_EBIT_PAGE);
-          lrow[x] = ok ? (uint32_t)(((long long)page * sh.Hkv + g) * kPage + (pos % kPage)) : 0u;
-          lmask[x] = ok ? all : (uint16_t)0;
+          row = ok ? (uint32_t)(((long long)page * sh.Hkv + g) * kPage + (pos % kPage)) : 0u;
+          mask = ok ? all : 0u;
         }
       }
-      const int tiles = (n + kTileRows - 1) / kTileRows;
-      __syncthreads();
-      // pad the last tile with copies of its first row (finite data), masked out
-      for (int x = n + tid; x < tiles * kTileRows; x += kThreads) {
-        lrow[x] = lrow[(tiles - 1) * kTileRows];
-        lmask[x] = 0;
-      }
-      __syncthreads();
-
-      // ---- stream the pass's tiles: warp w takes tiles w, w + kWarps, ... ---
-      const int mt = tiles > warp ? (tiles - warp + kWarps - 1) / kWarps : 0;
-      auto issue = [&](int q) {
-        if (q < mt) {
-          const int x0 = (warp + q * kWarps) * kTileRows;
-          const uint32_t dst = ring_w + (q % kTileRing) * kTileB + c_isv * (kTileRows * kPitch) + c_ch * 16 +
-                               c_sub * kPitch;
-          const unsigned char *src = (c_isv ? vbase : kbase) + c_ch * 16;
+    };
+    // copy tile q: rows past the segment repeat the tile's first row (finite
+    // data) and are masked out; the masks go to the warp's slot of tile q
+    auto issue = [&](int q, uint32_t row, uint32_t mask) {
+      if (q < mt) {
+        const long long gx0 = r0 + (long long)(warp + q * kWarps) * kTileRows;
+        const uint32_t first = __shfl_sync(kFull, row, 0);
+        if (gx0 + (lane & 15) >= r1) row = first;
+        if (lane < kTileRows) wmask[(q % kTileRing) * kTileRows + lane] = (uint16_t)mask;
+        const uint32_t dst = ring_w + (q % kTileRing) * kTileB + c_isv * (kTileRows * kPitch) + c_ch * 16 +
+                             c_sub * kPitch;
+        const unsigned char *src = (c_isv ? vbase : kbase) + c_ch * 16;
 #pragma unroll
-          for (int j = 0; j < kTileRows / RPI; ++j) {
-            const size_t row = lrow[x0 + j * RPI + c_sub];
-            cp_async16(dst + j * RPI * kPitch, src + row * kRowB, 16);
-          }
+        for (int j = 0; j < kTileRows / RPI; ++j) {
+          const uint32_t rj = __shfl_sync(kFull, row, j * RPI + c_sub);
+          cp_async16(dst + j * RPI * kPitch, src + (size_t)rj * kRowB, 16);
         }
-        cp_async_commit();
-      };
+      }
+      cp_async_commit();
+    };
+    uint32_t nrow, nmask;
+    fetch(0, nrow, nmask);
 #pragma unroll
-      for (int q = 0; q < kTileRing; ++q) issue(q);
+    for (int q = 0; q < kTileRing; ++q) {
+      const uint32_t row = nrow, mask = nmask;
+      fetch(q + 1, nrow, nmask);
+      issue(q, row, mask);
+    }
 
-      for (int q = 0; q < mt; ++q) {
-        cp_async_wait<kTileRing - 1>();
-        __syncwarp();
-        const uint32_t kt = ring_w + (q % kTileRing) * kTileB;
-        const int x0 = (warp + q * kWarps) * kTileRows;
+    for (int q = 0; q < mt; ++q) {
+      cp_async_wait<kTileRing - 1>();
+      __syncwarp();
+      const uint32_t kt = ring_w + (q % kTileRing) * kTileB;
         // S = Q K^T: n-tile j holds rows 8j .. 8j + 7 of the tile
         float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
@@ -569,8 +583,9 @@ attend_main_kernel(const AttendArgs a, const Shape sh, const Tables tb, const At
           }
         }
         // head masks of rows 2tq, 2tq + 1 (j = 0) and 8 + 2tq, 9 + 2tq (j = 1)
-        const uint32_t mk0 = *reinterpret_cast<const uint32_t *>(lmask + x0 + 2 * tq);
-        const uint32_t mk1 = *reinterpret_cast<const uint32_t *>(lmask + x0 + 8 + 2 * tq);
+        const uint16_t *ms = wmask + (q % kTileRing) * kTileRows;
+        const uint32_t mk0 = *reinterpret_cast<const uint32_t *>(ms + 2 * tq);
+        const uint32_t mk1 = *reinterpret_cast<const uint32_t *>(ms + 8 + 2 * tq);
         const uint32_t mr[4] = {mk0 & 0xFFFFu, mk0 >> 16, mk1 & 0xFFFFu, mk1 >> 16};
         float p[2][4];
 #pragma unroll
@@ -648,10 +663,13 @@ attend_main_kernel(const AttendArgs a, const Shape sh, const Tables tb, const At
           }
         }
         __syncwarp();
-        issue(q + kTileRing);
+        {
+          const uint32_t row = nrow, mask = nmask;
+          fetch(q + kTileRing + 1, nrow, nmask);
+          issue(q + kTileRing, row, mask);
+        }
       }
       cp_async_wait<0>();
-    }
     // per-lane partial sums of l -> per head
     l0 += __shfl_xor_sync(kFull, l0, 1);
     l0 += __shfl_xor_sync(kFull, l0, 2);
@@ -786,7 +804,7 @@ AttLayout att_layout(const Shape &sh, const Tables &tb, int batch) {
   L.plan_mask = o; o = align256(o + entries * 2);
   L.plan_cnt = o;  o = align256(o + (size_t)batch * tb.n_ret * p.ns * 4);
   L.tstart = o;    o = align256(o + (size_t)(p.ni + 1) * 8);
-  L.counters = o;  o = align256(o + ((size_t)p.ni * 2 + 1) * 4);     // item_rows, tickets, plan ticket
+  L.counters = o;  o = align256(o + (size_t)p.ni * 2 * 4);           // item_rows, tickets
   L.total = o;
   return L;
 }
@@ -837,13 +855,14 @@ cudaError_t launch_t(const AttendArgs &a, const Shape &sh, const Tables &tb, con
     e = set_smem(attend_plan_kernel<D, GR>, pbytes);
     if (e != cudaSuccess) return e;
     attend_plan_kernel<D, GR><<<dim3(p.ns, tb.n_ret, a.batch), kPlanThreads, pbytes, st>>>(a, sh, tb, p, ws);
-  } else {
-    attend_prefix_kernel<D><<<1, 256, 0, st>>>(a, sh, tb, p, ws);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
   }
+  attend_prefix_kernel<D><<<1, 1024, 0, st>>>(a, sh, tb, p, ws);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const size_t ring = (size_t)kWarps * kTileRing * (2 * kTileRows * (2 * D + 16));
-  const size_t lists = (size_t)kPassRows * 4 + (size_t)(kPassRows + kTileRows) * 2 + (size_t)(p.ns + 1) * 4;
+  const size_t lists = (size_t)kWarps * kTileRing * kTileRows * 2 + (size_t)(p.ns + 1) * 4;
   const size_t merge = (size_t)kWarps * 32 * 4 + (size_t)kWarps * GR * D * 4;
   const size_t bytes = std::max(ring + lists, merge);
   e = set_smem(attend_main_kernel<D, GR>, bytes);
@@ -885,8 +904,7 @@ cudaError_t launch_attend(const AttendArgs &a, const Shape &sh, const Tables &tb
   ws.tstart = reinterpret_cast<long long *>(base + L.tstart);
   ws.item_rows = reinterpret_cast<int *>(base + L.counters);
   ws.tickets = reinterpret_cast<unsigned *>(ws.item_rows + p.ni);
-  ws.plan_ticket = ws.tickets + p.ni;
-  cudaError_t e = cudaMemsetAsync(ws.item_rows, 0, ((size_t)p.ni * 2 + 1) * 4, st);
+  cudaError_t e = cudaMemsetAsync(ws.item_rows, 0, (size_t)p.ni * 2 * 4, st);
   if (e != cudaSuccess) return e;
   return sh.d == 128 ? dispatch_gr<128>(a, sh, tb, p, ws, st) : dispatch_gr<64>(a, sh, tb, p, ws, st);
 }

@@ -528,10 +528,10 @@ __device__ __forceinline__ void select_item(const SelectArgs &a, const Shape &sh
   }
 }
 
-// One cluster per work item (sequence, retrieval KV group).  With `flags`,
-// the grid's clusters stride over all items and process only the flagged
-// ones (items whose streaming top-k window missed); otherwise item =
-// blockIdx.y.
+// One cluster per work item (sequence, retrieval KV group).  With `flags`
+// (layout: a flag per item, then the count of flagged items, then their
+// list), the grid's clusters stride over the listed items only (items whose
+// streaming top-k window missed); otherwise item = blockIdx.y.
 template <int GR, bool TOPP, bool SMEM>
 __global__ void __launch_bounds__(kThreads, 1)
 select_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__ groups, int n_groups,
@@ -539,8 +539,9 @@ select_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__ grou
   __shared__ SelShared S;
   extern __shared__ __align__(16) unsigned char dyn[];
   const int n_items = a.batch * n_groups;
-  for (int item = blockIdx.y; item < n_items; item += gridDim.y) {
-    if (flags && flags[item] == 0u) continue;
+  const int n = flags ? (int)flags[n_items] : n_items;
+  for (int k = blockIdx.y; k < n; k += gridDim.y) {
+    const int item = flags ? (int)flags[n_items + 1 + k] : k;
     __syncthreads();
     select_item<GR, TOPP, SMEM>(a, sh, groups, n_groups, tc_cap, item, S, dyn);
   }
@@ -707,11 +708,11 @@ int smem_limit_bytes() {
 
 size_t select_workspace_bytes(const Shape &sh, const Tables &tb, int batch, size_t *flags_off) {
   // global score rows (used when the scores of a chunk do not fit on chip),
-  // then one flag per work item
+  // then one flag per work item, the count of flagged items and their list
   size_t rows = (size_t)batch * sh.H_ret * (size_t)sh.max_len * sizeof(float);
   rows = (rows + 255) / 256 * 256;
   if (flags_off) *flags_off = rows;
-  return rows + (size_t)batch * std::max(1, tb.n_ret) * sizeof(uint32_t);
+  return rows + (2 * (size_t)batch * std::max(1, tb.n_ret) + 1) * sizeof(uint32_t);
 }
 
 size_t select_topk_offset(const Shape &sh, const Tables &tb, int batch) {

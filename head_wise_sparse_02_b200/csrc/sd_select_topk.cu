@@ -25,9 +25,11 @@
 //   K2 resolve one CTA per (sequence, retrieval head): histograms the
 //              buffered scores over 512 bins of [t_lo, t_hi) (plus one bin for
 //              scores >= t_hi), scans from the top for the bin holding the
-//              k-th score, ranks the tokens of that bin exactly by (score
-//              desc, position asc), marks the selected positions in a bitmap
-//              of the context and writes them in ascending order.
+//              k-th score and, while that bin holds many tokens, splits it
+//              into 512 sub-bins and scans again (three levels at most); ranks
+//              the tokens of the final bin exactly by (score desc, position
+//              asc), marks the selected positions in a bitmap of the context
+//              and writes them in ascending order.
 // If the window misses (buffer overflow, k-th score outside the window, too
 // many tokens in the cut bin), K2 flags the work item and the exact general
 // kernel recomputes it.
@@ -51,6 +53,9 @@ constexpr int kRing = 12;             // K1: pages in flight per warp (even)
 // K1: staged buffer entries per (lane, head block); an iteration adds <= 4
 __host__ __device__ constexpr int stage_lane(int GR) { return GR <= 4 ? 10 : (GR == 8 ? 8 : 5); }
 constexpr int kCap = 2048;            // K2: cut-bin tokens ranked exactly
+constexpr int kLevels = 3;            // K2: histogram levels (the cut bin is split again)
+constexpr int kRefine = 64;           // K2: a cut bin above this many tokens is split again
+constexpr int kPer2 = 8;              // K2: buffer entries held in registers per thread
 constexpr int kPageBytes = kPage * kIndexDim * 2;   // 512 B: one page of one KV head
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
@@ -88,13 +93,49 @@ __device__ __forceinline__ int window_bin(float s, float tlo, float thi, float i
   return min(kBins - 1, max(0, __float2int_rz((s - tlo) * inv)));
 }
 
+// One warp: the highest bin c of hist[0, nb) (nb a multiple of 32, at most
+// 1024) whose suffix count sum_{b >= c} hist[b] reaches need (need >= 1);
+// -1 when the whole histogram holds fewer.  *above = sum_{b > c} hist[b],
+// *count = hist[c].  Each lane first sums its own nb / 32 consecutive bins,
+// one suffix scan over the 32 group totals picks the group, a second one
+// inside the group picks the bin.
+__device__ int warp_cut_bin(const uint32_t *hist, int nb, uint32_t need, int lane, uint32_t *above,
+                            uint32_t *count) {
+  const int G = nb >> 5;
+  uint32_t tot = 0;
+  for (int j = 0; j < G; ++j) tot += hist[lane * G + j];
+  uint32_t suf = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_down_sync(kFull, suf, o);
+    if (lane + o < 32) suf += y;
+  }
+  const unsigned bal = __ballot_sync(kFull, suf >= need);
+  if (!bal) return -1;
+  const int grp = 31 - __clz(bal);
+  const uint32_t acc = __shfl_sync(kFull, suf - tot, grp);     // bins of the groups above grp
+  const uint32_t c = lane < G ? hist[grp * G + lane] : 0u;
+  uint32_t s2 = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_down_sync(kFull, s2, o);
+    if (lane + o < 32) s2 += y;
+  }
+  const unsigned bal2 = __ballot_sync(kFull, lane < G && acc + s2 >= need);
+  const int j = 31 - __clz(bal2);                              // bal2 != 0: the group reaches need
+  *count = __shfl_sync(kFull, c, j);
+  *above = acc + __shfl_sync(kFull, s2, j) - *count;
+  return grp * G + j;
+}
+
 struct TopkWs {
   uint32_t *qsplit;                   // [rows][24]: bf16 pairs of the q~ terms hi, mid, lo
   float4 *win;                        // [rows]: t_lo, t_hi, 1 / bin width, unused
   uint32_t *bcount;                   // [rows] buffer entries written
   int *rowitem;                       // [rows] work item of the row
   unsigned long long *buf;            // [rows][cap]: order key << 32 | position
-  uint32_t *fail;                     // [items]
+  uint32_t *fail;                     // [items] flags, [1] count, [items] list of flagged items
+  int items;
   int cap;
 };
 
@@ -134,7 +175,7 @@ __device__ __forceinline__ long long topk_budget(const SelectArgs &a, long long 
 }
 
 // ------------------------------------------------------------------- K0
-constexpr int kT0 = 256;
+constexpr int kT0 = 512;
 
 template <int GR>
 __global__ void __launch_bounds__(kT0)
@@ -160,7 +201,10 @@ topk_window_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__
   long long N = a.seq_lens[b];
   N = N < 0 ? 0 : std::min<long long>(N, sh.max_len);
   const long long kb = topk_budget(a, N);
-  if (tid == 0) ws.fail[item] = 0u;
+  if (tid == 0) {
+    ws.fail[item] = 0u;
+    if (item == 0) ws.fail[ws.items] = 0u;           // count of flagged items
+  }
   if (tid < nr) {
     ws.bcount[(long long)b * sh.H_ret + grp.row[tid]] = 0u;
     ws.rowitem[(long long)b * sh.H_ret + grp.row[tid]] = item;
@@ -318,23 +362,9 @@ topk_window_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__
       const double mu = (double)m * (double)kb / (double)N;
       const double r = ceil(mu + 6.0 * sqrt(mu) + 8.0);
       if (r < (double)m) {
-        int blo = 0;
-        uint32_t acc = 0;
-        for (int top = kSampleBins; top > 0; top -= 32) {
-          const uint32_t c = shist[h][top - 32 + lane];
-          uint32_t suf = c;
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_down_sync(kFull, suf, o);
-            if (lane + o < 32) suf += y;
-          }
-          const unsigned bal = __ballot_sync(kFull, (double)(acc + suf) >= r);
-          if (bal) {
-            blo = top - 32 + (31 - __clz(bal));
-            break;
-          }
-          acc += __shfl_sync(kFull, suf, 0);
-        }
+        uint32_t above, cnt;
+        const int c = warp_cut_bin(shist[h], kSampleBins, (uint32_t)r, lane, &above, &cnt);
+        const int blo = c < 0 ? 0 : c;
         tlo = lo + (float)blo * ((hi - lo) / (float)kSampleBins);
       }
     }
@@ -497,8 +527,10 @@ topk_resolve_kernel(const SelectArgs a, const Shape sh, const TopkWs ws) {
   __shared__ unsigned long long cand[kCap];
   __shared__ uint32_t hist[kBins + 1];
   __shared__ uint32_t n_cand;
-  __shared__ int cut_s, fail_s;
+  __shared__ int fail_s, done_s;
   __shared__ long long need_s;
+  __shared__ int cutv[kLevels];
+  __shared__ float llo[kLevels], linv[kLevels];
   __shared__ uint32_t wtot[kT2 / 32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int b = blockIdx.y, hr = blockIdx.x;
@@ -521,67 +553,104 @@ topk_resolve_kernel(const SelectArgs a, const Shape sh, const TopkWs ws) {
   const int n = (int)std::min<uint32_t>(nbuf, (uint32_t)ws.cap);
   const int words = (int)((N + 31) / 32);
   for (int o = tid; o < words; o += kT2) bitmap[o] = 0u;
-  for (int o = tid; o <= kBins; o += kT2) hist[o] = 0u;
-  __syncthreads();
-  // window histogram of the buffered scores (all >= t_lo)
-  for (int e = tid; e < n; e += kT2) {
-    const uint32_t key = (uint32_t)(buf[e] >> 32);
-    atomicAdd(&hist[window_bin(key_to_float(key), w.x, w.y, w.z)], 1u);
+  if (tid == 0) {
+    llo[0] = w.x;
+    linv[0] = w.z;
+    need_s = kb;
+    fail_s = 0;
+    done_s = 0;
+    n_cand = 0u;
   }
-  __syncthreads();
-  // cut bin: warp 0 scans the histogram from the top, 32 bins at a time
-  if (warp == 0) {
-    const long long top = hist[kBins];
-    const long long need = kb - top;
-    long long acc = 0;
-    int cut = -1;
-    long long ncut = 0;
-    if (need > 0) {
-      for (int hi = kBins; hi > 0 && cut < 0; hi -= 32) {
-        const int bin = hi - 32 + lane;
-        const uint32_t c = hist[bin];
-        long long suf = c;
+  // bin of a score at level L: level 0 is the window histogram (bin kBins:
+  // scores >= t_hi); level L > 0 splits the cut bin of level L - 1 into kBins
+  // linear sub-bins.  Bins are non-decreasing in the score at every level.
+  auto bin_at = [&](float v, int L) -> int {
+    if (L == 0) return window_bin(v, w.x, w.y, w.z);
+    return min(kBins - 1, max(0, __float2int_rz((v - llo[L]) * linv[L])));
+  };
+  // this thread's first kPer2 entries, loaded once (the passes below reread
+  // only entries past kPer2 * kT2 from memory)
+  unsigned long long ent[kPer2];
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const long long y = __shfl_down_sync(kFull, suf, o);
-          if (lane + o < 32) suf += y;
-        }
-        const unsigned bal = __ballot_sync(kFull, c > 0u && acc + suf >= need);
-        if (bal) {
-          const int l = 31 - __clz(bal);
-          cut = hi - 32 + l;
-          ncut = __shfl_sync(kFull, (long long)c, l);
-          acc += __shfl_sync(kFull, suf, l) - ncut;
+  for (int j = 0; j < kPer2; ++j) {
+    const int e = tid + j * kT2;
+    ent[j] = e < n ? buf[e] : 0ull;
+  }
+  // the cut bin: refine while it holds more than kRefine tokens
+  int L = 0;
+  for (; L < kLevels; ++L) {
+    for (int o = tid; o <= kBins; o += kT2) hist[o] = 0u;
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kPer2; ++j) {
+      const int e = tid + j * kT2;
+      if (e < n) {
+        const float v = key_to_float((uint32_t)(ent[j] >> 32));
+        bool play = true;
+        for (int l = 0; l < L; ++l) play = play && bin_at(v, l) == cutv[l];
+        if (play) atomicAdd(&hist[bin_at(v, L)], 1u);
+      }
+    }
+    for (int e = tid + kPer2 * kT2; e < n; e += kT2) {
+      const float v = key_to_float((uint32_t)(buf[e] >> 32));
+      bool play = true;
+      for (int l = 0; l < L; ++l) play = play && bin_at(v, l) == cutv[l];
+      if (play) atomicAdd(&hist[bin_at(v, L)], 1u);
+    }
+    __syncthreads();
+    // warp 0 finds the bin holding the cut among the level's bins
+    if (warp == 0) {
+      const long long need = need_s - (L == 0 ? (long long)hist[kBins] : 0LL);
+      uint32_t above = 0, ncut = 0;
+      const int cut = need > 0 ? warp_cut_bin(hist, kBins, (uint32_t)need, lane, &above, &ncut) : -1;
+      const long long acc = above;
+      if (lane == 0) {
+        if (need <= 0 || cut < 0 || nbuf > (uint32_t)ws.cap) {
+          fail_s = 1;
         } else {
-          acc += __shfl_sync(kFull, suf, 0);
+          cutv[L] = cut;
+          need_s = need - acc;                       // tokens still to take from the cut bin
+          const bool last = ncut <= kRefine || L + 1 == kLevels;
+          if (last && ncut > kCap) fail_s = 1;
+          if (!last) {
+            llo[L + 1] = llo[L] + (float)cut / linv[L];
+            linv[L + 1] = linv[L] * (float)kBins;
+          }
+          done_s = last;
         }
       }
     }
-    if (lane == 0) {
-      const bool bad = need <= 0 || cut < 0 || ncut > kCap || nbuf > (uint32_t)ws.cap;
-      fail_s = bad;
-      cut_s = cut;
-      need_s = need - acc;                           // tokens to take from the cut bin
-      n_cand = 0u;
-    }
+    __syncthreads();
+    if (fail_s || done_s) break;
   }
-  __syncthreads();
   if (fail_s) {
-    if (tid == 0) atomicOr(&ws.fail[ws.rowitem[row]], 1u);
+    if (tid == 0) {
+      const int it = ws.rowitem[row];
+      if (atomicExch(&ws.fail[it], 1u) == 0u) ws.fail[ws.items + 1 + atomicAdd(&ws.fail[ws.items], 1u)] = (uint32_t)it;
+    }
     return;
   }
-  const int cut = cut_s;
-  for (int e = tid; e < n; e += kT2) {
-    const unsigned long long ent = buf[e];
-    const uint32_t key = (uint32_t)(ent >> 32), pos = (uint32_t)ent;
-    const int cls = window_bin(key_to_float(key), w.x, w.y, w.z);
-    if (cls > cut) {
+  const int nlev = L + 1;
+  // classify: above the cut path -> selected; on it -> candidate
+  auto classify = [&](unsigned long long en) {
+    const uint32_t key = (uint32_t)(en >> 32), pos = (uint32_t)en;
+    const float v = key_to_float(key);
+    int rel = 0;
+    for (int l = 0; l < nlev && rel == 0; ++l) {
+      const int bl = bin_at(v, l);
+      rel = bl > cutv[l] ? 1 : (bl < cutv[l] ? -1 : 0);
+    }
+    if (rel > 0) {
       atomicOr(&bitmap[pos >> 5], 1u << (pos & 31));
-    } else if (cls == cut) {
+    } else if (rel == 0) {
       const uint32_t at = atomicAdd(&n_cand, 1u);
       if (at < (uint32_t)kCap) cand[at] = ((unsigned long long)(~key) << 32) | pos;   // ascending = better first
     }
-  }
+  };
+#pragma unroll
+  for (int j = 0; j < kPer2; ++j)
+    if (tid + j * kT2 < n) classify(ent[j]);
+  for (int e = tid + kPer2 * kT2; e < n; e += kT2) classify(buf[e]);
   __syncthreads();
   // rank the cut bin exactly: the need_c best by (score desc, position asc)
   const int nc = (int)std::min<uint32_t>(n_cand, (uint32_t)kCap);
@@ -724,6 +793,7 @@ cudaError_t launch_select_topk_stream(const SelectArgs &a, const Shape &sh, cons
   ws.rowitem = reinterpret_cast<int *>(base + L.rowitem);
   ws.buf = reinterpret_cast<unsigned long long *>(base + L.buf);
   ws.fail = fail;
+  ws.items = a.batch * tb.n_ret;
   ws.cap = p.cap;
   int gr = 1;
   while (gr < tb.max_ret) gr <<= 1;
