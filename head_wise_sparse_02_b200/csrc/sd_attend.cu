@@ -100,6 +100,14 @@ __device__ __forceinline__ void mma_bf16_top(float (&d)[2], uint32_t a0, uint32_
       : "+f"(d[0]), "+f"(d[1]), "=f"(j0), "=f"(j1)
       : "r"(a0), "r"(zu), "r"(a2), "r"(b0), "r"(b1), "f"(zf));
 }
+// 2^x by the MUFU unit (PTX ex2.approx.ftz.f32: relative error below 2^-22,
+// subnormal results flushed to 0, exp2(-inf) = 0), far inside the float32
+// accumulation's own error here
+__device__ __forceinline__ float fast_exp2(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(r) : "f"(x));
+  return r;
+}
 // two floats -> bf16x2 (x in the low half), round to nearest even
 __device__ __forceinline__ uint32_t pack_bf16(float x, float y) {
   uint32_t r;
@@ -602,7 +610,7 @@ attend_main_kernel(const AttendArgs a, const Shape sh, const Tables tb, const At
         x0m = fmaxf(x0m, __shfl_xor_sync(kFull, x0m, 2));
         const float mn0 = fmaxf(m0, x0m);
         const float mu0 = mn0 == -INFINITY ? 0.f : mn0;
-        const float al0 = mn0 == m0 ? 1.f : exp2f(m0 - mu0);
+        const float al0 = mn0 == m0 ? 1.f : fast_exp2(m0 - mu0);
         m0 = mn0;
         float al1 = 1.f;
         if (HI) {
@@ -611,12 +619,12 @@ attend_main_kernel(const AttendArgs a, const Shape sh, const Tables tb, const At
           x1m = fmaxf(x1m, __shfl_xor_sync(kFull, x1m, 2));
           const float mn1 = fmaxf(m1, x1m);
           const float mu1 = mn1 == -INFINITY ? 0.f : mn1;
-          al1 = mn1 == m1 ? 1.f : exp2f(m1 - mu1);
+          al1 = mn1 == m1 ? 1.f : fast_exp2(m1 - mu1);
           m1 = mn1;
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
-            p[j][2] = exp2f(p[j][2] - mu1);
-            p[j][3] = exp2f(p[j][3] - mu1);
+            p[j][2] = fast_exp2(p[j][2] - mu1);
+            p[j][3] = fast_exp2(p[j][3] - mu1);
           }
           l1 = fmaf(l1, al1, (p[0][2] + p[0][3]) + (p[1][2] + p[1][3]));
         } else {
@@ -625,8 +633,8 @@ attend_main_kernel(const AttendArgs a, const Shape sh, const Tables tb, const At
         }
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
-          p[j][0] = exp2f(p[j][0] - mu0);
-          p[j][1] = exp2f(p[j][1] - mu0);
+          p[j][0] = fast_exp2(p[j][0] - mu0);
+          p[j][1] = fast_exp2(p[j][1] - mu0);
         }
         l0 = fmaf(l0, al0, (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]));
         if (__any_sync(kFull, al0 != 1.f || al1 != 1.f)) {

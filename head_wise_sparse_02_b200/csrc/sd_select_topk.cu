@@ -385,7 +385,10 @@ topk_stream_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__
   constexpr int SL = stage_lane(GR);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gq = lane >> 2, tq = lane & 3;
-  const int item = blockIdx.y;
+  // item fastest in the launch order: CTAs of all KV groups for the same
+  // chunk of pages run together, so reads of the groups' 512-byte slices of a
+  // page (adjacent in the index cache) meet in the same DRAM rows
+  const int item = blockIdx.x;
   const int b = item / n_groups, gi = item % n_groups;
   extern __shared__ __align__(128) unsigned char dyn1[];
   unsigned char (*ring)[kRing][kPageBytes] = reinterpret_cast<unsigned char (*)[kRing][kPageBytes]>(dyn1);
@@ -403,7 +406,7 @@ topk_stream_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__
   const long long kb = topk_budget(a, N);
   if (N == 0 || kb >= N) return;
   const int pages = (int)((N + kPage - 1) / kPage);
-  const int p0 = blockIdx.x * kChunkPages;
+  const int p0 = blockIdx.y * kChunkPages;
   if (p0 >= pages) return;
   const int np = pages - p0 < kChunkPages ? pages - p0 : kChunkPages;
   {
@@ -764,7 +767,7 @@ cudaError_t topk_launch(const SelectArgs &a, const Shape &sh, const Tables &tb, 
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int chunks = (int)((sh.max_pages + kChunkPages - 1) / kChunkPages);
-  topk_stream_kernel<GR><<<dim3(chunks, items), kT1, smem1, st>>>(a, sh, tb.ret, tb.n_ret, ws);
+  topk_stream_kernel<GR><<<dim3(items, chunks), kT1, smem1, st>>>(a, sh, tb.ret, tb.n_ret, ws);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   topk_resolve_kernel<<<dim3(sh.H_ret, a.batch), kT2, bitmap_bytes, st>>>(a, sh, ws);
