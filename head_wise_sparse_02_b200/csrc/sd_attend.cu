@@ -55,7 +55,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 // plan
 constexpr int kPlanThreads = 256;
 constexpr int kPlanWarps = kPlanThreads / 32;
-constexpr int kSpanMax = 8192;          // positions per plan CTA (max)
+constexpr int kSpanMax = 32768;         // positions per plan CTA (max)
 
 // main
 constexpr int kThreads = 128;
@@ -789,7 +789,7 @@ int group_rows_att(const Tables &tb) { return pow2_ceil(std::max(1, std::max(tb.
 AttParams att_params(const Shape &sh, const Tables &tb, int batch) {
   AttParams p{};
   const long long L = sh.max_len;
-  p.span = (int)std::max(256LL, std::min<long long>(kSpanMax, pow2_ceil((L + 15) / 16)));
+  p.span = (int)std::max(256LL, std::min<long long>(kSpanMax, pow2_ceil((L + 3) / 4)));   // ~4 spans per sequence
   p.ns = (int)((L + p.span - 1) / p.span);
   p.n_ret_items = batch * tb.n_ret;
   p.ni = batch * (tb.n_ret + tb.n_loc);

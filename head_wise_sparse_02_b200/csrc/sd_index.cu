@@ -38,9 +38,13 @@ index_keys_kernel(const uint16_t *__restrict__ k_pre, const int32_t *__restrict_
   const int row = threadIdx.x / kIndexDim, j = threadIdx.x % kIndexDim;
   const int t = t0 + row;
   if (t >= T) return;
-  double acc = 0.0;
+  // four interleaved partial sums (shorter dependent chains), added at the end
+  double acc4[4] = {0.0, 0.0, 0.0, 0.0};
 #pragma unroll 8
-  for (int i = 0; i < D; ++i) acc = fma(Ks[row][i], Ps[i][j], acc);
+  for (int i = 0; i < D; i += 4)
+#pragma unroll
+    for (int u = 0; u < 4; ++u) acc4[u] = fma(Ks[row][i + u], Ps[i + u][j], acc4[u]);
+  const double acc = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
   const long long slot = slots[t];
   if (slot < 0 || slot >= (long long)num_pages * kPage) {
     if (j == 0) raise_error(err, SD_EBIT_SLOT);

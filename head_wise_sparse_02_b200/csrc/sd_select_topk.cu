@@ -55,7 +55,7 @@ __host__ __device__ constexpr int stage_lane(int GR) { return GR <= 4 ? 10 : (GR
 constexpr int kCap = 2048;            // K2: cut-bin tokens ranked exactly
 constexpr int kLevels = 3;            // K2: histogram levels (the cut bin is split again)
 constexpr int kRefine = 64;           // K2: a cut bin above this many tokens is split again
-constexpr int kPer2 = 8;              // K2: buffer entries held in registers per thread
+constexpr int kPer2 = 16;             // K2: buffer entries held in registers per thread
 constexpr int kPageBytes = kPage * kIndexDim * 2;   // 512 B: one page of one KV head
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
@@ -522,9 +522,9 @@ topk_stream_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__
 }
 
 // ------------------------------------------------------------------- K2
-constexpr int kT2 = 512;
+constexpr int kT2 = 256;
 
-__global__ void __launch_bounds__(kT2)
+__global__ void __launch_bounds__(kT2, 4)
 topk_resolve_kernel(const SelectArgs a, const Shape sh, const TopkWs ws) {
   extern __shared__ uint32_t bitmap[];               // [max_len / 32]
   __shared__ unsigned long long cand[kCap];
