@@ -75,7 +75,8 @@ def barrier():
 
 class ClockSampler:
     """SM clock and throttle-reason samples during the timed region, read
-    through NVML every 10 ms (the data nvidia-smi reports; nothing is set).
+    through NVML every millisecond (the data nvidia-smi reports; nothing is
+    set): the timed region of a default run lasts a few milliseconds.
     Falls back to `nvidia-smi -lms 200` when NVML is unavailable."""
 
     # NVML clocks-event reason bits
@@ -119,7 +120,7 @@ class ClockSampler:
                                          int(getr(self.handle))))
                 except Exception:
                     pass
-                time.sleep(0.01)
+                time.sleep(0.001)
 
         self.thread = threading.Thread(target=loop, daemon=True)
         self.thread.start()
@@ -138,7 +139,7 @@ class ClockSampler:
                 if r & bit:
                     reasons.add(name)
         return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons),
-                "samples": len(sm), "source": "nvml 10 ms"}
+                "samples": len(sm), "source": "nvml 1 ms"}
 
 
 # ---------------------------------------------------------------- measurements
@@ -188,9 +189,11 @@ def ncu_traffic(kernel: str, algorithmic_bytes: float):
 def kernels_per_step(w) -> int:
     """Kernels of this library one step launches: index_keys; select (top-k:
     window, stream, resolve and the exact selector for flagged items; top-p:
-    the exact selector); attend (plan, or the item layout alone, and main)."""
-    n_sel = 0 if not any(w.head_is_retrieval) else (4 if w.mode == "top_k" else 1)
-    return 1 + n_sel + 2
+    the exact selector); attend (plan when there are retrieval heads, item
+    layout, main)."""
+    ret = any(w.head_is_retrieval)
+    n_sel = 0 if not ret else (4 if w.mode == "top_k" else 1)
+    return 1 + n_sel + (3 if ret else 2)
 
 
 def union_rows(sel_idx, sel_count, w):
