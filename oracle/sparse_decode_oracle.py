@@ -44,10 +44,12 @@ uint16 arrays holding raw bf16 bit patterns; both are widened exactly to
 float64 before any arithmetic.
 
 Parity pins: every function below is pinned by ``tests/test_oracle_pins.py``
-against closed forms, brute force or an independent library routine; the
-end-to-end composition (``decode_reference``) on realistic inputs has no
-external pin beyond those of its parts ("parity unpinned" for the composed
-result; see the test module).
+against closed forms, brute force or an independent library routine.  The
+end-to-end composition (``decode_reference``) is pinned on constructed cases:
+the degenerate settings that reduce to dense attention, and planted needles
+under a coordinate-selection projection, whose selected set is known by
+construction (compared with float64 SDPA over that set).  On general inputs
+the composition has no pin beyond those of its parts ("parity unpinned").
 """
 
 from __future__ import annotations

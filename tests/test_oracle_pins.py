@@ -332,3 +332,70 @@ def test_widen_accepts_bf16_bit_patterns():
     x = O.bf16_round(np.random.default_rng(9).standard_normal(100))
     bits = _bf16_bits(x.astype(np.float32)).astype(np.uint16)
     np.testing.assert_array_equal(O.widen(bits), x)
+
+
+# ---------------------------------------------------------------- composition
+
+def _planted_problem(seed, n=200, d=32, needles=(17, 64, 130, 199), gain=40.0):
+    """One sequence, Hq = 2 retrieval heads on KV head 0 plus 2 local heads on
+    KV head 1.  The projection selects the first 16 coordinates, so a key's
+    index entry is its first 16 coordinates.  Background keys are zero there
+    (index score exactly 0); needle i points along the query with scores
+    gain - 0.1 i (distinct, far above 0).  Pages are permuted."""
+    rng = np.random.default_rng(seed)
+    ps, r, Hq, Hkv = 16, 16, 4, 2
+    pages = math.ceil(n / ps)
+    perm = rng.permutation(pages)
+    pt = perm[None, :].astype(np.int64)
+    K = O.bf16_round(rng.standard_normal((n, Hkv, d)))
+    V = O.bf16_round(rng.standard_normal((n, Hkv, d)))
+    K[:, 0, :r] = 0.0
+    q = O.bf16_round(rng.standard_normal((1, Hq, d)))
+    # both retrieval heads share the first 16 query coordinates (unit-norm u)
+    u = rng.standard_normal(r)
+    u /= np.linalg.norm(u)
+    q[0, 0, :r] = O.bf16_round(u)
+    q[0, 1, :r] = O.bf16_round(u)
+    c = math.sqrt(d) / r
+    for i, j in enumerate(needles):
+        # index score = c * <q~, k~> with k~ = a u  =>  a = target / (c <q[:r], u>)
+        a = (gain - 0.1 * i) / (c * float(q[0, 0, :r] @ u))
+        K[j, 0, :r] = O.bf16_round(a * u)
+    kc = np.zeros((pages, Hkv, ps, d))
+    vc = np.zeros((pages, Hkv, ps, d))
+    for j in range(n):
+        kc[perm[j // ps], :, j % ps] = K[j]
+        vc[perm[j // ps], :, j % ps] = V[j]
+    proj = np.zeros((Hkv, d, r))
+    proj[:, :r, :] = np.eye(r)
+    prob = dict(proj=proj, q_pre=q, q=q, k_cache=kc, v_cache=vc, page_table=pt, seq_lens=np.array([n]))
+    return prob, K, V, Hq, Hkv, d, r
+
+
+@pytest.mark.parametrize("mode", ["top_k", "top_p"])
+def test_decode_step_composed_on_planted_needles(mode):
+    # index keys -> scores -> selection -> attention on a case whose selected
+    # set is known by construction; the output must equal float64 SDPA over
+    # exactly that set, and the local heads SDPA over sinks + window
+    needles = (17, 64, 130, 199)
+    prob, K, V, Hq, Hkv, d, r = _planted_problem(21, needles=needles)
+    retr = [1, 1, 0, 0]
+    if mode == "top_k":
+        cfg = O.OracleConfig(Hq, Hkv, d, r, 16, retr, 5, 2, "top_k", top_k=len(needles))
+    else:
+        # masses e^40, e^39.9, e^39.8, e^39.7 (cumulative 0.29, 0.55, 0.79, 1.0):
+        # p = 0.9 needs all four; the 196 zero scores add ~1e-15 of the mass
+        cfg = O.OracleConfig(Hq, Hkv, d, r, 16, retr, 5, 2, "top_p", top_p=0.9)
+    res = O.decode_reference(cfg, **prob, keep_scores=True)
+    for h in (0, 1):
+        np.testing.assert_array_equal(res.sets[(0, h)], np.array(needles))
+        s = res.scores[(0, h)]
+        assert np.all(s[np.setdiff1d(np.arange(200), needles)] == 0.0)
+        np.testing.assert_allclose(s[list(needles)], [40.0, 39.9, 39.8, 39.7], rtol=5e-3)
+        idx = np.array(needles)
+        want = _sdpa64(prob["q"][0, h], K[idx, 0], V[idx, 0], 1 / math.sqrt(d))
+        np.testing.assert_allclose(res.out[(0, h)], want, rtol=1e-11, atol=1e-12)
+    loc = np.array([0, 1, 195, 196, 197, 198, 199])       # sinks 0-1, window of 5
+    for h in (2, 3):
+        want = _sdpa64(prob["q"][0, h], K[loc, 1], V[loc, 1], 1 / math.sqrt(d))
+        np.testing.assert_allclose(res.out[(0, h)], want, rtol=1e-11, atol=1e-12)
