@@ -197,6 +197,30 @@ def test_host_side_argument_errors():
     st.close()
 
 
+# ------------------------------------------------------------------ group shapes
+
+# GQA group sizes and head dims beyond the named workloads: 16 heads per group
+# (all 16 rows of the attention MMA), 8 per group in top-k, MHA (1 per group),
+# d = 64 in top-k; ragged lengths, permuted pages
+SHAPES = [
+    ("g16_topk", [3001, 2500], 32, 2, 128, [1] * 32, 0, 0, "top_k", dict(top_k_frac=0.05)),
+    ("g16_mixed_topp", [2900, 1700], 32, 2, 128, [1] * 16 + [0] * 16, 300, 4, "top_p", dict(top_p=0.9)),
+    ("g8_topk", [4100, 777], 32, 4, 128, [1] * 32, 0, 0, "top_k", dict(top_k=100)),
+    ("d64_topk", [2000, 3333], 8, 2, 64, [1] * 8, 0, 0, "top_k", dict(top_k_frac=0.03)),
+    ("mha_mixed_topp", [1500, 2222], 8, 8, 128, [1, 0] * 4, 200, 2, "top_p", dict(top_p=0.8)),
+]
+
+
+@pytest.mark.parametrize("case", SHAPES, ids=[c[0] for c in SHAPES])
+def test_group_shapes(case):
+    from workloads.synthetic import _base, _gen, _plant_needles
+    name, lens, Hq, Hkv, d, retr, window, sinks, mode, kw = case
+    w = _base(name, 11, "cuda", lens, Hq, Hkv, d, retr, window, sinks, mode, permute=True, **kw)
+    if mode == "top_p":
+        _plant_needles(w, {b: [3] * sum(retr) for b in range(w.batch)}, _gen("cuda", 11, 6))
+    check_workload(w, label=name)
+
+
 # ------------------------------------------------------------------ top-k fallback
 
 def _group_query_keys(w, b, n, gain, noise, seed):
