@@ -422,12 +422,11 @@ attend_main_kernel(const AttendArgs a, const Shape sh, const Tables tb, const At
     if (lane == 0) S.item = i;
   }
 
-  // cp.async mapping: one instruction copies whole rows (coalesced): for
-  // d = 128 lanes 0-15 the K row and lanes 16-31 the V row of tile row j; for
-  // d = 64 lanes 0-7 / 8-15 the K / V row of tile row 2j, lanes 16-31 row 2j + 1
-  constexpr int RPI = 32 / (2 * CPR);                // tile rows per instruction
-  const int c_sub = lane / (2 * CPR);                // which of them
-  const int c_isv = (lane / CPR) & 1;                // K or V
+  // cp.async mapping: a tile's K rows and its V rows are copied separately
+  // (one commit group each), whole rows per instruction (coalesced): lanes
+  // [CPR c, CPR (c + 1)) copy row j RPH + c, one 16-byte chunk each
+  constexpr int RPH = 32 / CPR;                      // tile rows per copy instruction
+  const int c_sub = lane / CPR;                      // which of them
   const int c_ch = lane % CPR;                       // 16-byte chunk of the row
   const uint32_t ring_w = ring0 + warp * (kTileRing * kTileB);
   const unsigned char *kbase = reinterpret_cast<const unsigned char *>(a.k_cache);
@@ -542,21 +541,27 @@ attend_main_kernel(const AttendArgs a, const Shape sh, const Tables tb, const At
         }
       }
     };
-    // copy tile q: rows past the segment repeat the tile's first row (finite
+    // tile q's rows: rows past the segment repeat the tile's first row (finite
     // data) and are masked out; the masks go to the warp's slot of tile q
-    auto issue = [&](int q, uint32_t row, uint32_t mask) {
+    auto prep = [&](int q, uint32_t row, uint32_t mask) -> uint32_t {
       if (q < mt) {
         const long long gx0 = r0 + (long long)(warp + q * kWarps) * kTileRows;
         const uint32_t first = __shfl_sync(kFull, row, 0);
         if (gx0 + (lane & 15) >= r1) row = first;
         if (lane < kTileRows) wmask[(q % kTileRing) * kTileRows + lane] = (uint16_t)mask;
-        const uint32_t dst = ring_w + (q % kTileRing) * kTileB + c_isv * (kTileRows * kPitch) + c_ch * 16 +
+      }
+      return row;
+    };
+    // copy the K rows (half 0) or the V rows (half 1) of tile q: one commit group
+    auto issue_half = [&](int q, uint32_t row, int half) {
+      if (q < mt) {
+        const uint32_t dst = ring_w + (q % kTileRing) * kTileB + half * (kTileRows * kPitch) + c_ch * 16 +
                              c_sub * kPitch;
-        const unsigned char *src = (c_isv ? vbase : kbase) + c_ch * 16;
+        const unsigned char *src = (half ? vbase : kbase) + c_ch * 16;
 #pragma unroll
-        for (int j = 0; j < kTileRows / RPI; ++j) {
-          const uint32_t rj = __shfl_sync(kFull, row, j * RPI + c_sub);
-          cp_async16(dst + j * RPI * kPitch, src + (size_t)rj * kRowB, 16);
+        for (int j = 0; j < kTileRows / RPH; ++j) {
+          const uint32_t rj = __shfl_sync(kFull, row, j * RPH + c_sub);
+          cp_async16(dst + j * RPH * kPitch, src + (size_t)rj * kRowB, 16);
         }
       }
       cp_async_commit();
@@ -565,13 +570,18 @@ attend_main_kernel(const AttendArgs a, const Shape sh, const Tables tb, const At
     fetch(0, nrow, nmask);
 #pragma unroll
     for (int q = 0; q < kTileRing; ++q) {
-      const uint32_t row = nrow, mask = nmask;
+      const uint32_t row = prep(q, nrow, nmask);
       fetch(q + 1, nrow, nmask);
-      issue(q, row, mask);
+      issue_half(q, row, 0);
+      issue_half(q, row, 1);
     }
 
+    // Groups in flight: K and V of the next kTileRing tiles.  K of tile
+    // q + kTileRing is issued as soon as S(q) has read K(q) (during the
+    // softmax and P V of tile q), V of tile q + kTileRing after P V(q); at
+    // both waits 2 kTileRing - 1 younger groups may stay pending.
     for (int q = 0; q < mt; ++q) {
-      cp_async_wait<kTileRing - 1>();
+      cp_async_wait<2 * kTileRing - 1>();              // K(q)
       __syncwarp();
       const uint32_t kt = ring_w + (q % kTileRing) * kTileB;
         // S = Q K^T: n-tile j holds rows 8j .. 8j + 7 of the tile
@@ -595,6 +605,10 @@ attend_main_kernel(const AttendArgs a, const Shape sh, const Tables tb, const At
         const uint32_t mk0 = *reinterpret_cast<const uint32_t *>(ms + 2 * tq);
         const uint32_t mk1 = *reinterpret_cast<const uint32_t *>(ms + 8 + 2 * tq);
         const uint32_t mr[4] = {mk0 & 0xFFFFu, mk0 >> 16, mk1 & 0xFFFFu, mk1 >> 16};
+        __syncwarp();                                  // K(q) and the masks of q read by all lanes
+        const uint32_t rowR = prep(q + kTileRing, nrow, nmask);
+        fetch(q + kTileRing + 1, nrow, nmask);
+        issue_half(q + kTileRing, rowR, 0);
         float p[2][4];
 #pragma unroll
         for (int j = 0; j < 2; ++j)
@@ -647,6 +661,8 @@ attend_main_kernel(const AttendArgs a, const Shape sh, const Tables tb, const At
           }
         }
         // P as the A operand (heads x 16 rows), hi + lo
+        cp_async_wait<2 * kTileRing - 1>();            // V(q)
+        __syncwarp();
         uint32_t ph[4], pl[4];
         split_bf16(p[0][0], p[0][1], ph[0], pl[0]);  // head gq,     rows 2tq, 2tq+1
         split_bf16(p[0][2], p[0][3], ph[1], pl[1]);  // head gq + 8, rows 2tq, 2tq+1
@@ -671,11 +687,7 @@ attend_main_kernel(const AttendArgs a, const Shape sh, const Tables tb, const At
           }
         }
         __syncwarp();
-        {
-          const uint32_t row = nrow, mask = nmask;
-          fetch(q + kTileRing + 1, nrow, nmask);
-          issue(q + kTileRing, row, mask);
-        }
+        issue_half(q + kTileRing, rowR, 1);
       }
       cp_async_wait<0>();
     // per-lane partial sums of l -> per head
