@@ -49,7 +49,7 @@ constexpr int kBins = 512;            // window histogram bins (+1 slot: scores 
 __host__ __device__ constexpr int sample_pages(int GR) { return GR <= 4 ? 256 : (GR == 8 ? 192 : 96); }
 constexpr int kSampleBins = 256;
 constexpr int kChunkPages = 512;      // K1: pages per CTA
-constexpr int kRing = 12;             // K1: pages in flight per warp (even)
+constexpr int kRing = 8;              // K1: pages in flight per warp (even); 4 CTAs per SM
 // K1: staged buffer entries per (lane, head block); an iteration adds <= 4
 __host__ __device__ constexpr int stage_lane(int GR) { return GR <= 4 ? 10 : (GR == 8 ? 8 : 5); }
 constexpr int kCap = 2048;            // K2: cut-bin tokens ranked exactly
