@@ -162,7 +162,7 @@ def kernel_source_hash(files):
 
 
 KERNEL_SOURCES = {
-    "select": ["head_wise_sparse_02_b200/csrc/sd_select.cu", "head_wise_sparse_02_b200/csrc/sd_select_topk.cu",
+    "select": ["head_wise_sparse_02_b200/csrc/sd_select.cu", "head_wise_sparse_02_b200/csrc/sd_select_stream.cu",
                "head_wise_sparse_02_b200/csrc/sd_internal.cuh"],
     "attend": ["head_wise_sparse_02_b200/csrc/sd_attend.cu", "head_wise_sparse_02_b200/csrc/sd_internal.cuh"],
     "index_keys": ["head_wise_sparse_02_b200/csrc/sd_index.cu", "head_wise_sparse_02_b200/csrc/sd_internal.cuh"],
@@ -188,11 +188,11 @@ def ncu_traffic(kernel: str, algorithmic_bytes: float):
 
 def kernels_per_step(w) -> int:
     """Kernels of this library one step launches: index_keys; select (top-k:
-    window, stream, resolve and the exact selector for flagged items; top-p:
-    the exact selector); attend (plan when there are retrieval heads, item
-    layout, main)."""
+    window, stream, resolve; top-p: window, mass pass, cut pass, resolve;
+    then the exact selector for flagged items); attend (plan when there are
+    retrieval heads, item layout, main)."""
     ret = any(w.head_is_retrieval)
-    n_sel = 0 if not ret else (4 if w.mode == "top_k" else 1)
+    n_sel = 0 if not ret else (4 if w.mode == "top_k" else 5)
     return 1 + n_sel + (3 if ret else 2)
 
 

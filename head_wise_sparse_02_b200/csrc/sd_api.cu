@@ -57,7 +57,7 @@ WsLayout layout(const sd_ctx *ctx, int batch) {
   w.scores_bytes = align256(sd::select_workspace_bytes(ctx->sh, ctx->tb, batch, &foff));
   w.flags_off = w.scores_off + foff;
   w.topk_off = w.scores_off + w.scores_bytes;
-  w.topk_bytes = ctx->cfg.mode == SD_TOP_K ? align256(sd::topk_workspace_bytes(ctx->sh, ctx->tb, batch)) : 0;
+  w.topk_bytes = align256(sd::stream_workspace_bytes(ctx->sh, ctx->tb, batch, ctx->cfg.mode));
   w.att_off = w.topk_off + w.topk_bytes;
   w.total = align256(w.att_off + sd::attend_workspace_bytes(ctx->sh, ctx->tb, batch));
   return w;

@@ -92,8 +92,8 @@ struct SelectArgs {
   int top_k;
   float top_k_frac;
   float *score_ws;                // global score rows when they do not fit on chip
-  uint32_t *flags;                // [batch * n_ret] streaming top-k misses
-  void *topk_ws;                  // streaming top-k scratch (histograms, buffers)
+  uint32_t *flags;                // [batch * n_ret] streaming selection misses
+  void *topk_ws;                  // streaming selection scratch (histograms, buffers, bitmaps)
   unsigned *err;
   int batch;
 };
@@ -101,9 +101,12 @@ struct SelectArgs {
 size_t select_workspace_bytes(const Shape &sh, const Tables &tb, int batch, size_t *flags_off);
 size_t select_topk_offset(const Shape &sh, const Tables &tb, int batch);
 cudaError_t launch_select(const SelectArgs &a, const Shape &sh, const Tables &tb, cudaStream_t st);
-size_t topk_workspace_bytes(const Shape &sh, const Tables &tb, int batch);
-cudaError_t launch_select_topk_stream(const SelectArgs &a, const Shape &sh, const Tables &tb, uint32_t *fail,
-                                      void *ws_base, cudaStream_t st, bool *used);
+// Streaming selection (top-k and top-p): workspace bytes for a batch (0 when
+// the shapes are outside what it handles), and its launches; *used = false
+// when it did not run and the exact selector must take every item.
+size_t stream_workspace_bytes(const Shape &sh, const Tables &tb, int batch, int mode);
+cudaError_t launch_select_stream(const SelectArgs &a, const Shape &sh, const Tables &tb, uint32_t *fail,
+                                 void *ws_base, cudaStream_t st, bool *used);
 
 struct AttendArgs {
   const uint16_t *q;

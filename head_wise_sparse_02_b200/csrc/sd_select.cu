@@ -747,21 +747,18 @@ cudaError_t launch_select(const SelectArgs &a, const Shape &sh, const Tables &tb
     p.dyn_bytes = hist_bytes(group_rows(tb), topp);
   }
   const int items = a.batch * tb.n_ret;
-  if (!topp) {
-    bool used = false;
-    cudaError_t e = launch_select_topk_stream(a, sh, tb, a.flags, a.topk_ws, st, &used);
-    if (e != cudaSuccess) return e;
-    if (used) {
-      // exact recomputation of the items whose window missed (usually none)
-      const int gy = std::min(items, 16);
-      return p.smem ? dispatch_gr<false, true>(a, sh, tb, p, dev, st, a.flags, gy)
-                    : dispatch_gr<false, false>(a, sh, tb, p, dev, st, a.flags, gy);
-    }
-    return p.smem ? dispatch_gr<false, true>(a, sh, tb, p, dev, st, nullptr, items)
-                  : dispatch_gr<false, false>(a, sh, tb, p, dev, st, nullptr, items);
-  }
-  return p.smem ? dispatch_gr<true, true>(a, sh, tb, p, dev, st, nullptr, items)
-                : dispatch_gr<true, false>(a, sh, tb, p, dev, st, nullptr, items);
+  bool used = false;
+  cudaError_t e = launch_select_stream(a, sh, tb, a.flags, a.topk_ws, st, &used);
+  if (e != cudaSuccess) return e;
+  // after the streaming passes: exact recomputation of the items whose window
+  // missed (usually none); without them: every item
+  const uint32_t *flags = used ? a.flags : nullptr;
+  const int gy = used ? std::min(items, 16) : items;
+  if (topp)
+    return p.smem ? dispatch_gr<true, true>(a, sh, tb, p, dev, st, flags, gy)
+                  : dispatch_gr<true, false>(a, sh, tb, p, dev, st, flags, gy);
+  return p.smem ? dispatch_gr<false, true>(a, sh, tb, p, dev, st, flags, gy)
+                : dispatch_gr<false, false>(a, sh, tb, p, dev, st, flags, gy);
 }
 
 }  // namespace sd

@@ -1,0 +1,1295 @@
+// Streaming selection: top-k and top-p without a sort, in passes over the
+// index that no CTA waits on.
+//
+// RTPurbo page (gist.science/ar/paper/2605.16928), Methodology 2-3 and 5: the
+// tokens of a retrieval head are scored in the r = 16 index space; a fixed
+// top-k budget, or a dynamic top-p set (softmax mass of the index scores
+// accumulated from the top until it reaches p), is kept, and the threshold
+// comes from a histogram, without sorting.  ICS page
+// (gist.science/ar/paper/2605.24168), 2 and 3a: exact ("Oracle") top-k at ~2%
+// of the context.
+//
+// Every pass streams the index through per-warp cp.async rings (16 bytes per
+// lane, XOR-swizzled rows) and scores all heads of a KV group at once with
+// ldmatrix + mma.m16n8k16 (A = the 16 x 16 bf16 index page, B = the q~ terms).
+//
+// K0 window  one CTA per (sequence, KV group).  Computes q~ = c P_g^T q_pre
+//            (float64, rounded to float32, split exactly into three bf16
+//            terms) and scores a strided sample of <= 256 pages; from the
+//            sample it sets, per head, a score window [t_lo, t_hi): t_lo a
+//            sample quantile safely below the threshold, t_hi the sample
+//            maximum.  Zeroes the head's counters.
+//
+// top-k (three launches)
+//   K1 stream  many CTAs, each 512 pages of one (sequence, KV group): every
+//              score at or above t_lo goes, with its position, to a
+//              lane-private staging area in shared memory and from there, in
+//              batches, to a per-head buffer.  Most scores fail the single
+//              compare and cost nothing more.
+//   K2 resolve one CTA per (sequence, retrieval head): histograms the
+//              buffered scores over 512 bins of [t_lo, t_hi) (plus one bin for
+//              scores >= t_hi), scans from the top for the bin holding the
+//              k-th score and, while that bin holds many tokens, splits it
+//              into 512 sub-bins and scans again (three levels at most); ranks
+//              the tokens of the final bin exactly by (score desc, position
+//              asc), marks the selected positions in a bitmap of the context
+//              and writes them in ascending order.
+//
+// top-p (four launches; the softmax mass of a head is known only after a
+// whole pass, so the index is streamed twice)
+//   K1 mass    per chunk: the softmax weight w = 2^((s - t_hi) log2 e) of
+//              every score goes to a float64 sum (scores below t_lo) or to a
+//              1024-bin mass histogram of [t_lo, t_hi) plus one bin for scores
+//              >= t_hi, kept per CTA in shared memory and added to the head's
+//              histogram at the end.
+//   K1 cut     per chunk: every CTA derives the same cut bin from the head's
+//              histogram (the highest bin whose mass, with the mass above
+//              it, reaches p Z); tokens of higher bins go to a bitmap of the
+//              context, tokens of the cut bin to the head's candidate buffer.
+//   K2 resolve one CTA per (sequence, retrieval head): an exact radix search
+//              over the candidates' order keys (9 bits per level, float64
+//              mass per digit) finds the threshold score tau inside the cut
+//              bin; candidates >= tau join the bitmap, which is written out
+//              in ascending order.  Ties at tau are all kept.
+//
+// If the window misses (top-k: buffer overflow, k-th score outside the
+// window, too many tokens in the cut bin; top-p: the cut below t_lo, too many
+// candidates, a weight out of float range), K2 flags the work item and the
+// exact general kernel recomputes it.
+#include <cuda_bf16.h>
+
+#include <algorithm>
+#include <map>
+#include <mutex>
+
+#include "sd_internal.cuh"
+
+namespace sd {
+namespace {
+
+constexpr int kBins = 512;            // window histogram bins (+1 slot: scores >= t_hi)
+// K0: sampled pages per (sequence, group); the sample store is capped at 96 KB
+__host__ __device__ constexpr int sample_pages(int GR) { return GR <= 4 ? 256 : (GR == 8 ? 192 : 96); }
+constexpr int kSampleBins = 256;
+constexpr int kChunkPages = 512;      // K1: pages per CTA
+constexpr int kRing = 8;              // K1: pages in flight per warp (even); 4 CTAs per SM
+// K1: staged buffer entries per (lane, head block); an iteration adds <= 4
+__host__ __device__ constexpr int stage_lane(int GR) { return GR <= 4 ? 10 : (GR == 8 ? 8 : 5); }
+constexpr int kCap = 2048;            // K2: cut-bin tokens ranked exactly
+constexpr int kLevels = 3;            // K2: histogram levels (the cut bin is split again)
+constexpr int kRefine = 64;           // K2: a cut bin above this many tokens is split again
+constexpr int kPer2 = 16;             // K2: buffer entries held in registers per thread
+constexpr int kPageBytes = kPage * kIndexDim * 2;   // 512 B: one page of one KV head
+constexpr unsigned kFull = 0xFFFFFFFFu;
+// top-p window (K0): the sample's kExcl highest tokens are left out of its
+// mass estimate (one planted needle in the sample must not make the mass look
+// concentrated); the mass below t_lo is estimated kMassSafety times over; the
+// count above t_lo gets kCountSigmas standard deviations (plus 8) of margin
+constexpr int kExcl = 8;
+constexpr double kMassSafety = 2.0;
+constexpr double kCountSigmas = 6.0;
+constexpr int kBinsP = 1024;          // top-p window bins (+1 slot: scores >= t_hi); 32 per lane of a warp
+constexpr int kCapP = 4096;           // top-p: cut-bin candidates per head
+constexpr float kLog2e = 1.4426950408889634f;
+// top-p: a score this far above t_hi (nats) is flagged, so that no float
+// weight, nor a chunk's float sum of up to 512 x 16 x 16 of them, overflows
+constexpr float kMaxLogit = 60.0f;
+
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%10,%10,%10};\n"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.0f));
+}
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
+// byte offset of the 16-byte half `half` of row `row` inside a staged page;
+// halves of rows 4-7 and 12-15 are swapped so that the eight rows an ldmatrix
+// phase reads fall in distinct banks
+__device__ __forceinline__ uint32_t page_off(int row, int half) {
+  return (uint32_t)(row * 32 + ((half ^ ((row >> 2) & 1)) << 4));
+}
+__device__ __forceinline__ uint16_t bf16_rn(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
+__device__ __forceinline__ float bf16_val(uint16_t h) { return __uint_as_float(uint32_t(h) << 16); }
+
+// class of a score in the window of its head: kBins for scores >= t_hi, else
+// the linear bin of [t_lo, t_hi); the same arithmetic in K1 and K2
+template <int NB = kBins>
+__device__ __forceinline__ int window_bin(float s, float tlo, float thi, float inv) {
+  if (s >= thi) return NB;
+  return min(NB - 1, max(0, __float2int_rz((s - tlo) * inv)));
+}
+
+// One warp: the highest bin c of hist[0, nb) (nb a multiple of 32, at most
+// 1024) whose suffix count sum_{b >= c} hist[b] reaches need (need >= 1);
+// -1 when the whole histogram holds fewer.  *above = sum_{b > c} hist[b],
+// *count = hist[c].  Each lane first sums its own nb / 32 consecutive bins,
+// one suffix scan over the 32 group totals picks the group, a second one
+// inside the group picks the bin.
+__device__ int warp_cut_bin(const uint32_t *hist, int nb, uint32_t need, int lane, uint32_t *above,
+                            uint32_t *count) {
+  const int G = nb >> 5;
+  uint32_t tot = 0;
+  for (int j = 0; j < G; ++j) tot += hist[lane * G + j];
+  uint32_t suf = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_down_sync(kFull, suf, o);
+    if (lane + o < 32) suf += y;
+  }
+  const unsigned bal = __ballot_sync(kFull, suf >= need);
+  if (!bal) return -1;
+  const int grp = 31 - __clz(bal);
+  const uint32_t acc = __shfl_sync(kFull, suf - tot, grp);     // bins of the groups above grp
+  const uint32_t c = lane < G ? hist[grp * G + lane] : 0u;
+  uint32_t s2 = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_down_sync(kFull, s2, o);
+    if (lane + o < 32) s2 += y;
+  }
+  const unsigned bal2 = __ballot_sync(kFull, lane < G && acc + s2 >= need);
+  const int j = 31 - __clz(bal2);                              // bal2 != 0: the group reaches need
+  *count = __shfl_sync(kFull, c, j);
+  *above = acc + __shfl_sync(kFull, s2, j) - *count;
+  return grp * G + j;
+}
+
+// One warp, float64 masses: the cut bin of a top-p head.  hist[0, kBinsP)
+// holds the mass of the window's bins, hist[kBinsP] that of scores >= t_hi,
+// zlo that of scores below t_lo.  Returns the highest bin c whose mass plus
+// the mass above it reaches need = p Z (kBinsP when the top bin alone does),
+// with *above = the mass strictly above c; -1 when the window's bins together
+// fall short (the threshold lies below t_lo).  Every step is a fixed sequence
+// of shuffles, so every caller reading the same histogram gets the same bin.
+__device__ int warp_cut_mass(const double *hist, double zlo, double p, int lane, double *above, double *need) {
+  constexpr int G = kBinsP / 32;
+  double tot = 0.0;
+  for (int j = 0; j < G; ++j) tot += hist[lane * G + j];
+  double zw = tot;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) zw += __shfl_xor_sync(kFull, zw, o);   // the same on every lane
+  const double top = hist[kBinsP];
+  const double nd = p * ((zlo + zw) + top);
+  *need = nd;
+  *above = 0.0;
+  if (top >= nd) return kBinsP;
+  const double n2 = nd - top;
+  double suf = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double y = __shfl_down_sync(kFull, suf, o);
+    if (lane + o < 32) suf += y;
+  }
+  const unsigned bal = __ballot_sync(kFull, suf >= n2);
+  if (!bal) return -1;
+  const int grp = 31 - __clz(bal);
+  const double acc = __shfl_sync(kFull, suf - tot, grp);
+  const double c = lane < G ? hist[grp * G + lane] : 0.0;
+  double s2 = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double y = __shfl_down_sync(kFull, s2, o);
+    if (lane + o < 32) s2 += y;
+  }
+  unsigned bal2 = __ballot_sync(kFull, lane < G && acc + s2 >= n2);
+  // summed in another order the group may fall short by a rounding: its
+  // lowest bin with mass then
+  if (!bal2) {
+    const unsigned nz = __ballot_sync(kFull, lane < G && c > 0.0);
+    bal2 = nz & (0u - nz);
+  }
+  const int j = bal2 ? 31 - __clz(bal2) : 0;
+  *above = top + acc + __shfl_sync(kFull, s2, j) - __shfl_sync(kFull, c, j);
+  return grp * G + j;
+}
+
+struct StreamWs {
+  uint32_t *qsplit;                   // [rows][24]: bf16 pairs of the q~ terms hi, mid, lo
+  float4 *win;                        // [rows]: t_lo, t_hi, 1 / bin width, unused
+  uint32_t *bcount;                   // [rows] buffer entries written
+  int *rowitem;                       // [rows] work item of the row
+  unsigned long long *buf;            // [rows][cap]: order key << 32 | position
+  uint32_t *fail;                     // [items] flags, [1] count, [items] list of flagged items
+  double *hist;                       // top-p: [rows][kBinsP + 1] softmax mass per window bin
+  double *zlo;                        // top-p: [rows] softmax mass below t_lo
+  uint32_t *rflag;                    // top-p: [rows] nonzero: the window cannot resolve the row
+  uint32_t *bits;                     // top-p: [rows][bwords] tokens above the cut bin
+  long long bwords;
+  int items;
+  int cap;
+};
+
+// B fragments of mma.m16n8k16 for head block hb: column n = gq of the first
+// MMA carries head 4hb + gq/2, term gq%2 (hi, mid); of the second, the lo term
+// for even gq and zero for odd gq.
+struct BFrag {
+  uint32_t v[2][2];
+};
+__device__ __forceinline__ BFrag load_bfrag(const uint32_t *qs /* [16 heads][24] */, int hb, int gq, int tq) {
+  const int head = hb * 4 + (gq >> 1);
+  const int part = gq & 1;
+  const uint32_t *q = qs + head * 24;
+  BFrag f;
+  f.v[0][0] = q[part * 8 + tq];
+  f.v[0][1] = q[part * 8 + tq + 4];
+  f.v[1][0] = part == 0 ? q[16 + tq] : 0u;
+  f.v[1][1] = part == 0 ? q[16 + tq + 4] : 0u;
+  return f;
+}
+template <int HB>
+__device__ __forceinline__ void score_frag(const uint32_t (&af)[4], const BFrag (&bf)[HB], float (&out)[HB][2]) {
+#pragma unroll
+  for (int hb = 0; hb < HB; ++hb) {
+    float d[4], e[4];
+    mma_16816(d, af, bf[hb].v[0][0], bf[hb].v[0][1]);
+    mma_16816(e, af, bf[hb].v[1][0], bf[hb].v[1][1]);
+    out[hb][0] = (d[0] + d[1]) + e[0];               // row gq
+    out[hb][1] = (d[2] + d[3]) + e[2];               // row gq + 8
+  }
+}
+
+__device__ __forceinline__ long long topk_budget(const SelectArgs &a, long long N) {
+  long long kb = a.top_k > 0 ? (long long)a.top_k
+                             : std::max(1LL, (long long)floor((double)a.top_k_frac * (double)N));
+  return std::min(kb, N);
+}
+
+// ------------------------------------------------------------------- K0
+constexpr int kT0 = 512;
+
+// t_lo of a top-p head from its sample (one warp): m valid sample tokens out
+// of N, cnt / mass the sample's histograms over kSampleBins bins of [lo, hi]
+// (mass relative to the sample maximum hi).  The mass below a bin edge t is
+// estimated as (N / m) x the sample's mass below t; the total as that scaled
+// mass up to the bin of the kExcl-th highest sample token plus the mass above
+// it unscaled (heavy sampled tokens are real but need not be typical).  t_lo
+// is the highest edge whose estimated mass below, taken kMassSafety times,
+// stays within (1 - p) of the total, lowered further to hold kCountSigmas
+// standard deviations (plus 8) more sample tokens; the sample minimum when
+// that asks for more tokens than the sample has.
+__device__ float topp_window_lo(const uint32_t *cnt, const float *mass, float lo, float hi, long long m,
+                                long long N, double p, int lane) {
+  constexpr int PB = kSampleBins / 32;               // bins per lane
+  uint32_t above, ncut;
+  int cx = warp_cut_bin(cnt, kSampleBins, (uint32_t)kExcl, lane, &above, &ncut);
+  if (cx < 0) cx = 0;
+  double lm[PB];
+  double tot = 0.0;
+#pragma unroll
+  for (int j = 0; j < PB; ++j) {
+    lm[j] = (double)mass[lane * PB + j];
+    tot += lm[j];
+  }
+  double incl = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double y = __shfl_up_sync(kFull, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const double before = incl - tot;                  // mass of the bins below this lane's
+  const double total = __shfl_sync(kFull, incl, 31);
+  double upto = 0.0, run = before;
+#pragma unroll
+  for (int j = 0; j < PB; ++j) {
+    run += lm[j];
+    if (lane * PB + j == cx) upto = run;             // mass of bins <= cx
+  }
+  upto = __shfl_sync(kFull, upto, cx / PB);
+  const double sc = (double)N / (double)m;
+  const double thr = (1.0 - p) * (sc * upto + (total - upto));
+  int best = 0;
+  run = before;
+#pragma unroll
+  for (int j = 0; j < PB; ++j) {
+    const int c = lane * PB + j;
+    if (c <= cx && sc * run * kMassSafety <= thr) best = c;
+    run += lm[j];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) best = max(best, __shfl_xor_sync(kFull, best, o));
+  uint32_t cc = 0;
+#pragma unroll
+  for (int j = 0; j < PB; ++j)
+    if (lane * PB + j >= best) cc += cnt[lane * PB + j];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cc += __shfl_xor_sync(kFull, cc, o);
+  const double r = ceil((double)cc + kCountSigmas * sqrt((double)cc) + 8.0);
+  if (r >= (double)m) return lo;
+  const int c = warp_cut_bin(cnt, kSampleBins, (uint32_t)r, lane, &above, &ncut);
+  return lo + (float)(c < 0 ? 0 : c) * ((hi - lo) / (float)kSampleBins);
+}
+
+// keep every token: an empty context, k_b >= N_b (top-k) or p >= 1 (top-p)
+template <bool TOPP>
+__device__ __forceinline__ bool keeps_all(const SelectArgs &a, long long N) {
+  if (N == 0) return true;
+  if constexpr (TOPP) return a.top_p >= 1.0f;
+  else return topk_budget(a, N) >= N;
+}
+
+template <int GR, bool TOPP>
+__global__ void __launch_bounds__(kT0)
+window_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__ groups, int n_groups,
+              const StreamWs ws) {
+  constexpr int HB = (GR + 3) / 4;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gq = lane >> 2, tq = lane & 3;
+  const int item = blockIdx.x;
+  const int b = item / n_groups, gi = item % n_groups;
+  constexpr int SP = sample_pages(GR);
+  __shared__ Group grp;
+  __shared__ uint32_t qs[16 * 24];
+  __shared__ uint32_t smax[GR], smin[GR];
+  __shared__ float hlo[GR], hinv[GR], hhi[GR];
+  __shared__ int spage[SP];
+  extern __shared__ __align__(16) unsigned char dyn0[];
+  float (*sample)[SP * 16] = reinterpret_cast<float (*)[SP * 16]>(dyn0);
+  uint32_t (*shist)[kSampleBins] = reinterpret_cast<uint32_t (*)[kSampleBins]>(dyn0 + (size_t)GR * SP * 16 * 4);
+  // top-p: softmax mass of the sample per bin, relative to the sample maximum
+  float (*smass)[kSampleBins] =
+      reinterpret_cast<float (*)[kSampleBins]>(dyn0 + (size_t)GR * SP * 16 * 4 + (size_t)GR * kSampleBins * 4);
+  if (tid == 0) grp = groups[gi];
+  __syncthreads();
+  const int nr = grp.n, g = grp.kv_head;
+  long long N = a.seq_lens[b];
+  N = N < 0 ? 0 : std::min<long long>(N, sh.max_len);
+  const long long kb = TOPP ? 0 : topk_budget(a, N);
+  if (tid == 0) {
+    ws.fail[item] = 0u;
+    if (item == 0) ws.fail[ws.items] = 0u;           // count of flagged items
+  }
+  if (tid < nr) {
+    const long long row = (long long)b * sh.H_ret + grp.row[tid];
+    ws.bcount[row] = 0u;
+    ws.rowitem[row] = item;
+    if constexpr (TOPP) {
+      ws.zlo[row] = 0.0;
+      ws.rflag[row] = 0u;
+    }
+  }
+  if constexpr (TOPP) {
+    for (int o = tid; o < nr * (kBinsP + 1); o += kT0)
+      ws.hist[((long long)b * sh.H_ret + grp.row[o / (kBinsP + 1)]) * (kBinsP + 1) + o % (kBinsP + 1)] = 0.0;
+  }
+  if (keeps_all<TOPP>(a, N)) return;                 // K1 skips, K2 keeps everything
+
+  // q~ in float64 (one warp per head, lanes split d) -> float32 -> hi/mid/lo
+  for (int i = warp; i < 16; i += kT0 / 32) {
+    double acc[kIndexDim];
+#pragma unroll
+    for (int j = 0; j < kIndexDim; ++j) acc[j] = 0.0;
+    if (i < nr) {
+      const uint16_t *qrow = a.q_pre + ((long long)b * sh.Hq + grp.q_head[i]) * sh.d;
+      const uint16_t *P = a.proj + (long long)g * sh.d * kIndexDim;
+      for (int e = lane; e < sh.d; e += 32) {
+        const double qe = (double)bf16_to_f32(qrow[e]);
+        const uint4 p0 = __ldg(reinterpret_cast<const uint4 *>(P + e * kIndexDim));
+        const uint4 p1 = __ldg(reinterpret_cast<const uint4 *>(P + e * kIndexDim + 8));
+        const uint32_t pw[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          acc[2 * j] = fma(qe, (double)bf16_lo(pw[j]), acc[2 * j]);
+          acc[2 * j + 1] = fma(qe, (double)bf16_hi(pw[j]), acc[2 * j + 1]);
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kIndexDim; ++j)
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc[j] += __shfl_xor_sync(kFull, acc[j], o);
+    if (lane < kIndexDim) {
+      double v = 0.0;
+#pragma unroll
+      for (int j = 0; j < kIndexDim; ++j) v = (lane == j) ? acc[j] : v;
+      const float x = (float)(v * (double)a.index_scale);
+      const uint16_t hi = bf16_rn(x);
+      const float r1 = x - bf16_val(hi);             // exact in float32
+      const uint16_t mid = bf16_rn(r1);
+      const uint16_t lo = bf16_rn(r1 - bf16_val(mid));
+      uint16_t *q16 = reinterpret_cast<uint16_t *>(qs + i * 24);
+      q16[lane] = hi;
+      q16[16 + lane] = mid;
+      q16[32 + lane] = lo;
+    }
+  }
+  if (tid < GR) {
+    smax[tid] = 0u;
+    smin[tid] = 0xFFFFFFFFu;
+  }
+  for (int o = tid; o < GR * kSampleBins; o += kT0) {
+    (&shist[0][0])[o] = 0u;
+    if constexpr (TOPP) (&smass[0][0])[o] = 0.0f;
+  }
+  __syncthreads();
+  for (int o = tid; o < nr * 24; o += kT0)           // publish the q~ terms for K1
+    ws.qsplit[((long long)b * sh.H_ret + grp.row[o / 24]) * 24 + o % 24] = qs[o];
+
+  // sample: pages j * st, j < ns; their page ids first, all at once
+  const int pages = (int)((N + kPage - 1) / kPage);
+  int st = 1;
+  while ((long long)st * SP < pages) st <<= 1;
+  const int ns = (pages + st - 1) / st;
+  const int32_t *pt = a.page_table + (long long)b * sh.max_pages;
+  for (int j = tid; j < ns; j += kT0) {
+    const int page = pt[j * st];
+    const bool ok = page >= 0 && page < sh.num_pages;
+    spage[j] = ok ? page : -1;
+    if (!ok) raise_error(a.err, SD_EBIT_PAGE);
+  }
+  __syncthreads();
+  BFrag bf[HB];
+#pragma unroll
+  for (int hb = 0; hb < HB; ++hb) bf[hb] = load_bfrag(qs, hb, gq, tq);
+  const uint16_t *icache = a.index_cache + (long long)g * (kPage * kIndexDim);
+  const long long page_stride = (long long)sh.Hkv * (kPage * kIndexDim);
+  float smx[HB], smn[HB];
+#pragma unroll
+  for (int hb = 0; hb < HB; ++hb) {
+    smx[hb] = -INFINITY;
+    smn[hb] = INFINITY;
+  }
+  constexpr int U = 16;
+  for (int j0 = warp; j0 < ns; j0 += (kT0 / 32) * U) {
+    uint32_t af[U][4];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int j = j0 + u * (kT0 / 32);
+      af[u][0] = af[u][1] = af[u][2] = af[u][3] = 0u;
+      const int page = j < ns ? spage[j] : -1;
+      if (page >= 0) {
+        const uint32_t *pg = reinterpret_cast<const uint32_t *>(icache + page * page_stride);
+        af[u][0] = __ldg(pg + gq * 8 + tq);
+        af[u][1] = __ldg(pg + (gq + 8) * 8 + tq);
+        af[u][2] = __ldg(pg + gq * 8 + tq + 4);
+        af[u][3] = __ldg(pg + (gq + 8) * 8 + tq + 4);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int j = j0 + u * (kT0 / 32);
+      if (j >= ns) break;
+      const bool ok = spage[j] >= 0;
+      float sc[HB][2];
+      score_frag<HB>(af[u], bf, sc);
+#pragma unroll
+      for (int hb = 0; hb < HB; ++hb) {
+        const int h = hb * 4 + tq;
+        if (h >= GR) continue;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const int row = gq + 8 * r;
+          const bool valid = ok && (long long)j * st * kPage + row < N;
+          const float v = valid ? sc[hb][r] : -INFINITY;
+          sample[h][j * 16 + row] = v;
+          if (valid) {
+            smx[hb] = fmaxf(smx[hb], v);
+            smn[hb] = fminf(smn[hb], v);
+          }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int hb = 0; hb < HB; ++hb) {
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      smx[hb] = fmaxf(smx[hb], __shfl_xor_sync(kFull, smx[hb], o));
+      smn[hb] = fminf(smn[hb], __shfl_xor_sync(kFull, smn[hb], o));
+    }
+    const int h = hb * 4 + tq;
+    if (gq == 0 && h < nr && smx[hb] > -INFINITY) {
+      atomicMax(&smax[h], order_key(smx[hb]));
+      atomicMin(&smin[h], order_key(smn[hb]));
+    }
+  }
+  __syncthreads();
+  if (tid < nr) {
+    const float lo = key_to_float(smin[tid]), hi = key_to_float(smax[tid]);
+    hlo[tid] = lo;
+    hhi[tid] = hi;
+    hinv[tid] = (smax[tid] != 0u && hi > lo) ? (float)kSampleBins / (hi - lo) : 0.0f;
+  }
+  __syncthreads();
+  for (int o = tid; o < nr * ns * 16; o += kT0) {
+    const int h = o / (ns * 16), r = o % (ns * 16);
+    const float v = sample[h][r];
+    if (v == -INFINITY) continue;
+    const int bin = std::min(kSampleBins - 1, std::max(0, __float2int_rz((v - hlo[h]) * hinv[h])));
+    atomicAdd(&shist[h][bin], 1u);
+    if constexpr (TOPP) atomicAdd(&smass[h][bin], exp2f((v - hhi[h]) * kLog2e));
+  }
+  __syncthreads();
+  // one warp per head: the highest bin whose suffix count reaches r
+  for (int h = warp; h < nr; h += kT0 / 32) {
+    // valid sample tokens: every sampled page is full except possibly the last
+    const long long m = (long long)(ns - 1) * kPage + std::min<long long>(kPage, N - (long long)(ns - 1) * st * kPage);
+    const long long row = (long long)b * sh.H_ret + grp.row[h];
+    if constexpr (TOPP) {
+      // no valid sample token (bad page ids): nothing is binned, K2 flags the row
+      float tlo = INFINITY, thi = 0.0f;
+      if (smax[h] != 0u) {
+        thi = hhi[h];
+        tlo = topp_window_lo(shist[h], smass[h], hlo[h], thi, m, N, (double)a.top_p, lane);
+      } else if (lane == 0) {
+        ws.rflag[row] = 1u;
+      }
+      const float inv = thi > tlo ? (float)kBinsP / (thi - tlo) : 0.0f;
+      if (lane == 0) ws.win[row] = make_float4(tlo, thi, inv, 0.0f);
+      continue;
+    }
+    float tlo = -INFINITY, thi = INFINITY;
+    if (smax[h] != 0u) {
+      const float lo = hlo[h], hi = key_to_float(smax[h]);
+      thi = hi;
+      const double mu = (double)m * (double)kb / (double)N;
+      const double r = ceil(mu + 6.0 * sqrt(mu) + 8.0);
+      if (r < (double)m) {
+        uint32_t above, cnt;
+        const int c = warp_cut_bin(shist[h], kSampleBins, (uint32_t)r, lane, &above, &cnt);
+        const int blo = c < 0 ? 0 : c;
+        tlo = lo + (float)blo * ((hi - lo) / (float)kSampleBins);
+      }
+    }
+    const float inv = (tlo > -INFINITY && thi > tlo) ? (float)kBins / (thi - tlo) : 0.0f;
+    if (lane == 0) ws.win[row] = make_float4(tlo, thi, inv, 0.0f);
+  }
+}
+
+// ------------------------------------------------------------------- K1
+constexpr int kT1 = 256;
+constexpr int kW1 = kT1 / 32;
+
+// What a K1 launch does with each score.
+enum StreamMode { kStageTopk = 0, kMassTopp = 1, kCutTopp = 2 };
+
+// dynamic shared memory of a K1 launch: the rings, then the staging area
+// (kStageTopk, kCutTopp), the chunk's bitmap (kCutTopp) or the mass
+// histograms (kMassTopp)
+__host__ __device__ constexpr size_t stream_stage_bytes(int GR, int MODE) {
+  return MODE == kMassTopp ? 0 : (size_t)kW1 * ((GR + 3) / 4) * stage_lane(GR) * 32 * 8;
+}
+__host__ __device__ constexpr size_t stream_smem_bytes(int GR, int MODE) {
+  return (size_t)kW1 * kRing * kPageBytes + stream_stage_bytes(GR, MODE) +
+         (MODE == kMassTopp ? (size_t)GR * (kBinsP + 1) * 4 : 0) +
+         (MODE == kCutTopp ? (size_t)GR * (kChunkPages / 2) * 4 : 0);
+}
+
+template <int GR, int MODE>
+__global__ void __launch_bounds__(kT1)
+stream_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__ groups, int n_groups,
+              const StreamWs ws) {
+  constexpr int HB = (GR + 3) / 4;
+  constexpr int SL = stage_lane(GR);
+  constexpr bool TOPP = MODE != kStageTopk;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gq = lane >> 2, tq = lane & 3;
+  // item fastest in the launch order: CTAs of all KV groups for the same
+  // chunk of pages run together, so reads of the groups' 512-byte slices of a
+  // page (adjacent in the index cache) meet in the same DRAM rows
+  const int item = blockIdx.x;
+  const int b = item / n_groups, gi = item % n_groups;
+  extern __shared__ __align__(128) unsigned char dyn1[];
+  unsigned char (*ring)[kRing][kPageBytes] = reinterpret_cast<unsigned char (*)[kRing][kPageBytes]>(dyn1);
+  // lane-private staging: entry e of (warp, head block hb) for lane l at stage[warp][hb][e][l]
+  unsigned long long (*stage)[HB][SL][32] =
+      reinterpret_cast<unsigned long long (*)[HB][SL][32]>(dyn1 + (size_t)kW1 * kRing * kPageBytes);
+  unsigned char *tail = dyn1 + (size_t)kW1 * kRing * kPageBytes + stream_stage_bytes(GR, MODE);
+  // kMassTopp: per-head mass histograms; kCutTopp: per-head bitmap of the chunk
+  float (*shm)[kBinsP + 1] = reinterpret_cast<float (*)[kBinsP + 1]>(tail);
+  uint32_t (*sbits)[kChunkPages / 2] = reinterpret_cast<uint32_t (*)[kChunkPages / 2]>(tail);
+  __shared__ int32_t pt_s[kChunkPages];
+  __shared__ uint32_t qs[16 * 24];
+  __shared__ int cut_s[GR];
+  __shared__ Group grp;
+  if (tid == 0) grp = groups[gi];
+  __syncthreads();
+  const int nr = grp.n, g = grp.kv_head;
+  long long N = a.seq_lens[b];
+  N = N < 0 ? 0 : std::min<long long>(N, sh.max_len);
+  if (keeps_all<TOPP>(a, N)) return;
+  const int pages = (int)((N + kPage - 1) / kPage);
+  const int p0 = blockIdx.y * kChunkPages;
+  if (p0 >= pages) return;
+  const int np = pages - p0 < kChunkPages ? pages - p0 : kChunkPages;
+  {
+    // page id -> page * Hkv + g (the 512-byte index block of this KV head), or -1
+    const int32_t *pt = a.page_table + (long long)b * sh.max_pages + p0;
+    for (int o = tid; o < np; o += kT1) {
+      const int page = pt[o];
+      const bool ok = page >= 0 && page < sh.num_pages;
+      pt_s[o] = ok ? page * sh.Hkv + g : -1;
+      if (!ok) raise_error(a.err, SD_EBIT_PAGE);
+    }
+    for (int o = tid; o < 16 * 24; o += kT1) {
+      const int i = o / 24;
+      qs[o] = i < nr ? ws.qsplit[((long long)b * sh.H_ret + grp.row[i]) * 24 + o % 24] : 0u;
+    }
+    if constexpr (MODE == kMassTopp)
+      for (int o = tid; o < GR * (kBinsP + 1); o += kT1) (&shm[0][0])[o] = 0.0f;
+    if constexpr (MODE == kCutTopp) {
+      for (int o = tid; o < GR * (kChunkPages / 2); o += kT1) (&sbits[0][0])[o] = 0u;
+      // the cut bin of each head, from the mass pass (warp h, head h)
+      for (int h = warp; h < GR; h += kW1) {
+        int c = kBinsP + 1;                          // absent heads: nothing is above the cut
+        if (h < nr) {
+          const long long row = (long long)b * sh.H_ret + grp.row[h];
+          double above, need;
+          c = warp_cut_mass(ws.hist + row * (kBinsP + 1), ws.zlo[row], (double)a.top_p, lane, &above, &need);
+          if (c < 0) c = kBinsP + 1;                 // the threshold lies below t_lo: K2 flags the row
+        }
+        if (lane == 0) cut_s[h] = c;
+      }
+    }
+  }
+  __syncthreads();
+
+  // per-warp ring: this warp reads pages warp, warp + 8, ... of the chunk
+  const uint32_t ring_base = (uint32_t)__cvta_generic_to_shared(&ring[warp][0][0]);
+  const unsigned char *iblk = reinterpret_cast<const unsigned char *>(a.index_cache) + lane * 16;
+  const uint32_t st_off = page_off(lane >> 1, lane & 1);
+  const int nq = np > warp ? (np - warp + kW1 - 1) / kW1 : 0;
+  auto issue = [&](int q) {
+    if (q < nq) {
+      const int blk = pt_s[warp + q * kW1];
+      cp_async16(ring_base + (q % kRing) * kPageBytes + st_off, iblk + (size_t)(blk >= 0 ? blk : 0) * kPageBytes,
+                 blk >= 0 ? 16 : 0);
+    }
+    cp_async_commit();
+  };
+#pragma unroll
+  for (int q = 0; q < kRing; ++q) issue(q);
+
+  BFrag bf[HB];
+  float tlo[HB], thi[HB], inv[HB];
+  int cut[HB];
+  double zl[HB];                                     // kMassTopp: this lane's mass below t_lo
+  long long row_of[HB];
+#pragma unroll
+  for (int hb = 0; hb < HB; ++hb) {
+    bf[hb] = load_bfrag(qs, hb, gq, tq);
+    const int h = hb * 4 + tq;
+    row_of[hb] = h < nr ? (long long)b * sh.H_ret + grp.row[h] : 0;
+    const float4 wv = h < nr ? ws.win[row_of[hb]] : make_float4(INFINITY, 0.0f, 0.0f, 0.0f);
+    tlo[hb] = wv.x;                                  // absent heads keep nothing
+    thi[hb] = wv.y;
+    inv[hb] = wv.z;
+    cut[hb] = MODE == kCutTopp && h < GR ? cut_s[h] : 0;
+    zl[hb] = 0.0;
+  }
+  bool wide = false;                                 // kMassTopp: a weight beyond float range
+  uint32_t cnt[HB];
+#pragma unroll
+  for (int hb = 0; hb < HB; ++hb) cnt[hb] = 0u;
+  // move the warp's staged entries to the heads' buffers: the 8 lanes of a
+  // head (same tq) take consecutive ranges of one reservation
+  auto flush = [&]() {
+#pragma unroll
+    for (int hb = 0; hb < HB; ++hb) {
+      const int h = hb * 4 + tq;
+      uint32_t incl = cnt[hb];
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const uint32_t tot = __shfl_sync(kFull, incl, 28 + tq);
+      uint32_t base = 0u;
+      if (gq == 0 && h < nr && tot > 0u) base = atomicAdd(&ws.bcount[row_of[hb]], tot);
+      base = __shfl_sync(kFull, base, tq) + (incl - cnt[hb]);
+      if (h < nr) {
+        unsigned long long *dst = ws.buf + row_of[hb] * ws.cap;
+        for (uint32_t e = 0; e < cnt[hb]; ++e)
+          if (base + e < (uint32_t)ws.cap) dst[base + e] = stage[warp][hb][e][lane];
+      }
+      cnt[hb] = 0u;
+    }
+    __syncwarp();
+  };
+  const uint32_t ld = ring_base + page_off((lane & 7) + ((lane >> 3) & 1) * 8, lane >> 4);
+  const uint32_t n32 = (uint32_t)N;
+  // two pages per iteration (q, q + 1); one cp.async group per page
+  for (int q = 0; q < nq; q += 2) {
+    cp_async_wait<kRing - 2>();
+    __syncwarp();
+    uint32_t af[2][4];
+    ldmatrix_x4(af[0], ld + (q % kRing) * kPageBytes);
+    ldmatrix_x4(af[1], ld + ((q + 1) % kRing) * kPageBytes);
+    __syncwarp();
+    const int pl = warp + q * kW1;                   // page within the chunk
+    const bool ok0 = pt_s[pl] >= 0;
+    const bool ok1 = q + 1 < nq && pt_s[pl + kW1] >= 0;
+    issue(q + kRing);
+    issue(q + kRing + 1);
+    float sc[2][HB][2];
+    score_frag<HB>(af[0], bf, sc[0]);
+    score_frag<HB>(af[1], bf, sc[1]);
+    const uint32_t pos0 = (uint32_t)(p0 + pl) * kPage + gq;
+    bool full = false;
+#pragma unroll
+    for (int hb = 0; hb < HB; ++hb) {
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const uint32_t pos = pos0 + u * (kW1 * kPage) + 8 * r;
+          const float s = sc[u][hb][r];
+          const bool valid = (u ? ok1 : ok0) && pos < n32;
+          if constexpr (MODE == kStageTopk) {
+            if (valid && s >= tlo[hb]) {
+              stage[warp][hb][cnt[hb]][lane] = ((unsigned long long)order_key(s) << 32) | pos;
+              ++cnt[hb];
+            }
+          } else if constexpr (MODE == kMassTopp) {
+            const int h = hb * 4 + tq;
+            if (valid && h < nr) {
+              const float w = exp2f((s - thi[hb]) * kLog2e);
+              wide |= s - thi[hb] > kMaxLogit;
+              if (s < tlo[hb]) zl[hb] += (double)w;
+              else atomicAdd(&shm[h][window_bin<kBinsP>(s, tlo[hb], thi[hb], inv[hb])], w);
+            }
+          } else {
+            if (valid && hb * 4 + tq < nr && s >= tlo[hb]) {
+              const int bin = window_bin<kBinsP>(s, tlo[hb], thi[hb], inv[hb]);
+              if (bin > cut[hb]) {
+                const uint32_t loc = pos - (uint32_t)p0 * kPage;
+                atomicOr(&sbits[hb * 4 + tq][loc >> 5], 1u << (pos & 31));
+              } else if (bin == cut[hb]) {
+                stage[warp][hb][cnt[hb]][lane] = ((unsigned long long)order_key(s) << 32) | pos;
+                ++cnt[hb];
+              }
+            }
+          }
+        }
+      }
+      full |= cnt[hb] > (uint32_t)(SL - 4);
+    }
+    if constexpr (MODE != kMassTopp)
+      if (__any_sync(kFull, full)) flush();
+  }
+  if constexpr (MODE != kMassTopp) flush();
+  cp_async_wait<0>();
+  if constexpr (MODE == kMassTopp) {
+    // the chunk's masses join the heads' histograms; the lanes of a head
+    // (same tq) sum their float64 masses below t_lo first
+#pragma unroll
+    for (int hb = 0; hb < HB; ++hb) {
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) zl[hb] += __shfl_xor_sync(kFull, zl[hb], o);
+      if (gq == 0 && hb * 4 + tq < nr && zl[hb] != 0.0) atomicAdd(&ws.zlo[row_of[hb]], zl[hb]);
+    }
+    // a weight out of float range: the item goes to the exact selector
+    if (__any_sync(kFull, wide) && lane == 0) atomicOr(&ws.rflag[(long long)b * sh.H_ret + grp.row[0]], 2u);
+    __syncthreads();
+    for (int o = tid; o < nr * (kBinsP + 1); o += kT1) {
+      const int h = o / (kBinsP + 1), bin = o % (kBinsP + 1);
+      const float v = shm[h][bin];
+      if (v != 0.0f) atomicAdd(&ws.hist[((long long)b * sh.H_ret + grp.row[h]) * (kBinsP + 1) + bin], (double)v);
+    }
+  }
+  if constexpr (MODE == kCutTopp) {
+    // the chunk's words of the heads' bitmaps (512 pages = 256 words; the
+    // chunk starts on a word boundary)
+    __syncthreads();
+    const int nw = (np + 1) / 2;
+    for (int o = tid; o < nr * nw; o += kT1) {
+      const int h = o / nw, w = o % nw;
+      ws.bits[((long long)b * sh.H_ret + grp.row[h]) * ws.bwords + p0 / 2 + w] = sbits[h][w];
+    }
+  }
+}
+
+// ------------------------------------------------------------------- K2
+constexpr int kT2 = 256;
+
+// Block-wide: the positions set in bitmap[0, words) go to out in ascending
+// order (contiguous word ranges per thread, block-wide prefix), their number
+// to sel_count[row].  wtot: kT2 / 32 words of shared memory.
+__device__ void write_ascending(const SelectArgs &a, const uint32_t *bitmap, int words, int32_t *out, long long row,
+                                uint32_t *wtot) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int wpt = (words + kT2 - 1) / kT2;
+  const int w0 = tid * wpt, w1 = std::min(words, w0 + wpt);
+  uint32_t c = 0;
+  for (int x = w0; x < w1; ++x) c += __popc(bitmap[x]);
+  uint32_t incl = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(kFull, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) wtot[warp] = incl;
+  __syncthreads();
+  uint32_t base = 0, total = 0;
+  for (int x = 0; x < kT2 / 32; ++x) {
+    if (x < warp) base += wtot[x];
+    total += wtot[x];
+  }
+  long long o = base + incl - c;
+  for (int x = w0; x < w1; ++x) {
+    uint32_t bits = bitmap[x];
+    while (bits) {
+      const int bit = __ffs(bits) - 1;
+      bits &= bits - 1;
+      if (o < a.sel_stride) out[o] = x * 32 + bit;
+      else raise_error(a.err, SD_EBIT_SEL);
+      ++o;
+    }
+  }
+  if (tid == 0) {
+    if ((long long)total > a.sel_stride) raise_error(a.err, SD_EBIT_SEL);
+    a.sel_count[row] = (int32_t)std::min<long long>(total, a.sel_stride);
+  }
+}
+
+// Block-wide: every position 0 .. N - 1 (a head that keeps all its tokens).
+__device__ void write_all(const SelectArgs &a, long long N, int32_t *out, long long row) {
+  for (long long t = threadIdx.x; t < N; t += kT2) {
+    if (t < a.sel_stride) out[t] = (int32_t)t;
+    else raise_error(a.err, SD_EBIT_SEL);
+  }
+  if (threadIdx.x == 0) a.sel_count[row] = (int32_t)std::min(N, a.sel_stride);
+}
+
+// K2 flags the work item of a row whose window missed (once per item).
+__device__ void flag_item(const StreamWs &ws, long long row) {
+  const int it = ws.rowitem[row];
+  if (atomicExch(&ws.fail[it], 1u) == 0u) ws.fail[ws.items + 1 + atomicAdd(&ws.fail[ws.items], 1u)] = (uint32_t)it;
+}
+
+__global__ void __launch_bounds__(kT2, 4)
+topk_resolve_kernel(const SelectArgs a, const Shape sh, const StreamWs ws) {
+  extern __shared__ uint32_t bitmap[];               // [max_len / 32]
+  __shared__ unsigned long long cand[kCap];
+  __shared__ uint32_t hist[kBins + 1];
+  __shared__ uint32_t n_cand;
+  __shared__ int fail_s, done_s;
+  __shared__ long long need_s;
+  __shared__ int cutv[kLevels];
+  __shared__ float llo[kLevels], linv[kLevels];
+  __shared__ uint32_t wtot[kT2 / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int b = blockIdx.y, hr = blockIdx.x;
+  const long long row = (long long)b * sh.H_ret + hr;
+  int32_t *out = a.sel_idx + row * a.sel_stride;
+  long long N = a.seq_lens[b];
+  N = N < 0 ? 0 : std::min<long long>(N, sh.max_len);
+  const long long kb = topk_budget(a, N);
+  if (N == 0 || kb >= N) {
+    write_all(a, N, out, row);
+    return;
+  }
+  const float4 w = ws.win[row];
+  const uint32_t nbuf = ws.bcount[row];
+  const unsigned long long *buf = ws.buf + row * ws.cap;
+  const int n = (int)std::min<uint32_t>(nbuf, (uint32_t)ws.cap);
+  const int words = (int)((N + 31) / 32);
+  for (int o = tid; o < words; o += kT2) bitmap[o] = 0u;
+  if (tid == 0) {
+    llo[0] = w.x;
+    linv[0] = w.z;
+    need_s = kb;
+    fail_s = 0;
+    done_s = 0;
+    n_cand = 0u;
+  }
+  // bin of a score at level L: level 0 is the window histogram (bin kBins:
+  // scores >= t_hi); level L > 0 splits the cut bin of level L - 1 into kBins
+  // linear sub-bins.  Bins are non-decreasing in the score at every level.
+  auto bin_at = [&](float v, int L) -> int {
+    if (L == 0) return window_bin(v, w.x, w.y, w.z);
+    return min(kBins - 1, max(0, __float2int_rz((v - llo[L]) * linv[L])));
+  };
+  // this thread's first kPer2 entries, loaded once (the passes below reread
+  // only entries past kPer2 * kT2 from memory)
+  unsigned long long ent[kPer2];
+#pragma unroll
+  for (int j = 0; j < kPer2; ++j) {
+    const int e = tid + j * kT2;
+    ent[j] = e < n ? buf[e] : 0ull;
+  }
+  // the cut bin: refine while it holds more than kRefine tokens
+  int L = 0;
+  for (; L < kLevels; ++L) {
+    for (int o = tid; o <= kBins; o += kT2) hist[o] = 0u;
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kPer2; ++j) {
+      const int e = tid + j * kT2;
+      if (e < n) {
+        const float v = key_to_float((uint32_t)(ent[j] >> 32));
+        bool play = true;
+        for (int l = 0; l < L; ++l) play = play && bin_at(v, l) == cutv[l];
+        if (play) atomicAdd(&hist[bin_at(v, L)], 1u);
+      }
+    }
+    for (int e = tid + kPer2 * kT2; e < n; e += kT2) {
+      const float v = key_to_float((uint32_t)(buf[e] >> 32));
+      bool play = true;
+      for (int l = 0; l < L; ++l) play = play && bin_at(v, l) == cutv[l];
+      if (play) atomicAdd(&hist[bin_at(v, L)], 1u);
+    }
+    __syncthreads();
+    // warp 0 finds the bin holding the cut among the level's bins
+    if (warp == 0) {
+      const long long need = need_s - (L == 0 ? (long long)hist[kBins] : 0LL);
+      uint32_t above = 0, ncut = 0;
+      const int cut = need > 0 ? warp_cut_bin(hist, kBins, (uint32_t)need, lane, &above, &ncut) : -1;
+      const long long acc = above;
+      if (lane == 0) {
+        if (need <= 0 || cut < 0 || nbuf > (uint32_t)ws.cap) {
+          fail_s = 1;
+        } else {
+          cutv[L] = cut;
+          need_s = need - acc;                       // tokens still to take from the cut bin
+          const bool last = ncut <= kRefine || L + 1 == kLevels;
+          if (last && ncut > kCap) fail_s = 1;
+          if (!last) {
+            llo[L + 1] = llo[L] + (float)cut / linv[L];
+            linv[L + 1] = linv[L] * (float)kBins;
+          }
+          done_s = last;
+        }
+      }
+    }
+    __syncthreads();
+    if (fail_s || done_s) break;
+  }
+  if (fail_s) {
+    if (tid == 0) flag_item(ws, row);
+    return;
+  }
+  const int nlev = L + 1;
+  // classify: above the cut path -> selected; on it -> candidate
+  auto classify = [&](unsigned long long en) {
+    const uint32_t key = (uint32_t)(en >> 32), pos = (uint32_t)en;
+    const float v = key_to_float(key);
+    int rel = 0;
+    for (int l = 0; l < nlev && rel == 0; ++l) {
+      const int bl = bin_at(v, l);
+      rel = bl > cutv[l] ? 1 : (bl < cutv[l] ? -1 : 0);
+    }
+    if (rel > 0) {
+      atomicOr(&bitmap[pos >> 5], 1u << (pos & 31));
+    } else if (rel == 0) {
+      const uint32_t at = atomicAdd(&n_cand, 1u);
+      if (at < (uint32_t)kCap) cand[at] = ((unsigned long long)(~key) << 32) | pos;   // ascending = better first
+    }
+  };
+#pragma unroll
+  for (int j = 0; j < kPer2; ++j)
+    if (tid + j * kT2 < n) classify(ent[j]);
+  for (int e = tid + kPer2 * kT2; e < n; e += kT2) classify(buf[e]);
+  __syncthreads();
+  // rank the cut bin exactly: the need_c best by (score desc, position asc)
+  const int nc = (int)std::min<uint32_t>(n_cand, (uint32_t)kCap);
+  const long long need_c = need_s;
+  for (int e = tid; e < nc; e += kT2) {
+    const unsigned long long me = cand[e];
+    int rk = 0;
+    for (int j = 0; j < nc; ++j) rk += cand[j] < me;
+    if (rk < need_c) {
+      const uint32_t pos = (uint32_t)me;
+      atomicOr(&bitmap[pos >> 5], 1u << (pos & 31));
+    }
+  }
+  __syncthreads();
+  write_ascending(a, bitmap, words, out, row, wtot);
+}
+
+// One warp, over kBins radix digits with counts and float64 masses: the
+// highest non-empty digit whose mass plus the mass above it reaches need
+// (need <= 0: the highest non-empty digit).  When rounding leaves every digit
+// short, the lowest non-empty digit (all of the level is kept).  *above = the
+// mass of the digits above the one returned.
+__device__ int warp_cut_digit(const uint32_t *cnt, const double *mass, double need, int lane, double *above) {
+  constexpr int G = kBins / 32;
+  double tot = 0.0;
+  uint32_t nz = 0u;
+  for (int j = 0; j < G; ++j) {
+    tot += mass[lane * G + j];
+    nz += cnt[lane * G + j];
+  }
+  double suf = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double y = __shfl_down_sync(kFull, suf, o);
+    if (lane + o < 32) suf += y;
+  }
+  const unsigned bal = __ballot_sync(kFull, nz > 0u && suf >= need);
+  const unsigned any = __ballot_sync(kFull, nz > 0u);
+  const int grp = bal ? 31 - __clz(bal) : (any ? __ffs(any) - 1 : 0);
+  const double acc = __shfl_sync(kFull, suf - tot, grp);
+  const uint32_t c = lane < G ? cnt[grp * G + lane] : 0u;
+  const double m = lane < G ? mass[grp * G + lane] : 0.0;
+  double s2 = m;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double y = __shfl_down_sync(kFull, s2, o);
+    if (lane + o < 32) s2 += y;
+  }
+  const unsigned bal2 = __ballot_sync(kFull, lane < G && c > 0u && acc + s2 >= need);
+  const unsigned any2 = __ballot_sync(kFull, lane < G && c > 0u);
+  const int j = bal2 ? 31 - __clz(bal2) : (any2 ? __ffs(any2) - 1 : 0);
+  *above = acc + __shfl_sync(kFull, s2, j) - __shfl_sync(kFull, m, j);
+  return grp * G + j;
+}
+
+// top-p K2: one CTA per (sequence, retrieval head).
+__global__ void __launch_bounds__(kT2, 4)
+topp_resolve_kernel(const SelectArgs a, const Shape sh, const StreamWs ws) {
+  extern __shared__ uint32_t bitmap[];               // [max_len / 32]
+  __shared__ unsigned long long cand[kCapP];
+  __shared__ uint32_t dcnt[kBins];
+  __shared__ double dmass[kBins];
+  __shared__ int fail_s;
+  __shared__ double need_s;
+  __shared__ uint32_t kmin_s, kmax_s, prefix_s;
+  __shared__ uint32_t wtot[kT2 / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int b = blockIdx.y, hr = blockIdx.x;
+  const long long row = (long long)b * sh.H_ret + hr;
+  int32_t *out = a.sel_idx + row * a.sel_stride;
+  long long N = a.seq_lens[b];
+  N = N < 0 ? 0 : std::min<long long>(N, sh.max_len);
+  if (keeps_all<true>(a, N)) {
+    write_all(a, N, out, row);
+    return;
+  }
+  const float thi = ws.win[row].y;
+  if (warp == 0) {
+    double above, need;
+    const int c = warp_cut_mass(ws.hist + row * (kBinsP + 1), ws.zlo[row], (double)a.top_p, lane, &above, &need);
+    if (lane == 0) {
+      fail_s = c < 0 || ws.rflag[row] != 0u || ws.bcount[row] > (uint32_t)ws.cap;
+      need_s = need - above;                         // mass still to take from the cut bin
+      kmin_s = 0xFFFFFFFFu;
+      kmax_s = 0u;
+      prefix_s = 0u;
+    }
+  }
+  __syncthreads();
+  if (fail_s) {
+    if (tid == 0) flag_item(ws, row);
+    return;
+  }
+  // the bitmap of the tokens above the cut bin, and the cut bin's candidates
+  const int words = (int)((N + 31) / 32);
+  const uint32_t *bits = ws.bits + row * ws.bwords;
+  for (int o = tid; o < words; o += kT2) bitmap[o] = bits[o];
+  const int n = (int)ws.bcount[row];
+  const unsigned long long *buf = ws.buf + row * ws.cap;
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+  for (int e = tid; e < n; e += kT2) {
+    const unsigned long long v = buf[e];
+    cand[e] = v;
+    lo = min(lo, (uint32_t)(v >> 32));
+    hi = max(hi, (uint32_t)(v >> 32));
+  }
+  if (lo != 0xFFFFFFFFu) {
+    atomicMin(&kmin_s, lo);
+    atomicMax(&kmax_s, hi);
+  }
+  __syncthreads();
+  if (n > 0) {
+    // exact radix search over the order keys' offsets from the smallest:
+    // the largest key whose suffix mass reaches need (9 bits per level)
+    const uint32_t kmin = kmin_s, span = kmax_s - kmin;
+    int rem = span ? 32 - __clz(span) : 0;           // offset bits not yet decided
+    const int top = rem;
+    uint32_t prefix = 0u;
+    double need = need_s;
+    while (rem > 0) {
+      const int sh2 = rem > 9 ? rem - 9 : 0;
+      for (int o = tid; o < kBins; o += kT2) {
+        dcnt[o] = 0u;
+        dmass[o] = 0.0;
+      }
+      __syncthreads();
+      for (int e = tid; e < n; e += kT2) {
+        const uint32_t key = (uint32_t)(cand[e] >> 32), off = key - kmin;
+        if (rem != top && (off >> rem) != prefix) continue;
+        const uint32_t d = (off >> sh2) & ((1u << (rem - sh2)) - 1u);
+        atomicAdd(&dcnt[d], 1u);
+        atomicAdd(&dmass[d], (double)exp2f((key_to_float(key) - thi) * kLog2e));
+      }
+      __syncthreads();
+      if (warp == 0) {
+        double above;
+        const int d = warp_cut_digit(dcnt, dmass, need, lane, &above);
+        if (lane == 0) {
+          need_s = need - above;
+          prefix_s = (prefix << (rem - sh2)) | (uint32_t)d;
+        }
+      }
+      __syncthreads();
+      need = need_s;
+      prefix = prefix_s;
+      rem = sh2;
+    }
+    const uint32_t tau = kmin + prefix;              // the threshold's key: every candidate >= it is kept
+    for (int e = tid; e < n; e += kT2) {
+      const unsigned long long v = cand[e];
+      if ((uint32_t)(v >> 32) >= tau) {
+        const uint32_t pos = (uint32_t)v;
+        atomicOr(&bitmap[pos >> 5], 1u << (pos & 31));
+      }
+    }
+  }
+  __syncthreads();
+  write_ascending(a, bitmap, words, out, row, wtot);
+}
+
+// ------------------------------------------------------------------- host
+struct StreamPlan {
+  int cap;
+  size_t bitmap_bytes;
+  long long bwords;                   // top-p bitmap words per row
+  bool ok;
+};
+
+StreamPlan stream_plan(const Shape &sh, const Tables &tb, int mode) {
+  StreamPlan p{};
+  p.cap = mode == SD_TOP_P ? kCapP
+                           : (int)std::min<long long>(sh.max_len, std::max<long long>(4096, sh.max_len / 8));
+  p.bitmap_bytes = (size_t)((sh.max_len + 31) / 32) * 4;
+  p.bwords = mode == SD_TOP_P ? ((long long)sh.max_pages + 1) / 2 : 0;
+  p.ok = tb.max_ret <= 16 && p.bitmap_bytes <= 160 * 1024 && sh.max_len < (1LL << 31);
+  return p;
+}
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+struct StreamLayout {
+  size_t qsplit, win, bcount, rowitem, buf, hist, zlo, rflag, bits, total;
+};
+
+StreamLayout stream_layout(const Shape &sh, int batch, const StreamPlan &p) {
+  StreamLayout L{};
+  const size_t rows = (size_t)batch * std::max(1, sh.H_ret);
+  size_t o = 0;
+  L.qsplit = o;  o = align256(o + rows * 24 * 4);
+  L.win = o;     o = align256(o + rows * 16);
+  L.bcount = o;  o = align256(o + rows * 4);
+  L.rowitem = o; o = align256(o + rows * 4);
+  L.buf = o;     o = align256(o + rows * (size_t)p.cap * 8);
+  if (p.bwords) {
+    L.hist = o;  o = align256(o + rows * (kBinsP + 1) * 8);
+    L.zlo = o;   o = align256(o + rows * 8);
+    L.rflag = o; o = align256(o + rows * 4);
+    L.bits = o;  o = align256(o + rows * (size_t)p.bwords * 4);
+  }
+  L.total = o;
+  return L;
+}
+
+// dynamic shared memory attributes, set once per kernel and device
+template <typename K>
+cudaError_t set_smem_once(K kern, size_t bytes) {
+  static std::mutex mu;
+  static std::map<std::pair<const void *, int>, size_t> done;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lk(mu);
+  const auto key = std::make_pair((const void *)kern, dev);
+  auto it = done.find(key);
+  if (it != done.end() && it->second >= bytes) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) done[key] = bytes;
+  return e;
+}
+
+template <int GR>
+cudaError_t stream_launch(const SelectArgs &a, const Shape &sh, const Tables &tb, const StreamWs &ws,
+                          size_t bitmap_bytes, cudaStream_t st) {
+  const bool topp = a.mode == SD_TOP_P;
+  const int items = a.batch * tb.n_ret;
+  const int chunks = (int)((sh.max_pages + kChunkPages - 1) / kChunkPages);
+  const dim3 g1(items, chunks), g2(sh.H_ret, a.batch);
+  const size_t smem0 = (size_t)GR * sample_pages(GR) * 16 * 4 + (size_t)GR * kSampleBins * 4 * (topp ? 2 : 1);
+  cudaError_t e;
+  if (!topp) {
+    const size_t smem1 = stream_smem_bytes(GR, kStageTopk);
+    e = set_smem_once(window_kernel<GR, false>, smem0);
+    if (e == cudaSuccess) e = set_smem_once(stream_kernel<GR, kStageTopk>, smem1);
+    if (e == cudaSuccess) e = set_smem_once(topk_resolve_kernel, bitmap_bytes);
+    if (e != cudaSuccess) return e;
+    window_kernel<GR, false><<<items, kT0, smem0, st>>>(a, sh, tb.ret, tb.n_ret, ws);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    stream_kernel<GR, kStageTopk><<<g1, kT1, smem1, st>>>(a, sh, tb.ret, tb.n_ret, ws);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    topk_resolve_kernel<<<g2, kT2, bitmap_bytes, st>>>(a, sh, ws);
+    return cudaGetLastError();
+  }
+  const size_t smem_m = stream_smem_bytes(GR, kMassTopp), smem_c = stream_smem_bytes(GR, kCutTopp);
+  e = set_smem_once(window_kernel<GR, true>, smem0);
+  if (e == cudaSuccess) e = set_smem_once(stream_kernel<GR, kMassTopp>, smem_m);
+  if (e == cudaSuccess) e = set_smem_once(stream_kernel<GR, kCutTopp>, smem_c);
+  if (e == cudaSuccess) e = set_smem_once(topp_resolve_kernel, bitmap_bytes);
+  if (e != cudaSuccess) return e;
+  window_kernel<GR, true><<<items, kT0, smem0, st>>>(a, sh, tb.ret, tb.n_ret, ws);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  stream_kernel<GR, kMassTopp><<<g1, kT1, smem_m, st>>>(a, sh, tb.ret, tb.n_ret, ws);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  stream_kernel<GR, kCutTopp><<<g1, kT1, smem_c, st>>>(a, sh, tb.ret, tb.n_ret, ws);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  topp_resolve_kernel<<<g2, kT2, bitmap_bytes, st>>>(a, sh, ws);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t stream_workspace_bytes(const Shape &sh, const Tables &tb, int batch, int mode) {
+  const StreamPlan p = stream_plan(sh, tb, mode);
+  if (!p.ok) return 0;
+  return stream_layout(sh, batch, p).total;
+}
+
+cudaError_t launch_select_stream(const SelectArgs &a, const Shape &sh, const Tables &tb, uint32_t *fail,
+                                 void *ws_base, cudaStream_t st, bool *used) {
+  *used = false;
+  const StreamPlan p = stream_plan(sh, tb, a.mode);
+  if (!p.ok || ws_base == nullptr) return cudaSuccess;
+  const StreamLayout L = stream_layout(sh, a.batch, p);
+  char *base = static_cast<char *>(ws_base);
+  StreamWs ws{};
+  ws.qsplit = reinterpret_cast<uint32_t *>(base + L.qsplit);
+  ws.win = reinterpret_cast<float4 *>(base + L.win);
+  ws.bcount = reinterpret_cast<uint32_t *>(base + L.bcount);
+  ws.rowitem = reinterpret_cast<int *>(base + L.rowitem);
+  ws.buf = reinterpret_cast<unsigned long long *>(base + L.buf);
+  if (p.bwords) {
+    ws.hist = reinterpret_cast<double *>(base + L.hist);
+    ws.zlo = reinterpret_cast<double *>(base + L.zlo);
+    ws.rflag = reinterpret_cast<uint32_t *>(base + L.rflag);
+    ws.bits = reinterpret_cast<uint32_t *>(base + L.bits);
+  }
+  ws.bwords = p.bwords;
+  ws.fail = fail;
+  ws.items = a.batch * tb.n_ret;
+  ws.cap = p.cap;
+  int gr = 1;
+  while (gr < tb.max_ret) gr <<= 1;
+  cudaError_t e;
+  switch (gr) {
+    case 1: e = stream_launch<1>(a, sh, tb, ws, p.bitmap_bytes, st); break;
+    case 2: e = stream_launch<2>(a, sh, tb, ws, p.bitmap_bytes, st); break;
+    case 4: e = stream_launch<4>(a, sh, tb, ws, p.bitmap_bytes, st); break;
+    case 8: e = stream_launch<8>(a, sh, tb, ws, p.bitmap_bytes, st); break;
+    default: e = stream_launch<16>(a, sh, tb, ws, p.bitmap_bytes, st); break;
+  }
+  if (e == cudaSuccess) *used = true;
+  return e;
+}
+
+}  // namespace sd
