@@ -47,7 +47,7 @@ sd_status cuda_fail(sd_ctx *ctx, cudaError_t e, const char *what) {
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct WsLayout {
-  size_t scores_off, flags_off, scores_bytes, topk_off, topk_bytes, att_off, total;
+  size_t scores_off, flags_off, scores_bytes, stream_off, stream_bytes, att_off, total;
 };
 
 WsLayout layout(const sd_ctx *ctx, int batch) {
@@ -56,9 +56,9 @@ WsLayout layout(const sd_ctx *ctx, int batch) {
   size_t foff = 0;
   w.scores_bytes = align256(sd::select_workspace_bytes(ctx->sh, ctx->tb, batch, &foff));
   w.flags_off = w.scores_off + foff;
-  w.topk_off = w.scores_off + w.scores_bytes;
-  w.topk_bytes = align256(sd::stream_workspace_bytes(ctx->sh, ctx->tb, batch, ctx->cfg.mode));
-  w.att_off = w.topk_off + w.topk_bytes;
+  w.stream_off = w.scores_off + w.scores_bytes;
+  w.stream_bytes = align256(sd::stream_workspace_bytes(ctx->sh, ctx->tb, batch, ctx->cfg.mode));
+  w.att_off = w.stream_off + w.stream_bytes;
   w.total = align256(w.att_off + sd::attend_workspace_bytes(ctx->sh, ctx->tb, batch));
   return w;
 }
@@ -225,7 +225,7 @@ sd_status sparse_decode_select(sd_ctx *ctx, const void *q_pre, const void *index
   a.top_k_frac = ctx->cfg.top_k_frac;
   a.score_ws = reinterpret_cast<float *>(static_cast<char *>(workspace) + w.scores_off);
   a.flags = reinterpret_cast<uint32_t *>(static_cast<char *>(workspace) + w.flags_off);
-  a.topk_ws = w.topk_bytes ? static_cast<char *>(workspace) + w.topk_off : nullptr;
+  a.stream_ws = w.stream_bytes ? static_cast<char *>(workspace) + w.stream_off : nullptr;
   a.err = ctx->err_d;
   a.batch = batch;
   cudaError_t e = sd::launch_select(a, ctx->sh, ctx->tb, static_cast<cudaStream_t>(stream));

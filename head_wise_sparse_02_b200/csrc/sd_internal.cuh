@@ -93,13 +93,12 @@ struct SelectArgs {
   float top_k_frac;
   float *score_ws;                // global score rows when they do not fit on chip
   uint32_t *flags;                // [batch * n_ret] streaming selection misses
-  void *topk_ws;                  // streaming selection scratch (histograms, buffers, bitmaps)
+  void *stream_ws;                // streaming selection scratch (histograms, buffers, bitmaps)
   unsigned *err;
   int batch;
 };
 
 size_t select_workspace_bytes(const Shape &sh, const Tables &tb, int batch, size_t *flags_off);
-size_t select_topk_offset(const Shape &sh, const Tables &tb, int batch);
 cudaError_t launch_select(const SelectArgs &a, const Shape &sh, const Tables &tb, cudaStream_t st);
 // Streaming selection (top-k and top-p): workspace bytes for a batch (0 when
 // the shapes are outside what it handles), and its launches; *used = false

@@ -8,6 +8,10 @@
 //   Methodology 5  the threshold is found with a histogram, without sorting.
 // ICS page (gist.science/ar/paper/2605.24168), 2: "Oracle Top-K" = exact top-k.
 //
+// This is the exact selector.  It takes the items the streaming selectors
+// (sd_select_stream.cu) flag as misses, or every item when those cannot run
+// (shapes outside them).
+//
 // Design (one thread-block cluster per (sequence b, KV group g)):
 //   * the C CTAs of the cluster split the sequence's N_b tokens into C
 //     contiguous, page-aligned chunks;
@@ -531,7 +535,7 @@ __device__ __forceinline__ void select_item(const SelectArgs &a, const Shape &sh
 // One cluster per work item (sequence, retrieval KV group).  With `flags`
 // (layout: a flag per item, then the count of flagged items, then their
 // list), the grid's clusters stride over the listed items only (items whose
-// streaming top-k window missed); otherwise item = blockIdx.y.
+// streaming top-k or top-p window missed); otherwise item = blockIdx.y.
 template <int GR, bool TOPP, bool SMEM>
 __global__ void __launch_bounds__(kThreads, 1)
 select_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__ groups, int n_groups,
@@ -715,11 +719,6 @@ size_t select_workspace_bytes(const Shape &sh, const Tables &tb, int batch, size
   return rows + (2 * (size_t)batch * std::max(1, tb.n_ret) + 1) * sizeof(uint32_t);
 }
 
-size_t select_topk_offset(const Shape &sh, const Tables &tb, int batch) {
-  size_t f = 0;
-  return (select_workspace_bytes(sh, tb, batch, &f) + 255) / 256 * 256;
-}
-
 cudaError_t launch_select(const SelectArgs &a, const Shape &sh, const Tables &tb, cudaStream_t st) {
   if (tb.n_ret == 0 || a.batch == 0) return cudaSuccess;
   int dev = 0;
@@ -748,7 +747,7 @@ cudaError_t launch_select(const SelectArgs &a, const Shape &sh, const Tables &tb
   }
   const int items = a.batch * tb.n_ret;
   bool used = false;
-  cudaError_t e = launch_select_stream(a, sh, tb, a.flags, a.topk_ws, st, &used);
+  cudaError_t e = launch_select_stream(a, sh, tb, a.flags, a.stream_ws, st, &used);
   if (e != cudaSuccess) return e;
   // after the streaming passes: exact recomputation of the items whose window
   // missed (usually none); without them: every item
