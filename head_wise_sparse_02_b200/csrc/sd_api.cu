@@ -3,6 +3,7 @@
 #include <math.h>
 #include <stdio.h>
 
+#include <memory>
 #include <string>
 #include <vector>
 
@@ -83,6 +84,7 @@ const char *sparse_decode_status_string(sd_status s) {
     case SD_ERR_CUDA: return "CUDA error";
     case SD_ERR_TIMEOUT: return "device-side wait timed out";
     case SD_ERR_DEVICE_DATA: return "device-side check rejected input data";
+    case SD_ERR_HOST_MEMORY: return "host allocation failed";
   }
   return "unknown status";
 }
@@ -92,236 +94,267 @@ const char *sparse_decode_last_error(const sd_ctx *ctx) { return ctx ? ctx->last
 int sparse_decode_num_retrieval_heads(const sd_ctx *ctx) { return ctx ? ctx->sh.H_ret : 0; }
 
 sd_status sparse_decode_init(const sd_config *cfg, const void *proj, sd_ctx **out) {
-  if (!out) return SD_ERR_INVALID_ARG;
-  *out = nullptr;
-  if (!cfg || !proj || !cfg->head_is_retrieval) return SD_ERR_INVALID_ARG;
-  const sd_config &c = *cfg;
-  if (c.num_q_heads <= 0 || c.num_kv_heads <= 0 || c.num_q_heads % c.num_kv_heads != 0)
-    return SD_ERR_INVALID_ARG;
-  if (c.num_q_heads / c.num_kv_heads > sd::kMaxGroup) return SD_ERR_UNSUPPORTED;
-  if (c.head_dim != 64 && c.head_dim != 128) return SD_ERR_UNSUPPORTED;
-  if (c.index_dim != sd::kIndexDim || c.page_size != sd::kPage) return SD_ERR_UNSUPPORTED;
-  if (c.num_pages <= 0 || c.max_batch <= 0 || c.max_pages_per_seq <= 0) return SD_ERR_INVALID_ARG;
-  if ((long long)c.max_pages_per_seq * sd::kPage > (1LL << 25)) return SD_ERR_UNSUPPORTED;
-  // cache rows are addressed with 32-bit row numbers inside the kernels
-  if ((long long)c.num_pages * c.num_kv_heads * sd::kPage >= 0xFFFFFFFFLL) return SD_ERR_UNSUPPORTED;
-  if (c.window < 0 || c.num_sinks < 0) return SD_ERR_INVALID_ARG;
-  if (c.mode != SD_TOP_P && c.mode != SD_TOP_K) return SD_ERR_INVALID_ARG;
-  if (c.mode == SD_TOP_P && !(c.top_p > 0.0f && c.top_p <= 1.0f)) return SD_ERR_INVALID_ARG;
-  if (c.mode == SD_TOP_K) {
-    if (c.top_k < 0) return SD_ERR_INVALID_ARG;
-    if (c.top_k == 0 && !(c.top_k_frac > 0.0f && c.top_k_frac <= 1.0f)) return SD_ERR_INVALID_ARG;
-  }
-  for (int h = 0; h < c.num_q_heads; ++h)
-    if (c.head_is_retrieval[h] != 0 && c.head_is_retrieval[h] != 1) return SD_ERR_INVALID_ARG;
-
-  sd_ctx *ctx = new sd_ctx();
-  ctx->cfg = c;
-  ctx->retr.assign(c.head_is_retrieval, c.head_is_retrieval + c.num_q_heads);
-  ctx->cfg.head_is_retrieval = ctx->retr.data();
-  cudaGetDevice(&ctx->device);
-  const int Hq = c.num_q_heads, Hkv = c.num_kv_heads, G = Hq / Hkv;
-  int hr = 0;
-  for (int g = 0; g < Hkv; ++g) {
-    sd::Group r{}, l{};
-    r.kv_head = l.kv_head = g;
-    for (int j = 0; j < G; ++j) {
-      const int h = g * G + j;
-      if (ctx->retr[h]) {
-        r.q_head[r.n] = h;
-        r.row[r.n] = hr++;
-        r.n++;
-      } else {
-        l.q_head[l.n] = h;
-        l.row[l.n] = -1;
-        l.n++;
-      }
+  try {
+    if (!out) return SD_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (!cfg || !proj || !cfg->head_is_retrieval) return SD_ERR_INVALID_ARG;
+    const sd_config &c = *cfg;
+    if (c.num_q_heads <= 0 || c.num_kv_heads <= 0 || c.num_q_heads % c.num_kv_heads != 0)
+      return SD_ERR_INVALID_ARG;
+    if (c.num_q_heads / c.num_kv_heads > sd::kMaxGroup) return SD_ERR_UNSUPPORTED;
+    if (c.head_dim != 64 && c.head_dim != 128) return SD_ERR_UNSUPPORTED;
+    if (c.index_dim != sd::kIndexDim || c.page_size != sd::kPage) return SD_ERR_UNSUPPORTED;
+    if (c.num_pages <= 0 || c.max_batch <= 0 || c.max_pages_per_seq <= 0) return SD_ERR_INVALID_ARG;
+    if ((long long)c.max_pages_per_seq * sd::kPage > (1LL << 25)) return SD_ERR_UNSUPPORTED;
+    // cache rows are addressed with 32-bit row numbers inside the kernels
+    if ((long long)c.num_pages * c.num_kv_heads * sd::kPage >= 0xFFFFFFFFLL) return SD_ERR_UNSUPPORTED;
+    if (c.window < 0 || c.num_sinks < 0) return SD_ERR_INVALID_ARG;
+    if (c.mode != SD_TOP_P && c.mode != SD_TOP_K) return SD_ERR_INVALID_ARG;
+    if (c.mode == SD_TOP_P && !(c.top_p > 0.0f && c.top_p <= 1.0f)) return SD_ERR_INVALID_ARG;
+    if (c.mode == SD_TOP_K) {
+      if (c.top_k < 0) return SD_ERR_INVALID_ARG;
+      if (c.top_k == 0 && !(c.top_k_frac > 0.0f && c.top_k_frac <= 1.0f)) return SD_ERR_INVALID_ARG;
     }
-    if (r.n) ctx->ret_h.push_back(r);
-    if (l.n) ctx->loc_h.push_back(l);
-  }
-  ctx->sh.Hq = Hq;
-  ctx->sh.Hkv = Hkv;
-  ctx->sh.d = c.head_dim;
-  ctx->sh.num_pages = c.num_pages;
-  ctx->sh.max_pages = c.max_pages_per_seq;
-  ctx->sh.H_ret = hr;
-  ctx->sh.max_len = (long long)c.max_pages_per_seq * sd::kPage;
-  ctx->attn_scale = c.attn_scale > 0.f ? c.attn_scale : (float)(1.0 / sqrt((double)c.head_dim));
-  ctx->index_scale = c.index_scale > 0.f ? c.index_scale : (float)(sqrt((double)c.head_dim) / sd::kIndexDim);
+    for (int h = 0; h < c.num_q_heads; ++h)
+      if (c.head_is_retrieval[h] != 0 && c.head_is_retrieval[h] != 1) return SD_ERR_INVALID_ARG;
 
-  const size_t ng = ctx->ret_h.size() + ctx->loc_h.size();
-  const size_t proj_bytes = (size_t)Hkv * c.head_dim * sd::kIndexDim * sizeof(uint16_t);
-  cudaError_t e = cudaMalloc(&ctx->groups_d, ng * sizeof(sd::Group));
-  if (e == cudaSuccess) e = cudaMalloc(&ctx->proj_d, proj_bytes);
-  if (e == cudaSuccess) e = cudaMalloc(&ctx->err_d, sizeof(unsigned));
-  std::vector<sd::Group> all(ctx->ret_h);
-  all.insert(all.end(), ctx->loc_h.begin(), ctx->loc_h.end());
-  if (e == cudaSuccess) e = cudaMemcpy(ctx->groups_d, all.data(), ng * sizeof(sd::Group), cudaMemcpyHostToDevice);
-  if (e == cudaSuccess) e = cudaMemcpy(ctx->proj_d, proj, proj_bytes, cudaMemcpyDefault);
-  if (e == cudaSuccess) e = cudaMemset(ctx->err_d, 0, sizeof(unsigned));
-  if (e != cudaSuccess) {
-    sparse_decode_destroy(ctx);
-    return SD_ERR_CUDA;
+    std::unique_ptr<sd_ctx> holder(new sd_ctx());
+    sd_ctx *ctx = holder.get();
+    ctx->cfg = c;
+    ctx->retr.assign(c.head_is_retrieval, c.head_is_retrieval + c.num_q_heads);
+    ctx->cfg.head_is_retrieval = ctx->retr.data();
+    cudaGetDevice(&ctx->device);
+    const int Hq = c.num_q_heads, Hkv = c.num_kv_heads, G = Hq / Hkv;
+    int hr = 0;
+    for (int g = 0; g < Hkv; ++g) {
+      sd::Group r{}, l{};
+      r.kv_head = l.kv_head = g;
+      for (int j = 0; j < G; ++j) {
+        const int h = g * G + j;
+        if (ctx->retr[h]) {
+          r.q_head[r.n] = h;
+          r.row[r.n] = hr++;
+          r.n++;
+        } else {
+          l.q_head[l.n] = h;
+          l.row[l.n] = -1;
+          l.n++;
+        }
+      }
+      if (r.n) ctx->ret_h.push_back(r);
+      if (l.n) ctx->loc_h.push_back(l);
+    }
+    ctx->sh.Hq = Hq;
+    ctx->sh.Hkv = Hkv;
+    ctx->sh.d = c.head_dim;
+    ctx->sh.num_pages = c.num_pages;
+    ctx->sh.max_pages = c.max_pages_per_seq;
+    ctx->sh.H_ret = hr;
+    ctx->sh.max_len = (long long)c.max_pages_per_seq * sd::kPage;
+    ctx->attn_scale = c.attn_scale > 0.f ? c.attn_scale : (float)(1.0 / sqrt((double)c.head_dim));
+    ctx->index_scale = c.index_scale > 0.f ? c.index_scale : (float)(sqrt((double)c.head_dim) / sd::kIndexDim);
+
+    // every host allocation happens before the first device one, so a failed
+    // host allocation (caught below) leaves no device memory behind
+    const size_t ng = ctx->ret_h.size() + ctx->loc_h.size();
+    const size_t proj_bytes = (size_t)Hkv * c.head_dim * sd::kIndexDim * sizeof(uint16_t);
+    std::vector<sd::Group> all(ctx->ret_h);
+    all.insert(all.end(), ctx->loc_h.begin(), ctx->loc_h.end());
+    cudaError_t e = cudaMalloc(&ctx->groups_d, ng * sizeof(sd::Group));
+    if (e == cudaSuccess) e = cudaMalloc(&ctx->proj_d, proj_bytes);
+    if (e == cudaSuccess) e = cudaMalloc(&ctx->err_d, sizeof(unsigned));
+    if (e == cudaSuccess) e = cudaMemcpy(ctx->groups_d, all.data(), ng * sizeof(sd::Group), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(ctx->proj_d, proj, proj_bytes, cudaMemcpyDefault);
+    if (e == cudaSuccess) e = cudaMemset(ctx->err_d, 0, sizeof(unsigned));
+    if (e != cudaSuccess) {
+      sparse_decode_destroy(holder.release());
+      return SD_ERR_CUDA;
+    }
+    ctx->tb.ret = ctx->groups_d;
+    ctx->tb.loc = ctx->groups_d + ctx->ret_h.size();
+    ctx->tb.n_ret = (int)ctx->ret_h.size();
+    ctx->tb.n_loc = (int)ctx->loc_h.size();
+    for (auto &g : ctx->ret_h) ctx->tb.max_ret = std::max(ctx->tb.max_ret, g.n);
+    for (auto &g : ctx->loc_h) ctx->tb.max_loc = std::max(ctx->tb.max_loc, g.n);
+    *out = holder.release();
+    return SD_OK;
+  } catch (...) {
+    return SD_ERR_HOST_MEMORY;
   }
-  ctx->tb.ret = ctx->groups_d;
-  ctx->tb.loc = ctx->groups_d + ctx->ret_h.size();
-  ctx->tb.n_ret = (int)ctx->ret_h.size();
-  ctx->tb.n_loc = (int)ctx->loc_h.size();
-  for (auto &g : ctx->ret_h) ctx->tb.max_ret = std::max(ctx->tb.max_ret, g.n);
-  for (auto &g : ctx->loc_h) ctx->tb.max_loc = std::max(ctx->tb.max_loc, g.n);
-  *out = ctx;
-  return SD_OK;
 }
 
 sd_status sparse_decode_workspace_size(const sd_ctx *ctx, int batch, size_t *bytes) {
-  if (!ctx || !bytes) return SD_ERR_INVALID_ARG;
-  if (batch < 0 || batch > ctx->cfg.max_batch) return SD_ERR_INVALID_ARG;
-  *bytes = layout(ctx, batch).total;
-  return SD_OK;
+  try {
+    if (!ctx || !bytes) return SD_ERR_INVALID_ARG;
+    if (batch < 0 || batch > ctx->cfg.max_batch) return SD_ERR_INVALID_ARG;
+    *bytes = layout(ctx, batch).total;
+    return SD_OK;
+  } catch (...) {
+    return SD_ERR_HOST_MEMORY;
+  }
 }
 
 sd_status sparse_decode_index_keys(sd_ctx *ctx, const void *k_pre, const int32_t *slots, int num_tokens,
                                    void *index_cache, sd_stream stream) {
-  if (!ctx) return SD_ERR_INVALID_ARG;
-  if (num_tokens < 0) return fail(ctx, SD_ERR_INVALID_ARG, "num_tokens < 0");
-  if (num_tokens == 0) return SD_OK;
-  if (!k_pre || !slots || !index_cache) return fail(ctx, SD_ERR_INVALID_ARG, "null pointer");
-  DeviceGuard dg(ctx->device);
-  cudaError_t e = sd::launch_index_keys(static_cast<const uint16_t *>(k_pre), slots, num_tokens,
-                                        static_cast<uint16_t *>(index_cache), ctx->proj_d, ctx->sh,
-                                        ctx->err_d, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? SD_OK : cuda_fail(ctx, e, "index_keys launch");
+  try {
+    if (!ctx) return SD_ERR_INVALID_ARG;
+    if (num_tokens < 0) return fail(ctx, SD_ERR_INVALID_ARG, "num_tokens < 0");
+    if (num_tokens == 0) return SD_OK;
+    if (!k_pre || !slots || !index_cache) return fail(ctx, SD_ERR_INVALID_ARG, "null pointer");
+    DeviceGuard dg(ctx->device);
+    cudaError_t e = sd::launch_index_keys(static_cast<const uint16_t *>(k_pre), slots, num_tokens,
+                                          static_cast<uint16_t *>(index_cache), ctx->proj_d, ctx->sh,
+                                          ctx->err_d, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SD_OK : cuda_fail(ctx, e, "index_keys launch");
+  } catch (...) {
+    return SD_ERR_HOST_MEMORY;
+  }
 }
 
 sd_status sparse_decode_select(sd_ctx *ctx, const void *q_pre, const void *index_cache,
                                const int32_t *page_table, const int32_t *seq_lens, int batch,
                                int32_t *sel_idx, int32_t *sel_count, int sel_stride, void *workspace,
                                size_t ws_bytes, sd_stream stream) {
-  if (!ctx) return SD_ERR_INVALID_ARG;
-  if (batch < 0 || batch > ctx->cfg.max_batch) return fail(ctx, SD_ERR_INVALID_ARG, "batch out of range");
-  if (batch == 0 || ctx->sh.H_ret == 0) return SD_OK;
-  if (!q_pre || !index_cache || !page_table || !seq_lens || !sel_idx || !sel_count)
-    return fail(ctx, SD_ERR_INVALID_ARG, "null pointer");
-  const long long need_stride = ctx->cfg.mode == SD_TOP_P ? ctx->sh.max_len : max_topk(ctx);
-  if (sel_stride < need_stride)
-    return fail(ctx, SD_ERR_INVALID_ARG, "sel_stride smaller than the largest possible set");
-  const WsLayout w = layout(ctx, batch);
-  if (!workspace || ws_bytes < w.total) return fail(ctx, SD_ERR_WORKSPACE, "workspace too small");
-  DeviceGuard dg(ctx->device);
-  sd::SelectArgs a{};
-  a.q_pre = static_cast<const uint16_t *>(q_pre);
-  a.index_cache = static_cast<const uint16_t *>(index_cache);
-  a.page_table = page_table;
-  a.seq_lens = seq_lens;
-  a.sel_idx = sel_idx;
-  a.sel_count = sel_count;
-  a.sel_stride = sel_stride;
-  a.proj = ctx->proj_d;
-  a.index_scale = ctx->index_scale;
-  a.mode = ctx->cfg.mode;
-  a.top_p = ctx->cfg.top_p;
-  a.top_k = ctx->cfg.top_k;
-  a.top_k_frac = ctx->cfg.top_k_frac;
-  a.score_ws = reinterpret_cast<float *>(static_cast<char *>(workspace) + w.scores_off);
-  a.flags = reinterpret_cast<uint32_t *>(static_cast<char *>(workspace) + w.flags_off);
-  a.stream_ws = w.stream_bytes ? static_cast<char *>(workspace) + w.stream_off : nullptr;
-  a.err = ctx->err_d;
-  a.batch = batch;
-  cudaError_t e = sd::launch_select(a, ctx->sh, ctx->tb, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? SD_OK : cuda_fail(ctx, e, "select launch");
+  try {
+    if (!ctx) return SD_ERR_INVALID_ARG;
+    if (batch < 0 || batch > ctx->cfg.max_batch) return fail(ctx, SD_ERR_INVALID_ARG, "batch out of range");
+    if (batch == 0 || ctx->sh.H_ret == 0) return SD_OK;
+    if (!q_pre || !index_cache || !page_table || !seq_lens || !sel_idx || !sel_count)
+      return fail(ctx, SD_ERR_INVALID_ARG, "null pointer");
+    const long long need_stride = ctx->cfg.mode == SD_TOP_P ? ctx->sh.max_len : max_topk(ctx);
+    if (sel_stride < need_stride)
+      return fail(ctx, SD_ERR_INVALID_ARG, "sel_stride smaller than the largest possible set");
+    const WsLayout w = layout(ctx, batch);
+    if (!workspace || ws_bytes < w.total) return fail(ctx, SD_ERR_WORKSPACE, "workspace too small");
+    DeviceGuard dg(ctx->device);
+    sd::SelectArgs a{};
+    a.q_pre = static_cast<const uint16_t *>(q_pre);
+    a.index_cache = static_cast<const uint16_t *>(index_cache);
+    a.page_table = page_table;
+    a.seq_lens = seq_lens;
+    a.sel_idx = sel_idx;
+    a.sel_count = sel_count;
+    a.sel_stride = sel_stride;
+    a.proj = ctx->proj_d;
+    a.index_scale = ctx->index_scale;
+    a.mode = ctx->cfg.mode;
+    a.top_p = ctx->cfg.top_p;
+    a.top_k = ctx->cfg.top_k;
+    a.top_k_frac = ctx->cfg.top_k_frac;
+    a.score_ws = reinterpret_cast<float *>(static_cast<char *>(workspace) + w.scores_off);
+    a.flags = reinterpret_cast<uint32_t *>(static_cast<char *>(workspace) + w.flags_off);
+    a.stream_ws = w.stream_bytes ? static_cast<char *>(workspace) + w.stream_off : nullptr;
+    a.err = ctx->err_d;
+    a.batch = batch;
+    cudaError_t e = sd::launch_select(a, ctx->sh, ctx->tb, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SD_OK : cuda_fail(ctx, e, "select launch");
+  } catch (...) {
+    return SD_ERR_HOST_MEMORY;
+  }
 }
 
 sd_status sparse_decode_attend(sd_ctx *ctx, const void *q, const void *k_cache, const void *v_cache,
                                const int32_t *page_table, const int32_t *seq_lens, int batch,
                                const int32_t *sel_idx, const int32_t *sel_count, int sel_stride, float *out,
                                void *workspace, size_t ws_bytes, sd_stream stream) {
-  if (!ctx) return SD_ERR_INVALID_ARG;
-  if (batch < 0 || batch > ctx->cfg.max_batch) return fail(ctx, SD_ERR_INVALID_ARG, "batch out of range");
-  if (batch == 0) return SD_OK;
-  if (!q || !k_cache || !v_cache || !page_table || !seq_lens || !out)
-    return fail(ctx, SD_ERR_INVALID_ARG, "null pointer");
-  if (ctx->sh.H_ret > 0 && (!sel_idx || !sel_count || sel_stride <= 0))
-    return fail(ctx, SD_ERR_INVALID_ARG, "selection lists required for retrieval heads");
-  const WsLayout w = layout(ctx, batch);
-  if (!workspace || ws_bytes < w.total) return fail(ctx, SD_ERR_WORKSPACE, "workspace too small");
-  DeviceGuard dg(ctx->device);
-  sd::AttendArgs a{};
-  a.q = static_cast<const uint16_t *>(q);
-  a.k_cache = static_cast<const uint16_t *>(k_cache);
-  a.v_cache = static_cast<const uint16_t *>(v_cache);
-  a.page_table = page_table;
-  a.seq_lens = seq_lens;
-  a.sel_idx = sel_idx;
-  a.sel_count = sel_count;
-  a.sel_stride = sel_stride;
-  a.out = out;
-  a.attn_scale = ctx->attn_scale;
-  a.window = ctx->cfg.window;
-  a.num_sinks = ctx->cfg.num_sinks;
-  a.ws = static_cast<char *>(workspace) + w.att_off;
-  a.err = ctx->err_d;
-  a.batch = batch;
-  cudaError_t e = sd::launch_attend(a, ctx->sh, ctx->tb, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? SD_OK : cuda_fail(ctx, e, "attend launch");
+  try {
+    if (!ctx) return SD_ERR_INVALID_ARG;
+    if (batch < 0 || batch > ctx->cfg.max_batch) return fail(ctx, SD_ERR_INVALID_ARG, "batch out of range");
+    if (batch == 0) return SD_OK;
+    if (!q || !k_cache || !v_cache || !page_table || !seq_lens || !out)
+      return fail(ctx, SD_ERR_INVALID_ARG, "null pointer");
+    if (ctx->sh.H_ret > 0 && (!sel_idx || !sel_count || sel_stride <= 0))
+      return fail(ctx, SD_ERR_INVALID_ARG, "selection lists required for retrieval heads");
+    const WsLayout w = layout(ctx, batch);
+    if (!workspace || ws_bytes < w.total) return fail(ctx, SD_ERR_WORKSPACE, "workspace too small");
+    DeviceGuard dg(ctx->device);
+    sd::AttendArgs a{};
+    a.q = static_cast<const uint16_t *>(q);
+    a.k_cache = static_cast<const uint16_t *>(k_cache);
+    a.v_cache = static_cast<const uint16_t *>(v_cache);
+    a.page_table = page_table;
+    a.seq_lens = seq_lens;
+    a.sel_idx = sel_idx;
+    a.sel_count = sel_count;
+    a.sel_stride = sel_stride;
+    a.out = out;
+    a.attn_scale = ctx->attn_scale;
+    a.window = ctx->cfg.window;
+    a.num_sinks = ctx->cfg.num_sinks;
+    a.ws = static_cast<char *>(workspace) + w.att_off;
+    a.err = ctx->err_d;
+    a.batch = batch;
+    cudaError_t e = sd::launch_attend(a, ctx->sh, ctx->tb, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SD_OK : cuda_fail(ctx, e, "attend launch");
+  } catch (...) {
+    return SD_ERR_HOST_MEMORY;
+  }
 }
 
 sd_status sparse_decode_attend_noalloc(sd_ctx *ctx, const void *q, const void *k_cache, const void *v_cache,
                                        const int32_t *page_table, const int32_t *seq_lens, int batch,
                                        const int32_t *sel_idx, const int32_t *sel_count, int sel_stride,
                                        float *out, sd_stream stream) {
-  if (!ctx) return SD_ERR_INVALID_ARG;
-  if (batch < 0 || batch > ctx->cfg.max_batch) return fail(ctx, SD_ERR_INVALID_ARG, "batch out of range");
-  if (batch == 0) return SD_OK;
-  if (!q || !k_cache || !v_cache || !page_table || !seq_lens || !out)
-    return fail(ctx, SD_ERR_INVALID_ARG, "null pointer");
-  if (ctx->sh.H_ret > 0 && (!sel_idx || !sel_count || sel_stride <= 0))
-    return fail(ctx, SD_ERR_INVALID_ARG, "selection lists required for retrieval heads");
-  const size_t need = sd::attend_workspace_bytes(ctx->sh, ctx->tb, batch);
-  if (need > sd::kNoAllocScratchBytes)
-    return fail(ctx, SD_ERR_WORKSPACE,
-                "attend needs " + std::to_string(need) + " bytes of scratch for this batch; the built-in scratch holds " +
-                    std::to_string(sd::kNoAllocScratchBytes) + " (use sparse_decode_attend with a caller workspace)");
-  DeviceGuard dg(ctx->device);
-  void *scratch = nullptr;
-  cudaError_t e = sd::noalloc_scratch(&scratch);
-  if (e != cudaSuccess) return cuda_fail(ctx, e, "scratch lookup");
-  sd::AttendArgs a{};
-  a.q = static_cast<const uint16_t *>(q);
-  a.k_cache = static_cast<const uint16_t *>(k_cache);
-  a.v_cache = static_cast<const uint16_t *>(v_cache);
-  a.page_table = page_table;
-  a.seq_lens = seq_lens;
-  a.sel_idx = sel_idx;
-  a.sel_count = sel_count;
-  a.sel_stride = sel_stride;
-  a.out = out;
-  a.attn_scale = ctx->attn_scale;
-  a.window = ctx->cfg.window;
-  a.num_sinks = ctx->cfg.num_sinks;
-  a.ws = scratch;
-  a.err = ctx->err_d;
-  a.batch = batch;
-  e = sd::launch_attend(a, ctx->sh, ctx->tb, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? SD_OK : cuda_fail(ctx, e, "attend launch");
+  try {
+    if (!ctx) return SD_ERR_INVALID_ARG;
+    if (batch < 0 || batch > ctx->cfg.max_batch) return fail(ctx, SD_ERR_INVALID_ARG, "batch out of range");
+    if (batch == 0) return SD_OK;
+    if (!q || !k_cache || !v_cache || !page_table || !seq_lens || !out)
+      return fail(ctx, SD_ERR_INVALID_ARG, "null pointer");
+    if (ctx->sh.H_ret > 0 && (!sel_idx || !sel_count || sel_stride <= 0))
+      return fail(ctx, SD_ERR_INVALID_ARG, "selection lists required for retrieval heads");
+    const size_t need = sd::attend_workspace_bytes(ctx->sh, ctx->tb, batch);
+    if (need > sd::kNoAllocScratchBytes)
+      return fail(ctx, SD_ERR_WORKSPACE,
+                  "attend needs " + std::to_string(need) + " bytes of scratch for this batch; the built-in scratch holds " +
+                      std::to_string(sd::kNoAllocScratchBytes) + " (use sparse_decode_attend with a caller workspace)");
+    DeviceGuard dg(ctx->device);
+    void *scratch = nullptr;
+    cudaError_t e = sd::noalloc_scratch(&scratch);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "scratch lookup");
+    sd::AttendArgs a{};
+    a.q = static_cast<const uint16_t *>(q);
+    a.k_cache = static_cast<const uint16_t *>(k_cache);
+    a.v_cache = static_cast<const uint16_t *>(v_cache);
+    a.page_table = page_table;
+    a.seq_lens = seq_lens;
+    a.sel_idx = sel_idx;
+    a.sel_count = sel_count;
+    a.sel_stride = sel_stride;
+    a.out = out;
+    a.attn_scale = ctx->attn_scale;
+    a.window = ctx->cfg.window;
+    a.num_sinks = ctx->cfg.num_sinks;
+    a.ws = scratch;
+    a.err = ctx->err_d;
+    a.batch = batch;
+    e = sd::launch_attend(a, ctx->sh, ctx->tb, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SD_OK : cuda_fail(ctx, e, "attend launch");
+  } catch (...) {
+    return SD_ERR_HOST_MEMORY;
+  }
 }
 
 sd_status sparse_decode_error_word(sd_ctx *ctx, sd_stream stream, uint32_t *word) {
-  if (!ctx) return SD_ERR_INVALID_ARG;
-  DeviceGuard dg(ctx->device);
-  unsigned v = 0;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaMemcpyAsync(&v, ctx->err_d, sizeof(unsigned), cudaMemcpyDeviceToHost, st);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
-  if (e == cudaSuccess) e = cudaMemsetAsync(ctx->err_d, 0, sizeof(unsigned), st);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
-  if (e != cudaSuccess) return cuda_fail(ctx, e, "error word read");
-  if (word) *word = v;
-  if (v == 0) return SD_OK;
-  if (v & SD_EBIT_TIMEOUT) return fail(ctx, SD_ERR_TIMEOUT, "device-side wait timed out");
-  char buf[96];
-  snprintf(buf, sizeof(buf), "device-side check rejected input data (error word 0x%x)", v);
-  return fail(ctx, SD_ERR_DEVICE_DATA, buf);
+  try {
+    if (!ctx) return SD_ERR_INVALID_ARG;
+    DeviceGuard dg(ctx->device);
+    unsigned v = 0;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(&v, ctx->err_d, sizeof(unsigned), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ctx->err_d, 0, sizeof(unsigned), st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "error word read");
+    if (word) *word = v;
+    if (v == 0) return SD_OK;
+    if (v & SD_EBIT_TIMEOUT) return fail(ctx, SD_ERR_TIMEOUT, "device-side wait timed out");
+    char buf[96];
+    snprintf(buf, sizeof(buf), "device-side check rejected input data (error word 0x%x)", v);
+    return fail(ctx, SD_ERR_DEVICE_DATA, buf);
+  } catch (...) {
+    return SD_ERR_HOST_MEMORY;
+  }
 }
 
 void sparse_decode_destroy(sd_ctx *ctx) {

@@ -21,7 +21,7 @@ LIB_PATH = os.environ.get("SPARSE_DECODE_LIB") or os.path.join(
     os.path.dirname(os.path.abspath(__file__)), "lib", "libsparsedecode.so")
 
 SD_OK, SD_ERR_INVALID_ARG, SD_ERR_UNSUPPORTED, SD_ERR_WORKSPACE, SD_ERR_CUDA, SD_ERR_TIMEOUT, \
-    SD_ERR_DEVICE_DATA = range(7)
+    SD_ERR_DEVICE_DATA, SD_ERR_HOST_MEMORY = range(8)
 SD_TOP_P, SD_TOP_K = 0, 1
 SD_EBIT_PAGE, SD_EBIT_SEQLEN, SD_EBIT_SEL, SD_EBIT_SLOT, SD_EBIT_TIMEOUT = 1, 2, 4, 8, 16
 

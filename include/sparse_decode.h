@@ -89,7 +89,9 @@ typedef enum {
   SD_ERR_WORKSPACE = 3,     /* workspace missing or smaller than the size query */
   SD_ERR_CUDA = 4,          /* a CUDA runtime call or a kernel launch failed */
   SD_ERR_TIMEOUT = 5,       /* a bounded device-side wait gave up */
-  SD_ERR_DEVICE_DATA = 6    /* a device-side check rejected input data */
+  SD_ERR_DEVICE_DATA = 6,   /* a device-side check rejected input data */
+  SD_ERR_HOST_MEMORY = 7    /* a host allocation failed inside the call (no C++ exception ever
+                               leaves a call); work the call enqueued before it stays enqueued */
 } sd_status;
 
 /* Selection mode of retrieval heads (RTPurbo page, Methodology 3). */
@@ -168,7 +170,8 @@ typedef struct {
  * device error word.  Returns SD_ERR_INVALID_ARG or SD_ERR_UNSUPPORTED for a
  * bad or unsupported configuration (among them a pool whose
  * num_pages * Hkv * P cache rows do not fit 32-bit row numbers),
- * SD_ERR_CUDA if an allocation fails.
+ * SD_ERR_CUDA if a device allocation fails, SD_ERR_HOST_MEMORY if a host one
+ * does.
  */
 SD_API sd_status sparse_decode_init(const sd_config *cfg, const void *proj, sd_ctx **out);
 

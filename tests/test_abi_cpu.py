@@ -40,6 +40,7 @@ def test_status_strings():
     from head_wise_sparse_02_b200 import sparse_decode as sd
     assert sd.status_string(sd.SD_OK) == "ok"
     assert "workspace" in sd.status_string(sd.SD_ERR_WORKSPACE)
+    assert sd.status_string(sd.SD_ERR_HOST_MEMORY) == "host allocation failed"
     assert sd.status_string(99) == "unknown status"
 
 
