@@ -98,6 +98,22 @@ def _ptr(t: Optional[torch.Tensor], dtype: torch.dtype, name: str) -> Optional[i
     return t.data_ptr()
 
 
+def _check_sets(ctx: int, sel_idx, sel_count, batch: int) -> None:
+    """With retrieval heads, sel_idx must be [>= B, H_ret, stride] and sel_count
+    [>= B, H_ret]: the library addresses row (b, i) at (b * H_ret + i) * stride
+    through raw pointers and cannot see the tensors' extents.  Without
+    retrieval heads it reads neither."""
+    h_ret = sparse_decode_num_retrieval_heads(ctx) if ctx else 0
+    if h_ret == 0:
+        return
+    if sel_idx is None or sel_count is None:
+        raise ValueError("sel_idx and sel_count are required with retrieval heads")
+    if sel_idx.dim() != 3 or sel_idx.shape[0] < batch or sel_idx.shape[1] != h_ret:
+        raise ValueError(f"sel_idx must be [B >= {batch}, H_ret = {h_ret}, stride], got {tuple(sel_idx.shape)}")
+    if sel_count.dim() != 2 or sel_count.shape[0] < batch or sel_count.shape[1] != h_ret:
+        raise ValueError(f"sel_count must be [B >= {batch}, H_ret = {h_ret}], got {tuple(sel_count.shape)}")
+
+
 def _stream(stream) -> int:
     if stream is None:
         return torch.cuda.current_stream().cuda_stream
@@ -113,6 +129,8 @@ def sparse_decode_init(*, num_q_heads: int, num_kv_heads: int, head_dim: int,
                        top_k: int = 0, top_k_frac: float = 0.0, attn_scale: float = 0.0,
                        index_scale: float = 0.0, index_dim: int = 16, page_size: int = 16) -> int:
     """Create a context (returns the opaque handle)."""
+    if mode not in ("top_p", "top_k"):
+        raise ValueError(f"mode must be 'top_p' or 'top_k', got {mode!r}")
     retr = (c_int32 * num_q_heads)(*[int(x) for x in head_is_retrieval])
     cfg = SdConfig(num_q_heads, num_kv_heads, head_dim, index_dim, page_size, num_pages,
                    ctypes.cast(retr, POINTER(c_int32)), window, num_sinks,
@@ -140,6 +158,7 @@ def sparse_decode_index_keys(ctx: int, k_pre: torch.Tensor, slots: torch.Tensor,
 
 def sparse_decode_select(ctx: int, q_pre, index_cache, page_table, seq_lens, sel_idx, sel_count,
                          workspace, stream=None) -> None:
+    _check_sets(ctx, sel_idx, sel_count, int(seq_lens.numel()))
     _check(LIB.sparse_decode_select(
         ctx, _ptr(q_pre, torch.bfloat16, "q_pre"), _ptr(index_cache, torch.bfloat16, "index_cache"),
         _ptr(page_table, torch.int32, "page_table"), _ptr(seq_lens, torch.int32, "seq_lens"),
@@ -150,6 +169,7 @@ def sparse_decode_select(ctx: int, q_pre, index_cache, page_table, seq_lens, sel
 
 def sparse_decode_attend(ctx: int, q, k_cache, v_cache, page_table, seq_lens, sel_idx, sel_count,
                          out, workspace, stream=None) -> None:
+    _check_sets(ctx, sel_idx, sel_count, int(seq_lens.numel()))
     stride = int(sel_idx.shape[-1]) if sel_idx is not None else 0
     _check(LIB.sparse_decode_attend(
         ctx, _ptr(q, torch.bfloat16, "q"), _ptr(k_cache, torch.bfloat16, "k_cache"),
@@ -163,6 +183,7 @@ def sparse_decode_attend(ctx: int, q, k_cache, v_cache, page_table, seq_lens, se
 def sparse_decode_attend_noalloc(ctx: int, q, k_cache, v_cache, page_table, seq_lens, sel_idx, sel_count,
                                  out, stream=None) -> None:
     """attend on the library's built-in scratch (no workspace argument)."""
+    _check_sets(ctx, sel_idx, sel_count, int(seq_lens.numel()))
     stride = int(sel_idx.shape[-1]) if sel_idx is not None else 0
     _check(LIB.sparse_decode_attend_noalloc(
         ctx, _ptr(q, torch.bfloat16, "q"), _ptr(k_cache, torch.bfloat16, "k_cache"),

@@ -8,6 +8,7 @@ import os
 import re
 
 import pytest
+import torch
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -95,3 +96,29 @@ def test_binding_fails_loudly_without_the_library(tmp_path):
     from head_wise_sparse_02_b200 import sparse_decode as sd
     with pytest.raises(ImportError):
         sd._load(str(tmp_path / "missing.so"))
+
+
+def test_binding_checks_selection_shapes(monkeypatch):
+    """The library addresses selection rows through raw pointers, so the binding
+    checks their extents against the batch and the retrieval heads."""
+    from head_wise_sparse_02_b200 import sparse_decode as sd
+    monkeypatch.setattr(sd, "sparse_decode_num_retrieval_heads", lambda ctx: 4)
+    ok_idx, ok_cnt = torch.zeros((3, 4, 10), dtype=torch.int32), torch.zeros((3, 4), dtype=torch.int32)
+    sd._check_sets(1, ok_idx, ok_cnt, 3)
+    sd._check_sets(1, ok_idx, ok_cnt, 2)            # rows beyond the batch are not read
+    for idx, cnt in [(torch.zeros((3, 5, 10), dtype=torch.int32), ok_cnt),
+                     (torch.zeros((2, 4, 10), dtype=torch.int32), ok_cnt),
+                     (torch.zeros((3, 40), dtype=torch.int32), ok_cnt),
+                     (ok_idx, torch.zeros((3, 3), dtype=torch.int32)),
+                     (ok_idx, None)]:
+        with pytest.raises(ValueError):
+            sd._check_sets(1, idx, cnt, 3)
+    monkeypatch.setattr(sd, "sparse_decode_num_retrieval_heads", lambda ctx: 0)
+    sd._check_sets(1, None, None, 3)                 # no retrieval heads: nothing is read
+
+
+def test_binding_rejects_an_unknown_mode():
+    from head_wise_sparse_02_b200 import sparse_decode as sd
+    with pytest.raises(ValueError):
+        sd.sparse_decode_init(num_q_heads=4, num_kv_heads=2, head_dim=64, head_is_retrieval=[1] * 4,
+                              num_pages=4, max_batch=1, max_pages_per_seq=4, proj=None, mode="topk")
