@@ -70,3 +70,21 @@ def test_oracle_slab_step_matches_decode_reference():
         out = bench.oracle_slab_step(inp, cfg, 0, g, O.index_keys(inp["proj"][g], K))
         for i, h in enumerate(range(g * G, (g + 1) * G)):
             np.testing.assert_array_equal(out[i], ref.out[(0, h)])
+
+
+def test_reference_arm_prints_one_contract_line(capsys):
+    """`bench.py --impl reference` (the oracle on the host cores) prints one
+    JSON line with the keys the harness reads, on a shrunken workload."""
+    import json
+    bench.main(["--impl", "reference", "--workload", "tiny_ref", "--seq-len", "300", "--steps", "2",
+                "--warmup", "1"])
+    lines = [l for l in capsys.readouterr().out.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for k in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+              "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert k in d, k
+    assert d["impl"] == "reference" and d["steps"] == 2 and d["warmup"] == 3   # warm-up raised to 3
+    assert d["value"] > 0 and d["cpu_baseline"]["value"] == d["value"]
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
