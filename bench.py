@@ -431,7 +431,7 @@ def oracle_slab_step(inp, cfg, b, g, index_g):
     for h in range(g * G, (g + 1) * G):
         if cfg.head_is_retrieval[h]:
             s = O.index_scores(O.query_index(inp["proj"][g], inp["q_pre"][b, h]), index_g, index_scale)
-            S = (O.select_top_p(s, cfg.top_p) if cfg.mode == "top_p"
+            S = (O.select_top_p(s, O.stored_top_p(cfg.top_p)) if cfg.mode == "top_p"
                  else O.select_top_k(s, O.top_k_budget(n, cfg.top_k, cfg.top_k_frac)))
         else:
             S = O.local_positions(n, cfg.window, cfg.num_sinks)

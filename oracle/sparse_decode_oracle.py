@@ -68,6 +68,7 @@ __all__ = [
     "query_index",
     "index_scores",
     "select_top_p",
+    "stored_top_p",
     "select_top_k",
     "top_k_budget",
     "local_positions",
@@ -175,6 +176,15 @@ def select_top_p(scores, p: float) -> np.ndarray:
         return np.arange(n, dtype=np.int64)
     tau = s[order[first]]
     return np.flatnonzero(s >= tau).astype(np.int64)
+
+
+def stored_top_p(p: float) -> float:
+    """The mass p a top-p head must reach, as the float32 value the
+    configuration stores (the C interface holds p as a float; [RTP] §3 gives p,
+    e.g. 0.9, with no precision).  p and float32(p) differ by up to ~3e-8 of p;
+    near p = 1 that can move the threshold by a token whose score lies far
+    outside any tolerance band around it."""
+    return float(np.float32(p))
 
 
 def top_k_budget(n: int, top_k: int, top_k_frac: float) -> int:
@@ -313,7 +323,7 @@ def decode_reference(cfg: OracleConfig, proj, q_pre, q, k_cache, v_cache,
                 qi = query_index(proj[g], q_pre[b, h])
                 s = index_scores(qi, index_cache[(b, g)], index_scale)
                 if cfg.mode == "top_p":
-                    S = select_top_p(s, cfg.top_p)
+                    S = select_top_p(s, stored_top_p(cfg.top_p))
                 else:
                     S = select_top_k(s, top_k_budget(n, cfg.top_k, cfg.top_k_frac))
                 if keep_scores:

@@ -211,6 +211,29 @@ def test_top_p_zipf_closed_form(alpha, p):
     assert set(rank[S].tolist()) == set(range(1, n_expect + 1))
 
 
+def test_top_p_uses_the_float32_value_of_p():
+    # two tokens whose first holds mass 0.990000005: p = 0.99 keeps it alone,
+    # float32(0.99) = 0.99000000954 needs both; the configuration stores the
+    # float32 value, and the decode step applies exactly that
+    c1 = 0.990000005
+    s = np.array([math.log(c1 / (1.0 - c1)), 0.0])
+    assert O.select_top_p(s, 0.99).tolist() == [0]
+    assert O.stored_top_p(0.99) == float(np.float32(0.99)) > 0.99
+    assert O.select_top_p(s, O.stored_top_p(0.99)).tolist() == [0, 1]
+    assert O.stored_top_p(1.0) == 1.0 and O.stored_top_p(0.5) == 0.5
+
+
+def test_decode_step_applies_the_stored_top_p(monkeypatch):
+    import oracle.sparse_decode_oracle as OM
+    seen = []
+    real = OM.select_top_p
+    monkeypatch.setattr(OM, "select_top_p", lambda s, p: seen.append(p) or real(s, p))
+    prob, Hq, Hkv, d, r = _tiny_problem(12, page_perm=False)
+    cfg = O.OracleConfig(Hq, Hkv, d, r, 16, [1, 1, 0, 0], 8, 2, "top_p", top_p=0.99)
+    O.decode_reference(cfg, **prob)
+    assert seen and all(p == float(np.float32(0.99)) for p in seen)
+
+
 def test_top_p_one_keeps_everything_and_scale_invariance_of_order():
     s = np.array([3.0, -1.0, 2.0])
     assert O.select_top_p(s, 1.0).tolist() == [0, 1, 2]
