@@ -35,6 +35,7 @@ Readings taken where the pages are silent (each is listed in the design doc):
     even, from the exact value);
   * index score s_j = c * <q~, k~_j> with c = index_scale (default sqrt(d)/r);
   * top-p keeps every token whose score ties the threshold score;
+  * p and top-k's frac are the float32 values the configuration stores;
   * top-k breaks ties by the lower position;
   * p >= 1 keeps every token;
   * the attention logit scale is attn_scale (default 1/sqrt(d)).
