@@ -570,10 +570,10 @@ size_t hist_bytes(int GR, bool topp) {
 
 int group_rows(const Tables &tb) { return pow2_ceil(std::max(1, tb.max_ret)); }
 
-Plan make_plan(const Shape &sh, const Tables &tb, int batch, bool topp, int smem_limit) {
+Plan make_plan(const Shape &sh, const Tables &tb, int batch, bool topp, int smem_limit, int sms) {
   const int GR = group_rows(tb);
   const int items = std::max(1, batch * tb.n_ret);
-  int C = pow2_ceil((2 * 148 + items - 1) / items);
+  int C = pow2_ceil((2 * sms + items - 1) / items);      // about two CTAs per SM over all items
   C = std::min(C, kMaxCluster);
   const int max_c = std::max(1, std::min(kMaxCluster, 1 << (31 - __builtin_clz(std::max(1, sh.max_pages)))));
   C = std::min(C, max_c);
@@ -701,11 +701,19 @@ cudaError_t dispatch_gr(const SelectArgs &a, const Shape &sh, const Tables &tb, 
   }
 }
 
-int smem_limit_bytes() {
-  int dev = 0, v = 0;
+// Per device, looked up once: the opt-in shared memory per block and the
+// number of multiprocessors.
+struct DeviceLimits {
+  int smem;
+  int sms;
+};
+
+DeviceLimits device_limits() {
+  int dev = 0, v = 0, n = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-  return v > 0 ? v : 48 * 1024;
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return DeviceLimits{v > 0 ? v : 48 * 1024, n > 0 ? n : 1};
 }
 
 }  // namespace
@@ -725,15 +733,15 @@ cudaError_t launch_select(const SelectArgs &a, const Shape &sh, const Tables &tb
   cudaGetDevice(&dev);
   const bool topp = a.mode == SD_TOP_P;
   static std::mutex mu;
-  static std::map<int, int> smem_limit;
-  int lim;
+  static std::map<int, DeviceLimits> limits;
+  DeviceLimits lim;
   {
     std::lock_guard<std::mutex> lk(mu);
-    auto it = smem_limit.find(dev);
-    if (it == smem_limit.end()) it = smem_limit.emplace(dev, smem_limit_bytes()).first;
+    auto it = limits.find(dev);
+    if (it == limits.end()) it = limits.emplace(dev, device_limits()).first;
     lim = it->second;
   }
-  Plan p = make_plan(sh, tb, a.batch, topp, lim);
+  Plan p = make_plan(sh, tb, a.batch, topp, lim.smem, lim.sms);
   // A cluster whose CTAs cannot be co-resident would fail to launch: fall back
   // to the portable size with scores in the workspace.
   const int fits = topp ? (p.smem ? active_clusters_gr<true, true>(tb, p, dev) : active_clusters_gr<true, false>(tb, p, dev))
