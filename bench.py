@@ -445,7 +445,7 @@ def cpu_baseline(w, budget_s=15.0):
     import numpy as np
 
     import oracle as O
-    from tests.helpers import oracle_config, oracle_inputs
+    from oracle.workload_inputs import oracle_config, oracle_inputs
     cfg = oracle_config(w)
     G = w.num_q_heads // w.num_kv_heads
     done = 0
@@ -477,7 +477,7 @@ def run_reference(args):
         return
     import torch
 
-    from tests.helpers import oracle_config, oracle_inputs
+    from oracle.workload_inputs import oracle_config, oracle_inputs
     from workloads import make_workload
     import oracle as O
     dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")

@@ -2,9 +2,10 @@
 
     python -m head_wise_sparse_02_b200.build [--force] [-v]
 
-Each .cu under csrc/ is compiled to an object in _build/, then linked into
-lib/libsparsedecode.so with the CUDA runtime linked statically, so that the
-library loads (and exports its symbols) on a machine without a GPU.
+Each .cu under csrc/ is compiled to an object in a temporary directory
+(removed afterwards, so that only the library stays in the tree), then linked
+into lib/libsparsedecode.so with the CUDA runtime linked statically, so that
+the library loads (and exports its symbols) on a machine without a GPU.
 """
 
 from __future__ import annotations
@@ -15,12 +16,12 @@ import os
 import shutil
 import subprocess
 import sys
+import tempfile
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
-BUILD = os.path.join(HERE, "_build")
 LIBDIR = os.path.join(HERE, "lib")
 LIB = os.path.join(LIBDIR, "libsparsedecode.so")
 
@@ -52,16 +53,21 @@ def _stale(target, deps) -> bool:
 
 
 def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    os.makedirs(BUILD, exist_ok=True)
     os.makedirs(LIBDIR, exist_ok=True)
     deps = _deps() + [os.path.abspath(__file__)]
     if not force and not _stale(LIB, deps):
         return LIB
+    with tempfile.TemporaryDirectory(prefix="sd_build_") as tmp:
+        _compile_and_link(tmp, verbose, extra)
+    return LIB
+
+
+def _compile_and_link(build_dir: str, verbose: bool, extra) -> None:
     cc = nvcc()
     objs = []
     cmds = []
     for src in _sources():
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
         cmds.append([cc, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj])
 
@@ -79,7 +85,6 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     link = [cc, *ARCH, "-shared", "-cudart", "static", "-Xcompiler", "-fPIC", "-o", LIB + ".tmp", *objs]
     run(link)
     os.replace(LIB + ".tmp", LIB)
-    return LIB
 
 
 def main(argv=None):

@@ -11,6 +11,7 @@ import numpy as np
 import torch
 
 import oracle as O
+from oracle.workload_inputs import bf16_bits, oracle_config, oracle_inputs  # noqa: F401
 from workloads import Workload, keys_at, slots_of
 
 # Tolerances stated for the path: sets bit-exact except tokens whose oracle
@@ -19,45 +20,6 @@ from workloads import Workload, keys_at, slots_of
 BAND_REL = 1e-5
 OUT_MAX_ABS = 2e-3
 OUT_REL_L2 = 1e-3
-
-
-def bf16_bits(t: torch.Tensor) -> np.ndarray:
-    return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
-
-
-def oracle_config(w: Workload) -> O.OracleConfig:
-    return O.OracleConfig(w.num_q_heads, w.num_kv_heads, w.head_dim, w.index_dim, w.page_size,
-                          list(w.head_is_retrieval), w.window, w.num_sinks, w.mode, top_p=w.top_p,
-                          top_k=w.top_k, top_k_frac=w.top_k_frac,
-                          attn_scale=w.attn_scale or None, index_scale=w.index_scale or None)
-
-
-def oracle_inputs(w: Workload, seqs: Optional[Sequence[int]] = None):
-    """numpy inputs of the oracle for the sequences `seqs` (all by default).
-
-    Only the pages of those sequences are copied; they are renumbered in a
-    compact pool and the page table is remapped accordingly (a relabelling of
-    storage, which the page-table indirection makes invisible)."""
-    if seqs is None:
-        seqs = list(range(w.batch))
-    seqs = list(seqs)
-    lens = w.seq_lens.cpu().numpy()
-    pt = w.page_table.cpu().numpy()
-    pages = []
-    new_pt = -np.ones((len(seqs), pt.shape[1]), np.int64)
-    for i, b in enumerate(seqs):
-        m = math.ceil(int(lens[b]) / w.page_size)
-        ids = pt[b, :m].astype(np.int64)
-        new_pt[i, :m] = np.arange(len(pages), len(pages) + m)
-        pages.extend(ids.tolist())
-    idx = torch.tensor(pages, dtype=torch.long, device=w.k_cache.device)
-    kc = bf16_bits(w.k_cache.index_select(0, idx)) if len(pages) else np.zeros((0,) + tuple(w.k_cache.shape[1:]), np.uint16)
-    vc = bf16_bits(w.v_cache.index_select(0, idx)) if len(pages) else np.zeros_like(kc)
-    sel = torch.tensor(seqs, dtype=torch.long, device=w.q.device)
-    return dict(proj=w.proj.float().cpu().numpy(),
-                q_pre=w.q_pre.index_select(0, sel).float().cpu().numpy(),
-                q=w.q.index_select(0, sel).float().cpu().numpy(),
-                k_cache=kc, v_cache=vc, page_table=new_pt, seq_lens=lens[seqs])
 
 
 def make_step(w: Workload, build_index: bool = True):

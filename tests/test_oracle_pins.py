@@ -422,3 +422,65 @@ def test_decode_step_composed_on_planted_needles(mode):
     for h in (2, 3):
         want = _sdpa64(prob["q"][0, h], K[loc, 1], V[loc, 1], 1 / math.sqrt(d))
         np.testing.assert_allclose(res.out[(0, h)], want, rtol=1e-11, atol=1e-12)
+
+
+# ---------------------------------------------------------------- retained mass
+
+def test_mass_retained_closed_forms():
+    """Share of the full softmax mass on a kept set: the whole set gives 1, the
+    empty set 0, and two tokens with logits l0, l1 give the logistic of their
+    gap, 1 / (1 + e^(l1 - l0)) for keeping token 0 alone."""
+    rng = np.random.default_rng(3)
+    d = 16
+    K = rng.standard_normal((40, d)).astype(np.float32)
+    q = rng.standard_normal(d).astype(np.float32)
+    assert O.mass_retained(q, K, np.arange(40), 0.25) == pytest.approx(1.0, abs=1e-15)
+    assert O.mass_retained(q, K, np.zeros(0, np.int64), 0.25) == 0.0
+    # two keys along q: logits are scale * <q, k> computed by hand
+    q2 = np.zeros(d, np.float32)
+    q2[0] = 2.0
+    K2 = np.zeros((2, d), np.float32)
+    K2[0, 0], K2[1, 0] = 3.0, -1.5                       # logits 0.5 * (6, -3) = (3, -1.5)
+    want = 1.0 / (1.0 + math.exp(-1.5 - 3.0))
+    assert O.mass_retained(q2, K2, [0], 0.5) == pytest.approx(want, rel=1e-14)
+    assert O.mass_retained(q2, K2, [1], 0.5) == pytest.approx(1.0 - want, rel=1e-12)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_mass_retained_is_the_exact_share_on_small_integer_logits(seed):
+    """Logits that are small integers times ln 2 make every weight a power of
+    two, so the share is an exact rational: sum_{j in S} 2^{a_j} / sum_j 2^{a_j}.
+    Checked with Fraction arithmetic on every subset of a 7-token context (a
+    dropped term, a wrong index or a missing normalisation fails one)."""
+    rng = np.random.default_rng(100 + seed)
+    a = rng.integers(-6, 7, size=7)
+    d = 4
+    K = np.zeros((7, d), np.float64)
+    K[:, 0] = a * math.log(2.0)                          # logit_j = <q, k_j> = a_j ln 2
+    q = np.zeros(d)
+    q[0] = 1.0
+    tot = sum(Fraction(2) ** int(x) for x in a)
+    for mask in range(1 << 7):
+        S = [j for j in range(7) if mask >> j & 1]
+        want = sum((Fraction(2) ** int(a[j]) for j in S), Fraction(0)) / tot
+        got = O.mass_retained(q, K, S, 1.0)
+        assert got == pytest.approx(float(want), rel=1e-12, abs=1e-15)
+
+
+def test_mass_retained_of_a_top_p_set_on_full_logits_reaches_p():
+    """When the index scores are the attention logits themselves (identity
+    projection, index scale = attention scale), the top-p set of the index
+    holds at least p of the full softmax mass, and dropping its lowest-scored
+    token leaves less than p: the defining property, read through the
+    retained-mass diagnostic."""
+    rng = np.random.default_rng(9)
+    d = 16
+    K = O.bf16_round(rng.standard_normal((300, d)) * 2.0)
+    q = O.bf16_round(rng.standard_normal(d))
+    s = O.index_scores(q, K, 0.25)
+    for p in (0.5, 0.9, 0.99):
+        S = O.select_top_p(s, p)
+        m = O.mass_retained(q, K, S, 0.25)
+        assert m >= p - 1e-12
+        low = S[np.argmin(s[S])]
+        assert O.mass_retained(q, K, np.setdiff1d(S, [low]), 0.25) < p
