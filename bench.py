@@ -238,6 +238,103 @@ def union_rows(sel_idx, sel_count, w):
     return total, index_tokens
 
 
+L2_BYTES = 126 * 2 ** 20
+L2_FLUSH_BYTES = 512 * 2 ** 20
+# a step that streams at least this many bytes (4x the L2, in the same order
+# every step) leaves nothing useful in L2 for the next one: no flush is needed
+NO_FLUSH_ABOVE = 4 * L2_BYTES
+
+
+def streamed_bytes_lower_bound(w) -> int:
+    """Bytes every step reads whatever the selection: the index of every
+    retrieval (sequence, KV group) and the sink + window rows of every local
+    one (selected rows come on top)."""
+    G = w.num_q_heads // w.num_kv_heads
+    ret_groups = sum(1 for g in range(w.num_kv_heads) if any(w.head_is_retrieval[g * G:(g + 1) * G]))
+    loc_groups = sum(1 for g in range(w.num_kv_heads) if not all(w.head_is_retrieval[g * G:(g + 1) * G]))
+    total = 0
+    for n in w.seq_lens.cpu().tolist():
+        local_rows = min(n, w.num_sinks) + max(0, n - max(min(n, w.num_sinks), n - w.window))
+        total += ret_groups * 32 * n + loc_groups * local_rows * 4 * w.head_dim
+    return total
+
+
+def l2_flush_needed(mode: str, w) -> bool:
+    if mode == "on":
+        return True
+    if mode == "off":
+        return False
+    return streamed_bytes_lower_bound(w) < NO_FLUSH_ABOVE
+
+
+def workload_label(name: str, w) -> str:
+    lens = w.seq_lens
+    n = (f"N={int(lens.max())}" if int(lens.min()) == int(lens.max())
+         else f"N={int(lens.min())}..{int(lens.max())}")
+    mode = (f"top-k frac {w.top_k_frac}" if w.mode == "top_k" and not w.top_k
+            else f"top-k {w.top_k}" if w.mode == "top_k" else f"top-p {w.top_p}")
+    ret = sum(w.head_is_retrieval)
+    heads = f"{ret} retrieval ({mode})"
+    if ret < w.num_q_heads:
+        heads += f" + {w.num_q_heads - ret} local (window {w.window} + {w.num_sinks} sinks)"
+    return (f"{name}: B={w.batch}, Hq={w.num_q_heads}/Hkv={w.num_kv_heads}, d={w.head_dim}, {n}, "
+            f"{heads}" + (f", {w.notes['profile']}" if "profile" in w.notes else ""))
+
+
+def bench_config(args, w, ws: int, flush: bool):
+    """The `config` object of the JSON line; both arms print the same one."""
+    return {
+        "workload": workload_label(args.workload, w),
+        "batch_per_gpu": w.batch, "seq_len": int(w.seq_lens.max()),
+        "parallelism": f"replicas x{ws} (sequences sharded, no collective)",
+        "l2": ("flushed between steps (512 MiB write, untimed)" if flush
+               else "no flush: every step streams more than 4x the 126 MB L2"),
+    }
+
+
+def selection_diagnostics(w, st, budget_s: float = 20.0, max_pairs: int = 16):
+    """|S|/N of the retrieval heads and, on a sample of (sequence, retrieval
+    head) pairs, the share of the full-attention softmax mass that the GPU's
+    selected set holds (the oracle's mass_retained, float64 on the host).
+    Diagnostics only: nothing here is timed or compared."""
+    import numpy as np
+
+    import oracle as O
+    from oracle.workload_inputs import oracle_config, oracle_inputs
+    retr = [h for h in range(w.num_q_heads) if w.head_is_retrieval[h]]
+    if not retr:
+        return {"retrieval_heads": 0}
+    cnt = st.sel_count.cpu().numpy().astype(np.float64)
+    lens = w.seq_lens.cpu().numpy().astype(np.float64)
+    frac = cnt / np.maximum(lens[:, None], 1.0)
+    cfg = oracle_config(w)
+    attn_scale, _ = cfg.scales()
+    G = w.num_q_heads // w.num_kv_heads
+    rng = np.random.default_rng(0)
+    pairs = [(int(b), int(retr[i])) for b, i in zip(rng.integers(0, w.batch, max_pairs),
+                                                   rng.integers(0, len(retr), max_pairs))]
+    masses = []
+    t0 = time.perf_counter()
+    for b, h in pairs:
+        if time.perf_counter() - t0 > budget_s:
+            break
+        inp = oracle_inputs(w, [b])
+        n = int(inp["seq_lens"][0])
+        K = O.gather_rows(inp["k_cache"], inp["page_table"][0], n, h // G, cfg.page_size)
+        r = retr.index(h)
+        k = int(st.sel_count[b, r])
+        S = st.sel_idx[b, r, :k].cpu().numpy().astype(np.int64)
+        masses.append(O.mass_retained(inp["q"][0, h], K, S, attn_scale))
+    out = {"selected_frac": {"mean": round(float(frac.mean()), 5), "min": round(float(frac.min()), 5),
+                             "max": round(float(frac.max()), 5)}}
+    if masses:
+        out["mass_retained"] = {"mean": round(float(np.mean(masses)), 5), "min": round(float(np.min(masses)), 5),
+                                "sample": f"{len(masses)} random (sequence, retrieval head) pairs; float64 "
+                                          f"oracle on the host: share of the full softmax of q.k over all "
+                                          f"N tokens that falls on the GPU-selected set"}
+    return out
+
+
 def size_overrides(args):
     """--batch / --seq-len shrink the workload (profiling cases); the JSON
     config reports the sizes actually run."""
@@ -246,7 +343,24 @@ def size_overrides(args):
         kw["B"] = args.batch
     if args.seq_len:
         kw["N"] = args.seq_len
+    if args.top_p:
+        kw["top_p"] = args.top_p
+    if args.alpha:
+        kw["alpha"] = args.alpha
     return kw
+
+
+def workload_for_rank(args, device, rank: int):
+    """The rank's own seeded batch: the workload's default seed (or --seed)
+    offset per rank (weak scaling)."""
+    from workloads import make_workload
+    kw = size_overrides(args)
+    if args.seed is not None or rank:
+        import inspect
+        from workloads.synthetic import BUILDERS
+        base = args.seed if args.seed is not None else inspect.signature(BUILDERS[args.workload]).parameters["seed"].default
+        kw["seed"] = rank_seed(base, rank)
+    return make_workload(args.workload, device, **kw)
 
 
 def run_ours(args):
@@ -263,7 +377,7 @@ def run_ours(args):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
-    w = make_workload(args.workload, dev, seed=rank_seed(args.seed, rank), **size_overrides(args))
+    w = workload_for_rank(args, dev, rank)
     B, Hq, d = w.batch, w.num_q_heads, w.head_dim
     st = DecodeStep(k_cache=w.k_cache, v_cache=w.v_cache, page_table=w.page_table, seq_lens=w.seq_lens,
                     proj=w.proj, num_q_heads=Hq, head_is_retrieval=w.head_is_retrieval, window=w.window,
@@ -277,23 +391,24 @@ def run_ours(args):
     new_keys = keys_at(w, new_slots)
     stream = torch.cuda.current_stream()
 
-    ev = {k: [] for k in ("index_keys", "select", "attend")}
+    calls = ("index_keys", "select", "attend")
 
-    def step(record=False):
-        if record:
-            e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
-            e2 = torch.cuda.Event(enable_timing=True); e3 = torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
+    def step(ev=None):
+        """One decode step; with `ev`, an event pair around each call."""
+        if ev is not None:
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            e[0].record(stream)
         st.sd.index_keys(new_keys, new_slots, st.index_cache, stream)
-        if record:
-            e1.record(stream)
+        if ev is not None:
+            e[1].record(stream)
         st.select(w.q_pre, stream)
-        if record:
-            e2.record(stream)
+        if ev is not None:
+            e[2].record(stream)
         st.attend(w.q, stream=stream)
-        if record:
-            e3.record(stream)
-            ev["index_keys"].append((e0, e1)); ev["select"].append((e1, e2)); ev["attend"].append((e2, e3))
+        if ev is not None:
+            e[3].record(stream)
+            for i, k in enumerate(calls):
+                ev[k].append((e[i], e[i + 1]))
 
     for _ in range(args.warmup):
         step()
@@ -303,21 +418,52 @@ def run_ours(args):
         raise RuntimeError(f"device error word {word:#x} after warm-up")
     rows, index_tokens = union_rows(st.sel_idx, st.sel_count, w)
     sel_sizes = st.sel_count.float()
+    row_bytes = 4 * d                                   # K + V row, bf16
+    step_bytes = 32 * index_tokens + row_bytes * rows
+    flush = l2_flush_needed(args.l2_flush, w)
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev) if flush else None
+
+    def timed(n_steps, with_calls):
+        """Device time of n_steps steps (ms per step) and, with_calls, the
+        per-call event pairs.  Without an L2 flush one event pair brackets
+        all steps; with it, each step has its own pair and the flush (a
+        write of a buffer larger than L2) runs between them, untimed."""
+        ev = {k: [] for k in calls} if with_calls else None
+        if not flush:
+            a0 = torch.cuda.Event(enable_timing=True); a1 = torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            for _ in range(n_steps):
+                step(ev)
+            a1.record(stream)
+            torch.cuda.synchronize()
+            return a0.elapsed_time(a1) / n_steps, ev
+        pairs = []
+        for _ in range(n_steps):
+            flush_buf.zero_()
+            a0 = torch.cuda.Event(enable_timing=True); a1 = torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            step(ev)
+            a1.record(stream)
+            pairs.append((a0, a1))
+        torch.cuda.synchronize()
+        return sum(x.elapsed_time(y) for x, y in pairs) / n_steps, ev
 
     clocks = ClockSampler(local)
     clocks.start()
     barrier()
     torch.cuda.synchronize()
-    t0 = torch.cuda.Event(enable_timing=True); t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for _ in range(args.steps):
-        step(record=True)
-    t1.record(stream)
-    torch.cuda.synchronize()
+    ms, _ = timed(args.steps, False)
     barrier()
     clk = clocks.stop()
-    ms = t0.elapsed_time(t1) / args.steps
     ms_max = max_over_ranks(ms, dev)
+    # per-call device times: the same steps again, with an event pair around
+    # each call (events between calls keep a call's first kernel from
+    # overlapping the previous call's last one, so these sum to a little
+    # more than the step time above)
+    barrier()
+    torch.cuda.synchronize()
+    ms_calls, ev = timed(args.steps, True)
+    barrier()
     per = {k: sum(a.elapsed_time(b) for a, b in v) / len(v) for k, v in ev.items()}
 
     # ---- end to end through the public API with host buffers ----
@@ -341,27 +487,38 @@ def run_ours(args):
         e2e_step()
     torch.cuda.synchronize()
     barrier()
-    a0 = torch.cuda.Event(enable_timing=True); a1 = torch.cuda.Event(enable_timing=True)
-    a0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    a1.record(stream)
-    torch.cuda.synchronize()
+    if not flush:
+        a0 = torch.cuda.Event(enable_timing=True); a1 = torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        e2e_one = a0.elapsed_time(a1) / args.steps
+    else:
+        pairs = []
+        for _ in range(args.steps):
+            flush_buf.zero_()
+            a0 = torch.cuda.Event(enable_timing=True); a1 = torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            e2e_step()
+            a1.record(stream)
+            pairs.append((a0, a1))
+        torch.cuda.synchronize()
+        e2e_one = sum(x.elapsed_time(y) for x, y in pairs) / args.steps
     barrier()
-    e2e_ms = max_over_ranks(a0.elapsed_time(a1) / args.steps, dev)
+    e2e_ms = max_over_ranks(e2e_one, dev)
     word = st.error_word()
     if word:
         raise RuntimeError(f"device error word {word:#x} after timing")
 
     # ---- roofline of the dominant kernel ----
-    row_bytes = 4 * d                                   # K + V row, bf16
     index_bytes = 32 * index_tokens
     kv_bytes = row_bytes * rows
     kern_bytes = {"select": index_bytes, "attend": kv_bytes, "index_keys": B * w.num_kv_heads * (2 * d + 32)}
     dominant = max(per, key=per.get)
     peak, peak_kind = load_peak()
     achieved = kern_bytes[dominant] / (per[dominant] * 1e-3) / 1e9
-    step_bytes = index_bytes + kv_bytes
     head_steps = ws * B * Hq
     value = head_steps / (ms_max * 1e-3)
     res = {
@@ -369,18 +526,13 @@ def run_ours(args):
         "warmup": args.warmup, "ms_per_step": round(ms_max, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "storage_dtype": "bf16",
         "data": "synthetic (seeded; no datasets or trained weights)",
-        "config": {
-            "workload": f"{args.workload}: B={B}, Hq={Hq}/Hkv={w.num_kv_heads}, d={d}, "
-                        f"N={int(w.seq_lens.max())}, mode={w.mode}"
-                        + (f", top-k frac {w.top_k_frac}" if w.mode == "top_k" else f", top-p {w.top_p}"),
-            "batch_per_gpu": B, "seq_len": int(w.seq_lens.max()), "parallelism": f"replicas x{ws} (sequences sharded, no collective)",
-            "l2": "no flush: bytes touched per step exceed the 126 MB L2",
-        },
+        "config": bench_config(args, w, ws, flush),
         "tokens_per_s": round(ws * B / (ms_max * 1e-3), 1),
         "hbm_gbs_achieved_step": round(step_bytes / (ms * 1e-3) / 1e9, 1),
         "frac_of_8tbs_step": round(step_bytes / (ms * 1e-3) / 1e9 / CONTRACT_GBS, 4),
         "algorithmic_bytes_per_step": step_bytes,
         "ms_per_call": {k: round(v, 4) for k, v in per.items()},
+        "ms_per_step_with_call_events": round(ms_calls, 4),
         "algorithmic_bytes_per_call": kern_bytes,
         "selected_per_head": {"mean": round(float(sel_sizes.mean()), 1), "min": int(sel_sizes.min()),
                               "max": int(sel_sizes.max())},
@@ -395,6 +547,8 @@ def run_ours(args):
         "gpu_launches": kernels_per_step(w) * args.steps,
         "clocks": clk,
     }
+    if rank == 0 and ws == 1 and not args.no_diagnostics:
+        res["diagnostics"] = selection_diagnostics(w, st, budget_s=args.diag_budget)
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
     st.close()
@@ -481,7 +635,7 @@ def run_reference(args):
     from workloads import make_workload
     import oracle as O
     dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
-    w = make_workload(args.workload, dev, seed=rank_seed(args.seed, 0), **size_overrides(args))
+    w = workload_for_rank(args, dev, 0)
     cfg = oracle_config(w)
     G = w.num_q_heads // w.num_kv_heads
     inp = oracle_inputs(w, [0])
@@ -501,12 +655,12 @@ def run_reference(args):
     res = {"impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": UNIT, "n_gpus": ws,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-           "data": "synthetic (seeded)",
-           "config": {"workload": f"{args.workload}: B={w.batch}, Hq={w.num_q_heads}/Hkv={w.num_kv_heads}, "
-                                  f"d={w.head_dim}, N={int(w.seq_lens.max())}",
-                      "step_sample": f"one (sequence, KV group) slab = {G} head-steps per step"},
+           "data": "synthetic (seeded; no datasets or trained weights)",
+           "config": bench_config(args, w, ws, l2_flush_needed(args.l2_flush, w)),
            "cpu_baseline": {"kind": "oracle", "cores": _blas_threads(), "value": round(v, 3), "unit": UNIT,
-                            "sample": f"{args.steps} slabs of {G} heads, float64 numpy oracle"},
+                            "sample": f"each step: one (sequence, KV group) slab of the same workload = "
+                                      f"{G} head-steps, float64 numpy oracle, index prebuilt (untimed); "
+                                      f"{args.steps} slabs"},
            "e2e": {"value": round(v, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(res), flush=True)
 
@@ -518,11 +672,17 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="topk_128k")
-    ap.add_argument("--seed", type=int, default=2)
+    ap.add_argument("--seed", type=int, default=None, help="base seed (default: the workload's own)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling)")
     ap.add_argument("--seq-len", type=int, default=0, help="override the workload's context length")
+    ap.add_argument("--top-p", type=float, default=0.0, help="override the workload's top-p")
+    ap.add_argument("--alpha", type=float, default=0.0, help="long_zipf: Zipf exponent of the score profile")
+    ap.add_argument("--l2-flush", choices=["auto", "on", "off"], default="auto",
+                    help="flush L2 between timed steps (auto: when a step touches < 8x the L2)")
+    ap.add_argument("--no-diagnostics", action="store_true")
+    ap.add_argument("--diag-budget", type=float, default=20.0)
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)          # timing rule: at least 3 warm-up steps
     if args.impl == "reference":

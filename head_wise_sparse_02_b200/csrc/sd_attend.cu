@@ -20,9 +20,11 @@
 //         every union row is read once for all the group's heads that
 //         selected it.  The page of each row is resolved here, from a
 //         shared-memory copy of the span's page-table slice; the union sizes
-//         are summed per item.
-//   layout one CTA lays all items end to end and writes the first tile of
-//         each (a prefix sum over the items' tile counts).
+//         per span are written out.
+//   layout one CTA sums the plan's span counts of each retrieval item, lays
+//         all items end to end and writes the first tile of each (a prefix
+//         sum over the items' tile counts); it also clears the merge tickets,
+//         so that no call needs memory that starts at zero.
 //   main  a persistent grid, one CTA per resident slot.  CTA c takes the
 //         equal share [W c / P, W (c + 1) / P) of all W tiles and walks the
 //         items it overlaps (usually one or two), so that its rings run
@@ -64,8 +66,19 @@ constexpr int kTileRows = 16;
 constexpr int kTileRing = 3;            // tiles in flight per warp
 constexpr int kMaxGrid = 4096;          // persistent CTAs (partial slots are sized for this)
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, int src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+// 16-byte copy global -> shared, bypassing L1, with an L2 eviction-priority
+// hint: streamed cache rows are read once per call, so they are marked
+// evict-first and leave the small tables, lists and code of the surrounding
+// kernels in L2
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, int src_bytes, uint64_t policy) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;\n" ::"r"(dst), "l"(src),
+               "r"(src_bytes), "l"(policy)
+               : "memory");
+}
+__device__ __forceinline__ uint64_t evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(p));
+  return p;
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 template <int N>
@@ -165,8 +178,8 @@ struct AttWs {
   uint16_t *plan_mask;      // [B][n_ret][ns][span]: heads (bit i = i-th head of the group)
   int *plan_cnt;            // [B][n_ret][ns]
   long long *tstart;        // [ni + 1]: first tile of each item; tstart[ni] = all tiles
-  int *item_rows;           // [ni]: rows of each item           } zeroed before
-  unsigned *tickets;        // [ni]: partials merged per item     } every call
+  int *item_rows;           // [ni]: rows of each item (layout)
+  unsigned *tickets;        // [ni]: partials merged per item (cleared by the layout)
 };
 
 __device__ __forceinline__ const Group &item_group(const Tables &tb, const AttParams &ap, int i, int &b,
@@ -187,9 +200,10 @@ __device__ __forceinline__ long long clamp_len(const AttendArgs &a, const Shape 
 }
 
 // Tile counts and first tiles of all items, by one CTA (block size a multiple
-// of 32, at most 1024).  Retrieval items' rows were summed into item_rows by
-// the plan CTAs; local items' rows follow from N.  Items without rows get a
-// zero output here, since no main CTA visits them.
+// of 32, at most 1024).  A retrieval item's rows are the sum of its spans'
+// union counts (plan_cnt); a local item's rows follow from N.  Items without
+// rows get a zero output here, since no main CTA visits them.  The merge
+// tickets of the main kernel are cleared here.
 template <int D>
 __device__ void item_prefix(const AttendArgs &a, const Shape &sh, const Tables &tb, const AttParams &ap,
                             const AttWs &ws) {
@@ -208,15 +222,19 @@ __device__ void item_prefix(const AttendArgs &a, const Shape &sh, const Tables &
       long long rows;
       const long long N0 = a.seq_lens[b];
       if (N0 < 0 || N0 > sh.max_len) raise_error(a.err, SD_EBIT_SEQLEN);
+      const long long N = clamp_len(a, sh, b);
       if (is_ret) {
-        rows = __ldcg(ws.item_rows + i);
+        const int ns_item = (int)((N + ap.span - 1) / ap.span);
+        const int *cnt = ws.plan_cnt + ((long long)b * tb.n_ret + i % tb.n_ret) * ap.ns;
+        rows = 0;
+        for (int s = 0; s < ns_item; ++s) rows += __ldcg(cnt + s);
       } else {
-        const long long N = clamp_len(a, sh, b);
         const long long la = std::min<long long>(a.num_sinks, N);
         const long long lw = std::max<long long>(la, N - a.window);
         rows = la + (N - lw);
-        ws.item_rows[i] = (int)rows;
       }
+      ws.item_rows[i] = (int)rows;
+      ws.tickets[i] = 0u;
       nt = (rows + kTileRows - 1) / kTileRows;
       if (rows == 0)
         for (int x = 0; x < grp.n * D; ++x) a.out[((long long)b * sh.Hq + grp.q_head[x / D]) * D + x % D] = 0.0f;
@@ -247,12 +265,14 @@ __device__ void item_prefix(const AttendArgs &a, const Shape &sh, const Tables &
 template <int D>
 __global__ void __launch_bounds__(1024)
 attend_prefix_kernel(const AttendArgs a, const Shape sh, const Tables tb, const AttParams ap, const AttWs ws) {
+  pdl_wait();
+  pdl_trigger();
   item_prefix<D>(a, sh, tb, ap, ws);
 }
 
 // ============================================================== plan kernel
-// Union list of the span [p0, p1) of retrieval item (b, gi): plan_cnt[slot],
-// the list in plan_row / plan_mask, and the count added to the item's rows.
+// Union list of the span [p0, p1) of retrieval item (b, gi): its length in
+// plan_cnt[slot], the list in plan_row / plan_mask.
 // hbm: [GR][span / 32] bitmap words; pslice: the span's pages.
 template <int GR>
 __device__ void plan_span(const AttendArgs &a, const Shape &sh, const Tables &tb, const AttParams &ap,
@@ -357,10 +377,7 @@ __device__ void plan_span(const AttendArgs &a, const Shape &sh, const Tables &tb
       ++o;
     }
   }
-  if (tid == 0) {
-    ws.plan_cnt[slot] = (int)total;
-    if (total) atomicAdd(ws.item_rows + (long long)b * tb.n_ret + gi, (int)total);
-  }
+  if (tid == 0) ws.plan_cnt[slot] = (int)total;
 }
 
 // dynamic shared memory: [per-head bitmaps: GR x span / 32 words][page slice: span / 16 ints]
@@ -372,6 +389,8 @@ attend_plan_kernel(const AttendArgs a, const Shape sh, const Tables tb, const At
   __shared__ Group grp;
   extern __shared__ uint32_t plan_dyn[];
   if (tid == 0) grp = tb.ret[gi];
+  pdl_wait();
+  pdl_trigger();
   __syncthreads();
   plan_span<GR>(a, sh, tb, ap, ws, grp, b, gi, split, plan_dyn, reinterpret_cast<int *>(plan_dyn + GR * (ap.span / 32)));
 }
@@ -407,6 +426,8 @@ attend_main_kernel(const AttendArgs a, const Shape sh, const Tables tb, const At
   uint16_t *wmask = reinterpret_cast<uint16_t *>(dyn + (size_t)kWarps * kTileRing * kTileB) +
                     warp * (kTileRing * kTileRows);                       // this warp's tile masks
   int *pre = reinterpret_cast<int *>(dyn + (size_t)kWarps * kTileRing * kTileB + kWarps * kTileRing * kTileRows * 2);
+  pdl_wait();
+  pdl_trigger();
 
   // ---- this CTA's share of the tiles -----------------------------------------
   const long long W = __ldcg(ws.tstart + ap.ni);
@@ -436,6 +457,7 @@ attend_main_kernel(const AttendArgs a, const Shape sh, const Tables tb, const At
   const uint32_t k_lane = (lr + (lm >> 1) * 8) * kPitch + (lm & 1) * 16;   // K: rows (0-7 | 8-15) x chunk (2k | 2k+1)
   const uint32_t v_lane = kTileRows * kPitch + (lr + (lm & 1) * 8) * kPitch + (lm >> 1) * 16;   // V: rows x chunk (n | n+1)
   const float sc = a.attn_scale * kLog2e;
+  const uint64_t l2_stream = evict_first_policy();
   uint32_t zu = 0u;
   float zf = 0.0f;
   asm volatile("" : "+r"(zu), "+f"(zf));             // opaque zeros: one register each
@@ -561,7 +583,7 @@ attend_main_kernel(const AttendArgs a, const Shape sh, const Tables tb, const At
 #pragma unroll
         for (int j = 0; j < kTileRows / RPH; ++j) {
           const uint32_t rj = __shfl_sync(kFull, row, j * RPH + c_sub);
-          cp_async16(dst + j * RPH * kPitch, src + (size_t)rj * kRowB, 16);
+          cp_async16(dst + j * RPH * kPitch, src + (size_t)rj * kRowB, 16, l2_stream);
         }
       }
       cp_async_commit();
@@ -874,12 +896,11 @@ cudaError_t launch_t(const AttendArgs &a, const Shape &sh, const Tables &tb, con
     const size_t pbytes = (size_t)GR * (p.span / 32) * 4 + (size_t)(p.span / kPage) * 4;
     e = set_smem(attend_plan_kernel<D, GR>, pbytes);
     if (e != cudaSuccess) return e;
-    attend_plan_kernel<D, GR><<<dim3(p.ns, tb.n_ret, a.batch), kPlanThreads, pbytes, st>>>(a, sh, tb, p, ws);
-    e = cudaGetLastError();
+    e = launch_pdl(attend_plan_kernel<D, GR>, dim3(p.ns, tb.n_ret, a.batch), dim3(kPlanThreads), pbytes, st, 0,
+                   a, sh, tb, p, ws);
     if (e != cudaSuccess) return e;
   }
-  attend_prefix_kernel<D><<<1, 1024, 0, st>>>(a, sh, tb, p, ws);
-  e = cudaGetLastError();
+  e = launch_pdl(attend_prefix_kernel<D>, dim3(1), dim3(1024), 0, st, 0, a, sh, tb, p, ws);
   if (e != cudaSuccess) return e;
   const size_t ring = (size_t)kWarps * kTileRing * (2 * kTileRows * (2 * D + 16));
   const size_t lists = (size_t)kWarps * kTileRing * kTileRows * 2 + (size_t)(p.ns + 1) * 4;
@@ -889,8 +910,7 @@ cudaError_t launch_t(const AttendArgs &a, const Shape &sh, const Tables &tb, con
   if (e != cudaSuccess) return e;
   const int grid = resident_ctas(attend_main_kernel<D, GR>, kThreads, bytes);
   if (grid <= 0) return cudaErrorInvalidConfiguration;
-  attend_main_kernel<D, GR><<<grid, kThreads, bytes, st>>>(a, sh, tb, p, ws);
-  return cudaGetLastError();
+  return launch_pdl(attend_main_kernel<D, GR>, dim3(grid), dim3(kThreads), bytes, st, 0, a, sh, tb, p, ws);
 }
 
 template <int D>
@@ -924,8 +944,6 @@ cudaError_t launch_attend(const AttendArgs &a, const Shape &sh, const Tables &tb
   ws.tstart = reinterpret_cast<long long *>(base + L.tstart);
   ws.item_rows = reinterpret_cast<int *>(base + L.counters);
   ws.tickets = reinterpret_cast<unsigned *>(ws.item_rows + p.ni);
-  cudaError_t e = cudaMemsetAsync(ws.item_rows, 0, (size_t)p.ni * 2 * 4, st);
-  if (e != cudaSuccess) return e;
   return sh.d == 128 ? dispatch_gr<128>(a, sh, tb, p, ws, st) : dispatch_gr<64>(a, sh, tb, p, ws, st);
 }
 

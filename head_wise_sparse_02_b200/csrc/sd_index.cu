@@ -29,7 +29,9 @@ index_keys_kernel(const uint16_t *__restrict__ k_pre, const int32_t *__restrict_
   const int t0 = blockIdx.x * kRows;
   const uint16_t *P = proj + (size_t)g * D * kIndexDim;
   for (int i = threadIdx.x; i < D * kIndexDim; i += kThreads)
-    Ps[i / kIndexDim][i % kIndexDim] = (double)bf16_to_f32(P[i]);
+    Ps[i / kIndexDim][i % kIndexDim] = (double)bf16_to_f32(P[i]);    // the context's own copy
+  pdl_wait();
+  pdl_trigger();
   for (int i = threadIdx.x; i < kRows * D; i += kThreads) {
     const int row = i / D, c = i % D, t = t0 + row;
     Ks[row][c] = (t < T) ? (double)bf16_to_f32(k_pre[((size_t)t * Hkv + g) * D + c]) : 0.0;
@@ -61,12 +63,10 @@ cudaError_t launch_index_keys(const uint16_t *k_pre, const int32_t *slots, int T
   if (T <= 0) return cudaSuccess;
   dim3 grid((T + kRows - 1) / kRows, sh.Hkv);
   if (sh.d == 128)
-    index_keys_kernel<128><<<grid, kThreads, 0, st>>>(k_pre, slots, T, index_cache, proj, sh.Hkv,
-                                                      sh.num_pages, err);
-  else
-    index_keys_kernel<64><<<grid, kThreads, 0, st>>>(k_pre, slots, T, index_cache, proj, sh.Hkv,
-                                                     sh.num_pages, err);
-  return cudaGetLastError();
+    return launch_pdl(index_keys_kernel<128>, grid, dim3(kThreads), 0, st, 0, k_pre, slots, T, index_cache, proj,
+                      sh.Hkv, sh.num_pages, err);
+  return launch_pdl(index_keys_kernel<64>, grid, dim3(kThreads), 0, st, 0, k_pre, slots, T, index_cache, proj,
+                    sh.Hkv, sh.num_pages, err);
 }
 
 }  // namespace sd

@@ -71,6 +71,45 @@ __device__ __forceinline__ void raise_error(unsigned *err, unsigned bit) {
   if (err) atomicOr(err, bit);
 }
 
+// ------------------------------------------------ programmatic dependent launch
+// Every kernel of the library is launched with programmatic stream
+// serialization (launch_pdl below): its CTAs may be scheduled while the
+// previous kernel on the stream is still finishing.  Before its first access to
+// memory that earlier work on the stream writes or reads (inputs, outputs,
+// workspace), a kernel calls pdl_wait(), which returns once the previous grid
+// has completed and its writes are visible; it may only read the library's own
+// constant tables before that.  Every kernel calls pdl_wait() on every path,
+// early returns included, so that completion stays ordered along the stream.
+// pdl_trigger() lets the next kernel be scheduled before this one ends.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
+// cudaLaunchKernelEx with programmatic stream serialization, plus an optional
+// cluster shape (x CTAs per cluster; 0 = no cluster).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       int cluster_x, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  int n = 1;
+  if (cluster_x > 0) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster_x;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    n = 2;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // ---------------------------------------------------------------- launchers
 // Each returns cudaSuccess or the launch error.
 
@@ -129,7 +168,7 @@ cudaError_t launch_attend(const AttendArgs &a, const Shape &sh, const Tables &tb
 
 // Size of the built-in attend scratch of sparse_decode_attend_noalloc.
 constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;
-// This device's scratch address (looked up on the first call per device).
+// The current device's scratch address (looked up on every call).
 cudaError_t noalloc_scratch(void **ptr);
 
 }  // namespace sd

@@ -542,6 +542,8 @@ select_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__ grou
               int tc_cap, const uint32_t *__restrict__ flags) {
   __shared__ SelShared S;
   extern __shared__ __align__(16) unsigned char dyn[];
+  pdl_wait();
+  pdl_trigger();
   const int n_items = a.batch * n_groups;
   const int n = flags ? (int)flags[n_items] : n_items;
   for (int k = blockIdx.y; k < n; k += gridDim.y) {
@@ -663,19 +665,8 @@ cudaError_t launch_t(const SelectArgs &a, const Shape &sh, const Tables &tb, con
                      cudaStream_t st, const uint32_t *flags, int grid_y) {
   cudaError_t e = ensure_attrs<GR, TOPP, SMEM>(dev, p.dyn_bytes);
   if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.cluster, grid_y, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = p.dyn_bytes;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = p.cluster;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, select_kernel<GR, TOPP, SMEM>, a, sh, tb.ret, tb.n_ret, p.tc_cap, flags);
+  return launch_pdl(select_kernel<GR, TOPP, SMEM>, dim3(p.cluster, grid_y, 1), dim3(kThreads), p.dyn_bytes, st,
+                    p.cluster, a, sh, tb.ret, tb.n_ret, p.tc_cap, flags);
 }
 
 template <bool TOPP, bool SMEM>

@@ -107,8 +107,19 @@ __device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                : "r"(addr));
 }
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, int src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+// 16-byte copy global -> shared, bypassing L1, with an L2 eviction-priority
+// hint: streamed cache rows are read once per call, so they are marked
+// evict-first and leave the small tables, lists and code of the surrounding
+// kernels in L2
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, int src_bytes, uint64_t policy) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;\n" ::"r"(dst), "l"(src),
+               "r"(src_bytes), "l"(policy)
+               : "memory");
+}
+__device__ __forceinline__ uint64_t evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(p));
+  return p;
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 template <int N>
@@ -360,6 +371,8 @@ window_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__ grou
   float (*smass)[kSampleBins] =
       reinterpret_cast<float (*)[kSampleBins]>(dyn0 + (size_t)GR * SP * 16 * 4 + (size_t)GR * kSampleBins * 4);
   if (tid == 0) grp = groups[gi];
+  pdl_wait();
+  pdl_trigger();
   __syncthreads();
   const int nr = grp.n, g = grp.kv_head;
   long long N = a.seq_lens[b];
@@ -613,6 +626,8 @@ stream_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__ grou
   __shared__ int cut_s[GR];
   __shared__ Group grp;
   if (tid == 0) grp = groups[gi];
+  pdl_wait();
+  pdl_trigger();
   __syncthreads();
   const int nr = grp.n, g = grp.kv_head;
   long long N = a.seq_lens[b];
@@ -659,11 +674,12 @@ stream_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__ grou
   const unsigned char *iblk = reinterpret_cast<const unsigned char *>(a.index_cache) + lane * 16;
   const uint32_t st_off = page_off(lane >> 1, lane & 1);
   const int nq = np > warp ? (np - warp + kW1 - 1) / kW1 : 0;
+  const uint64_t l2_stream = evict_first_policy();
   auto issue = [&](int q) {
     if (q < nq) {
       const int blk = pt_s[warp + q * kW1];
       cp_async16(ring_base + (q % kRing) * kPageBytes + st_off, iblk + (size_t)(blk >= 0 ? blk : 0) * kPageBytes,
-                 blk >= 0 ? 16 : 0);
+                 blk >= 0 ? 16 : 0, l2_stream);
     }
     cp_async_commit();
   };
@@ -882,6 +898,8 @@ topk_resolve_kernel(const SelectArgs a, const Shape sh, const StreamWs ws) {
   const int b = blockIdx.y, hr = blockIdx.x;
   const long long row = (long long)b * sh.H_ret + hr;
   int32_t *out = a.sel_idx + row * a.sel_stride;
+  pdl_wait();
+  pdl_trigger();
   long long N = a.seq_lens[b];
   N = N < 0 ? 0 : std::min<long long>(N, sh.max_len);
   const long long kb = topk_budget(a, N);
@@ -1060,6 +1078,8 @@ topp_resolve_kernel(const SelectArgs a, const Shape sh, const StreamWs ws) {
   const int b = blockIdx.y, hr = blockIdx.x;
   const long long row = (long long)b * sh.H_ret + hr;
   int32_t *out = a.sel_idx + row * a.sel_stride;
+  pdl_wait();
+  pdl_trigger();
   long long N = a.seq_lens[b];
   N = N < 0 ? 0 : std::min<long long>(N, sh.max_len);
   if (keeps_all<true>(a, N)) {
@@ -1224,12 +1244,11 @@ cudaError_t stream_launch(const SelectArgs &a, const Shape &sh, const Tables &tb
     if (e == cudaSuccess) e = set_smem_once(stream_kernel<GR, kStageTopk>, smem1);
     if (e == cudaSuccess) e = set_smem_once(topk_resolve_kernel, bitmap_bytes);
     if (e != cudaSuccess) return e;
-    window_kernel<GR, false><<<items, kT0, smem0, st>>>(a, sh, tb.ret, tb.n_ret, ws);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    stream_kernel<GR, kStageTopk><<<g1, kT1, smem1, st>>>(a, sh, tb.ret, tb.n_ret, ws);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    topk_resolve_kernel<<<g2, kT2, bitmap_bytes, st>>>(a, sh, ws);
-    return cudaGetLastError();
+    e = launch_pdl(window_kernel<GR, false>, dim3(items), dim3(kT0), smem0, st, 0, a, sh, tb.ret, tb.n_ret, ws);
+    if (e == cudaSuccess)
+      e = launch_pdl(stream_kernel<GR, kStageTopk>, g1, dim3(kT1), smem1, st, 0, a, sh, tb.ret, tb.n_ret, ws);
+    if (e == cudaSuccess) e = launch_pdl(topk_resolve_kernel, g2, dim3(kT2), bitmap_bytes, st, 0, a, sh, ws);
+    return e;
   }
   const size_t smem_m = stream_smem_bytes(GR, kMassTopp), smem_c = stream_smem_bytes(GR, kCutTopp);
   e = set_smem_once(window_kernel<GR, true>, smem0);
@@ -1237,14 +1256,13 @@ cudaError_t stream_launch(const SelectArgs &a, const Shape &sh, const Tables &tb
   if (e == cudaSuccess) e = set_smem_once(stream_kernel<GR, kCutTopp>, smem_c);
   if (e == cudaSuccess) e = set_smem_once(topp_resolve_kernel, bitmap_bytes);
   if (e != cudaSuccess) return e;
-  window_kernel<GR, true><<<items, kT0, smem0, st>>>(a, sh, tb.ret, tb.n_ret, ws);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  stream_kernel<GR, kMassTopp><<<g1, kT1, smem_m, st>>>(a, sh, tb.ret, tb.n_ret, ws);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  stream_kernel<GR, kCutTopp><<<g1, kT1, smem_c, st>>>(a, sh, tb.ret, tb.n_ret, ws);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  topp_resolve_kernel<<<g2, kT2, bitmap_bytes, st>>>(a, sh, ws);
-  return cudaGetLastError();
+  e = launch_pdl(window_kernel<GR, true>, dim3(items), dim3(kT0), smem0, st, 0, a, sh, tb.ret, tb.n_ret, ws);
+  if (e == cudaSuccess)
+    e = launch_pdl(stream_kernel<GR, kMassTopp>, g1, dim3(kT1), smem_m, st, 0, a, sh, tb.ret, tb.n_ret, ws);
+  if (e == cudaSuccess)
+    e = launch_pdl(stream_kernel<GR, kCutTopp>, g1, dim3(kT1), smem_c, st, 0, a, sh, tb.ret, tb.n_ret, ws);
+  if (e == cudaSuccess) e = launch_pdl(topp_resolve_kernel, g2, dim3(kT2), bitmap_bytes, st, 0, a, sh, ws);
+  return e;
 }
 
 }  // namespace

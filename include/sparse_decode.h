@@ -273,15 +273,17 @@ SD_API sd_status sparse_decode_attend(sd_ctx *ctx, const void *q, const void *k_
  *     when this batch needs more than the built-in scratch (the amount
  *     sparse_decode_workspace_size reports for attend grows with the batch,
  *     the retrieval groups and max_pages_per_seq); nothing is launched then.
- *   - Nothing in the scratch has to start at zero: the call clears the
- *     counters it uses, on `stream`, before its kernels run.
+ *   - Nothing in the scratch has to start at zero: the call's own kernels
+ *     clear the counters they use, in stream order, before reading them.
  *   - The scratch is one area per device, shared by every context and stream
  *     of the process: two of these calls on the same device that are not
  *     ordered on one stream (other streams, threads or contexts) race and may
  *     give wrong outputs.  Order them, or use sparse_decode_attend with
  *     separate workspaces.
- *   - The first call on a device does a one-time set-up (it looks up the
- *     scratch address with cudaGetSymbolAddress); make that first call
+ *   - Every call looks up the scratch address of the current device with
+ *     cudaGetSymbolAddress (a cheap lookup; nothing is cached, so a device
+ *     reset between calls leaves no stale address).  The first call on a
+ *     device may load the library's device code there: make that first call
  *     outside any stream capture.
  */
 SD_API sd_status sparse_decode_attend_noalloc(sd_ctx *ctx, const void *q, const void *k_cache,

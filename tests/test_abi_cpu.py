@@ -26,7 +26,7 @@ def test_header_declares_the_boundary_calls():
     names = _declared()
     for n in ["sparse_decode_init", "sparse_decode_index_keys", "sparse_decode_select",
               "sparse_decode_attend", "sparse_decode_workspace_size", "sparse_decode_destroy",
-              "sparse_decode_error_word"]:
+              "sparse_decode_error_word", "sparse_decode_attend_noalloc"]:
         assert n in names
 
 
@@ -87,6 +87,11 @@ def test_null_arguments():
     n = ctypes.c_size_t()
     assert sd.LIB.sparse_decode_workspace_size(None, 1, ctypes.byref(n)) == sd.SD_ERR_INVALID_ARG
     assert sd.LIB.sparse_decode_select(None, None, None, None, None, 1, None, None, 1, None, 0, None) == sd.SD_ERR_INVALID_ARG
+    assert sd.LIB.sparse_decode_attend_noalloc(None, None, None, None, None, None, 1, None, None, 1, None,
+                                               None) == sd.SD_ERR_INVALID_ARG
+    assert sd.LIB.sparse_decode_attend(None, None, None, None, None, None, 1, None, None, 1, None, None, 0,
+                                       None) == sd.SD_ERR_INVALID_ARG
+    assert sd.LIB.sparse_decode_index_keys(None, None, None, 1, None, None) == sd.SD_ERR_INVALID_ARG
     assert sd.LIB.sparse_decode_num_retrieval_heads(None) == 0
     assert sd.LIB.sparse_decode_last_error(None) == b""
     sd.LIB.sparse_decode_destroy(None)

@@ -380,23 +380,38 @@ def test_topp_threshold_below_window_falls_back_to_exact():
 
 # ------------------------------------------------------------------ full sizes
 
+def _spread(lens, n_seq=8):
+    """n_seq sequences spread over the length range: the shortest, the
+    longest and the ones between them at evenly spaced length ranks."""
+    order = sorted(range(len(lens)), key=lambda b: lens[b])
+    return sorted({order[round(i * (len(lens) - 1) / (n_seq - 1))] for i in range(n_seq)})
+
+
+# Full-size workloads in the bench's launch configuration.  Every retrieval
+# head of the listed sequences is compared (sets and outputs), plus the first
+# and last local head; the long-context Zipf workload is run at every point of
+# its top-p x alpha sweep.
 FULL = [
-    ("llama3_8b_topp", dict(), [0, 3]),
+    ("llama3_8b_topp", dict(), [0, 1, 2, 3]),
     ("topk_128k", dict(), [0, 9, 15]),
-    ("long_zipf", dict(top_p=0.9, alpha=1.2), [0]),
-    ("long_zipf", dict(top_p=0.99, alpha=0.8), [0]),
-    ("ragged_paged", dict(), [0, 17, 63]),
+] + [("long_zipf", dict(top_p=p, alpha=a), [0]) for p in (0.5, 0.9, 0.99) for a in (0.8, 1.2)] + [
+    ("ragged_paged", dict(), "spread"),
 ]
 
 
 @pytest.mark.parametrize("name,kw,seqs", FULL, ids=[f"{n}-{i}" for i, (n, _, _) in enumerate(FULL)])
-def test_full_size_sampled(name, kw, seqs):
+def test_full_size_all_retrieval_heads(name, kw, seqs):
     w = make_workload(name, "cuda", **kw)
-    G = w.num_q_heads // w.num_kv_heads
-    # every retrieval head of two groups plus two local heads per sampled sequence
+    if seqs == "spread":
+        lens = w.seq_lens.cpu().tolist()
+        seqs = _spread(lens)
+        picked = [lens[b] for b in seqs]
+        assert len(seqs) == 8 and min(picked) == min(lens) and max(picked) == max(lens)
     retr = [h for h in range(w.num_q_heads) if w.head_is_retrieval[h]]
     loc = [h for h in range(w.num_q_heads) if not w.head_is_retrieval[h]]
-    heads = sorted(set(retr[:G] + retr[-G:] + loc[:1] + loc[-1:]))
-    check_workload(w, seqs=seqs, heads=heads, label=name)
+    heads = sorted(set(retr + loc[:1] + loc[-1:]))
+    band = check_workload(w, seqs=seqs, heads=heads, label=f"{name}{kw}")
+    print(f"{name} {kw} seqs {seqs}: {len(retr) * len(seqs)} retrieval sets compared, "
+          f"{band} tokens inside the threshold band")
     del w
     torch.cuda.empty_cache()

@@ -1,13 +1,15 @@
 """sparse_decode_attend_noalloc (attend on the library's built-in scratch)
-against sparse_decode_attend with a caller workspace, through the C ABI.
-Collected last on purpose: it must also pass after everything else ran in
-the same process."""
+against sparse_decode_attend with a caller workspace and against the float64
+oracle, through the C ABI.  Collected last on purpose: it must also pass
+after everything else ran in the same process."""
 
 import numpy as np
 import pytest
 import torch
 
-from tests.helpers import assert_out_close, make_step
+import oracle as O
+from oracle.workload_inputs import oracle_config, oracle_inputs
+from tests.helpers import assert_out_close, gpu_sets, make_step
 from workloads import make_workload
 
 pytestmark = pytest.mark.gpu
@@ -32,6 +34,29 @@ def test_noalloc_attend_matches_attend_twice_in_a_row():
         for b in range(w.batch):
             for h in range(w.num_q_heads):
                 assert_out_close(got[b, h], want[b, h], f"call {call} b={b} h={h}")
+    # and against the oracle: exact attention over the same selected sets
+    # (retrieval heads) and over sinks + window (local heads)
+    retr = [(b, h) for b in range(w.batch) for h in range(w.num_q_heads) if w.head_is_retrieval[h]]
+    ref = O.decode_reference(oracle_config(w), **oracle_inputs(w), sets_override=gpu_sets(st, w, retr))
+    for (b, h), o in ref.out.items():
+        assert_out_close(got[b, h], o, f"oracle b={b} h={h}")
+    st.close()
+
+
+def test_noalloc_attend_rejects_bad_arguments_before_launching():
+    from head_wise_sparse_02_b200 import sparse_decode as sd
+    w = make_workload("tiny_ref", "cuda")
+    st = make_step(w)
+    out = torch.empty((1, 4, 64), dtype=torch.float32, device="cuda")
+    lib, h = sd.LIB, st.sd.handle
+    args = [w.q.data_ptr(), st.k_cache.data_ptr(), st.v_cache.data_ptr(), st.page_table.data_ptr(),
+            st.seq_lens.data_ptr()]
+    sel = [st.sel_idx.data_ptr(), st.sel_count.data_ptr(), st.sel_idx.shape[-1], out.data_ptr(), None]
+    assert lib.sparse_decode_attend_noalloc(h, *args, 2, *sel) == sd.SD_ERR_INVALID_ARG      # batch > max_batch
+    assert lib.sparse_decode_attend_noalloc(h, *args, -1, *sel) == sd.SD_ERR_INVALID_ARG
+    assert lib.sparse_decode_attend_noalloc(h, None, *args[1:], 1, *sel) == sd.SD_ERR_INVALID_ARG
+    assert lib.sparse_decode_attend_noalloc(h, *args, 1, None, *sel[1:]) == sd.SD_ERR_INVALID_ARG
+    assert lib.sparse_decode_attend_noalloc(h, *args, 0, *sel) == sd.SD_OK                    # empty batch
     st.close()
 
 
