@@ -347,6 +347,8 @@ def size_overrides(args):
         kw["top_p"] = args.top_p
     if args.alpha:
         kw["alpha"] = args.alpha
+    if args.top_k_frac:
+        kw["top_k_frac"] = args.top_k_frac
     return kw
 
 
@@ -679,6 +681,7 @@ def main(argv=None):
     ap.add_argument("--seq-len", type=int, default=0, help="override the workload's context length")
     ap.add_argument("--top-p", type=float, default=0.0, help="override the workload's top-p")
     ap.add_argument("--alpha", type=float, default=0.0, help="long_zipf: Zipf exponent of the score profile")
+    ap.add_argument("--top-k-frac", type=float, default=0.0, help="override the workload's top-k fraction")
     ap.add_argument("--l2-flush", choices=["auto", "on", "off"], default="auto",
                     help="flush L2 between timed steps (auto: when a step touches < 8x the L2)")
     ap.add_argument("--no-diagnostics", action="store_true")

@@ -47,6 +47,10 @@ sd_status cuda_fail(sd_ctx *ctx, cudaError_t e, const char *what) {
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
+// Caches, keys and queries are read with 16-byte vector and asynchronous
+// copies: their base addresses must be 16-byte aligned.
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0u; }
+
 struct WsLayout {
   size_t scores_off, flags_off, scores_bytes, stream_off, stream_bytes, att_off, total;
 };
@@ -201,6 +205,8 @@ sd_status sparse_decode_index_keys(sd_ctx *ctx, const void *k_pre, const int32_t
     if (num_tokens < 0) return fail(ctx, SD_ERR_INVALID_ARG, "num_tokens < 0");
     if (num_tokens == 0) return SD_OK;
     if (!k_pre || !slots || !index_cache) return fail(ctx, SD_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(k_pre) || !aligned16(index_cache))
+      return fail(ctx, SD_ERR_INVALID_ARG, "k_pre and index_cache must be 16-byte aligned");
     DeviceGuard dg(ctx->device);
     cudaError_t e = sd::launch_index_keys(static_cast<const uint16_t *>(k_pre), slots, num_tokens,
                                           static_cast<uint16_t *>(index_cache), ctx->proj_d, ctx->sh,
@@ -221,6 +227,8 @@ sd_status sparse_decode_select(sd_ctx *ctx, const void *q_pre, const void *index
     if (batch == 0 || ctx->sh.H_ret == 0) return SD_OK;
     if (!q_pre || !index_cache || !page_table || !seq_lens || !sel_idx || !sel_count)
       return fail(ctx, SD_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(q_pre) || !aligned16(index_cache))
+      return fail(ctx, SD_ERR_INVALID_ARG, "q_pre and index_cache must be 16-byte aligned");
     const long long need_stride = ctx->cfg.mode == SD_TOP_P ? ctx->sh.max_len : max_topk(ctx);
     if (sel_stride < need_stride)
       return fail(ctx, SD_ERR_INVALID_ARG, "sel_stride smaller than the largest possible set");
@@ -263,6 +271,8 @@ sd_status sparse_decode_attend(sd_ctx *ctx, const void *q, const void *k_cache, 
     if (batch == 0) return SD_OK;
     if (!q || !k_cache || !v_cache || !page_table || !seq_lens || !out)
       return fail(ctx, SD_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+      return fail(ctx, SD_ERR_INVALID_ARG, "q, k_cache and v_cache must be 16-byte aligned");
     if (ctx->sh.H_ret > 0 && (!sel_idx || !sel_count || sel_stride <= 0))
       return fail(ctx, SD_ERR_INVALID_ARG, "selection lists required for retrieval heads");
     const WsLayout w = layout(ctx, batch);
@@ -301,6 +311,8 @@ sd_status sparse_decode_attend_noalloc(sd_ctx *ctx, const void *q, const void *k
     if (batch == 0) return SD_OK;
     if (!q || !k_cache || !v_cache || !page_table || !seq_lens || !out)
       return fail(ctx, SD_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+      return fail(ctx, SD_ERR_INVALID_ARG, "q, k_cache and v_cache must be 16-byte aligned");
     if (ctx->sh.H_ret > 0 && (!sel_idx || !sel_count || sel_stride <= 0))
       return fail(ctx, SD_ERR_INVALID_ARG, "selection lists required for retrieval heads");
     const size_t need = sd::attend_workspace_bytes(ctx->sh, ctx->tb, batch);

@@ -67,18 +67,11 @@ constexpr int kTileRing = 3;            // tiles in flight per warp
 constexpr int kMaxGrid = 4096;          // persistent CTAs (partial slots are sized for this)
 
 // 16-byte copy global -> shared, bypassing L1, with an L2 eviction-priority
-// hint: streamed cache rows are read once per call, so they are marked
-// evict-first and leave the small tables, lists and code of the surrounding
-// kernels in L2
+// hint (see evict_first_policy)
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, int src_bytes, uint64_t policy) {
   asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;\n" ::"r"(dst), "l"(src),
                "r"(src_bytes), "l"(policy)
                : "memory");
-}
-__device__ __forceinline__ uint64_t evict_first_policy() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(p));
-  return p;
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 template <int N>
@@ -336,46 +329,66 @@ __device__ void plan_span(const AttendArgs &a, const Shape &sh, const Tables &tb
     atomicOr(&hbm[i * bwords + (off >> 5)], 1u << (off & 31));
   }
   __syncthreads();
-  // ordered compaction of the union: contiguous word ranges per thread
-  const int wpt = (bwords + kPlanThreads - 1) / kPlanThreads;
-  const int w0 = tid * wpt, w1 = std::min(bwords, w0 + wpt);
+  // ordered compaction of the union: warp w owns a contiguous run of bitmap
+  // words, read lane-strided (32 consecutive words per step, no bank
+  // conflicts); a warp scan of the words' union bit counts places each lane's
+  // rows, a block-wide sum over the warp totals places the warp
+  const int steps = (bwords + kPlanThreads - 1) / kPlanThreads;   // 32-word steps per warp
+  const int x0 = warp * steps * 32;
   uint32_t c = 0;
-  for (int x = w0; x < w1; ++x) {
+  for (int r = 0; r < steps; ++r) {
+    const int x = x0 + r * 32 + lane;
     uint32_t u = 0;
-    for (int i = 0; i < nh; ++i) u |= hbm[i * bwords + x];
+    if (x < bwords)
+#pragma unroll
+      for (int i = 0; i < GR; ++i) u |= i < nh ? hbm[i * bwords + x] : 0u;
     c += __popc(u);
   }
-  uint32_t incl = c;
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t y = __shfl_up_sync(kFull, incl, o);
-    if (lane >= o) incl += y;
-  }
-  if (lane == 31) wtot[warp] = incl;
+  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(kFull, c, o);
+  if (lane == 0) wtot[warp] = c;
   __syncthreads();
-  uint32_t base = 0, total = 0;
+  uint32_t o = 0, total = 0;
+#pragma unroll
   for (int x = 0; x < kPlanWarps; ++x) {
-    if (x < warp) base += wtot[x];
+    o += x < warp ? wtot[x] : 0u;
     total += wtot[x];
   }
-  uint32_t o = base + incl - c;
   uint32_t *rows = ws.plan_row + slot * ap.span;
   uint16_t *masks = ws.plan_mask + slot * ap.span;
-  for (int x = w0; x < w1; ++x) {
+  const uint32_t row_g = (uint32_t)g * kPage;          // row of (page, g, slot) = (page * Hkv + g) * 16 + slot
+  const uint32_t row_page = (uint32_t)sh.Hkv * kPage;
+  for (int r = 0; r < steps; ++r) {
+    const int x = x0 + r * 32 + lane;
+    uint32_t hw[GR];
     uint32_t u = 0;
-    for (int i = 0; i < nh; ++i) u |= hbm[i * bwords + x];
+#pragma unroll
+    for (int i = 0; i < GR; ++i) {
+      hw[i] = (x < bwords && i < nh) ? hbm[i * bwords + x] : 0u;
+      u |= hw[i];
+    }
+    const uint32_t n = __popc(u);
+    uint32_t incl = n;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const uint32_t y = __shfl_up_sync(kFull, incl, d);
+      if (lane >= d) incl += y;
+    }
+    uint32_t at = o + incl - n;
     while (u) {
       const int bit = __ffs(u) - 1;
       u &= u - 1;
       uint32_t m = 0;
-      for (int i = 0; i < nh; ++i) m |= ((hbm[i * bwords + x] >> bit) & 1u) << i;
+#pragma unroll
+      for (int i = 0; i < GR; ++i) m |= ((hw[i] >> bit) & 1u) << i;
       const int off = x * 32 + bit;
-      const int page = pslice[off / kPage];
+      const int page = pslice[off >> 4];
       if (page < 0) raise_error(a.err, SD_EBIT_PAGE);
-      rows[o] = page >= 0 ? (uint32_t)(((long long)page * sh.Hkv + g) * kPage + (off % kPage)) : 0u;
-      masks[o] = (uint16_t)(page >= 0 ? m : 0u);
-      ++o;
+      rows[at] = page >= 0 ? (uint32_t)page * row_page + row_g + (uint32_t)(off & (kPage - 1)) : 0u;
+      masks[at] = (uint16_t)(page >= 0 ? m : 0u);
+      ++at;
     }
+    o += __shfl_sync(kFull, incl, 31);
   }
   if (tid == 0) ws.plan_cnt[slot] = (int)total;
 }

@@ -23,22 +23,44 @@ __global__ void __launch_bounds__(kThreads)
 index_keys_kernel(const uint16_t *__restrict__ k_pre, const int32_t *__restrict__ slots, int T,
                   uint16_t *__restrict__ index_cache, const uint16_t *__restrict__ proj, int Hkv,
                   int num_pages, unsigned *err) {
+  static_assert(D % 8 == 0, "whole 16-byte loads");
   __shared__ double Ps[D][kIndexDim];
   __shared__ double Ks[kRows][D + 1];
   const int g = blockIdx.y;
   const int t0 = blockIdx.x * kRows;
-  const uint16_t *P = proj + (size_t)g * D * kIndexDim;
-  for (int i = threadIdx.x; i < D * kIndexDim; i += kThreads)
-    Ps[i / kIndexDim][i % kIndexDim] = (double)bf16_to_f32(P[i]);    // the context's own copy
+  const int tid = threadIdx.x;
+  // the projection is the context's own copy: loaded before waiting for the
+  // previous kernel on the stream
+  const uint4 *P = reinterpret_cast<const uint4 *>(proj + (size_t)g * D * kIndexDim);
+#pragma unroll
+  for (int i = tid; i < D * kIndexDim / 8; i += kThreads) {
+    const uint4 v = __ldg(P + i);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = i * 8 + 2 * j;
+      Ps[e / kIndexDim][e % kIndexDim] = (double)bf16_lo(w[j]);
+      Ps[(e + 1) / kIndexDim][(e + 1) % kIndexDim] = (double)bf16_hi(w[j]);
+    }
+  }
   pdl_wait();
   pdl_trigger();
-  for (int i = threadIdx.x; i < kRows * D; i += kThreads) {
-    const int row = i / D, c = i % D, t = t0 + row;
-    Ks[row][c] = (t < T) ? (double)bf16_to_f32(k_pre[((size_t)t * Hkv + g) * D + c]) : 0.0;
+  const int row = tid / kIndexDim, j = tid % kIndexDim;
+  const int t = t0 + row;
+  const long long slot = t < T ? (long long)slots[t] : -1;     // issued with the key loads
+#pragma unroll
+  for (int i = tid; i < kRows * D / 8; i += kThreads) {
+    const int r = i / (D / 8), c = (i % (D / 8)) * 8, tr = t0 + r;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (tr < T) v = *reinterpret_cast<const uint4 *>(k_pre + ((size_t)tr * Hkv + g) * D + c);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      Ks[r][c + 2 * q] = (double)bf16_lo(w[q]);
+      Ks[r][c + 2 * q + 1] = (double)bf16_hi(w[q]);
+    }
   }
   __syncthreads();
-  const int row = threadIdx.x / kIndexDim, j = threadIdx.x % kIndexDim;
-  const int t = t0 + row;
   if (t >= T) return;
   // four interleaved partial sums (shorter dependent chains), added at the end
   double acc4[4] = {0.0, 0.0, 0.0, 0.0};
@@ -47,7 +69,6 @@ index_keys_kernel(const uint16_t *__restrict__ k_pre, const int32_t *__restrict_
 #pragma unroll
     for (int u = 0; u < 4; ++u) acc4[u] = fma(Ks[row][i + u], Ps[i + u][j], acc4[u]);
   const double acc = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
-  const long long slot = slots[t];
   if (slot < 0 || slot >= (long long)num_pages * kPage) {
     if (j == 0) raise_error(err, SD_EBIT_SLOT);
     return;

@@ -84,6 +84,14 @@ __device__ __forceinline__ void raise_error(unsigned *err, unsigned bit) {
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
 
+// L2 eviction priority of streamed data: cache rows and index pages are read
+// once per call, so they are marked evict-first and leave the small tables,
+// lists and code of the surrounding kernels in L2
+__device__ __forceinline__ uint64_t evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(p));
+  return p;
+}
 // cudaLaunchKernelEx with programmatic stream serialization, plus an optional
 // cluster shape (x CTAs per cluster; 0 = no cluster).
 template <typename... KArgs, typename... Args>

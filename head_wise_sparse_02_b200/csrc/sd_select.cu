@@ -751,7 +751,9 @@ cudaError_t launch_select(const SelectArgs &a, const Shape &sh, const Tables &tb
   // after the streaming passes: exact recomputation of the items whose window
   // missed (usually none); without them: every item
   const uint32_t *flags = used ? a.flags : nullptr;
-  const int gy = used ? std::min(items, 16) : items;
+  // with the streaming passes the exact selector usually has nothing to do:
+  // a few clusters stride over the flagged items (one wave of CTAs to launch)
+  const int gy = used ? std::min(items, 4) : items;
   if (topp)
     return p.smem ? dispatch_gr<true, true>(a, sh, tb, p, dev, st, flags, gy)
                   : dispatch_gr<true, false>(a, sh, tb, p, dev, st, flags, gy);

@@ -10,8 +10,11 @@
 // of the context.
 //
 // Every pass streams the index through per-warp cp.async rings (16 bytes per
-// lane, XOR-swizzled rows) and scores all heads of a KV group at once with
-// ldmatrix + mma.m16n8k16 (A = the 16 x 16 bf16 index page, B = the q~ terms).
+// lane, XOR-swizzled rows, L2 evict-first) and scores all heads of a KV group
+// at once with ldmatrix + mma.m16n8k16 (A = the 16 x 16 bf16 index page, B =
+// the q~ terms).  One bulk copy (cp.async.bulk) per 512-byte page, issued by
+// one lane and counted on an mbarrier, was measured 1.6x slower here: more
+// instructions per page and one CTA less per SM.
 //
 // K0 window  one CTA per (sequence, KV group).  Computes q~ = c P_g^T q_pre
 //            (float64, rounded to float32, split exactly into three bf16
@@ -75,9 +78,10 @@ constexpr int kChunkPages = 512;      // K1: pages per CTA
 constexpr int kRing = 8;              // K1: pages in flight per warp (even); 4 CTAs per SM
 // K1: staged buffer entries per (lane, head block); an iteration adds <= 4
 __host__ __device__ constexpr int stage_lane(int GR) { return GR <= 4 ? 10 : (GR == 8 ? 8 : 5); }
+constexpr int kBinsK = 2048;          // top-k K2: bins of the window and of each refinement level
 constexpr int kCap = 2048;            // K2: cut-bin tokens ranked exactly
 constexpr int kLevels = 3;            // K2: histogram levels (the cut bin is split again)
-constexpr int kRefine = 64;           // K2: a cut bin above this many tokens is split again
+constexpr int kRefine = 256;          // K2: a cut bin above this many tokens is split again
 constexpr int kPer2 = 16;             // K2: buffer entries held in registers per thread
 constexpr int kPageBytes = kPage * kIndexDim * 2;   // 512 B: one page of one KV head
 constexpr unsigned kFull = 0xFFFFFFFFu;
@@ -108,18 +112,11 @@ __device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
                : "r"(addr));
 }
 // 16-byte copy global -> shared, bypassing L1, with an L2 eviction-priority
-// hint: streamed cache rows are read once per call, so they are marked
-// evict-first and leave the small tables, lists and code of the surrounding
-// kernels in L2
+// hint (see evict_first_policy)
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, int src_bytes, uint64_t policy) {
   asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;\n" ::"r"(dst), "l"(src),
                "r"(src_bytes), "l"(policy)
                : "memory");
-}
-__device__ __forceinline__ uint64_t evict_first_policy() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(p));
-  return p;
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 template <int N>
@@ -397,12 +394,15 @@ window_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__ grou
   }
   if (keeps_all<TOPP>(a, N)) return;                 // K1 skips, K2 keeps everything
 
-  // q~ in float64 (one warp per head, lanes split d) -> float32 -> hi/mid/lo
-  for (int i = warp; i < 16; i += kT0 / 32) {
+  // q~ in float64 (one warp per head, lanes split d) -> float32 -> hi/mid/lo;
+  // the terms of absent heads stay zero
+  for (int o = tid; o < 16 * 24; o += kT0) qs[o] = 0u;
+  __syncthreads();
+  for (int i = warp; i < nr; i += kT0 / 32) {
     double acc[kIndexDim];
 #pragma unroll
     for (int j = 0; j < kIndexDim; ++j) acc[j] = 0.0;
-    if (i < nr) {
+    {
       const uint16_t *qrow = a.q_pre + ((long long)b * sh.Hq + grp.q_head[i]) * sh.d;
       const uint16_t *P = a.proj + (long long)g * sh.d * kIndexDim;
       for (int e = lane; e < sh.d; e += 32) {
@@ -534,13 +534,15 @@ window_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__ grou
     hinv[tid] = (smax[tid] != 0u && hi > lo) ? (float)kSampleBins / (hi - lo) : 0.0f;
   }
   __syncthreads();
-  for (int o = tid; o < nr * ns * 16; o += kT0) {
-    const int h = o / (ns * 16), r = o % (ns * 16);
-    const float v = sample[h][r];
-    if (v == -INFINITY) continue;
-    const int bin = std::min(kSampleBins - 1, std::max(0, __float2int_rz((v - hlo[h]) * hinv[h])));
-    atomicAdd(&shist[h][bin], 1u);
-    if constexpr (TOPP) atomicAdd(&smass[h][bin], exp2f((v - hhi[h]) * kLog2e));
+  for (int h = 0; h < nr; ++h) {
+    const float lo = hlo[h], iv = hinv[h], hi = hhi[h];
+    for (int r = tid; r < ns * 16; r += kT0) {
+      const float v = sample[h][r];
+      if (v == -INFINITY) continue;
+      const int bin = std::min(kSampleBins - 1, std::max(0, __float2int_rz((v - lo) * iv)));
+      atomicAdd(&shist[h][bin], 1u);
+      if constexpr (TOPP) atomicAdd(&smass[h][bin], exp2f((v - hi) * kLog2e));
+    }
   }
   __syncthreads();
   // one warp per head: the highest bin whose suffix count reaches r
@@ -574,7 +576,7 @@ window_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__ grou
         tlo = lo + (float)blo * ((hi - lo) / (float)kSampleBins);
       }
     }
-    const float inv = (tlo > -INFINITY && thi > tlo) ? (float)kBins / (thi - tlo) : 0.0f;
+    const float inv = (tlo > -INFINITY && thi > tlo) ? (float)kBinsK / (thi - tlo) : 0.0f;
     if (lane == 0) ws.win[row] = make_float4(tlo, thi, inv, 0.0f);
   }
 }
@@ -829,31 +831,44 @@ stream_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__ grou
 constexpr int kT2 = 256;
 
 // Block-wide: the positions set in bitmap[0, words) go to out in ascending
-// order (contiguous word ranges per thread, block-wide prefix), their number
-// to sel_count[row].  wtot: kT2 / 32 words of shared memory.
+// order, their number to sel_count[row].  Warp w owns a contiguous run of
+// words, read lane-strided (32 consecutive words per step, no bank
+// conflicts); a warp-wide scan of the words' bit counts places each lane's
+// positions, a block-wide sum over the warps' totals places the warp.  wtot:
+// kT2 / 32 words of shared memory.
 __device__ void write_ascending(const SelectArgs &a, const uint32_t *bitmap, int words, int32_t *out, long long row,
                                 uint32_t *wtot) {
+  constexpr int NW = kT2 / 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int wpt = (words + kT2 - 1) / kT2;
-  const int w0 = tid * wpt, w1 = std::min(words, w0 + wpt);
+  const int steps = (words + NW * 32 - 1) / (NW * 32);           // 32-word steps per warp
+  const int w0 = warp * steps * 32;
   uint32_t c = 0;
-  for (int x = w0; x < w1; ++x) c += __popc(bitmap[x]);
-  uint32_t incl = c;
+  for (int r = 0; r < steps; ++r) {
+    const int x = w0 + r * 32 + lane;
+    c += x < words ? __popc(bitmap[x]) : 0u;
+  }
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t y = __shfl_up_sync(kFull, incl, o);
-    if (lane >= o) incl += y;
-  }
-  if (lane == 31) wtot[warp] = incl;
+  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(kFull, c, o);
+  if (lane == 0) wtot[warp] = c;
   __syncthreads();
-  uint32_t base = 0, total = 0;
-  for (int x = 0; x < kT2 / 32; ++x) {
-    if (x < warp) base += wtot[x];
-    total += wtot[x];
+  uint32_t off = 0, total = 0;
+#pragma unroll
+  for (int x = 0; x < NW; ++x) {
+    const uint32_t t = wtot[x];
+    off += x < warp ? t : 0u;
+    total += t;
   }
-  long long o = base + incl - c;
-  for (int x = w0; x < w1; ++x) {
-    uint32_t bits = bitmap[x];
+  for (int r = 0; r < steps; ++r) {
+    const int x = w0 + r * 32 + lane;
+    uint32_t bits = x < words ? bitmap[x] : 0u;
+    const uint32_t n = __popc(bits);
+    uint32_t incl = n;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(kFull, incl, o);
+      if (lane >= o) incl += y;
+    }
+    long long o = (long long)off + (incl - n);
     while (bits) {
       const int bit = __ffs(bits) - 1;
       bits &= bits - 1;
@@ -861,6 +876,7 @@ __device__ void write_ascending(const SelectArgs &a, const uint32_t *bitmap, int
       else raise_error(a.err, SD_EBIT_SEL);
       ++o;
     }
+    off += __shfl_sync(kFull, incl, 31);
   }
   if (tid == 0) {
     if ((long long)total > a.sel_stride) raise_error(a.err, SD_EBIT_SEL);
@@ -883,101 +899,146 @@ __device__ void flag_item(const StreamWs &ws, long long row) {
   if (atomicExch(&ws.fail[it], 1u) == 0u) ws.fail[ws.items + 1 + atomicAdd(&ws.fail[ws.items], 1u)] = (uint32_t)it;
 }
 
+// Block-wide: the highest bin c of hist[0, kBinsK) whose suffix count reaches
+// need (need >= 1).  Thread t holds bins [8 t, 8 t + 8); a block-wide suffix
+// sum over the threads' totals finds the thread holding the cut, which scans
+// its own bins.  Writes c, the count strictly above it and hist[c] to res
+// (res[0] = -1 when the bins together hold fewer than need).  wsum: kT2 / 32
+// words of shared memory.
+__device__ void block_cut_bin(const uint32_t *hist, long long need, uint32_t *wsum, int *res) {
+  constexpr int PT = kBinsK / kT2;
+  static_assert(PT == 8, "two 16-byte loads per thread");
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint4 h0 = reinterpret_cast<const uint4 *>(hist)[2 * tid];
+  const uint4 h1 = reinterpret_cast<const uint4 *>(hist)[2 * tid + 1];
+  const uint32_t v[PT] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+  uint32_t tot = 0;
+#pragma unroll
+  for (int j = 0; j < PT; ++j) tot += v[j];
+  uint32_t suf = tot;                                  // sum over this and the higher lanes of the warp
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_down_sync(kFull, suf, o);
+    if (lane + o < 32) suf += y;
+  }
+  if (lane == 0) wsum[warp] = suf;
+  __syncthreads();
+  long long above = 0;
+#pragma unroll
+  for (int w = 0; w < kT2 / 32; ++w) above += w > warp ? wsum[w] : 0u;
+  long long run = above + (suf - tot);                 // count above this thread's bins
+  if (run < need && run + tot >= need) {
+#pragma unroll
+    for (int j = PT - 1; j >= 0; --j) {
+      if (run + v[j] >= need) {
+        res[0] = tid * PT + j;
+        res[1] = (int)run;
+        res[2] = (int)v[j];
+        break;
+      }
+      run += v[j];
+    }
+  }
+}
+
+// top-k K2: one CTA per (sequence, retrieval head).  The head's buffered
+// entries (every score >= t_lo) are histogrammed over kBinsK bins of
+// [t_lo, t_hi) plus one bin for scores >= t_hi; the bin holding the k-th
+// score is split again while it holds more than kRefine tokens (kLevels
+// levels at most); entries above the cut path are selected, the cut bin's are
+// ranked exactly by (score desc, position asc).
 __global__ void __launch_bounds__(kT2, 4)
 topk_resolve_kernel(const SelectArgs a, const Shape sh, const StreamWs ws) {
-  extern __shared__ uint32_t bitmap[];               // [max_len / 32]
+  extern __shared__ __align__(16) uint32_t bitmap[];  // [max_len / 32], rounded up to 16 bytes
   __shared__ unsigned long long cand[kCap];
-  __shared__ uint32_t hist[kBins + 1];
+  __shared__ __align__(16) uint32_t hist[kBinsK + 1];
   __shared__ uint32_t n_cand;
+  __shared__ int res[3];
   __shared__ int fail_s, done_s;
   __shared__ long long need_s;
   __shared__ int cutv[kLevels];
   __shared__ float llo[kLevels], linv[kLevels];
   __shared__ uint32_t wtot[kT2 / 32];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x, lane = tid & 31;
   const int b = blockIdx.y, hr = blockIdx.x;
   const long long row = (long long)b * sh.H_ret + hr;
   int32_t *out = a.sel_idx + row * a.sel_stride;
   pdl_wait();
   pdl_trigger();
+  // one round of independent loads: the length, the window, the buffer count
+  // and the first kPer2 * kT2 buffer slots (inside the row: reads stop at cap)
   long long N = a.seq_lens[b];
+  const float4 w = ws.win[row];
+  const uint32_t nbuf = ws.bcount[row];
+  const unsigned long long *buf = ws.buf + row * ws.cap;
+  unsigned long long ent[kPer2];
+#pragma unroll
+  for (int j = 0; j < kPer2; ++j) {
+    const int e = tid + j * kT2;
+    ent[j] = e < ws.cap ? __ldcg(buf + e) : 0ull;
+  }
   N = N < 0 ? 0 : std::min<long long>(N, sh.max_len);
   const long long kb = topk_budget(a, N);
   if (N == 0 || kb >= N) {
     write_all(a, N, out, row);
     return;
   }
-  const float4 w = ws.win[row];
-  const uint32_t nbuf = ws.bcount[row];
-  const unsigned long long *buf = ws.buf + row * ws.cap;
   const int n = (int)std::min<uint32_t>(nbuf, (uint32_t)ws.cap);
   const int words = (int)((N + 31) / 32);
-  for (int o = tid; o < words; o += kT2) bitmap[o] = 0u;
+  for (int o = tid; o < (words + 3) / 4; o += kT2) reinterpret_cast<uint4 *>(bitmap)[o] = make_uint4(0u, 0u, 0u, 0u);
   if (tid == 0) {
     llo[0] = w.x;
     linv[0] = w.z;
     need_s = kb;
-    fail_s = 0;
+    fail_s = nbuf > (uint32_t)ws.cap;
     done_s = 0;
     n_cand = 0u;
   }
-  // bin of a score at level L: level 0 is the window histogram (bin kBins:
-  // scores >= t_hi); level L > 0 splits the cut bin of level L - 1 into kBins
+  // bin of a score at level L: level 0 is the window histogram (bin kBinsK:
+  // scores >= t_hi); level L > 0 splits the cut bin of level L - 1 into kBinsK
   // linear sub-bins.  Bins are non-decreasing in the score at every level.
   auto bin_at = [&](float v, int L) -> int {
-    if (L == 0) return window_bin(v, w.x, w.y, w.z);
-    return min(kBins - 1, max(0, __float2int_rz((v - llo[L]) * linv[L])));
+    if (L == 0) return window_bin<kBinsK>(v, w.x, w.y, w.z);
+    return min(kBinsK - 1, max(0, __float2int_rz((v - llo[L]) * linv[L])));
   };
-  // this thread's first kPer2 entries, loaded once (the passes below reread
-  // only entries past kPer2 * kT2 from memory)
-  unsigned long long ent[kPer2];
-#pragma unroll
-  for (int j = 0; j < kPer2; ++j) {
-    const int e = tid + j * kT2;
-    ent[j] = e < n ? buf[e] : 0ull;
-  }
+  // the entries past the registers are read from the buffer (L2) at each pass
+  const int rest0 = kPer2 * kT2;
   // the cut bin: refine while it holds more than kRefine tokens
   int L = 0;
   for (; L < kLevels; ++L) {
-    for (int o = tid; o <= kBins; o += kT2) hist[o] = 0u;
+    for (int o = tid; o <= kBinsK; o += kT2) hist[o] = 0u;
     __syncthreads();
-#pragma unroll
-    for (int j = 0; j < kPer2; ++j) {
-      const int e = tid + j * kT2;
-      if (e < n) {
-        const float v = key_to_float((uint32_t)(ent[j] >> 32));
-        bool play = true;
-        for (int l = 0; l < L; ++l) play = play && bin_at(v, l) == cutv[l];
-        if (play) atomicAdd(&hist[bin_at(v, L)], 1u);
-      }
-    }
-    for (int e = tid + kPer2 * kT2; e < n; e += kT2) {
-      const float v = key_to_float((uint32_t)(buf[e] >> 32));
+    if (fail_s) break;
+    auto add = [&](unsigned long long en) {
+      const float v = key_to_float((uint32_t)(en >> 32));
       bool play = true;
       for (int l = 0; l < L; ++l) play = play && bin_at(v, l) == cutv[l];
       if (play) atomicAdd(&hist[bin_at(v, L)], 1u);
-    }
+    };
+#pragma unroll
+    for (int j = 0; j < kPer2; ++j)
+      if (tid + j * kT2 < n) add(ent[j]);
+    for (int e = rest0 + tid; e < n; e += kT2) add(__ldcg(buf + e));
+    if (tid == 0) res[0] = -1;
     __syncthreads();
-    // warp 0 finds the bin holding the cut among the level's bins
-    if (warp == 0) {
-      const long long need = need_s - (L == 0 ? (long long)hist[kBins] : 0LL);
-      uint32_t above = 0, ncut = 0;
-      const int cut = need > 0 ? warp_cut_bin(hist, kBins, (uint32_t)need, lane, &above, &ncut) : -1;
-      const long long acc = above;
-      if (lane == 0) {
-        if (need <= 0 || cut < 0 || nbuf > (uint32_t)ws.cap) {
-          fail_s = 1;
-        } else {
-          cutv[L] = cut;
-          need_s = need - acc;                       // tokens still to take from the cut bin
-          const bool last = ncut <= kRefine || L + 1 == kLevels;
-          if (last && ncut > kCap) fail_s = 1;
-          if (!last) {
-            llo[L + 1] = llo[L] + (float)cut / linv[L];
-            linv[L + 1] = linv[L] * (float)kBins;
-          }
-          done_s = last;
+    const long long need = need_s - (L == 0 ? (long long)hist[kBinsK] : 0LL);
+    if (need > 0) block_cut_bin(hist, need, wtot, res);
+    __syncthreads();
+    if (tid == 0) {
+      const int cut = res[0];
+      if (need <= 0 || cut < 0) {
+        fail_s = 1;
+      } else {
+        const uint32_t ncut = (uint32_t)res[2];
+        cutv[L] = cut;
+        need_s = need - res[1];                        // tokens still to take from the cut bin
+        const bool last = ncut <= (uint32_t)kRefine || L + 1 == kLevels;
+        if (last && ncut > (uint32_t)kCap) fail_s = 1;
+        if (!last) {
+          llo[L + 1] = llo[L] + (float)cut / linv[L];
+          linv[L + 1] = linv[L] * (float)kBinsK;
         }
+        done_s = last;
       }
     }
     __syncthreads();
@@ -988,8 +1049,10 @@ topk_resolve_kernel(const SelectArgs a, const Shape sh, const StreamWs ws) {
     return;
   }
   const int nlev = L + 1;
-  // classify: above the cut path -> selected; on it -> candidate
-  auto classify = [&](unsigned long long en) {
+  // classify: above the cut path -> selected; on it -> candidate.  Every lane
+  // of a warp takes part (invalid entries included) so that candidates are
+  // appended with one atomic per warp.
+  auto classify = [&](unsigned long long en, bool valid) {
     const uint32_t key = (uint32_t)(en >> 32), pos = (uint32_t)en;
     const float v = key_to_float(key);
     int rel = 0;
@@ -997,17 +1060,24 @@ topk_resolve_kernel(const SelectArgs a, const Shape sh, const StreamWs ws) {
       const int bl = bin_at(v, l);
       rel = bl > cutv[l] ? 1 : (bl < cutv[l] ? -1 : 0);
     }
-    if (rel > 0) {
-      atomicOr(&bitmap[pos >> 5], 1u << (pos & 31));
-    } else if (rel == 0) {
-      const uint32_t at = atomicAdd(&n_cand, 1u);
-      if (at < (uint32_t)kCap) cand[at] = ((unsigned long long)(~key) << 32) | pos;   // ascending = better first
+    if (valid && rel > 0) atomicOr(&bitmap[pos >> 5], 1u << (pos & 31));
+    const bool isc = valid && rel == 0;
+    const unsigned m = __ballot_sync(kFull, isc);
+    if (m) {
+      const int leader = __ffs(m) - 1;
+      uint32_t base = 0;
+      if (lane == leader) base = atomicAdd(&n_cand, (uint32_t)__popc(m));
+      base = __shfl_sync(kFull, base, leader);
+      const uint32_t at = base + __popc(m & ((1u << lane) - 1u));
+      if (isc && at < (uint32_t)kCap) cand[at] = ((unsigned long long)(~key) << 32) | pos;   // ascending = better first
     }
   };
 #pragma unroll
-  for (int j = 0; j < kPer2; ++j)
-    if (tid + j * kT2 < n) classify(ent[j]);
-  for (int e = tid + kPer2 * kT2; e < n; e += kT2) classify(buf[e]);
+  for (int j = 0; j < kPer2; ++j) classify(ent[j], tid + j * kT2 < n);
+  for (int e0 = rest0; e0 < n; e0 += kT2) {
+    const int e = e0 + tid;
+    classify(e < n ? __ldcg(buf + e) : 0ull, e < n);
+  }
   __syncthreads();
   // rank the cut bin exactly: the need_c best by (score desc, position asc)
   const int nc = (int)std::min<uint32_t>(n_cand, (uint32_t)kCap);
@@ -1182,7 +1252,7 @@ StreamPlan stream_plan(const Shape &sh, const Tables &tb, int mode) {
   StreamPlan p{};
   p.cap = mode == SD_TOP_P ? kCapP
                            : (int)std::min<long long>(sh.max_len, std::max<long long>(4096, sh.max_len / 8));
-  p.bitmap_bytes = (size_t)((sh.max_len + 31) / 32) * 4;
+  p.bitmap_bytes = (size_t)((sh.max_len + 127) / 128) * 16;      // whole 16-byte words
   p.bwords = mode == SD_TOP_P ? ((long long)sh.max_pages + 1) / 2 : 0;
   p.ok = tb.max_ret <= 16 && p.bitmap_bytes <= 160 * 1024 && sh.max_len < (1LL << 31);
   return p;

@@ -35,7 +35,10 @@
  *     current when sparse_decode_init ran.  The caller owns all of them; the
  *     library never frees caller memory.
  *   - bf16 tensors are raw IEEE bfloat16 bit patterns (uint16), row-major and
- *     densely packed in the order of their stated shapes.
+ *     densely packed in the order of their stated shapes.  The caches, k_pre,
+ *     q and q_pre must start on a 16-byte boundary (they are read with 16-byte
+ *     vector and asynchronous copies); a misaligned one is rejected with
+ *     SD_ERR_INVALID_ARG.
  *   - Hot calls (index_keys, select, attend) allocate nothing, never
  *     synchronise the host, and enqueue their work on `stream` (a
  *     cudaStream_t; NULL = the legacy default stream).  Argument errors are
