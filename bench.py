@@ -186,12 +186,15 @@ def ncu_traffic(kernel: str, algorithmic_bytes: float):
         return None
 
 
-def kernels_per_step(w) -> int:
+def kernels_per_step(w, score: str = "index") -> int:
     """Kernels of this library one step launches: index_keys; select (top-k:
     window, stream, resolve; top-p: window, mass pass, cut pass, resolve;
-    then the exact selector for flagged items); attend (plan when there are
-    retrieval heads, item layout, main)."""
+    then the exact selector for flagged items; exact-score mode: the score
+    kernel and the exact selector, no index_keys); attend (plan when there
+    are retrieval heads, item layout, main)."""
     ret = any(w.head_is_retrieval)
+    if score == "exact":
+        return (2 if ret else 0) + (3 if ret else 2)
     n_sel = 0 if not ret else (4 if w.mode == "top_k" else 5)
     return 1 + n_sel + (3 if ret else 2)
 
@@ -284,7 +287,7 @@ def workload_label(name: str, w) -> str:
 def bench_config(args, w, ws: int, flush: bool):
     """The `config` object of the JSON line; both arms print the same one."""
     return {
-        "workload": workload_label(args.workload, w),
+        "workload": workload_label(args.workload, w) + (", exact-score selection" if args.score == "exact" else ""),
         "batch_per_gpu": w.batch, "seq_len": int(w.seq_lens.max()),
         "parallelism": f"replicas x{ws} (sequences sharded, no collective)",
         "l2": ("flushed between steps (512 MiB write, untimed)" if flush
@@ -394,16 +397,23 @@ def run_ours(args):
     stream = torch.cuda.current_stream()
 
     calls = ("index_keys", "select", "attend")
+    exact = args.score == "exact"
 
     def step(ev=None):
-        """One decode step; with `ev`, an event pair around each call."""
+        """One decode step; with `ev`, an event pair around each call.  In
+        exact-score mode the sets come from the exact logits and no index is
+        kept (index_keys has nothing to do)."""
         if ev is not None:
             e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
             e[0].record(stream)
-        st.sd.index_keys(new_keys, new_slots, st.index_cache, stream)
+        if not exact:
+            st.sd.index_keys(new_keys, new_slots, st.index_cache, stream)
         if ev is not None:
             e[1].record(stream)
-        st.select(w.q_pre, stream)
+        if exact:
+            st.select_exact(w.q, stream)
+        else:
+            st.select(w.q_pre, stream)
         if ev is not None:
             e[2].record(stream)
         st.attend(w.q, stream=stream)
@@ -421,7 +431,8 @@ def run_ours(args):
     rows, index_tokens = union_rows(st.sel_idx, st.sel_count, w)
     sel_sizes = st.sel_count.float()
     row_bytes = 4 * d                                   # K + V row, bf16
-    step_bytes = 32 * index_tokens + row_bytes * rows
+    score_row = 2 * d if exact else 32                  # bytes scored per (token, retrieval group)
+    step_bytes = score_row * index_tokens + row_bytes * rows
     flush = l2_flush_needed(args.l2_flush, w)
     flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev) if flush else None
 
@@ -478,10 +489,14 @@ def run_ours(args):
     nk_d, ns_d = torch.empty_like(new_keys), torch.empty_like(new_slots)
 
     def e2e_step():
-        q_d.copy_(q_h, non_blocking=True); qp_d.copy_(qp_h, non_blocking=True)
-        nk_d.copy_(nk_h, non_blocking=True); ns_d.copy_(ns_h, non_blocking=True)
-        st.sd.index_keys(nk_d, ns_d, st.index_cache, stream)
-        st.select(qp_d, stream)
+        q_d.copy_(q_h, non_blocking=True)
+        if exact:
+            st.select_exact(q_d, stream)
+        else:
+            qp_d.copy_(qp_h, non_blocking=True)
+            nk_d.copy_(nk_h, non_blocking=True); ns_d.copy_(ns_h, non_blocking=True)
+            st.sd.index_keys(nk_d, ns_d, st.index_cache, stream)
+            st.select(qp_d, stream)
         st.attend(q_d, stream=stream)
         out_h.copy_(st.out, non_blocking=True)
 
@@ -515,9 +530,10 @@ def run_ours(args):
         raise RuntimeError(f"device error word {word:#x} after timing")
 
     # ---- roofline of the dominant kernel ----
-    index_bytes = 32 * index_tokens
+    index_bytes = score_row * index_tokens
     kv_bytes = row_bytes * rows
-    kern_bytes = {"select": index_bytes, "attend": kv_bytes, "index_keys": B * w.num_kv_heads * (2 * d + 32)}
+    kern_bytes = {"select": index_bytes, "attend": kv_bytes,
+                  "index_keys": 0 if exact else B * w.num_kv_heads * (2 * d + 32)}
     dominant = max(per, key=per.get)
     peak, peak_kind = load_peak()
     achieved = kern_bytes[dominant] / (per[dominant] * 1e-3) / 1e9
@@ -544,15 +560,16 @@ def run_ours(args):
                      "algorithmic_bytes_per_launch": kern_bytes[dominant],
                      "traffic": ncu_traffic(dominant, kern_bytes[dominant])},
         "e2e": {"value": round(head_steps / (e2e_ms * 1e-3), 1), "unit": UNIT,
-                "h2d_bytes_per_step": int(q_h.numel() * 2 + qp_h.numel() * 2 + nk_h.numel() * 2 + ns_h.numel() * 4),
+                "h2d_bytes_per_step": int(q_h.numel() * 2 + (0 if exact else
+                                                             qp_h.numel() * 2 + nk_h.numel() * 2 + ns_h.numel() * 4)),
                 "d2h_bytes_per_step": int(out_h.numel() * 4)},
-        "gpu_launches": kernels_per_step(w) * args.steps,
+        "gpu_launches": kernels_per_step(w, args.score) * args.steps,
         "clocks": clk,
     }
     if rank == 0 and ws == 1 and not args.no_diagnostics:
         res["diagnostics"] = selection_diagnostics(w, st, budget_s=args.diag_budget)
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
+        res["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget, score=args.score)
     st.close()
     if ws > 1:
         dist.destroy_process_group()
@@ -586,7 +603,8 @@ def oracle_slab_step(inp, cfg, b, g, index_g):
     outs = []
     for h in range(g * G, (g + 1) * G):
         if cfg.head_is_retrieval[h]:
-            s = O.index_scores(O.query_index(inp["proj"][g], inp["q_pre"][b, h]), index_g, index_scale)
+            s = (O.exact_scores(inp["q"][b, h], K, attn_scale) if cfg.score == "exact" else
+                 O.index_scores(O.query_index(inp["proj"][g], inp["q_pre"][b, h]), index_g, index_scale))
             S = (O.select_top_p(s, O.stored_top_p(cfg.top_p)) if cfg.mode == "top_p"
                  else O.select_top_k(s, O.top_k_budget(n, cfg.top_k, cfg.top_k_frac)))
         else:
@@ -595,7 +613,7 @@ def oracle_slab_step(inp, cfg, b, g, index_g):
     return np.stack(outs)
 
 
-def cpu_baseline(w, budget_s=15.0):
+def cpu_baseline(w, budget_s=15.0, score="index"):
     """Time the oracle as it stands on (b, KV group) slabs of the workload
     until ~budget_s of CPU work; head-steps/s over the slabs processed."""
     import numpy as np
@@ -603,6 +621,7 @@ def cpu_baseline(w, budget_s=15.0):
     import oracle as O
     from oracle.workload_inputs import oracle_config, oracle_inputs
     cfg = oracle_config(w)
+    cfg.score = score
     G = w.num_q_heads // w.num_kv_heads
     done = 0
     elapsed = 0.0
@@ -639,6 +658,7 @@ def run_reference(args):
     dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
     w = workload_for_rank(args, dev, 0)
     cfg = oracle_config(w)
+    cfg.score = args.score
     G = w.num_q_heads // w.num_kv_heads
     inp = oracle_inputs(w, [0])
     n = int(inp["seq_lens"][0])
@@ -682,6 +702,8 @@ def main(argv=None):
     ap.add_argument("--top-p", type=float, default=0.0, help="override the workload's top-p")
     ap.add_argument("--alpha", type=float, default=0.0, help="long_zipf: Zipf exponent of the score profile")
     ap.add_argument("--top-k-frac", type=float, default=0.0, help="override the workload's top-k fraction")
+    ap.add_argument("--score", choices=["index", "exact"], default="index",
+                    help="select by the r = 16 index (the method) or by the exact logits (reference selector)")
     ap.add_argument("--l2-flush", choices=["auto", "on", "off"], default="auto",
                     help="flush L2 between timed steps (auto: when a step touches < 8x the L2)")
     ap.add_argument("--no-diagnostics", action="store_true")

@@ -261,6 +261,51 @@ sd_status sparse_decode_select(sd_ctx *ctx, const void *q_pre, const void *index
   }
 }
 
+sd_status sparse_decode_select_exact(sd_ctx *ctx, const void *q, const void *k_cache, const int32_t *page_table,
+                                     const int32_t *seq_lens, int batch, int32_t *sel_idx, int32_t *sel_count,
+                                     int sel_stride, void *workspace, size_t ws_bytes, sd_stream stream) {
+  try {
+    if (!ctx) return SD_ERR_INVALID_ARG;
+    if (batch < 0 || batch > ctx->cfg.max_batch) return fail(ctx, SD_ERR_INVALID_ARG, "batch out of range");
+    if (batch == 0 || ctx->sh.H_ret == 0) return SD_OK;
+    if (!q || !k_cache || !page_table || !seq_lens || !sel_idx || !sel_count)
+      return fail(ctx, SD_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(q) || !aligned16(k_cache))
+      return fail(ctx, SD_ERR_INVALID_ARG, "q and k_cache must be 16-byte aligned");
+    const long long need_stride = ctx->cfg.mode == SD_TOP_P ? ctx->sh.max_len : max_topk(ctx);
+    if (sel_stride < need_stride)
+      return fail(ctx, SD_ERR_INVALID_ARG, "sel_stride smaller than the largest possible set");
+    const WsLayout w = layout(ctx, batch);
+    if (!workspace || ws_bytes < w.total) return fail(ctx, SD_ERR_WORKSPACE, "workspace too small");
+    DeviceGuard dg(ctx->device);
+    sd::SelectArgs a{};
+    a.page_table = page_table;
+    a.seq_lens = seq_lens;
+    a.sel_idx = sel_idx;
+    a.sel_count = sel_count;
+    a.sel_stride = sel_stride;
+    a.proj = ctx->proj_d;
+    a.index_scale = ctx->index_scale;
+    a.mode = ctx->cfg.mode;
+    a.top_p = ctx->cfg.top_p;
+    a.top_k = ctx->cfg.top_k;
+    a.top_k_frac = ctx->cfg.top_k_frac;
+    a.score_ws = reinterpret_cast<float *>(static_cast<char *>(workspace) + w.scores_off);
+    a.flags = reinterpret_cast<uint32_t *>(static_cast<char *>(workspace) + w.flags_off);
+    a.stream_ws = nullptr;
+    a.err = ctx->err_d;
+    a.batch = batch;
+    a.pre_scored = true;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = sd::launch_exact_scores(a, ctx->sh, ctx->tb, static_cast<const uint16_t *>(q),
+                                            static_cast<const uint16_t *>(k_cache), ctx->attn_scale, st);
+    if (e == cudaSuccess) e = sd::launch_select(a, ctx->sh, ctx->tb, st);
+    return e == cudaSuccess ? SD_OK : cuda_fail(ctx, e, "exact-score select launch");
+  } catch (...) {
+    return SD_ERR_HOST_MEMORY;
+  }
+}
+
 sd_status sparse_decode_attend(sd_ctx *ctx, const void *q, const void *k_cache, const void *v_cache,
                                const int32_t *page_table, const int32_t *seq_lens, int batch,
                                const int32_t *sel_idx, const int32_t *sel_count, int sel_stride, float *out,

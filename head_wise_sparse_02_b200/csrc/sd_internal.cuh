@@ -143,10 +143,15 @@ struct SelectArgs {
   void *stream_ws;                // streaming selection scratch (histograms, buffers, bitmaps)
   unsigned *err;
   int batch;
+  bool pre_scored;                // score_ws already holds every head's scores (exact-score mode)
 };
 
 size_t select_workspace_bytes(const Shape &sh, const Tables &tb, int batch, size_t *flags_off);
 cudaError_t launch_select(const SelectArgs &a, const Shape &sh, const Tables &tb, cudaStream_t st);
+// Exact-score selection: score_ws rows := attn_scale * q . k for every
+// retrieval head and cached token (then launch_select with pre_scored).
+cudaError_t launch_exact_scores(const SelectArgs &a, const Shape &sh, const Tables &tb, const uint16_t *q,
+                                const uint16_t *k_cache, float attn_scale, cudaStream_t st);
 // Streaming selection (top-k and top-p): workspace bytes for a batch (0 when
 // the shapes are outside what it handles), and its launches; *used = false
 // when it did not run and the exact selector must take every item.

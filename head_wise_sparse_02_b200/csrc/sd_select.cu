@@ -173,7 +173,8 @@ __device__ __forceinline__ void select_item(const SelectArgs &a, const Shape &sh
   };
 
   // ---- q~ = c * P_g^T q_pre (float64 accumulation) ----------------------
-  for (int o = tid; o < kMaxGroup * kIndexDim; o += kThreads) {
+  // (scores written beforehand by the exact-score kernel: only their maxima)
+  for (int o = tid; o < kMaxGroup * kIndexDim && !a.pre_scored; o += kThreads) {
     const int i = o / kIndexDim, j = o % kIndexDim;
     float v = 0.0f;
     if (i < nr) {
@@ -189,8 +190,21 @@ __device__ __forceinline__ void select_item(const SelectArgs &a, const Shape &sh
   if (tid < kMaxGroup) S.cmax_key[tid] = 0u;
   __syncthreads();
 
+  if constexpr (!SMEM) {
+    if (a.pre_scored) {
+      // ---- the score rows are given: the CTA's maxima only ------------------
+      for (int h = 0; h < nr; ++h) {
+        const float *sc = score_ptr(h);
+        float m = -INFINITY;
+        for (int i = tid; i < cnt; i += kThreads) m = fmaxf(m, sc[i]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
+        if (lane == 0 && m > -INFINITY) atomicMax(&S.cmax_key[h], order_key(m));
+      }
+    }
+  }
   // ---- stream the index, score, keep scores on chip ----------------------
-  {
+  if (!a.pre_scored) {
     constexpr int HPB = GR < 4 ? GR : 4;          // heads per thread
     constexpr int HB = GR / HPB;                  // head blocks (threads per token)
     const int hb = tid % HB;
@@ -744,10 +758,19 @@ cudaError_t launch_select(const SelectArgs &a, const Shape &sh, const Tables &tb
     p.tc_cap = (int)(((sh.max_len + c - 1) / c + kPage - 1) / kPage * kPage);
     p.dyn_bytes = hist_bytes(group_rows(tb), topp);
   }
+  if (a.pre_scored) {
+    // exact-score mode: the score rows are in the workspace already; every
+    // item goes through the exact selector, reading them there
+    p.smem = false;
+    p.tc_cap = (int)(((sh.max_len + p.cluster - 1) / p.cluster + kPage - 1) / kPage * kPage);
+    p.dyn_bytes = hist_bytes(group_rows(tb), topp);
+  }
   const int items = a.batch * tb.n_ret;
   bool used = false;
-  cudaError_t e = launch_select_stream(a, sh, tb, a.flags, a.stream_ws, st, &used);
-  if (e != cudaSuccess) return e;
+  if (!a.pre_scored) {
+    cudaError_t e = launch_select_stream(a, sh, tb, a.flags, a.stream_ws, st, &used);
+    if (e != cudaSuccess) return e;
+  }
   // after the streaming passes: exact recomputation of the items whose window
   // missed (usually none); without them: every item
   const uint32_t *flags = used ? a.flags : nullptr;

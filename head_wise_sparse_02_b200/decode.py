@@ -48,6 +48,11 @@ class DecodeStep:
         self.sd.select(q_pre, self.index_cache, self.page_table, self.seq_lens, self.sel_idx,
                        self.sel_count, self.workspace, stream)
 
+    def select_exact(self, q: torch.Tensor, stream=None):
+        """Sets by the exact attention logits (post-RoPE q against the K cache)."""
+        self.sd.select_exact(q, self.k_cache, self.page_table, self.seq_lens, self.sel_idx,
+                             self.sel_count, self.workspace, stream)
+
     def attend(self, q: torch.Tensor, sel_idx=None, sel_count=None, stream=None):
         self.sd.attend(q, self.k_cache, self.v_cache, self.page_table, self.seq_lens,
                        self.sel_idx if sel_idx is None else sel_idx,

@@ -52,6 +52,7 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sparse_decode_workspace_size": (c_int, [P, c_int, POINTER(c_size_t)]),
         "sparse_decode_index_keys": (c_int, [P, P, P, c_int, P, P]),
         "sparse_decode_select": (c_int, [P, P, P, P, P, c_int, P, P, c_int, P, c_size_t, P]),
+        "sparse_decode_select_exact": (c_int, [P, P, P, P, P, c_int, P, P, c_int, P, c_size_t, P]),
         "sparse_decode_attend": (c_int, [P, P, P, P, P, P, c_int, P, P, c_int, P, P, c_size_t, P]),
         "sparse_decode_attend_noalloc": (c_int, [P, P, P, P, P, P, c_int, P, P, c_int, P, P]),
         "sparse_decode_error_word": (c_int, [P, P, POINTER(c_uint32)]),
@@ -167,6 +168,18 @@ def sparse_decode_select(ctx: int, q_pre, index_cache, page_table, seq_lens, sel
         _ptr(workspace, torch.uint8, "workspace"), int(workspace.numel()), _stream(stream)), ctx)
 
 
+def sparse_decode_select_exact(ctx: int, q, k_cache, page_table, seq_lens, sel_idx, sel_count, workspace,
+                               stream=None) -> None:
+    """Sets chosen by the exact attention logits (post-RoPE q against the K cache)."""
+    _check_sets(ctx, sel_idx, sel_count, int(seq_lens.numel()))
+    _check(LIB.sparse_decode_select_exact(
+        ctx, _ptr(q, torch.bfloat16, "q"), _ptr(k_cache, torch.bfloat16, "k_cache"),
+        _ptr(page_table, torch.int32, "page_table"), _ptr(seq_lens, torch.int32, "seq_lens"),
+        int(seq_lens.numel()), _ptr(sel_idx, torch.int32, "sel_idx"),
+        _ptr(sel_count, torch.int32, "sel_count"), int(sel_idx.shape[-1]),
+        _ptr(workspace, torch.uint8, "workspace"), int(workspace.numel()), _stream(stream)), ctx)
+
+
 def sparse_decode_attend(ctx: int, q, k_cache, v_cache, page_table, seq_lens, sel_idx, sel_count,
                          out, workspace, stream=None) -> None:
     _check_sets(ctx, sel_idx, sel_count, int(seq_lens.numel()))
@@ -260,6 +273,10 @@ class SparseDecode:
     def select(self, q_pre, index_cache, page_table, seq_lens, sel_idx, sel_count, workspace, stream=None):
         sparse_decode_select(self.handle, q_pre, index_cache, page_table, seq_lens, sel_idx, sel_count,
                              workspace, stream)
+
+    def select_exact(self, q, k_cache, page_table, seq_lens, sel_idx, sel_count, workspace, stream=None):
+        sparse_decode_select_exact(self.handle, q, k_cache, page_table, seq_lens, sel_idx, sel_count,
+                                   workspace, stream)
 
     def attend(self, q, k_cache, v_cache, page_table, seq_lens, sel_idx, sel_count, out, workspace,
                stream=None):

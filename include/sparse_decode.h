@@ -234,6 +234,31 @@ SD_API sd_status sparse_decode_select(sd_ctx *ctx, const void *q_pre, const void
                                void *workspace, size_t ws_bytes, sd_stream stream);
 
 /*
+ * sparse_decode_select_exact -- per (sequence b, retrieval head h) token sets
+ * chosen by the exact attention logits instead of the index (ICS page, 2: the
+ * "Oracle Top-K" reference selector, applied here with top-k or top-p alike):
+ *
+ *   s_j = attn_scale * <q[b, h], k_j>           j < N_b, float32 accumulation
+ *   top-p / top-k over s_j exactly as for sparse_decode_select
+ *
+ *   q           device bf16 [B, Hq, d], post-RoPE queries (only retrieval
+ *               heads are read).
+ *   k_cache     device bf16 [num_pages, Hkv, P, d]; page_table, seq_lens as
+ *               described above.
+ *   sel_idx, sel_count, sel_stride, workspace, ws_bytes   as for
+ *               sparse_decode_select (the same workspace size).
+ *
+ * Every cached key of every retrieval KV group is read once per call
+ * (2 d bytes per token, against 2 r for the index): a ground truth for the
+ * index selection, not a substitute for it.  Errors as for
+ * sparse_decode_select.
+ */
+SD_API sd_status sparse_decode_select_exact(sd_ctx *ctx, const void *q, const void *k_cache,
+                                     const int32_t *page_table, const int32_t *seq_lens, int batch,
+                                     int32_t *sel_idx, int32_t *sel_count, int sel_stride,
+                                     void *workspace, size_t ws_bytes, sd_stream stream);
+
+/*
  * sparse_decode_attend -- attention output of every head (ICS page, 3c;
  * RTPurbo Methodology 1):
  *

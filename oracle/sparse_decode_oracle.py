@@ -68,6 +68,7 @@ __all__ = [
     "index_keys",
     "query_index",
     "index_scores",
+    "exact_scores",
     "select_top_p",
     "stored_top_p",
     "select_top_k",
@@ -145,6 +146,14 @@ def query_index(proj_g, q_row) -> np.ndarray:
 def index_scores(q_idx, k_idx, index_scale: float) -> np.ndarray:
     """Index scores s_j = c * <q~, k~_j> for every cached token j.  [RTP] §2."""
     return float(index_scale) * (np.asarray(k_idx, np.float64) @ np.asarray(q_idx, np.float64))
+
+
+def exact_scores(q, K, attn_scale: float) -> np.ndarray:
+    """Exact attention logits l_j = attn_scale * <q, k_j> of one query against
+    every cached key (post-RoPE q and the cached keys).  [ICS] §2: "Oracle
+    Top-K" selects the tokens by these true attention scores instead of an
+    approximate index."""
+    return float(attn_scale) * (widen(K) @ widen(q))
 
 
 # --------------------------------------------------------------------------
@@ -274,6 +283,7 @@ class OracleConfig:
     top_k_frac: float = 0.0
     attn_scale: Optional[float] = None
     index_scale: Optional[float] = None
+    score: str = "index"           # "index" (r-dim index, [RTP] §2) or "exact" ([ICS] §2)
 
     def scales(self) -> Tuple[float, float]:
         a = self.attn_scale if self.attn_scale else 1.0 / math.sqrt(self.head_dim)
@@ -296,7 +306,8 @@ def decode_reference(cfg: OracleConfig, proj, q_pre, q, k_cache, v_cache,
 
     For a retrieval head ([RTP] §1-§3): build the index of the sequence's keys
     of its KV head, score every cached token, select by top-p or top-k, attend
-    exactly over the selected rows.  For a local head ([RTP] §1, [AoH] §4):
+    exactly over the selected rows.  With cfg.score == "exact" the tokens are
+    scored by the exact attention logits instead of the index ([ICS] §2).  For a local head ([RTP] §1, [AoH] §4):
     attend over sinks plus the recent window.  Head h uses KV head
     h // (Hq / Hkv) (GQA).  ``sets_override`` replaces the selection of the
     given retrieval pairs (used to test attention alone).
@@ -319,10 +330,13 @@ def decode_reference(cfg: OracleConfig, proj, q_pre, q, k_cache, v_cache,
             if sets_override is not None and (b, h) in sets_override:
                 S = np.asarray(sets_override[(b, h)], dtype=np.int64)
             else:
-                if (b, g) not in index_cache:
-                    index_cache[(b, g)] = index_keys(proj[g], K)
-                qi = query_index(proj[g], q_pre[b, h])
-                s = index_scores(qi, index_cache[(b, g)], index_scale)
+                if cfg.score == "exact":
+                    s = exact_scores(q[b, h], K, attn_scale)
+                else:
+                    if (b, g) not in index_cache:
+                        index_cache[(b, g)] = index_keys(proj[g], K)
+                    qi = query_index(proj[g], q_pre[b, h])
+                    s = index_scores(qi, index_cache[(b, g)], index_scale)
                 if cfg.mode == "top_p":
                     S = select_top_p(s, stored_top_p(cfg.top_p))
                 else:

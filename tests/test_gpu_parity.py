@@ -31,16 +31,21 @@ def _pairs(w, seqs, heads=None):
     return [(b, h) for b in seqs for h in heads]
 
 
-def check_workload(w, seqs=None, heads=None, label=""):
+def check_workload(w, seqs=None, heads=None, label="", score="index"):
     """Run select + attend on the GPU and compare with the oracle on the given
-    sequences / heads.  Returns the number of band tokens reported."""
+    sequences / heads.  Returns the number of band tokens reported.  With
+    score="exact" the sets come from the exact attention logits on both sides."""
     st = make_step(w)
-    st.select(w.q_pre)
+    if score == "exact":
+        st.select_exact(w.q)
+    else:
+        st.select(w.q_pre)
     out_e2e = st.attend(w.q).clone()
     torch.cuda.synchronize()
     assert st.error_word() == 0
     seqs = list(range(w.batch)) if seqs is None else list(seqs)
     cfg = oracle_config(w)
+    cfg.score = score
     inp = oracle_inputs(w, seqs)
     local_pairs = _pairs(w, range(len(seqs)), heads)
     ref = O.decode_reference(cfg, **inp, pairs=local_pairs, keep_scores=True)
@@ -413,5 +418,46 @@ def test_full_size_all_retrieval_heads(name, kw, seqs):
     band = check_workload(w, seqs=seqs, heads=heads, label=f"{name}{kw}")
     print(f"{name} {kw} seqs {seqs}: {len(retr) * len(seqs)} retrieval sets compared, "
           f"{band} tokens inside the threshold band")
+    del w
+    torch.cuda.empty_cache()
+
+
+# ------------------------------------------------------------------ exact-score selection
+
+EXACT = [
+    ("tiny_ref", dict()),
+    ("tiny_ref", dict(N=69, permute=True, seed=4)),
+    ("llama3_8b_topp", dict(B=2, N=3001, window=256)),
+    ("topk_128k", dict(B=2, N=8192, permute=True)),
+    ("topk_128k", dict(B=1, N=4100, top_k=5)),
+    ("long_zipf", dict(N=20000, top_p=0.9, alpha=1.2)),
+    ("ragged_paged", dict(B=4, N_min=300, N_max=5000, window=200)),
+]
+
+
+@pytest.mark.parametrize("name,kw", EXACT, ids=[f"{n}-{i}" for i, (n, _) in enumerate(EXACT)])
+def test_exact_score_selection(name, kw):
+    """Sets chosen by the exact attention logits (the reference selector of
+    the ICS page) against the oracle in exact-score mode, then attention over
+    them, for top-p and top-k workloads, ragged and permuted."""
+    w = make_workload(name, "cuda", **kw)
+    check_workload(w, label=f"exact {name}{kw}", score="exact")
+
+
+def test_exact_score_selection_d64_and_group16():
+    from workloads.synthetic import _base
+    w = _base("d64_topk", 12, "cuda", [2000, 3333], 8, 2, 64, [1] * 8, 0, 0, "top_k", permute=True,
+              top_k_frac=0.03)
+    check_workload(w, label="exact d64", score="exact")
+    w = _base("g16_topp", 13, "cuda", [2900, 1700], 32, 2, 128, [1] * 16 + [0] * 16, 300, 4, "top_p",
+              permute=True, top_p=0.9)
+    check_workload(w, label="exact g16", score="exact")
+
+
+def test_exact_score_selection_full_size_128k():
+    """The 128K fixed-budget workload in exact-score mode, in the launch
+    configuration the bench times, on three sequences' heads."""
+    w = make_workload("topk_128k", "cuda")
+    check_workload(w, seqs=[0, 15], heads=list(range(0, 32, 3)), label="exact topk_128k", score="exact")
     del w
     torch.cuda.empty_cache()

@@ -484,3 +484,70 @@ def test_mass_retained_of_a_top_p_set_on_full_logits_reaches_p():
         assert m >= p - 1e-12
         low = S[np.argmin(s[S])]
         assert O.mass_retained(q, K, np.setdiff1d(S, [low]), 0.25) < p
+
+
+# ---------------------------------------------------------------- exact-score selection
+
+def test_exact_scores_equal_index_scores_under_an_identity_index():
+    """With r = d, P = I and c = attn_scale, the index of a key is the key
+    itself (bf16 values round to themselves) and q~ = q, so index scoring and
+    exact scoring coincide: the two selections must agree token for token."""
+    rng = np.random.default_rng(21)
+    d, n = 16, 400
+    K = O.bf16_round(rng.standard_normal((n, d)))
+    q = O.bf16_round(rng.standard_normal(d) * 2.0)
+    P = np.eye(d)
+    s_idx = O.index_scores(O.query_index(P, q), O.index_keys(P, K), 0.25)
+    s_ex = O.exact_scores(q, K, 0.25)
+    assert np.array_equal(s_idx, s_ex)
+    for p in (0.5, 0.9):
+        assert np.array_equal(O.select_top_p(s_idx, p), O.select_top_p(s_ex, p))
+    assert np.array_equal(O.select_top_k(s_idx, 37), O.select_top_k(s_ex, 37))
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_exact_top_p_is_the_smallest_set_holding_p_of_the_attention_mass(seed):
+    """Selecting by the exact logits, the top-p set is a minimum-size subset
+    whose share of the full softmax (mass_retained) reaches p, and among those
+    the one with the largest share: brute force over all subsets of a 10-token
+    context."""
+    rng = np.random.default_rng(300 + seed)
+    d, n = 8, 10
+    K = O.bf16_round(rng.standard_normal((n, d)) * 1.5)
+    q = O.bf16_round(rng.standard_normal(d))
+    p = float(rng.uniform(0.3, 0.95))
+    S = O.select_top_p(O.exact_scores(q, K, 0.5), p)
+    best = None
+    for size in range(1, n + 1):
+        cands = [c for c in itertools.combinations(range(n), size) if O.mass_retained(q, K, c, 0.5) >= p]
+        if cands:
+            best = (size, max(O.mass_retained(q, K, c, 0.5) for c in cands))
+            break
+    assert len(S) == best[0]
+    assert O.mass_retained(q, K, S, 0.5) == pytest.approx(best[1], rel=1e-12)
+
+
+def test_decode_step_with_exact_scores_selects_by_the_attention_logits():
+    """A decode step in exact-score mode on planted keys: under a projection
+    that hides the planted direction from the index, the index selection
+    misses the planted tokens while the exact selection keeps exactly them
+    (top-k = their number)."""
+    rng = np.random.default_rng(5)
+    d, n, G = 32, 64, 1
+    K = rng.standard_normal((n, d)) * 0.1
+    q = np.zeros(d)
+    q[0] = 4.0
+    planted = [5, 17, 40]
+    for j in planted:
+        K[j, 0] = 3.0                                    # large logits along q
+    K = O.bf16_round(K)
+    P = np.zeros((1, d, 16))
+    P[0, 1:17, :] = np.eye(16)                           # the index never sees dimension 0
+    kc = K.reshape(n // 16, 1, 16, d)
+    pt = np.arange(n // 16)[None, :]
+    base = dict(proj=P, q_pre=q[None, None, :], q=q[None, None, :], k_cache=kc, v_cache=kc,
+                page_table=pt, seq_lens=np.array([n]))
+    for score, want_all in (("exact", True), ("index", False)):
+        cfg = O.OracleConfig(1, 1, d, 16, 16, [1], 0, 0, "top_k", top_k=3, score=score)
+        S = O.decode_reference(cfg, **base).sets[(0, 0)]
+        assert (set(S.tolist()) == set(planted)) == want_all
