@@ -396,29 +396,31 @@ def run_ours(args):
     new_keys = keys_at(w, new_slots)
     stream = torch.cuda.current_stream()
 
-    calls = ("index_keys", "select", "attend")
     exact = args.score == "exact"
+    # the decode step through the public API: index_keys for the appended
+    # tokens, then the joined select + attend call (exact-score mode: the
+    # exact-score select, then attend; no index is kept)
+    calls = ("index_keys", "select", "attend") if exact else ("index_keys", "select_attend")
 
     def step(ev=None):
-        """One decode step; with `ev`, an event pair around each call.  In
-        exact-score mode the sets come from the exact logits and no index is
-        kept (index_keys has nothing to do)."""
+        """One decode step; with `ev`, an event pair around each call."""
         if ev is not None:
-            e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
             e[0].record(stream)
-        if not exact:
-            st.sd.index_keys(new_keys, new_slots, st.index_cache, stream)
-        if ev is not None:
-            e[1].record(stream)
         if exact:
+            if ev is not None:
+                e[1].record(stream)
             st.select_exact(w.q, stream)
+            if ev is not None:
+                e[2].record(stream)
+            st.attend(w.q, stream=stream)
         else:
-            st.select(w.q_pre, stream)
+            st.sd.index_keys(new_keys, new_slots, st.index_cache, stream)
+            if ev is not None:
+                e[1].record(stream)
+            st.select_attend(w.q_pre, w.q, stream)
         if ev is not None:
-            e[2].record(stream)
-        st.attend(w.q, stream=stream)
-        if ev is not None:
-            e[3].record(stream)
+            e[len(calls)].record(stream)
             for i, k in enumerate(calls):
                 ev[k].append((e[i], e[i + 1]))
 
@@ -492,12 +494,12 @@ def run_ours(args):
         q_d.copy_(q_h, non_blocking=True)
         if exact:
             st.select_exact(q_d, stream)
+            st.attend(q_d, stream=stream)
         else:
             qp_d.copy_(qp_h, non_blocking=True)
             nk_d.copy_(nk_h, non_blocking=True); ns_d.copy_(ns_h, non_blocking=True)
             st.sd.index_keys(nk_d, ns_d, st.index_cache, stream)
-            st.select(qp_d, stream)
-        st.attend(q_d, stream=stream)
+            st.select_attend(qp_d, q_d, stream)
         out_h.copy_(st.out, non_blocking=True)
 
     for _ in range(max(1, args.warmup)):
@@ -532,8 +534,8 @@ def run_ours(args):
     # ---- roofline of the dominant kernel ----
     index_bytes = score_row * index_tokens
     kv_bytes = row_bytes * rows
-    kern_bytes = {"select": index_bytes, "attend": kv_bytes,
-                  "index_keys": 0 if exact else B * w.num_kv_heads * (2 * d + 32)}
+    kern_bytes = ({"select": index_bytes, "attend": kv_bytes, "index_keys": 0} if exact else
+                  {"select_attend": index_bytes + kv_bytes, "index_keys": B * w.num_kv_heads * (2 * d + 32)})
     dominant = max(per, key=per.get)
     peak, peak_kind = load_peak()
     achieved = kern_bytes[dominant] / (per[dominant] * 1e-3) / 1e9

@@ -346,6 +346,83 @@ sd_status sparse_decode_attend(sd_ctx *ctx, const void *q, const void *k_cache, 
   }
 }
 
+sd_status sparse_decode_select_attend(sd_ctx *ctx, const void *q_pre, const void *q, const void *index_cache,
+                                     const void *k_cache, const void *v_cache, const int32_t *page_table,
+                                     const int32_t *seq_lens, int batch, int32_t *sel_idx, int32_t *sel_count,
+                                     int sel_stride, float *out, void *workspace, size_t ws_bytes, sd_stream stream) {
+  try {
+    if (!ctx) return SD_ERR_INVALID_ARG;
+    if (batch < 0 || batch > ctx->cfg.max_batch) return fail(ctx, SD_ERR_INVALID_ARG, "batch out of range");
+    if (batch == 0) return SD_OK;
+    if (!q || !k_cache || !v_cache || !page_table || !seq_lens || !out)
+      return fail(ctx, SD_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+      return fail(ctx, SD_ERR_INVALID_ARG, "q, k_cache and v_cache must be 16-byte aligned");
+    const bool ret = ctx->sh.H_ret > 0;
+    if (ret) {
+      if (!q_pre || !index_cache || !sel_idx || !sel_count) return fail(ctx, SD_ERR_INVALID_ARG, "null pointer");
+      if (!aligned16(q_pre) || !aligned16(index_cache))
+        return fail(ctx, SD_ERR_INVALID_ARG, "q_pre and index_cache must be 16-byte aligned");
+      const long long need_stride = ctx->cfg.mode == SD_TOP_P ? ctx->sh.max_len : max_topk(ctx);
+      if (sel_stride < need_stride)
+        return fail(ctx, SD_ERR_INVALID_ARG, "sel_stride smaller than the largest possible set");
+    }
+    const WsLayout w = layout(ctx, batch);
+    if (!workspace || ws_bytes < w.total) return fail(ctx, SD_ERR_WORKSPACE, "workspace too small");
+    DeviceGuard dg(ctx->device);
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char *wsb = static_cast<char *>(workspace);
+    bool unioned = false;
+    if (ret) {
+      sd::SelectArgs a{};
+      a.q_pre = static_cast<const uint16_t *>(q_pre);
+      a.index_cache = static_cast<const uint16_t *>(index_cache);
+      a.page_table = page_table;
+      a.seq_lens = seq_lens;
+      a.sel_idx = sel_idx;
+      a.sel_count = sel_count;
+      a.sel_stride = sel_stride;
+      a.proj = ctx->proj_d;
+      a.index_scale = ctx->index_scale;
+      a.mode = ctx->cfg.mode;
+      a.top_p = ctx->cfg.top_p;
+      a.top_k = ctx->cfg.top_k;
+      a.top_k_frac = ctx->cfg.top_k_frac;
+      a.score_ws = reinterpret_cast<float *>(wsb + w.scores_off);
+      a.flags = reinterpret_cast<uint32_t *>(wsb + w.flags_off);
+      a.stream_ws = w.stream_bytes ? wsb + w.stream_off : nullptr;
+      a.err = ctx->err_d;
+      a.batch = batch;
+      const sd::UnionOut uo = sd::attend_union_view(ctx->sh, ctx->tb, batch, wsb + w.att_off);
+      const cudaError_t e = sd::launch_select_union(a, ctx->sh, ctx->tb, uo, st, &unioned);
+      if (e != cudaSuccess) return cuda_fail(ctx, e, "select launch");
+    }
+    sd::AttendArgs at{};
+    at.q = static_cast<const uint16_t *>(q);
+    at.k_cache = static_cast<const uint16_t *>(k_cache);
+    at.v_cache = static_cast<const uint16_t *>(v_cache);
+    at.page_table = page_table;
+    at.seq_lens = seq_lens;
+    at.sel_idx = sel_idx;
+    at.sel_count = sel_count;
+    at.sel_stride = sel_stride;
+    at.out = out;
+    at.attn_scale = ctx->attn_scale;
+    at.window = ctx->cfg.window;
+    at.num_sinks = ctx->cfg.num_sinks;
+    at.ws = wsb + w.att_off;
+    at.err = ctx->err_d;
+    at.batch = batch;
+    // with the union lists built by select, attend plans only the items the
+    // exact selector redid (listed in the miss array)
+    const uint32_t *only = unioned ? reinterpret_cast<const uint32_t *>(wsb + w.flags_off) : nullptr;
+    const cudaError_t e = sd::launch_attend(at, ctx->sh, ctx->tb, st, only);
+    return e == cudaSuccess ? SD_OK : cuda_fail(ctx, e, "attend launch");
+  } catch (...) {
+    return SD_ERR_HOST_MEMORY;
+  }
+}
+
 sd_status sparse_decode_attend_noalloc(sd_ctx *ctx, const void *q, const void *k_cache, const void *v_cache,
                                        const int32_t *page_table, const int32_t *seq_lens, int batch,
                                        const int32_t *sel_idx, const int32_t *sel_count, int sel_stride,

@@ -73,6 +73,7 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, int sr
                "r"(src_bytes), "l"(policy)
                : "memory");
 }
+
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
@@ -358,8 +359,10 @@ __device__ void plan_span(const AttendArgs &a, const Shape &sh, const Tables &tb
   uint16_t *masks = ws.plan_mask + slot * ap.span;
   const uint32_t row_g = (uint32_t)g * kPage;          // row of (page, g, slot) = (page * Hkv + g) * 16 + slot
   const uint32_t row_page = (uint32_t)sh.Hkv * kPage;
+  bool bad_page = false;
   for (int r = 0; r < steps; ++r) {
-    const int x = x0 + r * 32 + lane;
+    const int xb = x0 + r * 32;
+    const int x = xb + lane;
     uint32_t hw[GR];
     uint32_t u = 0;
 #pragma unroll
@@ -367,45 +370,54 @@ __device__ void plan_span(const AttendArgs &a, const Shape &sh, const Tables &tb
       hw[i] = (x < bwords && i < nh) ? hbm[i * bwords + x] : 0u;
       u |= hw[i];
     }
-    const uint32_t n = __popc(u);
-    uint32_t incl = n;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-      const uint32_t y = __shfl_up_sync(kFull, incl, d);
-      if (lane >= d) incl += y;
-    }
-    uint32_t at = o + incl - n;
-    while (u) {
-      const int bit = __ffs(u) - 1;
-      u &= u - 1;
+    // union rows handed out 32 at a time: each store writes consecutive entries
+    o += (uint32_t)warp_emit_bits(u, lane, [&](bool valid, int k, int w, int bit) {
       uint32_t m = 0;
 #pragma unroll
-      for (int i = 0; i < GR; ++i) m |= ((hw[i] >> bit) & 1u) << i;
-      const int off = x * 32 + bit;
+      for (int i = 0; i < GR; ++i) m |= ((__shfl_sync(kFull, hw[i], w) >> bit) & 1u) << i;   // every lane
+      if (!valid) return;
+      const int off = (xb + w) * 32 + bit;
       const int page = pslice[off >> 4];
-      if (page < 0) raise_error(a.err, SD_EBIT_PAGE);
-      rows[at] = page >= 0 ? (uint32_t)page * row_page + row_g + (uint32_t)(off & (kPage - 1)) : 0u;
-      masks[at] = (uint16_t)(page >= 0 ? m : 0u);
-      ++at;
-    }
-    o += __shfl_sync(kFull, incl, 31);
+      bad_page |= page < 0;
+      rows[o + k] = page >= 0 ? (uint32_t)page * row_page + row_g + (uint32_t)(off & (kPage - 1)) : 0u;
+      masks[o + k] = (uint16_t)(page >= 0 ? m : 0u);
+    });
   }
+  if (bad_page) raise_error(a.err, SD_EBIT_PAGE);
   if (tid == 0) ws.plan_cnt[slot] = (int)total;
 }
 
 // dynamic shared memory: [per-head bitmaps: GR x span / 32 words][page slice: span / 16 ints]
+// Without `only`: CTA (split, gi, b) plans span `split` of retrieval item
+// (b, gi).  With `only` (the select's miss array: [items] flags, count, list),
+// the CTAs (split, y) stride over the listed items only.
 template <int D, int GR>
 __global__ void __launch_bounds__(kPlanThreads)
-attend_plan_kernel(const AttendArgs a, const Shape sh, const Tables tb, const AttParams ap, const AttWs ws) {
+attend_plan_kernel(const AttendArgs a, const Shape sh, const Tables tb, const AttParams ap, const AttWs ws,
+                   const uint32_t *only) {
   const int tid = threadIdx.x;
-  const int split = blockIdx.x, gi = blockIdx.y, b = blockIdx.z;
+  const int split = blockIdx.x;
   __shared__ Group grp;
   extern __shared__ uint32_t plan_dyn[];
-  if (tid == 0) grp = tb.ret[gi];
+  int *pslice = reinterpret_cast<int *>(plan_dyn + GR * (ap.span / 32));
+  if (only == nullptr && tid == 0) grp = tb.ret[blockIdx.y];
   pdl_wait();
   pdl_trigger();
   __syncthreads();
-  plan_span<GR>(a, sh, tb, ap, ws, grp, b, gi, split, plan_dyn, reinterpret_cast<int *>(plan_dyn + GR * (ap.span / 32)));
+  if (only == nullptr) {
+    plan_span<GR>(a, sh, tb, ap, ws, grp, blockIdx.z, blockIdx.y, split, plan_dyn, pslice);
+    return;
+  }
+  const int n_items = ap.n_ret_items;
+  const int listed = (int)__ldcg(only + n_items);
+  for (int k = blockIdx.y; k < listed; k += gridDim.y) {
+    const int item = (int)__ldcg(only + n_items + 1 + k);
+    const int b = item / tb.n_ret, gi = item % tb.n_ret;
+    if (tid == 0) grp = tb.ret[gi];
+    __syncthreads();
+    plan_span<GR>(a, sh, tb, ap, ws, grp, b, gi, split, plan_dyn, pslice);
+    __syncthreads();                                 // grp and the bitmaps are reused by the next item
+  }
 }
 
 // ============================================================== main kernel
@@ -903,14 +915,15 @@ int resident_ctas(K kern, int threads, size_t smem) {
 
 template <int D, int GR>
 cudaError_t launch_t(const AttendArgs &a, const Shape &sh, const Tables &tb, const AttParams &p, const AttWs &ws,
-                     cudaStream_t st) {
+                     cudaStream_t st, const uint32_t *only) {
   cudaError_t e;
   if (tb.n_ret > 0) {
     const size_t pbytes = (size_t)GR * (p.span / 32) * 4 + (size_t)(p.span / kPage) * 4;
     e = set_smem(attend_plan_kernel<D, GR>, pbytes);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(attend_plan_kernel<D, GR>, dim3(p.ns, tb.n_ret, a.batch), dim3(kPlanThreads), pbytes, st, 0,
-                   a, sh, tb, p, ws);
+    // the listed items only (usually none): a few CTAs per span stride over them
+    const dim3 grid = only ? dim3(p.ns, (unsigned)std::min(p.n_ret_items, 4), 1) : dim3(p.ns, tb.n_ret, a.batch);
+    e = launch_pdl(attend_plan_kernel<D, GR>, grid, dim3(kPlanThreads), pbytes, st, 0, a, sh, tb, p, ws, only);
     if (e != cudaSuccess) return e;
   }
   e = launch_pdl(attend_prefix_kernel<D>, dim3(1), dim3(1024), 0, st, 0, a, sh, tb, p, ws);
@@ -928,13 +941,13 @@ cudaError_t launch_t(const AttendArgs &a, const Shape &sh, const Tables &tb, con
 
 template <int D>
 cudaError_t dispatch_gr(const AttendArgs &a, const Shape &sh, const Tables &tb, const AttParams &p,
-                        const AttWs &ws, cudaStream_t st) {
+                        const AttWs &ws, cudaStream_t st, const uint32_t *only) {
   switch (group_rows_att(tb)) {
-    case 1: return launch_t<D, 1>(a, sh, tb, p, ws, st);
-    case 2: return launch_t<D, 2>(a, sh, tb, p, ws, st);
-    case 4: return launch_t<D, 4>(a, sh, tb, p, ws, st);
-    case 8: return launch_t<D, 8>(a, sh, tb, p, ws, st);
-    default: return launch_t<D, 16>(a, sh, tb, p, ws, st);
+    case 1: return launch_t<D, 1>(a, sh, tb, p, ws, st, only);
+    case 2: return launch_t<D, 2>(a, sh, tb, p, ws, st, only);
+    case 4: return launch_t<D, 4>(a, sh, tb, p, ws, st, only);
+    case 8: return launch_t<D, 8>(a, sh, tb, p, ws, st, only);
+    default: return launch_t<D, 16>(a, sh, tb, p, ws, st, only);
   }
 }
 
@@ -944,7 +957,16 @@ size_t attend_workspace_bytes(const Shape &sh, const Tables &tb, int batch) {
   return att_layout(sh, tb, batch).total;
 }
 
-cudaError_t launch_attend(const AttendArgs &a, const Shape &sh, const Tables &tb, cudaStream_t st) {
+UnionOut attend_union_view(const Shape &sh, const Tables &tb, int batch, void *attend_ws) {
+  const AttLayout L = att_layout(sh, tb, batch);
+  const AttParams p = att_params(sh, tb, batch);
+  char *base = static_cast<char *>(attend_ws);
+  return UnionOut{reinterpret_cast<uint32_t *>(base + L.plan_row), reinterpret_cast<uint16_t *>(base + L.plan_mask),
+                  reinterpret_cast<int *>(base + L.plan_cnt), p.span, p.ns};
+}
+
+cudaError_t launch_attend(const AttendArgs &a, const Shape &sh, const Tables &tb, cudaStream_t st,
+                          const uint32_t *plan_only) {
   if (a.batch == 0) return cudaSuccess;
   const AttLayout L = att_layout(sh, tb, a.batch);
   const AttParams p = att_params(sh, tb, a.batch);
@@ -957,7 +979,8 @@ cudaError_t launch_attend(const AttendArgs &a, const Shape &sh, const Tables &tb
   ws.tstart = reinterpret_cast<long long *>(base + L.tstart);
   ws.item_rows = reinterpret_cast<int *>(base + L.counters);
   ws.tickets = reinterpret_cast<unsigned *>(ws.item_rows + p.ni);
-  return sh.d == 128 ? dispatch_gr<128>(a, sh, tb, p, ws, st) : dispatch_gr<64>(a, sh, tb, p, ws, st);
+  return sh.d == 128 ? dispatch_gr<128>(a, sh, tb, p, ws, st, plan_only)
+                     : dispatch_gr<64>(a, sh, tb, p, ws, st, plan_only);
 }
 
 }  // namespace sd

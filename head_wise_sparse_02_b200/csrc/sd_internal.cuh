@@ -67,6 +67,102 @@ __device__ __forceinline__ uint16_t f64_to_bf16_rne(double x) {
   return sign | (uint16_t)(__float_as_uint(y) >> 16);
 }
 
+// Bit position of the n-th set bit (0-based) of v, n < popc(v): binary
+// search over halves by population count.
+__device__ __forceinline__ int nth_set_bit(uint32_t v, int n) {
+  int pos = 0;
+#pragma unroll
+  for (int s = 16; s > 0; s >>= 1) {
+    const uint32_t low = v & ((1u << s) - 1u);
+    const int c = __popc(low);
+    if (n >= c) {
+      n -= c;
+      v >>= s;
+      pos += s;
+    } else {
+      v = low;
+    }
+  }
+  return pos;
+}
+
+// One warp, 32 consecutive bitmap words (word x0 + lane in `bits`): the set
+// bits in ascending order are handed out 32 at a time, lane l taking the
+// (r + l)-th one, so that whatever a caller stores per bit goes out in
+// coalesced rows.  Every lane calls emit(valid, k, w, bit) in every round (so
+// that emit may shuffle); when valid, k in [0, total) is the rank of the set
+// bit it hands out, found in the word of lane w at bit position `bit`.
+// Returns the number of set bits of the 32 words.
+template <typename Emit>
+__device__ __forceinline__ int warp_emit_bits(uint32_t bits, int lane, Emit &&emit) {
+  const unsigned full = 0xFFFFFFFFu;
+  const int n = __popc(bits);
+  int incl = n;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(full, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const int total = __shfl_sync(full, incl, 31);
+  for (int r = 0; r < total; r += 32) {
+    const int k = r + lane;
+    // the word holding set bit k: the first lane whose inclusive count exceeds k
+    int w = 0;
+#pragma unroll
+    for (int st = 16; st > 0; st >>= 1) {
+      const int c = __shfl_sync(full, incl, w + st - 1);
+      if (c <= k) w += st;
+    }
+    const uint32_t wb = __shfl_sync(full, bits, w);
+    const int before = __shfl_sync(full, incl - n, w);
+    emit(k < total, k, w, nth_set_bit(wb, k - before));
+  }
+  return total;
+}
+
+// warp_emit_bits over W consecutive words per lane (lane l holds words
+// W l .. W l + W - 1 of a run of 32 W): fewer, longer steps for sparse bitmaps.
+// emit(valid, k, w, j, bit): set bit k of the run lies in word j of lane w.
+template <int W, typename Emit>
+__device__ __forceinline__ int warp_emit_bits_w(const uint32_t (&bits)[W], int lane, Emit &&emit) {
+  const unsigned full = 0xFFFFFFFFu;
+  int n = 0;
+#pragma unroll
+  for (int j = 0; j < W; ++j) n += __popc(bits[j]);
+  int incl = n;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(full, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const int total = __shfl_sync(full, incl, 31);
+  for (int r = 0; r < total; r += 32) {
+    const int k = r + lane;
+    int w = 0;
+#pragma unroll
+    for (int st = 16; st > 0; st >>= 1) {
+      const int c = __shfl_sync(full, incl, w + st - 1);
+      if (c <= k) w += st;
+    }
+    int rank = k - __shfl_sync(full, incl - n, w);    // rank of the bit among lane w's words
+    uint32_t word = 0;
+    int jw = 0;
+#pragma unroll
+    for (int j = 0; j < W; ++j) {
+      const uint32_t b = __shfl_sync(full, bits[j], w);
+      const int c = __popc(b);
+      if (jw == j && rank >= c && j + 1 < W) {
+        rank -= c;
+        jw = j + 1;
+      } else if (jw == j) {
+        word = b;
+      }
+    }
+    emit(k < total, k, w, jw, nth_set_bit(word, rank));
+  }
+  return total;
+}
+
 __device__ __forceinline__ void raise_error(unsigned *err, unsigned bit) {
   if (err) atomicOr(err, bit);
 }
@@ -146,6 +242,16 @@ struct SelectArgs {
   bool pre_scored;                // score_ws already holds every head's scores (exact-score mode)
 };
 
+// Where a fused select writes the union lists that attend reads: the plan
+// arrays of attend's workspace (union rows of (sequence, retrieval group,
+// span of positions): cache row and head mask of each, their count).
+struct UnionOut {
+  uint32_t *row;                  // [B][n_ret][ns][span]
+  uint16_t *mask;                 // [B][n_ret][ns][span]
+  int *cnt;                       // [B][n_ret][ns]
+  int span, ns;
+};
+
 size_t select_workspace_bytes(const Shape &sh, const Tables &tb, int batch, size_t *flags_off);
 cudaError_t launch_select(const SelectArgs &a, const Shape &sh, const Tables &tb, cudaStream_t st);
 // Exact-score selection: score_ws rows := attn_scale * q . k for every
@@ -156,8 +262,15 @@ cudaError_t launch_exact_scores(const SelectArgs &a, const Shape &sh, const Tabl
 // the shapes are outside what it handles), and its launches; *used = false
 // when it did not run and the exact selector must take every item.
 size_t stream_workspace_bytes(const Shape &sh, const Tables &tb, int batch, int mode);
+// With `uo` (not null) the last pass also builds attend's union lists (one CTA
+// per (sequence, retrieval group)) when the shapes allow it; *unioned tells.
 cudaError_t launch_select_stream(const SelectArgs &a, const Shape &sh, const Tables &tb, uint32_t *fail,
-                                 void *ws_base, cudaStream_t st, bool *used);
+                                 void *ws_base, cudaStream_t st, bool *used, const UnionOut *uo = nullptr,
+                                 bool *unioned = nullptr);
+// launch_select with the union lists built by the streaming pass where it can
+// (*unioned); the items it flags (exact selector) are left for attend's plan.
+cudaError_t launch_select_union(const SelectArgs &a, const Shape &sh, const Tables &tb, const UnionOut &uo,
+                                cudaStream_t st, bool *unioned);
 
 struct AttendArgs {
   const uint16_t *q;
@@ -177,7 +290,12 @@ struct AttendArgs {
 };
 
 size_t attend_workspace_bytes(const Shape &sh, const Tables &tb, int batch);
-cudaError_t launch_attend(const AttendArgs &a, const Shape &sh, const Tables &tb, cudaStream_t st);
+// plan_only: null = plan every retrieval item; else the select's miss array
+// ([items] flags, count, list): only the listed items are planned, the
+// others' union lists are already in the workspace.
+cudaError_t launch_attend(const AttendArgs &a, const Shape &sh, const Tables &tb, cudaStream_t st,
+                          const uint32_t *plan_only = nullptr);
+UnionOut attend_union_view(const Shape &sh, const Tables &tb, int batch, void *attend_ws);
 
 // Size of the built-in attend scratch of sparse_decode_attend_noalloc.
 constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;

@@ -732,7 +732,24 @@ size_t select_workspace_bytes(const Shape &sh, const Tables &tb, int batch, size
   return rows + (2 * (size_t)batch * std::max(1, tb.n_ret) + 1) * sizeof(uint32_t);
 }
 
+namespace {
+cudaError_t launch_select_impl(const SelectArgs &a, const Shape &sh, const Tables &tb, cudaStream_t st,
+                               const UnionOut *uo, bool *unioned);
+}  // namespace
+
 cudaError_t launch_select(const SelectArgs &a, const Shape &sh, const Tables &tb, cudaStream_t st) {
+  return launch_select_impl(a, sh, tb, st, nullptr, nullptr);
+}
+
+cudaError_t launch_select_union(const SelectArgs &a, const Shape &sh, const Tables &tb, const UnionOut &uo,
+                                cudaStream_t st, bool *unioned) {
+  return launch_select_impl(a, sh, tb, st, &uo, unioned);
+}
+
+namespace {
+cudaError_t launch_select_impl(const SelectArgs &a, const Shape &sh, const Tables &tb, cudaStream_t st,
+                               const UnionOut *uo, bool *unioned) {
+  if (unioned) *unioned = false;
   if (tb.n_ret == 0 || a.batch == 0) return cudaSuccess;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -768,7 +785,7 @@ cudaError_t launch_select(const SelectArgs &a, const Shape &sh, const Tables &tb
   const int items = a.batch * tb.n_ret;
   bool used = false;
   if (!a.pre_scored) {
-    cudaError_t e = launch_select_stream(a, sh, tb, a.flags, a.stream_ws, st, &used);
+    cudaError_t e = launch_select_stream(a, sh, tb, a.flags, a.stream_ws, st, &used, uo, unioned);
     if (e != cudaSuccess) return e;
   }
   // after the streaming passes: exact recomputation of the items whose window
@@ -783,5 +800,7 @@ cudaError_t launch_select(const SelectArgs &a, const Shape &sh, const Tables &tb
   return p.smem ? dispatch_gr<false, true>(a, sh, tb, p, dev, st, flags, gy)
                 : dispatch_gr<false, false>(a, sh, tb, p, dev, st, flags, gy);
 }
+
+}  // namespace
 
 }  // namespace sd

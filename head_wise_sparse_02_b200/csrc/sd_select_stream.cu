@@ -64,6 +64,7 @@
 #include <algorithm>
 #include <map>
 #include <mutex>
+#include <type_traits>
 
 #include "sd_internal.cuh"
 
@@ -830,67 +831,93 @@ stream_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__ grou
 // ------------------------------------------------------------------- K2
 constexpr int kT2 = 256;
 
-// Block-wide: the positions set in bitmap[0, words) go to out in ascending
+// K2 runs per head on a group of kT2 threads: alone in its CTA (the per-head
+// resolve kernels) or as one of several groups of a CTA that resolves every
+// retrieval head of a KV group and then builds the group's union list for
+// attend.  A group's barrier is __syncthreads when it is alone, otherwise the
+// named barrier 1 + id over its kT2 threads.
+struct HeadGroup {
+  int t;                    // thread index in the group
+  int id;                   // group index in the CTA
+  bool alone;
+  __device__ __forceinline__ void sync() const {
+    if (alone) __syncthreads();
+    else asm volatile("bar.sync %0, %1;\n" ::"r"(1 + id), "n"(kT2) : "memory");
+  }
+};
+
+// Group-wide: the positions set in bitmap[0, words) go to out in ascending
 // order, their number to sel_count[row].  Warp w owns a contiguous run of
-// words, read lane-strided (32 consecutive words per step, no bank
-// conflicts); a warp-wide scan of the words' bit counts places each lane's
-// positions, a block-wide sum over the warps' totals places the warp.  wtot:
-// kT2 / 32 words of shared memory.
-__device__ void write_ascending(const SelectArgs &a, const uint32_t *bitmap, int words, int32_t *out, long long row,
-                                uint32_t *wtot) {
+// words, 128 per step (four consecutive words per lane, one 16-byte load, no
+// bank conflicts); the set bits of a step are handed out 32 at a time, so
+// every store instruction writes consecutive positions; a group-wide sum over
+// the warps' totals places each warp.  The bitmap is read in whole 16-byte
+// words (its allocation is rounded up to them).  wtot: kT2 / 32 words of
+// shared memory.
+__device__ void write_ascending(const SelectArgs &a, const HeadGroup &hg, const uint32_t *bitmap, int words,
+                                int32_t *out, long long row, uint32_t *wtot) {
   constexpr int NW = kT2 / 32;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int steps = (words + NW * 32 - 1) / (NW * 32);           // 32-word steps per warp
-  const int w0 = warp * steps * 32;
+  constexpr int WPL = 4;                             // words per lane and step
+  const int lane = hg.t & 31, warp = hg.t >> 5;
+  const int steps = (words + NW * 32 * WPL - 1) / (NW * 32 * WPL);
+  const int w0 = warp * steps * 32 * WPL;
+  auto load = [&](int x, uint32_t (&v)[WPL]) {       // words x .. x + 3 (x a multiple of 4)
+    const uint4 q = x < words ? *reinterpret_cast<const uint4 *>(bitmap + x) : make_uint4(0u, 0u, 0u, 0u);
+    v[0] = q.x;
+    v[1] = x + 1 < words ? q.y : 0u;
+    v[2] = x + 2 < words ? q.z : 0u;
+    v[3] = x + 3 < words ? q.w : 0u;
+  };
   uint32_t c = 0;
   for (int r = 0; r < steps; ++r) {
-    const int x = w0 + r * 32 + lane;
-    c += x < words ? __popc(bitmap[x]) : 0u;
+    uint32_t v[WPL];
+    load(w0 + (r * 32 + lane) * WPL, v);
+#pragma unroll
+    for (int j = 0; j < WPL; ++j) c += __popc(v[j]);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(kFull, c, o);
   if (lane == 0) wtot[warp] = c;
-  __syncthreads();
-  uint32_t off = 0, total = 0;
+  hg.sync();
+  long long off = 0, total = 0;
 #pragma unroll
   for (int x = 0; x < NW; ++x) {
     const uint32_t t = wtot[x];
     off += x < warp ? t : 0u;
     total += t;
   }
+  bool over = false;
   for (int r = 0; r < steps; ++r) {
-    const int x = w0 + r * 32 + lane;
-    uint32_t bits = x < words ? bitmap[x] : 0u;
-    const uint32_t n = __popc(bits);
-    uint32_t incl = n;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(kFull, incl, o);
-      if (lane >= o) incl += y;
-    }
-    long long o = (long long)off + (incl - n);
-    while (bits) {
-      const int bit = __ffs(bits) - 1;
-      bits &= bits - 1;
-      if (o < a.sel_stride) out[o] = x * 32 + bit;
-      else raise_error(a.err, SD_EBIT_SEL);
-      ++o;
-    }
-    off += __shfl_sync(kFull, incl, 31);
+    const int x0 = w0 + r * 32 * WPL;
+    uint32_t v[WPL];
+    load(x0 + lane * WPL, v);
+    off += warp_emit_bits_w<WPL>(v, lane, [&](bool valid, int k, int w, int j, int bit) {
+      const long long o = off + k;
+      if (valid) {
+        if (o < a.sel_stride) out[o] = (x0 + w * WPL + j) * 32 + bit;
+        else over = true;
+      }
+    });
   }
-  if (tid == 0) {
-    if ((long long)total > a.sel_stride) raise_error(a.err, SD_EBIT_SEL);
+  if (over) raise_error(a.err, SD_EBIT_SEL);
+  if (hg.t == 0) {
+    if (total > a.sel_stride) raise_error(a.err, SD_EBIT_SEL);
     a.sel_count[row] = (int32_t)std::min<long long>(total, a.sel_stride);
   }
 }
 
-// Block-wide: every position 0 .. N - 1 (a head that keeps all its tokens).
-__device__ void write_all(const SelectArgs &a, long long N, int32_t *out, long long row) {
-  for (long long t = threadIdx.x; t < N; t += kT2) {
+// Group-wide: every position 0 .. N - 1 (a head that keeps all its tokens);
+// with `bitmap`, also every bit of [0, N) (for the union).
+__device__ void write_all(const SelectArgs &a, const HeadGroup &hg, long long N, int32_t *out, long long row,
+                          uint32_t *bitmap) {
+  for (long long t = hg.t; t < N; t += kT2) {
     if (t < a.sel_stride) out[t] = (int32_t)t;
     else raise_error(a.err, SD_EBIT_SEL);
   }
-  if (threadIdx.x == 0) a.sel_count[row] = (int32_t)std::min(N, a.sel_stride);
+  if (bitmap)
+    for (long long x = hg.t; x < (N + 31) / 32; x += kT2)
+      bitmap[x] = (x + 1) * 32 <= N ? 0xFFFFFFFFu : ((1u << (N & 31)) - 1u);
+  if (hg.t == 0) a.sel_count[row] = (int32_t)std::min(N, a.sel_stride);
 }
 
 // K2 flags the work item of a row whose window missed (once per item).
@@ -899,16 +926,16 @@ __device__ void flag_item(const StreamWs &ws, long long row) {
   if (atomicExch(&ws.fail[it], 1u) == 0u) ws.fail[ws.items + 1 + atomicAdd(&ws.fail[ws.items], 1u)] = (uint32_t)it;
 }
 
-// Block-wide: the highest bin c of hist[0, kBinsK) whose suffix count reaches
-// need (need >= 1).  Thread t holds bins [8 t, 8 t + 8); a block-wide suffix
+// Group-wide: the highest bin c of hist[0, kBinsK) whose suffix count reaches
+// need (need >= 1).  Thread t holds bins [8 t, 8 t + 8); a group-wide suffix
 // sum over the threads' totals finds the thread holding the cut, which scans
 // its own bins.  Writes c, the count strictly above it and hist[c] to res
 // (res[0] = -1 when the bins together hold fewer than need).  wsum: kT2 / 32
 // words of shared memory.
-__device__ void block_cut_bin(const uint32_t *hist, long long need, uint32_t *wsum, int *res) {
+__device__ void block_cut_bin(const HeadGroup &hg, const uint32_t *hist, long long need, uint32_t *wsum, int *res) {
   constexpr int PT = kBinsK / kT2;
   static_assert(PT == 8, "two 16-byte loads per thread");
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = hg.t, lane = tid & 31, warp = tid >> 5;
   const uint4 h0 = reinterpret_cast<const uint4 *>(hist)[2 * tid];
   const uint4 h1 = reinterpret_cast<const uint4 *>(hist)[2 * tid + 1];
   const uint32_t v[PT] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
@@ -922,7 +949,7 @@ __device__ void block_cut_bin(const uint32_t *hist, long long need, uint32_t *ws
     if (lane + o < 32) suf += y;
   }
   if (lane == 0) wsum[warp] = suf;
-  __syncthreads();
+  hg.sync();
   long long above = 0;
 #pragma unroll
   for (int w = 0; w < kT2 / 32; ++w) above += w > warp ? wsum[w] : 0u;
@@ -941,30 +968,32 @@ __device__ void block_cut_bin(const uint32_t *hist, long long need, uint32_t *ws
   }
 }
 
-// top-k K2: one CTA per (sequence, retrieval head).  The head's buffered
+// Shared memory of one top-k head group (besides its bitmap).
+struct TopkSmem {
+  unsigned long long cand[kCap];
+  __align__(16) uint32_t hist[kBinsK + 4];
+  uint32_t n_cand;
+  int res[3];
+  int fail, done;
+  long long need;
+  int cutv[kLevels];
+  float llo[kLevels], linv[kLevels];
+  uint32_t wtot[kT2 / 32];
+};
+
+// top-k K2 of one (sequence b, retrieval head row hr).  The head's buffered
 // entries (every score >= t_lo) are histogrammed over kBinsK bins of
 // [t_lo, t_hi) plus one bin for scores >= t_hi; the bin holding the k-th
 // score is split again while it holds more than kRefine tokens (kLevels
 // levels at most); entries above the cut path are selected, the cut bin's are
-// ranked exactly by (score desc, position asc).
-__global__ void __launch_bounds__(kT2, 4)
-topk_resolve_kernel(const SelectArgs a, const Shape sh, const StreamWs ws) {
-  extern __shared__ __align__(16) uint32_t bitmap[];  // [max_len / 32], rounded up to 16 bytes
-  __shared__ unsigned long long cand[kCap];
-  __shared__ __align__(16) uint32_t hist[kBinsK + 1];
-  __shared__ uint32_t n_cand;
-  __shared__ int res[3];
-  __shared__ int fail_s, done_s;
-  __shared__ long long need_s;
-  __shared__ int cutv[kLevels];
-  __shared__ float llo[kLevels], linv[kLevels];
-  __shared__ uint32_t wtot[kT2 / 32];
-  const int tid = threadIdx.x, lane = tid & 31;
-  const int b = blockIdx.y, hr = blockIdx.x;
+// ranked exactly by (score desc, position asc).  Leaves the set in `bitmap`
+// (bits of [0, N)) and writes it out; false when the window missed (the item
+// is flagged for the exact selector and nothing is written).
+__device__ bool resolve_topk(const SelectArgs &a, const Shape &sh, const StreamWs &ws, int b, int hr,
+                             const HeadGroup &hg, TopkSmem &S, uint32_t *bitmap, bool union_bits) {
+  const int tid = hg.t, lane = tid & 31;
   const long long row = (long long)b * sh.H_ret + hr;
   int32_t *out = a.sel_idx + row * a.sel_stride;
-  pdl_wait();
-  pdl_trigger();
   // one round of independent loads: the length, the window, the buffer count
   // and the first kPer2 * kT2 buffer slots (inside the row: reads stop at cap)
   long long N = a.seq_lens[b];
@@ -980,73 +1009,73 @@ topk_resolve_kernel(const SelectArgs a, const Shape sh, const StreamWs ws) {
   N = N < 0 ? 0 : std::min<long long>(N, sh.max_len);
   const long long kb = topk_budget(a, N);
   if (N == 0 || kb >= N) {
-    write_all(a, N, out, row);
-    return;
+    write_all(a, hg, N, out, row, union_bits ? bitmap : nullptr);
+    return true;
   }
   const int n = (int)std::min<uint32_t>(nbuf, (uint32_t)ws.cap);
   const int words = (int)((N + 31) / 32);
   for (int o = tid; o < (words + 3) / 4; o += kT2) reinterpret_cast<uint4 *>(bitmap)[o] = make_uint4(0u, 0u, 0u, 0u);
   if (tid == 0) {
-    llo[0] = w.x;
-    linv[0] = w.z;
-    need_s = kb;
-    fail_s = nbuf > (uint32_t)ws.cap;
-    done_s = 0;
-    n_cand = 0u;
+    S.llo[0] = w.x;
+    S.linv[0] = w.z;
+    S.need = kb;
+    S.fail = nbuf > (uint32_t)ws.cap;
+    S.done = 0;
+    S.n_cand = 0u;
   }
   // bin of a score at level L: level 0 is the window histogram (bin kBinsK:
   // scores >= t_hi); level L > 0 splits the cut bin of level L - 1 into kBinsK
   // linear sub-bins.  Bins are non-decreasing in the score at every level.
   auto bin_at = [&](float v, int L) -> int {
     if (L == 0) return window_bin<kBinsK>(v, w.x, w.y, w.z);
-    return min(kBinsK - 1, max(0, __float2int_rz((v - llo[L]) * linv[L])));
+    return min(kBinsK - 1, max(0, __float2int_rz((v - S.llo[L]) * S.linv[L])));
   };
   // the entries past the registers are read from the buffer (L2) at each pass
   const int rest0 = kPer2 * kT2;
   // the cut bin: refine while it holds more than kRefine tokens
   int L = 0;
   for (; L < kLevels; ++L) {
-    for (int o = tid; o <= kBinsK; o += kT2) hist[o] = 0u;
-    __syncthreads();
-    if (fail_s) break;
+    for (int o = tid; o <= kBinsK; o += kT2) S.hist[o] = 0u;
+    hg.sync();
+    if (S.fail) break;
     auto add = [&](unsigned long long en) {
       const float v = key_to_float((uint32_t)(en >> 32));
       bool play = true;
-      for (int l = 0; l < L; ++l) play = play && bin_at(v, l) == cutv[l];
-      if (play) atomicAdd(&hist[bin_at(v, L)], 1u);
+      for (int l = 0; l < L; ++l) play = play && bin_at(v, l) == S.cutv[l];
+      if (play) atomicAdd(&S.hist[bin_at(v, L)], 1u);
     };
 #pragma unroll
     for (int j = 0; j < kPer2; ++j)
       if (tid + j * kT2 < n) add(ent[j]);
     for (int e = rest0 + tid; e < n; e += kT2) add(__ldcg(buf + e));
-    if (tid == 0) res[0] = -1;
-    __syncthreads();
-    const long long need = need_s - (L == 0 ? (long long)hist[kBinsK] : 0LL);
-    if (need > 0) block_cut_bin(hist, need, wtot, res);
-    __syncthreads();
+    if (tid == 0) S.res[0] = -1;
+    hg.sync();
+    const long long need = S.need - (L == 0 ? (long long)S.hist[kBinsK] : 0LL);
+    if (need > 0) block_cut_bin(hg, S.hist, need, S.wtot, S.res);
+    hg.sync();
     if (tid == 0) {
-      const int cut = res[0];
+      const int cut = S.res[0];
       if (need <= 0 || cut < 0) {
-        fail_s = 1;
+        S.fail = 1;
       } else {
-        const uint32_t ncut = (uint32_t)res[2];
-        cutv[L] = cut;
-        need_s = need - res[1];                        // tokens still to take from the cut bin
+        const uint32_t ncut = (uint32_t)S.res[2];
+        S.cutv[L] = cut;
+        S.need = need - S.res[1];                      // tokens still to take from the cut bin
         const bool last = ncut <= (uint32_t)kRefine || L + 1 == kLevels;
-        if (last && ncut > (uint32_t)kCap) fail_s = 1;
+        if (last && ncut > (uint32_t)kCap) S.fail = 1;
         if (!last) {
-          llo[L + 1] = llo[L] + (float)cut / linv[L];
-          linv[L + 1] = linv[L] * (float)kBinsK;
+          S.llo[L + 1] = S.llo[L] + (float)cut / S.linv[L];
+          S.linv[L + 1] = S.linv[L] * (float)kBinsK;
         }
-        done_s = last;
+        S.done = last;
       }
     }
-    __syncthreads();
-    if (fail_s || done_s) break;
+    hg.sync();
+    if (S.fail || S.done) break;
   }
-  if (fail_s) {
+  if (S.fail) {
     if (tid == 0) flag_item(ws, row);
-    return;
+    return false;
   }
   const int nlev = L + 1;
   // classify: above the cut path -> selected; on it -> candidate.  Every lane
@@ -1058,7 +1087,7 @@ topk_resolve_kernel(const SelectArgs a, const Shape sh, const StreamWs ws) {
     int rel = 0;
     for (int l = 0; l < nlev && rel == 0; ++l) {
       const int bl = bin_at(v, l);
-      rel = bl > cutv[l] ? 1 : (bl < cutv[l] ? -1 : 0);
+      rel = bl > S.cutv[l] ? 1 : (bl < S.cutv[l] ? -1 : 0);
     }
     if (valid && rel > 0) atomicOr(&bitmap[pos >> 5], 1u << (pos & 31));
     const bool isc = valid && rel == 0;
@@ -1066,10 +1095,10 @@ topk_resolve_kernel(const SelectArgs a, const Shape sh, const StreamWs ws) {
     if (m) {
       const int leader = __ffs(m) - 1;
       uint32_t base = 0;
-      if (lane == leader) base = atomicAdd(&n_cand, (uint32_t)__popc(m));
+      if (lane == leader) base = atomicAdd(&S.n_cand, (uint32_t)__popc(m));
       base = __shfl_sync(kFull, base, leader);
       const uint32_t at = base + __popc(m & ((1u << lane) - 1u));
-      if (isc && at < (uint32_t)kCap) cand[at] = ((unsigned long long)(~key) << 32) | pos;   // ascending = better first
+      if (isc && at < (uint32_t)kCap) S.cand[at] = ((unsigned long long)(~key) << 32) | pos;   // ascending = better first
     }
   };
 #pragma unroll
@@ -1078,21 +1107,22 @@ topk_resolve_kernel(const SelectArgs a, const Shape sh, const StreamWs ws) {
     const int e = e0 + tid;
     classify(e < n ? __ldcg(buf + e) : 0ull, e < n);
   }
-  __syncthreads();
+  hg.sync();
   // rank the cut bin exactly: the need_c best by (score desc, position asc)
-  const int nc = (int)std::min<uint32_t>(n_cand, (uint32_t)kCap);
-  const long long need_c = need_s;
+  const int nc = (int)std::min<uint32_t>(S.n_cand, (uint32_t)kCap);
+  const long long need_c = S.need;
   for (int e = tid; e < nc; e += kT2) {
-    const unsigned long long me = cand[e];
+    const unsigned long long me = S.cand[e];
     int rk = 0;
-    for (int j = 0; j < nc; ++j) rk += cand[j] < me;
+    for (int j = 0; j < nc; ++j) rk += S.cand[j] < me;
     if (rk < need_c) {
       const uint32_t pos = (uint32_t)me;
       atomicOr(&bitmap[pos >> 5], 1u << (pos & 31));
     }
   }
-  __syncthreads();
-  write_ascending(a, bitmap, words, out, row, wtot);
+  hg.sync();
+  write_ascending(a, hg, bitmap, words, out, row, S.wtot);
+  return true;
 }
 
 // One warp, over kBins radix digits with counts and float64 masses: the
@@ -1133,45 +1163,49 @@ __device__ int warp_cut_digit(const uint32_t *cnt, const double *mass, double ne
   return grp * G + j;
 }
 
-// top-p K2: one CTA per (sequence, retrieval head).
-__global__ void __launch_bounds__(kT2, 4)
-topp_resolve_kernel(const SelectArgs a, const Shape sh, const StreamWs ws) {
-  extern __shared__ uint32_t bitmap[];               // [max_len / 32]
-  __shared__ unsigned long long cand[kCapP];
-  __shared__ uint32_t dcnt[kBins];
-  __shared__ double dmass[kBins];
-  __shared__ int fail_s;
-  __shared__ double need_s;
-  __shared__ uint32_t kmin_s, kmax_s, prefix_s;
-  __shared__ uint32_t wtot[kT2 / 32];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int b = blockIdx.y, hr = blockIdx.x;
+// Shared memory of one top-p head group (besides its bitmap).
+struct ToppSmem {
+  unsigned long long cand[kCapP];
+  uint32_t dcnt[kBins];
+  double dmass[kBins];
+  int fail;
+  double need;
+  uint32_t kmin, kmax, prefix;
+  uint32_t wtot[kT2 / 32];
+};
+
+// top-p K2 of one (sequence b, retrieval head row hr): the tokens above the
+// cut bin (the cut pass's bitmap) plus the cut bin's candidates at or above
+// the exact threshold, found by a radix search over their order keys with
+// float64 mass per digit.  As resolve_topk for the bitmap, the output and a
+// miss.
+__device__ bool resolve_topp(const SelectArgs &a, const Shape &sh, const StreamWs &ws, int b, int hr,
+                             const HeadGroup &hg, ToppSmem &S, uint32_t *bitmap, bool union_bits) {
+  const int tid = hg.t, lane = tid & 31, warp = tid >> 5;
   const long long row = (long long)b * sh.H_ret + hr;
   int32_t *out = a.sel_idx + row * a.sel_stride;
-  pdl_wait();
-  pdl_trigger();
   long long N = a.seq_lens[b];
   N = N < 0 ? 0 : std::min<long long>(N, sh.max_len);
   if (keeps_all<true>(a, N)) {
-    write_all(a, N, out, row);
-    return;
+    write_all(a, hg, N, out, row, union_bits ? bitmap : nullptr);
+    return true;
   }
   const float thi = ws.win[row].y;
   if (warp == 0) {
     double above, need;
     const int c = warp_cut_mass(ws.hist + row * (kBinsP + 1), ws.zlo[row], (double)a.top_p, lane, &above, &need);
     if (lane == 0) {
-      fail_s = c < 0 || ws.rflag[row] != 0u || ws.bcount[row] > (uint32_t)ws.cap;
-      need_s = need - above;                         // mass still to take from the cut bin
-      kmin_s = 0xFFFFFFFFu;
-      kmax_s = 0u;
-      prefix_s = 0u;
+      S.fail = c < 0 || ws.rflag[row] != 0u || ws.bcount[row] > (uint32_t)ws.cap;
+      S.need = need - above;                           // mass still to take from the cut bin
+      S.kmin = 0xFFFFFFFFu;
+      S.kmax = 0u;
+      S.prefix = 0u;
     }
   }
-  __syncthreads();
-  if (fail_s) {
+  hg.sync();
+  if (S.fail) {
     if (tid == 0) flag_item(ws, row);
-    return;
+    return false;
   }
   // the bitmap of the tokens above the cut bin, and the cut bin's candidates
   const int words = (int)((N + 31) / 32);
@@ -1182,62 +1216,190 @@ topp_resolve_kernel(const SelectArgs a, const Shape sh, const StreamWs ws) {
   uint32_t lo = 0xFFFFFFFFu, hi = 0u;
   for (int e = tid; e < n; e += kT2) {
     const unsigned long long v = buf[e];
-    cand[e] = v;
+    S.cand[e] = v;
     lo = min(lo, (uint32_t)(v >> 32));
     hi = max(hi, (uint32_t)(v >> 32));
   }
   if (lo != 0xFFFFFFFFu) {
-    atomicMin(&kmin_s, lo);
-    atomicMax(&kmax_s, hi);
+    atomicMin(&S.kmin, lo);
+    atomicMax(&S.kmax, hi);
   }
-  __syncthreads();
+  hg.sync();
   if (n > 0) {
     // exact radix search over the order keys' offsets from the smallest:
     // the largest key whose suffix mass reaches need (9 bits per level)
-    const uint32_t kmin = kmin_s, span = kmax_s - kmin;
+    const uint32_t kmin = S.kmin, span = S.kmax - kmin;
     int rem = span ? 32 - __clz(span) : 0;           // offset bits not yet decided
     const int top = rem;
     uint32_t prefix = 0u;
-    double need = need_s;
+    double need = S.need;
     while (rem > 0) {
       const int sh2 = rem > 9 ? rem - 9 : 0;
       for (int o = tid; o < kBins; o += kT2) {
-        dcnt[o] = 0u;
-        dmass[o] = 0.0;
+        S.dcnt[o] = 0u;
+        S.dmass[o] = 0.0;
       }
-      __syncthreads();
+      hg.sync();
       for (int e = tid; e < n; e += kT2) {
-        const uint32_t key = (uint32_t)(cand[e] >> 32), off = key - kmin;
+        const uint32_t key = (uint32_t)(S.cand[e] >> 32), off = key - kmin;
         if (rem != top && (off >> rem) != prefix) continue;
         const uint32_t d = (off >> sh2) & ((1u << (rem - sh2)) - 1u);
-        atomicAdd(&dcnt[d], 1u);
-        atomicAdd(&dmass[d], (double)exp2f((key_to_float(key) - thi) * kLog2e));
+        atomicAdd(&S.dcnt[d], 1u);
+        atomicAdd(&S.dmass[d], (double)exp2f((key_to_float(key) - thi) * kLog2e));
       }
-      __syncthreads();
+      hg.sync();
       if (warp == 0) {
         double above;
-        const int d = warp_cut_digit(dcnt, dmass, need, lane, &above);
+        const int d = warp_cut_digit(S.dcnt, S.dmass, need, lane, &above);
         if (lane == 0) {
-          need_s = need - above;
-          prefix_s = (prefix << (rem - sh2)) | (uint32_t)d;
+          S.need = need - above;
+          S.prefix = (prefix << (rem - sh2)) | (uint32_t)d;
         }
       }
-      __syncthreads();
-      need = need_s;
-      prefix = prefix_s;
+      hg.sync();
+      need = S.need;
+      prefix = S.prefix;
       rem = sh2;
     }
     const uint32_t tau = kmin + prefix;              // the threshold's key: every candidate >= it is kept
     for (int e = tid; e < n; e += kT2) {
-      const unsigned long long v = cand[e];
+      const unsigned long long v = S.cand[e];
       if ((uint32_t)(v >> 32) >= tau) {
         const uint32_t pos = (uint32_t)v;
         atomicOr(&bitmap[pos >> 5], 1u << (pos & 31));
       }
     }
   }
+  hg.sync();
+  write_ascending(a, hg, bitmap, words, out, row, S.wtot);
+  return true;
+}
+
+// Per-head K2: one CTA per (sequence, retrieval head).  dynamic shared
+// memory: the head's bitmap of the context [max_len / 32 words, rounded up to
+// 16 bytes].
+__global__ void __launch_bounds__(kT2, 4)
+topk_resolve_kernel(const SelectArgs a, const Shape sh, const StreamWs ws) {
+  extern __shared__ __align__(16) uint32_t bitmap[];
+  __shared__ TopkSmem S;
+  pdl_wait();
+  pdl_trigger();
+  const HeadGroup hg{(int)threadIdx.x, 0, true};
+  resolve_topk(a, sh, ws, blockIdx.y, blockIdx.x, hg, S, bitmap, false);
+}
+
+__global__ void __launch_bounds__(kT2, 4)
+topp_resolve_kernel(const SelectArgs a, const Shape sh, const StreamWs ws) {
+  extern __shared__ __align__(16) uint32_t bitmap[];
+  __shared__ ToppSmem S;
+  pdl_wait();
+  pdl_trigger();
+  const HeadGroup hg{(int)threadIdx.x, 0, true};
+  resolve_topp(a, sh, ws, blockIdx.y, blockIdx.x, hg, S, bitmap, false);
+}
+
+// K2 of the decode step with the union: one CTA per (sequence, retrieval KV
+// group), one group of kT2 threads per retrieval head of the group (NG >= the
+// group's heads).  Each group resolves its head into a bitmap of the context
+// and writes the head's list; then the whole CTA walks the heads' bitmaps span
+// by span (the spans of attend's plan) and writes the group's union list
+// there: (cache row, head mask) in ascending position order, and its length.
+// An item with a missed window is left to the exact selector and to attend's
+// plan.  dynamic shared memory: [NG bitmaps of bm_bytes][NG head smem].
+template <bool TOPP, int NG>
+__global__ void __launch_bounds__(NG * kT2, 1)
+resolve_union_kernel(const SelectArgs a, const Shape sh, const StreamWs ws, const Group *__restrict__ groups,
+                     int n_groups, const UnionOut uo, int bm_bytes) {
+  using Smem = typename std::conditional<TOPP, ToppSmem, TopkSmem>::type;
+  constexpr int NWC = NG * kT2 / 32;                 // warps of the CTA
+  extern __shared__ __align__(16) unsigned char dynu[];
+  __shared__ Group grp;
+  __shared__ int any_fail;
+  __shared__ uint32_t ctot[NWC];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int item = blockIdx.x;
+  const int b = item / n_groups, gi = item % n_groups;
+  if (tid == 0) {
+    grp = groups[gi];
+    any_fail = 0;
+  }
+  pdl_wait();
+  pdl_trigger();
   __syncthreads();
-  write_ascending(a, bitmap, words, out, row, wtot);
+  const int nr = grp.n, g = grp.kv_head;
+  const int k = tid / kT2;
+  const HeadGroup hg{tid % kT2, k, false};
+  auto bitmap_of = [&](int i) { return reinterpret_cast<uint32_t *>(dynu + (size_t)i * bm_bytes); };
+  Smem &S = *reinterpret_cast<Smem *>(dynu + (size_t)NG * bm_bytes + (size_t)k * sizeof(Smem));
+  if (k < nr) {
+    const bool ok = TOPP ? resolve_topp(a, sh, ws, b, grp.row[k], hg, reinterpret_cast<ToppSmem &>(S), bitmap_of(k), true)
+                         : resolve_topk(a, sh, ws, b, grp.row[k], hg, reinterpret_cast<TopkSmem &>(S), bitmap_of(k), true);
+    if (!ok && hg.t == 0) any_fail = 1;
+  }
+  __syncthreads();
+  if (any_fail) return;                              // planned by attend after the exact selector
+
+  // ---- the group's union list, span by span ------------------------------------
+  long long N = a.seq_lens[b];
+  N = N < 0 ? 0 : std::min<long long>(N, sh.max_len);
+  const int words = (int)((N + 31) / 32);
+  const int span_words = uo.span / 32;
+  const int ns_item = (int)((N + uo.span - 1) / uo.span);
+  const uint32_t row_g = (uint32_t)g * kPage;        // row of (page, g, slot) = (page * Hkv + g) * 16 + slot
+  const uint32_t row_page = (uint32_t)sh.Hkv * kPage;
+  const int32_t *pt = a.page_table + (long long)b * sh.max_pages;
+  bool bad_page = false;
+  for (int sp = 0; sp < ns_item; ++sp) {
+    const int x_lo = sp * span_words, x_hi = std::min(words, x_lo + span_words);
+    const int steps = (x_hi - x_lo + NWC * 32 - 1) / (NWC * 32);
+    const int w0 = x_lo + warp * steps * 32;
+    uint32_t c = 0;
+    for (int r = 0; r < steps; ++r) {
+      const int x = w0 + r * 32 + lane;
+      uint32_t u = 0;
+#pragma unroll
+      for (int i = 0; i < NG; ++i) u |= (x < x_hi && i < nr) ? bitmap_of(i)[x] : 0u;
+      c += __popc(u);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(kFull, c, o);
+    if (lane == 0) ctot[warp] = c;
+    __syncthreads();
+    uint32_t off = 0, total = 0;
+    for (int x = 0; x < NWC; ++x) {
+      off += x < warp ? ctot[x] : 0u;
+      total += ctot[x];
+    }
+    const long long slot = ((long long)b * n_groups + gi) * uo.ns + sp;   // attend's plan slot
+    uint32_t *rows = uo.row + slot * uo.span;
+    uint16_t *masks = uo.mask + slot * uo.span;
+    for (int r = 0; r < steps; ++r) {
+      const int xb = w0 + r * 32;
+      const int x = xb + lane;
+      uint32_t hw[NG];
+      uint32_t u = 0;
+#pragma unroll
+      for (int i = 0; i < NG; ++i) {
+        hw[i] = (x < x_hi && i < nr) ? bitmap_of(i)[x] : 0u;
+        u |= hw[i];
+      }
+      off += (uint32_t)warp_emit_bits(u, lane, [&](bool valid, int kk, int w, int bit) {
+        uint32_t m = 0;
+#pragma unroll
+        for (int i = 0; i < NG; ++i) m |= ((__shfl_sync(kFull, hw[i], w) >> bit) & 1u) << i;   // every lane
+        if (!valid) return;
+        const int pos = (xb + w) * 32 + bit;
+        const int page = pt[pos >> 4];
+        const bool ok = page >= 0 && page < sh.num_pages;
+        bad_page |= !ok;
+        rows[off + kk] = ok ? (uint32_t)page * row_page + row_g + (uint32_t)(pos & (kPage - 1)) : 0u;
+        masks[off + kk] = (uint16_t)(ok ? m : 0u);
+      });
+    }
+    if (tid == 0) uo.cnt[slot] = (int)total;
+    __syncthreads();                                 // ctot is reused by the next span
+  }
+  if (bad_page) raise_error(a.err, SD_EBIT_PAGE);
 }
 
 // ------------------------------------------------------------------- host
@@ -1299,39 +1461,71 @@ cudaError_t set_smem_once(K kern, size_t bytes) {
   return e;
 }
 
+// The last pass: the per-head resolve, or, with `uo`, at most four retrieval
+// heads per group whose bitmaps and scratch fit in one CTA, and enough items
+// to fill half the multiprocessors, the resolve with the group's union list
+// (*unioned).
+template <bool TOPP, int GR>
+cudaError_t launch_resolve(const SelectArgs &a, const Shape &sh, const Tables &tb, const StreamWs &ws,
+                           size_t bitmap_bytes, const UnionOut *uo, bool *unioned, cudaStream_t st) {
+  using Smem = typename std::conditional<TOPP, ToppSmem, TopkSmem>::type;
+  auto *per_head = TOPP ? topp_resolve_kernel : topk_resolve_kernel;
+  constexpr int NG = GR <= 4 ? GR : 4;
+  const size_t ubytes = (size_t)NG * (bitmap_bytes + sizeof(Smem));
+  if (unioned) *unioned = false;
+  // one CTA per item: worth it when the items fill at least half the GPU
+  // (fewer, and the per-head CTAs' parallelism wins)
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
+      sms = n;
+  }
+  if (uo && GR <= 4 && ubytes <= 227 * 1024 && 2 * a.batch * tb.n_ret >= std::max(sms, 1)) {
+    auto *kern = resolve_union_kernel<TOPP, NG>;
+    cudaError_t e = set_smem_once(kern, ubytes);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(kern, dim3(a.batch * tb.n_ret), dim3(NG * kT2), ubytes, st, 0, a, sh, ws, tb.ret, tb.n_ret, *uo,
+                   (int)bitmap_bytes);
+    if (e == cudaSuccess && unioned) *unioned = true;
+    return e;
+  }
+  cudaError_t e = set_smem_once(per_head, bitmap_bytes);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(per_head, dim3(sh.H_ret, a.batch), dim3(kT2), bitmap_bytes, st, 0, a, sh, ws);
+}
+
 template <int GR>
 cudaError_t stream_launch(const SelectArgs &a, const Shape &sh, const Tables &tb, const StreamWs &ws,
-                          size_t bitmap_bytes, cudaStream_t st) {
+                          size_t bitmap_bytes, const UnionOut *uo, bool *unioned, cudaStream_t st) {
   const bool topp = a.mode == SD_TOP_P;
   const int items = a.batch * tb.n_ret;
   const int chunks = (int)((sh.max_pages + kChunkPages - 1) / kChunkPages);
-  const dim3 g1(items, chunks), g2(sh.H_ret, a.batch);
+  const dim3 g1(items, chunks);
   const size_t smem0 = (size_t)GR * sample_pages(GR) * 16 * 4 + (size_t)GR * kSampleBins * 4 * (topp ? 2 : 1);
   cudaError_t e;
   if (!topp) {
     const size_t smem1 = stream_smem_bytes(GR, kStageTopk);
     e = set_smem_once(window_kernel<GR, false>, smem0);
     if (e == cudaSuccess) e = set_smem_once(stream_kernel<GR, kStageTopk>, smem1);
-    if (e == cudaSuccess) e = set_smem_once(topk_resolve_kernel, bitmap_bytes);
     if (e != cudaSuccess) return e;
     e = launch_pdl(window_kernel<GR, false>, dim3(items), dim3(kT0), smem0, st, 0, a, sh, tb.ret, tb.n_ret, ws);
     if (e == cudaSuccess)
       e = launch_pdl(stream_kernel<GR, kStageTopk>, g1, dim3(kT1), smem1, st, 0, a, sh, tb.ret, tb.n_ret, ws);
-    if (e == cudaSuccess) e = launch_pdl(topk_resolve_kernel, g2, dim3(kT2), bitmap_bytes, st, 0, a, sh, ws);
+    if (e == cudaSuccess) e = launch_resolve<false, GR>(a, sh, tb, ws, bitmap_bytes, uo, unioned, st);
     return e;
   }
   const size_t smem_m = stream_smem_bytes(GR, kMassTopp), smem_c = stream_smem_bytes(GR, kCutTopp);
   e = set_smem_once(window_kernel<GR, true>, smem0);
   if (e == cudaSuccess) e = set_smem_once(stream_kernel<GR, kMassTopp>, smem_m);
   if (e == cudaSuccess) e = set_smem_once(stream_kernel<GR, kCutTopp>, smem_c);
-  if (e == cudaSuccess) e = set_smem_once(topp_resolve_kernel, bitmap_bytes);
   if (e != cudaSuccess) return e;
   e = launch_pdl(window_kernel<GR, true>, dim3(items), dim3(kT0), smem0, st, 0, a, sh, tb.ret, tb.n_ret, ws);
   if (e == cudaSuccess)
     e = launch_pdl(stream_kernel<GR, kMassTopp>, g1, dim3(kT1), smem_m, st, 0, a, sh, tb.ret, tb.n_ret, ws);
   if (e == cudaSuccess)
     e = launch_pdl(stream_kernel<GR, kCutTopp>, g1, dim3(kT1), smem_c, st, 0, a, sh, tb.ret, tb.n_ret, ws);
-  if (e == cudaSuccess) e = launch_pdl(topp_resolve_kernel, g2, dim3(kT2), bitmap_bytes, st, 0, a, sh, ws);
+  if (e == cudaSuccess) e = launch_resolve<true, GR>(a, sh, tb, ws, bitmap_bytes, uo, unioned, st);
   return e;
 }
 
@@ -1344,8 +1538,9 @@ size_t stream_workspace_bytes(const Shape &sh, const Tables &tb, int batch, int 
 }
 
 cudaError_t launch_select_stream(const SelectArgs &a, const Shape &sh, const Tables &tb, uint32_t *fail,
-                                 void *ws_base, cudaStream_t st, bool *used) {
+                                 void *ws_base, cudaStream_t st, bool *used, const UnionOut *uo, bool *unioned) {
   *used = false;
+  if (unioned) *unioned = false;
   const StreamPlan p = stream_plan(sh, tb, a.mode);
   if (!p.ok || ws_base == nullptr) return cudaSuccess;
   const StreamLayout L = stream_layout(sh, a.batch, p);
@@ -1370,11 +1565,11 @@ cudaError_t launch_select_stream(const SelectArgs &a, const Shape &sh, const Tab
   while (gr < tb.max_ret) gr <<= 1;
   cudaError_t e;
   switch (gr) {
-    case 1: e = stream_launch<1>(a, sh, tb, ws, p.bitmap_bytes, st); break;
-    case 2: e = stream_launch<2>(a, sh, tb, ws, p.bitmap_bytes, st); break;
-    case 4: e = stream_launch<4>(a, sh, tb, ws, p.bitmap_bytes, st); break;
-    case 8: e = stream_launch<8>(a, sh, tb, ws, p.bitmap_bytes, st); break;
-    default: e = stream_launch<16>(a, sh, tb, ws, p.bitmap_bytes, st); break;
+    case 1: e = stream_launch<1>(a, sh, tb, ws, p.bitmap_bytes, uo, unioned, st); break;
+    case 2: e = stream_launch<2>(a, sh, tb, ws, p.bitmap_bytes, uo, unioned, st); break;
+    case 4: e = stream_launch<4>(a, sh, tb, ws, p.bitmap_bytes, uo, unioned, st); break;
+    case 8: e = stream_launch<8>(a, sh, tb, ws, p.bitmap_bytes, uo, unioned, st); break;
+    default: e = stream_launch<16>(a, sh, tb, ws, p.bitmap_bytes, uo, unioned, st); break;
   }
   if (e == cudaSuccess) *used = true;
   return e;

@@ -60,13 +60,18 @@ class DecodeStep:
                        self.out, self.workspace, stream)
         return self.out
 
+    def select_attend(self, q_pre: torch.Tensor, q: torch.Tensor, stream=None) -> torch.Tensor:
+        """select then attend on the same sets, joined in one call."""
+        self.sd.select_attend(q_pre, q, self.index_cache, self.k_cache, self.v_cache, self.page_table,
+                              self.seq_lens, self.sel_idx, self.sel_count, self.out, self.workspace, stream)
+        return self.out
+
     def step(self, q_pre: torch.Tensor, q: torch.Tensor, new_keys: Optional[torch.Tensor] = None,
              new_slots: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-        """One decode step: index the appended tokens, select, attend."""
+        """One decode step: index the appended tokens, then select and attend."""
         if new_keys is not None:
             self.sd.index_keys(new_keys, new_slots, self.index_cache, stream)
-        self.select(q_pre, stream)
-        return self.attend(q, stream=stream)
+        return self.select_attend(q_pre, q, stream)
 
     def error_word(self, stream=None) -> int:
         return self.sd.error_word(stream)

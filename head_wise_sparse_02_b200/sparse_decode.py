@@ -54,6 +54,7 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sparse_decode_select": (c_int, [P, P, P, P, P, c_int, P, P, c_int, P, c_size_t, P]),
         "sparse_decode_select_exact": (c_int, [P, P, P, P, P, c_int, P, P, c_int, P, c_size_t, P]),
         "sparse_decode_attend": (c_int, [P, P, P, P, P, P, c_int, P, P, c_int, P, P, c_size_t, P]),
+        "sparse_decode_select_attend": (c_int, [P, P, P, P, P, P, P, P, c_int, P, P, c_int, P, P, c_size_t, P]),
         "sparse_decode_attend_noalloc": (c_int, [P, P, P, P, P, P, c_int, P, P, c_int, P, P]),
         "sparse_decode_error_word": (c_int, [P, P, POINTER(c_uint32)]),
         "sparse_decode_num_retrieval_heads": (c_int, [P]),
@@ -193,6 +194,21 @@ def sparse_decode_attend(ctx: int, q, k_cache, v_cache, page_table, seq_lens, se
         int(workspace.numel()), _stream(stream)), ctx)
 
 
+def sparse_decode_select_attend(ctx: int, q_pre, q, index_cache, k_cache, v_cache, page_table, seq_lens,
+                                sel_idx, sel_count, out, workspace, stream=None) -> None:
+    """select followed by attend on the same sets, in one call."""
+    _check_sets(ctx, sel_idx, sel_count, int(seq_lens.numel()))
+    stride = int(sel_idx.shape[-1]) if sel_idx is not None else 0
+    _check(LIB.sparse_decode_select_attend(
+        ctx, _ptr(q_pre, torch.bfloat16, "q_pre"), _ptr(q, torch.bfloat16, "q"),
+        _ptr(index_cache, torch.bfloat16, "index_cache"), _ptr(k_cache, torch.bfloat16, "k_cache"),
+        _ptr(v_cache, torch.bfloat16, "v_cache"), _ptr(page_table, torch.int32, "page_table"),
+        _ptr(seq_lens, torch.int32, "seq_lens"), int(seq_lens.numel()),
+        _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_count, torch.int32, "sel_count"), stride,
+        _ptr(out, torch.float32, "out"), _ptr(workspace, torch.uint8, "workspace"), int(workspace.numel()),
+        _stream(stream)), ctx)
+
+
 def sparse_decode_attend_noalloc(ctx: int, q, k_cache, v_cache, page_table, seq_lens, sel_idx, sel_count,
                                  out, stream=None) -> None:
     """attend on the library's built-in scratch (no workspace argument)."""
@@ -282,6 +298,11 @@ class SparseDecode:
                stream=None):
         sparse_decode_attend(self.handle, q, k_cache, v_cache, page_table, seq_lens, sel_idx, sel_count,
                              out, workspace, stream)
+
+    def select_attend(self, q_pre, q, index_cache, k_cache, v_cache, page_table, seq_lens, sel_idx, sel_count,
+                      out, workspace, stream=None):
+        sparse_decode_select_attend(self.handle, q_pre, q, index_cache, k_cache, v_cache, page_table, seq_lens,
+                                    sel_idx, sel_count, out, workspace, stream)
 
     def error_word(self, stream=None) -> int:
         return sparse_decode_error_word(self.handle, stream)

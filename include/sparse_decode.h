@@ -285,6 +285,27 @@ SD_API sd_status sparse_decode_attend(sd_ctx *ctx, const void *q, const void *k_
                                void *workspace, size_t ws_bytes, sd_stream stream);
 
 /*
+ * sparse_decode_select_attend -- sparse_decode_select followed by
+ * sparse_decode_attend on the same sets, in one call: the decode step of the
+ * layer (RTPurbo page, Methodology 1-3 and 5; ICS page, 3c).  The arguments
+ * are the union of theirs (q_pre and index_cache for the selection, q and the
+ * K/V caches for the attention; sel_idx / sel_count receive the sets as
+ * sparse_decode_select writes them); the results are identical to the two
+ * calls in a row.
+ *
+ * Joined, the last selection pass writes each (sequence, retrieval KV group)'s
+ * union of selected rows straight into the workspace instead of attend
+ * rebuilding it from sel_idx (when a group has at most four retrieval heads and
+ * their context bitmaps fit one CTA's shared memory; otherwise the two calls
+ * run as they are).  Errors as for the two calls.
+ */
+SD_API sd_status sparse_decode_select_attend(sd_ctx *ctx, const void *q_pre, const void *q,
+                                      const void *index_cache, const void *k_cache, const void *v_cache,
+                                      const int32_t *page_table, const int32_t *seq_lens, int batch,
+                                      int32_t *sel_idx, int32_t *sel_count, int sel_stride, float *out,
+                                      void *workspace, size_t ws_bytes, sd_stream stream);
+
+/*
  * sparse_decode_attend_noalloc -- sparse_decode_attend without a workspace
  * argument: the call uses a fixed scratch area compiled into the library
  * (64 MiB per device) and allocates nothing.  An addition of this library;

@@ -461,3 +461,92 @@ def test_exact_score_selection_full_size_128k():
     check_workload(w, seqs=[0, 15], heads=list(range(0, 32, 3)), label="exact topk_128k", score="exact")
     del w
     torch.cuda.empty_cache()
+
+
+# ------------------------------------------------------------------ joined select + attend
+
+# The joined call builds the union lists in the selection when the items
+# ((sequence, retrieval group) pairs) fill at least half the GPU: the cases
+# with 80 or more items take that path, the small ones the separate one.
+JOINED = [
+    ("tiny_ref", dict()),
+    ("tiny_ref", dict(N=1)),
+    ("tiny_ref", dict(N=67, permute=True, seed=5)),
+    ("llama3_8b_topp", dict(B=3, N=5000, permute=True, window=100, sinks=0)),
+    ("llama3_8b_topp", dict(B=40, N=3000, permute=True, window=100)),
+    ("topk_128k", dict(B=2, N=8192, permute=True)),
+    ("topk_128k", dict(B=10, N=8192, permute=True)),
+    ("topk_128k", dict(B=10, N=3001, top_k_frac=0.3)),
+    ("long_zipf", dict(N=20000, top_p=0.99, alpha=0.8, window=333)),
+    ("ragged_paged", dict(B=5, N_min=300, N_max=3000, window=200)),
+    ("ragged_paged", dict(B=40, N_min=1, N_max=4000, window=200)),
+]
+
+
+def _joined_vs_separate(w, label, oracle_seqs=None):
+    """The joined call against select then attend: identical sets and outputs
+    (both build the same union lists in the same order), and the outputs
+    against the oracle over the selected sets."""
+    st = make_step(w)
+    st.select(w.q_pre)
+    ref_out = st.attend(w.q).clone()
+    ref_idx, ref_cnt = st.sel_idx.clone(), st.sel_count.clone()
+    torch.cuda.synchronize()
+    assert st.error_word() == 0
+    st.sel_idx.fill_(-7)
+    st.sel_count.fill_(-7)
+    st.out.fill_(float("nan"))
+    out = st.select_attend(w.q_pre, w.q).clone()
+    torch.cuda.synchronize()
+    assert st.error_word() == 0
+    assert torch.equal(st.sel_count, ref_cnt), label
+    for b in range(w.batch):
+        for r in range(st.sel_count.shape[1]):
+            n = int(ref_cnt[b, r])
+            assert torch.equal(st.sel_idx[b, r, :n], ref_idx[b, r, :n]), f"{label} b={b} row={r}"
+    assert torch.equal(out, ref_out), f"{label}: joined and separate outputs differ"
+    seqs = list(range(w.batch)) if oracle_seqs is None else list(oracle_seqs)
+    retr = [(i, h) for i in range(len(seqs)) for h in range(w.num_q_heads) if w.head_is_retrieval[h]]
+    got = gpu_sets(st, w, [(seqs[i], h) for i, h in retr])
+    ref = O.decode_reference(oracle_config(w), **oracle_inputs(w, seqs),
+                             sets_override={(i, h): got[(seqs[i], h)] for i, h in retr})
+    for (i, h), o in ref.out.items():
+        assert_out_close(out[seqs[i], h].cpu().numpy(), o, f"{label} oracle b={seqs[i]} h={h}")
+    st.close()
+
+
+@pytest.mark.parametrize("name,kw", JOINED, ids=[f"{n}-{i}" for i, (n, _) in enumerate(JOINED)])
+def test_select_attend_joined(name, kw):
+    w = make_workload(name, "cuda", **kw)
+    _joined_vs_separate(w, f"joined {name}{kw}")
+
+
+@pytest.mark.parametrize("case", SHAPES, ids=[c[0] for c in SHAPES])
+def test_select_attend_joined_group_shapes(case):
+    """Group shapes where the joined call builds the union in the selection
+    (1, 2 and 4 retrieval heads per group) and where it falls back (8, 16)."""
+    from workloads.synthetic import _base, _gen, _plant_needles
+    name, lens, Hq, Hkv, d, retr, window, sinks, mode, kw = case
+    w = _base(name, 11, "cuda", lens, Hq, Hkv, d, retr, window, sinks, mode, permute=True, **kw)
+    if mode == "top_p":
+        _plant_needles(w, {b: [3] * sum(retr) for b in range(w.batch)}, _gen("cuda", 11, 6))
+    _joined_vs_separate(w, f"joined {name}")
+
+
+def test_select_attend_joined_with_exact_fallback():
+    """Planted keys on the sampled pages make the window miss for many groups
+    (the construction of test_topk_sample_overestimate_falls_back_to_exact):
+    those items are redone by the exact selector and planned by attend, the
+    others come with their union lists from the selection."""
+    w = make_workload("topk_128k", "cuda", B=10, N=32768)
+    for b in range(w.batch):
+        pos = [p * 16 + s for p in range(0, 2048, 8) for s in range(16)]
+        _set_keys(w, b, pos, _group_query_keys(w, b, len(pos), 2.0, 0.5, 100 + b))
+    _joined_vs_separate(w, "joined with fallback", oracle_seqs=[0, 5, 9])
+
+
+def test_select_attend_joined_full_size_128k():
+    w = make_workload("topk_128k", "cuda", B=10)
+    _joined_vs_separate(w, "joined topk_128k B=10", oracle_seqs=[0, 9])
+    del w
+    torch.cuda.empty_cache()
