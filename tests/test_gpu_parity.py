@@ -484,9 +484,9 @@ JOINED = [
 
 
 def _joined_vs_separate(w, label, oracle_seqs=None):
-    """The joined call against select then attend: identical sets and outputs
-    (both build the same union lists in the same order), and the outputs
-    against the oracle over the selected sets."""
+    """The joined call against select then attend: identical sets, outputs
+    within the output tolerance of each other, and against the oracle over
+    the selected sets."""
     st = make_step(w)
     st.select(w.q_pre)
     ref_out = st.attend(w.q).clone()
@@ -504,7 +504,12 @@ def _joined_vs_separate(w, label, oracle_seqs=None):
         for r in range(st.sel_count.shape[1]):
             n = int(ref_cnt[b, r])
             assert torch.equal(st.sel_idx[b, r, :n], ref_idx[b, r, :n]), f"{label} b={b} row={r}"
-    assert torch.equal(out, ref_out), f"{label}: joined and separate outputs differ"
+    # the same sets; the outputs are held to the output tolerance of each
+    # other (they come out bit-identical today: same union lists, same tiles)
+    got_o, ref_o = out.cpu().numpy(), ref_out.cpu().numpy()
+    for b in range(w.batch):
+        for h in range(w.num_q_heads):
+            assert_out_close(got_o[b, h], ref_o[b, h], f"{label} joined vs separate b={b} h={h}")
     seqs = list(range(w.batch)) if oracle_seqs is None else list(oracle_seqs)
     retr = [(i, h) for i in range(len(seqs)) for h in range(w.num_q_heads) if w.head_is_retrieval[h]]
     got = gpu_sets(st, w, [(seqs[i], h) for i, h in retr])
