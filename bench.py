@@ -186,17 +186,32 @@ def ncu_traffic(kernel: str, algorithmic_bytes: float):
         return None
 
 
-def kernels_per_step(w, score: str = "index") -> int:
+def kernels_per_step(w, score: str = "index", split: bool = False) -> int:
     """Kernels of this library one step launches: index_keys; select (top-k:
     window, stream, resolve; top-p: window, mass pass, cut pass, resolve;
     then the exact selector for flagged items; exact-score mode: the score
     kernel and the exact selector, no index_keys); attend (plan when there
-    are retrieval heads, item layout, main)."""
+    are retrieval heads, item layout, main); split layout: local_append of
+    the new tokens when there are local heads."""
     ret = any(w.head_is_retrieval)
+    loc = not all(w.head_is_retrieval)
     if score == "exact":
         return (2 if ret else 0) + (3 if ret else 2)
     n_sel = 0 if not ret else (4 if w.mode == "top_k" else 5)
-    return 1 + n_sel + (3 if ret else 2)
+    return 1 + (1 if split and loc else 0) + n_sel + (3 if ret else 2)
+
+
+def kv_cache_bytes(w) -> dict:
+    """K + V bytes the sequences of `w` occupy: every KV head keeps the whole
+    context (full layout), or only the retrieval groups do and each local
+    group keeps num_sinks + window rows (split layout)."""
+    G = w.num_q_heads // w.num_kv_heads
+    ret_groups = sum(1 for g in range(w.num_kv_heads) if any(w.head_is_retrieval[g * G:(g + 1) * G]))
+    loc_groups = sum(1 for g in range(w.num_kv_heads) if not all(w.head_is_retrieval[g * G:(g + 1) * G]))
+    row = 4 * w.head_dim
+    tokens = sum(w.seq_lens.cpu().tolist())
+    return {"full": tokens * w.num_kv_heads * row,
+            "split": tokens * ret_groups * row + w.batch * loc_groups * (w.num_sinks + w.window) * row}
 
 
 def union_rows(sel_idx, sel_count, w):
@@ -287,7 +302,8 @@ def workload_label(name: str, w) -> str:
 def bench_config(args, w, ws: int, flush: bool):
     """The `config` object of the JSON line; both arms print the same one."""
     return {
-        "workload": workload_label(args.workload, w) + (", exact-score selection" if args.score == "exact" else ""),
+        "workload": workload_label(args.workload, w) + (", exact-score selection" if args.score == "exact" else "")
+        + (", split KV layout (compacted local caches)" if getattr(args, "kv_layout", "full") == "split" else ""),
         "batch_per_gpu": w.batch, "seq_len": int(w.seq_lens.max()),
         "parallelism": f"replicas x{ws} (sequences sharded, no collective)",
         "l2": ("flushed between steps (512 MiB write, untimed)" if flush
@@ -397,10 +413,25 @@ def run_ours(args):
     stream = torch.cuda.current_stream()
 
     exact = args.score == "exact"
+    split = args.kv_layout == "split"
     # the decode step through the public API: index_keys for the appended
     # tokens, then the joined select + attend call (exact-score mode: the
-    # exact-score select, then attend; no index is kept)
-    calls = ("index_keys", "select", "attend") if exact else ("index_keys", "select_attend")
+    # exact-score select, then attend; no index is kept; split layout: the
+    # appended tokens also go to the compacted local caches, and the joined
+    # call reads the split caches)
+    if split:
+        st.make_split()                                   # setup, untimed
+        pos_new = (lens - 1).to(torch.int32)
+        seq_new = torch.arange(B, device=dev, dtype=torch.int32)
+        page_new = w.page_table[seq_new.long(), (lens - 1) // 16].long()
+        kn_new = w.k_cache[page_new, :, (lens - 1) % 16].contiguous()    # [B, Hkv, d] of the new tokens
+        vn_new = w.v_cache[page_new, :, (lens - 1) % 16].contiguous()
+    if exact:
+        calls = ("index_keys", "select", "attend")
+    elif split:
+        calls = ("index_keys", "local_append", "select_attend_split")
+    else:
+        calls = ("index_keys", "select_attend")
 
     def step(ev=None):
         """One decode step; with `ev`, an event pair around each call."""
@@ -414,6 +445,14 @@ def run_ours(args):
             if ev is not None:
                 e[2].record(stream)
             st.attend(w.q, stream=stream)
+        elif split:
+            st.sd.index_keys(new_keys, new_slots, st.index_cache, stream)
+            if ev is not None:
+                e[1].record(stream)
+            st.sd.local_append(kn_new, vn_new, seq_new, pos_new, st.local_k, st.local_v, stream)
+            if ev is not None:
+                e[2].record(stream)
+            st.select_attend_split(w.q_pre, w.q, stream)
         else:
             st.sd.index_keys(new_keys, new_slots, st.index_cache, stream)
             if ev is not None:
@@ -490,11 +529,22 @@ def run_ours(args):
     q_d, qp_d = torch.empty_like(w.q), torch.empty_like(w.q_pre)
     nk_d, ns_d = torch.empty_like(new_keys), torch.empty_like(new_slots)
 
+    if split:
+        kn_h, vn_h = kn_new.cpu().pin_memory(), vn_new.cpu().pin_memory()
+        kn_d, vn_d = torch.empty_like(kn_new), torch.empty_like(vn_new)
+
     def e2e_step():
         q_d.copy_(q_h, non_blocking=True)
         if exact:
             st.select_exact(q_d, stream)
             st.attend(q_d, stream=stream)
+        elif split:
+            qp_d.copy_(qp_h, non_blocking=True)
+            nk_d.copy_(nk_h, non_blocking=True); ns_d.copy_(ns_h, non_blocking=True)
+            kn_d.copy_(kn_h, non_blocking=True); vn_d.copy_(vn_h, non_blocking=True)
+            st.sd.index_keys(nk_d, ns_d, st.index_cache, stream)
+            st.sd.local_append(kn_d, vn_d, seq_new, pos_new, st.local_k, st.local_v, stream)
+            st.select_attend_split(qp_d, q_d, stream)
         else:
             qp_d.copy_(qp_h, non_blocking=True)
             nk_d.copy_(nk_h, non_blocking=True); ns_d.copy_(ns_h, non_blocking=True)
@@ -534,8 +584,16 @@ def run_ours(args):
     # ---- roofline of the dominant kernel ----
     index_bytes = score_row * index_tokens
     kv_bytes = row_bytes * rows
-    kern_bytes = ({"select": index_bytes, "attend": kv_bytes, "index_keys": 0} if exact else
-                  {"select_attend": index_bytes + kv_bytes, "index_keys": B * w.num_kv_heads * (2 * d + 32)})
+    if exact:
+        kern_bytes = {"select": index_bytes, "attend": kv_bytes, "index_keys": 0}
+    else:
+        kern_bytes = {"select_attend": index_bytes + kv_bytes, "index_keys": B * w.num_kv_heads * (2 * d + 32)}
+    if split:
+        n_loc = sum(1 for g in range(w.num_kv_heads)
+                    if not all(w.head_is_retrieval[g * (Hq // w.num_kv_heads):(g + 1) * (Hq // w.num_kv_heads)]))
+        kern_bytes["select_attend_split"] = kern_bytes.pop("select_attend")
+        kern_bytes["local_append"] = 2 * B * n_loc * 4 * d           # read and write K + V rows
+        step_bytes += kern_bytes["local_append"]
     dominant = max(per, key=per.get)
     peak, peak_kind = load_peak()
     achieved = kern_bytes[dominant] / (per[dominant] * 1e-3) / 1e9
@@ -563,9 +621,11 @@ def run_ours(args):
                      "traffic": ncu_traffic(dominant, kern_bytes[dominant])},
         "e2e": {"value": round(head_steps / (e2e_ms * 1e-3), 1), "unit": UNIT,
                 "h2d_bytes_per_step": int(q_h.numel() * 2 + (0 if exact else
-                                                             qp_h.numel() * 2 + nk_h.numel() * 2 + ns_h.numel() * 4)),
+                                                             qp_h.numel() * 2 + nk_h.numel() * 2 + ns_h.numel() * 4)
+                                          + (kn_h.numel() * 4 if split else 0)),
                 "d2h_bytes_per_step": int(out_h.numel() * 4)},
-        "gpu_launches": kernels_per_step(w, args.score) * args.steps,
+        "gpu_launches": kernels_per_step(w, args.score, split) * args.steps,
+        "kv_cache_bytes": dict(kv_cache_bytes(w), layout=args.kv_layout),
         "clocks": clk,
     }
     if rank == 0 and ws == 1 and not args.no_diagnostics:
@@ -708,6 +768,8 @@ def main(argv=None):
                     help="select by the r = 16 index (the method) or by the exact logits (reference selector)")
     ap.add_argument("--l2-flush", choices=["auto", "on", "off"], default="auto",
                     help="flush L2 between timed steps (auto: when a step touches < 8x the L2)")
+    ap.add_argument("--kv-layout", choices=["full", "split"], default="full",
+                    help="split: paged caches of the retrieval groups only, compacted local caches")
     ap.add_argument("--no-diagnostics", action="store_true")
     ap.add_argument("--diag-budget", type=float, default=20.0)
     args = ap.parse_args(argv)

@@ -75,6 +75,101 @@ long long max_topk(const sd_ctx *ctx) {
   return std::min(k, L);
 }
 
+// Rows per (sequence, local KV group) of a compacted local cache.
+long long local_rows(const sd_ctx *ctx) { return (long long)ctx->cfg.num_sinks + ctx->cfg.window; }
+
+// attend, alone (joined = false) or after the selection of the same sets
+// (joined = true), on the full paged caches (split = false) or on caches of the
+// retrieval groups plus compacted local caches (split = true)
+sd_status attend_impl(sd_ctx *ctx, const void *q_pre, const void *q, const void *index_cache, const void *k_cache,
+                      const void *v_cache, const void *local_k, const void *local_v, const int32_t *page_table,
+                      const int32_t *seq_lens, int batch, int32_t *sel_idx, int32_t *sel_count, int sel_stride,
+                      float *out, void *workspace, size_t ws_bytes, sd_stream stream, bool joined, bool split) {
+  if (!ctx) return SD_ERR_INVALID_ARG;
+  if (batch < 0 || batch > ctx->cfg.max_batch) return fail(ctx, SD_ERR_INVALID_ARG, "batch out of range");
+  if (batch == 0) return SD_OK;
+  const bool ret = ctx->sh.H_ret > 0;
+  if (!q || !page_table || !seq_lens || !out) return fail(ctx, SD_ERR_INVALID_ARG, "null pointer");
+  // with the split layout, caches of a kind of head that is absent may be NULL
+  const bool need_paged = !split || ret;
+  const bool need_local = split && ctx->tb.n_loc > 0 && local_rows(ctx) > 0;
+  if (need_paged && (!k_cache || !v_cache)) return fail(ctx, SD_ERR_INVALID_ARG, "null pointer");
+  if (need_local && (!local_k || !local_v)) return fail(ctx, SD_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || (need_paged && (!aligned16(k_cache) || !aligned16(v_cache))) ||
+      (need_local && (!aligned16(local_k) || !aligned16(local_v))))
+    return fail(ctx, SD_ERR_INVALID_ARG, "q and the K/V caches must be 16-byte aligned");
+  // local cache rows are addressed with 32-bit row numbers inside the kernels
+  if (need_local && (long long)batch * ctx->tb.n_loc * local_rows(ctx) >= 0xFFFFFFFFLL)
+    return fail(ctx, SD_ERR_UNSUPPORTED, "local caches too large for 32-bit row numbers");
+  if (ret) {
+    if (!sel_idx || !sel_count) return fail(ctx, SD_ERR_INVALID_ARG, "selection lists required for retrieval heads");
+    if (joined) {
+      if (!q_pre || !index_cache) return fail(ctx, SD_ERR_INVALID_ARG, "null pointer");
+      if (!aligned16(q_pre) || !aligned16(index_cache))
+        return fail(ctx, SD_ERR_INVALID_ARG, "q_pre and index_cache must be 16-byte aligned");
+      const long long need_stride = ctx->cfg.mode == SD_TOP_P ? ctx->sh.max_len : max_topk(ctx);
+      if (sel_stride < need_stride)
+        return fail(ctx, SD_ERR_INVALID_ARG, "sel_stride smaller than the largest possible set");
+    } else if (sel_stride <= 0) {
+      return fail(ctx, SD_ERR_INVALID_ARG, "selection lists required for retrieval heads");
+    }
+  }
+  const WsLayout w = layout(ctx, batch);
+  if (!workspace || ws_bytes < w.total) return fail(ctx, SD_ERR_WORKSPACE, "workspace too small");
+  DeviceGuard dg(ctx->device);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char *wsb = static_cast<char *>(workspace);
+  bool unioned = false;
+  if (joined && ret) {
+    sd::SelectArgs a{};
+    a.q_pre = static_cast<const uint16_t *>(q_pre);
+    a.index_cache = static_cast<const uint16_t *>(index_cache);
+    a.page_table = page_table;
+    a.seq_lens = seq_lens;
+    a.sel_idx = sel_idx;
+    a.sel_count = sel_count;
+    a.sel_stride = sel_stride;
+    a.proj = ctx->proj_d;
+    a.index_scale = ctx->index_scale;
+    a.mode = ctx->cfg.mode;
+    a.top_p = ctx->cfg.top_p;
+    a.top_k = ctx->cfg.top_k;
+    a.top_k_frac = ctx->cfg.top_k_frac;
+    a.score_ws = reinterpret_cast<float *>(wsb + w.scores_off);
+    a.flags = reinterpret_cast<uint32_t *>(wsb + w.flags_off);
+    a.stream_ws = w.stream_bytes ? wsb + w.stream_off : nullptr;
+    a.err = ctx->err_d;
+    a.batch = batch;
+    const sd::UnionOut uo = sd::attend_union_view(ctx->sh, ctx->tb, batch, wsb + w.att_off, split);
+    const cudaError_t e = sd::launch_select_union(a, ctx->sh, ctx->tb, uo, st, &unioned);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "select launch");
+  }
+  sd::AttendArgs at{};
+  at.q = static_cast<const uint16_t *>(q);
+  at.k_cache = static_cast<const uint16_t *>(k_cache);
+  at.v_cache = static_cast<const uint16_t *>(v_cache);
+  at.page_table = page_table;
+  at.seq_lens = seq_lens;
+  at.sel_idx = sel_idx;
+  at.sel_count = sel_count;
+  at.sel_stride = sel_stride;
+  at.out = out;
+  at.attn_scale = ctx->attn_scale;
+  at.window = ctx->cfg.window;
+  at.num_sinks = ctx->cfg.num_sinks;
+  at.ws = wsb + w.att_off;
+  at.err = ctx->err_d;
+  at.batch = batch;
+  at.split = split;
+  at.local_k = static_cast<const uint16_t *>(local_k);
+  at.local_v = static_cast<const uint16_t *>(local_v);
+  // with the union lists built by select, attend plans only the items the
+  // exact selector redid (listed in the miss array)
+  const uint32_t *only = unioned ? reinterpret_cast<const uint32_t *>(wsb + w.flags_off) : nullptr;
+  const cudaError_t e = sd::launch_attend(at, ctx->sh, ctx->tb, st, only);
+  return e == cudaSuccess ? SD_OK : cuda_fail(ctx, e, "attend launch");
+}
+
 }  // namespace
 
 extern "C" {
@@ -311,36 +406,9 @@ sd_status sparse_decode_attend(sd_ctx *ctx, const void *q, const void *k_cache, 
                                const int32_t *sel_idx, const int32_t *sel_count, int sel_stride, float *out,
                                void *workspace, size_t ws_bytes, sd_stream stream) {
   try {
-    if (!ctx) return SD_ERR_INVALID_ARG;
-    if (batch < 0 || batch > ctx->cfg.max_batch) return fail(ctx, SD_ERR_INVALID_ARG, "batch out of range");
-    if (batch == 0) return SD_OK;
-    if (!q || !k_cache || !v_cache || !page_table || !seq_lens || !out)
-      return fail(ctx, SD_ERR_INVALID_ARG, "null pointer");
-    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
-      return fail(ctx, SD_ERR_INVALID_ARG, "q, k_cache and v_cache must be 16-byte aligned");
-    if (ctx->sh.H_ret > 0 && (!sel_idx || !sel_count || sel_stride <= 0))
-      return fail(ctx, SD_ERR_INVALID_ARG, "selection lists required for retrieval heads");
-    const WsLayout w = layout(ctx, batch);
-    if (!workspace || ws_bytes < w.total) return fail(ctx, SD_ERR_WORKSPACE, "workspace too small");
-    DeviceGuard dg(ctx->device);
-    sd::AttendArgs a{};
-    a.q = static_cast<const uint16_t *>(q);
-    a.k_cache = static_cast<const uint16_t *>(k_cache);
-    a.v_cache = static_cast<const uint16_t *>(v_cache);
-    a.page_table = page_table;
-    a.seq_lens = seq_lens;
-    a.sel_idx = sel_idx;
-    a.sel_count = sel_count;
-    a.sel_stride = sel_stride;
-    a.out = out;
-    a.attn_scale = ctx->attn_scale;
-    a.window = ctx->cfg.window;
-    a.num_sinks = ctx->cfg.num_sinks;
-    a.ws = static_cast<char *>(workspace) + w.att_off;
-    a.err = ctx->err_d;
-    a.batch = batch;
-    cudaError_t e = sd::launch_attend(a, ctx->sh, ctx->tb, static_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? SD_OK : cuda_fail(ctx, e, "attend launch");
+    return attend_impl(ctx, nullptr, q, nullptr, k_cache, v_cache, nullptr, nullptr, page_table, seq_lens, batch,
+                       const_cast<int32_t *>(sel_idx), const_cast<int32_t *>(sel_count), sel_stride, out, workspace,
+                       ws_bytes, stream, false, false);
   } catch (...) {
     return SD_ERR_HOST_MEMORY;
   }
@@ -351,73 +419,62 @@ sd_status sparse_decode_select_attend(sd_ctx *ctx, const void *q_pre, const void
                                      const int32_t *seq_lens, int batch, int32_t *sel_idx, int32_t *sel_count,
                                      int sel_stride, float *out, void *workspace, size_t ws_bytes, sd_stream stream) {
   try {
+    return attend_impl(ctx, q_pre, q, index_cache, k_cache, v_cache, nullptr, nullptr, page_table, seq_lens, batch,
+                       sel_idx, sel_count, sel_stride, out, workspace, ws_bytes, stream, true, false);
+  } catch (...) {
+    return SD_ERR_HOST_MEMORY;
+  }
+}
+
+sd_status sparse_decode_attend_split(sd_ctx *ctx, const void *q, const void *k_ret, const void *v_ret,
+                                     const void *local_k, const void *local_v, const int32_t *page_table,
+                                     const int32_t *seq_lens, int batch, const int32_t *sel_idx,
+                                     const int32_t *sel_count, int sel_stride, float *out, void *workspace,
+                                     size_t ws_bytes, sd_stream stream) {
+  try {
+    return attend_impl(ctx, nullptr, q, nullptr, k_ret, v_ret, local_k, local_v, page_table, seq_lens, batch,
+                       const_cast<int32_t *>(sel_idx), const_cast<int32_t *>(sel_count), sel_stride, out, workspace,
+                       ws_bytes, stream, false, true);
+  } catch (...) {
+    return SD_ERR_HOST_MEMORY;
+  }
+}
+
+sd_status sparse_decode_select_attend_split(sd_ctx *ctx, const void *q_pre, const void *q, const void *index_cache,
+                                           const void *k_ret, const void *v_ret, const void *local_k,
+                                           const void *local_v, const int32_t *page_table, const int32_t *seq_lens,
+                                           int batch, int32_t *sel_idx, int32_t *sel_count, int sel_stride,
+                                           float *out, void *workspace, size_t ws_bytes, sd_stream stream) {
+  try {
+    return attend_impl(ctx, q_pre, q, index_cache, k_ret, v_ret, local_k, local_v, page_table, seq_lens, batch,
+                       sel_idx, sel_count, sel_stride, out, workspace, ws_bytes, stream, true, true);
+  } catch (...) {
+    return SD_ERR_HOST_MEMORY;
+  }
+}
+
+int sparse_decode_num_retrieval_groups(const sd_ctx *ctx) { return ctx ? ctx->tb.n_ret : 0; }
+
+int sparse_decode_num_local_groups(const sd_ctx *ctx) { return ctx ? ctx->tb.n_loc : 0; }
+
+sd_status sparse_decode_local_append(sd_ctx *ctx, const void *k_new, const void *v_new, const int32_t *seq_ids,
+                                     const int32_t *positions, int num_tokens, void *local_k, void *local_v,
+                                     sd_stream stream) {
+  try {
     if (!ctx) return SD_ERR_INVALID_ARG;
-    if (batch < 0 || batch > ctx->cfg.max_batch) return fail(ctx, SD_ERR_INVALID_ARG, "batch out of range");
-    if (batch == 0) return SD_OK;
-    if (!q || !k_cache || !v_cache || !page_table || !seq_lens || !out)
+    if (num_tokens < 0) return fail(ctx, SD_ERR_INVALID_ARG, "num_tokens < 0");
+    const long long rows = local_rows(ctx);
+    if (num_tokens == 0 || ctx->tb.n_loc == 0 || rows == 0) return SD_OK;
+    if (!k_new || !v_new || !seq_ids || !positions || !local_k || !local_v)
       return fail(ctx, SD_ERR_INVALID_ARG, "null pointer");
-    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
-      return fail(ctx, SD_ERR_INVALID_ARG, "q, k_cache and v_cache must be 16-byte aligned");
-    const bool ret = ctx->sh.H_ret > 0;
-    if (ret) {
-      if (!q_pre || !index_cache || !sel_idx || !sel_count) return fail(ctx, SD_ERR_INVALID_ARG, "null pointer");
-      if (!aligned16(q_pre) || !aligned16(index_cache))
-        return fail(ctx, SD_ERR_INVALID_ARG, "q_pre and index_cache must be 16-byte aligned");
-      const long long need_stride = ctx->cfg.mode == SD_TOP_P ? ctx->sh.max_len : max_topk(ctx);
-      if (sel_stride < need_stride)
-        return fail(ctx, SD_ERR_INVALID_ARG, "sel_stride smaller than the largest possible set");
-    }
-    const WsLayout w = layout(ctx, batch);
-    if (!workspace || ws_bytes < w.total) return fail(ctx, SD_ERR_WORKSPACE, "workspace too small");
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(local_k) || !aligned16(local_v))
+      return fail(ctx, SD_ERR_INVALID_ARG, "k_new, v_new and the local caches must be 16-byte aligned");
     DeviceGuard dg(ctx->device);
-    const cudaStream_t st = static_cast<cudaStream_t>(stream);
-    char *wsb = static_cast<char *>(workspace);
-    bool unioned = false;
-    if (ret) {
-      sd::SelectArgs a{};
-      a.q_pre = static_cast<const uint16_t *>(q_pre);
-      a.index_cache = static_cast<const uint16_t *>(index_cache);
-      a.page_table = page_table;
-      a.seq_lens = seq_lens;
-      a.sel_idx = sel_idx;
-      a.sel_count = sel_count;
-      a.sel_stride = sel_stride;
-      a.proj = ctx->proj_d;
-      a.index_scale = ctx->index_scale;
-      a.mode = ctx->cfg.mode;
-      a.top_p = ctx->cfg.top_p;
-      a.top_k = ctx->cfg.top_k;
-      a.top_k_frac = ctx->cfg.top_k_frac;
-      a.score_ws = reinterpret_cast<float *>(wsb + w.scores_off);
-      a.flags = reinterpret_cast<uint32_t *>(wsb + w.flags_off);
-      a.stream_ws = w.stream_bytes ? wsb + w.stream_off : nullptr;
-      a.err = ctx->err_d;
-      a.batch = batch;
-      const sd::UnionOut uo = sd::attend_union_view(ctx->sh, ctx->tb, batch, wsb + w.att_off);
-      const cudaError_t e = sd::launch_select_union(a, ctx->sh, ctx->tb, uo, st, &unioned);
-      if (e != cudaSuccess) return cuda_fail(ctx, e, "select launch");
-    }
-    sd::AttendArgs at{};
-    at.q = static_cast<const uint16_t *>(q);
-    at.k_cache = static_cast<const uint16_t *>(k_cache);
-    at.v_cache = static_cast<const uint16_t *>(v_cache);
-    at.page_table = page_table;
-    at.seq_lens = seq_lens;
-    at.sel_idx = sel_idx;
-    at.sel_count = sel_count;
-    at.sel_stride = sel_stride;
-    at.out = out;
-    at.attn_scale = ctx->attn_scale;
-    at.window = ctx->cfg.window;
-    at.num_sinks = ctx->cfg.num_sinks;
-    at.ws = wsb + w.att_off;
-    at.err = ctx->err_d;
-    at.batch = batch;
-    // with the union lists built by select, attend plans only the items the
-    // exact selector redid (listed in the miss array)
-    const uint32_t *only = unioned ? reinterpret_cast<const uint32_t *>(wsb + w.flags_off) : nullptr;
-    const cudaError_t e = sd::launch_attend(at, ctx->sh, ctx->tb, st, only);
-    return e == cudaSuccess ? SD_OK : cuda_fail(ctx, e, "attend launch");
+    const cudaError_t e = sd::launch_local_append(
+        static_cast<const uint16_t *>(k_new), static_cast<const uint16_t *>(v_new), seq_ids, positions, num_tokens,
+        static_cast<uint16_t *>(local_k), static_cast<uint16_t *>(local_v), ctx->sh, ctx->tb, ctx->cfg.max_batch,
+        ctx->cfg.num_sinks, ctx->cfg.window, ctx->err_d, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SD_OK : cuda_fail(ctx, e, "local_append launch");
   } catch (...) {
     return SD_ERR_HOST_MEMORY;
   }

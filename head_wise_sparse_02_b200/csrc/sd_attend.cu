@@ -357,8 +357,11 @@ __device__ void plan_span(const AttendArgs &a, const Shape &sh, const Tables &tb
   }
   uint32_t *rows = ws.plan_row + slot * ap.span;
   uint16_t *masks = ws.plan_mask + slot * ap.span;
-  const uint32_t row_g = (uint32_t)g * kPage;          // row of (page, g, slot) = (page * Hkv + g) * 16 + slot
-  const uint32_t row_page = (uint32_t)sh.Hkv * kPage;
+  // row of (page, head, slot) = (page * heads + head) * 16 + slot; with a
+  // compacted local cache the paged caches hold the retrieval groups only
+  const bool ret_only = a.split;
+  const uint32_t row_g = (uint32_t)(ret_only ? gi : g) * kPage;
+  const uint32_t row_page = (uint32_t)(ret_only ? tb.n_ret : sh.Hkv) * kPage;
   bool bad_page = false;
   for (int r = 0; r < steps; ++r) {
     const int xb = x0 + r * 32;
@@ -475,7 +478,7 @@ attend_main_kernel(const AttendArgs a, const Shape sh, const Tables tb, const At
   const int c_sub = lane / CPR;                      // which of them
   const int c_ch = lane % CPR;                       // 16-byte chunk of the row
   const uint32_t ring_w = ring0 + warp * (kTileRing * kTileB);
-  const unsigned char *kbase = reinterpret_cast<const unsigned char *>(a.k_cache);
+  const unsigned char *kbase = reinterpret_cast<const unsigned char *>(a.k_cache);   // per item, below
   const unsigned char *vbase = reinterpret_cast<const unsigned char *>(a.v_cache);
   // ldmatrix lane addresses inside a tile (plus a constant per k-step / n-tile)
   const int lm = lane >> 3, lr = lane & 7;
@@ -533,6 +536,11 @@ attend_main_kernel(const AttendArgs a, const Shape sh, const Tables tb, const At
     const int g = S.grp.kv_head;
     const long long loc_a = std::min<long long>(a.num_sinks, N);
     const long long loc_w = std::max<long long>(loc_a, N - a.window);
+    // compacted local cache: rows of (b, local group) start here; the caches
+    // the tiles are copied from
+    const long long local_base = is_ret ? 0 : (long long)(item - ap.n_ret_items) * (a.num_sinks + a.window);
+    kbase = reinterpret_cast<const unsigned char *>(!is_ret && a.split ? a.local_k : a.k_cache);
+    vbase = reinterpret_cast<const unsigned char *>(!is_ret && a.split ? a.local_v : a.v_cache);
 
     // ---- queries: A fragments of Q (heads on M), bf16 ----------------------
     uint32_t qa[KS][4];
@@ -580,11 +588,16 @@ attend_main_kernel(const AttendArgs a, const Shape sh, const Tables tb, const At
           mask = __ldcg(ws.plan_mask + e);
         } else {
           const long long pos = gx < loc_a ? gx : loc_w + (gx - loc_a);
-          const int page = pt[pos / kPage];
-          const bool ok = page >= 0 && page < sh.num_pages;
-          if (!ok) raise_error(a.err, SD_EBIT_PAGE);
-          row = ok ? (uint32_t)(((long long)page * sh.Hkv + g) * kPage + (pos % kPage)) : 0u;
-          mask = ok ? all : 0u;
+          if (a.split) {                               // compacted: sinks, then a ring of the window
+            row = (uint32_t)(local_base + local_slot(pos, a.num_sinks, a.window));
+            mask = all;
+          } else {
+            const int page = pt[pos / kPage];
+            const bool ok = page >= 0 && page < sh.num_pages;
+            if (!ok) raise_error(a.err, SD_EBIT_PAGE);
+            row = ok ? (uint32_t)(((long long)page * sh.Hkv + g) * kPage + (pos % kPage)) : 0u;
+            mask = ok ? all : 0u;
+          }
         }
       }
     };
@@ -957,12 +970,12 @@ size_t attend_workspace_bytes(const Shape &sh, const Tables &tb, int batch) {
   return att_layout(sh, tb, batch).total;
 }
 
-UnionOut attend_union_view(const Shape &sh, const Tables &tb, int batch, void *attend_ws) {
+UnionOut attend_union_view(const Shape &sh, const Tables &tb, int batch, void *attend_ws, bool ret_only) {
   const AttLayout L = att_layout(sh, tb, batch);
   const AttParams p = att_params(sh, tb, batch);
   char *base = static_cast<char *>(attend_ws);
   return UnionOut{reinterpret_cast<uint32_t *>(base + L.plan_row), reinterpret_cast<uint16_t *>(base + L.plan_mask),
-                  reinterpret_cast<int *>(base + L.plan_cnt), p.span, p.ns};
+                  reinterpret_cast<int *>(base + L.plan_cnt), p.span, p.ns, ret_only};
 }
 
 cudaError_t launch_attend(const AttendArgs &a, const Shape &sh, const Tables &tb, cudaStream_t st,

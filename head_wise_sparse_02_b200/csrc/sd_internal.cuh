@@ -250,6 +250,7 @@ struct UnionOut {
   uint16_t *mask;                 // [B][n_ret][ns][span]
   int *cnt;                       // [B][n_ret][ns]
   int span, ns;
+  bool ret_only;                  // rows address caches of the retrieval groups only
 };
 
 size_t select_workspace_bytes(const Shape &sh, const Tables &tb, int batch, size_t *flags_off);
@@ -287,7 +288,25 @@ struct AttendArgs {
   void *ws;                       // attend's part of the workspace (partials, union lists, tickets)
   unsigned *err;
   int batch;
+  // split layout: the paged caches hold only the retrieval KV groups (in
+  // ascending KV-head order) and the local groups read the compacted caches
+  // local_k / local_v [B][n_loc][num_sinks + window][d]
+  bool split;
+  const uint16_t *local_k;
+  const uint16_t *local_v;
 };
+
+// Slot of position `pos` in a compacted local-head cache: sinks first, then a
+// ring of `window` slots; -1 when the position is kept nowhere (no window).
+__host__ __device__ __forceinline__ long long local_slot(long long pos, int num_sinks, int window) {
+  if (pos < num_sinks) return pos;
+  return window > 0 ? num_sinks + pos % window : -1;
+}
+
+cudaError_t launch_local_append(const uint16_t *k_new, const uint16_t *v_new, const int32_t *seq_ids,
+                                const int32_t *positions, int T, uint16_t *local_k, uint16_t *local_v,
+                                const Shape &sh, const Tables &tb, int max_batch, int num_sinks, int window,
+                                unsigned *err, cudaStream_t st);
 
 size_t attend_workspace_bytes(const Shape &sh, const Tables &tb, int batch);
 // plan_only: null = plan every retrieval item; else the select's miss array
@@ -295,7 +314,7 @@ size_t attend_workspace_bytes(const Shape &sh, const Tables &tb, int batch);
 // others' union lists are already in the workspace.
 cudaError_t launch_attend(const AttendArgs &a, const Shape &sh, const Tables &tb, cudaStream_t st,
                           const uint32_t *plan_only = nullptr);
-UnionOut attend_union_view(const Shape &sh, const Tables &tb, int batch, void *attend_ws);
+UnionOut attend_union_view(const Shape &sh, const Tables &tb, int batch, void *attend_ws, bool ret_only);
 
 // Size of the built-in attend scratch of sparse_decode_attend_noalloc.
 constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;

@@ -1345,8 +1345,10 @@ resolve_union_kernel(const SelectArgs a, const Shape sh, const StreamWs ws, cons
   const int words = (int)((N + 31) / 32);
   const int span_words = uo.span / 32;
   const int ns_item = (int)((N + uo.span - 1) / uo.span);
-  const uint32_t row_g = (uint32_t)g * kPage;        // row of (page, g, slot) = (page * Hkv + g) * 16 + slot
-  const uint32_t row_page = (uint32_t)sh.Hkv * kPage;
+  // row of (page, head, slot) = (page * heads + head) * 16 + slot, over all KV
+  // heads or over the retrieval groups only
+  const uint32_t row_g = (uint32_t)(uo.ret_only ? gi : g) * kPage;
+  const uint32_t row_page = (uint32_t)(uo.ret_only ? n_groups : sh.Hkv) * kPage;
   const int32_t *pt = a.page_table + (long long)b * sh.max_pages;
   bool bad_page = false;
   for (int sp = 0; sp < ns_item; ++sp) {

@@ -73,6 +73,51 @@ class DecodeStep:
             self.sd.index_keys(new_keys, new_slots, self.index_cache, stream)
         return self.select_attend(q_pre, q, stream)
 
+    # ---- split layout: paged caches of the retrieval groups, compacted local caches
+
+    def make_split(self, stream=None):
+        """Build the split layout from the full caches: k_ret / v_ret keep the
+        retrieval KV groups, and local_append copies every sequence's sinks
+        and window (its local positions, in order) into compacted caches."""
+        retr = self.sd.cfg["head_is_retrieval"]
+        Hkv = self.k_cache.shape[1]
+        G = self.num_q_heads // Hkv
+        ret_g = [g for g in range(Hkv) if any(retr[g * G:(g + 1) * G])]
+        if ret_g == list(range(Hkv)):                                  # every group retrieves
+            self.k_ret, self.v_ret = self.k_cache, self.v_cache
+        else:
+            self.k_ret = self.k_cache[:, ret_g].contiguous()
+            self.v_ret = self.v_cache[:, ret_g].contiguous()
+        self.local_k, self.local_v = self.sd.local_cache()
+        window, sinks = self.sd.cfg.get("window", 0), self.sd.cfg.get("num_sinks", 0)
+        lens = self.seq_lens.tolist()
+        seq, pos = [], []
+        for b, n in enumerate(lens):
+            keep = sorted(set(range(min(sinks, n))) | set(range(max(0, n - window), n)))
+            seq += [b] * len(keep)
+            pos += keep
+        if pos:
+            dev = self.k_cache.device
+            seq_t = torch.tensor(seq, dtype=torch.int32, device=dev)
+            pos_t = torch.tensor(pos, dtype=torch.int32, device=dev)
+            page = self.page_table[seq_t.long(), (pos_t // 16).long()].long()
+            off = (pos_t % 16).long()
+            k_new = self.k_cache[page, :, off].contiguous()           # [T, Hkv, d]
+            v_new = self.v_cache[page, :, off].contiguous()
+            self.sd.local_append(k_new, v_new, seq_t, pos_t, self.local_k, self.local_v, stream)
+
+    def attend_split(self, q: torch.Tensor, sel_idx=None, sel_count=None, stream=None):
+        self.sd.attend_split(q, self.k_ret, self.v_ret, self.local_k, self.local_v, self.page_table,
+                             self.seq_lens, self.sel_idx if sel_idx is None else sel_idx,
+                             self.sel_count if sel_count is None else sel_count, self.out, self.workspace, stream)
+        return self.out
+
+    def select_attend_split(self, q_pre: torch.Tensor, q: torch.Tensor, stream=None) -> torch.Tensor:
+        self.sd.select_attend_split(q_pre, q, self.index_cache, self.k_ret, self.v_ret, self.local_k,
+                                    self.local_v, self.page_table, self.seq_lens, self.sel_idx, self.sel_count,
+                                    self.out, self.workspace, stream)
+        return self.out
+
     def error_word(self, stream=None) -> int:
         return self.sd.error_word(stream)
 

@@ -57,6 +57,12 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sparse_decode_select_attend": (c_int, [P, P, P, P, P, P, P, P, c_int, P, P, c_int, P, P, c_size_t, P]),
         "sparse_decode_attend_noalloc": (c_int, [P, P, P, P, P, P, c_int, P, P, c_int, P, P]),
         "sparse_decode_error_word": (c_int, [P, P, POINTER(c_uint32)]),
+        "sparse_decode_attend_split": (c_int, [P, P, P, P, P, P, P, P, c_int, P, P, c_int, P, P, c_size_t, P]),
+        "sparse_decode_select_attend_split": (c_int, [P, P, P, P, P, P, P, P, P, P, c_int, P, P, c_int, P, P,
+                                                      c_size_t, P]),
+        "sparse_decode_local_append": (c_int, [P, P, P, P, P, c_int, P, P, P]),
+        "sparse_decode_num_retrieval_groups": (c_int, [P]),
+        "sparse_decode_num_local_groups": (c_int, [P]),
         "sparse_decode_num_retrieval_heads": (c_int, [P]),
         "sparse_decode_last_error": (c_char_p, [P]),
         "sparse_decode_status_string": (c_char_p, [c_int]),
@@ -209,6 +215,71 @@ def sparse_decode_select_attend(ctx: int, q_pre, q, index_cache, k_cache, v_cach
         _stream(stream)), ctx)
 
 
+def _check_local(ctx: int, local_k, local_v, rows_needed: int) -> None:
+    """The compacted local caches are addressed through raw pointers: check that
+    both hold at least `rows_needed` sequences of [Lg, num_sinks + window, d]."""
+    for name, t in (("local_k", local_k), ("local_v", local_v)):
+        if t is None:
+            continue
+        if t.dim() != 4 or t.shape[0] < rows_needed or t.shape[1] != sparse_decode_num_local_groups(ctx):
+            raise ValueError(f"{name} must be [>= {rows_needed}, Lg = {sparse_decode_num_local_groups(ctx)}, "
+                             f"num_sinks + window, d], got {tuple(t.shape)}")
+
+
+def sparse_decode_attend_split(ctx: int, q, k_ret, v_ret, local_k, local_v, page_table, seq_lens, sel_idx,
+                               sel_count, out, workspace, stream=None) -> None:
+    """attend on the split layout: paged caches of the retrieval groups only,
+    compacted sink + window caches of the local groups."""
+    _check_sets(ctx, sel_idx, sel_count, int(seq_lens.numel()))
+    _check_local(ctx, local_k, local_v, int(seq_lens.numel()))
+    stride = int(sel_idx.shape[-1]) if sel_idx is not None else 0
+    _check(LIB.sparse_decode_attend_split(
+        ctx, _ptr(q, torch.bfloat16, "q"), _ptr(k_ret, torch.bfloat16, "k_ret"),
+        _ptr(v_ret, torch.bfloat16, "v_ret"), _ptr(local_k, torch.bfloat16, "local_k"),
+        _ptr(local_v, torch.bfloat16, "local_v"), _ptr(page_table, torch.int32, "page_table"),
+        _ptr(seq_lens, torch.int32, "seq_lens"), int(seq_lens.numel()),
+        _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_count, torch.int32, "sel_count"), stride,
+        _ptr(out, torch.float32, "out"), _ptr(workspace, torch.uint8, "workspace"),
+        int(workspace.numel()), _stream(stream)), ctx)
+
+
+def sparse_decode_select_attend_split(ctx: int, q_pre, q, index_cache, k_ret, v_ret, local_k, local_v,
+                                      page_table, seq_lens, sel_idx, sel_count, out, workspace,
+                                      stream=None) -> None:
+    """select_attend on the split layout."""
+    _check_sets(ctx, sel_idx, sel_count, int(seq_lens.numel()))
+    _check_local(ctx, local_k, local_v, int(seq_lens.numel()))
+    stride = int(sel_idx.shape[-1]) if sel_idx is not None else 0
+    _check(LIB.sparse_decode_select_attend_split(
+        ctx, _ptr(q_pre, torch.bfloat16, "q_pre"), _ptr(q, torch.bfloat16, "q"),
+        _ptr(index_cache, torch.bfloat16, "index_cache"), _ptr(k_ret, torch.bfloat16, "k_ret"),
+        _ptr(v_ret, torch.bfloat16, "v_ret"), _ptr(local_k, torch.bfloat16, "local_k"),
+        _ptr(local_v, torch.bfloat16, "local_v"), _ptr(page_table, torch.int32, "page_table"),
+        _ptr(seq_lens, torch.int32, "seq_lens"), int(seq_lens.numel()),
+        _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_count, torch.int32, "sel_count"), stride,
+        _ptr(out, torch.float32, "out"), _ptr(workspace, torch.uint8, "workspace"), int(workspace.numel()),
+        _stream(stream)), ctx)
+
+
+def sparse_decode_local_append(ctx: int, k_new, v_new, seq_ids, positions, local_k, local_v, max_batch: int,
+                               stream=None) -> None:
+    """Copy new tokens' keys and values ([T, Hkv, d]) of the local groups into
+    the compacted caches ([max_batch, Lg, num_sinks + window, d])."""
+    _check_local(ctx, local_k, local_v, max_batch)
+    _check(LIB.sparse_decode_local_append(
+        ctx, _ptr(k_new, torch.bfloat16, "k_new"), _ptr(v_new, torch.bfloat16, "v_new"),
+        _ptr(seq_ids, torch.int32, "seq_ids"), _ptr(positions, torch.int32, "positions"), int(seq_ids.numel()),
+        _ptr(local_k, torch.bfloat16, "local_k"), _ptr(local_v, torch.bfloat16, "local_v"), _stream(stream)), ctx)
+
+
+def sparse_decode_num_retrieval_groups(ctx: int) -> int:
+    return int(LIB.sparse_decode_num_retrieval_groups(ctx))
+
+
+def sparse_decode_num_local_groups(ctx: int) -> int:
+    return int(LIB.sparse_decode_num_local_groups(ctx))
+
+
 def sparse_decode_attend_noalloc(ctx: int, q, k_cache, v_cache, page_table, seq_lens, sel_idx, sel_count,
                                  out, stream=None) -> None:
     """attend on the library's built-in scratch (no workspace argument)."""
@@ -303,6 +374,33 @@ class SparseDecode:
                       out, workspace, stream=None):
         sparse_decode_select_attend(self.handle, q_pre, q, index_cache, k_cache, v_cache, page_table, seq_lens,
                                     sel_idx, sel_count, out, workspace, stream)
+
+    def attend_split(self, q, k_ret, v_ret, local_k, local_v, page_table, seq_lens, sel_idx, sel_count, out,
+                     workspace, stream=None):
+        sparse_decode_attend_split(self.handle, q, k_ret, v_ret, local_k, local_v, page_table, seq_lens,
+                                   sel_idx, sel_count, out, workspace, stream)
+
+    def select_attend_split(self, q_pre, q, index_cache, k_ret, v_ret, local_k, local_v, page_table, seq_lens,
+                            sel_idx, sel_count, out, workspace, stream=None):
+        sparse_decode_select_attend_split(self.handle, q_pre, q, index_cache, k_ret, v_ret, local_k, local_v,
+                                          page_table, seq_lens, sel_idx, sel_count, out, workspace, stream)
+
+    def local_append(self, k_new, v_new, seq_ids, positions, local_k, local_v, stream=None):
+        sparse_decode_local_append(self.handle, k_new, v_new, seq_ids, positions, local_k, local_v,
+                                   self.cfg["max_batch"], stream)
+
+    def num_retrieval_groups(self) -> int:
+        return sparse_decode_num_retrieval_groups(self.handle)
+
+    def num_local_groups(self) -> int:
+        return sparse_decode_num_local_groups(self.handle)
+
+    def local_cache(self, max_batch: Optional[int] = None):
+        """Zeroed compacted local caches (K, V) for `max_batch` sequences."""
+        rows = self.cfg.get("window", 0) + self.cfg.get("num_sinks", 0)
+        shape = (max_batch or self.cfg["max_batch"], self.num_local_groups(), rows, self.cfg["head_dim"])
+        return (torch.zeros(shape, dtype=torch.bfloat16, device=self.device),
+                torch.zeros(shape, dtype=torch.bfloat16, device=self.device))
 
     def error_word(self, stream=None) -> int:
         return sparse_decode_error_word(self.handle, stream)

@@ -39,9 +39,10 @@
  *     q and q_pre must start on a 16-byte boundary (they are read with 16-byte
  *     vector and asynchronous copies); a misaligned one is rejected with
  *     SD_ERR_INVALID_ARG.
- *   - Hot calls (index_keys, select, attend) allocate nothing, never
- *     synchronise the host, and enqueue their work on `stream` (a
- *     cudaStream_t; NULL = the legacy default stream).  Argument errors are
+ *   - Hot calls (index_keys, local_append, select, attend and their joined
+ *     and split forms) allocate nothing, never synchronise the host, and
+ *     enqueue their work on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream).  Argument errors are
  *     detected on the host before any launch and nothing is enqueued.
  *   - Data-dependent errors found on the device (a page id outside
  *     [0, num_pages), a sequence length above max_pages_per_seq * page_size,
@@ -304,6 +305,90 @@ SD_API sd_status sparse_decode_select_attend(sd_ctx *ctx, const void *q_pre, con
                                       const int32_t *page_table, const int32_t *seq_lens, int batch,
                                       int32_t *sel_idx, int32_t *sel_count, int sel_stride, float *out,
                                       void *workspace, size_t ws_bytes, sd_stream stream);
+
+/*
+ * Split cache layout (RTPurbo page, Methodology 1: local heads only ever see
+ * the sinks and the recent window; AoH page, Methodology 4: the KV memory of
+ * streaming heads is the saving).  The paged caches then hold only the
+ * retrieval KV groups, and each local KV group keeps a compacted cache of
+ * num_sinks + window rows per sequence instead of the whole context:
+ *
+ *   k_ret, v_ret      bf16 [num_pages, R, P, d], R = number of retrieval KV
+ *                     groups (KV heads with at least one retrieval query head,
+ *                     in ascending KV-head order); token j of sequence b,
+ *                     i-th retrieval group, at [page_table[b][j / P], i, j % P, :].
+ *   local_k, local_v  bf16 [max_batch, Lg, num_sinks + window, d], Lg = number
+ *                     of local KV groups (KV heads with at least one local
+ *                     query head, ascending); position j of sequence b,
+ *                     i-th local group, at [b, i, slot(j), :] with
+ *                     slot(j) = j for j < num_sinks, else
+ *                     num_sinks + j % window.  Row b is sequence b of a call's
+ *                     batch, like row b of page_table.
+ *
+ * A KV group with both kinds of query heads is kept in both.  The index cache
+ * keeps its layout.  Every position in [0, num_sinks) U [N_b - window, N_b)
+ * has its own slot, so after the tokens of a sequence are appended in
+ * position order the compacted rows hold exactly the rows its local heads
+ * attend to at length N_b; the outputs equal those of the full layout.
+ */
+
+/* R and Lg of the split layout (0 on a NULL context). */
+SD_API int sparse_decode_num_retrieval_groups(const sd_ctx *ctx);
+SD_API int sparse_decode_num_local_groups(const sd_ctx *ctx);
+
+/*
+ * sparse_decode_local_append -- copy the keys and values of `num_tokens` new
+ * tokens into the compacted local caches:
+ *
+ *   local_k[s_t, i, slot(p_t), :] = k_new[t, g_i, :]   (and likewise v)
+ *
+ * for every local KV group i (KV head g_i), s_t = seq_ids[t], p_t = positions[t].
+ *
+ *   k_new, v_new      device bf16 [num_tokens, Hkv, d], post-RoPE keys and the
+ *                     values of the new tokens (the rows of every KV head; only
+ *                     local groups are read).
+ *   seq_ids           device int32 [num_tokens], in [0, max_batch).
+ *   positions         device int32 [num_tokens], in [0, L).
+ *   local_k, local_v  device bf16, the split layout's compacted caches.
+ *
+ * A token whose sequence or position is out of range sets SD_EBIT_SLOT and is
+ * skipped.  Positions >= num_sinks with window == 0 are kept nowhere (no
+ * error).  Tokens of one call that land on the same slot of the same
+ * sequence (more than `window` positions past the sinks of one sequence in a
+ * call) race: which one stays is unspecified; append at most the last
+ * `window` such positions of a sequence per call.  num_tokens == 0, or no
+ * local group, is a no-op.
+ */
+SD_API sd_status sparse_decode_local_append(sd_ctx *ctx, const void *k_new, const void *v_new,
+                                     const int32_t *seq_ids, const int32_t *positions, int num_tokens,
+                                     void *local_k, void *local_v, sd_stream stream);
+
+/*
+ * sparse_decode_attend_split -- sparse_decode_attend on the split layout:
+ * retrieval heads read k_ret / v_ret, local heads their compacted caches.
+ * Same arguments otherwise; the outputs equal those of sparse_decode_attend
+ * on the full caches holding the same data.  k_ret / v_ret may be NULL
+ * without retrieval heads, local_k / local_v without local heads (or with
+ * num_sinks + window == 0).  Returns SD_ERR_UNSUPPORTED when
+ * batch * Lg * (num_sinks + window) reaches 2^32 rows.
+ */
+SD_API sd_status sparse_decode_attend_split(sd_ctx *ctx, const void *q, const void *k_ret, const void *v_ret,
+                                     const void *local_k, const void *local_v, const int32_t *page_table,
+                                     const int32_t *seq_lens, int batch, const int32_t *sel_idx,
+                                     const int32_t *sel_count, int sel_stride, float *out,
+                                     void *workspace, size_t ws_bytes, sd_stream stream);
+
+/*
+ * sparse_decode_select_attend_split -- sparse_decode_select_attend on the split
+ * layout (the index cache keeps its layout).  Arguments, results and errors as
+ * for sparse_decode_select_attend and sparse_decode_attend_split.
+ */
+SD_API sd_status sparse_decode_select_attend_split(sd_ctx *ctx, const void *q_pre, const void *q,
+                                            const void *index_cache, const void *k_ret, const void *v_ret,
+                                            const void *local_k, const void *local_v,
+                                            const int32_t *page_table, const int32_t *seq_lens, int batch,
+                                            int32_t *sel_idx, int32_t *sel_count, int sel_stride, float *out,
+                                            void *workspace, size_t ws_bytes, sd_stream stream);
 
 /*
  * sparse_decode_attend_noalloc -- sparse_decode_attend without a workspace

@@ -74,6 +74,8 @@ __all__ = [
     "select_top_k",
     "top_k_budget",
     "local_positions",
+    "local_slot",
+    "compact_local_rows",
     "attend_set",
     "gather_rows",
     "OracleConfig",
@@ -229,6 +231,34 @@ def local_positions(n: int, window: int, num_sinks: int) -> np.ndarray:
     sinks = np.arange(min(num_sinks, n))
     win = np.arange(max(0, n - window), n)
     return np.union1d(sinks, win).astype(np.int64)
+
+
+def local_slot(pos: int, window: int, num_sinks: int) -> int:
+    """Row of position ``pos`` in a compacted local-head cache of
+    num_sinks + window rows: a sink keeps its own row, every later position
+    cycles through a ring of ``window`` rows; -1 when the position is kept
+    nowhere (window 0).  Storage reading: the pages fix only which positions a
+    local head attends to ([RTP] §1, [AoH] §4); keeping just those rows is the
+    KV saving that [AoH] §4 attributes to streaming heads."""
+    if pos < num_sinks:
+        return int(pos)
+    if window == 0:
+        return -1
+    return int(num_sinks + pos % window)
+
+
+def compact_local_rows(rows, window: int, num_sinks: int) -> np.ndarray:
+    """Compacted cache of one (sequence, local KV head) after the rows of
+    positions 0..n-1 (``rows[j]``, n = len(rows)) were written in position
+    order, each to its ``local_slot``; a row never written stays zero.  Keeps
+    the dtype of ``rows`` (raw bf16 bit patterns stay bit patterns)."""
+    rows = np.asarray(rows)
+    out = np.zeros((num_sinks + window,) + rows.shape[1:], dtype=rows.dtype)
+    for j in range(rows.shape[0]):
+        s = local_slot(j, window, num_sinks)
+        if s >= 0:
+            out[s] = rows[j]
+    return out
 
 
 # --------------------------------------------------------------------------

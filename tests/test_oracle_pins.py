@@ -149,6 +149,44 @@ def test_local_positions_hand_worked_cases():
         assert O.local_positions(c["n"], c["window"], c["sinks"]).tolist() == want, c
 
 
+# ---------------------------------------------------------------- compacted local cache
+
+@pytest.mark.parametrize("sinks", [0, 1, 3, 8])
+@pytest.mark.parametrize("window", [0, 1, 5, 16])
+def test_compacted_local_rows_hold_exactly_the_local_positions(window, sinks):
+    """After positions 0..n-1 are written in order, the compacted rows hold
+    each position a local head attends to at length n exactly once and
+    nothing else (marker rows: row j carries j + 1).  A ring that ignored the
+    sinks, or a slot off by one, overwrites a kept row and fails here."""
+    for n in range(0, 70):
+        rows = (np.arange(n, dtype=np.int64) + 1)[:, None]
+        comp = O.compact_local_rows(rows, window, sinks)
+        assert comp.shape == (sinks + window, 1)
+        held = sorted(int(x) - 1 for x in comp[:, 0] if x != 0)
+        assert held == O.local_positions(n, window, sinks).tolist(), (n, window, sinks)
+
+
+def test_local_slot_hand_cases():
+    # sinks keep their rows; the ring starts after them and wraps every `window`
+    assert [O.local_slot(p, 4, 2) for p in range(11)] == [0, 1, 4, 5, 2, 3, 4, 5, 2, 3, 4]
+    assert [O.local_slot(p, 0, 2) for p in range(4)] == [0, 1, -1, -1]
+    assert [O.local_slot(p, 3, 0) for p in range(5)] == [0, 1, 2, 0, 1]
+
+
+def test_local_attention_over_compacted_rows_equals_the_paged_one():
+    rng = np.random.default_rng(3)
+    n, d, window, sinks = 57, 8, 16, 4
+    K, V, q = rng.normal(size=(n, d)), rng.normal(size=(n, d)), rng.normal(size=d)
+    keep = O.local_positions(n, window, sinks)
+    ck = O.compact_local_rows(K, window, sinks)
+    cv = O.compact_local_rows(V, window, sinks)
+    slots = [O.local_slot(j, window, sinks) for j in keep]
+    assert len(set(slots)) == len(slots)
+    got = O.attend_set(q, ck, cv, slots, 0.3)
+    want = O.attend_set(q, K, V, keep, 0.3)
+    assert np.allclose(got, want, rtol=1e-13, atol=1e-13)
+
+
 # ---------------------------------------------------------------- top-p
 
 def _mass(s):
