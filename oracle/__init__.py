@@ -7,3 +7,4 @@ imports it.
 """
 
 from .sparse_decode_oracle import *  # noqa: F401,F403
+from .head_classifier_oracle import *  # noqa: F401,F403
