@@ -22,6 +22,7 @@ a bounded sample of the same workload.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import hashlib
 import json
 import math
@@ -749,6 +750,208 @@ def run_reference(args):
     print(json.dumps(res), flush=True)
 
 
+# ---------------------------------------------------------------- head classifier
+
+# float64 peak of the part: 148 SMs x 64 FP64 FMA per clock x 2 flops x 1965 MHz
+# (the recipe's SM count and maximum clock; 64 FP64 lanes per SM)
+FP64_PEAK_TFLOPS = 148 * 64 * 2 * 1.965e9 / 1e12
+CLASSIFY_METRIC = "AoH data-free head classification: query heads classified/s (effective rank of W_K^T W_Q)"
+
+
+def classifier_flops(L, Hq, Hkv, D, d_model) -> dict:
+    """Algorithmic float64 flops of one call: the symmetric Gram matrices
+    (D (D+1)/2 entries of d_model products each, query and key blocks), their
+    Cholesky factors (D^3/3) and X = L_k^T L_q (triangular, D^3/3
+    multiply-adds).  The Jacobi sweeps are iterative and not counted."""
+    mats = L * (Hq + Hkv)
+    return {"gram": 2.0 * mats * D * (D + 1) / 2 * d_model, "cholesky": mats * D ** 3 / 3.0,
+            "x_product": L * Hq * 2.0 * D ** 3 / 3.0}
+
+
+def run_classifier(args):
+    import torch
+    import torch.distributed as dist
+
+    from head_wise_sparse_02_b200 import sparse_decode as sd
+    from workloads import make_projections
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    L = args.layers
+    p = make_projections(dev, seed=rank_seed(7 if args.seed is None else args.seed, rank), num_layers=L)
+    Hq, Hkv, D, dm = p.num_q_heads, p.num_kv_heads, p.head_dim, p.d_model
+    n = ctypes.c_size_t()
+    sd._check(sd.LIB.sparse_decode_head_er_workspace_size(L, Hq, Hkv, D, ctypes.byref(n)))
+    wsb = torch.empty(n.value, dtype=torch.uint8, device=dev)
+    er = torch.empty((L, Hq), dtype=torch.float64, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        sd.sparse_decode_head_effective_rank(p.w_q, p.w_k, Hq, Hkv, D, eff_rank=er, workspace=wsb, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if not bool(torch.isfinite(er).all()):
+        raise RuntimeError("a head's Jacobi sweeps did not converge")
+    weight_bytes = (p.w_q.numel() + p.w_k.numel()) * 2
+    flush = weight_bytes < NO_FLUSH_ABOVE
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev) if flush else None
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    pairs = []
+    for _ in range(args.steps):
+        if flush:
+            flush_buf.zero_()
+        a0 = torch.cuda.Event(enable_timing=True); a1 = torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        step()
+        a1.record(stream)
+        pairs.append((a0, a1))
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms = sum(a.elapsed_time(b) for a, b in pairs) / args.steps
+    ms_max = max_over_ranks(ms, dev)
+
+    # end to end: the weights from pinned host memory, the call, the ERs back,
+    # and the per-layer classification on the host
+    wq_h, wk_h = p.w_q.cpu().pin_memory(), p.w_k.cpu().pin_memory()
+    wq_d, wk_d = torch.empty_like(p.w_q), torch.empty_like(p.w_k)
+    er_h = torch.empty((L, Hq), dtype=torch.float64).pin_memory()
+    n_ret = Hkv // 2
+
+    def e2e_step():
+        wq_d.copy_(wq_h, non_blocking=True)
+        wk_d.copy_(wk_h, non_blocking=True)
+        sd.sparse_decode_head_effective_rank(wq_d, wk_d, Hq, Hkv, D, eff_rank=er, workspace=wsb, stream=stream)
+        er_h.copy_(er, non_blocking=True)
+        stream.synchronize()
+        return [sd.sparse_decode_classify_heads(er_h[l], Hkv, n_ret) for l in range(L)]
+
+    e2e_step()
+    barrier()
+    t0 = torch.cuda.Event(enable_timing=True); t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, dev)
+
+    fl = classifier_flops(L, Hq, Hkv, D, dm)
+    total_fl = sum(fl.values())
+    achieved = total_fl / (ms * 1e-3) / 1e12
+    heads = ws * L * Hq
+    res = {
+        "metric": CLASSIFY_METRIC, "value": round(heads / (ms_max * 1e-3), 1), "unit": "heads/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "storage_dtype": "bf16",
+        "data": "synthetic (seeded bf16 projections with planted spectra; no trained weights)",
+        "config": {"workload": f"aoh_llama3_8b: {L} layers, d_model {dm}, Hq {Hq} / Hkv {Hkv}, d_head {D} "
+                               f"(Llama-3.1-8B attention shapes), {n_ret} of {Hkv} groups retrieval",
+                   "parallelism": f"replicas x{ws}",
+                   "l2": ("flushed between steps (512 MiB write, untimed)" if flush
+                          else f"no flush: every step reads {weight_bytes / 1e9:.2f} GB of weights")},
+        "roofline": {"kernel": "head_effective_rank (gram + cholesky + jacobi launches)", "bound": "alu",
+                     "achieved": round(achieved, 3), "peak": round(FP64_PEAK_TFLOPS, 1),
+                     "peak_kind": "derived fp64: 148 SMs x 64 FMA/clk x 2 x 1965 MHz", "unit": "TFLOP/s",
+                     "frac": round(achieved / FP64_PEAK_TFLOPS, 4), "algorithmic_flops_per_launch": fl,
+                     "traffic": None},
+        "weights_hbm_gbs": round(weight_bytes / (ms * 1e-3) / 1e9, 1),
+        "e2e": {"value": round(heads / (e2e_ms * 1e-3), 1), "unit": "heads/s",
+                "h2d_bytes_per_step": int(weight_bytes), "d2h_bytes_per_step": int(L * Hq * 8)},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = classifier_cpu_baseline(p, budget_s=args.cpu_budget)
+    if ws > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+def classifier_cpu_baseline(p, budget_s: float = 15.0):
+    """The oracle's eigenvalue route (C_h, float64 numpy), head by head over
+    the layers in order, until the budget runs out: heads/s."""
+    import numpy as np
+
+    import oracle as O
+    G = p.num_q_heads // p.num_kv_heads
+    done, t0 = 0, time.perf_counter()
+    for layer in range(p.num_layers):
+        wq = p.w_q[layer].float().cpu().numpy().astype(np.float64)
+        wk = p.w_k[layer].float().cpu().numpy().astype(np.float64)
+        for h in range(p.num_q_heads):
+            O.effective_rank_of_spectrum(O.singular_values_sylvester(
+                O.head_block(wq, h, p.head_dim), O.head_block(wk, h // G, p.head_dim)))
+            done += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+        if time.perf_counter() - t0 > budget_s:
+            break
+    el = time.perf_counter() - t0
+    return {"kind": "oracle", "value": round(done / el, 2), "unit": "heads/s", "cores": _blas_threads(),
+            "sample": f"{done} heads of the same synthetic weights (layers in order), float64 numpy, "
+                      "eigenvalues of C_h per head"}
+
+
+def run_classifier_reference(args):
+    """The oracle as the classifier's reference arm: each step one query head
+    of the same synthetic weights by the eigenvalue route, on the host."""
+    ws, rank, local = dist_env()
+    if rank != 0:
+        return
+    import numpy as np
+    import torch
+
+    import oracle as O
+    from workloads import make_projections
+    dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
+    L = args.layers
+    p = make_projections(dev, seed=7 if args.seed is None else args.seed, num_layers=L)
+    G = p.num_q_heads // p.num_kv_heads
+    wq = p.w_q[0].float().cpu().numpy().astype(np.float64)
+    wk = p.w_k[0].float().cpu().numpy().astype(np.float64)
+
+    def one(i):
+        h = i % p.num_q_heads
+        O.effective_rank_of_spectrum(O.singular_values_sylvester(O.head_block(wq, h, p.head_dim),
+                                                                 O.head_block(wk, h // G, p.head_dim)))
+
+    for i in range(args.warmup):
+        one(i)
+    t = time.perf_counter()
+    for i in range(args.steps):
+        one(i)
+    el = time.perf_counter() - t
+    v = args.steps / el
+    flush = (p.w_q.numel() + p.w_k.numel()) * 2 < NO_FLUSH_ABOVE
+    res = {"impl": "reference", "metric": CLASSIFY_METRIC, "value": round(v, 3), "unit": "heads/s", "n_gpus": ws,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic (seeded bf16 projections with planted spectra; no trained weights)",
+           "config": {"workload": f"aoh_llama3_8b: {L} layers, d_model {p.d_model}, Hq {p.num_q_heads} / Hkv "
+                                  f"{p.num_kv_heads}, d_head {p.head_dim} (Llama-3.1-8B attention shapes), "
+                                  f"{p.num_kv_heads // 2} of {p.num_kv_heads} groups retrieval",
+                      "parallelism": f"replicas x{ws}",
+                      "l2": ("flushed between steps (512 MiB write, untimed)" if flush
+                             else f"no flush: every step reads {(p.w_q.numel() + p.w_k.numel()) * 2 / 1e9:.2f} "
+                                  "GB of weights")},
+           "cpu_baseline": {"kind": "oracle", "cores": _blas_threads(), "value": round(v, 3), "unit": "heads/s",
+                            "sample": f"each step: one query head of layer 0 (eigenvalues of C_h, float64 "
+                                      f"numpy); {args.steps} heads"},
+           "e2e": {"value": round(v, 3), "unit": "heads/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -772,9 +975,15 @@ def main(argv=None):
                     help="split: paged caches of the retrieval groups only, compacted local caches")
     ap.add_argument("--no-diagnostics", action="store_true")
     ap.add_argument("--diag-budget", type=float, default=20.0)
+    ap.add_argument("--layers", type=int, default=32, help="aoh_llama3_8b: layers classified per step")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)          # timing rule: at least 3 warm-up steps
-    if args.impl == "reference":
+    if args.workload == "aoh_llama3_8b":
+        if args.impl == "reference":
+            run_classifier_reference(args)
+        else:
+            run_classifier(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

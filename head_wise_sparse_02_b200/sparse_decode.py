@@ -63,6 +63,10 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sparse_decode_local_append": (c_int, [P, P, P, P, P, c_int, P, P, P]),
         "sparse_decode_num_retrieval_groups": (c_int, [P]),
         "sparse_decode_num_local_groups": (c_int, [P]),
+        "sparse_decode_head_er_workspace_size": (c_int, [c_int, c_int, c_int, c_int, POINTER(c_size_t)]),
+        "sparse_decode_head_effective_rank": (c_int, [P, P, c_int, c_int, c_int, c_int, c_int, P, P, c_size_t,
+                                                      P]),
+        "sparse_decode_classify_heads": (c_int, [P, c_int, c_int, c_int, P]),
         "sparse_decode_num_retrieval_heads": (c_int, [P]),
         "sparse_decode_last_error": (c_char_p, [P]),
         "sparse_decode_status_string": (c_char_p, [c_int]),
@@ -278,6 +282,40 @@ def sparse_decode_num_retrieval_groups(ctx: int) -> int:
 
 def sparse_decode_num_local_groups(ctx: int) -> int:
     return int(LIB.sparse_decode_num_local_groups(ctx))
+
+
+def sparse_decode_head_effective_rank(w_q, w_k, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                                      eff_rank=None, workspace=None, stream=None) -> torch.Tensor:
+    """ER of every query head from the frozen projections w_q [L, Hq*d_head,
+    d_model] and w_k [L, Hkv*d_head, d_model] (bf16, CUDA); returns float64
+    [L, Hq] on the device."""
+    if w_q.dim() != 3 or w_k.dim() != 3 or w_q.shape[0] != w_k.shape[0] or w_q.shape[2] != w_k.shape[2]:
+        raise ValueError(f"w_q / w_k must be [L, H*d_head, d_model], got {tuple(w_q.shape)} / {tuple(w_k.shape)}")
+    L, d_model = int(w_q.shape[0]), int(w_q.shape[2])
+    if w_q.shape[1] != num_q_heads * head_dim or w_k.shape[1] != num_kv_heads * head_dim:
+        raise ValueError("w_q / w_k rows do not match the head counts")
+    n = c_size_t()
+    _check(LIB.sparse_decode_head_er_workspace_size(L, num_q_heads, num_kv_heads, head_dim, ctypes.byref(n)))
+    if workspace is None:
+        workspace = torch.empty(n.value, dtype=torch.uint8, device=w_q.device)
+    if eff_rank is None:
+        eff_rank = torch.empty((L, num_q_heads), dtype=torch.float64, device=w_q.device)
+    if eff_rank.numel() < L * num_q_heads:
+        raise ValueError("eff_rank too small")
+    _check(LIB.sparse_decode_head_effective_rank(
+        _ptr(w_q, torch.bfloat16, "w_q"), _ptr(w_k, torch.bfloat16, "w_k"), L, d_model, num_q_heads, num_kv_heads,
+        head_dim, _ptr(eff_rank, torch.float64, "eff_rank"), _ptr(workspace, torch.uint8, "workspace"),
+        int(workspace.numel()), _stream(stream)))
+    return eff_rank
+
+
+def sparse_decode_classify_heads(eff_rank, num_kv_heads: int, num_retrieval_groups: int) -> list:
+    """head_is_retrieval of one layer from its heads' ER (host float64 [Hq])."""
+    er = torch.as_tensor(eff_rank, dtype=torch.float64).detach().cpu().contiguous()
+    out = torch.zeros(er.numel(), dtype=torch.int32)
+    _check(LIB.sparse_decode_classify_heads(er.data_ptr(), int(er.numel()), num_kv_heads, num_retrieval_groups,
+                                            out.data_ptr()))
+    return out.tolist()
 
 
 def sparse_decode_attend_noalloc(ctx: int, q, k_cache, v_cache, page_table, seq_lens, sel_idx, sel_count,

@@ -30,7 +30,8 @@ Readings taken where the page is silent or garbled (each is listed in the design doc)
     eps * lambda_max, so its square root only to about sqrt(eps) * sigma_max);
   * a head with no nonzero singular value has ER = exp(0) = 1 (the empty sum);
   * §4's "k lowest" is a count of GQA groups given by the caller; equal pooled
-    scores go to the lower group index.
+    scores go to the lower group index; a NaN score ranks after every number;
+    the pooled mean sums the group's heads in head order, then divides.
 
 Pins (``tests/test_classifier_pins.py``): closed forms of the entropy, weights
 built with a known spectrum (equal singular values, rank one, a prescribed
@@ -40,6 +41,7 @@ against each other on random weights.
 
 from __future__ import annotations
 
+import math
 from typing import Sequence
 
 import numpy as np
@@ -126,6 +128,8 @@ def classify_groups(eff_rank: Sequence[float], num_kv_heads: int, num_retrieval_
         for h in range(g * group, (g + 1) * group):    # in head order, one rounding per add
             total += float(er[h])
         pooled.append(total / group)
-    order = sorted(range(num_kv_heads), key=lambda g: (pooled[g], g))
+    # a NaN (no converged spectrum) ranks after every number
+    order = sorted(range(num_kv_heads), key=lambda g: (math.isnan(pooled[g]),
+                                                       0.0 if math.isnan(pooled[g]) else pooled[g], g))
     chosen = set(order[:num_retrieval_groups])
     return np.array([1 if h // group in chosen else 0 for h in range(er.size)], dtype=np.int32)

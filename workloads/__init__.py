@@ -2,3 +2,4 @@
 
 from .synthetic import (BUILDERS, WORKLOAD_NAMES, Workload, keys_at, make_workload,  # noqa: F401
                         slots_of)
+from .projections import ProjectionWeights, make_projections  # noqa: F401
