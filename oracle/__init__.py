@@ -8,3 +8,4 @@ imports it.
 
 from .sparse_decode_oracle import *  # noqa: F401,F403
 from .head_classifier_oracle import *  # noqa: F401,F403
+from .prefill_oracle import *  # noqa: F401,F403
