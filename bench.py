@@ -903,6 +903,227 @@ def classifier_cpu_baseline(p, budget_s: float = 15.0):
                       "eigenvalues of C_h per head"}
 
 
+# ---------------------------------------------------------------- head-wise prefill
+
+PREFILL_METRIC = "head-wise prefill tokens/s (retrieval heads dense causal, local heads sinks + window)"
+
+
+def load_bf16_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+def prefill_flops(w, chunk_lens) -> float:
+    """Algorithmic flops of a prefill: 4 d per (query, head, key seen) (Q K^T
+    and P V, two flops per multiply-add)."""
+    import numpy as np
+    total = 0.0
+    n_ret = sum(1 for x in w.head_is_retrieval if x)
+    n_loc = w.num_q_heads - n_ret
+    for n, t in zip(w.seq_lens.cpu().tolist(), chunk_lens):
+        pos = np.arange(n - t, n, dtype=np.float64)
+        total += n_ret * float(np.sum(pos + 1))                           # keys 0 .. pos
+        sinks = np.minimum(pos + 1, w.num_sinks)                           # keys [0, S) within [0, pos]
+        win = np.maximum(0.0, pos - np.maximum(w.num_sinks, pos - w.window + 1) + 1)
+        total += n_loc * float(np.sum(sinks + win))
+    return 4.0 * w.head_dim * total
+
+
+def prefill_workload(args, device, rank):
+    from workloads import make_workload
+    N = args.seq_len or 32768
+    return make_workload("llama3_8b_topp", device, B=1, N=N, permute=True,
+                         seed=rank_seed(1 if args.seed is None else args.seed, rank))
+
+
+def run_prefill(args):
+    import torch
+    import torch.distributed as dist
+
+    from head_wise_sparse_02_b200.sparse_decode import SparseDecode
+    from workloads import prefill_inputs
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    w = prefill_workload(args, dev, rank)
+    N = int(w.seq_lens[0])
+    sd = SparseDecode(num_q_heads=w.num_q_heads, num_kv_heads=w.num_kv_heads, head_dim=w.head_dim,
+                      head_is_retrieval=w.head_is_retrieval, num_pages=int(w.k_cache.shape[0]), max_batch=1,
+                      max_pages_per_seq=int(w.page_table.shape[1]), proj=w.proj, window=w.window,
+                      num_sinks=w.num_sinks, mode=w.mode, top_p=w.top_p)
+    q, starts = prefill_inputs(w, [N], seed=5)
+    out = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        sd.prefill(q, w.k_cache, w.v_cache, w.page_table, w.seq_lens, starts, out, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if sd.error_word():
+        raise RuntimeError("device error word set after warm-up")
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    pairs = []
+    for _ in range(args.steps):
+        flush_buf.zero_()
+        a0 = torch.cuda.Event(enable_timing=True); a1 = torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        step()
+        a1.record(stream)
+        pairs.append((a0, a1))
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms = sum(a.elapsed_time(b) for a, b in pairs) / args.steps
+    ms_max = max_over_ranks(ms, dev)
+
+    # dense causal attention of every head over the same keys (torch SDPA,
+    # bf16): the dense baseline the pages compare prefill against
+    G = w.num_q_heads // w.num_kv_heads
+    pages = w.page_table[0, :(N + 15) // 16].long()
+    Kc = w.k_cache[pages].permute(1, 0, 2, 3).reshape(w.num_kv_heads, -1, w.head_dim)[:, :N]
+    Vc = w.v_cache[pages].permute(1, 0, 2, 3).reshape(w.num_kv_heads, -1, w.head_dim)[:, :N]
+    Kd = Kc.repeat_interleave(G, dim=0)[None].contiguous()
+    Vd = Vc.repeat_interleave(G, dim=0)[None].contiguous()
+    Qd = q.permute(1, 0, 2)[None].contiguous()
+    dense = lambda: torch.nn.functional.scaled_dot_product_attention(Qd, Kd, Vd, is_causal=True)  # noqa: E731
+    for _ in range(2):
+        dense()
+    torch.cuda.synchronize()
+    d_pairs = []
+    for _ in range(max(1, args.steps // 2)):
+        flush_buf.zero_()
+        a0 = torch.cuda.Event(enable_timing=True); a1 = torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        dense()
+        a1.record(stream)
+        d_pairs.append((a0, a1))
+    torch.cuda.synchronize()
+    dense_ms = sum(a.elapsed_time(b) for a, b in d_pairs) / len(d_pairs)
+    del Kd, Vd, Qd
+
+    # end to end: queries from pinned host memory, the call, outputs back
+    q_h = q.cpu().pin_memory()
+    out_h = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+    q_d = torch.empty_like(q)
+
+    def e2e_step():
+        q_d.copy_(q_h, non_blocking=True)
+        sd.prefill(q_d, w.k_cache, w.v_cache, w.page_table, w.seq_lens, starts, out, stream)
+        out_h.copy_(out, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    t0 = torch.cuda.Event(enable_timing=True); t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, dev)
+
+    fl = prefill_flops(w, [N])
+    peak, kind = load_bf16_peak()
+    achieved = fl / (ms * 1e-3) / 1e12
+    tokens = ws * N
+    n_ret = sum(w.head_is_retrieval)
+    res = {
+        "metric": PREFILL_METRIC, "value": round(tokens / (ms_max * 1e-3), 1), "unit": "tokens/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "storage_dtype": "bf16",
+        "data": "synthetic (seeded; no datasets or trained weights)",
+        "config": {"workload": f"prefill_llama3_8b: B=1, N={N} full prefill, Hq={w.num_q_heads}/Hkv="
+                               f"{w.num_kv_heads}, d={w.head_dim}, {n_ret} retrieval heads (dense causal) + "
+                               f"{w.num_q_heads - n_ret} local (window {w.window} + {w.num_sinks} sinks)",
+                   "parallelism": f"replicas x{ws}", "l2": "flushed between steps (512 MiB write, untimed)"},
+        "roofline": {"kernel": "prefill_kernel", "bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
+                     "peak_kind": f"{kind} bf16_tflops (cuBLAS bf16 GEMM)", "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "algorithmic_flops_per_launch": fl, "traffic": None,
+                     "note": "P V runs as two bf16 MMAs (P split hi + lo): 1.5x the algorithmic MMA work"},
+        "dense_causal_sdpa_ms": round(dense_ms, 3),
+        "speedup_vs_dense_sdpa": round(dense_ms / ms, 3),
+        "e2e": {"value": round(tokens / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(q_h.numel() * 2), "d2h_bytes_per_step": int(out_h.numel() * 4)},
+        "gpu_launches": args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = prefill_cpu_baseline(w, q, starts, budget_s=args.cpu_budget)
+    sd.close()
+    if ws > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+def prefill_cpu_baseline(w, q, starts, budget_s: float = 15.0):
+    """The oracle on the host: query rows of the last positions (the longest
+    key ranges) for every head, until the budget runs out; tokens/s."""
+    import oracle as O
+    from oracle.workload_inputs import oracle_config, oracle_inputs
+    inp = oracle_inputs(w)
+    cfg = oracle_config(w)
+    qn = q.float().cpu().numpy()
+    st = starts.cpu().numpy()
+    total = int(st[-1])
+    done, t0 = 0, time.perf_counter()
+    r = total - 1
+    while r >= 0 and time.perf_counter() - t0 < budget_s:
+        O.prefill_reference(cfg, qn, inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_lens"], st,
+                            pairs=[(r, h) for h in range(w.num_q_heads)])
+        done += 1
+        r -= 1
+    el = time.perf_counter() - t0
+    return {"kind": "oracle", "value": round(done / el, 3), "unit": "tokens/s", "cores": _blas_threads(),
+            "sample": f"the last {done} query positions (all heads) of the same prefill, float64 numpy "
+                      "(the longest key ranges: a lower bound on the average rate)"}
+
+
+def run_prefill_reference(args):
+    """The oracle as the prefill's reference arm: each step one query position
+    (all heads) of the same prefill, from the last position down."""
+    ws, rank, local = dist_env()
+    if rank != 0:
+        return
+    import torch
+
+    from workloads import prefill_inputs
+    dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
+    w = prefill_workload(args, dev, 0)
+    N = int(w.seq_lens[0])
+    q, starts = prefill_inputs(w, [N], seed=5)
+    t = time.perf_counter()
+    base = prefill_cpu_baseline(w, q, starts, budget_s=args.cpu_budget)
+    el = time.perf_counter() - t
+    v = base["value"]
+    n_ret = sum(w.head_is_retrieval)
+    res = {"impl": "reference", "metric": PREFILL_METRIC, "value": v, "unit": "tokens/s", "n_gpus": ws,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 / v, 3) if v else None,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic (seeded; no datasets or trained weights)",
+           "config": {"workload": f"prefill_llama3_8b: B=1, N={N} full prefill, Hq={w.num_q_heads}/Hkv="
+                                  f"{w.num_kv_heads}, d={w.head_dim}, {n_ret} retrieval heads (dense causal) + "
+                                  f"{w.num_q_heads - n_ret} local (window {w.window} + {w.num_sinks} sinks)",
+                      "parallelism": f"replicas x{ws}", "l2": "flushed between steps (512 MiB write, untimed)"},
+           "cpu_baseline": dict(base, sample=base["sample"] + f"; {el:.1f} s"),
+           "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+
+
 def run_classifier_reference(args):
     """The oracle as the classifier's reference arm: each step one query head
     of the same synthetic weights by the eigenvalue route, on the host."""
@@ -978,7 +1199,12 @@ def main(argv=None):
     ap.add_argument("--layers", type=int, default=32, help="aoh_llama3_8b: layers classified per step")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)          # timing rule: at least 3 warm-up steps
-    if args.workload == "aoh_llama3_8b":
+    if args.workload == "prefill_llama3_8b":
+        if args.impl == "reference":
+            run_prefill_reference(args)
+        else:
+            run_prefill(args)
+    elif args.workload == "aoh_llama3_8b":
         if args.impl == "reference":
             run_classifier_reference(args)
         else:

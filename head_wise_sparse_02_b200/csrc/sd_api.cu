@@ -453,6 +453,30 @@ sd_status sparse_decode_select_attend_split(sd_ctx *ctx, const void *q_pre, cons
   }
 }
 
+sd_status sparse_decode_prefill(sd_ctx *ctx, const void *q, const void *k_cache, const void *v_cache,
+                                const int32_t *page_table, const int32_t *seq_lens, const int32_t *q_starts,
+                                int batch, int total_q, float *out, sd_stream stream) {
+  try {
+    if (!ctx) return SD_ERR_INVALID_ARG;
+    if (batch < 0 || batch > ctx->cfg.max_batch) return fail(ctx, SD_ERR_INVALID_ARG, "batch out of range");
+    if (total_q < 0) return fail(ctx, SD_ERR_INVALID_ARG, "total_q < 0");
+    if (batch == 0 || total_q == 0) return SD_OK;
+    if (!q || !k_cache || !v_cache || !page_table || !seq_lens || !q_starts || !out)
+      return fail(ctx, SD_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+      return fail(ctx, SD_ERR_INVALID_ARG, "q, the caches and out must be 16-byte aligned");
+    DeviceGuard dg(ctx->device);
+    const cudaError_t e = sd::launch_prefill(
+        static_cast<const uint16_t *>(q), static_cast<const uint16_t *>(k_cache),
+        static_cast<const uint16_t *>(v_cache), page_table, seq_lens, q_starts, batch, total_q, out,
+        ctx->attn_scale, ctx->cfg.window, ctx->cfg.num_sinks, ctx->sh, ctx->tb, ctx->err_d,
+        static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SD_OK : cuda_fail(ctx, e, "prefill launch");
+  } catch (...) {
+    return SD_ERR_HOST_MEMORY;
+  }
+}
+
 int sparse_decode_num_retrieval_groups(const sd_ctx *ctx) { return ctx ? ctx->tb.n_ret : 0; }
 
 int sparse_decode_num_local_groups(const sd_ctx *ctx) { return ctx ? ctx->tb.n_loc : 0; }

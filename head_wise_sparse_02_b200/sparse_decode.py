@@ -61,6 +61,7 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sparse_decode_select_attend_split": (c_int, [P, P, P, P, P, P, P, P, P, P, c_int, P, P, c_int, P, P,
                                                       c_size_t, P]),
         "sparse_decode_local_append": (c_int, [P, P, P, P, P, c_int, P, P, P]),
+        "sparse_decode_prefill": (c_int, [P, P, P, P, P, P, P, c_int, c_int, P, P]),
         "sparse_decode_num_retrieval_groups": (c_int, [P]),
         "sparse_decode_num_local_groups": (c_int, [P]),
         "sparse_decode_head_er_workspace_size": (c_int, [c_int, c_int, c_int, c_int, POINTER(c_size_t)]),
@@ -276,6 +277,23 @@ def sparse_decode_local_append(ctx: int, k_new, v_new, seq_ids, positions, local
         _ptr(local_k, torch.bfloat16, "local_k"), _ptr(local_v, torch.bfloat16, "local_v"), _stream(stream)), ctx)
 
 
+def sparse_decode_prefill(ctx: int, q, k_cache, v_cache, page_table, seq_lens, q_starts, out,
+                          stream=None) -> None:
+    """Head-wise prefill: q [total_q, Hq, d] packed by sequence (q_starts
+    [B + 1], device int32), out float32 of q's shape."""
+    B = int(seq_lens.numel())
+    if q_starts.numel() != B + 1:
+        raise ValueError(f"q_starts must hold batch + 1 = {B + 1} entries, got {q_starts.numel()}")
+    if q.dim() != 3 or tuple(out.shape) != tuple(q.shape):
+        raise ValueError(f"q must be [total_q, Hq, d] and out the same shape, got {tuple(q.shape)} / "
+                         f"{tuple(out.shape)}")
+    _check(LIB.sparse_decode_prefill(
+        ctx, _ptr(q, torch.bfloat16, "q"), _ptr(k_cache, torch.bfloat16, "k_cache"),
+        _ptr(v_cache, torch.bfloat16, "v_cache"), _ptr(page_table, torch.int32, "page_table"),
+        _ptr(seq_lens, torch.int32, "seq_lens"), _ptr(q_starts, torch.int32, "q_starts"), B, int(q.shape[0]),
+        _ptr(out, torch.float32, "out"), _stream(stream)), ctx)
+
+
 def sparse_decode_num_retrieval_groups(ctx: int) -> int:
     return int(LIB.sparse_decode_num_retrieval_groups(ctx))
 
@@ -426,6 +444,9 @@ class SparseDecode:
     def local_append(self, k_new, v_new, seq_ids, positions, local_k, local_v, stream=None):
         sparse_decode_local_append(self.handle, k_new, v_new, seq_ids, positions, local_k, local_v,
                                    self.cfg["max_batch"], stream)
+
+    def prefill(self, q, k_cache, v_cache, page_table, seq_lens, q_starts, out, stream=None):
+        sparse_decode_prefill(self.handle, q, k_cache, v_cache, page_table, seq_lens, q_starts, out, stream)
 
     def num_retrieval_groups(self) -> int:
         return sparse_decode_num_retrieval_groups(self.handle)

@@ -391,6 +391,38 @@ SD_API sd_status sparse_decode_select_attend_split(sd_ctx *ctx, const void *q_pr
                                             void *workspace, size_t ws_bytes, sd_stream stream);
 
 /*
+ * sparse_decode_prefill -- attention outputs of the queries of a prefill
+ * chunk (RTPurbo page, Methodology 1: retrieval heads keep their full KV
+ * through prefill, local heads use the sliding window with sinks; AoH page,
+ * Methodology 4: streaming heads keep sinks + a recent window, with chunked
+ * prefill).  Sequence b's chunk is its last T_b = q_starts[b+1] - q_starts[b]
+ * positions, N_b - T_b .. N_b - 1, whose keys and values are already in the
+ * caches (written by the caller, like every earlier position).  The query at
+ * position i of head h attends to
+ *
+ *   retrieval head  keys 0 .. i                              (dense causal)
+ *   local head      keys [0, num_sinks) U [i - window + 1, i], within [0, i]
+ *
+ * with one softmax over those keys (scale attn_scale, float32 accumulation;
+ * an empty set gives zeros).
+ *
+ *   q          device bf16 [total_q, Hq, d], post-RoPE queries packed by
+ *              sequence: sequence b's chunk at rows q_starts[b] ..
+ *              q_starts[b+1] - 1.
+ *   q_starts   device int32 [batch + 1], nondecreasing, q_starts[0] = 0,
+ *              q_starts[batch] = total_q, T_b <= N_b.
+ *   k_cache, v_cache, page_table, seq_lens   as described above (N_b =
+ *              seq_lens[b] includes the chunk).
+ *   out        device float32 [total_q, Hq, d], 16-byte aligned.
+ *
+ * No workspace.  A sequence whose q_starts or length is inconsistent sets
+ * SD_EBIT_SEQLEN and is skipped; page ids as for attend.
+ */
+SD_API sd_status sparse_decode_prefill(sd_ctx *ctx, const void *q, const void *k_cache, const void *v_cache,
+                                const int32_t *page_table, const int32_t *seq_lens, const int32_t *q_starts,
+                                int batch, int total_q, float *out, sd_stream stream);
+
+/*
  * sparse_decode_attend_noalloc -- sparse_decode_attend without a workspace
  * argument: the call uses a fixed scratch area compiled into the library
  * (64 MiB per device) and allocates nothing.  An addition of this library;

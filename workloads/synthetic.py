@@ -317,6 +317,21 @@ BUILDERS = {
 }
 
 
+def prefill_inputs(w: Workload, chunk_lens, seed: int = 0, scale: float = 1.0):
+    """Queries of a prefill chunk per sequence: the last chunk_lens[b] positions
+    of sequence b (clamped to its length), packed by sequence.  Returns
+    (q bf16 [total_q, Hq, d] drawn N(0, scale^2), q_starts int32 [B + 1])."""
+    lens = w.seq_lens.tolist()
+    t = [max(0, min(int(c), n)) for c, n in zip(chunk_lens, lens)]
+    starts = [0]
+    for x in t:
+        starts.append(starts[-1] + x)
+    dev = w.k_cache.device
+    q = (_randn_bf16((max(1, starts[-1]), w.num_q_heads, w.head_dim), _gen(dev, seed, 7), dev).float()
+         * scale).to(torch.bfloat16)[:starts[-1]].contiguous()
+    return q, torch.tensor(starts, dtype=torch.int32, device=dev)
+
+
 def make_workload(name: str, device="cuda", **overrides) -> Workload:
     return BUILDERS[name](device=device, **overrides)
 
