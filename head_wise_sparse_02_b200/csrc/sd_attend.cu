@@ -65,6 +65,7 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kTileRows = 16;
 constexpr int kTileRing = 3;            // tiles in flight per warp
 constexpr int kMaxGrid = 4096;          // persistent CTAs (partial slots are sized for this)
+constexpr int kMergeChunk = 64;         // partial slots weighed per step of the final merge
 
 // 16-byte copy global -> shared, bypassing L1, with an L2 eviction-priority
 // hint (see evict_first_policy)
@@ -823,24 +824,74 @@ attend_main_kernel(const AttendArgs a, const Shape sh, const Tables tb, const At
       __syncthreads();
       if (S.last) {
         __threadfence();
-        // the last segment of the item: merge partial slots first + item .. last + item
-        for (int x = tid; x < nh * D; x += kThreads) {
-          const int i = x / D, cc = x % D;
+        // the last segment of the item: merge partial slots first + item .. last
+        // + item.  Per head i the reference M_i = max_s m_s; then, kMergeChunk
+        // slots at a time, the weights f_is = 2^(m_s - M_i) (0 for an empty
+        // slot) go to shared memory and every output sums f_is o_s[cc] with
+        // independent loads (an item can span a few hundred CTAs)
+        const int np = (int)(last - first + 1);
+        constexpr long long PS = (long long)GR * (D + 2);            // stride of the partial slots
+        constexpr int OPT = (GR * D + kThreads - 1) / kThreads;     // outputs per thread, at most
+        const float *pbase = ws.partials + (first + item) * PS;
+        float *fw = reinterpret_cast<float *>(dyn);                  // [GR][kMergeChunk]
+        float *sM = fw + GR * kMergeChunk;                           // [GR]
+        float *sden = sM + GR;                                       // [GR]
+        for (int i = warp; i < nh; i += kWarps) {
           float M = -INFINITY;
-          for (long long s = first; s <= last; ++s)
-            M = fmaxf(M, __ldcg(ws.partials + ((s + item) * GR + i) * (long long)(D + 2)));
-          float num = 0.0f, den = 0.0f;
-          if (M > -INFINITY) {
-            for (long long s = first; s <= last; ++s) {
-              const float *pp = ws.partials + ((s + item) * GR + i) * (long long)(D + 2);
-              const float ms = __ldcg(pp);
-              if (ms == -INFINITY) continue;
-              const float f = exp2f(ms - M);
-              den = fmaf(f, __ldcg(pp + 1), den);
-              num = fmaf(f, __ldcg(pp + 2 + cc), num);
+          for (int s = lane; s < np; s += 32) M = fmaxf(M, __ldcg(pbase + s * PS + i * (D + 2)));
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, off));
+          if (lane == 0) {
+            sM[i] = M;
+            sden[i] = 0.0f;
+          }
+        }
+        float num[OPT];
+#pragma unroll
+        for (int u = 0; u < OPT; ++u) num[u] = 0.0f;
+        for (int s0 = 0; s0 < np; s0 += kMergeChunk) {
+          const int nc = np - s0 < kMergeChunk ? np - s0 : kMergeChunk;
+          __syncthreads();                             // M ready; the previous chunk's weights consumed
+          for (int x = tid; x < nh * kMergeChunk; x += kThreads) {
+            const int i = x / kMergeChunk, sl = x % kMergeChunk;
+            float f = 0.0f;
+            if (sl < nc) {
+              const float ms = __ldcg(pbase + (s0 + sl) * PS + i * (D + 2));
+              f = (ms == -INFINITY || sM[i] == -INFINITY) ? 0.0f : exp2f(ms - sM[i]);
+            }
+            fw[i * kMergeChunk + sl] = f;
+          }
+          __syncthreads();
+          for (int i = warp; i < nh; i += kWarps) {
+            float dsum = 0.0f;
+            for (int sl = lane; sl < nc; sl += 32)
+              dsum = fmaf(fw[i * kMergeChunk + sl], __ldcg(pbase + (s0 + sl) * PS + i * (D + 2) + 1), dsum);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) dsum += __shfl_xor_sync(kFull, dsum, off);
+            if (lane == 0) sden[i] += dsum;
+          }
+#pragma unroll
+          for (int u = 0; u < OPT; ++u) {
+            const int x = tid + u * kThreads;
+            if (x < nh * D) {
+              const int i = x / D, cc = x % D;
+              const float *pp = pbase + s0 * PS + i * (D + 2) + 2 + cc;
+              const float *fi = fw + i * kMergeChunk;
+              float acc = num[u];
+#pragma unroll 8
+              for (int sl = 0; sl < nc; ++sl) acc = fmaf(fi[sl], __ldcg(pp + sl * PS), acc);
+              num[u] = acc;
             }
           }
-          a.out[((long long)b * sh.Hq + S.grp.q_head[i]) * D + cc] = den > 0.0f ? num / den : 0.0f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int u = 0; u < OPT; ++u) {
+          const int x = tid + u * kThreads;
+          if (x < nh * D) {
+            const int i = x / D, cc = x % D;
+            a.out[((long long)b * sh.Hq + S.grp.q_head[i]) * D + cc] = sden[i] > 0.0f ? num[u] / sden[i] : 0.0f;
+          }
         }
       }
     }
@@ -943,7 +994,8 @@ cudaError_t launch_t(const AttendArgs &a, const Shape &sh, const Tables &tb, con
   if (e != cudaSuccess) return e;
   const size_t ring = (size_t)kWarps * kTileRing * (2 * kTileRows * (2 * D + 16));
   const size_t lists = (size_t)kWarps * kTileRing * kTileRows * 2 + (size_t)(p.ns + 1) * 4;
-  const size_t merge = (size_t)kWarps * 32 * 4 + (size_t)kWarps * GR * D * 4;
+  const size_t merge = std::max((size_t)kWarps * 32 * 4 + (size_t)kWarps * GR * D * 4,
+                                (size_t)GR * (kMergeChunk + 2) * 4);
   const size_t bytes = std::max(ring + lists, merge);
   e = set_smem(attend_main_kernel<D, GR>, bytes);
   if (e != cudaSuccess) return e;
