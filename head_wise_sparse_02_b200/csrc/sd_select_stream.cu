@@ -75,7 +75,7 @@ constexpr int kBins = 512;            // window histogram bins (+1 slot: scores 
 // K0: sampled pages per (sequence, group); the sample store is capped at 96 KB
 __host__ __device__ constexpr int sample_pages(int GR) { return GR <= 4 ? 256 : (GR == 8 ? 192 : 96); }
 constexpr int kSampleBins = 256;
-constexpr int kChunkPages = 512;      // K1: pages per CTA
+constexpr int kChunkPages = 512;      // K1: pages per CTA (at most; fewer when the items are few)
 constexpr int kRing = 8;              // K1: pages in flight per warp (even); 4 CTAs per SM
 // K1: staged buffer entries per (lane, head block); an iteration adds <= 4
 __host__ __device__ constexpr int stage_lane(int GR) { return GR <= 4 ? 10 : (GR == 8 ? 8 : 5); }
@@ -604,7 +604,7 @@ __host__ __device__ constexpr size_t stream_smem_bytes(int GR, int MODE) {
 template <int GR, int MODE>
 __global__ void __launch_bounds__(kT1)
 stream_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__ groups, int n_groups,
-              const StreamWs ws) {
+              const StreamWs ws, int chunk) {
   constexpr int HB = (GR + 3) / 4;
   constexpr int SL = stage_lane(GR);
   constexpr bool TOPP = MODE != kStageTopk;
@@ -637,9 +637,9 @@ stream_kernel(const SelectArgs a, const Shape sh, const Group *__restrict__ grou
   N = N < 0 ? 0 : std::min<long long>(N, sh.max_len);
   if (keeps_all<TOPP>(a, N)) return;
   const int pages = (int)((N + kPage - 1) / kPage);
-  const int p0 = blockIdx.y * kChunkPages;
+  const int p0 = blockIdx.y * chunk;                 // chunk: a multiple of 64 pages, at most kChunkPages
   if (p0 >= pages) return;
-  const int np = pages - p0 < kChunkPages ? pages - p0 : kChunkPages;
+  const int np = pages - p0 < chunk ? pages - p0 : chunk;
   {
     // page id -> page * Hkv + g (the 512-byte index block of this KV head), or -1
     const int32_t *pt = a.page_table + (long long)b * sh.max_pages + p0;
@@ -1467,6 +1467,17 @@ cudaError_t set_smem_once(K kern, size_t bytes) {
 // heads per group whose bitmaps and scratch fit in one CTA, and enough items
 // to fill half the multiprocessors, the resolve with the group's union list
 // (*unioned).
+// SMs of the current device (looked up once; 1 if the query fails)
+int sm_count() {
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
+      sms = n;
+  }
+  return std::max(sms, 1);
+}
+
 template <bool TOPP, int GR>
 cudaError_t launch_resolve(const SelectArgs &a, const Shape &sh, const Tables &tb, const StreamWs &ws,
                            size_t bitmap_bytes, const UnionOut *uo, bool *unioned, cudaStream_t st) {
@@ -1477,13 +1488,7 @@ cudaError_t launch_resolve(const SelectArgs &a, const Shape &sh, const Tables &t
   if (unioned) *unioned = false;
   // one CTA per item: worth it when the items fill at least half the GPU
   // (fewer, and the per-head CTAs' parallelism wins)
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0, n = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
-      sms = n;
-  }
-  if (uo && GR <= 4 && ubytes <= 227 * 1024 && 2 * a.batch * tb.n_ret >= std::max(sms, 1)) {
+  if (uo && GR <= 4 && ubytes <= 227 * 1024 && 2 * a.batch * tb.n_ret >= sm_count()) {
     auto *kern = resolve_union_kernel<TOPP, NG>;
     cudaError_t e = set_smem_once(kern, ubytes);
     if (e != cudaSuccess) return e;
@@ -1502,7 +1507,11 @@ cudaError_t stream_launch(const SelectArgs &a, const Shape &sh, const Tables &tb
                           size_t bitmap_bytes, const UnionOut *uo, bool *unioned, cudaStream_t st) {
   const bool topp = a.mode == SD_TOP_P;
   const int items = a.batch * tb.n_ret;
-  const int chunks = (int)((sh.max_pages + kChunkPages - 1) / kChunkPages);
+  // pages per K1 CTA: 512, or fewer (a multiple of 64) when items x chunks
+  // would leave SMs idle, so that small batches still spread over the GPU
+  int chunk = kChunkPages;
+  while (chunk > 64 && (long long)items * ((sh.max_pages + chunk - 1) / chunk) < 2LL * sm_count()) chunk /= 2;
+  const int chunks = (int)((sh.max_pages + chunk - 1) / chunk);
   const dim3 g1(items, chunks);
   const size_t smem0 = (size_t)GR * sample_pages(GR) * 16 * 4 + (size_t)GR * kSampleBins * 4 * (topp ? 2 : 1);
   cudaError_t e;
@@ -1513,7 +1522,7 @@ cudaError_t stream_launch(const SelectArgs &a, const Shape &sh, const Tables &tb
     if (e != cudaSuccess) return e;
     e = launch_pdl(window_kernel<GR, false>, dim3(items), dim3(kT0), smem0, st, 0, a, sh, tb.ret, tb.n_ret, ws);
     if (e == cudaSuccess)
-      e = launch_pdl(stream_kernel<GR, kStageTopk>, g1, dim3(kT1), smem1, st, 0, a, sh, tb.ret, tb.n_ret, ws);
+      e = launch_pdl(stream_kernel<GR, kStageTopk>, g1, dim3(kT1), smem1, st, 0, a, sh, tb.ret, tb.n_ret, ws, chunk);
     if (e == cudaSuccess) e = launch_resolve<false, GR>(a, sh, tb, ws, bitmap_bytes, uo, unioned, st);
     return e;
   }
@@ -1524,9 +1533,9 @@ cudaError_t stream_launch(const SelectArgs &a, const Shape &sh, const Tables &tb
   if (e != cudaSuccess) return e;
   e = launch_pdl(window_kernel<GR, true>, dim3(items), dim3(kT0), smem0, st, 0, a, sh, tb.ret, tb.n_ret, ws);
   if (e == cudaSuccess)
-    e = launch_pdl(stream_kernel<GR, kMassTopp>, g1, dim3(kT1), smem_m, st, 0, a, sh, tb.ret, tb.n_ret, ws);
+    e = launch_pdl(stream_kernel<GR, kMassTopp>, g1, dim3(kT1), smem_m, st, 0, a, sh, tb.ret, tb.n_ret, ws, chunk);
   if (e == cudaSuccess)
-    e = launch_pdl(stream_kernel<GR, kCutTopp>, g1, dim3(kT1), smem_c, st, 0, a, sh, tb.ret, tb.n_ret, ws);
+    e = launch_pdl(stream_kernel<GR, kCutTopp>, g1, dim3(kT1), smem_c, st, 0, a, sh, tb.ret, tb.n_ret, ws, chunk);
   if (e == cudaSuccess) e = launch_resolve<true, GR>(a, sh, tb, ws, bitmap_bytes, uo, unioned, st);
   return e;
 }
