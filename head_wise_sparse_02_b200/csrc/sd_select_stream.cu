@@ -1385,13 +1385,19 @@ resolve_union_kernel(const SelectArgs a, const Shape sh, const StreamWs ws, cons
         hw[i] = (x < x_hi && i < nr) ? bitmap_of(i)[x] : 0u;
         u |= hw[i];
       }
+      // the two pages of this lane's word, loaded before the emission needs
+      // them (pages at or past the sequence's end are never read)
+      const long long q0 = (long long)x * 32;
+      const int pg0 = (x < x_hi && q0 < N) ? pt[q0 >> 4] : -1;
+      const int pg1 = (x < x_hi && q0 + 16 < N) ? pt[(q0 >> 4) + 1] : -1;
       off += (uint32_t)warp_emit_bits(u, lane, [&](bool valid, int kk, int w, int bit) {
         uint32_t m = 0;
 #pragma unroll
         for (int i = 0; i < NG; ++i) m |= ((__shfl_sync(kFull, hw[i], w) >> bit) & 1u) << i;   // every lane
+        const int pa = __shfl_sync(kFull, pg0, w), pb = __shfl_sync(kFull, pg1, w);
         if (!valid) return;
         const int pos = (xb + w) * 32 + bit;
-        const int page = pt[pos >> 4];
+        const int page = bit < 16 ? pa : pb;
         const bool ok = page >= 0 && page < sh.num_pages;
         bad_page |= !ok;
         rows[off + kk] = ok ? (uint32_t)page * row_page + row_g + (uint32_t)(pos & (kPage - 1)) : 0u;
