@@ -1240,12 +1240,32 @@ __device__ bool resolve_topp(const SelectArgs &a, const Shape &sh, const StreamW
         S.dmass[o] = 0.0;
       }
       hg.sync();
-      for (int e = tid; e < n; e += kT2) {
-        const uint32_t key = (uint32_t)(S.cand[e] >> 32), off = key - kmin;
-        if (rem != top && (off >> rem) != prefix) continue;
-        const uint32_t d = (off >> sh2) & ((1u << (rem - sh2)) - 1u);
-        atomicAdd(&S.dcnt[d], 1u);
-        atomicAdd(&S.dmass[d], (double)exp2f((key_to_float(key) - thi) * kLog2e));
+      // lanes of a warp holding the same digit add their count and mass
+      // first, and one of them updates the shared bins (the candidates of a
+      // cut bin crowd into a few digits at the first levels)
+      for (int e0 = 0; e0 < n; e0 += kT2) {
+        const int e = e0 + tid;
+        bool part = false;
+        uint32_t d = 0u;
+        double wt = 0.0;
+        if (e < n) {
+          const uint32_t key = (uint32_t)(S.cand[e] >> 32), off = key - kmin;
+          part = rem == top || (off >> rem) == prefix;
+          if (part) {
+            d = (off >> sh2) & ((1u << (rem - sh2)) - 1u);
+            wt = (double)exp2f((key_to_float(key) - thi) * kLog2e);
+          }
+        }
+        const unsigned pm = __ballot_sync(kFull, part);
+        if (part) {
+          const unsigned peers = __match_any_sync(pm, d);
+          double sum = 0.0;
+          for (unsigned m = peers; m; m &= m - 1u) sum += __shfl_sync(peers, wt, __ffs(m) - 1);
+          if (lane == __ffs(peers) - 1) {
+            atomicAdd(&S.dcnt[d], (uint32_t)__popc(peers));
+            atomicAdd(&S.dmass[d], sum);
+          }
+        }
       }
       hg.sync();
       if (warp == 0) {
