@@ -66,6 +66,7 @@ constexpr int kTileRows = 16;
 constexpr int kTileRing = 3;            // tiles in flight per warp
 constexpr int kMaxGrid = 4096;          // persistent CTAs (partial slots are sized for this)
 constexpr int kMergeChunk = 64;         // partial slots weighed per step of the final merge
+constexpr int kDensePlanBits = 256;     // union bits per warp step above which lanes write their own rows
 
 // 16-byte copy global -> shared, bypassing L1, with an L2 eviction-priority
 // hint (see evict_first_policy)
@@ -373,6 +374,34 @@ __device__ void plan_span(const AttendArgs &a, const Shape &sh, const Tables &tb
     for (int i = 0; i < GR; ++i) {
       hw[i] = (x < bwords && i < nh) ? hbm[i * bwords + x] : 0u;
       u |= hw[i];
+    }
+    const int nl = __popc(u);
+    const int step_bits = __reduce_add_sync(kFull, (unsigned)nl);
+    if (step_bits >= kDensePlanBits) {
+      // dense run: each lane writes the rows of its own word's bits
+      int incl = nl;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int y = __shfl_up_sync(kFull, incl, d);
+        if (lane >= d) incl += y;
+      }
+      uint32_t at = o + (uint32_t)(incl - nl);
+      uint32_t bits = u;
+      while (bits) {
+        const int bit = __ffs(bits) - 1;
+        bits &= bits - 1u;
+        uint32_t m = 0;
+#pragma unroll
+        for (int i = 0; i < GR; ++i) m |= ((hw[i] >> bit) & 1u) << i;
+        const int off = x * 32 + bit;
+        const int page = pslice[off >> 4];
+        bad_page |= page < 0;
+        rows[at] = page >= 0 ? (uint32_t)page * row_page + row_g + (uint32_t)(off & (kPage - 1)) : 0u;
+        masks[at] = (uint16_t)(page >= 0 ? m : 0u);
+        ++at;
+      }
+      o += (uint32_t)step_bits;
+      continue;
     }
     // union rows handed out 32 at a time: each store writes consecutive entries
     o += (uint32_t)warp_emit_bits(u, lane, [&](bool valid, int k, int w, int bit) {

@@ -179,6 +179,32 @@ __global__ void __launch_bounds__(kThreads) cholesky_kernel(double *__restrict__
     for (int j = lane; j < D; j += 32) G[i * D + j] = j <= i ? at(i, j) : 0.0;
 }
 
+// Rotation of a column pair (alpha = |x_p|^2, beta = |x_q|^2, gamma = x_p.x_q)
+// that makes the pair orthogonal: tan = t, the root of t^2 + 2 zeta t - 1 = 0
+// of smaller magnitude, zeta = (beta - alpha) / (2 gamma) (Rutishauser's
+// form).  t is taken in float32 (fast reciprocal and root): an angle off by
+// ~1e-7 relative only leaves a residual gamma ~1e-7 times the old one for a
+// later sweep.  cos = (1 + t^2)^(-1/2) must keep cos^2 + sin^2 = 1 to float64
+// rounding (the rotations must preserve the column norms), so it starts from
+// the float32 reciprocal square root and takes two Newton steps in float64,
+// y <- y (3 - x y^2) / 2, each squaring the relative error (1e-7 -> 1e-14 ->
+// below double rounding).  Returns cos; *t gets the tangent.
+__device__ __forceinline__ double rot_cos(double alpha, double beta, double gamma, double &t) {
+  const float den = 2.0f * (float)gamma;
+  float tf = 0.0f;                                   // gamma below float range: no rotation
+  if (den != 0.0f) {
+    const float zeta = (float)(beta - alpha) / den;
+    const float az = fabsf(zeta);
+    tf = (zeta >= 0.0f ? 1.0f : -1.0f) / (az + sqrtf(fmaf(az, az, 1.0f)));   // 0 when zeta^2 overflows
+  }
+  t = (double)tf;
+  const double x = fma(t, t, 1.0);
+  double y = (double)rsqrtf((float)x);
+  y = y * fma(-0.5 * x * y, y, 1.5);
+  y = y * fma(-0.5 * x * y, y, 1.5);
+  return y;
+}
+
 template <int D>
 __host__ __device__ constexpr size_t jacobi_smem() {
   return (size_t)D * D * sizeof(double) + 2 * (size_t)16 * D * sizeof(double);
@@ -246,7 +272,7 @@ jacobi_kernel(const double *__restrict__ gram, int Hq, int Hkv, double *__restri
   for (int sweep = 0; sweep < kMaxSweeps && !converged; ++sweep) {
     int rotated = 0;
     for (int r = 0; r < D - 1; ++r) {
-      double al[PPW], be[PPW], ga[PPW];
+      double al[PPW], be[PPW], ga[PPW], t_of[PPW];
       int cp[PPW], cq[PPW];
 #pragma unroll
       for (int j = 0; j < PPW; ++j) {
@@ -273,9 +299,8 @@ jacobi_kernel(const double *__restrict__ gram, int Hq, int Hkv, double *__restri
 #pragma unroll
       for (int j = 0; j < PPW; ++j) {
         if (ga[j] * ga[j] > tol2 * (al[j] * be[j])) {  // |gamma| > tol sqrt(alpha beta), without the root
-          const double zeta = (be[j] - al[j]) / (2.0 * ga[j]);
-          const double t = (zeta >= 0.0 ? 1.0 : -1.0) / (fabs(zeta) + sqrt(1.0 + zeta * zeta));
-          const double c = rsqrt(1.0 + t * t), s = c * t;
+          const double c = rot_cos(al[j], be[j], ga[j], t_of[j]);
+          const double s = c * t_of[j];
 #pragma unroll
           for (int e = 0; e < RPL; ++e) {
             double *xp = Xc + cp[j] * D + lane + 32 * e, *xq = Xc + cq[j] * D + lane + 32 * e;

@@ -75,6 +75,9 @@ constexpr int kBins = 512;            // window histogram bins (+1 slot: scores 
 // K0: sampled pages per (sequence, group); the sample store is capped at 96 KB
 __host__ __device__ constexpr int sample_pages(int GR) { return GR <= 4 ? 256 : (GR == 8 ? 192 : 96); }
 constexpr int kSampleBins = 256;
+// set bits per warp step above which write_ascending's lanes write their own
+// bits (the union lists keep the coalesced emission: measured faster there)
+constexpr int kDenseBits = 256;
 constexpr int kChunkPages = 512;      // K1: pages per CTA (at most; fewer when the items are few)
 constexpr int kRing = 8;              // K1: pages in flight per warp (even); 4 CTAs per SM
 // K1: staged buffer entries per (lane, head block); an iteration adds <= 4
@@ -891,13 +894,42 @@ __device__ void write_ascending(const SelectArgs &a, const HeadGroup &hg, const 
     const int x0 = w0 + r * 32 * WPL;
     uint32_t v[WPL];
     load(x0 + lane * WPL, v);
-    off += warp_emit_bits_w<WPL>(v, lane, [&](bool valid, int k, int w, int j, int bit) {
-      const long long o = off + k;
-      if (valid) {
-        if (o < a.sel_stride) out[o] = (x0 + w * WPL + j) * 32 + bit;
-        else over = true;
+    int nl = 0;
+#pragma unroll
+    for (int j = 0; j < WPL; ++j) nl += __popc(v[j]);
+    const int step_bits = __reduce_add_sync(kFull, (unsigned)nl);
+    if (step_bits >= kDenseBits) {
+      // dense run: each lane writes its own bits (consecutive slots per lane),
+      // far fewer instructions than handing bits out 32 at a time
+      int incl = nl;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += y;
       }
-    });
+      long long o = off + incl - nl;
+#pragma unroll
+      for (int j = 0; j < WPL; ++j) {
+        uint32_t bits = v[j];
+        const int base = (x0 + lane * WPL + j) * 32;
+        while (bits) {
+          const int bit = __ffs(bits) - 1;
+          bits &= bits - 1u;
+          if (o < a.sel_stride) out[o] = base + bit;
+          else over = true;
+          ++o;
+        }
+      }
+      off += step_bits;
+    } else {
+      off += warp_emit_bits_w<WPL>(v, lane, [&](bool valid, int k, int w, int j, int bit) {
+        const long long o = off + k;
+        if (valid) {
+          if (o < a.sel_stride) out[o] = (x0 + w * WPL + j) * 32 + bit;
+          else over = true;
+        }
+      });
+    }
   }
   if (over) raise_error(a.err, SD_EBIT_SEL);
   if (hg.t == 0) {
