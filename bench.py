@@ -167,6 +167,9 @@ KERNEL_SOURCES = {
                "head_wise_sparse_02_b200/csrc/sd_internal.cuh"],
     "attend": ["head_wise_sparse_02_b200/csrc/sd_attend.cu", "head_wise_sparse_02_b200/csrc/sd_internal.cuh"],
     "index_keys": ["head_wise_sparse_02_b200/csrc/sd_index.cu", "head_wise_sparse_02_b200/csrc/sd_internal.cuh"],
+    # the joined call: the selection and attend kernels one step launches
+    "select_attend": ["head_wise_sparse_02_b200/csrc/sd_select.cu", "head_wise_sparse_02_b200/csrc/sd_select_stream.cu",
+                      "head_wise_sparse_02_b200/csrc/sd_attend.cu", "head_wise_sparse_02_b200/csrc/sd_internal.cuh"],
 }
 
 
