@@ -308,6 +308,11 @@ cudaError_t launch_prefill(const uint16_t *q, const uint16_t *k_cache, const uin
                            int total_q, float *out, float attn_scale, int window, int num_sinks, const Shape &sh,
                            const Tables &tb, unsigned *err, cudaStream_t st);
 
+cudaError_t launch_prefill_tc(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                              const int32_t *page_table, const int32_t *seq_lens, const int32_t *q_starts, int batch,
+                              int total_q, float *out, float attn_scale, int window, int num_sinks, const Shape &sh,
+                              const Tables &tb, unsigned *err, cudaStream_t st);
+
 cudaError_t launch_local_append(const uint16_t *k_new, const uint16_t *v_new, const int32_t *seq_ids,
                                 const int32_t *positions, int T, uint16_t *local_k, uint16_t *local_v,
                                 const Shape &sh, const Tables &tb, int max_batch, int num_sinks, int window,

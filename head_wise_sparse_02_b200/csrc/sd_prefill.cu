@@ -197,19 +197,24 @@ prefill_kernel(const PrefillArgs a, const Shape sh, const Tables tb) {
   auto issue = [&](int kt, int st) {
     const uint32_t kdst = sbase + st * (uint32_t)stage_bytes<D>();
     const uint32_t vdst = kdst + kKT * PITCH;
+    // the tile's four page ids first (independent loads), then the copies
+    int pg[kKT / kPage];
+#pragma unroll
+    for (int u = 0; u < kKT / kPage; ++u) {
+      const long long key = (long long)kt * kKT + u * kPage;
+      int page = key <= p_last ? pt[key / kPage] : -1;
+      if (key <= p_last && (page < 0 || page >= sh.num_pages)) {
+        raise_error(a.err, SD_EBIT_PAGE);
+        page = -1;
+      }
+      pg[u] = page;
+    }
 #pragma unroll
     for (int x = 0; x < kKT * CPR / kThreads; ++x) {
       const int c = tid + kThreads * x;
       const int r = c / CPR, ch = c % CPR;
       const long long key = (long long)kt * kKT + r;
-      int page = -1;
-      if (key <= p_last) {
-        page = pt[key / kPage];
-        if (page < 0 || page >= sh.num_pages) {
-          raise_error(a.err, SD_EBIT_PAGE);
-          page = -1;
-        }
-      }
+      const int page = key <= p_last ? pg[r / kPage] : -1;
       const size_t off = page >= 0 ? (((size_t)page * sh.Hkv + g) * kPage + (size_t)(key % kPage)) * (2 * D) + ch * 16 : 0;
       const int bytes = page >= 0 ? 16 : 0;          // rows past p_last or on a bad page are zero-filled
       cp_async16(kdst + r * PITCH + ch * 16, reinterpret_cast<const unsigned char *>(a.k_cache) + off, bytes);
@@ -390,9 +395,13 @@ cudaError_t launch_prefill(const uint16_t *q, const uint16_t *k_cache, const uin
                            int total_q, float *out, float attn_scale, int window, int num_sinks, const Shape &sh,
                            const Tables &tb, unsigned *err, cudaStream_t st) {
   if (batch == 0 || total_q == 0 || tb.n_ret + tb.n_loc == 0) return cudaSuccess;
+  // d = 128 runs on the tcgen05 kernel (sd_prefill_tc.cu); this mma.sync one serves d = 64
+  if (sh.d == 128)
+    return launch_prefill_tc(q, k_cache, v_cache, page_table, seq_lens, q_starts, batch, total_q, out, attn_scale,
+                             window, num_sinks, sh, tb, err, st);
   PrefillArgs a{q, k_cache, v_cache, page_table, seq_lens, q_starts, out, attn_scale, window, num_sinks, batch,
                 total_q, err};
-  return sh.d == 128 ? launch_d<128>(a, sh, tb, total_q, st) : launch_d<64>(a, sh, tb, total_q, st);
+  return launch_d<64>(a, sh, tb, total_q, st);
 }
 
 }  // namespace sd

@@ -83,6 +83,28 @@ def test_llama3_8b_shapes_sampled_rows():
     _run(w, [4096], rows=rows, label="llama3 4096")
 
 
+@pytest.mark.parametrize("scale", [0.25, 4.0])
+def test_peaked_and_flat_softmax(scale):
+    """Query scales that make the softmax nearly flat (0.25) or sharply peaked
+    with row maxima jumping between key tiles (4.0: the running maximum moves
+    and the partial outputs are rescaled), 700 positions, ragged pages."""
+    from workloads.synthetic import _base
+    w = _base("scaled", 12, "cuda", [700, 300], 8, 2, 128, [1, 1, 0, 0, 1, 0, 0, 1], 160, 4, "top_p", permute=True)
+    sd = _ctx(w)
+    q, starts = prefill_inputs(w, [700, 250], seed=4, scale=scale)
+    out = torch.full(q.shape, float("nan"), dtype=torch.float32, device="cuda")
+    sd.prefill(q, w.k_cache, w.v_cache, w.page_table, w.seq_lens, starts, out)
+    torch.cuda.synchronize()
+    assert sd.error_word() == 0
+    inp = oracle_inputs(w)
+    ref = O.prefill_reference(oracle_config(w), q.float().cpu().numpy(), inp["k_cache"], inp["v_cache"],
+                              inp["page_table"], inp["seq_lens"], starts.cpu().numpy())
+    got = out.cpu().numpy()
+    for (r, h), o in ref.items():
+        assert_out_close(got[r, h], o, f"scale {scale} row={r} h={h}")
+    sd.close()
+
+
 def test_inconsistent_chunk_sets_error_word_without_fault():
     from head_wise_sparse_02_b200.sparse_decode import SD_EBIT_SEQLEN
     w = make_workload("tiny_ref", "cuda", N=100)
