@@ -204,6 +204,7 @@ prefill_tc_kernel(const TcArgs a, const Shape sh, const Tables tb) {
   __shared__ __align__(8) uint64_t mbar[2];          // 0: S ready, 1: P V done
   __shared__ uint32_t tslot;
   __shared__ int s_b, s_t, s_bad;
+  __shared__ int s_pg[128 * (kN / kPage)];
   __shared__ Group s_grp;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gr = blockIdx.y, hidx = blockIdx.z;
@@ -276,27 +277,36 @@ prefill_tc_kernel(const TcArgs a, const Shape sh, const Tables tb) {
       cp_async16(sbase + kOffQ + (r >> 3) * 2048 + c8 * 128 + (r & 7) * 16, src, ok ? 16 : 0);
     }
   }
-  // the four pages of key tile kt, looked up once (one round of independent
-  // loads) before any copy is issued: -1 past p_last or for a bad page id
-  auto tile_pages = [&](int kt, int (&pg)[kN / kPage]) {
-#pragma unroll
-    for (int u = 0; u < kN / kPage; ++u) {
-      const long long key = (long long)kt * kN + u * kPage;
-      int page = key <= p_last ? pt[key / kPage] : -1;
-      if (key <= p_last && (page < 0 || page >= sh.num_pages)) {
-        raise_error(a.err, SD_EBIT_PAGE);
-        page = -1;
+  // Page ids of the CTA's key tiles, 4 per tile, in a shared ring of 128
+  // tiles filled 64 tiles at a time, 64 tiles ahead of their copies, so that
+  // no page-table load sits on the path of a tile (-1: past p_last or a bad id)
+  auto fill_pages = [&](int t0) {
+    for (int e = tid; e < 64 * (kN / kPage); e += kThreads) {
+      const int t = t0 + e / (kN / kPage), u = e % (kN / kPage);
+      int val = -1;
+      if (t < ntiles) {
+        const long long key = (long long)tr.at(t) * kN + u * kPage;
+        if (key <= p_last) {
+          val = pt[key / kPage];
+          if (val < 0 || val >= sh.num_pages) {
+            raise_error(a.err, SD_EBIT_PAGE);
+            val = -1;
+          }
+        }
       }
-      pg[u] = page;
+      s_pg[(t & 127) * (kN / kPage) + u] = val;
     }
   };
+  fill_pages(0);
+  fill_pages(64);
+  __syncthreads();
   // Copies of a tile: thread tid takes the 16-byte chunk c8 = tid % 16 of rows
   // r0 + 8 x (r0 = tid / 16, x < 8), so its rows are r0 and r0 + 8 of the tile's
   // four pages and its shared-memory offsets are fixed up to x.
   const int r0 = tid >> 4, c8 = tid & 15;
-  auto issue_kv = [&](int kt, const uint16_t *cache, uint32_t dst0, uint32_t xstride) {
-    int pg[kN / kPage];
-    tile_pages(kt, pg);
+  auto issue_kv = [&](int t, const uint16_t *cache, uint32_t dst0, uint32_t xstride) {
+    const int kt = tr.at(t);
+    const int *pg = s_pg + (t & 127) * (kN / kPage);
     const unsigned char *base = reinterpret_cast<const unsigned char *>(cache) + c8 * 16;
 #pragma unroll
     for (int x = 0; x < 8; ++x) {
@@ -309,17 +319,17 @@ prefill_tc_kernel(const TcArgs a, const Shape sh, const Tables tb) {
     }
   };
   // K: K-major (8-row group x -> 2048 bytes); V: MN-major (8-key group x -> 128 bytes)
-  auto issue_k = [&](int kt, int buf) {
-    issue_kv(kt, a.k_cache, sbase + kOffK + buf * kKBytes + c8 * 128 + r0 * 16, 2048u);
+  auto issue_k = [&](int t, int buf) {                // t: position in the CTA's tile list
+    issue_kv(t, a.k_cache, sbase + kOffK + buf * kKBytes + c8 * 128 + r0 * 16, 2048u);
   };
-  auto issue_v = [&](int kt, int buf) {
-    issue_kv(kt, a.v_cache, sbase + kOffV + buf * kVBytes + c8 * 1024 + r0 * 16, 128u);
+  auto issue_v = [&](int t, int buf) {
+    issue_kv(t, a.v_cache, sbase + kOffV + buf * kVBytes + c8 * 1024 + r0 * 16, 128u);
   };
-  if (ntiles > 0) issue_k(tr.at(0), 0);
+  if (ntiles > 0) issue_k(0, 0);
   cp_async_commit();
-  if (ntiles > 1) issue_k(tr.at(1), 1);
+  if (ntiles > 1) issue_k(1, 1);
   cp_async_commit();
-  if (ntiles > 0) issue_v(tr.at(0), 0);
+  if (ntiles > 0) issue_v(0, 0);
   cp_async_commit();
 
   // ---- barriers and tensor memory
@@ -345,29 +355,33 @@ prefill_tc_kernel(const TcArgs a, const Shape sh, const Tables tb) {
   const float sc = a.attn_scale * kLog2e;
   float m_ref = -INFINITY, l = 0.0f;
   bool waited_ok = true;
+  // S(0) before the loop; then in iteration i the tensor cores compute S(i + 1)
+  // while the CTA turns S(i) into P(i), and P V(i) while it reads S(i + 1)
+  auto issue_s = [&](int t) {
+    const uint32_t kb = sbase + kOffK + (t & 1) * kKBytes;
+#pragma unroll
+    for (int s = 0; s < kD / 16; ++s)
+      umma(t_s, sdesc(sbase + kOffQ + s * 256, 128, 2048), sdesc(kb + s * 256, 128, 2048), idesc(kN, false),
+           s > 0 ? 1u : 0u);
+    umma_commit(mb_s);
+  };
+  cp_async_wait2();                                   // Q and K(0)
+  fence_async_smem();
+  __syncthreads();
+  if (tid == 0 && ntiles > 0) {
+    tc_after_sync();
+    issue_s(0);
+  }
   for (int i = 0; i < ntiles; ++i) {
     const long long j0 = (long long)tr.at(i) * kN;
-    cp_async_wait2();                                 // K(i) (and Q) landed
-    fence_async_smem();
-    __syncthreads();                                  // ... for every thread and the tensor cores
-    if (s_bad) break;
-    if (tid == 0) {
-      tc_after_sync();
-      const uint32_t kb = sbase + kOffK + (i & 1) * kKBytes;
-#pragma unroll
-      for (int s = 0; s < kD / 16; ++s)
-        umma(t_s, sdesc(sbase + kOffQ + s * 256, 128, 2048), sdesc(kb + s * 256, 128, 2048), idesc(kN, false),
-             s > 0 ? 1u : 0u);
-      umma_commit(mb_s);
-    }
-    if (!mbar_wait(mb_s, (uint32_t)(i & 1))) {
+    if (!mbar_wait(mb_s, (uint32_t)(i & 1))) {        // S(i) is in tensor memory, K(i)'s buffer is free
       waited_ok = false;
       s_bad = 1;
     }
     tc_after_sync();
-    if (i + 2 < ntiles) issue_k(tr.at(i + 2), i & 1);   // S(i) has read K(i)
+    if (i + 2 < ntiles) issue_k(i + 2, i & 1);
     cp_async_commit();
-    // ---- this row's scores, masked, and its softmax weights
+    // ---- this row's scores
     float p[kN];
     {
       float v[32];
@@ -378,6 +392,17 @@ prefill_tc_kernel(const TcArgs a, const Shape sh, const Tables tb) {
 #pragma unroll
       for (int j = 0; j < 32; ++j) p[32 + j] = v[j];
     }
+    cp_async_wait2();                                 // K(i + 1) landed
+    fence_async_smem();
+    tc_before_sync();
+    __syncthreads();                                  // S(i) read by every thread: its columns may be rewritten
+    if (s_bad) break;
+    if (tid == 0 && i + 1 < ntiles) {
+      tc_after_sync();
+      issue_s(i + 1);
+    }
+    if ((i & 63) == 0 && i > 0) fill_pages(i + 64);  // the ring slots of tiles i - 64 .. i - 1 are done with
+    // ---- masked softmax weights of S(i)
     float mt = -INFINITY;
     // every row of the CTA sees the whole tile: keys at or before p0 and, for
     // local rows, all sinks or all inside the window of the last row
@@ -422,7 +447,7 @@ prefill_tc_kernel(const TcArgs a, const Shape sh, const Tables tb) {
       s_bad = 1;
     }
     tc_after_sync();
-    if (i + 1 < ntiles) issue_v(tr.at(i + 1), (i + 1) & 1);
+    if (i + 1 < ntiles) issue_v(i + 1, (i + 1) & 1);
     cp_async_commit();
     if (__any_sync(kFull, factor != 1.0f)) {          // rescale this warp's rows of O
 #pragma unroll 1
