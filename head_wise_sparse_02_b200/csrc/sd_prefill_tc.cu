@@ -4,9 +4,11 @@
 // the sinks and the window ending at i (RTPurbo page, Methodology 1; AoH page,
 // Methodology 4).
 //
-// One CTA (4 warps) per (128 consecutive query positions of one sequence, one
-// query head).  Thread r owns query row r: its tensor-memory lane holds that
-// row of S and of O, so the online softmax needs no shuffles.  Per key tile of
+// One CTA (8 warps) per (128 consecutive query positions of one sequence, one
+// query head).  Two threads own query row r (warps w and w + 4 read the same
+// TMEM lane quarter), each one half of the row's columns of S and O; they
+// trade their partial row maximum and sum through shared memory at the
+// barriers the tile already has.  Per key tile of
 // 64 positions:
 //   S[128 x 64]  = Q[128 x 128] K^T     one tcgen05.mma per 16 dims (A = Q, B = K,
 //                                       both K-major in shared memory), into TMEM
@@ -38,7 +40,7 @@ namespace {
 
 constexpr unsigned kFull = 0xFFFFFFFFu;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;                // 8 warps: two per TMEM lane quarter
 constexpr int kD = 128;                 // head dimension
 constexpr int kM = 128;                 // query rows per CTA
 constexpr int kN = 64;                  // keys per tile
@@ -87,6 +89,13 @@ __device__ __forceinline__ void tmem_st32u(uint32_t addr, const uint32_t (&v)[32
       "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]),
       "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
       "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st16u(uint32_t addr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(addr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
       : "memory");
 }
 __device__ __forceinline__ void umma_commit(uint32_t mbar) {
@@ -205,6 +214,7 @@ prefill_tc_kernel(const TcArgs a, const Shape sh, const Tables tb) {
   __shared__ uint32_t tslot;
   __shared__ int s_b, s_t, s_bad;
   __shared__ int s_pg[128 * (kN / kPage)];
+  __shared__ float s_max[2][kM], s_sum[2][kM];         // per row: the two column halves' partial max / sum
   __shared__ Group s_grp;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gr = blockIdx.y, hidx = blockIdx.z;
@@ -300,30 +310,30 @@ prefill_tc_kernel(const TcArgs a, const Shape sh, const Tables tb) {
   fill_pages(0);
   fill_pages(64);
   __syncthreads();
-  // Copies of a tile: thread tid takes the 16-byte chunk c8 = tid % 16 of rows
-  // r0 + 8 x (r0 = tid / 16, x < 8), so its rows are r0 and r0 + 8 of the tile's
-  // four pages and its shared-memory offsets are fixed up to x.
+  // Copies of a tile: thread tid takes the 16-byte chunk c8 = tid % 16 of row
+  // r0 = tid / 16 of each of the tile's four pages (x = page), so its
+  // shared-memory offsets are fixed up to x (rows r0 + 16 x: 8-row group
+  // r0 / 8 + 2 x, row r0 % 8 within it).
   const int r0 = tid >> 4, c8 = tid & 15;
   auto issue_kv = [&](int t, const uint16_t *cache, uint32_t dst0, uint32_t xstride) {
     const int kt = tr.at(t);
     const int *pg = s_pg + (t & 127) * (kN / kPage);
     const unsigned char *base = reinterpret_cast<const unsigned char *>(cache) + c8 * 16;
 #pragma unroll
-    for (int x = 0; x < 8; ++x) {
-      const int page = pg[x >> 1];
-      const int rp = r0 + 8 * (x & 1);                 // row within the page
-      const bool ok = page >= 0 && (long long)kt * kN + (x >> 1) * kPage + rp <= p_last;
+    for (int x = 0; x < kN / kPage; ++x) {
+      const int page = pg[x];
+      const bool ok = page >= 0 && (long long)kt * kN + x * kPage + r0 <= p_last;
       const unsigned char *src =
-          ok ? base + ((((size_t)page * sh.Hkv + g) * kPage + rp) * (size_t)(2 * kD)) : base;
+          ok ? base + ((((size_t)page * sh.Hkv + g) * kPage + r0) * (size_t)(2 * kD)) : base;
       cp_async16(dst0 + x * xstride, src, ok ? 16 : 0);
     }
   };
-  // K: K-major (8-row group x -> 2048 bytes); V: MN-major (8-key group x -> 128 bytes)
+  // K: K-major (8-row group -> 2048 bytes); V: MN-major (8-key group -> 128 bytes)
   auto issue_k = [&](int t, int buf) {                // t: position in the CTA's tile list
-    issue_kv(t, a.k_cache, sbase + kOffK + buf * kKBytes + c8 * 128 + r0 * 16, 2048u);
+    issue_kv(t, a.k_cache, sbase + kOffK + buf * kKBytes + (r0 >> 3) * 2048 + c8 * 128 + (r0 & 7) * 16, 2u * 2048u);
   };
   auto issue_v = [&](int t, int buf) {
-    issue_kv(t, a.v_cache, sbase + kOffV + buf * kVBytes + c8 * 1024 + r0 * 16, 128u);
+    issue_kv(t, a.v_cache, sbase + kOffV + buf * kVBytes + c8 * 1024 + (r0 >> 3) * 128 + (r0 & 7) * 16, 2u * 128u);
   };
   if (ntiles > 0) issue_k(0, 0);
   cp_async_commit();
@@ -349,9 +359,11 @@ prefill_tc_kernel(const TcArgs a, const Shape sh, const Tables tb) {
   tc_after_sync();
   const uint32_t tmem = tslot;
   const uint32_t t_o = tmem, t_s = tmem + 128, t_ph = tmem + 192, t_pl = tmem + 224;
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;   // this warp's TMEM lanes
-
-  const long long pos = p0 + tid;                     // this thread's query row
+  // warp w reads TMEM lanes 32 (w % 4) .. + 31 (rows) and column half w / 4
+  const int quarter = warp & 3, half = warp >> 2;
+  const int row = quarter * 32 + lane;                // this thread's query row
+  const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+  const long long pos = p0 + row;
   const float sc = a.attn_scale * kLog2e;
   float m_ref = -INFINITY, l = 0.0f;
   bool waited_ok = true;
@@ -382,15 +394,34 @@ prefill_tc_kernel(const TcArgs a, const Shape sh, const Tables tb) {
     if (i + 2 < ntiles) issue_k(i + 2, i & 1);
     cp_async_commit();
     // ---- this row's scores
-    float p[kN];
+    constexpr int kH = kN / 2;                        // this thread's columns of S
+    float p[kH];
+    tmem_ld32(t_s + lane_off + half * kH, p);
+    const long long jb = j0 + half * kH;              // position of column 0 of this half
+    // ---- masked scores of this half; the row's partial maximum goes to the
+    // other half's thread through shared memory at the barrier below.  Every row
+    // of the CTA sees the whole tile when its keys lie at or before p0 and, for
+    // local rows, are all sinks or all inside the last row's window.
+    const bool full = j0 + kN - 1 <= p0 &&
+                      (ret || j0 + kN - 1 < a.num_sinks || j0 > p_last - a.window);
+    if (!full) {
+      const int jr = (int)(pos - jb);                 // column j is seen when j <= jr and, for a local
+      const int js = a.num_sinks - (int)jb;           // head, j < js (a sink) or j > jw (in the window)
+      const int jw = jr - a.window;
+#pragma unroll
+      for (int j = 0; j < kH; ++j) {
+        const bool ok = j <= jr && (ret || j < js || j > jw);
+        p[j] = ok ? p[j] : -INFINITY;
+      }
+    }
     {
-      float v[32];
-      tmem_ld32(t_s + lane_off, v);
+      float mx8[8];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) p[j] = v[j];
-      tmem_ld32(t_s + lane_off + 32, v);
+      for (int u = 0; u < 8; ++u) mx8[u] = p[u];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) p[32 + j] = v[j];
+      for (int j = 8; j < kH; ++j) mx8[j & 7] = fmaxf(mx8[j & 7], p[j]);
+      s_max[half][row] = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
     }
     cp_async_wait2();                                 // K(i + 1) landed
     fence_async_smem();
@@ -402,29 +433,8 @@ prefill_tc_kernel(const TcArgs a, const Shape sh, const Tables tb) {
       issue_s(i + 1);
     }
     if ((i & 63) == 0 && i > 0) fill_pages(i + 64);  // the ring slots of tiles i - 64 .. i - 1 are done with
-    // ---- masked softmax weights of S(i)
-    float mt = -INFINITY;
-    // every row of the CTA sees the whole tile: keys at or before p0 and, for
-    // local rows, all sinks or all inside the window of the last row
-    const bool full = j0 + kN - 1 <= p0 &&
-                      (ret || j0 + kN - 1 < a.num_sinks || j0 > p_last - a.window);
-    if (full) {
-#pragma unroll
-      for (int j = 0; j < kN; ++j) {
-        p[j] *= sc;
-        mt = fmaxf(mt, p[j]);
-      }
-    } else {
-      const int jr = (int)(pos - j0);                 // key j of the tile is seen when j <= jr and, for a
-      const int js = a.num_sinks - (int)j0;           // local head, j < js (a sink) or j > jw (in the window)
-      const int jw = jr - a.window;
-#pragma unroll
-      for (int j = 0; j < kN; ++j) {
-        const bool ok = j <= jr && (ret || j < js || j > jw);
-        p[j] = ok ? p[j] * sc : -INFINITY;
-        mt = fmaxf(mt, p[j]);
-      }
-    }
+    // ---- softmax weights (the scale folded into the exponent: p = 2^(s sc - m))
+    const float mt = fmaxf(s_max[0][row], s_max[1][row]) * sc;   // the same on both halves' threads
     float factor = 1.0f;
     if (mt > -INFINITY) {
       if (m_ref == -INFINITY) {
@@ -434,13 +444,14 @@ prefill_tc_kernel(const TcArgs a, const Shape sh, const Tables tb) {
         m_ref = mt;
       }
     }
-    float ps = 0.0f;
+    const float nm = m_ref == -INFINITY ? 0.0f : -m_ref;
+    float ps8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int j = 0; j < kN; ++j) {
-      p[j] = p[j] == -INFINITY ? 0.0f : fast_exp2(p[j] - m_ref);
-      ps += p[j];
+    for (int j = 0; j < kH; ++j) {
+      p[j] = fast_exp2(fmaf(p[j], sc, nm));           // 2^(-inf) = 0 for masked keys
+      ps8[j & 7] += p[j];
     }
-    l = l * factor + ps;
+    s_sum[half][row] = ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) + ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
     // ---- P V(i - 1) must be done before O or P change and before V(i - 1)'s buffer is refilled
     if (i > 0 && !mbar_wait(mb_o, (uint32_t)((i - 1) & 1))) {
       waited_ok = false;
@@ -449,9 +460,9 @@ prefill_tc_kernel(const TcArgs a, const Shape sh, const Tables tb) {
     tc_after_sync();
     if (i + 1 < ntiles) issue_v(i + 1, (i + 1) & 1);
     cp_async_commit();
-    if (__any_sync(kFull, factor != 1.0f)) {          // rescale this warp's rows of O
+    if (__any_sync(kFull, factor != 1.0f)) {          // rescale this warp's rows of O (its column half)
 #pragma unroll 1
-      for (int c = 0; c < kD; c += 32) {
+      for (int c = half * (kD / 2); c < (half + 1) * (kD / 2); c += 32) {
         float o[32];
         tmem_ld32(t_o + lane_off + c, o);
 #pragma unroll
@@ -461,21 +472,22 @@ prefill_tc_kernel(const TcArgs a, const Shape sh, const Tables tb) {
     }
     // P = hi + lo in bf16 into tensor memory: column c holds keys 2c (low half) and 2c + 1
     {
-      uint32_t h[32], w[32];
+      uint32_t h[kH / 2], w[kH / 2];
 #pragma unroll
-      for (int c = 0; c < kN / 2; ++c) {
+      for (int c = 0; c < kH / 2; ++c) {
         const float x = p[2 * c], y = p[2 * c + 1];
         h[c] = pack_bf16(x, y);
         w[c] = pack_bf16(x - __uint_as_float(h[c] << 16), y - __uint_as_float(h[c] & 0xFFFF0000u));
       }
-      tmem_st32u(t_ph + lane_off, h);
-      tmem_st32u(t_pl + lane_off, w);
+      tmem_st16u(t_ph + lane_off + half * (kH / 2), h);
+      tmem_st16u(t_pl + lane_off + half * (kH / 2), w);
     }
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
     cp_async_wait2();                                 // V(i) landed
     fence_async_smem();
     tc_before_sync();
     __syncthreads();                                  // P and O in place, V(i) visible: the tensor cores may go
+    l = l * factor + (s_sum[half][row] + s_sum[half ^ 1][row]);
     if (s_bad) break;
     if (tid == 0) {
       tc_after_sync();
@@ -493,17 +505,17 @@ prefill_tc_kernel(const TcArgs a, const Shape sh, const Tables tb) {
   if (ntiles > 0 && !s_bad && !mbar_wait(mb_o, (uint32_t)((ntiles - 1) & 1))) waited_ok = false;
   tc_after_sync();
 
-  // ---- O / l to the output rows
-  float *orow = a.out + ((long long)(qs + row0 + tid) * sh.Hq + qh) * kD;
+  // ---- O / l to the output rows (this thread: its row's column half)
+  float *orow = a.out + ((long long)(qs + row0 + row) * sh.Hq + qh) * kD;
   const float inv = l > 0.0f ? 1.0f / l : 0.0f;
   const bool use_o = ntiles > 0 && !__syncthreads_or(!waited_ok || s_bad);
 #pragma unroll 1
-  for (int c = 0; c < kD; c += 32) {
+  for (int c = half * (kD / 2); c < (half + 1) * (kD / 2); c += 32) {
     float o[32];
     if (use_o) tmem_ld32(t_o + lane_off + c, o);
 #pragma unroll
     for (int j = 0; j < 32; ++j) o[j] = use_o ? o[j] * inv : 0.0f;
-    if (tid < nrows)
+    if (row < nrows)
 #pragma unroll
       for (int j = 0; j < 32; j += 4) *reinterpret_cast<float4 *>(orow + c + j) = make_float4(o[j], o[j + 1], o[j + 2], o[j + 3]);
   }
