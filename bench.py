@@ -170,19 +170,27 @@ KERNEL_SOURCES = {
     # the joined call: the selection and attend kernels one step launches
     "select_attend": ["head_wise_sparse_02_b200/csrc/sd_select.cu", "head_wise_sparse_02_b200/csrc/sd_select_stream.cu",
                       "head_wise_sparse_02_b200/csrc/sd_attend.cu", "head_wise_sparse_02_b200/csrc/sd_internal.cuh"],
+    # exact-score selection: the score kernel and the exact selector
+    "select_exact": ["head_wise_sparse_02_b200/csrc/sd_exact.cu", "head_wise_sparse_02_b200/csrc/sd_select.cu",
+                     "head_wise_sparse_02_b200/csrc/sd_internal.cuh"],
 }
+# the split layout's joined call runs the same kernels as the joined call
+KERNEL_SOURCES["select_attend_split"] = KERNEL_SOURCES["select_attend"]
+# ncu_traffic.json key of a call's dominant kernel, per score mode
+TRAFFIC_KEY = {("exact", "select"): "select_exact"}
 
 
-def ncu_traffic(kernel: str, algorithmic_bytes: float):
-    """DRAM bytes per call from a committed ncu summary, if it was taken on
-    the current kernel source (else None).  The summary stores DRAM bytes per
-    algorithmic byte of the captured (smaller) case; both grow with the rows
-    a call processes, so the ratio scales the capture to this call."""
+def ncu_traffic(kernel: str, workload: str, algorithmic_bytes: float):
+    """DRAM bytes per call from a committed ncu summary of this call on this
+    workload, if it was taken on the current kernel source (else None).  The
+    summary stores DRAM bytes per algorithmic byte of the captured case (the
+    bench's own size, or a smaller one that takes the same code path); both
+    grow with the rows a call processes, so the ratio scales it to this call."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(p) as f:
             d = json.load(f)
-        e = d[kernel]
+        e = d[f"{kernel}@{workload}"]
         if e.get("source_hash") != kernel_source_hash(KERNEL_SOURCES[kernel]):
             return None
         return round(float(e["dram_bytes_per_algorithmic_byte"]) * algorithmic_bytes)
@@ -364,7 +372,10 @@ def size_overrides(args):
     kw = {}
     if args.batch:
         kw["B"] = args.batch
-    if args.seq_len:
+    if args.seq_len and args.workload == "ragged_paged":
+        kw["N_max"] = args.seq_len                  # lengths U[min(4096, N), N]
+        kw["N_min"] = min(4096, args.seq_len)
+    elif args.seq_len:
         kw["N"] = args.seq_len
     if args.top_p:
         kw["top_p"] = args.top_p
@@ -622,7 +633,8 @@ def run_ours(args):
                      "peak_kind": f"{peak_kind} hbm_gbs (copy bandwidth)", "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
                      "algorithmic_bytes_per_launch": kern_bytes[dominant],
-                     "traffic": ncu_traffic(dominant, kern_bytes[dominant])},
+                     "traffic": ncu_traffic(TRAFFIC_KEY.get((args.score, dominant), dominant), args.workload,
+                                            kern_bytes[dominant])},
         "e2e": {"value": round(head_steps / (e2e_ms * 1e-3), 1), "unit": UNIT,
                 "h2d_bytes_per_step": int(q_h.numel() * 2 + (0 if exact else
                                                              qp_h.numel() * 2 + nk_h.numel() * 2 + ns_h.numel() * 4)
@@ -1073,7 +1085,8 @@ def run_prefill(args):
                                f"{w.num_kv_heads}, d={w.head_dim}, {n_ret} retrieval heads (dense causal) + "
                                f"{w.num_q_heads - n_ret} local (window {w.window} + {w.num_sinks} sinks)",
                    "parallelism": f"replicas x{ws}", "l2": "flushed between steps (512 MiB write, untimed)"},
-        "roofline": {"kernel": "prefill_kernel", "bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
+        "roofline": {"kernel": ("prefill_tc_kernel (tcgen05, accumulators in tensor memory)" if w.head_dim == 128
+                                else "prefill_kernel (mma.sync)"), "bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
                      "peak_kind": f"{kind} bf16_tflops (cuBLAS bf16 GEMM)", "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "algorithmic_flops_per_launch": fl, "traffic": None,
                      "note": "P V runs as two bf16 MMAs (P split hi + lo): 1.5x the algorithmic MMA work"},
