@@ -52,6 +52,16 @@ def test_full_prefill_tiny(N):
     _run(w, [N], label=f"N={N}")
 
 
+@pytest.mark.parametrize("N", [1, 17, 64, 65, 128, 129, 200])
+def test_full_prefill_d128(N):
+    """d = 128 (the tcgen05 kernel) at the edges of its 128-row query tile and
+    64-key tile: one retrieval and one local head per KV group, so each CTA
+    holds two heads, and a group whose second head slot is empty."""
+    from workloads.synthetic import _base
+    w = _base("d128", N, "cuda", [N], 6, 2, 128, [1, 0, 0, 1, 1, 0], 40, 3, "top_p", permute=True)
+    _run(w, [N], seed=N, label=f"d128 N={N}")
+
+
 def test_later_chunks_ragged_permuted():
     from workloads.synthetic import _base
     w = _base("chunks", 5, "cuda", [300, 1000, 77], 8, 2, 128, [1, 1, 0, 0, 0, 1, 0, 0], 96, 4, "top_p",
