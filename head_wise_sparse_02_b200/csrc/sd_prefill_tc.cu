@@ -517,25 +517,34 @@ prefill_tc_kernel(const TcArgs a, const Shape sh, const Tables tb) {
     // cp.async.mbarrier.arrive.noinc counts on the buffer's "full" barrier once
     // all its copies so far have landed (the MMA thread fences them to the
     // async proxy after its wait), so up to kStages tiles are in flight.
+    // page ids of the tile after the current one are loaded while the current
+    // tile's copies are issued (kPastEnd past p_last); checked one iteration later
+    constexpr int kPastEnd = -0x7FFFFFFF - 1;
+    auto raw_pages = [&](int t) {
+      const long long k0 = (long long)tr.at(t) * kN;
+      int4 v;
+      v.x = k0 <= p_last ? pt[k0 / kPage] : kPastEnd;
+      v.y = k0 + kPage <= p_last ? pt[k0 / kPage + 1] : kPastEnd;
+      v.z = k0 + 2 * kPage <= p_last ? pt[k0 / kPage + 2] : kPastEnd;
+      v.w = k0 + 3 * kPage <= p_last ? pt[k0 / kPage + 3] : kPastEnd;
+      return v;
+    };
+    auto checked = [&](int id) {                      // -1: zero-fill; a bad id also sets the error bit
+      if (id == kPastEnd) return -1;
+      if (id < 0 || id >= sh.num_pages) {
+        raise_error(a.err, SD_EBIT_PAGE);
+        return -1;
+      }
+      return id;
+    };
     bool ok = true;
+    int4 nxt = ntiles > 0 ? raw_pages(0) : make_int4(kPastEnd, kPastEnd, kPastEnd, kPastEnd);
     for (int i = 0; i < ntiles; ++i) {
       const int bi = i % kStages;
       const uint32_t par = (uint32_t)(((i / kStages) + 1) & 1);   // completion i / kStages - 1: tile i - kStages
       const long long k0 = (long long)tr.at(i) * kN;
-      int pgs[kN / kPage];                            // page ids of the tile (-1: past p_last or a bad id)
-#pragma unroll
-      for (int u = 0; u < kN / kPage; ++u) {
-        const long long key = k0 + u * kPage;
-        int val = -1;
-        if (key <= p_last) {
-          val = pt[key / kPage];
-          if (val < 0 || val >= sh.num_pages) {
-            raise_error(a.err, SD_EBIT_PAGE);
-            val = -1;
-          }
-        }
-        pgs[u] = val;
-      }
+      const int pgs[kN / kPage] = {checked(nxt.x), checked(nxt.y), checked(nxt.z), checked(nxt.w)};
+      if (i + 1 < ntiles) nxt = raw_pages(i + 1);
       long long so[kN / 4];                           // byte offsets of this thread's rows (-1: zero-fill)
 #pragma unroll
       for (int x = 0; x < kN / 4; ++x) {

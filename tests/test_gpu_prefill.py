@@ -128,3 +128,24 @@ def test_inconsistent_chunk_sets_error_word_without_fault():
     assert sd.error_word() & SD_EBIT_SEQLEN
     assert float(out.abs().sum()) == 0.0                                     # nothing written
     sd.close()
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_bad_page_ids_error_word_without_fault(d):
+    """Page-table entries outside the pool (past its end, negative) inside a
+    sequence's range: the kernel reads zeros in their place, sets the page
+    error bit and leaves every output finite."""
+    from head_wise_sparse_02_b200.sparse_decode import SD_EBIT_PAGE
+    from workloads.synthetic import _base
+    w = _base("badpage", 3, "cuda", [300], 4, 2, d, [1, 0, 0, 1], 64, 2, "top_p", permute=True)
+    pt = w.page_table.clone()
+    pt[0, 5] = int(w.k_cache.shape[0]) + 7
+    pt[0, 9] = -3
+    sd = _ctx(w)
+    q, starts = prefill_inputs(w, [300], seed=2)
+    out = torch.full(q.shape, float("nan"), dtype=torch.float32, device="cuda")
+    sd.prefill(q, w.k_cache, w.v_cache, pt, w.seq_lens, starts, out)
+    torch.cuda.synchronize()
+    assert sd.error_word() & SD_EBIT_PAGE
+    assert bool(torch.isfinite(out).all())
+    sd.close()
