@@ -28,8 +28,9 @@
 // one head's softmax runs, the tensor cores work on the other head.
 // The hand-offs are mbarriers, no CTA-wide barrier inside the loop: a K / V
 // buffer is full when every copy thread's cp.async.mbarrier.arrive has fired
-// (its copies landed; the MMA thread then fences them to the async proxy) and
-// free when tcgen05.commit says the MMAs that read it are done; S_s is full
+// (its copies landed; the MMA warp then fences them to the async proxy), and a
+// buffer slot (K and V of one tile) is free when tcgen05.commit says that the
+// tile's S and P V MMAs of both heads are done; S_s is full
 // when tcgen05.commit arrives; P_s is stored when each softmax warp arrives.
 // Every wait is bounded (a poll count and 2 s of the global timer) and also
 // ends when another role has given up (a shared flag): the CTA then sets
@@ -281,7 +282,7 @@ prefill_tc_kernel(const TcArgs a, const Shape sh, const Tables tb) {
   // mbarriers: K / V buffer full (copy warps) and free (MMA commit); per head
   // slot Q stored and P stored (softmax warps), S full (MMA commit: S(i) and
   // the P V before it), the last P V done (MMA commit); the MMA thread's drain
-  __shared__ __align__(8) uint64_t bar_kfull[kStages], bar_kfree[kStages], bar_vfull[kStages], bar_vfree[kStages];
+  __shared__ __align__(8) uint64_t bar_kfull[kStages], bar_vfull[kStages], bar_free[kStages];
   __shared__ __align__(8) uint64_t bar_qfull[2], bar_sfull[2], bar_pfull[2], bar_odone[2], bar_drain;
   __shared__ uint32_t tslot;
   __shared__ int s_b, s_t;
@@ -351,8 +352,7 @@ prefill_tc_kernel(const TcArgs a, const Shape sh, const Tables tb) {
     for (int k = 0; k < kStages; ++k) {
       mbar_init(bar(&bar_kfull[k]), kLoadThreads);
       mbar_init(bar(&bar_vfull[k]), kLoadThreads);
-      mbar_init(bar(&bar_kfree[k]), 1);
-      mbar_init(bar(&bar_vfree[k]), 1);
+      mbar_init(bar(&bar_free[k]), 1);
     }
     for (int k = 0; k < 2; ++k) {
       mbar_init(bar(&bar_sfull[k]), 1);
@@ -554,15 +554,13 @@ prefill_tc_kernel(const TcArgs a, const Shape sh, const Tables tb) {
                     ? (long long)((((size_t)page * sh.Hkv + g) * kPage + (r % kPage)) * (size_t)(2 * kD))
                     : -1;
       }
-      if (i >= kStages) ok = __all_sync(kFull, mbar_wait(bar(&bar_kfree[bi]), par, &s_bad));
+      if (i >= kStages) ok = __all_sync(kFull, mbar_wait(bar(&bar_free[bi]), par, &s_bad));
       if (!ok) break;
 #pragma unroll
       for (int x = 0; x < kN / 4; ++x)
         cp_async16(k_dst + bi * kKBytes + (x >> 1) * 2048 + (x & 1) * 64, so[x] >= 0 ? kbase + so[x] : kbase,
                    so[x] >= 0 ? 16 : 0);
       cp_async_arrive_noinc(bar(&bar_kfull[bi]));
-      if (i >= kStages) ok = __all_sync(kFull, mbar_wait(bar(&bar_vfree[bi]), par, &s_bad));
-      if (!ok) break;
 #pragma unroll
       for (int x = 0; x < kN / 4; ++x)
         cp_async16(v_dst + bi * kVBytes + (x >> 1) * 128 + (x & 1) * 64, so[x] >= 0 ? vbase + so[x] : vbase,
@@ -604,10 +602,13 @@ prefill_tc_kernel(const TcArgs a, const Shape sh, const Tables tb) {
       tc_after_sync();
       if (ok) issue_s(0, s);
     }
-    if (ok) umma_commit(bar(&bar_kfree[0]));
     for (int i = 0; i < ntiles && ok; ++i) {
       const bool more = i + 1 < ntiles;
+      // V(i) and K(i + 1) landed; one fence to the async proxy for both
       ok = __all_sync(kFull, mbar_wait(bar(&bar_vfull[i % kStages]), (uint32_t)((i / kStages) & 1), &s_bad));
+      if (ok && more)
+        ok = __all_sync(kFull, mbar_wait(bar(&bar_kfull[(i + 1) % kStages]), (uint32_t)(((i + 1) / kStages) & 1),
+                                         &s_bad));
       fence_async_smem();
       // per head: P V(i), then S(i + 1) into the same columns
       for (int s = 0; s < nh && ok; ++s) {
@@ -615,22 +616,11 @@ prefill_tc_kernel(const TcArgs a, const Shape sh, const Tables tb) {
         tc_after_sync();
         if (!ok) break;
         issue_pv(i, s);
-        if (!more) {
-          umma_commit(bar(&bar_odone[s]));
-          continue;
-        }
-        if (s == 0) {
-          ok = __all_sync(kFull, mbar_wait(bar(&bar_kfull[(i + 1) % kStages]), (uint32_t)(((i + 1) / kStages) & 1),
-                                           &s_bad));
-          fence_async_smem();
-          tc_after_sync();
-          if (!ok) break;
-        }
-        issue_s(i + 1, s);
+        if (more) issue_s(i + 1, s);
+        else umma_commit(bar(&bar_odone[s]));
       }
       if (!ok) break;
-      umma_commit(bar(&bar_vfree[i % kStages]));
-      if (more) umma_commit(bar(&bar_kfree[(i + 1) % kStages]));
+      umma_commit(bar(&bar_free[i % kStages]));       // K(i) and V(i): S(i) and P V(i) of both heads are done
     }
     // every MMA issued above completes before tensor memory is freed (this
     // wait ignores the abort flag; the MMAs depend on nothing and finish)
