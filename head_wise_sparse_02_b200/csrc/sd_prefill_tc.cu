@@ -37,9 +37,12 @@
 // SD_EBIT_TIMEOUT, waits for its own MMAs and copies, writes zeros and frees
 // its tensor memory.
 //
-// The running maximum of a row is only moved when a tile raises it by more than
-// 8 (log2 units); O is then rescaled in tensor memory (ld, scale, st), so most
-// tiles skip that round trip and P stays below 2^8.
+// The softmax reference of a row (log2 units) is set by the first keys it sees
+// and moved only when a tile's weights against it sum past 2^64 or overflow;
+// then S is read again, the reference becomes the tile's maximum and O is
+// rescaled in tensor memory (ld, scale, st).  Most tiles so skip both the row
+// maximum and the rescale; P (hi + lo) and O keep their relative precision at
+// any magnitude up to 2^64.
 //
 // Shared-memory operand layouts are the canonical no-swizzle ones: 8 rows x
 // 16 bytes per core matrix (128 contiguous bytes); for the K-major K the two
@@ -65,7 +68,7 @@ constexpr int kD = 128;                 // head dimension
 constexpr int kM = 128;                 // query rows per CTA
 constexpr int kN = 64;                  // keys per tile
 constexpr int kStages = 4;              // K and V buffers
-constexpr float kRescale = 8.0f;        // log2 growth of a row maximum that triggers a rescale of O
+constexpr float kBig = 1.8446744e19f;   // 2^64: a tile whose weights sum past this moves the reference
 constexpr long long kWaitSpins = 1LL << 26;
 constexpr unsigned long long kWaitNs = 2000000000ull;
 
@@ -415,44 +418,66 @@ prefill_tc_kernel(const TcArgs a, const Shape sh, const Tables tb) {
         if (!ok) break;
         tc_after_sync();
         float p[kN];
-        tmem_ld32x2(t_s, p);
         // ---- masked scores.  Every row of the CTA sees the whole tile when its
         // keys lie at or before p0 and, for local rows, are all sinks or all
         // inside the last row's window.
         const bool full = j0 + kN - 1 <= p0 && (ret || j0 + kN - 1 < a.num_sinks || j0 > p_last - a.window);
-        if (!full) {
-          const int jr = (int)(pos - j0);             // column j is seen when j <= jr and, for a local
-          const int js = a.num_sinks - (int)j0;       // head, j < js (a sink) or j > jw (in the window)
-          const int jw = jr - a.window;
+        auto load_scores = [&]() {                    // warp-collective
+          tmem_ld32x2(t_s, p);
+          if (!full) {
+            const int jr = (int)(pos - j0);           // column j is seen when j <= jr and, for a local
+            const int js = a.num_sinks - (int)j0;     // head, j < js (a sink) or j > jw (in the window)
+            const int jw = jr - a.window;
+#pragma unroll
+            for (int j = 0; j < kN; ++j) {
+              const bool seen = j <= jr && (ret || j < js || j > jw);
+              p[j] = seen ? p[j] : -INFINITY;
+            }
+          }
+        };
+        auto scaled_max = [&]() {                     // the tile's maximum of this row, times sc
+          float mx8[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) mx8[u] = p[u];
+#pragma unroll
+          for (int j = 8; j < kN; ++j) mx8[j & 7] = fmaxf(mx8[j & 7], p[j]);
+          return fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * sc;
+        };
+        float ps8[8];
+        auto weights = [&]() {                        // p = 2^(s sc - m_ref); 2^(-inf) = 0 for masked keys
+          const float nm = m_ref == -INFINITY ? 0.0f : -m_ref;
+#pragma unroll
+          for (int u = 0; u < 8; ++u) ps8[u] = 0.0f;
 #pragma unroll
           for (int j = 0; j < kN; ++j) {
-            const bool seen = j <= jr && (ret || j < js || j > jw);
-            p[j] = seen ? p[j] : -INFINITY;
+            p[j] = fast_exp2(fmaf(p[j], sc, nm));
+            ps8[j & 7] += p[j];
           }
-        }
-        float mx8[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) mx8[u] = p[u];
-#pragma unroll
-        for (int j = 8; j < kN; ++j) mx8[j & 7] = fmaxf(mx8[j & 7], p[j]);
-        const float mt = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * sc;
-        // ---- softmax weights (the scale folded into the exponent: p = 2^(s sc - m))
+          return ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) + ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
+        };
+        load_scores();
+        // ---- softmax weights against the row's reference m_ref (log2 units),
+        // which is set by the first keys the row sees and only moved when a
+        // tile's weights against it sum past kBig (or overflow): then S is read
+        // again, m_ref becomes the tile's maximum and O is rescaled.  Most tiles
+        // thus skip the row maximum altogether; P and O keep their relative
+        // precision at any magnitude up to kBig.
         float factor = 1.0f;
-        if (mt > -INFINITY) {
-          if (m_ref == -INFINITY) {
-            m_ref = mt;                               // first keys of the row: O and l are still zero
-          } else if (mt > m_ref + kRescale) {
+        if (__any_sync(kFull, m_ref == -INFINITY)) {
+          const float mt = scaled_max();
+          if (m_ref == -INFINITY) m_ref = mt;         // O and l are still zero; -inf again if no key is seen
+        }
+        float psum = weights();
+        if (__any_sync(kFull, !(psum <= kBig))) {
+          const bool moved = !(psum <= kBig);
+          load_scores();
+          const float mt = scaled_max();
+          if (moved && mt > m_ref) {
             factor = fast_exp2(m_ref - mt);
             m_ref = mt;
           }
-        }
-        const float nm = m_ref == -INFINITY ? 0.0f : -m_ref;
-        float ps8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int j = 0; j < kN; ++j) {
-          p[j] = fast_exp2(fmaf(p[j], sc, nm));       // 2^(-inf) = 0 for masked keys
-          ps8[j & 7] += p[j];
+          psum = weights();
         }
         if (__any_sync(kFull, factor != 1.0f)) {      // rescale this warp's rows of O
 #pragma unroll 1
@@ -480,7 +505,7 @@ prefill_tc_kernel(const TcArgs a, const Shape sh, const Tables tb) {
         tc_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(b_pfull);          // P(i) and O in place: P V(i) may go
-        l = l * factor + (((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) + ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7])));
+        l = l * factor + psum;
       }
       if (ok && ntiles > 0) {                         // the last P V
         ok = __all_sync(kFull, mbar_wait(bar(&bar_odone[s]), 0u, &s_bad));

@@ -93,11 +93,13 @@ def test_llama3_8b_shapes_sampled_rows():
     _run(w, [4096], rows=rows, label="llama3 4096")
 
 
-@pytest.mark.parametrize("scale", [0.25, 4.0])
+@pytest.mark.parametrize("scale", [0.25, 4.0, 48.0])
 def test_peaked_and_flat_softmax(scale):
     """Query scales that make the softmax nearly flat (0.25) or sharply peaked
-    with row maxima jumping between key tiles (4.0: the running maximum moves
-    and the partial outputs are rescaled), 700 positions, ragged pages."""
+    with row maxima jumping between key tiles (4.0; 48.0: logits spread over
+    hundreds of log2 units, so later tiles' weights against the row's first
+    reference overflow it, the reference moves and the partial outputs are
+    rescaled), 700 positions, ragged pages."""
     from workloads.synthetic import _base
     w = _base("scaled", 12, "cuda", [700, 300], 8, 2, 128, [1, 1, 0, 0, 1, 0, 0, 1], 160, 4, "top_p", permute=True)
     sd = _ctx(w)
