@@ -1,5 +1,6 @@
 // C ABI of the sparse decode library: argument validation, the context, the
 // workspace layout and the launches.  See include/sparse_decode.h.
+#include <atomic>
 #include <math.h>
 #include <stdio.h>
 
@@ -8,6 +9,10 @@
 #include <vector>
 
 #include "sd_internal.cuh"
+
+namespace sd {
+extern std::atomic<int> g_prefill_stall;      // sd_prefill_tc.cu: testing switch of the d = 128 prefill
+}
 
 struct sd_ctx {
   sd_config cfg;                      // head_is_retrieval points into `retr`
@@ -549,6 +554,8 @@ sd_status sparse_decode_attend_noalloc(sd_ctx *ctx, const void *q, const void *k
     return SD_ERR_HOST_MEMORY;
   }
 }
+
+void sparse_decode_testing_stall_prefill(int on) { sd::g_prefill_stall.store(on != 0 ? 1 : 0); }
 
 sd_status sparse_decode_error_word(sd_ctx *ctx, sd_stream stream, uint32_t *word) {
   try {

@@ -52,6 +52,7 @@
 // operand (Q, P) has one row per lane and two 16-bit K elements per 32-bit
 // column.
 #include <algorithm>
+#include <atomic>
 
 #include "sd_internal.cuh"
 
@@ -245,6 +246,7 @@ struct TcArgs {
   float attn_scale;
   int window, num_sinks, batch, total_q;
   unsigned *err;
+  int stall;                      // testing: the MMA warp first waits on a barrier nothing arrives at
 };
 
 // Key tiles (64 positions) of a CTA, ascending, without repeats: retrieval rows
@@ -286,7 +288,7 @@ prefill_tc_kernel(const TcArgs a, const Shape sh, const Tables tb) {
   // slot Q stored and P stored (softmax warps), S full (MMA commit: S(i) and
   // the P V before it), the last P V done (MMA commit); the MMA thread's drain
   __shared__ __align__(8) uint64_t bar_kfull[kStages], bar_vfull[kStages], bar_free[kStages];
-  __shared__ __align__(8) uint64_t bar_qfull[2], bar_sfull[2], bar_pfull[2], bar_odone[2], bar_drain;
+  __shared__ __align__(8) uint64_t bar_qfull[2], bar_sfull[2], bar_pfull[2], bar_odone[2], bar_drain, bar_never;
   __shared__ uint32_t tslot;
   __shared__ int s_b, s_t;
   __shared__ volatile int s_bad;
@@ -364,6 +366,7 @@ prefill_tc_kernel(const TcArgs a, const Shape sh, const Tables tb) {
       mbar_init(bar(&bar_odone[k]), 1);
     }
     mbar_init(bar(&bar_drain), 1);
+    mbar_init(bar(&bar_never), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == kMmaWarp) {
@@ -620,7 +623,9 @@ prefill_tc_kernel(const TcArgs a, const Shape sh, const Tables tb) {
 #pragma unroll
       for (int k = 0; k < kN / 16; ++k) umma_ts<true>(to, to + 160 + k * 8, dv + k * 16, id_o);
     };
-    bool ok = __all_sync(kFull, mbar_wait(bar(&bar_kfull[0]), 0u, &s_bad));
+    bool ok = true;
+    if (a.stall) ok = __all_sync(kFull, mbar_wait(bar(&bar_never), 0u, &s_bad));   // runs out: the test of the bounds
+    ok = ok && __all_sync(kFull, mbar_wait(bar(&bar_kfull[0]), 0u, &s_bad));
     fence_async_smem();                               // the copy warps' writes, to the async proxy
     for (int s = 0; s < nh && ok; ++s) {
       ok = __all_sync(kFull, mbar_wait(bar(&bar_qfull[s]), 0u, &s_bad));
@@ -665,6 +670,8 @@ prefill_tc_kernel(const TcArgs a, const Shape sh, const Tables tb) {
 
 }  // namespace
 
+std::atomic<int> g_prefill_stall{0};
+
 cudaError_t launch_prefill_tc(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
                               const int32_t *page_table, const int32_t *seq_lens, const int32_t *q_starts, int batch,
                               int total_q, float *out, float attn_scale, int window, int num_sinks, const Shape &sh,
@@ -673,7 +680,8 @@ cudaError_t launch_prefill_tc(const uint16_t *q, const uint16_t *k_cache, const 
   static_assert(kSmem > 114 * 1024 && kSmem <= 227 * 1024, "one CTA per SM: it holds all 512 TMEM columns");
   cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
-  TcArgs a{q, k_cache, v_cache, page_table, seq_lens, q_starts, out, attn_scale, window, num_sinks, batch, total_q, err};
+  TcArgs a{q, k_cache, v_cache, page_table, seq_lens, q_starts, out, attn_scale, window, num_sinks, batch, total_q, err,
+           g_prefill_stall.load()};
   const long long tiles = (long long)(total_q + kM - 1) / kM + batch;   // >= sum_b ceil(T_b / 128)
   const int heads = std::max(tb.max_ret, tb.max_loc);
   const dim3 grid((unsigned)tiles, (unsigned)(tb.n_ret + tb.n_loc), (unsigned)((heads + 1) / 2));

@@ -69,6 +69,7 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
                                                       P]),
         "sparse_decode_classify_heads": (c_int, [P, c_int, c_int, c_int, P]),
         "sparse_decode_num_retrieval_heads": (c_int, [P]),
+        "sparse_decode_testing_stall_prefill": (None, [c_int]),
         "sparse_decode_last_error": (c_char_p, [P]),
         "sparse_decode_status_string": (c_char_p, [c_int]),
         "sparse_decode_destroy": (None, [P]),
@@ -356,6 +357,12 @@ def sparse_decode_error_word(ctx: int, stream=None) -> int:
     if st not in (SD_OK, SD_ERR_DEVICE_DATA, SD_ERR_TIMEOUT):
         _check(st, ctx)
     return int(w.value)
+
+
+def sparse_decode_testing_stall_prefill(on: bool) -> None:
+    """Testing only: while on, the d = 128 prefill's device-side waits cannot
+    end and run out after their bound (outputs zero, SD_EBIT_TIMEOUT)."""
+    LIB.sparse_decode_testing_stall_prefill(1 if on else 0)
 
 
 def sparse_decode_num_retrieval_heads(ctx: int) -> int:

@@ -466,6 +466,18 @@ SD_API sd_status sparse_decode_attend_noalloc(sd_ctx *ctx, const void *q, const 
  */
 SD_API sd_status sparse_decode_error_word(sd_ctx *ctx, sd_stream stream, uint32_t *word);
 
+/*
+ * sparse_decode_testing_stall_prefill -- testing only, off by default.  While
+ * on != 0, every CTA of the d = 128 prefill kernel first waits on an mbarrier
+ * that nothing arrives at: a device-side wait that cannot end.  Its bound (2 s
+ * of the global timer) runs out, the CTA's other roles stop at their next wait,
+ * its MMAs and copies are drained, its outputs are written as zeros and the
+ * error word gets SD_EBIT_TIMEOUT; the context stays usable.  The tests use it
+ * to check that the bounded waits end and are reported.  Process-wide; set it
+ * back to 0 before production calls.
+ */
+SD_API void sparse_decode_testing_stall_prefill(int on);
+
 /* Number of retrieval heads (rows per sequence in sel_idx / sel_count). */
 SD_API int sparse_decode_num_retrieval_heads(const sd_ctx *ctx);
 

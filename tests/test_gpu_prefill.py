@@ -151,3 +151,41 @@ def test_bad_page_ids_error_word_without_fault(d):
     assert sd.error_word() & SD_EBIT_PAGE
     assert bool(torch.isfinite(out).all())
     sd.close()
+
+
+def test_bounded_wait_runs_out_and_is_reported():
+    """A device-side wait that cannot end (the testing switch makes the MMA warp
+    of every CTA wait on an mbarrier that nothing arrives at) runs out after its
+    bound; the other roles stop, the outputs are zero, the error word reports
+    SD_EBIT_TIMEOUT, and the next call on the same context is correct."""
+    import time
+
+    from head_wise_sparse_02_b200 import sparse_decode as S
+    from workloads.synthetic import _base
+    w = _base("stall", 65, "cuda", [65], 6, 2, 128, [1, 0, 0, 1, 1, 0], 40, 3, "top_p", permute=True)
+    sd = _ctx(w)
+    q, starts = prefill_inputs(w, [65], seed=1)
+    out = torch.full(q.shape, float("nan"), dtype=torch.float32, device="cuda")
+    S.sparse_decode_testing_stall_prefill(True)
+    try:
+        t0 = time.time()
+        sd.prefill(q, w.k_cache, w.v_cache, w.page_table, w.seq_lens, starts, out)
+        torch.cuda.synchronize()
+        took = time.time() - t0
+    finally:
+        S.sparse_decode_testing_stall_prefill(False)
+    assert sd.error_word() & S.SD_EBIT_TIMEOUT
+    assert float(out.abs().sum()) == 0.0
+    assert took < 60.0
+    # the context and the GPU stay usable: the same call again, checked against the oracle
+    out.fill_(float("nan"))
+    sd.prefill(q, w.k_cache, w.v_cache, w.page_table, w.seq_lens, starts, out)
+    torch.cuda.synchronize()
+    assert sd.error_word() == 0
+    inp = oracle_inputs(w)
+    ref = O.prefill_reference(oracle_config(w), q.float().cpu().numpy(), inp["k_cache"], inp["v_cache"],
+                              inp["page_table"], inp["seq_lens"], starts.cpu().numpy())
+    got = out.cpu().numpy()
+    for (r, h), o in ref.items():
+        assert_out_close(got[r, h], o, f"after stall row={r} h={h}")
+    sd.close()
