@@ -93,6 +93,18 @@ def test_llama3_8b_shapes_sampled_rows():
     _run(w, [4096], rows=rows, label="llama3 4096")
 
 
+def test_prefill_32k_sampled_rows():
+    """The bench's prefill at full size (prefill_llama3_8b: one 32768-token
+    chunk, 8 retrieval + 24 local heads, window 1024 + 4 sinks, d = 128, the
+    tcgen05 kernel), every head of sampled rows: tile edges, the window edge and
+    the longest key ranges at the end of the sequence."""
+    w = make_workload("llama3_8b_topp", "cuda", B=1, N=32768, permute=True, seed=1)
+    rng = np.random.default_rng(7)
+    rows = sorted(set(rng.integers(0, 32768, size=10).tolist())
+                  | {0, 1, 63, 64, 127, 128, 1023, 1024, 1028, 16383, 32640, 32766, 32767})
+    _run(w, [32768], seed=5, rows=rows, label="32K")
+
+
 @pytest.mark.parametrize("scale", [0.25, 4.0, 48.0])
 def test_peaked_and_flat_softmax(scale):
     """Query scales that make the softmax nearly flat (0.25) or sharply peaked
