@@ -22,7 +22,8 @@
 //                    d_head * eps * max diag G zeroes its column (rank-deficient
 //                    blocks factor as semi-definite)
 //   jacobi_kernel    X = L_k^T L_q in shared memory, parallel cyclic Jacobi
-//                    sweeps (round-robin pairings, one warp per column pair),
+//                    sweeps (round-robin pairings; each warp takes several
+//                    column pairs of a round, their reductions interleaved),
 //                    then ER from the column norms
 //
 // Everything is float64: this runs once per model, and its output is a
