@@ -190,17 +190,26 @@ __device__ __forceinline__ void select_item(const SelectArgs &a, const Shape &sh
   if (tid < kMaxGroup) S.cmax_key[tid] = 0u;
   __syncthreads();
 
-  if constexpr (!SMEM) {
-    if (a.pre_scored) {
-      // ---- the score rows are given: the CTA's maxima only ------------------
-      for (int h = 0; h < nr; ++h) {
-        const float *sc = score_ptr(h);
-        float m = -INFINITY;
-        for (int i = tid; i < cnt; i += kThreads) m = fmaxf(m, sc[i]);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
-        if (lane == 0 && m > -INFINITY) atomicMax(&S.cmax_key[h], order_key(m));
+  if (a.pre_scored) {
+    // ---- the score rows are given (exact-score mode): the CTA's maxima, and
+    // with room on chip a copy of its chunk of every row, read once here
+    // instead of at every radix pass
+    for (int h = 0; h < nr; ++h) {
+      const float *src = a.score_ws + ((long long)b * sh.H_ret + S.grp.row[h]) * sh.max_len + t0;
+      float m = -INFINITY;
+      if constexpr (SMEM) {
+        float *dst = score_ptr(h);
+        for (int i = tid; i < cnt; i += kThreads) {
+          const float v = __ldcg(src + i);
+          dst[i] = v;
+          m = fmaxf(m, v);
+        }
+      } else {
+        for (int i = tid; i < cnt; i += kThreads) m = fmaxf(m, src[i]);
       }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
+      if (lane == 0 && m > -INFINITY) atomicMax(&S.cmax_key[h], order_key(m));
     }
   }
   // ---- stream the index, score, keep scores on chip ----------------------
@@ -775,13 +784,9 @@ cudaError_t launch_select_impl(const SelectArgs &a, const Shape &sh, const Table
     p.tc_cap = (int)(((sh.max_len + c - 1) / c + kPage - 1) / kPage * kPage);
     p.dyn_bytes = hist_bytes(group_rows(tb), topp);
   }
-  if (a.pre_scored) {
-    // exact-score mode: the score rows are in the workspace already; every
-    // item goes through the exact selector, reading them there
-    p.smem = false;
-    p.tc_cap = (int)(((sh.max_len + p.cluster - 1) / p.cluster + kPage - 1) / kPage * kPage);
-    p.dyn_bytes = hist_bytes(group_rows(tb), topp);
-  }
+  // exact-score mode: the score rows are in the workspace already and every
+  // item goes through the exact selector; a CTA copies its chunk of them on
+  // chip when the plan has room for it (else it reads them there at each pass)
   const int items = a.batch * tb.n_ret;
   bool used = false;
   if (!a.pre_scored) {
