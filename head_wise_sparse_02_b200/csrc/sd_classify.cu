@@ -264,16 +264,18 @@ jacobi_kernel(const double *__restrict__ gram, int Hq, int Hkv, double *__restri
   // to D * eps relative; round r pairs (r, D-1) and ((r+m) mod (D-1),
   // (r-m) mod (D-1)) for m = 1 .. D/2-1, every pair once per sweep
   // Warp w takes pairs m = w * PPW .. w * PPW + PPW - 1 of each round, all at
-  // once: their partial sums, butterfly reductions and rotations interleave,
-  // so the shuffle latency of one pair hides behind the others'.
+  // once: their partial sums, reductions and rotations interleave, so the
+  // shuffle latency of one pair hides behind the others'.
   constexpr int PPW = D / 2 / kWarps;                // pairs per warp and round
+  static_assert(PPW % 4 == 0, "the pair sums are split over the four quarters of a warp");
   constexpr int RPL = D / 32;                        // rows per lane
   const double tol2 = (D * DBL_EPSILON) * (D * DBL_EPSILON);
   bool converged = false;
   for (int sweep = 0; sweep < kMaxSweeps && !converged; ++sweep) {
     int rotated = 0;
     for (int r = 0; r < D - 1; ++r) {
-      double al[PPW], be[PPW], ga[PPW], t_of[PPW];
+      double al[PPW], be[PPW], ga[PPW];
+      double xu[PPW][RPL], xv[PPW][RPL];             // this lane's rows of the pairs' columns, read once
       int cp[PPW], cq[PPW];
 #pragma unroll
       for (int j = 0; j < PPW; ++j) {
@@ -284,32 +286,75 @@ jacobi_kernel(const double *__restrict__ gram, int Hq, int Hkv, double *__restri
 #pragma unroll
         for (int e = 0; e < RPL; ++e) {
           const double u = Xc[cp[j] * D + lane + 32 * e], v = Xc[cq[j] * D + lane + 32 * e];
+          xu[j][e] = u;
+          xv[j][e] = v;
           al[j] = fma(u, u, al[j]);
           be[j] = fma(v, v, be[j]);
           ga[j] = fma(u, v, ga[j]);
         }
       }
+      // The pairs' sums (al, be, ga) over the warp, reduce-scatter style: two
+      // halving exchanges leave each quarter of the warp (lane bits 4 and 3)
+      // with the partial sums of NP of the pairs, a butterfly over those lanes
+      // completes them, the quarter computes their rotations, and three
+      // exchanges give every lane the rotations of all PPW pairs.
+      constexpr int NV = 3 * PPW, NP = PPW / 4;
+      const int b4 = (lane >> 4) & 1, b3 = (lane >> 3) & 1;
+      double w1[NV / 2], w2[NV / 4];
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1)               // butterfly sums: identical on every lane
+      for (int k = 0; k < NV / 2; ++k) {             // lanes 0-15 keep pairs 0 .. PPW/2-1, lanes 16-31 the rest
+        const int lo = k, hi = NV / 2 + k;
+        const double vlo = lo % 3 == 0 ? al[lo / 3] : (lo % 3 == 1 ? be[lo / 3] : ga[lo / 3]);
+        const double vhi = hi % 3 == 0 ? al[hi / 3] : (hi % 3 == 1 ? be[hi / 3] : ga[hi / 3]);
+        w1[k] = (b4 ? vhi : vlo) + __shfl_xor_sync(kFull, b4 ? vlo : vhi, 16);
+      }
 #pragma unroll
-        for (int j = 0; j < PPW; ++j) {
-          al[j] += __shfl_xor_sync(kFull, al[j], o);
-          be[j] += __shfl_xor_sync(kFull, be[j], o);
-          ga[j] += __shfl_xor_sync(kFull, ga[j], o);
+      for (int k = 0; k < NV / 4; ++k) {             // then lane bit 3 halves the kept pairs again
+        const double vlo = w1[k], vhi = w1[NV / 4 + k];
+        w2[k] = (b3 ? vhi : vlo) + __shfl_xor_sync(kFull, b3 ? vlo : vhi, 8);
+      }
+#pragma unroll
+      for (int o = 4; o > 0; o >>= 1)
+#pragma unroll
+        for (int k = 0; k < NV / 4; ++k) w2[k] += __shfl_xor_sync(kFull, w2[k], o);
+      // this quarter's pairs G4 * PPW/2 + G3 * NP + p (G4 = b4, G3 = b3): c, s
+      // (s = 0: no rotation; a rotating pair has |t| > 0, so s != 0)
+      double cg[NP], sg[NP];
+#pragma unroll
+      for (int q = 0; q < NP; ++q) {
+        const double A = w2[3 * q], Bv = w2[3 * q + 1], Gv = w2[3 * q + 2];
+        cg[q] = 1.0;
+        sg[q] = 0.0;
+        if (Gv * Gv > tol2 * (A * Bv)) {             // |gamma| > tol sqrt(alpha beta), without the root
+          double t;
+          cg[q] = rot_cos(A, Bv, Gv, t);
+          sg[q] = cg[q] * t;
+          rotated = 1;
         }
+      }
+      double c8[NP], s8[NP], c16[NP], s16[NP], c24[NP], s24[NP];
+#pragma unroll
+      for (int q = 0; q < NP; ++q) {
+        c8[q] = __shfl_xor_sync(kFull, cg[q], 8);
+        s8[q] = __shfl_xor_sync(kFull, sg[q], 8);
+        c16[q] = __shfl_xor_sync(kFull, cg[q], 16);
+        s16[q] = __shfl_xor_sync(kFull, sg[q], 16);
+        c24[q] = __shfl_xor_sync(kFull, cg[q], 24);
+        s24[q] = __shfl_xor_sync(kFull, sg[q], 24);
+      }
 #pragma unroll
       for (int j = 0; j < PPW; ++j) {
-        if (ga[j] * ga[j] > tol2 * (al[j] * be[j])) {  // |gamma| > tol sqrt(alpha beta), without the root
-          const double c = rot_cos(al[j], be[j], ga[j], t_of[j]);
-          const double s = c * t_of[j];
+        const int G4 = j / (PPW / 2), G3 = (j / NP) & 1, q = j % NP;
+        const bool f4 = G4 != b4, f3 = G3 != b3;
+        const double c = f4 ? (f3 ? c24[q] : c16[q]) : (f3 ? c8[q] : cg[q]);
+        const double sn = f4 ? (f3 ? s24[q] : s16[q]) : (f3 ? s8[q] : sg[q]);
+        if (sn != 0.0) {
 #pragma unroll
           for (int e = 0; e < RPL; ++e) {
-            double *xp = Xc + cp[j] * D + lane + 32 * e, *xq = Xc + cq[j] * D + lane + 32 * e;
-            const double u = *xp, v = *xq;
-            *xp = c * u - s * v;
-            *xq = s * u + c * v;
+            const double u = xu[j][e], v = xv[j][e];
+            Xc[cp[j] * D + lane + 32 * e] = c * u - sn * v;
+            Xc[cq[j] * D + lane + 32 * e] = sn * u + c * v;
           }
-          rotated = 1;
         }
       }
       __syncthreads();
