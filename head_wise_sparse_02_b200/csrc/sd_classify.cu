@@ -212,11 +212,19 @@ __host__ __device__ constexpr size_t jacobi_smem() {
 }
 
 // One CTA per (layer, query head): X = L_k^T L_q, one-sided Jacobi, ER.
+// threads of the Jacobi kernel: 4 column pairs per warp and round
 template <int D>
-__global__ void __launch_bounds__(kThreads)
+__host__ __device__ constexpr int jacobi_threads() {
+  return D / 2 / 4 * 32;
+}
+
+template <int D>
+__global__ void __launch_bounds__(jacobi_threads<D>(), 1)
 jacobi_kernel(const double *__restrict__ gram, int Hq, int Hkv, double *__restrict__ eff_rank) {
-  constexpr int TI = D / 16;                         // rows / columns of X per thread (register tile)
-  constexpr int kWarps = kThreads / 32;
+  constexpr int kJThreads = jacobi_threads<D>();
+  constexpr int kWarps = kJThreads / 32;
+  constexpr int TR = D / (kJThreads / 16), TC = D / 16;   // rows, columns of X per thread (register tile)
+  static_assert(TR >= 1 && D % (kJThreads / 16) == 0, "X tile");
   extern __shared__ __align__(16) double smem[];
   double *Xc = smem;                                 // X column-major: Xc[j * D + i] = X_ij
   double *sk = smem + D * D;                         // 16 staged rows of L_k
@@ -229,34 +237,35 @@ jacobi_kernel(const double *__restrict__ gram, int Hq, int Hkv, double *__restri
   const double *Lq = gram + ((size_t)layer * (Hq + Hkv) + h) * D * D;
   const double *Lk = gram + ((size_t)layer * (Hq + Hkv) + Hq + g) * D * D;
 
-  // ---- X_ij = sum_k Lk[k][i] Lq[k][j]: rows i = ty + 16 a, columns j = tx + 16 c
+  // ---- X_ij = sum_k Lk[k][i] Lq[k][j]: rows i = ty + (threads / 16) a,
+  // columns j = tx + 16 c
   {
-    double acc[TI][TI] = {};
+    constexpr int RS = kJThreads / 16;               // row stride of a thread's tile
+    double acc[TR][TC] = {};
     for (int k0 = 0; k0 < D; k0 += 16) {
-      for (int x = tid; x < 16 * D; x += kThreads) {
+      for (int x = tid; x < 16 * D; x += kJThreads) {
         sk[x] = Lk[(size_t)k0 * D + x];
         sq[x] = Lq[(size_t)k0 * D + x];
       }
       __syncthreads();
 #pragma unroll 2
       for (int k = 0; k < 16; ++k) {
-        double u[TI], v[TI];
+        double u[TR], v[TC];
 #pragma unroll
-        for (int t = 0; t < TI; ++t) {
-          u[t] = sk[k * D + ty + 16 * t];
-          v[t] = sq[k * D + tx + 16 * t];
-        }
+        for (int t = 0; t < TR; ++t) u[t] = sk[k * D + ty + RS * t];
 #pragma unroll
-        for (int a = 0; a < TI; ++a)
+        for (int t = 0; t < TC; ++t) v[t] = sq[k * D + tx + 16 * t];
 #pragma unroll
-          for (int c = 0; c < TI; ++c) acc[a][c] = fma(u[a], v[c], acc[a][c]);
+        for (int a = 0; a < TR; ++a)
+#pragma unroll
+          for (int c = 0; c < TC; ++c) acc[a][c] = fma(u[a], v[c], acc[a][c]);
       }
       __syncthreads();
     }
 #pragma unroll
-    for (int a = 0; a < TI; ++a)
+    for (int a = 0; a < TR; ++a)
 #pragma unroll
-      for (int c = 0; c < TI; ++c) Xc[(tx + 16 * c) * D + ty + 16 * a] = acc[a][c];
+      for (int c = 0; c < TC; ++c) Xc[(tx + 16 * c) * D + ty + RS * a] = acc[a][c];
   }
   __syncthreads();
 
@@ -407,7 +416,7 @@ cudaError_t launch_er_d(const uint16_t *w_q, const uint16_t *w_k, int L, int d_m
   static_assert(jacobi_smem<D>() + D * sizeof(double) <= 227 * 1024, "Jacobi tile fits in shared memory");
   e = cudaFuncSetAttribute(jacobi_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)jacobi_smem<D>());
   if (e != cudaSuccess) return e;
-  return launch_pdl(jacobi_kernel<D>, dim3(L * Hq), dim3(kThreads), jacobi_smem<D>(), st, 0,
+  return launch_pdl(jacobi_kernel<D>, dim3(L * Hq), dim3(jacobi_threads<D>()), jacobi_smem<D>(), st, 0,
                     (const double *)gram, Hq, Hkv, er);
 }
 
