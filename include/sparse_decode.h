@@ -89,7 +89,7 @@ typedef void *sd_stream;               /* a cudaStream_t */
 typedef enum {
   SD_OK = 0,
   SD_ERR_INVALID_ARG = 1,   /* a null pointer, a bad size or an inconsistent shape */
-  SD_ERR_UNSUPPORTED = 2,   /* a valid request this build does not implement */
+  SD_ERR_UNSUPPORTED = 2,   /* a valid request the library does not implement */
   SD_ERR_WORKSPACE = 3,     /* workspace missing or smaller than the size query */
   SD_ERR_CUDA = 4,          /* a CUDA runtime call or a kernel launch failed */
   SD_ERR_TIMEOUT = 5,       /* a bounded device-side wait gave up */

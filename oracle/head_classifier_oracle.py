@@ -17,7 +17,7 @@ Query-Key Geometry", gist.science/ar/paper/2608.06849, Methodology:
   §4  heads ranked by ER, the k lowest become retrieval heads; under GQA the
       head scores are mean-pooled to the group.
 
-Readings taken where the page is silent or garbled (each is listed in the design doc):
+Readings taken where the page is silent or garbled:
   * W_Q^h is the d_head x d_model block of rows h*d_head .. (h+1)*d_head - 1
     of the query projection weight [Hq*d_head, d_model] (q = W x), and W_K^g
     likewise of the key projection; head h pairs with KV head g = h // (Hq/Hkv);

@@ -25,7 +25,7 @@ position i of head h attends, causally, to
     retrieval head:  keys 0 .. i                         (dense causal)
     local head:      keys [0, num_sinks) U [i - window + 1, i], within [0, i]
 
-Readings (listed in the design doc): the window counts the query's own position,
+Readings: the window counts the query's own position,
 so a local head's keys at position i are the decode local set at length
 i + 1; the chunk's own keys and values are already in the cache; earlier
 chunks' keys are read from the cache like any other.

@@ -28,7 +28,7 @@ Sources (gist.science summary pages; cited below by the short tag):
       Geometry", gist.science/ar/paper/2608.06849.  Methodology §4 deployment:
       streaming (local) heads keep a fixed sink prefix plus a recent window.
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
   * one projection P_g of shape [d, r] per KV head g, shared by the keys of
     that head and the queries of its GQA group;
   * the index cache stores k~ = P_g^T k rounded to bf16 (round to nearest
