@@ -62,6 +62,15 @@ def test_full_prefill_d128(N):
     _run(w, [N], seed=N, label=f"d128 N={N}")
 
 
+def test_empty_chunk_between_sequences_d128():
+    """Three sequences, the middle one with an empty chunk (no query rows): the
+    query tiles of the others map to the right sequences and positions."""
+    from workloads.synthetic import _base
+    w = _base("emptychunk", 8, "cuda", [150, 90, 300], 8, 2, 128, [1, 0, 1, 1, 0, 0, 1, 0], 50, 2, "top_p",
+              permute=True)
+    _run(w, [150, 0, 130], seed=2, label="empty chunk")
+
+
 def test_later_chunks_ragged_permuted():
     from workloads.synthetic import _base
     w = _base("chunks", 5, "cuda", [300, 1000, 77], 8, 2, 128, [1, 1, 0, 0, 0, 1, 0, 0], 96, 4, "top_p",
