@@ -58,6 +58,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kPlanThreads = 256;
 constexpr int kPlanWarps = kPlanThreads / 32;
 constexpr int kSpanMax = 32768;         // positions per plan CTA (max)
+constexpr int kPlanCtas = 296;          // plan CTAs aimed for when the items are few (two per SM)
 
 // main
 constexpr int kThreads = 128;
@@ -941,7 +942,11 @@ int group_rows_att(const Tables &tb) { return pow2_ceil(std::max(1, std::max(tb.
 AttParams att_params(const Shape &sh, const Tables &tb, int batch) {
   AttParams p{};
   const long long L = sh.max_len;
-  p.span = (int)std::max(256LL, std::min<long long>(kSpanMax, pow2_ceil((L + 3) / 4)));   // ~4 spans per sequence
+  // spans per sequence: about four, more when the retrieval items are few, so
+  // that the plan still has about kPlanCtas CTAs (its work is split by span)
+  const long long items = std::max(1LL, (long long)batch * tb.n_ret);
+  const long long want = std::max(4LL, (kPlanCtas + items - 1) / items);
+  p.span = (int)std::max(256LL, std::min<long long>(kSpanMax, pow2_ceil((L + want - 1) / want)));
   p.ns = (int)((L + p.span - 1) / p.span);
   p.n_ret_items = batch * tb.n_ret;
   p.ni = batch * (tb.n_ret + tb.n_loc);
