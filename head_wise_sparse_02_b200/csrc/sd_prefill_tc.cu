@@ -21,7 +21,7 @@
 //                                          shared memory)
 // Q in tensor memory keeps the S MMAs off the shared-memory bandwidth (only K
 // is read there), and P over S keeps two heads within the 512 columns.  The MMA
-// thread issues, per head, P V(i) and then S(i + 1) into the same columns (the
+// warp issues, per head, P V(i) and then S(i + 1) into the same columns (the
 // tensor cores run one thread's MMAs in order, so S(i + 1) overwrites P(i) only
 // after P V(i) has read it), and commits both to one mbarrier: its arrival
 // tells the softmax warps that S(i + 1) is there and that O holds P V(i).  While
@@ -35,7 +35,9 @@
 // Every wait is bounded (a poll count and 2 s of the global timer) and also
 // ends when another role has given up (a shared flag): the CTA then sets
 // SD_EBIT_TIMEOUT, waits for its own MMAs and copies, writes zeros and frees
-// its tensor memory.
+// its tensor memory.  A test-only switch (sparse_decode_testing_stall_prefill)
+// makes the MMA warp first wait on an mbarrier that nothing arrives at, so
+// that the tests can check this path.
 //
 // The softmax reference of a row (log2 units) is set by the first keys it sees
 // and moved only when a tile's weights against it sum past 2^64 or overflow;
