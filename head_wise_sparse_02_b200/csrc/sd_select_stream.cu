@@ -86,7 +86,14 @@ constexpr int kBinsK = 2048;          // top-k K2: bins of the window and of eac
 constexpr int kCap = 2048;            // K2: cut-bin tokens ranked exactly
 constexpr int kLevels = 3;            // K2: histogram levels (the cut bin is split again)
 constexpr int kRefine = 256;          // K2: a cut bin above this many tokens is split again
-constexpr int kPer2 = 16;             // K2: buffer entries held in registers per thread
+// K2: buffer entries held in registers per thread (the rest of the buffer is
+// read from L2 at each pass), by the launch's register budget: with 64
+// registers a thread, 16 entries (32 registers) spilled; the fused union
+// resolve, whose union walk needs more of them, holds 8
+__host__ __device__ constexpr int per_thread_entries(int cta_threads, int ctas_per_sm) {
+  return 65536 / (cta_threads * ctas_per_sm) > 64 ? 16 : (cta_threads >= 1024 ? 8 : 12);
+}
+constexpr int kRestBatch = 4;         // K2: buffer entries past the registers loaded at once per thread
 constexpr int kPageBytes = kPage * kIndexDim * 2;   // 512 B: one page of one KV head
 constexpr unsigned kFull = 0xFFFFFFFFu;
 // top-p window (K0): the sample's kExcl highest tokens are left out of its
@@ -1020,21 +1027,23 @@ struct TopkSmem {
 // levels at most); entries above the cut path are selected, the cut bin's are
 // ranked exactly by (score desc, position asc).  Leaves the set in `bitmap`
 // (bits of [0, N)) and writes it out; false when the window missed (the item
-// is flagged for the exact selector and nothing is written).
+// is flagged for the exact selector and nothing is written).  PER: buffer
+// entries held in registers per thread.
+template <int PER>
 __device__ bool resolve_topk(const SelectArgs &a, const Shape &sh, const StreamWs &ws, int b, int hr,
                              const HeadGroup &hg, TopkSmem &S, uint32_t *bitmap, bool union_bits) {
   const int tid = hg.t, lane = tid & 31;
   const long long row = (long long)b * sh.H_ret + hr;
   int32_t *out = a.sel_idx + row * a.sel_stride;
   // one round of independent loads: the length, the window, the buffer count
-  // and the first kPer2 * kT2 buffer slots (inside the row: reads stop at cap)
+  // and the first PER * kT2 buffer slots (inside the row: reads stop at cap)
   long long N = a.seq_lens[b];
   const float4 w = ws.win[row];
   const uint32_t nbuf = ws.bcount[row];
   const unsigned long long *buf = ws.buf + row * ws.cap;
-  unsigned long long ent[kPer2];
+  unsigned long long ent[PER];
 #pragma unroll
-  for (int j = 0; j < kPer2; ++j) {
+  for (int j = 0; j < PER; ++j) {
     const int e = tid + j * kT2;
     ent[j] = e < ws.cap ? __ldcg(buf + e) : 0ull;
   }
@@ -1063,7 +1072,7 @@ __device__ bool resolve_topk(const SelectArgs &a, const Shape &sh, const StreamW
     return min(kBinsK - 1, max(0, __float2int_rz((v - S.llo[L]) * S.linv[L])));
   };
   // the entries past the registers are read from the buffer (L2) at each pass
-  const int rest0 = kPer2 * kT2;
+  const int rest0 = PER * kT2;
   // the cut bin: refine while it holds more than kRefine tokens
   int L = 0;
   for (; L < kLevels; ++L) {
@@ -1077,9 +1086,16 @@ __device__ bool resolve_topk(const SelectArgs &a, const Shape &sh, const StreamW
       if (play) atomicAdd(&S.hist[bin_at(v, L)], 1u);
     };
 #pragma unroll
-    for (int j = 0; j < kPer2; ++j)
+    for (int j = 0; j < PER; ++j)
       if (tid + j * kT2 < n) add(ent[j]);
-    for (int e = rest0 + tid; e < n; e += kT2) add(__ldcg(buf + e));
+    for (int e0 = rest0 + tid; e0 < n; e0 += kRestBatch * kT2) {
+      unsigned long long v[kRestBatch];              // independent loads first
+#pragma unroll
+      for (int u = 0; u < kRestBatch; ++u) v[u] = e0 + u * kT2 < n ? __ldcg(buf + e0 + u * kT2) : 0ull;
+#pragma unroll
+      for (int u = 0; u < kRestBatch; ++u)
+        if (e0 + u * kT2 < n) add(v[u]);
+    }
     if (tid == 0) S.res[0] = -1;
     hg.sync();
     const long long need = S.need - (L == 0 ? (long long)S.hist[kBinsK] : 0LL);
@@ -1134,10 +1150,16 @@ __device__ bool resolve_topk(const SelectArgs &a, const Shape &sh, const StreamW
     }
   };
 #pragma unroll
-  for (int j = 0; j < kPer2; ++j) classify(ent[j], tid + j * kT2 < n);
-  for (int e0 = rest0; e0 < n; e0 += kT2) {
-    const int e = e0 + tid;
-    classify(e < n ? __ldcg(buf + e) : 0ull, e < n);
+  for (int j = 0; j < PER; ++j) classify(ent[j], tid + j * kT2 < n);
+  for (int e0 = rest0; e0 < n; e0 += kRestBatch * kT2) {
+    unsigned long long v[kRestBatch];
+#pragma unroll
+    for (int u = 0; u < kRestBatch; ++u) {
+      const int e = e0 + u * kT2 + tid;
+      v[u] = e < n ? __ldcg(buf + e) : 0ull;
+    }
+#pragma unroll
+    for (int u = 0; u < kRestBatch; ++u) classify(v[u], e0 + u * kT2 + tid < n);
   }
   hg.sync();
   // rank the cut bin exactly: the need_c best by (score desc, position asc)
@@ -1337,7 +1359,7 @@ topk_resolve_kernel(const SelectArgs a, const Shape sh, const StreamWs ws) {
   pdl_wait();
   pdl_trigger();
   const HeadGroup hg{(int)threadIdx.x, 0, true};
-  resolve_topk(a, sh, ws, blockIdx.y, blockIdx.x, hg, S, bitmap, false);
+  resolve_topk<per_thread_entries(kT2, 4)>(a, sh, ws, blockIdx.y, blockIdx.x, hg, S, bitmap, false);
 }
 
 __global__ void __launch_bounds__(kT2, 4)
@@ -1353,9 +1375,10 @@ topp_resolve_kernel(const SelectArgs a, const Shape sh, const StreamWs ws) {
 // K2 of the decode step with the union: one CTA per (sequence, retrieval KV
 // group), one group of kT2 threads per retrieval head of the group (NG >= the
 // group's heads).  Each group resolves its head into a bitmap of the context
-// and writes the head's list; then the whole CTA walks the heads' bitmaps span
-// by span (the spans of attend's plan) and writes the group's union list
-// there: (cache row, head mask) in ascending position order, and its length.
+// and writes the head's list; then the whole CTA walks the heads' bitmaps over
+// the spans of attend's plan (the item's spans side by side, a share of the
+// warps each) and writes each span's union list there: (cache row, head mask)
+// in ascending position order, and its length.
 // An item with a missed window is left to the exact selector and to attend's
 // plan.  dynamic shared memory: [NG bitmaps of bm_bytes][NG head smem].
 template <bool TOPP, int NG>
@@ -1385,13 +1408,14 @@ resolve_union_kernel(const SelectArgs a, const Shape sh, const StreamWs ws, cons
   Smem &S = *reinterpret_cast<Smem *>(dynu + (size_t)NG * bm_bytes + (size_t)k * sizeof(Smem));
   if (k < nr) {
     const bool ok = TOPP ? resolve_topp(a, sh, ws, b, grp.row[k], hg, reinterpret_cast<ToppSmem &>(S), bitmap_of(k), true)
-                         : resolve_topk(a, sh, ws, b, grp.row[k], hg, reinterpret_cast<TopkSmem &>(S), bitmap_of(k), true);
+                         : resolve_topk<per_thread_entries(NG * kT2, 1)>(a, sh, ws, b, grp.row[k], hg,
+                                                                      reinterpret_cast<TopkSmem &>(S), bitmap_of(k), true);
     if (!ok && hg.t == 0) any_fail = 1;
   }
   __syncthreads();
   if (any_fail) return;                              // planned by attend after the exact selector
 
-  // ---- the group's union list, span by span ------------------------------------
+  // ---- the group's union list: the item's spans side by side ---------------------
   long long N = a.seq_lens[b];
   N = N < 0 ? 0 : std::min<long long>(N, sh.max_len);
   const int words = (int)((N + 31) / 32);
@@ -1403,10 +1427,32 @@ resolve_union_kernel(const SelectArgs a, const Shape sh, const StreamWs ws, cons
   const uint32_t row_page = (uint32_t)(uo.ret_only ? n_groups : sh.Hkv) * kPage;
   const int32_t *pt = a.page_table + (long long)b * sh.max_pages;
   bool bad_page = false;
-  for (int sp = 0; sp < ns_item; ++sp) {
-    const int x_lo = sp * span_words, x_hi = std::min(words, x_lo + span_words);
-    const int steps = (x_hi - x_lo + NWC * 32 - 1) / (NWC * 32);
-    const int w0 = x_lo + warp * steps * 32;
+  // P spans at a time, WPS warps on each: warp `sub` of a span takes its words
+  // [sub * steps * 32, (sub + 1) * steps * 32) in steps of 32 (one per lane)
+  constexpr int kPre = 4;                            // steps whose page ids are loaded up front
+  const int P = ns_item < NWC ? ns_item : NWC;
+  const int WPS = P > 0 ? NWC / P : NWC;
+  const int sub = warp % WPS, first = warp - sub;
+  for (int sp0 = 0; sp0 < ns_item; sp0 += P) {
+    const int sp = sp0 + warp / WPS;
+    const bool act = warp / WPS < P && sp < ns_item;
+    const int x_lo = act ? sp * span_words : 0;
+    const int x_hi = act ? std::min(words, x_lo + span_words) : 0;
+    const int steps = (x_hi - x_lo + WPS * 32 - 1) / (WPS * 32);
+    const int w0 = x_lo + sub * steps * 32;
+    // the two pages of each word of the first steps, in flight during the
+    // count (pages at or past the sequence's end are never read)
+    auto pages_of = [&](int x, int &p0, int &p1) {
+      const long long q0 = (long long)x * 32;
+      p0 = (x < x_hi && q0 < N) ? pt[q0 >> 4] : -1;
+      p1 = (x < x_hi && q0 + 16 < N) ? pt[(q0 >> 4) + 1] : -1;
+    };
+    int pre0[kPre], pre1[kPre];
+#pragma unroll
+    for (int r = 0; r < kPre; ++r) {
+      pre0[r] = pre1[r] = -1;
+      if (r < steps) pages_of(w0 + r * 32 + lane, pre0[r], pre1[r]);
+    }
     uint32_t c = 0;
     for (int r = 0; r < steps; ++r) {
       const int x = w0 + r * 32 + lane;
@@ -1420,14 +1466,14 @@ resolve_union_kernel(const SelectArgs a, const Shape sh, const StreamWs ws, cons
     if (lane == 0) ctot[warp] = c;
     __syncthreads();
     uint32_t off = 0, total = 0;
-    for (int x = 0; x < NWC; ++x) {
+    for (int x = first; x < first + WPS; ++x) {
       off += x < warp ? ctot[x] : 0u;
       total += ctot[x];
     }
-    const long long slot = ((long long)b * n_groups + gi) * uo.ns + sp;   // attend's plan slot
+    const long long slot = ((long long)b * n_groups + gi) * uo.ns + (act ? sp : 0);   // attend's plan slot
     uint32_t *rows = uo.row + slot * uo.span;
     uint16_t *masks = uo.mask + slot * uo.span;
-    for (int r = 0; r < steps; ++r) {
+    auto step = [&](int r, int pg0, int pg1) {       // warp-wide: words w0 + 32 r + lane
       const int xb = w0 + r * 32;
       const int x = xb + lane;
       uint32_t hw[NG];
@@ -1437,11 +1483,6 @@ resolve_union_kernel(const SelectArgs a, const Shape sh, const StreamWs ws, cons
         hw[i] = (x < x_hi && i < nr) ? bitmap_of(i)[x] : 0u;
         u |= hw[i];
       }
-      // the two pages of this lane's word, loaded before the emission needs
-      // them (pages at or past the sequence's end are never read)
-      const long long q0 = (long long)x * 32;
-      const int pg0 = (x < x_hi && q0 < N) ? pt[q0 >> 4] : -1;
-      const int pg1 = (x < x_hi && q0 + 16 < N) ? pt[(q0 >> 4) + 1] : -1;
       off += (uint32_t)warp_emit_bits(u, lane, [&](bool valid, int kk, int w, int bit) {
         uint32_t m = 0;
 #pragma unroll
@@ -1455,9 +1496,17 @@ resolve_union_kernel(const SelectArgs a, const Shape sh, const StreamWs ws, cons
         rows[off + kk] = ok ? (uint32_t)page * row_page + row_g + (uint32_t)(pos & (kPage - 1)) : 0u;
         masks[off + kk] = (uint16_t)(ok ? m : 0u);
       });
+    };
+#pragma unroll
+    for (int r = 0; r < kPre; ++r)
+      if (r < steps) step(r, pre0[r], pre1[r]);
+    for (int r = kPre; r < steps; ++r) {
+      int p0, p1;
+      pages_of(w0 + r * 32 + lane, p0, p1);
+      step(r, p0, p1);
     }
-    if (tid == 0) uo.cnt[slot] = (int)total;
-    __syncthreads();                                 // ctot is reused by the next span
+    if (act && sub == 0 && lane == 0) uo.cnt[slot] = (int)total;
+    __syncthreads();                                 // ctot is reused by the next spans
   }
   if (bad_page) raise_error(a.err, SD_EBIT_PAGE);
 }
