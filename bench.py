@@ -27,6 +27,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import subprocess
 import sys
 import threading
@@ -154,11 +155,38 @@ def load_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def code_only(text: bytes) -> bytes:
+    """A C++/CUDA source without its comments (// and /* */ outside string and
+    character literals) and with every run of whitespace made one space: the
+    code the compiler sees, so that an edit of the comments alone keeps a
+    capture taken on the source valid."""
+    out, i, n = bytearray(), 0, len(text)
+    while i < n:
+        c = text[i:i + 1]
+        if c in (b'"', b"'"):
+            j = i + 1
+            while j < n and text[j:j + 1] != c:
+                j += 2 if text[j:j + 1] == b"\\" else 1
+            out += text[i:j + 1]
+            i = j + 1
+        elif text.startswith(b"//", i):
+            j = text.find(b"\n", i)
+            i = n if j < 0 else j
+        elif text.startswith(b"/*", i):
+            j = text.find(b"*/", i + 2)
+            i = n if j < 0 else j + 2
+            out += b" "
+        else:
+            out += c
+            i += 1
+    return re.sub(rb"\s+", b" ", bytes(out)).strip()
+
+
 def kernel_source_hash(files):
     h = hashlib.sha256()
     for f in files:
         with open(os.path.join(ROOT, f), "rb") as fh:
-            h.update(fh.read())
+            h.update(code_only(fh.read()))
     return h.hexdigest()[:16]
 
 

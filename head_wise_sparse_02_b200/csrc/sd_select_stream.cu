@@ -30,13 +30,17 @@
 //              batches, to a per-head buffer.  Most scores fail the single
 //              compare and cost nothing more.
 //   K2 resolve one CTA per (sequence, retrieval head): histograms the
-//              buffered scores over 512 bins of [t_lo, t_hi) (plus one bin for
-//              scores >= t_hi), scans from the top for the bin holding the
-//              k-th score and, while that bin holds many tokens, splits it
-//              into 512 sub-bins and scans again (three levels at most); ranks
-//              the tokens of the final bin exactly by (score desc, position
-//              asc), marks the selected positions in a bitmap of the context
-//              and writes them in ascending order.
+//              buffered scores over 2048 bins of [t_lo, t_hi) (plus one bin
+//              for scores >= t_hi), scans from the top for the bin holding
+//              the k-th score and, while that bin holds many tokens, splits
+//              it into 2048 sub-bins and scans again (three levels at most);
+//              ranks the tokens of the final bin exactly by (score desc,
+//              position asc), marks the selected positions in a bitmap of the
+//              context and writes them in ascending order.
+//
+// In the joined select + attend call with many items, K2 of either mode runs
+// fused: one CTA per (sequence, retrieval KV group) resolves all its heads and
+// writes the group's union list straight into attend's workspace.
 //
 // top-p (four launches; the softmax mass of a head is known only after a
 // whole pass, so the index is streamed twice)

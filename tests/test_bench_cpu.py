@@ -88,3 +88,17 @@ def test_reference_arm_prints_one_contract_line(capsys):
     assert d["value"] > 0 and d["cpu_baseline"]["value"] == d["value"]
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_kernel_hash_ignores_comments_only():
+    """roofline.traffic stays tied to the code it was captured on: the hash
+    leaves comments and whitespace out, and changes with any code token."""
+    src = (b'// header\n#include <x.h>\n/* block\n comment */ int f(int a) {  // why\n'
+           b'  const char *s = "a // not a comment /* nor this */";\n  return a + \'/\';\n}\n')
+    edited = (b'// a new header, longer\n\n#include <x.h>\n/* other */ int f(int a) {\n'
+              b'  const char *s = "a // not a comment /* nor this */";   // note\n  return a + \'/\';\n}\n')
+    changed = src.replace(b"a + '/'", b"a - '/'")
+    assert bench.code_only(src) == bench.code_only(edited)
+    assert bench.code_only(src) != bench.code_only(changed)
+    assert b'"a // not a comment /* nor this */"' in bench.code_only(src)
+    assert b"header" not in bench.code_only(src) and b"why" not in bench.code_only(src)
